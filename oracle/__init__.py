@@ -1,0 +1,198 @@
+"""Plain fp64 CPU oracle for the FLARE / FLARE++ mixer forward.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` are the only code
+allowed to import this package.  The CUDA library never calls it and shares no
+code with it.
+
+The arithmetic lives in ``flare_oracle.c`` (plain loops, fp64, two-pass
+softmax in ascending index order, OpenMP over independent rows); this module
+only marshals numpy arrays.  Every function cites the passage of the FLARE++
+paper (arXiv 2608.11519, section "Method") it follows:
+
+  project   eq. 7 / eq. 9   K_h = X W_{K,h}, heads = column blocks of width D
+  encode    eq. 5 / 8 / 10  Z_h = softmax_n(Q_h K_h^T / sqrt(D)) V_h
+  decode    eq. 6 / 11      Y_h = softmax_m(K_h Q_h^T / sqrt(D)) Z_h
+
+Pins (tests/test_oracle_pins.py): torch float64 SDPA chain, the materialised
+rank-M mixing matrix, closed forms (two tokens, identical keys, zero queries,
+one latent), token-permutation equivariance, the masked/unmasked identity and
+the shard-combine identity of section "Multi-GPU context parallelism" (eq. 14).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "flare_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "libflare_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with gcc (OpenMP, IEEE semantics, no FMA contraction)."""
+    if not force and os.path.exists(_LIB_PATH) and \
+            os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC):
+        return _LIB_PATH
+    os.makedirs(_BUILD, exist_ok=True)
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fPIC",
+           "-shared", "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int32)
+        lp = ctypes.POINTER(ctypes.c_int64)
+        L = ctypes.c_long
+        lib.flare_oracle_project.argtypes = [dp, dp, dp, L, L, L, L, L]
+        lib.flare_oracle_project.restype = None
+        lib.flare_oracle_encode.argtypes = [dp, ctypes.c_int, dp, dp, ip, ctypes.c_double,
+                                            L, L, L, L, L, dp, dp]
+        lib.flare_oracle_encode.restype = None
+        lib.flare_oracle_decode.argtypes = [dp, dp, ctypes.c_int, dp, ip, ctypes.c_double,
+                                            L, L, L, L, L, lp, L, dp]
+        lib.flare_oracle_decode.restype = None
+        lib.flare_oracle_num_threads.argtypes = []
+        lib.flare_oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def num_threads() -> int:
+    return int(_load().flare_oracle_num_threads())
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _dptr(a: Optional[np.ndarray]):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _lens(lengths, B):
+    if lengths is None:
+        return None, None
+    arr = np.ascontiguousarray(lengths, dtype=np.int32)
+    assert arr.shape == (B,)
+    return arr, arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def project(X, W, H: int) -> np.ndarray:
+    """eq. 7 / eq. 9: X [B][N][C] @ W [C][C], split into H heads -> [B][H][N][D]."""
+    X, W = _f64(X), _f64(W)
+    B, N, C = X.shape
+    assert W.shape == (C, C) and C % H == 0
+    D = C // H
+    out = np.empty((B, H, N, D), dtype=np.float64)
+    _load().flare_oracle_project(_dptr(X), _dptr(W), _dptr(out), B, N, C, H, D)
+    return out
+
+
+def encode(Q, K, V, lengths=None, scale: Optional[float] = None,
+           return_lse: bool = False):
+    """eq. 5 (FLARE encoder), eq. 8 (query synthesis), eq. 10 (encode with Q(X)).
+
+    Q: [H][M][D] (shared over the batch) or [B][H][M][D] (one set per sample).
+    K, V: [B][H][N][D].  Returns Z [B][H][M][D] (and the row log-normaliser
+    lse [B][H][M] = max + log(sum exp) when ``return_lse``)."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    B, H, N, D = K.shape
+    assert V.shape == K.shape
+    if Q.ndim == 3:
+        per_batch, M = 0, Q.shape[1]
+        assert Q.shape == (H, M, D)
+    else:
+        per_batch, M = 1, Q.shape[2]
+        assert Q.shape == (B, H, M, D)
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    lens, lp = _lens(lengths, B)
+    Z = np.empty((B, H, M, D), dtype=np.float64)
+    lse = np.empty((B, H, M), dtype=np.float64) if return_lse else None
+    _load().flare_oracle_encode(_dptr(Q), per_batch, _dptr(K), _dptr(V), lp, float(scale),
+                                B, H, N, M, D, _dptr(Z), _dptr(lse))
+    return (Z, lse) if return_lse else Z
+
+
+def decode(K, Q, Z, lengths=None, scale: Optional[float] = None, rows=None) -> np.ndarray:
+    """eq. 6 (FLARE decoder) / eq. 11 (decode with Q(X)).
+
+    K [B][H][N][D]; Q [H][M][D] or [B][H][M][D]; Z [B][H][M][D].
+    ``rows``: optional token indices (same for every head); the output is then
+    [B][H][len(rows)][D].  Masked tokens (n >= lengths[b]) give zero rows."""
+    K, Q, Z = _f64(K), _f64(Q), _f64(Z)
+    B, H, N, D = K.shape
+    if Q.ndim == 3:
+        per_batch, M = 0, Q.shape[1]
+    else:
+        per_batch, M = 1, Q.shape[2]
+    assert Z.shape == (B, H, M, D)
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    lens, lp = _lens(lengths, B)
+    if rows is None:
+        rp, nrows = None, N
+    else:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        assert rows.ndim == 1 and (rows.size == 0 or (rows.min() >= 0 and rows.max() < N))
+        rp, nrows = rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), rows.size
+    Y = np.empty((B, H, nrows, D), dtype=np.float64)
+    _load().flare_oracle_decode(_dptr(K), _dptr(Q), per_batch, _dptr(Z), lp, float(scale),
+                                B, H, N, M, D, rp, nrows, _dptr(Y))
+    return Y
+
+
+def flare_forward(K, V, Q, lengths=None, scale=None, rows=None) -> dict:
+    """FLARE mixer (section "FLARE: fixed-query latent routing", eq. 5-6)."""
+    Z = encode(Q, K, V, lengths, scale)
+    Y = decode(K, Q, Z, lengths, scale, rows)
+    return {"Z": Z, "Y": Y}
+
+
+def flarepp_forward(X, Wk, Wv, Wk_syn, Wv_syn, Q0, H: int, lengths=None, scale=None,
+                    rows=None, keep_projections: bool = False) -> dict:
+    """FLARE++ mixer (section "FLARE++: dynamic token routing", eq. 7-11):
+    K~ = X W~_K, V~ = X W~_V, Q(X) = SDPA(Q~, K~, V~); K = X W_K, V = X W_V,
+    Z = SDPA(Q(X), K, V), Y = SDPA(K, Q(X), Z)."""
+    Kt = project(X, Wk_syn, H)
+    Vt = project(X, Wv_syn, H)
+    Qx = encode(Q0, Kt, Vt, lengths, scale)
+    if not keep_projections:
+        del Kt, Vt
+    K = project(X, Wk, H)
+    V = project(X, Wv, H)
+    Z = encode(Qx, K, V, lengths, scale)
+    Y = decode(K, Qx, Z, lengths, scale, rows)
+    out = {"Qx": Qx, "Z": Z, "Y": Y}
+    if keep_projections:
+        out.update(Kt=Kt, Vt=Vt, K=K, V=V)
+    return out
+
+
+def forward_workload(w, rows=None, keep_projections: bool = False) -> dict:
+    """Run the oracle on a ``workloads.Workload`` (bf16 bits widened to fp64)."""
+    from workloads import bf16_bits_to_f64 as f64
+    if w.variant == "flare":
+        return flare_forward(f64(w.K), f64(w.V), f64(w.Q), w.lengths, w.scale, rows)
+    return flarepp_forward(f64(w.X), f64(w.Wk), f64(w.Wv), f64(w.Wk_syn), f64(w.Wv_syn),
+                           f64(w.Q0), w.H, w.lengths, w.scale, rows, keep_projections)

@@ -1,0 +1,80 @@
+"""The oracle pins must catch plausible mistakes in the oracle.
+
+Each case compiles a copy of ``oracle/flare_oracle.c`` with one planted mistake
+(a dropped term, a wrong index, a transposed operand, an off-by-one mask),
+swaps it in, and checks that at least one pin of ``test_oracle_pins`` fails.
+Everything runs on the CPU.
+"""
+import contextlib
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import tests.test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "flare_oracle.c")
+
+MUTATIONS = {
+    "decode_exp_drops_scale": ("double p = exp(scale * dot(k, Qg + m * D, D) - nu);",
+                               "double p = exp(dot(k, Qg + m * D, D) - nu);"),
+    "encode_wrong_normaliser": ("den += w;", "den += 1.0;"),
+    "encode_uses_keys_as_values": ("z[d] += w * Vh[n * D + d];", "z[d] += w * Kh[n * D + d];"),
+    "project_transposed_weight": ("x[c] * W[c * C + h * D + d]", "x[c] * W[(h * D + d) * C + c]"),
+    "decode_mask_off_by_one": ("if (n >= L) continue;", "if (n > L) continue;"),
+    "encode_mask_ignored": ("long L = valid_len(lengths, b, N);\n        for (long d = 0; d < D; ++d) z[d] = 0.0;",
+                            "long L = N;\n        for (long d = 0; d < D; ++d) z[d] = 0.0;"),
+    "encode_query_group_ignores_batch": ("long g = q_per_batch ? b * H + h : h;\n        const double *q",
+                                         "long g = h;\n        const double *q"),
+    "decode_max_not_subtracted_sign": ("double p = exp(scale * dot(k, Qg + m * D, D) - nu);",
+                                       "double p = exp(scale * dot(k, Qg + m * D, D) + nu);"),
+}
+
+PIN_FUNCS = [
+    lambda m: pins.test_flarepp_matches_torch_sdpa_chain(m, True),
+    lambda m: pins.test_flare_matches_torch_sdpa_chain(m),
+    lambda m: pins.test_project_matches_matmul(m),
+    lambda m: pins.test_materialised_mixing_matrix(m, "flarepp"),
+    lambda m: pins.test_two_tokens_one_latent_closed_form(m),
+    lambda m: pins.test_identical_keys_give_token_mean(m),
+    lambda m: pins.test_zero_queries_give_uniform_routing(m),
+    lambda m: pins.test_zero_seeds_give_mean_synthesis_values(m),
+    lambda m: pins.test_mask_equals_truncation(m),
+    lambda m: pins.test_hard_max_limit(m),
+]
+
+
+@contextlib.contextmanager
+def mutated_oracle(tmp_path, name):
+    old, new = MUTATIONS[name]
+    text = open(SRC).read()
+    assert text.count(old) == 1, name
+    src = tmp_path / f"{name}.c"
+    src.write_text(text.replace(old, new))
+    so = tmp_path / f"lib{name}.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fPIC",
+                    "-shared", "-o", str(so), str(src), "-lm"], check=True)
+    good = oracle._load()
+    bad = ctypes.CDLL(str(so))
+    for fn in ("flare_oracle_project", "flare_oracle_encode", "flare_oracle_decode"):
+        getattr(bad, fn).argtypes = getattr(good, fn).argtypes
+        getattr(bad, fn).restype = None
+    oracle._lib = bad
+    try:
+        yield
+    finally:
+        oracle._lib = good
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(tmp_path, name):
+    failures = 0
+    with mutated_oracle(tmp_path, name):
+        for f in PIN_FUNCS:
+            try:
+                f(oracle)
+            except AssertionError:
+                failures += 1
+    assert failures >= 1, f"no pin caught the planted mistake {name}"
