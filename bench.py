@@ -1,0 +1,458 @@
+#!/usr/bin/env python
+"""Benchmark of the FLARE++ mixer forward on B200.
+
+One step = one ``flarepp_mixer_fwd`` call over the N = 1,048,576-token
+workload (B=1, C=128, H=8, D=16, M=512; 3-D point cloud lifted to C features):
+the four per-head projections, the query-synthesis encode, the encode with
+the synthesised queries, both log-sum-exp merges and the decode.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  ``value`` is whole-job token*heads/s with the
+inputs resident in HBM, timed with CUDA events on the launching stream over
+exactly K steps (max over ranks).  ``e2e`` is the same metric with the
+host->device copy of the step's inputs (pinned memory) and the device->host
+copy of Y inside the timed region.  ``roofline`` reports the dominant kernel
+against the exp-unit (MUFU) peak, ``cpu_baseline`` the fp64 oracle on a
+bounded sample of the same workload on this host's cores.  ``--impl
+reference`` times the oracle itself as the reference arm.
+
+With ``--gpus N`` (launched through torch.distributed.run) every rank runs an
+independent copy of the workload on its own synthetic input (weak scaling; the
+heads and samples of the mixer are independent, so there is no data-path
+collective).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import make_workload  # noqa: E402
+
+METRIC = "mixer fwd token·heads/s at N=1M (1×B200) and % of roofline (HBM/MMA/MUFU)"
+UNIT = "token·heads/s"
+WORKLOAD = "flarepp_n1m_mesh3d"
+MUFU_PER_CLK_PER_SM = 16          # ex2 results per clock per SM (special-function unit)
+NUM_SM = 148
+STAGES_PP = ["project", "synth_encode", "synth_merge", "encode", "merge", "decode"]
+KERNEL_SOURCES = {"project": "project.cu", "synth_encode": "encode.cu", "encode": "encode.cu",
+                  "synth_merge": "merge.cu", "merge": "merge.cu", "decode": "decode.cu"}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "sm_max_mhz": d.get("sm_max_mhz", 1965.0), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0,
+            "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML, read only)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x4: "sw_power_cap", 0x1: "gpu_idle",
+               0x2: "applications_clocks_setting", 0x100: "sync_boost"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception as e:  # pragma: no cover - depends on the host
+            log("clock sampling unavailable:", e)
+        self.period = period_s
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._ok:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per stage (FLARE++), per launch
+# ---------------------------------------------------------------------------
+
+def stage_work(w):
+    B, N, C, H, D, M = w.B, w.N, w.C, w.H, w.D, w.M
+    Nv = w.valid_tokens() // B if w.lengths is not None else N
+    th = B * H * Nv                                   # token*heads
+    proj_bytes = B * N * C * 2 + 4 * C * C * 2 + 4 * B * H * N * D * 2
+    enc_exps = th * M                                 # one exponential per (latent, token) score
+    enc_flops = 4 * th * M * D                        # Q K^T and P V
+    enc_bytes = 2 * B * H * N * D * 2
+    dec_bytes = 2 * B * H * N * D * 2                 # read K, write Y
+    return {
+        "project": {"bytes": proj_bytes, "flops": 8 * B * N * C * C, "exps": 0},
+        "synth_encode": {"bytes": enc_bytes, "flops": enc_flops, "exps": enc_exps},
+        "synth_merge": {"bytes": 0, "flops": 0, "exps": 0},
+        "encode": {"bytes": enc_bytes, "flops": enc_flops, "exps": enc_exps},
+        "merge": {"bytes": 0, "flops": 0, "exps": 0},
+        "decode": {"bytes": dec_bytes, "flops": enc_flops, "exps": enc_exps},
+    }
+
+
+def kernel_traffic(kernel_file: str, workload: str):
+    """dram bytes per launch from a committed ncu summary, if that summary was
+    taken on the current source of the kernel (else None)."""
+    prof = os.path.join(ROOT, "profiles")
+    src = os.path.join(ROOT, "rank_latent_routing_flare_b200", "csrc", kernel_file)
+    if not os.path.isdir(prof) or not os.path.exists(src):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    for f in sorted(os.listdir(prof)):
+        if not f.endswith(".md"):
+            continue
+        text = open(os.path.join(prof, f)).read()
+        m_src = re.search(r"kernel_source_sha256_16:\s*(\w+)", text)
+        m_w = re.search(r"workload:\s*(\S+)", text)
+        m_k = re.search(r"kernel_file:\s*(\S+)", text)
+        m_t = re.search(r"dram_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text)
+        if m_src and m_t and m_k and m_w and m_src.group(1) == sha and m_k.group(1) == kernel_file \
+                and m_w.group(1) == workload:
+            return float(m_t.group(1))
+    return None
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample of the workload
+# ---------------------------------------------------------------------------
+
+def oracle_sample_rate(w, target_s: float):
+    import oracle
+    from workloads import bf16_bits_to_f64 as f64
+    oracle.build()
+    W = [f64(a) for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn)]
+    Q0 = f64(w.Q0)
+
+    def run(ns):
+        X = f64(w.X[:, :ns])
+        t0 = time.perf_counter()
+        oracle.flarepp_forward(X, *W, Q0, w.H, None, w.scale)
+        return time.perf_counter() - t0
+
+    ns = min(4096, w.N)
+    t = run(ns)
+    while t < target_s / 4 and ns < w.N:
+        ns = min(w.N, int(ns * min(8.0, max(2.0, target_s / max(t, 1e-3)))))
+        t = run(ns)
+    rate = w.B * w.H * ns / t
+    return rate, ns, t, oracle.num_threads()
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle timed as it stands
+# ---------------------------------------------------------------------------
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    w = make_workload(args.workload)
+    import oracle
+    from workloads import bf16_bits_to_f64 as f64
+    oracle.build()
+    W = [f64(a) for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn)]
+    Q0 = f64(w.Q0)
+    # each step: the full FLARE++ forward on a bounded token sample, sized so
+    # that the whole run stays within a few minutes
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    rate, ns, t, threads = oracle_sample_rate(w, min(budget, 20.0))
+    X = f64(w.X[:, :ns])
+    for _ in range(args.warmup):
+        oracle.flarepp_forward(X, *W, Q0, w.H, None, w.scale)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.flarepp_forward(X, *W, Q0, w.H, None, w.scale)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = w.B * w.H * ns / dt
+    sample = (f"FLARE++ forward (projections, synthesis, encode, decode) on the first {ns} of "
+              f"{w.N} tokens, B={w.B} H={w.H} M={w.M} D={w.D} C={w.C}; fp64 oracle, {threads} threads, "
+              f"{cpu_model()}")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "N": w.N, "C": w.C, "H": w.H, "D": w.D, "M": w.M,
+                       "sample_tokens": ns},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        log("warm-up raised to the minimum of 3 steps")
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    import rank_latent_routing_flare_b200 as fl
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    fl.load_library()
+
+    # inputs: each rank its own synthetic sample of the workload (weak scaling)
+    w = make_workload(args.workload, seed=None if rank == 0 else 1000 + rank)
+    assert w.variant == "flarepp"
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    X = to_dev(w.X)
+    Ws = [to_dev(a) for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn)]
+    Q0 = to_dev(w.Q0)
+    lengths = None if w.lengths is None else torch.from_numpy(w.lengths).to(dev)
+    Y = torch.empty((w.B, w.H, w.N, w.D), dtype=torch.bfloat16, device=dev)
+    nbytes = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLAREPP, w.B, w.H, w.N, w.M, w.D, w.C)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+
+    def step(events=None):
+        fl.flarepp_mixer_fwd(X, *Ws, Q0, lengths=lengths, Y=Y, workspace=ws, stream=stream, check=False,
+                             stage_events=events)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st = fl.flare_last_device_status(ws)
+    if st != fl.Status.OK:
+        raise RuntimeError(f"device status after warm-up: {st!r}")
+
+    # ---------------- timed region (inputs resident in HBM) ----------------
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(stage_ev[i])
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    th_per_rank = w.B * w.H * (w.valid_tokens() // w.B if w.lengths is not None else w.N)
+    value = world * th_per_rank / (ms * 1e-3)
+
+    # per-stage device times (same timed steps, same stream)
+    stage_ms = {s: 0.0 for s in STAGES_PP}
+    for evs in stage_ev:
+        for j, s in enumerate(STAGES_PP):
+            stage_ms[s] += evs[j].elapsed_time(evs[j + 1]) / args.steps
+    work = stage_work(w)
+    peaks = load_peaks()
+    clk = clocks.summary()
+    mufu_peak_max = MUFU_PER_CLK_PER_SM * NUM_SM * peaks["sm_max_mhz"] * 1e6
+    stages = {}
+    for s in STAGES_PP:
+        t = stage_ms[s] * 1e-3
+        wk = work[s]
+        stages[s] = {"ms": round(stage_ms[s], 4),
+                     "GB_s": round(wk["bytes"] / t / 1e9, 1) if wk["bytes"] else None,
+                     "TFLOP_s": round(wk["flops"] / t / 1e12, 2) if wk["flops"] else None,
+                     "Gexp_s": round(wk["exps"] / t / 1e9, 1) if wk["exps"] else None}
+    # the dominant kernel: largest share of the step (the two encoder launches
+    # are one kernel)
+    kern_ms = {"encode": stage_ms["synth_encode"] + stage_ms["encode"], "decode": stage_ms["decode"],
+               "project": stage_ms["project"], "merge": stage_ms["synth_merge"] + stage_ms["merge"]}
+    dom = max(kern_ms, key=kern_ms.get)
+    if dom in ("encode", "decode"):
+        per_launch_ms = kern_ms[dom] / (2 if dom == "encode" else 1)
+        exps = work["encode" if dom == "encode" else "decode"]["exps"]
+        achieved = exps / (per_launch_ms * 1e-3) / 1e9
+        roof = {"kernel": f"{dom}_kernel", "bound": "alu", "achieved": round(achieved, 1),
+                "peak": round(mufu_peak_max / 1e9, 1), "unit": "Gexp/s",
+                "frac": round(achieved / (mufu_peak_max / 1e9), 4),
+                "peak_basis": f"{MUFU_PER_CLK_PER_SM} ex2/clk/SM x {NUM_SM} SMs x {peaks['sm_max_mhz']:.0f} MHz",
+                "per_launch_ms": round(per_launch_ms, 4),
+                "traffic": kernel_traffic(f"{dom}.cu", w.name)}
+        if clk.get("sm_mhz"):
+            roof["frac_at_observed_clock"] = round(
+                achieved / (MUFU_PER_CLK_PER_SM * NUM_SM * clk["sm_mhz"] * 1e-3), 4)
+    elif dom == "project":
+        per = kern_ms[dom]
+        achieved = work["project"]["bytes"] / (per * 1e-3) / 1e9
+        roof = {"kernel": "project_kernel", "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "per_launch_ms": round(per, 4), "traffic": kernel_traffic("project.cu", w.name)}
+    else:
+        roof = {"kernel": "merge_kernel", "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": None, "traffic": None}
+    roof["peak_source"] = peaks["source"]
+    # whole-step roofline of the benchmark spec: max(bytes/HBM, MMA/tensor, exps/MUFU)
+    tot_bytes = 3 * w.B * w.N * w.C * 2 + w.B * w.H * w.N * w.D * 2
+    tot_exps = sum(work[s]["exps"] for s in STAGES_PP)
+    tot_flops = sum(work[s]["flops"] for s in STAGES_PP)
+    t_roof = max(tot_bytes / (peaks["hbm_gbs"] * 1e9), tot_flops / (peaks["bf16_tflops"] * 1e12),
+                 tot_exps / mufu_peak_max)
+    step_roofline = {"t_roof_ms": round(t_roof * 1e3, 4), "frac": round(t_roof / (ms * 1e-3), 4),
+                     "terms_ms": {"hbm": round(tot_bytes / (peaks["hbm_gbs"] * 1e9) * 1e3, 4),
+                                  "mma": round(tot_flops / (peaks["bf16_tflops"] * 1e12) * 1e3, 4),
+                                  "mufu": round(tot_exps / mufu_peak_max * 1e3, 4)}}
+
+    # ---------------- end to end through the public API ----------------
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).pin_memory()  # noqa: E731
+    hX = pin(w.X)
+    hW = [pin(a) for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn)]
+    hQ0 = pin(w.Q0)
+    hY = torch.empty((w.B, w.H, w.N, w.D), dtype=torch.int16).pin_memory()
+    dX = X.view(torch.int16)
+    dW = [a.view(torch.int16) for a in Ws]
+    dQ0 = Q0.view(torch.int16)
+    h2d = hX.numel() * 2 + sum(a.numel() * 2 for a in hW) + hQ0.numel() * 2
+    d2h = hY.numel() * 2
+
+    def e2e_step():
+        dX.copy_(hX, non_blocking=True)
+        for d, h in zip(dW, hW):
+            d.copy_(h, non_blocking=True)
+        dQ0.copy_(hQ0, non_blocking=True)
+        step()
+        hY.copy_(Y.view(torch.int16), non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+    e2e_value = world * th_per_rank / (e2e_ms * 1e-3)
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            rate, ns, t, threads = oracle_sample_rate(w, args.cpu_seconds)
+            cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+                   "sample": f"fp64 oracle, full FLARE++ forward on the first {ns} of {w.N} tokens "
+                             f"(B={w.B} H={w.H} M={w.M} D={w.D} C={w.C}) in {t:.1f} s; {cpu_model()}"}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "N": w.N, "C": w.C, "H": w.H, "D": w.D, "M": w.M,
+                       "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": "inputs larger than L2 (X 256 MiB; K~,V~,K,V 1 GiB per step)"},
+            "roofline": roof,
+            "step_roofline": step_roofline,
+            "stages": stages,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": 6 * args.steps,
+            "clocks": clk,
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

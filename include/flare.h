@@ -1,0 +1,172 @@
+/*
+ * flare.h - C ABI of the B200 (sm_100a) FLARE / FLARE++ mixer forward.
+ *
+ * What the calls compute (FLARE++ paper, arXiv 2608.11519, section "Method"):
+ *
+ *   flare_mixer_fwd      FLARE, section "FLARE: fixed-query latent routing"
+ *                        (eq. 5-6): per head h, with learned queries Q_h (M x D)
+ *                          Z_h = softmax_n(Q_h K_h^T * scale) V_h        (encode)
+ *                          Y_h = softmax_m(K_h Q_h^T * scale) Z_h        (decode)
+ *
+ *   flarepp_mixer_fwd    FLARE++, section "FLARE++: dynamic token routing"
+ *                        (eq. 7-11): per head h
+ *                          K~_h = X W~_K,h,  V~_h = X W~_V,h             (eq. 7)
+ *                          Q_h(X) = softmax_n(Q~_h K~_h^T * scale) V~_h  (eq. 8)
+ *                          K_h = X W_K,h,  V_h = X W_V,h                 (eq. 9)
+ *                          Z_h = softmax_n(Q_h(X) K_h^T * scale) V_h     (eq. 10)
+ *                          Y_h = softmax_m(K_h Q_h(X)^T * scale) Z_h     (eq. 11)
+ *                        W_{.,h} is column block [h*D, (h+1)*D) of the C x C
+ *                        matrix W (section "Full self-attention": H heads of
+ *                        width D = C/H).
+ *
+ * The head concatenation and the output projection W_O are not part of these
+ * calls; Y is returned per head.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *   - bf16 tensors are passed as pointers to 16-bit bit patterns (flare_bf16),
+ *     float tensors as float*.  All tensors are dense, row-major, in DEVICE
+ *     memory, and every pointer must be 16-byte aligned.
+ *   - Layouts: X [B][N][C]; W [C][C] with K = X @ W (row-vector convention);
+ *     K, V, Y [B][H][N][D]; Q, Q0 [H][M][D] (shared by the whole batch);
+ *     debug outputs Q(X) and Z are float [B][H][M][D].
+ *   - Supported sizes: B, H, N >= 1; D in {16, 32}; M a multiple of 16 in
+ *     [16, 512]; FLARE++ also needs C = H*D, C a multiple of 64, C <= 256.
+ *   - lengths: optional DEVICE int32[B] (NULL = every token valid).  Tokens
+ *     n >= lengths[b] are padding: they are not keys of the synthesis and
+ *     encode softmaxes and their rows of Y are written as zeros.  A length
+ *     outside [1, N] is clamped to [0, N] and reported by
+ *     flare_last_device_status() as FLARE_ERR_SHAPE.
+ *   - scale <= 0 selects the default 1/sqrt(D).
+ *   - workspace: caller-owned DEVICE scratch of at least
+ *     flare_workspace_bytes(...) bytes, 256-byte aligned.  The library never
+ *     allocates or frees memory and keeps no state between calls; two calls
+ *     that may run concurrently need two workspaces.
+ *   - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Every call only enqueues work on that stream and returns; inputs must
+ *     stay valid until the stream has executed the work.  No call
+ *     synchronises except flare_last_device_status().
+ *   - Results are deterministic: the same inputs give bitwise-identical
+ *     outputs on every run (fixed split count and fixed merge order, no
+ *     floating-point atomics).
+ *   - Errors: argument errors are detected on the host before anything is
+ *     enqueued and returned as a flare_status.  A CUDA error while
+ *     enqueueing returns FLARE_ERR_LAUNCH.  Errors found while the kernels
+ *     run (a bounded wait that expired, an invalid length) are recorded in
+ *     the workspace and returned by flare_last_device_status().  No call
+ *     traps the device.
+ */
+#ifndef FLARE_H_
+#define FLARE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FLARE_API __attribute__((visibility("default")))
+#else
+#define FLARE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t flare_bf16; /* bfloat16 bit pattern */
+
+typedef enum {
+  FLARE_OK = 0,
+  FLARE_ERR_NULL = 1,        /* a required pointer is NULL                        */
+  FLARE_ERR_SHAPE = 2,       /* a size is out of range or inconsistent            */
+  FLARE_ERR_UNSUPPORTED = 3, /* valid math, but a size this build does not cover  */
+  FLARE_ERR_ALIGN = 4,       /* a pointer is not 16-byte (workspace: 256) aligned */
+  FLARE_ERR_WORKSPACE = 5,   /* workspace smaller than flare_workspace_bytes()    */
+  FLARE_ERR_LAUNCH = 6,      /* CUDA error while enqueueing (no sm_100 device...) */
+  FLARE_ERR_TIMEOUT = 7      /* a device-side bounded wait expired                */
+} flare_status;
+
+/* Variant selector for flare_workspace_bytes(). */
+#define FLARE_VARIANT_FLARE 0
+#define FLARE_VARIANT_FLAREPP 1
+
+/*
+ * Workspace size in bytes for one call with these sizes (C is ignored for
+ * FLARE).  Returns 0 when the sizes are not supported.  Pure host function.
+ */
+FLARE_API size_t flare_workspace_bytes(int variant, int B, int H, int N, int M, int D, int C);
+
+/*
+ * FLARE mixer forward (eq. 5-6).
+ *   K, V    [B][H][N][D] bf16, read only
+ *   Q       [H][M][D]    bf16, read only (learned latent queries)
+ *   Y       [B][H][N][D] bf16, written
+ *   Z_out   [B][H][M][D] float, written if not NULL (latent values, debug)
+ */
+FLARE_API flare_status flare_mixer_fwd(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, flare_bf16* Y,
+                             int B, int H, int N, int M, int D, const int32_t* lengths, float scale,
+                             void* workspace, size_t workspace_bytes, void* stream, float* Z_out);
+
+/*
+ * FLARE++ mixer forward (eq. 7-11).
+ *   X                       [B][N][C] bf16, read only
+ *   Wk, Wv, Wk_syn, Wv_syn  [C][C]    bf16, read only (W_K, W_V, W~_K, W~_V)
+ *   Q0                      [H][M][D] bf16, read only (learned seeds Q~)
+ *   Y                       [B][H][N][D] bf16, written
+ *   Qx_out, Z_out           [B][H][M][D] float, written if not NULL (the
+ *                           synthesised routing queries Q(X) and the latent
+ *                           values Z, for inspection)
+ */
+FLARE_API flare_status flarepp_mixer_fwd(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                               const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0,
+                               flare_bf16* Y, int B, int N, int C, int H, int M, int D,
+                               const int32_t* lengths, float scale, void* workspace, size_t workspace_bytes,
+                               void* stream, float* Qx_out, float* Z_out);
+
+/*
+ * Profiling variants: identical work, plus cudaEventRecord() of caller-created
+ * events (cudaEvent_t passed as void*) on `stream` between the stages, so a
+ * caller can time each kernel on the stream it runs on.  A NULL array (or a
+ * NULL entry) records nothing.
+ *   flare_mixer_fwd_profiled:   5 events around key norms | encode | merge |
+ *                               decode   (events[i] precedes stage i,
+ *                               events[4] follows the decode)
+ *   flarepp_mixer_fwd_profiled: 7 events around projections | synthesis
+ *                               encode | synthesis merge | encode | merge |
+ *                               decode   (events[6] follows the decode)
+ */
+FLARE_API flare_status flare_mixer_fwd_profiled(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q,
+                                                flare_bf16* Y, int B, int H, int N, int M, int D,
+                                                const int32_t* lengths, float scale, void* workspace,
+                                                size_t workspace_bytes, void* stream, float* Z_out,
+                                                void* const* stage_events);
+FLARE_API flare_status flarepp_mixer_fwd_profiled(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                                                  const flare_bf16* Wk_syn, const flare_bf16* Wv_syn,
+                                                  const flare_bf16* Q0, flare_bf16* Y, int B, int N, int C, int H,
+                                                  int M, int D, const int32_t* lengths, float scale,
+                                                  void* workspace, size_t workspace_bytes, void* stream,
+                                                  float* Qx_out, float* Z_out, void* const* stage_events);
+
+/*
+ * Synchronises `stream`, reads the device error word of `workspace` and
+ * returns FLARE_OK, FLARE_ERR_TIMEOUT or FLARE_ERR_SHAPE (invalid lengths).
+ * The word is cleared at the start of every mixer call.
+ */
+FLARE_API flare_status flare_last_device_status(void* workspace, void* stream);
+
+/* Static, human-readable name of a status. */
+FLARE_API const char* flare_status_string(flare_status status);
+
+/*
+ * Self-test of the bounded-wait error path: enqueues one small kernel that
+ * waits on an mbarrier nothing ever completes, with a limit of `timeout_ns`
+ * nanoseconds (clamped to [1e3, 1e9]).  The wait expires, the kernel records
+ * FLARE_ERR_TIMEOUT in the workspace error word and returns normally; read
+ * it with flare_last_device_status().  workspace needs 256 bytes.
+ */
+FLARE_API flare_status flare_selftest_wait_timeout(void* workspace, void* stream, unsigned long long timeout_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLARE_H_ */

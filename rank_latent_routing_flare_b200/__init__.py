@@ -1,0 +1,22 @@
+"""B200 (sm_100a) FLARE / FLARE++ mixer forward.
+
+The compute lives in ``libflare.so`` (hand-written CUDA kernels behind the C
+ABI of ``include/flare.h``).  This package is a thin ctypes binding: it checks
+tensor types, passes device pointers and sizes, and raises ``FlareError`` on a
+non-OK status.  PyTorch only provides device memory and streams.  There is no
+CPU fallback: if the library cannot be loaded, every call raises.
+"""
+from ._binding import (  # noqa: F401
+    FLARE_VARIANT_FLARE,
+    FLARE_VARIANT_FLAREPP,
+    FlareError,
+    Status,
+    flare_last_device_status,
+    flare_mixer_fwd,
+    flare_selftest_wait_timeout,
+    flare_status_string,
+    flare_workspace_bytes,
+    flarepp_mixer_fwd,
+    library_path,
+    load_library,
+)

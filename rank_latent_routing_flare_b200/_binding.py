@@ -1,0 +1,207 @@
+"""ctypes binding of include/flare.h (argument marshalling only)."""
+from __future__ import annotations
+
+import ctypes
+import enum
+import os
+import threading
+from typing import Optional
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libflare.so")
+_lock = threading.Lock()
+_lib = None
+
+FLARE_VARIANT_FLARE = 0
+FLARE_VARIANT_FLAREPP = 1
+
+
+class Status(enum.IntEnum):
+    OK = 0
+    ERR_NULL = 1
+    ERR_SHAPE = 2
+    ERR_UNSUPPORTED = 3
+    ERR_ALIGN = 4
+    ERR_WORKSPACE = 5
+    ERR_LAUNCH = 6
+    ERR_TIMEOUT = 7
+
+
+class FlareError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = Status(status)
+        super().__init__(f"{where}: {flare_status_string(status)}")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library(build_if_missing: bool = True):
+    """Load libflare.so, compiling it with nvcc first if it is missing or stale."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        from . import build as _build
+        if build_if_missing and not _build.up_to_date():
+            _build.build()
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"FLARE CUDA library not found at {_LIB_PATH}")
+        lib = ctypes.CDLL(_LIB_PATH)
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        lib.flare_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+        lib.flare_workspace_bytes.restype = sz
+        lib.flare_mixer_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, vp, f, vp, sz, vp, vp]
+        lib.flare_mixer_fwd.restype = i
+        lib.flarepp_mixer_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, f, vp, sz, vp, vp, vp]
+        lib.flarepp_mixer_fwd.restype = i
+        lib.flare_mixer_fwd_profiled.argtypes = lib.flare_mixer_fwd.argtypes + [vp]
+        lib.flare_mixer_fwd_profiled.restype = i
+        lib.flarepp_mixer_fwd_profiled.argtypes = lib.flarepp_mixer_fwd.argtypes + [vp]
+        lib.flarepp_mixer_fwd_profiled.restype = i
+        lib.flare_last_device_status.argtypes = [vp, vp]
+        lib.flare_last_device_status.restype = i
+        lib.flare_status_string.argtypes = [i]
+        lib.flare_status_string.restype = ctypes.c_char_p
+        lib.flare_selftest_wait_timeout.argtypes = [vp, vp, ctypes.c_ulonglong]
+        lib.flare_selftest_wait_timeout.restype = i
+        _lib = lib
+        return lib
+
+
+def flare_status_string(status: int) -> str:
+    return load_library().flare_status_string(int(status)).decode()
+
+
+def flare_workspace_bytes(variant: int, B: int, H: int, N: int, M: int, D: int, C: int = 0) -> int:
+    return int(load_library().flare_workspace_bytes(variant, B, H, N, M, D, C))
+
+
+# ----------------------------------------------------------------------------
+# torch helpers (plumbing only)
+# ----------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _check_dev(name, t, dtype, shape=None):
+    torch = _torch()
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _stream_ptr(stream, device) -> int:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return int(stream.cuda_stream)
+
+
+def _workspace(workspace, nbytes, device):
+    torch = _torch()
+    if workspace is None:
+        return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+    _check_dev("workspace", workspace, torch.uint8)
+    if workspace.numel() < nbytes:
+        raise ValueError(f"workspace has {workspace.numel()} bytes, needs {nbytes}")
+    return workspace
+
+
+def _event_array(events):
+    """cudaEvent_t handles of torch.cuda.Event objects (each recorded once so
+    that its handle exists) as a ctypes void* array."""
+    if events is None:
+        return None
+    handles = []
+    for e in events:
+        if e.cuda_event == 0:
+            e.record()
+        handles.append(e.cuda_event)
+    return (ctypes.c_void_p * len(handles))(*handles)
+
+
+def flare_mixer_fwd(K, V, Q, lengths=None, scale: float = 0.0, Y=None, workspace=None, stream=None,
+                    Z_out=None, check: bool = True, stage_events=None):
+    """FLARE forward (eq. 5-6).  K, V: [B,H,N,D] bf16; Q: [H,M,D] bf16 -> Y [B,H,N,D] bf16."""
+    torch = _torch()
+    B, H, N, D = K.shape
+    M = Q.shape[1]
+    if check:
+        _check_dev("K", K, torch.bfloat16)
+        _check_dev("V", V, torch.bfloat16, K.shape)
+        _check_dev("Q", Q, torch.bfloat16, (H, M, D))
+        _check_dev("lengths", lengths, torch.int32, (B,))
+        _check_dev("Z_out", Z_out, torch.float32, (B, H, M, D))
+    if Y is None:
+        Y = torch.empty_like(K)
+    nbytes = flare_workspace_bytes(FLARE_VARIANT_FLARE, B, H, N, M, D)
+    workspace = _workspace(workspace, nbytes, K.device)
+    args = (_ptr(K), _ptr(V), _ptr(Q), _ptr(Y), B, H, N, M, D, _ptr(lengths), float(scale), _ptr(workspace),
+            workspace.numel(), _stream_ptr(stream, K.device), _ptr(Z_out))
+    if stage_events is None:
+        st = load_library().flare_mixer_fwd(*args)
+    else:
+        assert len(stage_events) == 5
+        st = load_library().flare_mixer_fwd_profiled(*args, _event_array(stage_events))
+    if st != 0:
+        raise FlareError(st, "flare_mixer_fwd")
+    return Y
+
+
+def flarepp_mixer_fwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, lengths=None, scale: float = 0.0, Y=None,
+                      workspace=None, stream=None, Qx_out=None, Z_out=None, check: bool = True,
+                      stage_events=None):
+    """FLARE++ forward (eq. 7-11).  X: [B,N,C] bf16; W*: [C,C] bf16; Q0: [H,M,D] bf16
+    -> Y [B,H,N,D] bf16."""
+    torch = _torch()
+    B, N, C = X.shape
+    H, M, D = Q0.shape
+    if check:
+        _check_dev("X", X, torch.bfloat16)
+        for nm, w in (("Wk", Wk), ("Wv", Wv), ("Wk_syn", Wk_syn), ("Wv_syn", Wv_syn)):
+            _check_dev(nm, w, torch.bfloat16, (C, C))
+        _check_dev("Q0", Q0, torch.bfloat16)
+        _check_dev("lengths", lengths, torch.int32, (B,))
+        _check_dev("Qx_out", Qx_out, torch.float32, (B, H, M, D))
+        _check_dev("Z_out", Z_out, torch.float32, (B, H, M, D))
+    if Y is None:
+        Y = torch.empty((B, H, N, D), dtype=torch.bfloat16, device=X.device)
+    nbytes = flare_workspace_bytes(FLARE_VARIANT_FLAREPP, B, H, N, M, D, C)
+    workspace = _workspace(workspace, nbytes, X.device)
+    args = (_ptr(X), _ptr(Wk), _ptr(Wv), _ptr(Wk_syn), _ptr(Wv_syn), _ptr(Q0), _ptr(Y), B, N, C, H, M, D,
+            _ptr(lengths), float(scale), _ptr(workspace), workspace.numel(), _stream_ptr(stream, X.device),
+            _ptr(Qx_out), _ptr(Z_out))
+    if stage_events is None:
+        st = load_library().flarepp_mixer_fwd(*args)
+    else:
+        assert len(stage_events) == 7
+        st = load_library().flarepp_mixer_fwd_profiled(*args, _event_array(stage_events))
+    if st != 0:
+        raise FlareError(st, "flarepp_mixer_fwd")
+    return Y
+
+
+def flare_last_device_status(workspace, stream=None) -> Status:
+    return Status(load_library().flare_last_device_status(_ptr(workspace), _stream_ptr(stream, workspace.device)))
+
+
+def flare_selftest_wait_timeout(workspace, timeout_ns: int, stream=None) -> None:
+    st = load_library().flare_selftest_wait_timeout(_ptr(workspace), _stream_ptr(stream, workspace.device),
+                                                    int(timeout_ns))
+    if st != 0:
+        raise FlareError(st, "flare_selftest_wait_timeout")

@@ -1,0 +1,384 @@
+// Host entry points of the C ABI declared in include/flare.h: argument
+// validation (before anything is enqueued), workspace layout, TMA tensor maps
+// and the launch sequence of the FLARE / FLARE++ forward.
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "flare.h"
+#include "flare_internal.h"
+
+namespace flare {
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn tensor_map_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+unsigned long long wait_timeout_ns() {
+  static unsigned long long t = [] {
+    const char* e = std::getenv("FLARE_WAIT_TIMEOUT_NS");
+    unsigned long long v = e ? std::strtoull(e, nullptr, 10) : 0ull;
+    return v > 0 ? v : 4000000000ull;  // 4 s per wait
+  }();
+  return t;
+}
+
+// 3-D bf16 tensor map: dims (d0 innermost, d1, d2), dense, box (b0, b1, 1).
+bool map3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1,
+           CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = tensor_map_encoder();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  const cuuint32_t box[3] = {b0, b1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool map2d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint32_t b0, uint32_t b1,
+           CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = tensor_map_encoder();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {d0, d1};
+  const cuuint64_t strides[1] = {d0 * 2};
+  const cuuint32_t box[2] = {b0, b1};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+CUtensorMapSwizzle row_swizzle(int D) { return D == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+long cdiv(long a, long b) { return (a + b - 1) / b; }
+
+// Number of token splits of the encoder: at least 8 tiles per split, chosen
+// to fill the SMs' CTA slots in whole waves.  Depends on the sizes only, so a
+// given problem always uses the same split count (and gives the same bits).
+int choose_splits(long units, long ntiles) {
+  const long slots = static_cast<long>(kNumSM) * kSlotsPerSM;
+  const long smax = std::max(1L, std::min(ntiles / 8, 1024L));
+  int best = 1;
+  double best_eff = -1.0;
+  for (long s = 1; s <= smax; ++s) {
+    const long ctas = units * s;
+    const long waves = cdiv(ctas, slots);
+    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = static_cast<int>(s);
+    }
+  }
+  return best;
+}
+
+struct Plan {
+  int S = 1, tps = 1, LB = 1;            // encoder splits, tiles per split, latent blocks
+  int dec_ctas = 1, dec_tiles = 1;       // decoder CTAs per head, tiles per CTA
+  int G32 = 1;
+  size_t off_err = 0, off_kt = 0, off_vt = 0, off_kp = 0, off_vp = 0, off_kn_syn = 0, off_kn = 0, off_part = 0,
+         off_qx32 = 0, off_qx16 = 0, off_z32 = 0, off_z16 = 0, total = 0;
+};
+
+Plan make_plan(int variant, long B, long H, long N, long M, long D) {
+  Plan p;
+  const long BH = B * H;
+  const long ntiles = cdiv(N, kEncTile);
+  p.LB = static_cast<int>(cdiv(M, kLatBlock));
+  p.S = choose_splits(BH * p.LB, ntiles);
+  p.tps = static_cast<int>(cdiv(ntiles, p.S));
+  p.S = static_cast<int>(cdiv(ntiles, p.tps));
+  const long dtiles = cdiv(N, kDecTile);
+  long per = std::max(1L, static_cast<long>(kNumSM) * kSlotsPerSM / BH);
+  per = std::min(per, dtiles);
+  p.dec_tiles = static_cast<int>(cdiv(dtiles, per));
+  p.dec_ctas = static_cast<int>(cdiv(dtiles, p.dec_tiles));
+  p.G32 = static_cast<int>(cdiv(N, kNormGroup));
+  size_t off = 0;
+  p.off_err = off;
+  off += 256;
+  const size_t proj = align256(static_cast<size_t>(BH * N * D) * 2);
+  if (variant == FLARE_VARIANT_FLAREPP) {
+    p.off_kt = off; off += proj;
+    p.off_vt = off; off += proj;
+    p.off_kp = off; off += proj;
+    p.off_vp = off; off += proj;
+    p.off_kn_syn = off; off += align256(static_cast<size_t>(BH) * p.G32 * 4);
+  }
+  p.off_kn = off; off += align256(static_cast<size_t>(BH) * p.G32 * 4);
+  p.off_part = off; off += align256(static_cast<size_t>(BH) * p.S * M * (D + 2) * 4);
+  const size_t lat32 = align256(static_cast<size_t>(BH * M * D) * 4), lat16 = align256(static_cast<size_t>(BH * M * D) * 2);
+  if (variant == FLARE_VARIANT_FLAREPP) {
+    p.off_qx32 = off; off += lat32;
+    p.off_qx16 = off; off += lat16;
+  }
+  p.off_z32 = off; off += lat32;
+  p.off_z16 = off; off += lat16;
+  p.total = off;
+  return p;
+}
+
+// Records stage event i (a cudaEvent_t passed as void*) when profiling is on.
+bool record(void* const* ev, int i, cudaStream_t s) {
+  if (ev == nullptr || ev[i] == nullptr) return true;
+  return cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) == cudaSuccess;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+flare_status check_common(int B, int H, int N, int M, int D) {
+  if (B < 1 || H < 1 || N < 1 || M < 1 || D < 1) return FLARE_ERR_SHAPE;
+  if (D != 16 && D != 32) return FLARE_ERR_UNSUPPORTED;
+  if (M % 16 != 0 || M > 512) return FLARE_ERR_UNSUPPORTED;
+  // element offsets stay below 2^31 per head row index; whole tensors may be larger
+  if (static_cast<long>(N) * D >= (1L << 31) || static_cast<long>(B) * H > (1L << 20)) return FLARE_ERR_UNSUPPORTED;
+  return FLARE_OK;
+}
+
+float resolve_scale(float scale, int D) { return scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(D)); }
+
+// Encoder pass + merge: queries (bf16, [G][M][D]) against keys/values.
+flare_status run_encode(const Plan& pl, uint8_t* ws, const void* q, int q_per_batch, const void* k, const void* v,
+                        const float* knorm, float* out32, uint16_t* out16, int B, int H, int N, int M, int D,
+                        const int32_t* lengths, float scale, cudaStream_t st, void* const* ev, int ev0) {
+  const long BH = static_cast<long>(B) * H;
+  const long G = q_per_batch ? BH : H;
+  CUtensorMap tq, tk, tv;
+  if (!map3d(&tq, q, D, M, G, D, std::min(M, kLatBlock), row_swizzle(D)) ||
+      !map3d(&tk, k, D, N, BH, D, kEncTile, row_swizzle(D)) || !map3d(&tv, v, D, N, BH, D, kEncTile, row_swizzle(D)))
+    return FLARE_ERR_LAUNCH;
+  EncodeParams ep{};
+  ep.B = B; ep.H = H; ep.N = N; ep.M = M; ep.D = D;
+  ep.q_per_batch = q_per_batch;
+  ep.n_splits = pl.S; ep.tiles_per_split = pl.tps; ep.n_lblocks = pl.LB; ep.n_groups32 = pl.G32;
+  ep.q_rows = std::min(M, kLatBlock);
+  ep.c = scale * 1.4426950408889634f;
+  ep.lengths = lengths;
+  ep.knorm = knorm;
+  ep.q = static_cast<const uint16_t*>(q);
+  ep.part = reinterpret_cast<float*>(ws + pl.off_part);
+  ep.err = reinterpret_cast<uint32_t*>(ws + pl.off_err);
+  ep.timeout_ns = wait_timeout_ns();
+  if (launch_encode(tq, tk, tv, ep, st) != cudaSuccess || !record(ev, ev0, st)) return FLARE_ERR_LAUNCH;
+  MergeParams mp{};
+  mp.B = B; mp.H = H; mp.N = N; mp.M = M; mp.D = D;
+  mp.q_per_batch = q_per_batch;
+  mp.n_splits = pl.S; mp.tiles_per_split = pl.tps;
+  mp.scale = scale; mp.c = ep.c;
+  mp.lengths = lengths;
+  mp.part = ep.part;
+  mp.q = ep.q;
+  mp.k = static_cast<const uint16_t*>(k);
+  mp.v = static_cast<const uint16_t*>(v);
+  mp.out_f32 = out32;
+  mp.out_bf16 = out16;
+  if (launch_merge(mp, st) != cudaSuccess || !record(ev, ev0 + 1, st)) return FLARE_ERR_LAUNCH;
+  return FLARE_OK;
+}
+
+flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_batch, const uint16_t* z16,
+                        const void* k, void* y, int B, int H, int N, int M, int D, const int32_t* lengths,
+                        float scale, cudaStream_t st) {
+  const long BH = static_cast<long>(B) * H;
+  const long G = q_per_batch ? BH : H;
+  CUtensorMap tq, tz, tk;
+  const int chunk_rows = std::min(M, kDecChunk);
+  if (!map3d(&tq, q, D, M, G, D, chunk_rows, row_swizzle(D)) || !map3d(&tz, z16, D, M, BH, D, chunk_rows, row_swizzle(D)) ||
+      !map3d(&tk, k, D, N, BH, D, kDecTile, row_swizzle(D)))
+    return FLARE_ERR_LAUNCH;
+  DecodeParams dp{};
+  dp.B = B; dp.H = H; dp.N = N; dp.M = M; dp.D = D;
+  dp.q_per_batch = q_per_batch;
+  dp.tiles_per_cta = pl.dec_tiles; dp.ctas_per_head = pl.dec_ctas;
+  dp.chunk_rows = chunk_rows;
+  dp.scale = scale; dp.c = scale * 1.4426950408889634f;
+  dp.lengths = lengths;
+  dp.q = static_cast<const uint16_t*>(q);
+  dp.z = z16;
+  dp.k = static_cast<const uint16_t*>(k);
+  dp.y = static_cast<uint16_t*>(y);
+  dp.err = reinterpret_cast<uint32_t*>(ws + pl.off_err);
+  dp.timeout_ns = wait_timeout_ns();
+  if (launch_decode(tq, tz, tk, dp, st) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  return FLARE_OK;
+}
+
+}  // namespace
+}  // namespace flare
+
+using namespace flare;
+
+extern "C" {
+
+size_t flare_workspace_bytes(int variant, int B, int H, int N, int M, int D, int C) {
+  if (variant != FLARE_VARIANT_FLARE && variant != FLARE_VARIANT_FLAREPP) return 0;
+  if (check_common(B, H, N, M, D) != FLARE_OK) return 0;
+  if (variant == FLARE_VARIANT_FLAREPP && (C != H * D || C % 64 != 0 || C > 256)) return 0;
+  return make_plan(variant, B, H, N, M, D).total;
+}
+
+const char* flare_status_string(flare_status s) {
+  switch (s) {
+    case FLARE_OK: return "FLARE_OK";
+    case FLARE_ERR_NULL: return "FLARE_ERR_NULL: a required pointer is NULL";
+    case FLARE_ERR_SHAPE: return "FLARE_ERR_SHAPE: a size is out of range or inconsistent";
+    case FLARE_ERR_UNSUPPORTED: return "FLARE_ERR_UNSUPPORTED: size not covered by this build";
+    case FLARE_ERR_ALIGN: return "FLARE_ERR_ALIGN: pointer not 16-byte (workspace 256-byte) aligned";
+    case FLARE_ERR_WORKSPACE: return "FLARE_ERR_WORKSPACE: workspace too small";
+    case FLARE_ERR_LAUNCH: return "FLARE_ERR_LAUNCH: CUDA error while enqueueing";
+    case FLARE_ERR_TIMEOUT: return "FLARE_ERR_TIMEOUT: a device-side bounded wait expired";
+  }
+  return "unknown flare_status";
+}
+
+flare_status flare_mixer_fwd_profiled(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, flare_bf16* Y,
+                                      int B, int H, int N, int M, int D, const int32_t* lengths, float scale,
+                                      void* workspace, size_t workspace_bytes, void* stream, float* Z_out,
+                                      void* const* stage_events) {
+  if (!K || !V || !Q || !Y || !workspace) return FLARE_ERR_NULL;
+  flare_status st = check_common(B, H, N, M, D);
+  if (st != FLARE_OK) return st;
+  if (!aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(Y) || !aligned16(lengths) || !aligned16(Z_out) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FLARE_ERR_ALIGN;
+  const Plan pl = make_plan(FLARE_VARIANT_FLARE, B, H, N, M, D);
+  if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
+  const float sc = resolve_scale(scale, D);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(ws + pl.off_err, 0, 4, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  if (!record(stage_events, 0, s)) return FLARE_ERR_LAUNCH;
+  KnormParams kp{B * H, N, D, pl.G32, reinterpret_cast<const uint16_t*>(K), reinterpret_cast<float*>(ws + pl.off_kn)};
+  if (launch_knorm(kp, s) != cudaSuccess || !record(stage_events, 1, s)) return FLARE_ERR_LAUNCH;
+  float* z32 = Z_out ? Z_out : reinterpret_cast<float*>(ws + pl.off_z32);
+  uint16_t* z16 = reinterpret_cast<uint16_t*>(ws + pl.off_z16);
+  st = run_encode(pl, ws, Q, 0, K, V, kp.knorm, z32, z16, B, H, N, M, D, lengths, sc, s, stage_events, 2);
+  if (st != FLARE_OK) return st;
+  st = run_decode(pl, ws, Q, 0, z16, K, Y, B, H, N, M, D, lengths, sc, s);
+  if (st != FLARE_OK) return st;
+  return record(stage_events, 4, s) ? FLARE_OK : FLARE_ERR_LAUNCH;
+}
+
+flare_status flare_mixer_fwd(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, flare_bf16* Y, int B,
+                             int H, int N, int M, int D, const int32_t* lengths, float scale, void* workspace,
+                             size_t workspace_bytes, void* stream, float* Z_out) {
+  return flare_mixer_fwd_profiled(K, V, Q, Y, B, H, N, M, D, lengths, scale, workspace, workspace_bytes, stream,
+                                  Z_out, nullptr);
+}
+
+flare_status flarepp_mixer_fwd_profiled(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                                        const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0,
+                                        flare_bf16* Y, int B, int N, int C, int H, int M, int D,
+                                        const int32_t* lengths, float scale, void* workspace,
+                                        size_t workspace_bytes, void* stream, float* Qx_out, float* Z_out,
+                                        void* const* stage_events) {
+  if (!X || !Wk || !Wv || !Wk_syn || !Wv_syn || !Q0 || !Y || !workspace) return FLARE_ERR_NULL;
+  flare_status st = check_common(B, H, N, M, D);
+  if (st != FLARE_OK) return st;
+  if (C != H * D) return FLARE_ERR_SHAPE;
+  if (C % 64 != 0 || C > 256) return FLARE_ERR_UNSUPPORTED;
+  if (!aligned16(X) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(Wk_syn) || !aligned16(Wv_syn) ||
+      !aligned16(Q0) || !aligned16(Y) || !aligned16(lengths) || !aligned16(Qx_out) || !aligned16(Z_out) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FLARE_ERR_ALIGN;
+  const Plan pl = make_plan(FLARE_VARIANT_FLAREPP, B, H, N, M, D);
+  if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
+  const float sc = resolve_scale(scale, D);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(ws + pl.off_err, 0, 4, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+
+  // eq. 7 and eq. 9: the four per-head projections
+  CUtensorMap tx, tw[4];
+  if (!map3d(&tx, X, C, N, B, 64, kProjTile, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map2d(&tw[0], Wk_syn, C, C, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map2d(&tw[1], Wv_syn, C, C, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map2d(&tw[2], Wk, C, C, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map2d(&tw[3], Wv, C, C, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return FLARE_ERR_LAUNCH;
+  uint16_t* kt = reinterpret_cast<uint16_t*>(ws + pl.off_kt);
+  uint16_t* vt = reinterpret_cast<uint16_t*>(ws + pl.off_vt);
+  uint16_t* kk = reinterpret_cast<uint16_t*>(ws + pl.off_kp);
+  uint16_t* vv = reinterpret_cast<uint16_t*>(ws + pl.off_vp);
+  float* kn_syn = reinterpret_cast<float*>(ws + pl.off_kn_syn);
+  float* kn = reinterpret_cast<float*>(ws + pl.off_kn);
+  if (!record(stage_events, 0, s)) return FLARE_ERR_LAUNCH;
+  ProjParams pp{};
+  pp.B = B; pp.N = N; pp.C = C; pp.H = H; pp.D = D;
+  pp.tiles_per_b = static_cast<int>(cdiv(N, kProjTile));
+  pp.n_tiles = B * pp.tiles_per_b;
+  const int slots = C == 256 ? kNumSM : kNumSM * kSlotsPerSM;
+  pp.groups = std::max(1, std::min(pp.n_tiles, slots / 4));
+  pp.n_groups32 = pl.G32;
+  pp.out[0] = kt; pp.out[1] = vt; pp.out[2] = kk; pp.out[3] = vv;
+  pp.knorm[0] = kn_syn; pp.knorm[1] = nullptr; pp.knorm[2] = kn; pp.knorm[3] = nullptr;
+  pp.err = reinterpret_cast<uint32_t*>(ws + pl.off_err);
+  pp.timeout_ns = wait_timeout_ns();
+  if (launch_project(tx, tw, pp, s) != cudaSuccess || !record(stage_events, 1, s)) return FLARE_ERR_LAUNCH;
+
+  // eq. 8: query synthesis with the learned seeds
+  float* qx32 = Qx_out ? Qx_out : reinterpret_cast<float*>(ws + pl.off_qx32);
+  uint16_t* qx16 = reinterpret_cast<uint16_t*>(ws + pl.off_qx16);
+  st = run_encode(pl, ws, Q0, 0, kt, vt, kn_syn, qx32, qx16, B, H, N, M, D, lengths, sc, s, stage_events, 2);
+  if (st != FLARE_OK) return st;
+  // eq. 10: encode with the synthesised queries
+  float* z32 = Z_out ? Z_out : reinterpret_cast<float*>(ws + pl.off_z32);
+  uint16_t* z16 = reinterpret_cast<uint16_t*>(ws + pl.off_z16);
+  st = run_encode(pl, ws, qx16, 1, kk, vv, kn, z32, z16, B, H, N, M, D, lengths, sc, s, stage_events, 4);
+  if (st != FLARE_OK) return st;
+  // eq. 11: decode
+  st = run_decode(pl, ws, qx16, 1, z16, kk, Y, B, H, N, M, D, lengths, sc, s);
+  if (st != FLARE_OK) return st;
+  return record(stage_events, 6, s) ? FLARE_OK : FLARE_ERR_LAUNCH;
+}
+
+flare_status flarepp_mixer_fwd(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                               const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0,
+                               flare_bf16* Y, int B, int N, int C, int H, int M, int D, const int32_t* lengths,
+                               float scale, void* workspace, size_t workspace_bytes, void* stream, float* Qx_out,
+                               float* Z_out) {
+  return flarepp_mixer_fwd_profiled(X, Wk, Wv, Wk_syn, Wv_syn, Q0, Y, B, N, C, H, M, D, lengths, scale, workspace,
+                                    workspace_bytes, stream, Qx_out, Z_out, nullptr);
+}
+
+flare_status flare_last_device_status(void* workspace, void* stream) {
+  if (!workspace) return FLARE_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, workspace, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  if (word & FLARE_DEV_TIMEOUT) return FLARE_ERR_TIMEOUT;
+  if (word & FLARE_DEV_BAD_LENGTH) return FLARE_ERR_SHAPE;
+  return FLARE_OK;
+}
+
+flare_status flare_selftest_wait_timeout(void* workspace, void* stream, unsigned long long timeout_ns) {
+  if (!workspace) return FLARE_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FLARE_ERR_ALIGN;
+  if (timeout_ns < 1000ull) timeout_ns = 1000ull;
+  if (timeout_ns > 1000000000ull) timeout_ns = 1000000000ull;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, 4, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  if (launch_wait_selftest(static_cast<uint32_t*>(workspace), timeout_ns, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  return FLARE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,119 @@
+// Internal definitions shared by the FLARE kernels and the host entry points.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+// Device error word bits (first 4 bytes of the workspace).
+#define FLARE_DEV_TIMEOUT 0x1u
+#define FLARE_DEV_BAD_LENGTH 0x2u
+
+namespace flare {
+
+constexpr int kSlotsPerSM = 2;     // co-resident CTAs per SM for the softmax kernels
+constexpr int kNumSM = 148;        // B200
+constexpr int kEncTile = 64;       // tokens per encode tile
+constexpr int kLatBlock = 128;     // latents per encode CTA (UMMA M)
+constexpr int kDecTile = 128;      // tokens per decode tile (UMMA M)
+constexpr int kDecChunk = 64;      // latents per decode chunk (UMMA N)
+constexpr int kNormGroup = 32;     // tokens per key-norm group
+constexpr int kProjTile = 128;     // tokens per projection tile
+
+// ---------------------------------------------------------------------------
+// Projection: out[p][b][h][n][:] = X[b][n][:] @ W_p[:, h*D:(h+1)*D]
+// ---------------------------------------------------------------------------
+struct ProjParams {
+  int B, N, C, H, D;
+  int tiles_per_b;     // ceil(N / kProjTile)
+  int n_tiles;         // B * tiles_per_b
+  int groups;          // CTAs per projection
+  int n_groups32;      // ceil(N / kNormGroup)
+  uint16_t* out[4];    // [B][H][N][D] bf16
+  float* knorm[4];     // [B*H][n_groups32] max key norm per group, or nullptr
+  uint32_t* err;
+  unsigned long long timeout_ns;
+};
+
+// ---------------------------------------------------------------------------
+// Key norms for the FLARE path (keys given by the caller)
+// ---------------------------------------------------------------------------
+struct KnormParams {
+  int BH, N, D, n_groups32;
+  const uint16_t* k;   // [BH][N][D]
+  float* knorm;        // [BH][n_groups32]
+};
+
+// ---------------------------------------------------------------------------
+// Split-N encode: partial softmax sums of one (b, h, latent block, split)
+// ---------------------------------------------------------------------------
+struct EncodeParams {
+  int B, H, N, M, D;
+  int q_per_batch;      // queries [B*H][M][D] (1) or [H][M][D] (0)
+  int n_splits;         // S
+  int tiles_per_split;  // in kEncTile tiles
+  int n_lblocks;        // ceil(M / kLatBlock)
+  int n_groups32;
+  int q_rows;           // rows of one query box: min(M, kLatBlock)
+  float c;              // scale * log2(e)
+  const int32_t* lengths;
+  const float* knorm;   // [B*H][n_groups32]
+  const uint16_t* q;    // bf16 queries
+  float* part;          // [B*H][S][M][D+2]: shift, sum, D partial outputs
+  uint32_t* err;
+  unsigned long long timeout_ns;
+};
+
+// ---------------------------------------------------------------------------
+// Merge of the split partials (log-sum-exp combine) + exact fallback rows
+// ---------------------------------------------------------------------------
+struct MergeParams {
+  int B, H, N, M, D;
+  int q_per_batch;
+  int n_splits, tiles_per_split;
+  float scale, c;
+  const int32_t* lengths;
+  const float* part;
+  const uint16_t* q;    // bf16 queries of this encode
+  const uint16_t* k;    // bf16 keys   [B*H][N][D]
+  const uint16_t* v;    // bf16 values [B*H][N][D]
+  float* out_f32;       // [B*H][M][D]
+  uint16_t* out_bf16;   // [B*H][M][D]
+};
+
+// ---------------------------------------------------------------------------
+// Decode: Y = softmax_m(K Q^T * scale) Z per token
+// ---------------------------------------------------------------------------
+struct DecodeParams {
+  int B, H, N, M, D;
+  int q_per_batch;
+  int tiles_per_cta;    // in kDecTile tiles
+  int ctas_per_head;
+  int chunk_rows;       // rows of one Q/Z box: min(M, kDecChunk)
+  float scale, c;
+  const int32_t* lengths;
+  const uint16_t* q;    // bf16 [G][M][D]
+  const uint16_t* z;    // bf16 [B*H][M][D]
+  const uint16_t* k;    // bf16 [B*H][N][D]
+  uint16_t* y;          // bf16 [B*H][N][D]
+  uint32_t* err;
+  unsigned long long timeout_ns;
+};
+
+// Host-side launchers (each returns the cudaError_t of the launch).
+cudaError_t launch_project(const CUtensorMap& tm_x, const CUtensorMap (&tm_w)[4], const ProjParams& p,
+                           cudaStream_t s);
+cudaError_t launch_knorm(const KnormParams& p, cudaStream_t s);
+cudaError_t launch_encode(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                          const EncodeParams& p, cudaStream_t s);
+cudaError_t launch_merge(const MergeParams& p, cudaStream_t s);
+cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_z, const CUtensorMap& tm_k,
+                          const DecodeParams& p, cudaStream_t s);
+cudaError_t launch_wait_selftest(uint32_t* err, unsigned long long timeout_ns, cudaStream_t s);
+
+// Shared-memory footprints (bytes) of the pipelined kernels.
+size_t encode_smem_bytes(int D);
+size_t decode_smem_bytes(int D, int M);
+size_t project_smem_bytes(int C);
+
+}  // namespace flare

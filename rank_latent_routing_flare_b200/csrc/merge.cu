@@ -1,0 +1,172 @@
+// Small kernels around the encoder:
+//  - merge_kernel: combines the per-split partial softmax sums of the encoder
+//    with the log-sum-exp rule of the FLARE++ paper (arXiv 2608.11519,
+//    section "Multi-GPU context parallelism", eq. 14), used here across the
+//    CTAs of one GPU instead of across ranks.  Splits are visited in
+//    ascending order, so the result is bitwise reproducible.  A row whose
+//    fast-path sums lost mass to underflow is recomputed exactly (two-pass
+//    softmax in fp32 over all valid tokens) by the warp that owns it.
+//  - knorm_kernel: largest key norm of every 32-token group (keys given by
+//    the caller, FLARE path); the encoder's softmax shift bound.
+//  - wait_selftest_kernel: exercises the bounded-wait error path.
+#include "ptx.cuh"
+
+namespace flare {
+namespace {
+
+// Exact encoder row: z = sum_n softmax_n(<q, k_n> * scale) v_n over n < L,
+// fp32, two passes, lanes stride over tokens, fixed butterfly reductions.
+template <int D>
+__device__ float merge_exact_row(const MergeParams& p, const uint16_t* qrow, const uint16_t* kh,
+                                 const uint16_t* vh, int L, int lane) {
+  if (L <= 0) return 0.f;
+  float q[D];
+#pragma unroll
+  for (int d = 0; d < D; ++d) q[d] = __uint_as_float(static_cast<uint32_t>(qrow[d]) << 16);
+  float mx = -INFINITY;
+  for (int n = lane; n < L; n += 32) {
+    float s = 0.f;
+#pragma unroll
+    for (int d = 0; d < D; ++d) s = fmaf(q[d], __uint_as_float(static_cast<uint32_t>(kh[static_cast<size_t>(n) * D + d]) << 16), s);
+    mx = fmaxf(mx, s * p.c);
+  }
+  mx = warp_max(mx);
+  float acc[D];
+#pragma unroll
+  for (int d = 0; d < D; ++d) acc[d] = 0.f;
+  float den = 0.f;
+  for (int n = lane; n < L; n += 32) {
+    float s = 0.f;
+#pragma unroll
+    for (int d = 0; d < D; ++d) s = fmaf(q[d], __uint_as_float(static_cast<uint32_t>(kh[static_cast<size_t>(n) * D + d]) << 16), s);
+    const float e = exp2f(s * p.c - mx);
+    den += e;
+#pragma unroll
+    for (int d = 0; d < D; ++d) acc[d] = fmaf(e, __uint_as_float(static_cast<uint32_t>(vh[static_cast<size_t>(n) * D + d]) << 16), acc[d]);
+  }
+  den = warp_sum(den);
+  float mine = 0.f;
+#pragma unroll
+  for (int d = 0; d < D; ++d) {
+    const float t = warp_sum(acc[d]);
+    if (d == lane) mine = t;
+  }
+  return mine / den;
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= p.B * p.H * p.M) return;
+  const int bh = row / p.M, m = row % p.M;
+  const int b = bh / p.H, h = bh % p.H;
+  int L = p.N;
+  if (p.lengths) L = min(max(p.lengths[b], 0), p.N);
+  const int ntv = (L + kEncTile - 1) / kEncTile;
+  const int S = p.n_splits;
+  const size_t stride = static_cast<size_t>(p.M) * (D + 2);
+  const float* base = p.part + static_cast<size_t>(bh) * S * stride + static_cast<size_t>(m) * (D + 2);
+
+  // log2 of the total weight: G = max_s (U_s + log2 l_s); bound of the mass
+  // lost to flushed exponentials: sum_s n_s 2^(U_s - 126)
+  float G = -INFINITY, lost = -INFINITY;
+  for (int s = 0; s < S; ++s) {
+    const int t0 = s * p.tiles_per_split, t1 = min(t0 + p.tiles_per_split, ntv);
+    if (t1 <= t0) continue;
+    const float U = base[s * stride], l = base[s * stride + 1];
+    if (l > 0.f) G = fmaxf(G, U + log2f(l));
+    lost = fmaxf(lost, U - 126.f + log2f(static_cast<float>((t1 - t0) * kEncTile)));
+  }
+  const bool exact = !(G > -INFINITY) || (lost + log2f(static_cast<float>(S)) - G > -27.f);
+  float z = 0.f;
+  if (!exact) {
+    float num = 0.f, den = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const int t0 = s * p.tiles_per_split, t1 = min(t0 + p.tiles_per_split, ntv);
+      if (t1 <= t0) continue;
+      const float* e = base + s * stride;
+      const float l = e[1];
+      if (!(l > 0.f)) continue;
+      const float w = exp2f(e[0] - G);
+      den = fmaf(w, l, den);
+      if (lane < D) num = fmaf(w, e[2 + lane], num);
+    }
+    z = num / den;
+  } else {
+    const int g = p.q_per_batch ? bh : h;
+    z = merge_exact_row<D>(p, p.q + (static_cast<size_t>(g) * p.M + m) * D, p.k + static_cast<size_t>(bh) * p.N * D,
+                           p.v + static_cast<size_t>(bh) * p.N * D, L, lane);
+  }
+  if (lane < D) {
+    const size_t o = static_cast<size_t>(row) * D + lane;
+    p.out_f32[o] = z;
+    p.out_bf16[o] = static_cast<uint16_t>(pack_bf16x2(z, 0.f) & 0xFFFFu);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) knorm_kernel(const KnormParams p) {
+  const long grp = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (grp >= static_cast<long>(p.BH) * p.n_groups32) return;
+  const int bh = static_cast<int>(grp / p.n_groups32), gi = static_cast<int>(grp % p.n_groups32);
+  const int n = gi * kNormGroup + lane;
+  float s = 0.f;
+  if (n < p.N) {
+    const uint4* row = reinterpret_cast<const uint4*>(p.k + (static_cast<size_t>(bh) * p.N + n) * D);
+#pragma unroll
+    for (int u = 0; u < D / 8; ++u) {
+      const uint4 v = row[u];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float a = bf16_lo(w[t]), b = bf16_hi(w[t]);
+        s = fmaf(a, a, fmaf(b, b, s));
+      }
+    }
+  }
+  const float nm = warp_max(sqrtf(s));
+  if (lane == 0) p.knorm[grp] = nm;
+}
+
+__global__ void wait_selftest_kernel(uint32_t* err, unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // nothing ever arrives on `bar`: the wait runs out and records the error
+    const WaitCtx w{err, &abort_flag, timeout_ns};
+    mbar_wait(&bar, 0, w);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_merge(const MergeParams& p, cudaStream_t s) {
+  const long rows = static_cast<long>(p.B) * p.H * p.M;
+  const dim3 grid(static_cast<unsigned>((rows * 32 + 255) / 256));
+  if (p.D == 16) merge_kernel<16><<<grid, 256, 0, s>>>(p);
+  else merge_kernel<32><<<grid, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_knorm(const KnormParams& p, cudaStream_t s) {
+  const long groups = static_cast<long>(p.BH) * p.n_groups32;
+  const dim3 grid(static_cast<unsigned>((groups * 32 + 255) / 256));
+  if (p.D == 16) knorm_kernel<16><<<grid, 256, 0, s>>>(p);
+  else knorm_kernel<32><<<grid, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_selftest(uint32_t* err, unsigned long long timeout_ns, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 32, 0, s>>>(err, timeout_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace flare

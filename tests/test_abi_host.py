@@ -1,0 +1,144 @@
+"""Host-only checks of the C ABI (no GPU needed, no kernel is launched).
+
+The library must load on a machine without a GPU, export every function that
+include/flare.h declares, size workspaces from the shapes alone and reject
+invalid arguments on the host, before anything is enqueued.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import rank_latent_routing_flare_b200 as fl
+from rank_latent_routing_flare_b200 import Status
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "flare.h")
+
+# fake, 256-byte aligned "device" addresses: never dereferenced, because every
+# call below fails validation before it touches CUDA
+A = 0x10000
+W = 0x20000
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"FLARE_API\s+[\w\s\*]+?\b(flare\w*)\s*\(", text)))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    assert names == sorted(["flare_workspace_bytes", "flare_mixer_fwd", "flarepp_mixer_fwd",
+                            "flare_mixer_fwd_profiled", "flarepp_mixer_fwd_profiled",
+                            "flare_last_device_status", "flare_status_string",
+                            "flare_selftest_wait_timeout"])
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = fl.load_library()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = os.popen(f"nm -D --defined-only {fl.library_path()}").read()
+    exported = set(re.findall(r"\bT (\w+)", out))
+    assert set(declared_functions()) <= exported
+    # nothing else leaks out of the library except the C ABI
+    assert all(e.startswith("flare") or e.startswith("_") for e in exported), exported
+
+
+def test_library_needs_no_libcuda_at_load_time():
+    out = os.popen(f"ldd {fl.library_path()}").read()
+    assert "libcuda.so" not in out and "libcudart" not in out
+
+
+def test_status_strings():
+    for s in Status:
+        txt = fl.flare_status_string(int(s))
+        assert txt.startswith("FLARE_" if s else "FLARE_OK")
+    assert "unknown" in fl.flare_status_string(99)
+
+
+@pytest.mark.parametrize("cfg", [
+    (1, 4, 1024, 32, 16, 64, 1),
+    (1, 8, 8192, 64, 16, 128, 8),
+    (0, 8, 65536, 256, 16, 128, 4),
+    (1, 8, 65536, 256, 16, 128, 4),
+    (1, 8, 1048576, 512, 16, 128, 1),
+    (1, 8, 4096, 128, 32, 256, 32),
+])
+def test_workspace_sizes(cfg):
+    variant, H, N, M, D, C, B = cfg
+    n = fl.flare_workspace_bytes(variant, B, H, N, M, D, C)
+    proj = B * H * N * D * 2
+    lat = B * H * M * D * 4
+    assert n > 0 and n % 256 == 0
+    if variant == 1:
+        assert n >= 4 * proj + 2 * lat      # K~, V~, K, V and the fp32 Q(X), Z
+    else:
+        assert n >= lat
+    # shape-only: the same question always gets the same answer
+    assert n == fl.flare_workspace_bytes(variant, B, H, N, M, D, C)
+
+
+def test_workspace_unsupported_sizes_return_zero():
+    assert fl.flare_workspace_bytes(0, 1, 1, 64, 32, 8, 0) == 0        # D not in {16, 32}
+    assert fl.flare_workspace_bytes(0, 1, 1, 64, 24, 16, 0) == 0       # M not a multiple of 16
+    assert fl.flare_workspace_bytes(0, 1, 1, 64, 528, 16, 0) == 0      # M > 512
+    assert fl.flare_workspace_bytes(1, 1, 2, 64, 32, 16, 48) == 0      # C != H*D
+    assert fl.flare_workspace_bytes(1, 1, 3, 64, 32, 16, 48) == 0      # C not a multiple of 64
+    assert fl.flare_workspace_bytes(2, 1, 1, 64, 32, 16, 16) == 0      # bad variant
+    assert fl.flare_workspace_bytes(0, 0, 1, 64, 32, 16, 0) == 0       # B = 0
+
+
+def flare_call(K=A, V=A, Q=A, Y=A, B=1, H=2, N=100, M=32, D=16, lengths=None, ws=W, ws_bytes=1 << 40,
+               Z=None):
+    lib = fl.load_library()
+    return lib.flare_mixer_fwd(K, V, Q, Y, B, H, N, M, D, lengths, 0.0, ws, ws_bytes, None, Z)
+
+
+def flarepp_call(X=A, Wk=A, Wv=A, Wks=A, Wvs=A, Q0=A, Y=A, B=1, N=100, C=64, H=4, M=32, D=16,
+                 lengths=None, ws=W, ws_bytes=1 << 40, Qx=None, Z=None):
+    lib = fl.load_library()
+    return lib.flarepp_mixer_fwd(X, Wk, Wv, Wks, Wvs, Q0, Y, B, N, C, H, M, D, lengths, 0.0, ws, ws_bytes,
+                                 None, Qx, Z)
+
+
+def test_flare_argument_errors():
+    assert flare_call(K=None) == Status.ERR_NULL
+    assert flare_call(Y=None) == Status.ERR_NULL
+    assert flare_call(ws=None) == Status.ERR_NULL
+    assert flare_call(N=0) == Status.ERR_SHAPE
+    assert flare_call(B=-1) == Status.ERR_SHAPE
+    assert flare_call(D=64) == Status.ERR_UNSUPPORTED
+    assert flare_call(M=40) == Status.ERR_UNSUPPORTED
+    assert flare_call(K=A + 8) == Status.ERR_ALIGN
+    assert flare_call(lengths=A + 4) == Status.ERR_ALIGN
+    assert flare_call(Z=A + 2) == Status.ERR_ALIGN
+    assert flare_call(ws=W + 16) == Status.ERR_ALIGN
+    need = fl.flare_workspace_bytes(0, 1, 2, 100, 32, 16)
+    assert flare_call(ws_bytes=need - 1) == Status.ERR_WORKSPACE
+
+
+def test_flarepp_argument_errors():
+    assert flarepp_call(Wvs=None) == Status.ERR_NULL
+    assert flarepp_call(Q0=None) == Status.ERR_NULL
+    assert flarepp_call(C=128) == Status.ERR_SHAPE                  # C != H*D
+    assert flarepp_call(C=48, H=3) == Status.ERR_UNSUPPORTED        # C % 64 != 0
+    assert flarepp_call(C=512, H=16, D=32) == Status.ERR_UNSUPPORTED
+    assert flarepp_call(X=A + 2) == Status.ERR_ALIGN
+    assert flarepp_call(Qx=A + 4) == Status.ERR_ALIGN
+    need = fl.flare_workspace_bytes(1, 1, 4, 100, 32, 16, 64)
+    assert flarepp_call(ws_bytes=need - 256) == Status.ERR_WORKSPACE
+
+
+def test_valid_call_without_gpu_reports_launch_error():
+    """With valid arguments the library reaches CUDA; on a machine without a
+    GPU that fails cleanly with ERR_LAUNCH instead of crashing."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert flare_call() == Status.ERR_LAUNCH
+    assert flarepp_call() == Status.ERR_LAUNCH
+    lib = fl.load_library()
+    assert lib.flare_selftest_wait_timeout(W, None, 1000) == Status.ERR_LAUNCH
+    assert lib.flare_last_device_status(None, None) == Status.ERR_NULL
