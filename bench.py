@@ -31,7 +31,6 @@ import os
 import re
 import statistics
 import sys
-import threading
 import time
 
 import numpy as np
@@ -71,56 +70,68 @@ def load_peaks():
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    REASONS = {0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
-               0x80: "hw_power_brake_slowdown", 0x4: "sw_power_cap", 0x1: "gpu_idle",
-               0x2: "applications_clocks_setting", 0x100: "sync_boost"}
+    """Samples SM clock, power and clock-event reasons with ``nvidia-smi -lms``
+    (a separate process, read only) while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
-        self.samples = []
-        self.reasons = set()
-        self.max_mhz = None
-        self._stop = threading.Event()
-        self._ok = False
-        try:
-            import pynvml
-            pynvml.nvmlInit()
-            self._nv = pynvml
-            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
-            self._ok = True
-        except Exception as e:  # pragma: no cover - depends on the host
-            log("clock sampling unavailable:", e)
-        self.period = period_s
-        self._t = threading.Thread(target=self._run, daemon=True)
-
-    def _run(self):
-        nv = self._nv
-        while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-                for bit, name in self.REASONS.items():
-                    if r & bit and name != "gpu_idle":
-                        self.reasons.add(name)
-            except Exception:
-                pass
-            time.sleep(self.period)
+    def __init__(self, device_index: int, period_ms: int = 20, path: str | None = None):
+        import tempfile
+        self.dev = device_index
+        self.period = period_ms
+        self.path = path or tempfile.mktemp(prefix="flare_clocks_", suffix=".csv")
+        self.proc = None
+        self.lines = []
 
     def __enter__(self):
-        if self._ok:
-            self._t.start()
+        import shutil
+        import subprocess
+        if shutil.which("nvidia-smi") is None:
+            log("nvidia-smi not found: no clock samples")
+            return self
+        self.fh = open(self.path, "w")
+        self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                      f"-lms={self.period}", "-i", str(self.dev)], stdout=self.fh,
+                                     stderr=subprocess.DEVNULL)
+        t0 = time.time()
+        while time.time() - t0 < 10 and os.path.getsize(self.path) == 0:
+            time.sleep(0.01)
+        self.skip = sum(1 for _ in open(self.path))   # samples taken before the timed region
         return self
 
     def __exit__(self, *exc):
-        self._stop.set()
-        if self._ok:
-            self._t.join()
+        if self.proc is None:
+            return
+        time.sleep(self.period / 1000.0)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.fh.close()
+        self.lines = [ln.strip() for ln in open(self.path) if ln.strip()][self.skip:]
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
 
     def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
-        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        mhz, mx, pw, reasons = [], None, [], set()
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                mx = float(f[2])
+                pw.append(float(f[3]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": float(statistics.median(mhz)) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz),
+                "power_w_median": float(statistics.median(pw)) if pw else None}
 
 
 # ---------------------------------------------------------------------------
@@ -250,10 +261,12 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override N (smaller cases for profiling; not a bench line)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -280,7 +293,7 @@ def main():
     fl.load_library()
 
     # inputs: each rank its own synthetic sample of the workload (weak scaling)
-    w = make_workload(args.workload, seed=None if rank == 0 else 1000 + rank)
+    w = make_workload(args.workload, N=args.tokens, seed=None if rank == 0 else 1000 + rank)
     assert w.variant == "flarepp"
 
     def to_dev(bits):
@@ -404,17 +417,19 @@ def main():
         step()
         hY.copy_(Y.view(torch.int16), non_blocking=True)
 
-    e2e_step()
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
+    e2e_ms = float("nan")
+    if args.e2e_steps > 0:
         e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
     if world > 1:
         t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)

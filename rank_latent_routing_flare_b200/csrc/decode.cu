@@ -39,7 +39,11 @@ struct DecCfg {
   static constexpr int OFF_BAR = OFF_K + NST * KT_B;
   static constexpr int OFF_MISC = OFF_BAR + 8 * 32;
   static constexpr int BYTES = OFF_MISC + 64;
-  static constexpr uint32_t TMEM_COLS = 256;            // S/P buffers [0,128), Y buffers at 128, 192
+  // TMEM columns: S[0..1] at 0 and 64 (fp32 scores), P[0..1] at 128 and 160
+  // (bf16 pairs), Y at 192 (+32): two buffers for D = 16, one for D = 32
+  static constexpr uint32_t TMEM_COLS = 256;
+  static constexpr uint32_t COL_S = 0, COL_P = 128, COL_Y = 192;
+  static constexpr int NYB = (D == 16) ? 2 : 1;
 };
 
 __device__ __forceinline__ float bf16_row_norm2(const uint4* row, int n16) {
@@ -103,11 +107,12 @@ __global__ void __launch_bounds__(192, 2)
   uint64_t* qz_full = bars;
   uint64_t* k_full = bars + 1;
   uint64_t* k_empty = bars + 1 + NST;
-  uint64_t* s_full = bars + 1 + 2 * NST;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* buf_free = p_full + 2;
-  uint64_t* y_full = buf_free + 2;
-  uint64_t* y_free = y_full + 2;
+  uint64_t* s_full = bars + 1 + 2 * NST;  // S[j] computed
+  uint64_t* s_free = s_full + 2;           // S[j] loaded by the softmax warps
+  uint64_t* p_full = s_free + 2;           // P[j] stored
+  uint64_t* p_free = p_full + 2;           // P[j] consumed by the value MMA
+  uint64_t* y_full = p_free + 2;           // Y[yb] of a tile complete
+  uint64_t* y_free = y_full + 2;           // Y[yb] read by the epilogue
   uint64_t* mma_done = y_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(sm + Cfg::OFF_MISC + 4);
@@ -155,8 +160,9 @@ __global__ void __launch_bounds__(192, 2)
     }
     for (int j = 0; j < 2; ++j) {
       mbar_init(s_full + j, 1);
+      mbar_init(s_free + j, 128);
       mbar_init(p_full + j, 128);
-      mbar_init(buf_free + j, 1);
+      mbar_init(p_free + j, 1);
       mbar_init(y_full + j, 1);
       mbar_init(y_free + j, 128);
     }
@@ -202,13 +208,32 @@ __global__ void __launch_bounds__(192, 2)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Chunk sequence q = tile * nc + c.  S(q+2) is issued as soon as the
+    // softmax warps have loaded S(q); P(q) [Z_c | 1] accumulates into Y of
+    // the tile once P(q) is stored.
     if (lane == 0) {
       const uint32_t idesc_y = idesc_bf16_f32(128, Cfg::NY, false, true);
       const uint32_t sq_a = smem_u32(sq), sz_a = smem_u32(sz), ones_a = smem_u32(sones);
       auto chunk_n = [&](int c) { return min(kDecChunk, p.M - c * kDecChunk); };
+      auto issue_s = [&](int q) -> bool {
+        const int tile = q / nc, c = q % nc, j = q & 1;
+        const int st = tile % NST;
+        if (c == 0 && !mbar_wait(k_full + st, (tile / NST) & 1, wc)) return false;
+        if (q >= 2 && !mbar_wait(s_free + j, ((q >> 1) - 1) & 1, wc)) return false;
+        tc_fence_after();
+        const uint32_t k_a = smem_u32(sk + st * Cfg::KT_B);
+        const uint32_t idesc_s = idesc_bf16_f32(128, chunk_n(c), false, false);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          umma_ss(tmem + Cfg::COL_S + j * 64, umma_desc(k_a + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT),
+                  umma_desc(sq_a + c * Cfg::CH_B + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full + j);
+        return true;
+      };
       auto issue_pv = [&](int q) -> bool {
-        const int tile = q / nc, c = q % nc, j = q & 1, yb = tile & 1;
-        if (c == 0 && tile >= 2 && !mbar_wait(y_free + yb, ((tile >> 1) - 1) & 1, wc)) return false;
+        const int tile = q / nc, c = q % nc, j = q & 1, yb = tile % Cfg::NYB;
+        if (c == 0 && tile >= Cfg::NYB && !mbar_wait(y_free + yb, ((tile / Cfg::NYB) - 1) & 1, wc)) return false;
         if (!mbar_wait(p_full + j, (q >> 1) & 1, wc)) return false;
         tc_fence_after();
         const uint32_t z_a = sz_a + c * Cfg::CH_B;
@@ -216,9 +241,10 @@ __global__ void __launch_bounds__(192, 2)
         const int nks = chunk_n(c) / 16;
         for (int ks = 0; ks < nks; ++ks) {
           const uint64_t bdesc = umma_desc(z_a + ks * 16 * Cfg::ROWB, lbo, Cfg::SBO, Cfg::LAYOUT);
-          umma_ts(tmem + 128 + yb * 64, tmem + j * 64 + ks * 8, bdesc, idesc_y, (c > 0 || ks > 0) ? 1u : 0u);
+          umma_ts(tmem + Cfg::COL_Y + yb * 32, tmem + Cfg::COL_P + j * 32 + ks * 8, bdesc, idesc_y,
+                  (c > 0 || ks > 0) ? 1u : 0u);
         }
-        umma_commit(buf_free + j);
+        umma_commit(p_free + j);
         if (c == nc - 1) {
           umma_commit(y_full + yb);
           umma_commit(k_empty + (tile % NST));
@@ -227,23 +253,11 @@ __global__ void __launch_bounds__(192, 2)
       };
       bool ok = mbar_wait(qz_full, 0, wc);
       const int total = ntiles * nc;
+      for (int q = 0; ok && q < min(2, total); ++q) ok = issue_s(q);
       for (int q = 0; ok && q < total; ++q) {
-        const int tile = q / nc, c = q % nc, j = q & 1;
-        const int st = tile % NST;
-        if (c == 0 && !mbar_wait(k_full + st, (tile / NST) & 1, wc)) { ok = false; break; }
-        if (q >= 2 && !mbar_wait(buf_free + j, ((q >> 1) - 1) & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t k_a = smem_u32(sk + st * Cfg::KT_B);
-        const uint32_t idesc_s = idesc_bf16_f32(128, chunk_n(c), false, false);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          umma_ss(tmem + j * 64, umma_desc(k_a + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT),
-                  umma_desc(sq_a + c * Cfg::CH_B + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT), idesc_s, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(s_full + j);
-        if (q >= 1 && !issue_pv(q - 1)) { ok = false; break; }
+        if (q + 2 < total && !issue_s(q + 2)) { ok = false; break; }
+        if (!issue_pv(q)) { ok = false; break; }
       }
-      if (ok) issue_pv(total - 1);
       // drain: every MMA issued above must be complete before TMEM is freed
       umma_commit(mma_done);
       mbar_wait_drain(mma_done, 0, p.timeout_ns);
@@ -268,68 +282,27 @@ __global__ void __launch_bounds__(192, 2)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     int q = 0;  // global chunk counter (same sequence as the MMA issuer)
     bool ok = true;
-    for (int i = 0; ok && i < ntiles; ++i) {
-      const int n = (ta + i) * kDecTile + r;
-      const bool in_range = n < p.N;
-      const bool valid = n < L;
-      float kn = 0.f;
-      if (in_range) kn = sqrtf(bf16_row_norm2(reinterpret_cast<const uint4*>(kh + static_cast<size_t>(n) * D), D / 8));
-      const float nu = c * kn * qm;
-      for (int cc = 0; cc < nc; ++cc, ++q) {
-        const int j = q & 1;
-        if (!mbar_wait_warp(s_full + j, (q >> 1) & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-        const int cn = min(kDecChunk, p.M - cc * kDecChunk);
-        uint32_t sa[32], pk[32];
-        tmem_ld32(lane_base + j * 64, sa);
-        if (cn > 32) {
-          uint32_t sb[32];
-          tmem_ld32(lane_base + j * 64 + 32, sb);
-          tmem_wait_ld();
-          if (cn == 64) {
+    // this thread's key row, loaded one tile ahead so that the norm never
+    // waits on memory
+    uint4 krow[D / 8];
+    auto load_krow = [&](int tile_idx) {
+      const int nn = (ta + tile_idx) * kDecTile + r;
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              pk[k] = pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sa[2 * k]), c, -nu)),
-                                  ex2_mufu(fmaf(__uint_as_float(sa[2 * k + 1]), c, -nu)));
-              pk[16 + k] = pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sb[2 * k]), c, -nu)),
-                                       ex2_mufu(fmaf(__uint_as_float(sb[2 * k + 1]), c, -nu)));
-            }
-          } else {  // 48 latents
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-              pk[k] = pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sa[2 * k]), c, -nu)),
-                                  ex2_mufu(fmaf(__uint_as_float(sa[2 * k + 1]), c, -nu)));
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              pk[16 + k] = pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sb[2 * k]), c, -nu)),
-                                       ex2_mufu(fmaf(__uint_as_float(sb[2 * k + 1]), c, -nu)));
-#pragma unroll
-            for (int k = 8; k < 16; ++k) pk[16 + k] = 0u;
-          }
-        } else {
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            pk[k] = (2 * k < cn) ? pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sa[2 * k]), c, -nu)),
-                                               ex2_mufu(fmaf(__uint_as_float(sa[2 * k + 1]), c, -nu)))
-                                 : 0u;
-            pk[16 + k] = 0u;
-          }
-        }
-        tmem_st32(lane_base + j * 64, pk);  // P overwrites the first 32 columns of S
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(p_full + j);
-      }
-      if (!ok) break;
-      // epilogue of tile i
-      const int yb = i & 1;
-      if (!mbar_wait_warp(y_full + yb, (i >> 1) & 1, wc)) { ok = false; break; }
+      for (int u = 0; u < D / 8; ++u)
+        krow[u] = nn < p.N ? reinterpret_cast<const uint4*>(kh + static_cast<size_t>(nn) * D)[u]
+                           : make_uint4(0, 0, 0, 0);
+    };
+    // Epilogue of tile i: Y = acc / sum, zero rows for padding, bf16 stores.
+    // It runs one chunk late (after chunk 0 of tile i+1) so that the softmax
+    // warps never wait for the last value MMA of a tile.
+    auto epilogue = [&](int i) -> bool {
+      const int yb = i % Cfg::NYB;
+      if (!mbar_wait_warp(y_full + yb, (i / Cfg::NYB) & 1, wc)) return false;
       tc_fence_after();
       uint32_t o[32];
       float l;
       float y[D];
-      tmem_ld32(lane_base + 128 + yb * 64, o);
+      tmem_ld32(lane_base + Cfg::COL_Y + yb * 32, o);
       if constexpr (D == 16) {
         tmem_wait_ld();
         l = __uint_as_float(o[16]);
@@ -337,7 +310,7 @@ __global__ void __launch_bounds__(192, 2)
         for (int d = 0; d < 16; ++d) y[d] = __uint_as_float(o[d]);
       } else {
         uint32_t o2[16];
-        tmem_ld16(lane_base + 128 + yb * 64 + 32, o2);
+        tmem_ld16(lane_base + Cfg::COL_Y + yb * 32 + 32, o2);
         tmem_wait_ld();
         l = __uint_as_float(o2[0]);
 #pragma unroll
@@ -345,7 +318,8 @@ __global__ void __launch_bounds__(192, 2)
       }
       tc_fence_before();
       mbar_arrive(y_free + yb);
-      if (valid) {
+      const int n = (ta + i) * kDecTile + r;
+      if (n < L) {
         // lost mass < M * 2^-126 per token; 2^-90 keeps it below 2^-27 relative
         if (!(l >= 0x1p-90f)) {
           decode_token_exact<D>(p, kh + static_cast<size_t>(n) * D, qg, zh, y);
@@ -358,14 +332,64 @@ __global__ void __launch_bounds__(192, 2)
 #pragma unroll
         for (int d = 0; d < D; ++d) y[d] = 0.f;
       }
-      if (in_range) {
+      if (n < p.N) {
         uint4* dst = reinterpret_cast<uint4*>(yh + static_cast<size_t>(n) * D);
 #pragma unroll
         for (int u = 0; u < D / 8; ++u)
           dst[u] = make_uint4(pack_bf16x2(y[8 * u + 0], y[8 * u + 1]), pack_bf16x2(y[8 * u + 2], y[8 * u + 3]),
                               pack_bf16x2(y[8 * u + 4], y[8 * u + 5]), pack_bf16x2(y[8 * u + 6], y[8 * u + 7]));
       }
+      return true;
+    };
+    load_krow(0);
+    for (int i = 0; ok && i < ntiles; ++i) {
+      const float kn = sqrtf(bf16_row_norm2(krow, D / 8));
+      if (i + 1 < ntiles) load_krow(i + 1);
+      const float nu = c * kn * qm;
+      for (int cc = 0; cc < nc; ++cc, ++q) {
+        const int j = q & 1;
+        if (!mbar_wait_warp(s_full + j, (q >> 1) & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        const int cn = min(kDecChunk, p.M - cc * kDecChunk);
+        uint32_t sa[32], sb[32], pk[32];
+        tmem_ld32(lane_base + Cfg::COL_S + j * 64, sa);
+        if (cn > 32) tmem_ld32(lane_base + Cfg::COL_S + j * 64 + 32, sb);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(s_free + j);  // the tensor pipe may now overwrite S[j]
+        if (cn == 64) {
+          exp2_chunk64<FLARE_DEC_POLY_PAIRS>(sa, sb, c, nu, pk);
+        } else if (cn > 32) {  // 48 latents
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            pk[k] = pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sa[2 * k]), c, -nu)),
+                                ex2_mufu(fmaf(__uint_as_float(sa[2 * k + 1]), c, -nu)));
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            pk[16 + k] = pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sb[2 * k]), c, -nu)),
+                                     ex2_mufu(fmaf(__uint_as_float(sb[2 * k + 1]), c, -nu)));
+#pragma unroll
+          for (int k = 8; k < 16; ++k) pk[16 + k] = 0u;
+        } else {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            pk[k] = (2 * k < cn) ? pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sa[2 * k]), c, -nu)),
+                                               ex2_mufu(fmaf(__uint_as_float(sa[2 * k + 1]), c, -nu)))
+                                 : 0u;
+            pk[16 + k] = 0u;
+          }
+        }
+        // P[j] was last read by the value MMA of chunk q-2
+        if (q >= 2 && !mbar_wait_warp(p_free + j, ((q >> 1) - 1) & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        tmem_st32(lane_base + Cfg::COL_P + j * 32, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full + j);
+        if (cc == 0 && i >= 1 && !epilogue(i - 1)) { ok = false; break; }
+      }
     }
+    if (ok && ntiles > 0) epilogue(ntiles - 1);
   }
   tc_fence_before();
   __syncthreads();

@@ -37,7 +37,10 @@ struct EncCfg {
   static constexpr int OFF_BAR = OFF_ONES + TILE_B;
   static constexpr int OFF_MISC = OFF_BAR + 8 * 32;
   static constexpr int BYTES = OFF_MISC + 64;
-  static constexpr uint32_t TMEM_COLS = 256;           // S buffers [0,128), O at 128
+  // TMEM columns: S[0..1] at 0 and 64 (fp32 scores), P[0..1] at 128 and 160
+  // (bf16 pairs), O at 192 (D values + the row-sum block)
+  static constexpr uint32_t TMEM_COLS = 256;
+  static constexpr uint32_t COL_S = 0, COL_P = 128, COL_O = 192;
 };
 
 template <int D>
@@ -56,10 +59,11 @@ __global__ void __launch_bounds__(192, 2)
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = bars + 1 + NST;
-  uint64_t* s_full = bars + 1 + 2 * NST;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* buf_free = p_full + 2;
-  uint64_t* o_full = buf_free + 2;
+  uint64_t* s_full = bars + 1 + 2 * NST;  // S[j] computed
+  uint64_t* s_free = s_full + 2;           // S[j] loaded by the softmax warps
+  uint64_t* p_full = s_free + 2;           // P[j] stored by the softmax warps
+  uint64_t* p_free = p_full + 2;           // P[j] consumed by the value MMA
+  uint64_t* o_full = p_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(sm + Cfg::OFF_MISC + 4);
   float* red = reinterpret_cast<float*>(sm + Cfg::OFF_MISC + 16);
@@ -108,8 +112,9 @@ __global__ void __launch_bounds__(192, 2)
     }
     for (int j = 0; j < 2; ++j) {
       mbar_init(s_full + j, 1);
+      mbar_init(s_free + j, 128);
       mbar_init(p_full + j, 128);
-      mbar_init(buf_free + j, 1);
+      mbar_init(p_free + j, 1);
     }
     mbar_init(o_full, 1);
     *abort_flag = 0;
@@ -153,43 +158,51 @@ __global__ void __launch_bounds__(192, 2)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Order: S(i+2) is issued as soon as the softmax warps have loaded S(i)
+    // (early release of the score buffer), then P(i) V(i) once P(i) is in
+    // TMEM.  Two score and two probability buffers keep a full tile of slack
+    // between the tensor pipe and the softmax warps.
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, kEncTile, false, false);
       const uint32_t idesc_pv = idesc_bf16_f32(128, Cfg::NO, false, true);
-      const uint32_t tO = tmem + 128;
+      const uint32_t tO = tmem + Cfg::COL_O;
       const uint32_t sq_a = smem_u32(sq);
       const uint32_t ones_a = smem_u32(sones);
-      auto issue_pv = [&](int q) -> bool {
-        const int j = q & 1, st = q % NST;
-        if (!mbar_wait(p_full + j, (q >> 1) & 1, wc)) return false;
+      auto issue_s = [&](int i) -> bool {
+        const int st = i % NST, j = i & 1;
+        if (!mbar_wait(kv_full + st, (i / NST) & 1, wc)) return false;
+        if (i >= 2 && !mbar_wait(s_free + j, ((i >> 1) - 1) & 1, wc)) return false;
+        tc_fence_after();
+        const uint32_t k_a = smem_u32(sk + st * Cfg::TILE_B);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          umma_ss(tmem + Cfg::COL_S + j * 64, umma_desc(sq_a + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT),
+                  umma_desc(k_a + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full + j);
+        return true;
+      };
+      auto issue_pv = [&](int i) -> bool {
+        const int j = i & 1, st = i % NST;
+        if (!mbar_wait(p_full + j, (i >> 1) & 1, wc)) return false;
         tc_fence_after();
         const uint32_t v_a = smem_u32(sv + st * Cfg::TILE_B);
         const uint32_t lbo = ones_a - v_a;  // [V | 1] : second N-atom = ones block
 #pragma unroll
         for (int ks = 0; ks < kEncTile / 16; ++ks) {
           const uint64_t bdesc = umma_desc(v_a + ks * 16 * Cfg::ROWB, lbo, Cfg::SBO, Cfg::LAYOUT);
-          umma_ts(tO, tmem + j * 64 + ks * 8, bdesc, idesc_pv, (q > 0 || ks > 0) ? 1u : 0u);
+          umma_ts(tO, tmem + Cfg::COL_P + j * 32 + ks * 8, bdesc, idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
         }
-        umma_commit(buf_free + j);
+        umma_commit(p_free + j);
         umma_commit(kv_empty + st);
         return true;
       };
       bool ok = mbar_wait(q_full, 0, wc);
+      for (int i = 0; ok && i < min(2, ntiles); ++i) ok = issue_s(i);
       for (int i = 0; ok && i < ntiles; ++i) {
-        const int st = i % NST, j = i & 1;
-        if (!mbar_wait(kv_full + st, (i / NST) & 1, wc)) { ok = false; break; }
-        if (i >= 2 && !mbar_wait(buf_free + j, ((i >> 1) - 1) & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t k_a = smem_u32(sk + st * Cfg::TILE_B);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          umma_ss(tmem + j * 64, umma_desc(sq_a + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT),
-                  umma_desc(k_a + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT), idesc_s, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(s_full + j);
-        if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
+        if (i + 2 < ntiles && !issue_s(i + 2)) { ok = false; break; }
+        if (!issue_pv(i)) { ok = false; break; }
       }
-      if (ok) issue_pv(ntiles - 1);
       umma_commit(o_full);  // completes once every MMA issued above is done
       mbar_wait_drain(o_full, 0, p.timeout_ns);
     }
@@ -233,20 +246,18 @@ __global__ void __launch_bounds__(192, 2)
       const int j = i & 1;
       if (!mbar_wait_warp(s_full + j, (i >> 1) & 1, wc)) { ok = false; break; }
       tc_fence_after();
+      uint32_t sa[32], sb[32], pk[32];
       if (warp_live) {
-        uint32_t sa[32], sb[32], pk[32];
-        tmem_ld32(lane_base + j * 64, sa);
-        tmem_ld32(lane_base + j * 64 + 32, sb);
+        tmem_ld32(lane_base + Cfg::COL_S + j * 64, sa);
+        tmem_ld32(lane_base + Cfg::COL_S + j * 64 + 32, sb);
         tmem_wait_ld();
+      }
+      tc_fence_before();
+      mbar_arrive(s_free + j);  // the tensor pipe may now overwrite S[j]
+      if (warp_live) {
         const int valid = L - (t0 + i) * kEncTile;
         if (valid >= kEncTile) {
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            pk[k] = pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sa[2 * k]), c, -U)),
-                                ex2_mufu(fmaf(__uint_as_float(sa[2 * k + 1]), c, -U)));
-            pk[16 + k] = pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sb[2 * k]), c, -U)),
-                                     ex2_mufu(fmaf(__uint_as_float(sb[2 * k + 1]), c, -U)));
-          }
+          exp2_chunk64<FLARE_ENC_POLY_PAIRS>(sa, sb, c, U, pk);
         } else {  // last, partial tile of the valid range: padded tokens get weight 0
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
@@ -259,7 +270,12 @@ __global__ void __launch_bounds__(192, 2)
             pk[16 + k] = pack_bf16x2(e2, e3);
           }
         }
-        tmem_st32(lane_base + j * 64, pk);  // P overwrites the first 32 columns of S
+      }
+      // P[j] was last read by the value MMA of tile i-2
+      if (i >= 2 && !mbar_wait_warp(p_free + j, ((i >> 1) - 1) & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+      if (warp_live) {
+        tmem_st32(lane_base + Cfg::COL_P + j * 32, pk);
         tmem_wait_st();
       }
       tc_fence_before();
@@ -269,14 +285,14 @@ __global__ void __launch_bounds__(192, 2)
       tc_fence_after();
       if (warp_live) {
         uint32_t o[32];
-        tmem_ld32(lane_base + 128, o);
+        tmem_ld32(lane_base + Cfg::COL_O, o);
         float l;
         if constexpr (D == 16) {
           tmem_wait_ld();
           l = __uint_as_float(o[16]);
         } else {
           uint32_t o2[16];
-          tmem_ld16(lane_base + 128 + 32, o2);
+          tmem_ld16(lane_base + Cfg::COL_O + 32, o2);
           tmem_wait_ld();
           l = __uint_as_float(o2[0]);
         }

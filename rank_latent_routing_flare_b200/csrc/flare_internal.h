@@ -20,6 +20,16 @@ constexpr int kDecChunk = 64;      // latents per decode chunk (UMMA N)
 constexpr int kNormGroup = 32;     // tokens per key-norm group
 constexpr int kProjTile = 128;     // tokens per projection tile
 
+// Of the 32 score pairs of each 64-column softmax chunk, how many are
+// exponentiated on the FMA pipe (polynomial) instead of the MUFU; chosen by
+// measurement on B200.
+#ifndef FLARE_ENC_POLY_PAIRS
+#define FLARE_ENC_POLY_PAIRS 0
+#endif
+#ifndef FLARE_DEC_POLY_PAIRS
+#define FLARE_DEC_POLY_PAIRS 0
+#endif
+
 // ---------------------------------------------------------------------------
 // Projection: out[p][b][h][n][:] = X[b][n][:] @ W_p[:, h*D:(h+1)*D]
 // ---------------------------------------------------------------------------

@@ -246,12 +246,55 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 // ----------------------------------------------------------------------------
 // arithmetic helpers
 // ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi);
+
 // 2^x on the special-function unit (flushes subnormal results to zero).
 __device__ __forceinline__ float ex2_mufu(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 2^x on the FMA pipe, for x <= ~0 (inputs below -125 are clamped; the
+// result is then 2^-125 instead of 0, which the callers' sums absorb).
+// Cody-Waite range reduction x = j + f, j = rint(x), f in [-1/2, 1/2]:
+// t = x + 1.5*2^23 leaves j in the low mantissa bits of t, so (bits(t) << 23)
+// is j shifted into the exponent field; p(f) ~ 2^f is the degree-3 minimax
+// polynomial (max relative error 7.5e-5) derived by gen_exp2_poly.py.
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  float p = fmaf(0x1.c3f76p-5f, f, 0x1.f0de1ap-3f);
+  p = fmaf(p, f, 0x1.62f31ap-1f);
+  p = fmaf(p, f, 0x1.fff692p-1f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Exponentials of one 64-column chunk of scores (raw fp32 bits in a[0..31],
+// b[0..31]): e = 2^(s * c - shift), packed to bf16 pairs.  NPOLY of the 32
+// pairs use ex2_poly (FMA pipe), spread evenly; the rest use the MUFU.
+template <int NPOLY>
+__device__ __forceinline__ void exp2_chunk64(const uint32_t (&a)[32], const uint32_t (&b)[32], float c, float shift,
+                                             uint32_t (&pk)[32]) {
+#pragma unroll
+  for (int q = 0; q < 32; ++q) {
+    const uint32_t* src = q < 16 ? a : b;
+    const int k = q & 15;
+    const float x0 = fmaf(__uint_as_float(src[2 * k]), c, -shift);
+    const float x1 = fmaf(__uint_as_float(src[2 * k + 1]), c, -shift);
+    const bool poly = ((q * NPOLY) % 32) < NPOLY;
+    float e0, e1;
+    if (poly) {
+      e0 = ex2_poly(x0);
+      e1 = ex2_poly(x1);
+    } else {
+      e0 = ex2_mufu(x0);
+      e1 = ex2_mufu(x1);
+    }
+    pk[q] = pack_bf16x2(e0, e1);
+  }
+}
+
 // Pack two floats to bf16x2 (round to nearest even): lo -> bits [0,16), hi -> [16,32).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
