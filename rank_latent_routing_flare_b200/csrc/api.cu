@@ -70,20 +70,22 @@ CUtensorMapSwizzle row_swizzle(int D) { return D == 16 ? CU_TENSOR_MAP_SWIZZLE_3
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 long cdiv(long a, long b) { return (a + b - 1) / b; }
 
-// Number of token splits of the encoder: at least 8 tiles per split, chosen
-// to fill the SMs' CTA slots in whole waves.  Depends on the sizes only, so a
-// given problem always uses the same split count (and gives the same bits).
-int choose_splits(long units, long ntiles) {
-  const long slots = static_cast<long>(kNumSM) * kSlotsPerSM;
-  const long smax = std::max(1L, std::min(ntiles / 8, 1024L));
+// Number of token splits of the encoder.  Cost model: the CTAs run in
+// waves of `slots` (CTAs resident on the whole GPU); a wave lasts as long as
+// one split (its tiles plus a fixed set-up cost worth kSplitSetupTiles
+// tiles).  Depends on the sizes only, so a given problem always uses the same
+// split count (and gives the same bits).
+constexpr long kSplitSetupTiles = 8;
+int choose_splits(long units, long ntiles, long slots) {
+  const long smax = std::max(1L, std::min(ntiles, 1024L));
   int best = 1;
-  double best_eff = -1.0;
+  long best_cost = -1;
   for (long s = 1; s <= smax; ++s) {
-    const long ctas = units * s;
-    const long waves = cdiv(ctas, slots);
-    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
+    const long tps = cdiv(ntiles, s);
+    if (s > 1 && cdiv(ntiles, tps) < s) continue;  // same tiling as a smaller s
+    const long cost = cdiv(units * s, slots) * (tps + kSplitSetupTiles);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
       best = static_cast<int>(s);
     }
   }
@@ -95,7 +97,7 @@ struct Plan {
   int dec_ctas = 1, dec_tiles = 1;       // decoder CTAs per head, tiles per CTA
   int G32 = 1;
   size_t off_err = 0, off_kt = 0, off_vt = 0, off_kp = 0, off_vp = 0, off_kn_syn = 0, off_kn = 0, off_part = 0,
-         off_qx32 = 0, off_qx16 = 0, off_z32 = 0, off_z16 = 0, total = 0;
+         off_qx32 = 0, off_qx16 = 0, off_z32 = 0, off_z16 = 0, off_fb = 0, total = 0;
 };
 
 Plan make_plan(int variant, long B, long H, long N, long M, long D) {
@@ -103,11 +105,11 @@ Plan make_plan(int variant, long B, long H, long N, long M, long D) {
   const long BH = B * H;
   const long ntiles = cdiv(N, kEncTile);
   p.LB = static_cast<int>(cdiv(M, kLatBlock));
-  p.S = choose_splits(BH * p.LB, ntiles);
+  p.S = choose_splits(BH * p.LB, ntiles, static_cast<long>(kNumSM) * enc_ctas_per_sm(static_cast<int>(D)));
   p.tps = static_cast<int>(cdiv(ntiles, p.S));
   p.S = static_cast<int>(cdiv(ntiles, p.tps));
   const long dtiles = cdiv(N, kDecTile);
-  long per = std::max(1L, static_cast<long>(kNumSM) * kSlotsPerSM / BH);
+  long per = std::max(1L, static_cast<long>(kNumSM) * dec_ctas_per_sm(static_cast<int>(D)) / BH);
   per = std::min(per, dtiles);
   p.dec_tiles = static_cast<int>(cdiv(dtiles, per));
   p.dec_ctas = static_cast<int>(cdiv(dtiles, p.dec_tiles));
@@ -132,6 +134,7 @@ Plan make_plan(int variant, long B, long H, long N, long M, long D) {
   }
   p.off_z32 = off; off += lat32;
   p.off_z16 = off; off += lat16;
+  p.off_fb = off; off += align256(static_cast<size_t>(BH) * N * 8);
   p.total = off;
   return p;
 }
@@ -216,6 +219,8 @@ flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
   dp.k = static_cast<const uint16_t*>(k);
   dp.y = static_cast<uint16_t*>(y);
   dp.err = reinterpret_cast<uint32_t*>(ws + pl.off_err);
+  dp.fb_count = reinterpret_cast<uint32_t*>(ws + pl.off_err) + 1;
+  dp.fb_list = reinterpret_cast<uint64_t*>(ws + pl.off_fb);
   dp.timeout_ns = wait_timeout_ns();
   if (launch_decode(tq, tz, tk, dp, st) != cudaSuccess) return FLARE_ERR_LAUNCH;
   return FLARE_OK;
@@ -264,7 +269,7 @@ flare_status flare_mixer_fwd_profiled(const flare_bf16* K, const flare_bf16* V, 
   const float sc = resolve_scale(scale, D);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  if (cudaMemsetAsync(ws + pl.off_err, 0, 4, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  if (cudaMemsetAsync(ws + pl.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   if (!record(stage_events, 0, s)) return FLARE_ERR_LAUNCH;
   KnormParams kp{B * H, N, D, pl.G32, reinterpret_cast<const uint16_t*>(K), reinterpret_cast<float*>(ws + pl.off_kn)};
   if (launch_knorm(kp, s) != cudaSuccess || !record(stage_events, 1, s)) return FLARE_ERR_LAUNCH;
@@ -304,7 +309,7 @@ flare_status flarepp_mixer_fwd_profiled(const flare_bf16* X, const flare_bf16* W
   const float sc = resolve_scale(scale, D);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  if (cudaMemsetAsync(ws + pl.off_err, 0, 4, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  if (cudaMemsetAsync(ws + pl.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
 
   // eq. 7 and eq. 9: the four per-head projections
   CUtensorMap tx, tw[4];
@@ -325,7 +330,7 @@ flare_status flarepp_mixer_fwd_profiled(const flare_bf16* X, const flare_bf16* W
   pp.B = B; pp.N = N; pp.C = C; pp.H = H; pp.D = D;
   pp.tiles_per_b = static_cast<int>(cdiv(N, kProjTile));
   pp.n_tiles = B * pp.tiles_per_b;
-  const int slots = C == 256 ? kNumSM : kNumSM * kSlotsPerSM;
+  const int slots = C == 256 ? kNumSM : kNumSM * 2;
   pp.groups = std::max(1, std::min(pp.n_tiles, slots / 4));
   pp.n_groups32 = pl.G32;
   pp.out[0] = kt; pp.out[1] = vt; pp.out[2] = kk; pp.out[3] = vv;

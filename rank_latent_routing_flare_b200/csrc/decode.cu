@@ -15,8 +15,11 @@
 // whose sum underflows (only possible when the bound is very loose) is
 // recomputed exactly by its own thread from global memory.
 //
-// Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer + TMEM owner,
-// warps 2..5 = softmax + epilogue (thread <-> TMEM lane <-> token).
+// Warp roles (5 warps): warp 0 lane 0 is the control thread: it loads Q and
+// Z, keeps the key-tile ring full (TMA) and issues the MMAs in program order,
+// blocking on exactly the next event.  Warps 1..4 are the softmax warps
+// (thread <-> TMEM lane <-> token).  A CTA needs 128 TMEM columns for D = 16,
+// so three CTAs share an SM.
 #include "ptx.cuh"
 
 namespace flare {
@@ -39,11 +42,12 @@ struct DecCfg {
   static constexpr int OFF_BAR = OFF_K + NST * KT_B;
   static constexpr int OFF_MISC = OFF_BAR + 8 * 32;
   static constexpr int BYTES = OFF_MISC + 64;
-  // TMEM columns: S[0..1] at 0 and 64 (fp32 scores), P[0..1] at 128 and 160
-  // (bf16 pairs), Y at 192 (+32): two buffers for D = 16, one for D = 32
-  static constexpr uint32_t TMEM_COLS = 256;
-  static constexpr uint32_t COL_S = 0, COL_P = 128, COL_Y = 192;
-  static constexpr int NYB = (D == 16) ? 2 : 1;
+  // TMEM columns: S at 0 (fp32 scores of one 64-latent chunk), P at 64 (bf16
+  // pairs), Y at 96 (D values + the row-sum block)
+  static constexpr uint32_t COL_S = 0, COL_P = 64, COL_Y = 96;
+  static constexpr uint32_t TMEM_COLS = (COL_Y + NY <= 128) ? 128 : 256;
+  static constexpr int THREADS = 160;
+  static constexpr int CTAS_PER_SM = dec_ctas_per_sm(D);
 };
 
 __device__ __forceinline__ float bf16_row_norm2(const uint4* row, int n16) {
@@ -60,39 +64,56 @@ __device__ __forceinline__ float bf16_row_norm2(const uint4* row, int n16) {
   return s;
 }
 
-// Exact two-pass softmax over the M latents for one token (fallback when the
-// fast path's row sum underflowed).  fp32 throughout, from global memory.
+// Exact two-pass softmax over the M latents for one token, written straight
+// to its output row: the fallback for tokens whose fast-path row sum
+// underflowed (only possible when the norm bound is very loose).  fp32 from
+// global memory; one thread per listed token.
 template <int D>
-__device__ void decode_token_exact(const DecodeParams& p, const uint16_t* krow, const uint16_t* qg,
-                                   const uint16_t* zh, float (&y)[D]) {
-  float k[D];
+__global__ void __launch_bounds__(128) decode_fallback_kernel(const DecodeParams p) {
+  const uint32_t count = *p.fb_count;
+  for (uint32_t e = blockIdx.x * blockDim.x + threadIdx.x; e < count; e += gridDim.x * blockDim.x) {
+    const uint64_t tok = p.fb_list[e];
+    const int bh = static_cast<int>(tok / static_cast<uint64_t>(p.N));
+    const int n = static_cast<int>(tok % static_cast<uint64_t>(p.N));
+    const int g = p.q_per_batch ? bh : bh % p.H;
+    const uint16_t* krow = p.k + (static_cast<size_t>(bh) * p.N + n) * D;
+    const uint16_t* qg = p.q + static_cast<size_t>(g) * p.M * D;
+    const uint16_t* zh = p.z + static_cast<size_t>(bh) * p.M * D;
+    float k[D], y[D];
 #pragma unroll
-  for (int d = 0; d < D; ++d) k[d] = __uint_as_float(static_cast<uint32_t>(krow[d]) << 16);
-  float mx = -INFINITY;
-  for (int m = 0; m < p.M; ++m) {
-    float s = 0.f;
+    for (int d = 0; d < D; ++d) k[d] = __uint_as_float(static_cast<uint32_t>(krow[d]) << 16);
+    float mx = -INFINITY;
+    for (int m = 0; m < p.M; ++m) {
+      float s = 0.f;
 #pragma unroll
-    for (int d = 0; d < D; ++d) s = fmaf(k[d], __uint_as_float(static_cast<uint32_t>(qg[m * D + d]) << 16), s);
-    mx = fmaxf(mx, s * p.c);
+      for (int d = 0; d < D; ++d) s = fmaf(k[d], __uint_as_float(static_cast<uint32_t>(qg[m * D + d]) << 16), s);
+      mx = fmaxf(mx, s * p.c);
+    }
+    float den = 0.f;
+#pragma unroll
+    for (int d = 0; d < D; ++d) y[d] = 0.f;
+    for (int m = 0; m < p.M; ++m) {
+      float s = 0.f;
+#pragma unroll
+      for (int d = 0; d < D; ++d) s = fmaf(k[d], __uint_as_float(static_cast<uint32_t>(qg[m * D + d]) << 16), s);
+      const float w = exp2f(s * p.c - mx);
+      den += w;
+#pragma unroll
+      for (int d = 0; d < D; ++d) y[d] = fmaf(w, __uint_as_float(static_cast<uint32_t>(zh[m * D + d]) << 16), y[d]);
+    }
+    const float inv = 1.f / den;
+    uint4* dst = reinterpret_cast<uint4*>(p.y + (static_cast<size_t>(bh) * p.N + n) * D);
+#pragma unroll
+    for (int u = 0; u < D / 8; ++u)
+      dst[u] = make_uint4(pack_bf16x2(y[8 * u + 0] * inv, y[8 * u + 1] * inv),
+                          pack_bf16x2(y[8 * u + 2] * inv, y[8 * u + 3] * inv),
+                          pack_bf16x2(y[8 * u + 4] * inv, y[8 * u + 5] * inv),
+                          pack_bf16x2(y[8 * u + 6] * inv, y[8 * u + 7] * inv));
   }
-  float den = 0.f;
-#pragma unroll
-  for (int d = 0; d < D; ++d) y[d] = 0.f;
-  for (int m = 0; m < p.M; ++m) {
-    float s = 0.f;
-#pragma unroll
-    for (int d = 0; d < D; ++d) s = fmaf(k[d], __uint_as_float(static_cast<uint32_t>(qg[m * D + d]) << 16), s);
-    const float e = exp2f(s * p.c - mx);
-    den += e;
-#pragma unroll
-    for (int d = 0; d < D; ++d) y[d] = fmaf(e, __uint_as_float(static_cast<uint32_t>(zh[m * D + d]) << 16), y[d]);
-  }
-#pragma unroll
-  for (int d = 0; d < D; ++d) y[d] /= den;
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 2)
+__global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
     decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_z,
                   const __grid_constant__ CUtensorMap tm_k, const DecodeParams p) {
   using Cfg = DecCfg<D>;
@@ -107,13 +128,13 @@ __global__ void __launch_bounds__(192, 2)
   uint64_t* qz_full = bars;
   uint64_t* k_full = bars + 1;
   uint64_t* k_empty = bars + 1 + NST;
-  uint64_t* s_full = bars + 1 + 2 * NST;  // S[j] computed
-  uint64_t* s_free = s_full + 2;           // S[j] loaded by the softmax warps
-  uint64_t* p_full = s_free + 2;           // P[j] stored
-  uint64_t* p_free = p_full + 2;           // P[j] consumed by the value MMA
-  uint64_t* y_full = p_free + 2;           // Y[yb] of a tile complete
-  uint64_t* y_free = y_full + 2;           // Y[yb] read by the epilogue
-  uint64_t* mma_done = y_free + 2;
+  uint64_t* s_full = bars + 1 + 2 * NST;  // S computed
+  uint64_t* s_free = s_full + 1;           // S loaded by every softmax warp
+  uint64_t* p_full = s_full + 2;           // P stored by every softmax warp
+  uint64_t* p_free = s_full + 3;           // P consumed by the value MMA
+  uint64_t* y_full = s_full + 4;           // Y of a tile complete
+  uint64_t* y_free = s_full + 5;           // Y read by every softmax warp
+  uint64_t* mma_done = s_full + 6;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(sm + Cfg::OFF_MISC + 4);
   float* red = reinterpret_cast<float*>(sm + Cfg::OFF_MISC + 16);
@@ -158,14 +179,12 @@ __global__ void __launch_bounds__(192, 2)
       mbar_init(k_full + i, 1);
       mbar_init(k_empty + i, 1);
     }
-    for (int j = 0; j < 2; ++j) {
-      mbar_init(s_full + j, 1);
-      mbar_init(s_free + j, 128);
-      mbar_init(p_full + j, 128);
-      mbar_init(p_free + j, 1);
-      mbar_init(y_full + j, 1);
-      mbar_init(y_free + j, 128);
-    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 4);
+    mbar_init(p_full, 4);
+    mbar_init(p_free, 1);
+    mbar_init(y_full, 1);
+    mbar_init(y_free, 4);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -173,7 +192,7 @@ __global__ void __launch_bounds__(192, 2)
   for (int i = threadIdx.x; i < Cfg::CH_B / 4; i += blockDim.x)
     reinterpret_cast<uint32_t*>(sones)[i] = 0x3F803F80u;  // bf16 1.0 pairs
   fence_proxy_async_smem();
-  if (warp == 1) {
+  if (warp == 0) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
@@ -184,7 +203,7 @@ __global__ void __launch_bounds__(192, 2)
   const WaitCtx wc{p.err, abort_flag, p.timeout_ns};
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ control thread
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_z);
@@ -194,82 +213,81 @@ __global__ void __launch_bounds__(192, 2)
         tma_load_3d(sq + c * Cfg::CH_B, &tm_q, qz_full, 0, c * kDecChunk, g);
         tma_load_3d(sz + c * Cfg::CH_B, &tm_z, qz_full, 0, c * kDecChunk, bh);
       }
-      int issued = 0;
-      for (int i = 0; i < ntiles; ++i) {
-        const int st = i % NST;
-        if (!mbar_wait(k_empty + st, ((i / NST) & 1) ^ 1, wc)) break;
-        mbar_arrive_expect_tx(k_full + st, Cfg::KT_B);
-        tma_load_3d(sk + st * Cfg::KT_B, &tm_k, k_full + st, 0, (ta + i) * kDecTile, bh);
-        issued = i + 1;
-      }
-      for (int i = max(0, issued - NST); i < issued; ++i)
-        mbar_wait_drain(k_full + (i % NST), (i / NST) & 1, p.timeout_ns);
-      mbar_wait_drain(qz_full, 0, p.timeout_ns);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    // Chunk sequence q = tile * nc + c.  S(q+2) is issued as soon as the
-    // softmax warps have loaded S(q); P(q) [Z_c | 1] accumulates into Y of
-    // the tile once P(q) is stored.
-    if (lane == 0) {
       const uint32_t idesc_y = idesc_bf16_f32(128, Cfg::NY, false, true);
       const uint32_t sq_a = smem_u32(sq), sz_a = smem_u32(sz), ones_a = smem_u32(sones);
-      auto chunk_n = [&](int c) { return min(kDecChunk, p.M - c * kDecChunk); };
-      auto issue_s = [&](int q) -> bool {
-        const int tile = q / nc, c = q % nc, j = q & 1;
+      auto chunk_n = [&](int cc) { return min(kDecChunk, p.M - cc * kDecChunk); };
+      int n_load = 0;
+      auto load = [&]() {
+        const int st = n_load % NST;
+        mbar_arrive_expect_tx(k_full + st, Cfg::KT_B);
+        tma_load_3d(sk + st * Cfg::KT_B, &tm_k, k_full + st, 0, (ta + n_load) * kDecTile, bh);
+        ++n_load;
+      };
+      auto refill = [&]() {
+        while (n_load < ntiles && mbar_test(k_empty + n_load % NST, ((n_load / NST) & 1) ^ 1)) load();
+      };
+      auto issue_s = [&](int qq) -> bool {
+        const int tile = qq / nc, cc = qq - tile * nc;
         const int st = tile % NST;
-        if (c == 0 && !mbar_wait(k_full + st, (tile / NST) & 1, wc)) return false;
-        if (q >= 2 && !mbar_wait(s_free + j, ((q >> 1) - 1) & 1, wc)) return false;
+        if (cc == 0) {
+          while (n_load <= tile) {
+            if (!mbar_wait(k_empty + n_load % NST, ((n_load / NST) & 1) ^ 1, wc)) return false;
+            load();
+          }
+          if (!mbar_wait(k_full + st, (tile / NST) & 1, wc)) return false;
+        }
         tc_fence_after();
         const uint32_t k_a = smem_u32(sk + st * Cfg::KT_B);
-        const uint32_t idesc_s = idesc_bf16_f32(128, chunk_n(c), false, false);
+        const uint32_t idesc_s = idesc_bf16_f32(128, chunk_n(cc), false, false);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          umma_ss(tmem + Cfg::COL_S + j * 64, umma_desc(k_a + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT),
-                  umma_desc(sq_a + c * Cfg::CH_B + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT), idesc_s, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(s_full + j);
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ss(tmem + Cfg::COL_S, umma_desc(k_a + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT),
+                  umma_desc(sq_a + cc * Cfg::CH_B + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT), idesc_s, kk > 0 ? 1u : 0u);
+        umma_commit(s_full);
         return true;
       };
-      auto issue_pv = [&](int q) -> bool {
-        const int tile = q / nc, c = q % nc, j = q & 1, yb = tile % Cfg::NYB;
-        if (c == 0 && tile >= Cfg::NYB && !mbar_wait(y_free + yb, ((tile / Cfg::NYB) - 1) & 1, wc)) return false;
-        if (!mbar_wait(p_full + j, (q >> 1) & 1, wc)) return false;
+      auto issue_pv = [&](int qq) -> bool {
+        const int tile = qq / nc, cc = qq - tile * nc;
+        // the first value MMA of a tile overwrites Y: the previous tile's
+        // epilogue must have read it
+        if (cc == 0 && tile >= 1 && !mbar_wait(y_free, (tile - 1) & 1, wc)) return false;
+        if (!mbar_wait(p_full, qq & 1, wc)) return false;
         tc_fence_after();
-        const uint32_t z_a = sz_a + c * Cfg::CH_B;
+        const uint32_t z_a = sz_a + cc * Cfg::CH_B;
         const uint32_t lbo = ones_a - z_a;  // [Z_c | 1]: second N-atom = ones block
-        const int nks = chunk_n(c) / 16;
+        const int nks = chunk_n(cc) / 16;
         for (int ks = 0; ks < nks; ++ks) {
           const uint64_t bdesc = umma_desc(z_a + ks * 16 * Cfg::ROWB, lbo, Cfg::SBO, Cfg::LAYOUT);
-          umma_ts(tmem + Cfg::COL_Y + yb * 32, tmem + Cfg::COL_P + j * 32 + ks * 8, bdesc, idesc_y,
-                  (c > 0 || ks > 0) ? 1u : 0u);
+          umma_ts(tmem + Cfg::COL_Y, tmem + Cfg::COL_P + ks * 8, bdesc, idesc_y, (cc > 0 || ks > 0) ? 1u : 0u);
         }
-        umma_commit(p_free + j);
-        if (c == nc - 1) {
-          umma_commit(y_full + yb);
+        umma_commit(p_free);
+        if (cc == nc - 1) {
+          umma_commit(y_full);
           umma_commit(k_empty + (tile % NST));
         }
         return true;
       };
-      bool ok = mbar_wait(qz_full, 0, wc);
       const int total = ntiles * nc;
-      for (int q = 0; ok && q < min(2, total); ++q) ok = issue_s(q);
-      for (int q = 0; ok && q < total; ++q) {
-        if (q + 2 < total && !issue_s(q + 2)) { ok = false; break; }
-        if (!issue_pv(q)) { ok = false; break; }
+      refill();
+      bool ok = mbar_wait(qz_full, 0, wc) && issue_s(0);
+      for (int qq = 1; ok && qq < total; ++qq) {
+        ok = mbar_wait(s_free, (qq - 1) & 1, wc) && issue_s(qq);  // S(q-1) loaded -> S(q)
+        if (ok) ok = issue_pv(qq - 1);                              // P(q-1) stored -> P(q-1) [Z | 1]
+        if (ok) refill();
       }
-      // drain: every MMA issued above must be complete before TMEM is freed
-      umma_commit(mma_done);
+      if (ok) issue_pv(total - 1);
+      umma_commit(mma_done);  // every MMA issued above is complete before TMEM is freed
       mbar_wait_drain(mma_done, 0, p.timeout_ns);
+      for (int i = max(0, n_load - NST); i < n_load; ++i)
+        mbar_wait_drain(k_full + (i % NST), (i / NST) & 1, p.timeout_ns);
+      mbar_wait_drain(qz_full, 0, p.timeout_ns);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     const int wq = warp & 3;
     const int r = wq * 32 + lane;                     // token row within the tile
-    const int tid = threadIdx.x - 64;
+    const int tid = threadIdx.x - 32;
     const uint16_t* qg = p.q + static_cast<size_t>(g) * p.M * D;
-    const uint16_t* zh = p.z + static_cast<size_t>(bh) * p.M * D;
-    const uint16_t* kh = p.k + static_cast<size_t>(bh) * p.N * D;
     // largest query norm of the head
     float qm = 0.f;
     for (int m = tid; m < p.M; m += 128)
@@ -280,29 +298,16 @@ __global__ void __launch_bounds__(192, 2)
     qm = sqrtf(fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])));
     const float c = p.c;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    int q = 0;  // global chunk counter (same sequence as the MMA issuer)
-    bool ok = true;
-    // this thread's key row, loaded one tile ahead so that the norm never
-    // waits on memory
-    uint4 krow[D / 8];
-    auto load_krow = [&](int tile_idx) {
-      const int nn = (ta + tile_idx) * kDecTile + r;
-#pragma unroll
-      for (int u = 0; u < D / 8; ++u)
-        krow[u] = nn < p.N ? reinterpret_cast<const uint4*>(kh + static_cast<size_t>(nn) * D)[u]
-                           : make_uint4(0, 0, 0, 0);
-    };
     // Epilogue of tile i: Y = acc / sum, zero rows for padding, bf16 stores.
-    // It runs one chunk late (after chunk 0 of tile i+1) so that the softmax
-    // warps never wait for the last value MMA of a tile.
+    // It runs inside chunk 0 of tile i+1, after the P store (the value MMA of
+    // the tile's last chunk has completed by then).
     auto epilogue = [&](int i) -> bool {
-      const int yb = i % Cfg::NYB;
-      if (!mbar_wait_warp(y_full + yb, (i / Cfg::NYB) & 1, wc)) return false;
+      if (!mbar_wait_warp(y_full, i & 1, wc)) return false;
       tc_fence_after();
       uint32_t o[32];
       float l;
       float y[D];
-      tmem_ld32(lane_base + Cfg::COL_Y + yb * 32, o);
+      tmem_ld32(lane_base + Cfg::COL_Y, o);
       if constexpr (D == 16) {
         tmem_wait_ld();
         l = __uint_as_float(o[16]);
@@ -310,29 +315,29 @@ __global__ void __launch_bounds__(192, 2)
         for (int d = 0; d < 16; ++d) y[d] = __uint_as_float(o[d]);
       } else {
         uint32_t o2[16];
-        tmem_ld16(lane_base + Cfg::COL_Y + yb * 32 + 32, o2);
+        tmem_ld16(lane_base + Cfg::COL_Y + 32, o2);
         tmem_wait_ld();
         l = __uint_as_float(o2[0]);
 #pragma unroll
         for (int d = 0; d < 32; ++d) y[d] = __uint_as_float(o[d]);
       }
       tc_fence_before();
-      mbar_arrive(y_free + yb);
+      mbar_arrive_warp(y_free);  // the next tile's first value MMA may overwrite Y
       const int n = (ta + i) * kDecTile + r;
+      // lost mass < M * 2^-126 per token; 2^-90 keeps it below 2^-27 relative
+      const bool exact = n < L && !(l >= 0x1p-90f);
       if (n < L) {
-        // lost mass < M * 2^-126 per token; 2^-90 keeps it below 2^-27 relative
-        if (!(l >= 0x1p-90f)) {
-          decode_token_exact<D>(p, kh + static_cast<size_t>(n) * D, qg, zh, y);
-        } else {
-          const float inv = 1.f / l;
+        const float inv = 1.f / l;
 #pragma unroll
-          for (int d = 0; d < D; ++d) y[d] *= inv;
-        }
+        for (int d = 0; d < D; ++d) y[d] *= inv;
       } else {
 #pragma unroll
         for (int d = 0; d < D; ++d) y[d] = 0.f;
       }
-      if (n < p.N) {
+      if (exact) {  // recomputed exactly by decode_fallback_kernel
+        const uint32_t e = atomicAdd(p.fb_count, 1u);
+        p.fb_list[e] = static_cast<uint64_t>(bh) * p.N + n;
+      } else if (n < p.N) {
         uint4* dst = reinterpret_cast<uint4*>(yh + static_cast<size_t>(n) * D);
 #pragma unroll
         for (int u = 0; u < D / 8; ++u)
@@ -341,59 +346,63 @@ __global__ void __launch_bounds__(192, 2)
       }
       return true;
     };
-    load_krow(0);
-    for (int i = 0; ok && i < ntiles; ++i) {
-      const float kn = sqrtf(bf16_row_norm2(krow, D / 8));
-      if (i + 1 < ntiles) load_krow(i + 1);
-      const float nu = c * kn * qm;
-      for (int cc = 0; cc < nc; ++cc, ++q) {
-        const int j = q & 1;
-        if (!mbar_wait_warp(s_full + j, (q >> 1) & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-        const int cn = min(kDecChunk, p.M - cc * kDecChunk);
-        uint32_t sa[32], sb[32], pk[32];
-        tmem_ld32(lane_base + Cfg::COL_S + j * 64, sa);
-        if (cn > 32) tmem_ld32(lane_base + Cfg::COL_S + j * 64 + 32, sb);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(s_free + j);  // the tensor pipe may now overwrite S[j]
-        if (cn == 64) {
-          exp2_chunk64<FLARE_DEC_POLY_PAIRS>(sa, sb, c, nu, pk);
-        } else if (cn > 32) {  // 48 latents
-#pragma unroll
-          for (int k = 0; k < 16; ++k)
-            pk[k] = pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sa[2 * k]), c, -nu)),
-                                ex2_mufu(fmaf(__uint_as_float(sa[2 * k + 1]), c, -nu)));
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            pk[16 + k] = pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sb[2 * k]), c, -nu)),
-                                     ex2_mufu(fmaf(__uint_as_float(sb[2 * k + 1]), c, -nu)));
-#pragma unroll
-          for (int k = 8; k < 16; ++k) pk[16 + k] = 0u;
-        } else {
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            pk[k] = (2 * k < cn) ? pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sa[2 * k]), c, -nu)),
-                                               ex2_mufu(fmaf(__uint_as_float(sa[2 * k + 1]), c, -nu)))
-                                 : 0u;
-            pk[16 + k] = 0u;
-          }
-        }
-        // P[j] was last read by the value MMA of chunk q-2
-        if (q >= 2 && !mbar_wait_warp(p_free + j, ((q >> 1) - 1) & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-        tmem_st32(lane_base + Cfg::COL_P + j * 32, pk);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(p_full + j);
-        if (cc == 0 && i >= 1 && !epilogue(i - 1)) { ok = false; break; }
+    const int total = ntiles * nc;
+    bool ok = true;
+    float nu = 0.f;
+    for (int qq = 0; qq < total; ++qq) {
+      const int tile = qq / nc, cc = qq - tile * nc;
+      if (!mbar_wait_warp(s_full, qq & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+      const int cn = min(kDecChunk, p.M - cc * kDecChunk);
+      uint32_t sa[32], sb[32], pk[32];
+      tmem_ld32(lane_base + Cfg::COL_S, sa);
+      if (cn > 32) tmem_ld32(lane_base + Cfg::COL_S + 32, sb);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive_warp(s_free);  // the tensor pipe may now write S(q+1)
+      if (cc == 0) {
+        // |k_n| from the key tile in shared memory (the swizzle only permutes
+        // 16-byte halves inside each row, which a sum of squares ignores);
+        // the tile stays resident until the tile's last value MMA completes
+        const uint4* krow_s = reinterpret_cast<const uint4*>(sk + (tile % NST) * Cfg::KT_B + r * Cfg::ROWB);
+        nu = c * sqrtf(bf16_row_norm2(krow_s, D / 8)) * qm;
       }
+      if (cn == kDecChunk) {
+        exp2_chunk64<FLARE_DEC_POLY_PAIRS>(sa, sb, c, nu, pk);
+      } else if (cn > 32) {  // 48 latents
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          pk[k] = pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sa[2 * k]), c, -nu)),
+                              ex2_mufu(fmaf(__uint_as_float(sa[2 * k + 1]), c, -nu)));
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          pk[16 + k] = pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sb[2 * k]), c, -nu)),
+                                   ex2_mufu(fmaf(__uint_as_float(sb[2 * k + 1]), c, -nu)));
+#pragma unroll
+        for (int k = 8; k < 16; ++k) pk[16 + k] = 0u;
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          pk[k] = (2 * k < cn) ? pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sa[2 * k]), c, -nu)),
+                                             ex2_mufu(fmaf(__uint_as_float(sa[2 * k + 1]), c, -nu)))
+                               : 0u;
+          pk[16 + k] = 0u;
+        }
+      }
+      // P was last read by the value MMA of chunk q-1
+      if (qq >= 1 && !mbar_wait_warp(p_free, (qq - 1) & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+      tmem_st32(lane_base + Cfg::COL_P, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive_warp(p_full);
+      if (cc == 0 && tile >= 1 && !epilogue(tile - 1)) { ok = false; break; }
     }
     if (ok && ntiles > 0) epilogue(ntiles - 1);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::TMEM_COLS);
   }
@@ -403,7 +412,9 @@ __global__ void __launch_bounds__(192, 2)
 
 size_t decode_smem_bytes(int D, int /*M*/) {
   const size_t need = (D == 16 ? DecCfg<16>::BYTES : DecCfg<32>::BYTES) + 1024;
-  return need > 90 * 1024 ? need : 90 * 1024;
+  // at most dec_ctas_per_sm(D) CTAs per SM (TMEM columns)
+  const size_t floor = dec_ctas_per_sm(D) >= 3 ? 70 * 1024 : 100 * 1024;
+  return need > floor ? need : floor;
 }
 
 cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_z, const CUtensorMap& tm_k,
@@ -414,13 +425,17 @@ cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_z, cons
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    decode_kernel<16><<<grid, 192, smem, s>>>(tm_q, tm_z, tm_k, p);
+    decode_kernel<16><<<grid, DecCfg<16>::THREADS, smem, s>>>(tm_q, tm_z, tm_k, p);
   } else {
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    decode_kernel<32><<<grid, 192, smem, s>>>(tm_q, tm_z, tm_k, p);
+    decode_kernel<32><<<grid, DecCfg<32>::THREADS, smem, s>>>(tm_q, tm_z, tm_k, p);
   }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (p.D == 16) decode_fallback_kernel<16><<<kNumSM, 128, 0, s>>>(p);
+  else decode_fallback_kernel<32><<<kNumSM, 128, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -14,8 +14,13 @@
 // (U_m, sum_m, O_m) and the merge kernel combines splits with the exact
 // log-sum-exp rule of section "Multi-GPU context parallelism" (eq. 14).
 //
-// Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer + TMEM owner,
-// warps 2..5 = softmax (thread <-> TMEM lane <-> latent row).
+// Warp roles (5 warps): warp 0 lane 0 is the control thread: it keeps the
+// K/V ring full (TMA) and issues the MMAs in program order, blocking on
+// exactly the next event (S(i+1) once every softmax warp has loaded S(i);
+// P(i) [V(i) | 1] once every softmax warp has stored P(i)).  Warps 1..4 are
+// the softmax warps (thread <-> TMEM lane <-> latent row).  A CTA needs 128
+// TMEM columns for D = 16: three CTAs (three softmax warps per SM
+// sub-partition) share an SM.
 #include "ptx.cuh"
 
 namespace flare {
@@ -23,13 +28,17 @@ namespace {
 
 template <int D>
 struct EncCfg {
+  static constexpr int T = kEncTile;                   // tokens per tile (64)
   static constexpr int ROWB = D * 2;                   // bytes of one K/V/Q row
-  static constexpr int TILE_B = kEncTile * ROWB;       // bytes of one K or V tile
+  static constexpr int TILE_B = T * ROWB;              // bytes of one K or V tile
   static constexpr int Q_B = kLatBlock * ROWB;
   static constexpr int NST = 8;                        // K/V ring stages
   static constexpr uint32_t LAYOUT = (D == 16) ? LAYOUT_SW32 : LAYOUT_SW64;
   static constexpr uint32_t SBO = 8 * ROWB;            // stride of 8-row core-matrix groups
   static constexpr int NO = D + 16;                    // O columns: D values + 16 copies of the sum
+  // TMEM columns: S at 0 (fp32 scores), P at T (bf16 pairs), O at 3T/2
+  static constexpr uint32_t COL_S = 0, COL_P = T, COL_O = T + T / 2;
+  static constexpr uint32_t TMEM_COLS = (COL_O + NO <= 128) ? 128 : 256;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_B;
   static constexpr int OFF_V = OFF_K + NST * TILE_B;
@@ -37,18 +46,16 @@ struct EncCfg {
   static constexpr int OFF_BAR = OFF_ONES + TILE_B;
   static constexpr int OFF_MISC = OFF_BAR + 8 * 32;
   static constexpr int BYTES = OFF_MISC + 64;
-  // TMEM columns: S[0..1] at 0 and 64 (fp32 scores), P[0..1] at 128 and 160
-  // (bf16 pairs), O at 192 (D values + the row-sum block)
-  static constexpr uint32_t TMEM_COLS = 256;
-  static constexpr uint32_t COL_S = 0, COL_P = 128, COL_O = 192;
+  static constexpr int THREADS = 160;
+  static constexpr int CTAS_PER_SM = enc_ctas_per_sm(D);
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 2)
+__global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
     encode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const EncodeParams p) {
   using Cfg = EncCfg<D>;
-  constexpr int NST = Cfg::NST;
+  constexpr int NST = Cfg::NST, T = Cfg::T;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sq = sm + Cfg::OFF_Q;
@@ -59,11 +66,11 @@ __global__ void __launch_bounds__(192, 2)
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = bars + 1 + NST;
-  uint64_t* s_full = bars + 1 + 2 * NST;  // S[j] computed
-  uint64_t* s_free = s_full + 2;           // S[j] loaded by the softmax warps
-  uint64_t* p_full = s_free + 2;           // P[j] stored by the softmax warps
-  uint64_t* p_free = p_full + 2;           // P[j] consumed by the value MMA
-  uint64_t* o_full = p_free + 2;
+  uint64_t* s_full = bars + 1 + 2 * NST;  // S computed
+  uint64_t* s_free = s_full + 1;           // S loaded by every softmax warp (one arrive per warp)
+  uint64_t* p_full = s_full + 2;           // P stored by every softmax warp (one arrive per warp)
+  uint64_t* p_free = s_full + 3;           // P consumed by the value MMA
+  uint64_t* o_full = s_full + 4;           // every MMA of the CTA done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(sm + Cfg::OFF_MISC + 4);
   float* red = reinterpret_cast<float*>(sm + Cfg::OFF_MISC + 16);
@@ -83,7 +90,7 @@ __global__ void __launch_bounds__(192, 2)
     }
     L = l;
   }
-  const int ntiles_valid = (L + kEncTile - 1) / kEncTile;
+  const int ntiles_valid = (L + T - 1) / T;
   const int t0 = s * p.tiles_per_split;
   const int t1 = min(t0 + p.tiles_per_split, ntiles_valid);
   const int ntiles = max(0, t1 - t0);
@@ -110,12 +117,10 @@ __global__ void __launch_bounds__(192, 2)
       mbar_init(kv_full + i, 1);
       mbar_init(kv_empty + i, 1);
     }
-    for (int j = 0; j < 2; ++j) {
-      mbar_init(s_full + j, 1);
-      mbar_init(s_free + j, 128);
-      mbar_init(p_full + j, 128);
-      mbar_init(p_free + j, 1);
-    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 4);
+    mbar_init(p_full, 4);
+    mbar_init(p_free, 1);
     mbar_init(o_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -123,7 +128,7 @@ __global__ void __launch_bounds__(192, 2)
   for (int i = threadIdx.x; i < Cfg::TILE_B / 4; i += blockDim.x)
     reinterpret_cast<uint32_t*>(sones)[i] = 0x3F803F80u;  // bf16 1.0 pairs
   fence_proxy_async_smem();
-  if (warp == 1) {
+  if (warp == 0) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
@@ -134,77 +139,72 @@ __global__ void __launch_bounds__(192, 2)
   const WaitCtx wc{p.err, abort_flag, p.timeout_ns};
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ control thread
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       mbar_arrive_expect_tx(q_full, p.q_rows * Cfg::ROWB);
       tma_load_3d(sq, &tm_q, q_full, 0, lb * kLatBlock, g);
-      int issued = 0;
-      for (int i = 0; i < ntiles; ++i) {
-        const int st = i % NST;
-        if (!mbar_wait(kv_empty + st, ((i / NST) & 1) ^ 1, wc)) break;
+      const uint32_t idesc_s = idesc_bf16_f32(128, T, false, false);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, Cfg::NO, false, true);
+      const uint32_t sq_a = smem_u32(sq), ones_a = smem_u32(sones);
+      int n_load = 0;
+      auto load = [&]() {
+        const int st = n_load % NST;
         mbar_arrive_expect_tx(kv_full + st, 2 * Cfg::TILE_B);
-        const int tok = (t0 + i) * kEncTile;
+        const int tok = (t0 + n_load) * T;
         tma_load_3d(sk + st * Cfg::TILE_B, &tm_k, kv_full + st, 0, tok, bh);
         tma_load_3d(sv + st * Cfg::TILE_B, &tm_v, kv_full + st, 0, tok, bh);
-        issued = i + 1;
-      }
-      // every issued copy must have landed before the CTA may exit
-      for (int i = max(0, issued - NST); i < issued; ++i)
-        mbar_wait_drain(kv_full + (i % NST), (i / NST) & 1, p.timeout_ns);
-      mbar_wait_drain(q_full, 0, p.timeout_ns);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    // Order: S(i+2) is issued as soon as the softmax warps have loaded S(i)
-    // (early release of the score buffer), then P(i) V(i) once P(i) is in
-    // TMEM.  Two score and two probability buffers keep a full tile of slack
-    // between the tensor pipe and the softmax warps.
-    if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(128, kEncTile, false, false);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, Cfg::NO, false, true);
-      const uint32_t tO = tmem + Cfg::COL_O;
-      const uint32_t sq_a = smem_u32(sq);
-      const uint32_t ones_a = smem_u32(sones);
+        ++n_load;
+      };
+      // refill every ring stage whose previous tile's value MMA has completed
+      auto refill = [&]() {
+        while (n_load < ntiles && mbar_test(kv_empty + n_load % NST, ((n_load / NST) & 1) ^ 1)) load();
+      };
       auto issue_s = [&](int i) -> bool {
-        const int st = i % NST, j = i & 1;
-        if (!mbar_wait(kv_full + st, (i / NST) & 1, wc)) return false;
-        if (i >= 2 && !mbar_wait(s_free + j, ((i >> 1) - 1) & 1, wc)) return false;
-        tc_fence_after();
-        const uint32_t k_a = smem_u32(sk + st * Cfg::TILE_B);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          umma_ss(tmem + Cfg::COL_S + j * 64, umma_desc(sq_a + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT),
-                  umma_desc(k_a + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT), idesc_s, kk > 0 ? 1u : 0u);
+        while (n_load <= i) {  // tile i not requested yet: wait for its stage
+          if (!mbar_wait(kv_empty + n_load % NST, ((n_load / NST) & 1) ^ 1, wc)) return false;
+          load();
         }
-        umma_commit(s_full + j);
+        if (!mbar_wait(kv_full + i % NST, (i / NST) & 1, wc)) return false;
+        tc_fence_after();
+        const uint32_t k_a = smem_u32(sk + (i % NST) * Cfg::TILE_B);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ss(tmem + Cfg::COL_S, umma_desc(sq_a + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT),
+                  umma_desc(k_a + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT), idesc_s, kk > 0 ? 1u : 0u);
+        umma_commit(s_full);
         return true;
       };
       auto issue_pv = [&](int i) -> bool {
-        const int j = i & 1, st = i % NST;
-        if (!mbar_wait(p_full + j, (i >> 1) & 1, wc)) return false;
+        if (!mbar_wait(p_full, i & 1, wc)) return false;
         tc_fence_after();
+        const int st = i % NST;
         const uint32_t v_a = smem_u32(sv + st * Cfg::TILE_B);
         const uint32_t lbo = ones_a - v_a;  // [V | 1] : second N-atom = ones block
 #pragma unroll
-        for (int ks = 0; ks < kEncTile / 16; ++ks) {
+        for (int ks = 0; ks < T / 16; ++ks) {
           const uint64_t bdesc = umma_desc(v_a + ks * 16 * Cfg::ROWB, lbo, Cfg::SBO, Cfg::LAYOUT);
-          umma_ts(tO, tmem + Cfg::COL_P + j * 32 + ks * 8, bdesc, idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
+          umma_ts(tmem + Cfg::COL_O, tmem + Cfg::COL_P + ks * 8, bdesc, idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
         }
-        umma_commit(p_free + j);
+        umma_commit(p_free);
         umma_commit(kv_empty + st);
         return true;
       };
-      bool ok = mbar_wait(q_full, 0, wc);
-      for (int i = 0; ok && i < min(2, ntiles); ++i) ok = issue_s(i);
-      for (int i = 0; ok && i < ntiles; ++i) {
-        if (i + 2 < ntiles && !issue_s(i + 2)) { ok = false; break; }
-        if (!issue_pv(i)) { ok = false; break; }
+      refill();
+      bool ok = mbar_wait(q_full, 0, wc) && issue_s(0);
+      for (int i = 1; ok && i < ntiles; ++i) {
+        ok = mbar_wait(s_free, (i - 1) & 1, wc) && issue_s(i);  // S(i-1) loaded -> S(i)
+        if (ok) ok = issue_pv(i - 1);                             // P(i-1) stored -> P(i-1) V(i-1)
+        if (ok) refill();
       }
+      if (ok) issue_pv(ntiles - 1);
       umma_commit(o_full);  // completes once every MMA issued above is done
       mbar_wait_drain(o_full, 0, p.timeout_ns);
+      for (int i = max(0, n_load - NST); i < n_load; ++i)  // copies in flight must land
+        mbar_wait_drain(kv_full + (i % NST), (i / NST) & 1, p.timeout_ns);
+      mbar_wait_drain(q_full, 0, p.timeout_ns);
     }
   } else {
     // ------------------------------------------------------------ softmax
@@ -213,12 +213,12 @@ __global__ void __launch_bounds__(192, 2)
     const int m = lb * kLatBlock + r;
     const bool row_ok = m < p.M;
     const bool warp_live = lb * kLatBlock + wq * 32 < p.M;
-    const int tid = threadIdx.x - 64;
+    const int tid = threadIdx.x - 32;
     // bound of the key norms over this split
     float km = 0.f;
     const float* kn = p.knorm + static_cast<size_t>(bh) * p.n_groups32;
-    const int g_end = min(t1 * (kEncTile / kNormGroup), p.n_groups32);
-    for (int gi = t0 * (kEncTile / kNormGroup) + tid; gi < g_end; gi += 128) km = fmaxf(km, kn[gi]);
+    const int g_end = min(t1 * (T / kNormGroup), p.n_groups32);
+    for (int gi = t0 * (T / kNormGroup) + tid; gi < g_end; gi += 128) km = fmaxf(km, kn[gi]);
     km = warp_max(km);
     if (lane == 0) red[wq] = km;
     named_bar_sync(1, 128);
@@ -243,20 +243,19 @@ __global__ void __launch_bounds__(192, 2)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
-      const int j = i & 1;
-      if (!mbar_wait_warp(s_full + j, (i >> 1) & 1, wc)) { ok = false; break; }
+      if (!mbar_wait_warp(s_full, i & 1, wc)) { ok = false; break; }
       tc_fence_after();
       uint32_t sa[32], sb[32], pk[32];
       if (warp_live) {
-        tmem_ld32(lane_base + Cfg::COL_S + j * 64, sa);
-        tmem_ld32(lane_base + Cfg::COL_S + j * 64 + 32, sb);
+        tmem_ld32(lane_base + Cfg::COL_S, sa);
+        tmem_ld32(lane_base + Cfg::COL_S + 32, sb);
         tmem_wait_ld();
       }
       tc_fence_before();
-      mbar_arrive(s_free + j);  // the tensor pipe may now overwrite S[j]
+      mbar_arrive_warp(s_free);  // the tensor pipe may now write S(i+1)
       if (warp_live) {
-        const int valid = L - (t0 + i) * kEncTile;
-        if (valid >= kEncTile) {
+        const int valid = L - (t0 + i) * T;
+        if (valid >= T) {
           exp2_chunk64<FLARE_ENC_POLY_PAIRS>(sa, sb, c, U, pk);
         } else {  // last, partial tile of the valid range: padded tokens get weight 0
 #pragma unroll
@@ -271,15 +270,15 @@ __global__ void __launch_bounds__(192, 2)
           }
         }
       }
-      // P[j] was last read by the value MMA of tile i-2
-      if (i >= 2 && !mbar_wait_warp(p_free + j, ((i >> 1) - 1) & 1, wc)) { ok = false; break; }
+      // P was last read by the value MMA of tile i-1
+      if (i >= 1 && !mbar_wait_warp(p_free, (i - 1) & 1, wc)) { ok = false; break; }
       tc_fence_after();
       if (warp_live) {
-        tmem_st32(lane_base + Cfg::COL_P + j * 32, pk);
+        tmem_st32(lane_base + Cfg::COL_P, pk);
         tmem_wait_st();
       }
       tc_fence_before();
-      mbar_arrive(p_full + j);
+      mbar_arrive_warp(p_full);
     }
     if (ok && mbar_wait_warp(o_full, 0, wc)) {
       tc_fence_after();
@@ -308,7 +307,7 @@ __global__ void __launch_bounds__(192, 2)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::TMEM_COLS);
   }
@@ -318,9 +317,10 @@ __global__ void __launch_bounds__(192, 2)
 
 size_t encode_smem_bytes(int D) {
   const size_t need = (D == 16 ? EncCfg<16>::BYTES : EncCfg<32>::BYTES) + 1024;
-  // Reserve enough shared memory that at most kSlotsPerSM CTAs share an SM:
-  // each CTA holds 256 of the 512 TMEM columns.
-  return need > 90 * 1024 ? need : 90 * 1024;
+  // Reserve enough shared memory that at most enc_ctas_per_sm(D) CTAs share
+  // an SM, so that every resident CTA finds its TMEM columns free.
+  const size_t floor = enc_ctas_per_sm(D) >= 3 ? 70 * 1024 : 100 * 1024;
+  return need > floor ? need : floor;
 }
 
 cudaError_t launch_encode(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
@@ -331,12 +331,12 @@ cudaError_t launch_encode(const CUtensorMap& tm_q, const CUtensorMap& tm_k, cons
     cudaError_t e = cudaFuncSetAttribute(encode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    encode_kernel<16><<<grid, 192, smem, s>>>(tm_q, tm_k, tm_v, p);
+    encode_kernel<16><<<grid, EncCfg<16>::THREADS, smem, s>>>(tm_q, tm_k, tm_v, p);
   } else {
     cudaError_t e = cudaFuncSetAttribute(encode_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    encode_kernel<32><<<grid, 192, smem, s>>>(tm_q, tm_k, tm_v, p);
+    encode_kernel<32><<<grid, EncCfg<32>::THREADS, smem, s>>>(tm_q, tm_k, tm_v, p);
   }
   return cudaGetLastError();
 }

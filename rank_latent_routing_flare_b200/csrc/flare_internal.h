@@ -11,7 +11,6 @@
 
 namespace flare {
 
-constexpr int kSlotsPerSM = 2;     // co-resident CTAs per SM for the softmax kernels
 constexpr int kNumSM = 148;        // B200
 constexpr int kEncTile = 64;       // tokens per encode tile
 constexpr int kLatBlock = 128;     // latents per encode CTA (UMMA M)
@@ -20,11 +19,20 @@ constexpr int kDecChunk = 64;      // latents per decode chunk (UMMA N)
 constexpr int kNormGroup = 32;     // tokens per key-norm group
 constexpr int kProjTile = 128;     // tokens per projection tile
 
+// Co-resident CTAs per SM of the encoder: 128 TMEM columns per CTA for
+// D = 16 (three CTAs), 256 for D = 32 (two).
+__host__ __device__ constexpr int enc_ctas_per_sm(int D) { return D == 16 ? 3 : 2; }
+// Same for the decoder.
+#ifndef FLARE_DEC_CTAS_D16
+#define FLARE_DEC_CTAS_D16 3
+#endif
+__host__ __device__ constexpr int dec_ctas_per_sm(int D) { return D == 16 ? FLARE_DEC_CTAS_D16 : 2; }
+
 // Of the 32 score pairs of each 64-column softmax chunk, how many are
 // exponentiated on the FMA pipe (polynomial) instead of the MUFU; chosen by
-// measurement on B200.
+// measurement on B200 (the encoder gains ~2% with 4, the decoder loses).
 #ifndef FLARE_ENC_POLY_PAIRS
-#define FLARE_ENC_POLY_PAIRS 0
+#define FLARE_ENC_POLY_PAIRS 4
 #endif
 #ifndef FLARE_DEC_POLY_PAIRS
 #define FLARE_DEC_POLY_PAIRS 0
@@ -106,6 +114,8 @@ struct DecodeParams {
   const uint16_t* z;    // bf16 [B*H][M][D]
   const uint16_t* k;    // bf16 [B*H][N][D]
   uint16_t* y;          // bf16 [B*H][N][D]
+  uint32_t* fb_count;   // number of listed tokens (zeroed before the decoder runs)
+  uint64_t* fb_list;    // tokens (bh * N + n) whose row sum underflowed, capacity B*H*N
   uint32_t* err;
   unsigned long long timeout_ns;
 };

@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int j = 0; j < 2; ++j) {
       mbar_init(acc_full + j, 1);
-      mbar_init(acc_free + j, 128);
+      mbar_init(acc_free + j, 4);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(acc_free + ab);
+      mbar_arrive_warp(acc_free + ab);
     }
   }
   tc_fence_before();
