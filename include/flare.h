@@ -157,6 +157,36 @@ FLARE_API flare_status flare_last_device_status(void* workspace, void* stream);
 FLARE_API const char* flare_status_string(flare_status status);
 
 /*
+ * FLARE mixer forward for callers that cannot allocate device memory.
+ *
+ * The paper has no counterpart to this call; it exists for callers that
+ * must not call cudaMalloc (or any allocating routine) themselves, for
+ * example code running where device allocation is forbidden or has to stay
+ * under a fixed budget.  It computes exactly what flare_mixer_fwd computes,
+ * with the same arguments minus the workspace: its scratch lives in a
+ * fixed array of FLARE_STATIC_SCRATCH_BYTES bytes inside the library's
+ * device image, which every GPU that loads the library keeps until the
+ * process exits.  The call allocates nothing.
+ *
+ *   - Sizes whose workspace (flare_workspace_bytes(FLARE_VARIANT_FLARE, ...))
+ *     exceeds FLARE_STATIC_SCRATCH_BYTES are rejected with
+ *     FLARE_ERR_WORKSPACE before anything is enqueued.
+ *   - The first call on each device looks up the array's device address
+ *     with that device current (cudaGetSymbolAddress); make that first call
+ *     before any stream capture.
+ *   - Every call, on every stream, shares the one array, and the array keeps
+ *     the last call's contents (the words that must start at zero are
+ *     cleared by each call).  Calls whose execution overlaps on the GPU race
+ *     on the scratch and give wrong results: serialise them.
+ *   - The device error word lives in the shared array, so
+ *     flare_last_device_status() cannot be used with this call.
+ */
+#define FLARE_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
+FLARE_API flare_status flare_mixer_fwd_static(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q,
+                                              flare_bf16* Y, int B, int H, int N, int M, int D,
+                                              const int32_t* lengths, float scale, void* stream, float* Z_out);
+
+/*
  * Self-test of the bounded-wait error path: enqueues one small kernel that
  * waits on an mbarrier nothing ever completes, with a limit of `timeout_ns`
  * nanoseconds (clamped to [1e3, 1e9]).  The wait expires, the kernel records

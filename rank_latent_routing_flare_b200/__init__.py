@@ -13,6 +13,7 @@ from ._binding import (  # noqa: F401
     Status,
     flare_last_device_status,
     flare_mixer_fwd,
+    flare_mixer_fwd_static,
     flare_selftest_wait_timeout,
     flare_status_string,
     flare_workspace_bytes,

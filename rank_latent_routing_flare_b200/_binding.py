@@ -60,6 +60,8 @@ def load_library(build_if_missing: bool = True):
         lib.flare_mixer_fwd_profiled.restype = i
         lib.flarepp_mixer_fwd_profiled.argtypes = lib.flarepp_mixer_fwd.argtypes + [vp]
         lib.flarepp_mixer_fwd_profiled.restype = i
+        lib.flare_mixer_fwd_static.argtypes = [vp, vp, vp, vp, i, i, i, i, i, vp, f, vp, vp]
+        lib.flare_mixer_fwd_static.restype = i
         lib.flare_last_device_status.argtypes = [vp, vp]
         lib.flare_last_device_status.restype = i
         lib.flare_status_string.argtypes = [i]
@@ -193,6 +195,30 @@ def flarepp_mixer_fwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, lengths=None, scale: float 
         st = load_library().flarepp_mixer_fwd_profiled(*args, _event_array(stage_events))
     if st != 0:
         raise FlareError(st, "flarepp_mixer_fwd")
+    return Y
+
+
+FLARE_STATIC_SCRATCH_BYTES = 64 << 20
+
+
+def flare_mixer_fwd_static(K, V, Q, lengths=None, scale: float = 0.0, Y=None, stream=None, Z_out=None):
+    """FLARE forward without a caller-provided workspace (the library's fixed
+    device scratch of FLARE_STATIC_SCRATCH_BYTES is used; nothing is
+    allocated by the library).  Calls must not overlap on the GPU."""
+    torch = _torch()
+    B, H, N, D = K.shape
+    M = Q.shape[1]
+    _check_dev("K", K, torch.bfloat16)
+    _check_dev("V", V, torch.bfloat16, K.shape)
+    _check_dev("Q", Q, torch.bfloat16, (H, M, D))
+    _check_dev("lengths", lengths, torch.int32, (B,))
+    _check_dev("Z_out", Z_out, torch.float32, (B, H, M, D))
+    if Y is None:
+        Y = torch.empty_like(K)
+    st = load_library().flare_mixer_fwd_static(_ptr(K), _ptr(V), _ptr(Q), _ptr(Y), B, H, N, M, D, _ptr(lengths),
+                                               float(scale), _stream_ptr(stream, K.device), _ptr(Z_out))
+    if st != 0:
+        raise FlareError(st, "flare_mixer_fwd_static")
     return Y
 
 

@@ -229,6 +229,35 @@ flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
 }  // namespace
 }  // namespace flare
 
+namespace flare {
+namespace {
+
+// Scratch for callers that cannot allocate device memory (see
+// flare_mixer_fwd_static): a fixed array in the library's device image.
+// Every device that loads the library holds it until the process exits.
+static __device__ __align__(256) unsigned char g_static_scratch[FLARE_STATIC_SCRATCH_BYTES];
+
+// Device address of g_static_scratch on the current device.  Host code must
+// not pass the symbol itself to a kernel (on the host it is only a stand-in);
+// its device address is looked up once per device, with that device current.
+flare_status static_scratch_address(void** out) {
+  static std::mutex mu;
+  static void* addr[256] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return FLARE_ERR_LAUNCH;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return FLARE_ERR_LAUNCH;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return FLARE_OK;
+}
+
+}  // namespace
+}  // namespace flare
+
 using namespace flare;
 
 extern "C" {
@@ -362,6 +391,24 @@ flare_status flarepp_mixer_fwd(const flare_bf16* X, const flare_bf16* Wk, const 
                                float* Z_out) {
   return flarepp_mixer_fwd_profiled(X, Wk, Wv, Wk_syn, Wv_syn, Q0, Y, B, N, C, H, M, D, lengths, scale, workspace,
                                     workspace_bytes, stream, Qx_out, Z_out, nullptr);
+}
+
+flare_status flare_mixer_fwd_static(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, flare_bf16* Y,
+                                    int B, int H, int N, int M, int D, const int32_t* lengths, float scale,
+                                    void* stream, float* Z_out) {
+  // Same argument checks as flare_mixer_fwd, then the size limit of the
+  // static scratch, all before any CUDA call.
+  if (!K || !V || !Q || !Y) return FLARE_ERR_NULL;
+  flare_status st = check_common(B, H, N, M, D);
+  if (st != FLARE_OK) return st;
+  if (!aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(Y) || !aligned16(lengths) || !aligned16(Z_out))
+    return FLARE_ERR_ALIGN;
+  if (make_plan(FLARE_VARIANT_FLARE, B, H, N, M, D).total > FLARE_STATIC_SCRATCH_BYTES) return FLARE_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  st = static_scratch_address(&scratch);
+  if (st != FLARE_OK) return st;
+  return flare_mixer_fwd(K, V, Q, Y, B, H, N, M, D, lengths, scale, scratch, FLARE_STATIC_SCRATCH_BYTES, stream,
+                         Z_out);
 }
 
 flare_status flare_last_device_status(void* workspace, void* stream) {

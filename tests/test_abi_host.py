@@ -30,7 +30,7 @@ def declared_functions():
 def test_header_declares_the_abi():
     names = declared_functions()
     assert names == sorted(["flare_workspace_bytes", "flare_mixer_fwd", "flarepp_mixer_fwd",
-                            "flare_mixer_fwd_profiled", "flarepp_mixer_fwd_profiled",
+                            "flare_mixer_fwd_profiled", "flarepp_mixer_fwd_profiled", "flare_mixer_fwd_static",
                             "flare_last_device_status", "flare_status_string",
                             "flare_selftest_wait_timeout"])
 
@@ -142,3 +142,13 @@ def test_valid_call_without_gpu_reports_launch_error():
     lib = fl.load_library()
     assert lib.flare_selftest_wait_timeout(W, None, 1000) == Status.ERR_LAUNCH
     assert lib.flare_last_device_status(None, None) == Status.ERR_NULL
+
+
+def test_static_scratch_entry_point_rejects_oversized_problems():
+    """Sizes whose workspace exceeds the fixed scratch are refused on the host."""
+    lib = fl.load_library()
+    assert fl.flare_workspace_bytes(0, 64, 8, 1 << 20, 512, 16) > fl._binding.FLARE_STATIC_SCRATCH_BYTES
+    st = lib.flare_mixer_fwd_static(A, A, A, A, 64, 8, 1 << 20, 512, 16, None, 0.0, None, None)
+    assert st == Status.ERR_WORKSPACE
+    assert lib.flare_mixer_fwd_static(None, A, A, A, 1, 1, 64, 16, 16, None, 0.0, None, None) == Status.ERR_NULL
+    assert lib.flare_mixer_fwd_static(A, A, A, A + 2, 1, 1, 64, 16, 16, None, 0.0, None, None) == Status.ERR_ALIGN
