@@ -159,12 +159,17 @@ def stage_work(w):
 
 def kernel_traffic(kernel_file: str, workload: str):
     """dram bytes per launch from a committed ncu summary, if that summary was
-    taken on the current source of the kernel (else None)."""
+    taken on the current source of the kernel (its .cu file, ptx.cuh and
+    flare_internal.h); else None."""
     prof = os.path.join(ROOT, "profiles")
-    src = os.path.join(ROOT, "rank_latent_routing_flare_b200", "csrc", kernel_file)
-    if not os.path.isdir(prof) or not os.path.exists(src):
+    csrc = os.path.join(ROOT, "rank_latent_routing_flare_b200", "csrc")
+    srcs = [os.path.join(csrc, f) for f in (kernel_file, "ptx.cuh", "flare_internal.h")]
+    if not os.path.isdir(prof) or not all(os.path.exists(f) for f in srcs):
         return None
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for f in srcs:
+        h.update(open(f, "rb").read())
+    sha = h.hexdigest()[:16]
     for f in sorted(os.listdir(prof)):
         if not f.endswith(".md"):
             continue
@@ -177,6 +182,34 @@ def kernel_traffic(kernel_file: str, workload: str):
                 and m_w.group(1) == workload:
             return float(m_t.group(1))
     return None
+
+
+# ---------------------------------------------------------------------------
+# ranks (weak scaling: every rank runs its own copy of the workload)
+# ---------------------------------------------------------------------------
+
+LAUNCHES_PER_STEP = 7   # project, synth encode, synth merge, encode, merge, decode, decode fallback
+
+
+def rank_seed(rank: int):
+    """Seed of a rank's synthetic input: rank 0 uses the workload's own seed."""
+    return None if rank == 0 else 1000 + rank
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest value of x over all ranks (every rank gets it)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_rank: float, ms: float) -> float:
+    """Units processed by all ranks per second, timed by the slowest rank."""
+    return world * units_per_rank / (ms * 1e-3)
 
 
 # ---------------------------------------------------------------------------
@@ -293,7 +326,7 @@ def main():
     fl.load_library()
 
     # inputs: each rank its own synthetic sample of the workload (weak scaling)
-    w = make_workload(args.workload, N=args.tokens, seed=None if rank == 0 else 1000 + rank)
+    w = make_workload(args.workload, N=args.tokens, seed=rank_seed(rank))
     assert w.variant == "flarepp"
 
     def to_dev(bits):
@@ -333,13 +366,9 @@ def main():
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
-    ms = ev0.elapsed_time(ev1) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world, dev)
     th_per_rank = w.B * w.H * (w.valid_tokens() // w.B if w.lengths is not None else w.N)
-    value = world * th_per_rank / (ms * 1e-3)
+    value = whole_job_rate(world, th_per_rank, ms)
 
     # per-stage device times (same timed steps, same stream)
     stage_ms = {s: 0.0 for s in STAGES_PP}
@@ -430,12 +459,10 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
     if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         dist.barrier()
-    e2e_value = world * th_per_rank / (e2e_ms * 1e-3)
+    e2e_value = whole_job_rate(world, th_per_rank, e2e_ms)
 
     line = None
     if rank == 0:
@@ -458,7 +485,7 @@ def main():
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms},
-            "gpu_launches": 6 * args.steps,
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": clk,
         }
     if world > 1:

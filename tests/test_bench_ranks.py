@@ -1,0 +1,75 @@
+"""Host logic of bench.py's multi-rank path (weak scaling), on CPU.
+
+With --gpus N every rank runs its own copy of the workload on its own seed;
+the step time is the slowest rank's and the whole-job rate counts the units
+of all ranks.  The reference arm does its work on rank 0 only.  The timing
+reduction runs here on two gloo ranks."""
+import datetime
+import multiprocessing
+import os
+import socket
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from workloads import make_workload  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, ms, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        got = bench.max_over_ranks(ms[rank], world, "cpu")
+        out.put((rank, got, bench.whole_job_rate(world, 8 * 1024, got)))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_step_time_is_the_slowest_rank_and_rate_counts_all_ranks():
+    world, ms = 2, [3.0, 5.0]
+    ctx = multiprocessing.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, ms, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = sorted(out.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, got, rate in results:
+        assert got == 5.0
+        assert rate == world * 8 * 1024 / 5e-3
+
+
+def test_single_rank_needs_no_process_group():
+    assert bench.max_over_ranks(4.5, 1, None) == 4.5
+    assert bench.whole_job_rate(1, 1000, 2.0) == 500_000.0
+
+
+def test_each_rank_draws_its_own_input_of_the_same_shape():
+    w0 = make_workload(bench.WORKLOAD, N=256, seed=bench.rank_seed(0))
+    w1 = make_workload(bench.WORKLOAD, N=256, seed=bench.rank_seed(1))
+    assert w0.seed == 3 and w1.seed != w0.seed
+    assert w0.X.shape == w1.X.shape and not np.array_equal(w0.X, w1.X)
+    assert np.array_equal(w0.Wk, make_workload(bench.WORKLOAD, N=256).Wk)
+
+
+def test_reference_arm_works_on_rank_zero_only(capsys):
+    class Args:
+        workload, steps, warmup = bench.WORKLOAD, 1, 3
+    assert bench.run_reference(Args, rank=1, world=2) == 0
+    assert capsys.readouterr().out == ""
