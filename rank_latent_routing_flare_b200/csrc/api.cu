@@ -103,7 +103,7 @@ struct Plan {
 Plan make_plan(int variant, long B, long H, long N, long M, long D) {
   Plan p;
   const long BH = B * H;
-  const long ntiles = cdiv(N, kEncTile);
+  const long ntiles = cdiv(N, enc_tile(static_cast<int>(D)));
   p.LB = static_cast<int>(cdiv(M, kLatBlock));
   p.S = choose_splits(BH * p.LB, ntiles, static_cast<long>(kNumSM) * enc_ctas_per_sm(static_cast<int>(D)));
   p.tps = static_cast<int>(cdiv(ntiles, p.S));
@@ -166,7 +166,7 @@ flare_status run_encode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
   const long G = q_per_batch ? BH : H;
   CUtensorMap tq, tk, tv;
   if (!map3d(&tq, q, D, M, G, D, std::min(M, kLatBlock), row_swizzle(D)) ||
-      !map3d(&tk, k, D, N, BH, D, kEncTile, row_swizzle(D)) || !map3d(&tv, v, D, N, BH, D, kEncTile, row_swizzle(D)))
+      !map3d(&tk, k, D, N, BH, D, enc_tile(D), row_swizzle(D)) || !map3d(&tv, v, D, N, BH, D, enc_tile(D), row_swizzle(D)))
     return FLARE_ERR_LAUNCH;
   EncodeParams ep{};
   ep.B = B; ep.H = H; ep.N = N; ep.M = M; ep.D = D;
@@ -203,15 +203,15 @@ flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
   const long BH = static_cast<long>(B) * H;
   const long G = q_per_batch ? BH : H;
   CUtensorMap tq, tz, tk;
-  const int chunk_rows = std::min(M, kDecChunk);
-  if (!map3d(&tq, q, D, M, G, D, chunk_rows, row_swizzle(D)) || !map3d(&tz, z16, D, M, BH, D, chunk_rows, row_swizzle(D)) ||
+  const int box_rows = std::min(M, 256);
+  if (!map3d(&tq, q, D, M, G, D, box_rows, row_swizzle(D)) || !map3d(&tz, z16, D, M, BH, D, box_rows, row_swizzle(D)) ||
       !map3d(&tk, k, D, N, BH, D, kDecTile, row_swizzle(D)))
     return FLARE_ERR_LAUNCH;
   DecodeParams dp{};
   dp.B = B; dp.H = H; dp.N = N; dp.M = M; dp.D = D;
   dp.q_per_batch = q_per_batch;
   dp.tiles_per_cta = pl.dec_tiles; dp.ctas_per_head = pl.dec_ctas;
-  dp.chunk_rows = chunk_rows;
+  dp.qz_box_rows = box_rows;
   dp.scale = scale; dp.c = scale * 1.4426950408889634f;
   dp.lengths = lengths;
   dp.q = static_cast<const uint16_t*>(q);

@@ -4,22 +4,32 @@
 //
 // One CTA owns one head (b, h) and a contiguous range of 128-token tiles.  The
 // head's queries Q (M x D) and latent values Z (M x D) stay resident in shared
-// memory; key tiles stream through a TMA ring.  Per tile and per 64-latent
-// chunk c:
-//   S = K_tile Q_c^T               UMMA M=128 (tokens) x N=64 (latents), fp32 TMEM
+// memory; key tiles stream through a TMA ring.  Per tile and per chunk of C
+// latents (C = dec_chunk(D); the last chunk may be shorter):
+//   S = K_tile Q_c^T               UMMA M=128 (tokens) x N=C (latents), fp32 TMEM
 //   P = 2^(S * c - nu_n)           softmax threads, one token row per thread
 //   Y += P [Z_c | 1]               UMMA with A = P read from TMEM; column D of Y
 //                                  accumulates the row sum
 // nu_n = c * |k_n| * max_m |q_m| bounds the token's scaled scores from above
 // (Cauchy-Schwarz), so the latent chunks need no running maximum.  A token
-// whose sum underflows (only possible when the bound is very loose) is
-// recomputed exactly by its own thread from global memory.
+// whose sum underflows (only possible when the bound is very loose) is listed
+// and recomputed exactly by decode_fallback_kernel.
 //
-// Warp roles (5 warps): warp 0 lane 0 is the control thread: it loads Q and
-// Z, keeps the key-tile ring full (TMA) and issues the MMAs in program order,
-// blocking on exactly the next event.  Warps 1..4 are the softmax warps
-// (thread <-> TMEM lane <-> token).  A CTA needs 128 TMEM columns for D = 16,
-// so three CTAs share an SM.
+// The chunks of all tiles form one sequence q = tile * nc + chunk.  TMEM holds
+// two score buffers (chunk q uses buffer q % 2; the softmax threads write P_q
+// over the first C/2 columns of S_q once S_q is in registers) and the Y
+// accumulator.  The MMA thread computes S_{q+1} while the softmax threads work
+// on S_q; S_{q+2} reuses the buffer once the value MMA of chunk q is done.
+// Every barrier reused across chunks exists once per buffer, so no party can
+// run a full phase ahead of the party that waits on it.  The epilogue of a
+// tile (Y / sum, bf16 stores) runs after the first chunk of the next tile.
+//
+// Warp roles (5 warps): warp 0 lane 0 is the MMA thread (it also loads Q, Z
+// and the first key tiles).  Warps 1..4 are the softmax warps (thread <->
+// TMEM lane <-> token); one of them, in rotation, refills the key ring.  A
+// CTA needs 128 TMEM columns for D = 16, so four CTAs share an SM.
+#include <type_traits>
+
 #include "ptx.cuh"
 
 namespace flare {
@@ -27,27 +37,29 @@ namespace {
 
 template <int D>
 struct DecCfg {
+  static constexpr int C = dec_chunk(D);                // latents per chunk
   static constexpr int ROWB = D * 2;
   static constexpr int KT_B = kDecTile * ROWB;          // one key tile
-  static constexpr int CH_B = kDecChunk * ROWB;         // one 64-latent chunk of Q or Z
-  static constexpr int MAXCH = 512 / kDecChunk;         // M <= 512
-  static constexpr int NST = 4;
+  static constexpr int QZ_B = 512 * ROWB;               // all of Q (or Z): M <= 512
+  static constexpr int NST = 4;                         // key ring stages
   static constexpr uint32_t LAYOUT = (D == 16) ? LAYOUT_SW32 : LAYOUT_SW64;
   static constexpr uint32_t SBO = 8 * ROWB;
   static constexpr int NY = D + 16;                     // Y columns: D values + sums
-  static constexpr int OFF_Q = 0;                       // MAXCH * CH_B
-  static constexpr int OFF_Z = OFF_Q + MAXCH * CH_B;
-  static constexpr int OFF_ONES = OFF_Z + MAXCH * CH_B; // CH_B
-  static constexpr int OFF_K = OFF_ONES + CH_B;         // NST * KT_B
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_Z = OFF_Q + QZ_B;
+  static constexpr int OFF_ONES = OFF_Z + QZ_B;         // C x ROWB block of ones
+  static constexpr int OFF_K = OFF_ONES + C * ROWB;     // NST * KT_B
   static constexpr int OFF_BAR = OFF_K + NST * KT_B;
   static constexpr int OFF_MISC = OFF_BAR + 8 * 32;
-  static constexpr int BYTES = OFF_MISC + 64;
-  // TMEM columns: S at 0 (fp32 scores of one 64-latent chunk), P at 64 (bf16
-  // pairs), Y at 96 (D values + the row-sum block)
-  static constexpr uint32_t COL_S = 0, COL_P = 64, COL_Y = 96;
+  static constexpr int BYTES = OFF_MISC + 64 + NST * 4;
+  // TMEM columns: score buffers at 0 and C (each later holds its P), Y at 2C
+  static constexpr uint32_t COL_Y = 2 * C;
   static constexpr uint32_t TMEM_COLS = (COL_Y + NY <= 128) ? 128 : 256;
   static constexpr int THREADS = 160;
   static constexpr int CTAS_PER_SM = dec_ctas_per_sm(D);
+  static_assert(TMEM_COLS <= 512 / CTAS_PER_SM, "TMEM columns of the co-resident CTAs exceed 512");
+  static_assert(OFF_K % 512 == 0 || D == 16, "key tiles must start on a swizzle atom");
+  static_assert(OFF_K % 256 == 0, "key tiles must start on a swizzle atom");
 };
 
 __device__ __forceinline__ float bf16_row_norm2(const uint4* row, int n16) {
@@ -117,7 +129,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
     decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_z,
                   const __grid_constant__ CUtensorMap tm_k, const DecodeParams p) {
   using Cfg = DecCfg<D>;
-  constexpr int NST = Cfg::NST;
+  constexpr int NST = Cfg::NST, C = Cfg::C;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sq = sm + Cfg::OFF_Q;
@@ -126,18 +138,17 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
   uint8_t* sk = sm + Cfg::OFF_K;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Cfg::OFF_BAR);
   uint64_t* qz_full = bars;
-  uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = bars + 1 + NST;
-  uint64_t* s_full = bars + 1 + 2 * NST;  // S computed
-  uint64_t* s_free = s_full + 1;           // S loaded by every softmax warp
-  uint64_t* p_full = s_full + 2;           // P stored by every softmax warp
-  uint64_t* p_free = s_full + 3;           // P consumed by the value MMA
-  uint64_t* y_full = s_full + 4;           // Y of a tile complete
-  uint64_t* y_free = s_full + 5;           // Y read by every softmax warp
-  uint64_t* mma_done = s_full + 6;
+  uint64_t* k_full = bars + 1;             // [NST] key tile landed
+  uint64_t* s_full = bars + 1 + NST;       // [2] score buffer computed
+  uint64_t* pv_done = s_full + 2;          // [2] value MMA done reading the buffer's P
+  uint64_t* p_full = s_full + 4;           // [2] P stored by every softmax warp
+  uint64_t* y_full = s_full + 6;           // Y of a tile complete
+  uint64_t* y_free = s_full + 7;           // Y read by every softmax warp
+  uint64_t* mma_done = s_full + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(sm + Cfg::OFF_MISC + 4);
   float* red = reinterpret_cast<float*>(sm + Cfg::OFF_MISC + 16);
+  volatile int* last_load = reinterpret_cast<volatile int*>(sm + Cfg::OFF_MISC + 64);  // per stage
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.x / p.ctas_per_head;
@@ -159,7 +170,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
   const int tb = min(ta + p.tiles_per_cta, tiles_head);
   const int tc_end = min(tb, tiles_valid);            // tiles [ta, tc_end) are computed
   const int ntiles = max(0, tc_end - ta);
-  const int nc = (p.M + kDecChunk - 1) / kDecChunk;   // latent chunks
+  const int nc = (p.M + C - 1) / C;                   // latent chunks
   uint16_t* yh = p.y + static_cast<size_t>(bh) * p.N * D;
 
   // tiles entirely past the valid length: zero rows
@@ -177,19 +188,20 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
     mbar_init(qz_full, 1);
     for (int i = 0; i < NST; ++i) {
       mbar_init(k_full + i, 1);
-      mbar_init(k_empty + i, 1);
+      last_load[i] = -1;
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 4);
-    mbar_init(p_full, 4);
-    mbar_init(p_free, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full + i, 1);
+      mbar_init(pv_done + i, 1);
+      mbar_init(p_full + i, 4);
+    }
     mbar_init(y_full, 1);
     mbar_init(y_free, 4);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  for (int i = threadIdx.x; i < Cfg::CH_B / 4; i += blockDim.x)
+  for (int i = threadIdx.x; i < C * Cfg::ROWB / 4; i += blockDim.x)
     reinterpret_cast<uint32_t*>(sones)[i] = 0x3F803F80u;  // bf16 1.0 pairs
   fence_proxy_async_smem();
   if (warp == 0) {
@@ -201,86 +213,97 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{p.err, abort_flag, p.timeout_ns};
+  // key tile n (of this CTA's range) into ring stage n % NST (one thread)
+  auto load_tile = [&](int n) {
+    const int st = n % NST;
+    mbar_arrive_expect_tx(k_full + st, Cfg::KT_B);
+    tma_load_3d(sk + st * Cfg::KT_B, &tm_k, k_full + st, 0, (ta + n) * kDecTile, bh);
+    last_load[st] = n;
+  };
+  const int total = ntiles * nc;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ control thread
+    // ------------------------------------------------------------ MMA thread
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_z);
       tma_prefetch_desc(&tm_k);
-      mbar_arrive_expect_tx(qz_full, 2 * nc * p.chunk_rows * Cfg::ROWB);
-      for (int c = 0; c < nc; ++c) {
-        tma_load_3d(sq + c * Cfg::CH_B, &tm_q, qz_full, 0, c * kDecChunk, g);
-        tma_load_3d(sz + c * Cfg::CH_B, &tm_z, qz_full, 0, c * kDecChunk, bh);
+      const int nbox = (p.M + p.qz_box_rows - 1) / p.qz_box_rows;
+      mbar_arrive_expect_tx(qz_full, 2 * nbox * p.qz_box_rows * Cfg::ROWB);
+      for (int bx = 0; bx < nbox; ++bx) {
+        tma_load_3d(sq + bx * p.qz_box_rows * Cfg::ROWB, &tm_q, qz_full, 0, bx * p.qz_box_rows, g);
+        tma_load_3d(sz + bx * p.qz_box_rows * Cfg::ROWB, &tm_z, qz_full, 0, bx * p.qz_box_rows, bh);
       }
+      for (int n = 0; n < min(NST, ntiles); ++n) load_tile(n);
       const uint32_t idesc_y = idesc_bf16_f32(128, Cfg::NY, false, true);
-      const uint32_t sq_a = smem_u32(sq), sz_a = smem_u32(sz), ones_a = smem_u32(sones);
-      auto chunk_n = [&](int cc) { return min(kDecChunk, p.M - cc * kDecChunk); };
-      int n_load = 0;
-      auto load = [&]() {
-        const int st = n_load % NST;
-        mbar_arrive_expect_tx(k_full + st, Cfg::KT_B);
-        tma_load_3d(sk + st * Cfg::KT_B, &tm_k, k_full + st, 0, (ta + n_load) * kDecTile, bh);
-        ++n_load;
+      const uint32_t sz_a = smem_u32(sz), ones_a = smem_u32(sones);
+      const uint64_t q_desc = umma_desc(smem_u32(sq), 16, Cfg::SBO, Cfg::LAYOUT);
+      const uint64_t k_desc = umma_desc(smem_u32(sk), 16, Cfg::SBO, Cfg::LAYOUT);
+      // chunk q = tile * nc + cc, tracked incrementally (no division per chunk)
+      struct Cursor {
+        int q, tile, cc;
       };
-      auto refill = [&]() {
-        while (n_load < ntiles && mbar_test(k_empty + n_load % NST, ((n_load / NST) & 1) ^ 1)) load();
-      };
-      auto issue_s = [&](int qq) -> bool {
-        const int tile = qq / nc, cc = qq - tile * nc;
-        const int st = tile % NST;
-        if (cc == 0) {
-          while (n_load <= tile) {
-            if (!mbar_wait(k_empty + n_load % NST, ((n_load / NST) & 1) ^ 1, wc)) return false;
-            load();
-          }
-          if (!mbar_wait(k_full + st, (tile / NST) & 1, wc)) return false;
+      auto advance = [&](Cursor& x) {
+        ++x.q;
+        if (++x.cc == nc) {
+          x.cc = 0;
+          ++x.tile;
         }
+      };
+      const int last_n = p.M - (nc - 1) * C;            // latents of the last chunk
+      const uint32_t idesc_full = idesc_bf16_f32(128, C, false, false);
+      const uint32_t idesc_last = idesc_bf16_f32(128, last_n, false, false);
+      constexpr uint64_t CH_STEP = (C * Cfg::ROWB) >> 4;  // descriptor units per chunk
+      // [Z_c | 1]: chunk c starts CH_STEP * c further on, and its ones block
+      // (leading byte offset) is that much closer
+      const uint64_t z_desc = umma_desc(sz_a, ones_a - sz_a, Cfg::SBO, Cfg::LAYOUT);
+      // S_q = K_tile Q_c^T into buffer q % 2, once the key tile has landed and
+      // P_{q-2} has been consumed
+      auto issue_s = [&](const Cursor& x) -> bool {
+        const int buf = x.q & 1, st = x.tile % NST;
+        if (x.cc == 0 && !mbar_wait(k_full + st, (x.tile / NST) & 1, wc)) return false;
+        if (x.q >= 2 && !mbar_wait(pv_done + buf, ((x.q - 2) >> 1) & 1, wc)) return false;
         tc_fence_after();
-        const uint32_t k_a = smem_u32(sk + st * Cfg::KT_B);
-        const uint32_t idesc_s = idesc_bf16_f32(128, chunk_n(cc), false, false);
+        const uint32_t idesc_s = x.cc == nc - 1 ? idesc_last : idesc_full;
+        const uint64_t kd = k_desc + static_cast<uint64_t>(st) * (Cfg::KT_B >> 4);
+        const uint64_t qd = q_desc + static_cast<uint64_t>(x.cc) * CH_STEP;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          umma_ss(tmem + Cfg::COL_S, umma_desc(k_a + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT),
-                  umma_desc(sq_a + cc * Cfg::CH_B + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT), idesc_s, kk > 0 ? 1u : 0u);
-        umma_commit(s_full);
+          umma_ss(tmem + buf * C, kd + 2 * kk, qd + 2 * kk, idesc_s, kk > 0 ? 1u : 0u);
+        umma_commit(s_full + buf);
         return true;
       };
-      auto issue_pv = [&](int qq) -> bool {
-        const int tile = qq / nc, cc = qq - tile * nc;
-        // the first value MMA of a tile overwrites Y: the previous tile's
-        // epilogue must have read it
-        if (cc == 0 && tile >= 1 && !mbar_wait(y_free, (tile - 1) & 1, wc)) return false;
-        if (!mbar_wait(p_full, qq & 1, wc)) return false;
+      // Y += P_q [Z_c | 1] once every softmax warp has stored P_q (and, for a
+      // tile's first chunk, has read the previous tile's Y)
+      auto issue_pv = [&](const Cursor& x) -> bool {
+        const int buf = x.q & 1;
+        if (!mbar_wait(p_full + buf, (x.q >> 1) & 1, wc)) return false;
+        if (x.cc == 0 && x.tile >= 1 && !mbar_wait(y_free, (x.tile - 1) & 1, wc)) return false;
         tc_fence_after();
-        const uint32_t z_a = sz_a + cc * Cfg::CH_B;
-        const uint32_t lbo = ones_a - z_a;  // [Z_c | 1]: second N-atom = ones block
-        const int nks = chunk_n(cc) / 16;
-        for (int ks = 0; ks < nks; ++ks) {
-          const uint64_t bdesc = umma_desc(z_a + ks * 16 * Cfg::ROWB, lbo, Cfg::SBO, Cfg::LAYOUT);
-          umma_ts(tmem + Cfg::COL_Y, tmem + Cfg::COL_P + ks * 8, bdesc, idesc_y, (cc > 0 || ks > 0) ? 1u : 0u);
-        }
-        umma_commit(p_free);
-        if (cc == nc - 1) {
-          umma_commit(y_full);
-          umma_commit(k_empty + (tile % NST));
-        }
+        const uint64_t step = static_cast<uint64_t>(x.cc) * CH_STEP;
+        const uint64_t zd = z_desc + step - (step << 16);
+        const int nks = (x.cc == nc - 1 ? last_n : C) / 16;
+        for (int ks = 0; ks < nks; ++ks)
+          umma_ts(tmem + Cfg::COL_Y, tmem + buf * C + ks * 8, zd + static_cast<uint64_t>((ks * 16 * Cfg::ROWB) >> 4),
+                  idesc_y, (x.cc > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(pv_done + buf);
+        if (x.cc == nc - 1) umma_commit(y_full);
         return true;
       };
-      const int total = ntiles * nc;
-      refill();
-      bool ok = mbar_wait(qz_full, 0, wc) && issue_s(0);
-      for (int qq = 1; ok && qq < total; ++qq) {
-        ok = mbar_wait(s_free, (qq - 1) & 1, wc) && issue_s(qq);  // S(q-1) loaded -> S(q)
-        if (ok) ok = issue_pv(qq - 1);                              // P(q-1) stored -> P(q-1) [Z | 1]
-        if (ok) refill();
+      Cursor cs{0, 0, 0}, cp{0, 0, 0};
+      bool ok = mbar_wait(qz_full, 0, wc) && issue_s(cs);
+      advance(cs);
+      if (ok && total > 1) ok = issue_s(cs);
+      advance(cs);
+      for (; ok && cp.q < total; advance(cp)) {
+        ok = issue_pv(cp);
+        if (ok && cs.q < total) {
+          ok = issue_s(cs);
+          advance(cs);
+        }
       }
-      if (ok) issue_pv(total - 1);
       umma_commit(mma_done);  // every MMA issued above is complete before TMEM is freed
       mbar_wait_drain(mma_done, 0, p.timeout_ns);
-      for (int i = max(0, n_load - NST); i < n_load; ++i)
-        mbar_wait_drain(k_full + (i % NST), (i / NST) & 1, p.timeout_ns);
-      mbar_wait_drain(qz_full, 0, p.timeout_ns);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -299,8 +322,6 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
     const float c = p.c;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     // Epilogue of tile i: Y = acc / sum, zero rows for padding, bf16 stores.
-    // It runs inside chunk 0 of tile i+1, after the P store (the value MMA of
-    // the tile's last chunk has completed by then).
     auto epilogue = [&](int i) -> bool {
       if (!mbar_wait_warp(y_full, i & 1, wc)) return false;
       tc_fence_after();
@@ -346,63 +367,66 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
       }
       return true;
     };
-    const int total = ntiles * nc;
+    // exponentials of one chunk of CN latents in buffer column base cb: the
+    // first 16 columns are exponentiated while the rest are read from TMEM
+    auto run_chunk = [&](auto cn_tag, uint32_t cb, float nu) {
+      constexpr int CN = decltype(cn_tag)::value;
+      uint32_t s0[16], pk[CN / 2];
+      tmem_ld16(cb, s0);
+      tmem_wait_ld();
+      if constexpr (CN > 16) {
+        uint32_t s1[CN - 16];
+        tmem_ld_cols<CN - 16>(cb + 16, s1);
+        exp2_row<16, FLARE_DEC_POLY_PAIRS>(s0, c, nu, *reinterpret_cast<uint32_t(*)[8]>(&pk[0]));
+        tmem_wait_ld();
+        exp2_row<CN - 16, FLARE_DEC_POLY_PAIRS>(s1, c, nu, *reinterpret_cast<uint32_t(*)[(CN - 16) / 2]>(&pk[8]));
+      } else {
+        exp2_row<16, FLARE_DEC_POLY_PAIRS>(s0, c, nu, pk);
+      }
+      tmem_st_cols<CN / 2>(cb, pk);  // P over the first CN/2 columns of the chunk's scores
+      tmem_wait_st();
+    };
     bool ok = true;
     float nu = 0.f;
-    for (int qq = 0; qq < total; ++qq) {
-      const int tile = qq / nc, cc = qq - tile * nc;
-      if (!mbar_wait_warp(s_full, qq & 1, wc)) { ok = false; break; }
+    for (int q = 0, tile = 0, cc = 0; q < total; ++q) {
+      const int buf = q & 1;
+      if (!mbar_wait_warp(s_full + buf, (q >> 1) & 1, wc)) { ok = false; break; }
       tc_fence_after();
-      const int cn = min(kDecChunk, p.M - cc * kDecChunk);
-      uint32_t sa[32], sb[32], pk[32];
-      tmem_ld32(lane_base + Cfg::COL_S, sa);
-      if (cn > 32) tmem_ld32(lane_base + Cfg::COL_S + 32, sb);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive_warp(s_free);  // the tensor pipe may now write S(q+1)
       if (cc == 0) {
         // |k_n| from the key tile in shared memory (the swizzle only permutes
-        // 16-byte halves inside each row, which a sum of squares ignores);
-        // the tile stays resident until the tile's last value MMA completes
+        // 16-byte pieces inside each row, which a sum of squares ignores); the
+        // tile's stage is refilled only after every warp is past this point
+        if (!mbar_wait_warp(k_full + tile % NST, (tile / NST) & 1, wc)) { ok = false; break; }
         const uint4* krow_s = reinterpret_cast<const uint4*>(sk + (tile % NST) * Cfg::KT_B + r * Cfg::ROWB);
         nu = c * sqrtf(bf16_row_norm2(krow_s, D / 8)) * qm;
       }
-      if (cn == kDecChunk) {
-        exp2_chunk64<FLARE_DEC_POLY_PAIRS>(sa, sb, c, nu, pk);
-      } else if (cn > 32) {  // 48 latents
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-          pk[k] = pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sa[2 * k]), c, -nu)),
-                              ex2_mufu(fmaf(__uint_as_float(sa[2 * k + 1]), c, -nu)));
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          pk[16 + k] = pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sb[2 * k]), c, -nu)),
-                                   ex2_mufu(fmaf(__uint_as_float(sb[2 * k + 1]), c, -nu)));
-#pragma unroll
-        for (int k = 8; k < 16; ++k) pk[16 + k] = 0u;
-      } else {
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          pk[k] = (2 * k < cn) ? pack_bf16x2(ex2_mufu(fmaf(__uint_as_float(sa[2 * k]), c, -nu)),
-                                             ex2_mufu(fmaf(__uint_as_float(sa[2 * k + 1]), c, -nu)))
-                               : 0u;
-          pk[16 + k] = 0u;
-        }
-      }
-      // P was last read by the value MMA of chunk q-1
-      if (qq >= 1 && !mbar_wait_warp(p_free, (qq - 1) & 1, wc)) { ok = false; break; }
-      tc_fence_after();
-      tmem_st32(lane_base + Cfg::COL_P, pk);
-      tmem_wait_st();
+      const int cn = min(C, p.M - cc * C);
+      const uint32_t cb = lane_base + buf * C;
+      if (cn == C) run_chunk(std::integral_constant<int, C>{}, cb, nu);
+      else if (cn == 48) run_chunk(std::integral_constant<int, 48>{}, cb, nu);
+      else if (cn == 32) run_chunk(std::integral_constant<int, 32>{}, cb, nu);
+      else run_chunk(std::integral_constant<int, 16>{}, cb, nu);
       tc_fence_before();
-      mbar_arrive_warp(p_full);
+      mbar_arrive_warp(p_full + buf);
+      if (cc == 0 && tile >= 2 && tile - 2 + NST < ntiles && wq == (tile & 3) && lane == 0)
+        load_tile(tile - 2 + NST);  // every MMA and norm read of tile - 2 is done
+      __syncwarp();
       if (cc == 0 && tile >= 1 && !epilogue(tile - 1)) { ok = false; break; }
+      if (++cc == nc) {
+        cc = 0;
+        ++tile;
+      }
     }
-    if (ok && ntiles > 0) epilogue(ntiles - 1);
+    if (ok) epilogue(ntiles - 1);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
+    if (lane == 0) {  // copies still in flight (only after an abort) must land before exit
+      for (int st = 0; st < NST; ++st)
+        if (last_load[st] >= 0) mbar_wait_drain(k_full + st, (last_load[st] / NST) & 1, p.timeout_ns);
+      mbar_wait_drain(qz_full, 0, p.timeout_ns);
+    }
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::TMEM_COLS);
   }
@@ -412,8 +436,9 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
 
 size_t decode_smem_bytes(int D, int /*M*/) {
   const size_t need = (D == 16 ? DecCfg<16>::BYTES : DecCfg<32>::BYTES) + 1024;
-  // at most dec_ctas_per_sm(D) CTAs per SM (TMEM columns)
-  const size_t floor = dec_ctas_per_sm(D) >= 3 ? 70 * 1024 : 100 * 1024;
+  // at most dec_ctas_per_sm(D) CTAs per SM (228 KB each, 1 KB of it
+  // reserved per CTA), so that every resident CTA finds its TMEM columns free
+  const size_t floor = (228 * 1024) / (dec_ctas_per_sm(D) + 1) + 1024;
   return need > floor ? need : floor;
 }
 

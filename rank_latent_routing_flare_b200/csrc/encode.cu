@@ -3,10 +3,10 @@
 // eq. 5, which is also the query synthesis of eq. 8 and the encode of eq. 10).
 //
 // One CTA owns (b, h, a block of 128 latents, a contiguous range of token
-// tiles).  Per 64-token tile:
-//   S = Q_blk K_tile^T            UMMA M=128 (latents) x N=64 (tokens), fp32 in TMEM
-//   P = 2^(S * c - U_m)           softmax threads, one latent row per thread
-//   O += P [V_tile | 1]           UMMA with A = P read from TMEM; the ones block
+// tiles of T tokens, T = enc_tile(D)).  Per tile i:
+//   S_i = Q_blk K_i^T             UMMA M=128 (latents) x N=T (tokens), fp32 in TMEM
+//   P_i = 2^(S_i * c - U_m)       softmax threads, one latent row per thread
+//   O  += P_i [V_i | 1]           UMMA with A = P_i read from TMEM; the ones block
 //                                 makes column D of O the running row sum
 // The shift U_m = c * |q_m| * max_{n in split} |k_n| is an upper bound of the
 // row's scaled scores (Cauchy-Schwarz), fixed for the whole split, so no
@@ -14,13 +14,23 @@
 // (U_m, sum_m, O_m) and the merge kernel combines splits with the exact
 // log-sum-exp rule of section "Multi-GPU context parallelism" (eq. 14).
 //
-// Warp roles (5 warps): warp 0 lane 0 is the control thread: it keeps the
-// K/V ring full (TMA) and issues the MMAs in program order, blocking on
-// exactly the next event (S(i+1) once every softmax warp has loaded S(i);
-// P(i) [V(i) | 1] once every softmax warp has stored P(i)).  Warps 1..4 are
-// the softmax warps (thread <-> TMEM lane <-> latent row).  A CTA needs 128
-// TMEM columns for D = 16: three CTAs (three softmax warps per SM
-// sub-partition) share an SM.
+// TMEM holds two score buffers; tile i uses buffer i % 2, and the softmax
+// threads write P_i (bf16 pairs) over the first T/2 columns of S_i once they
+// hold S_i in registers.  S_{i+2} reuses the buffer after the value MMA of
+// tile i has completed.  The MMA thread therefore computes S_{i+1} while the
+// softmax threads work on S_i, and the softmax threads wait on a single
+// barrier per tile (S_i ready); their only other barrier operation is the
+// arrive that hands P_i to the MMA thread.  Every barrier that is reused
+// across tiles exists once per buffer, so no party can run a full phase
+// ahead of the party that waits on it.
+//
+// Warp roles (5 warps): warp 0 lane 0 is the MMA thread, issuing in program
+// order S_0, S_1, P_0 V_0, S_2, P_1 V_1, S_3, ...  Warps 1..4 are the softmax
+// warps (thread <-> TMEM lane <-> latent row).  They also refill the K/V
+// ring: S_i was issued after P_{i-2} V_{i-2}, so once S_i is complete the
+// ring stage of tile i-2 is free, and one softmax warp, in rotation, loads
+// tile i-2+NST into it.  A CTA needs 128 TMEM columns for D = 16: three CTAs
+// (three softmax warps per SM sub-partition) share an SM.
 #include "ptx.cuh"
 
 namespace flare {
@@ -28,7 +38,7 @@ namespace {
 
 template <int D>
 struct EncCfg {
-  static constexpr int T = kEncTile;                   // tokens per tile (64)
+  static constexpr int T = enc_tile(D);                // tokens per tile
   static constexpr int ROWB = D * 2;                   // bytes of one K/V/Q row
   static constexpr int TILE_B = T * ROWB;              // bytes of one K or V tile
   static constexpr int Q_B = kLatBlock * ROWB;
@@ -36,18 +46,21 @@ struct EncCfg {
   static constexpr uint32_t LAYOUT = (D == 16) ? LAYOUT_SW32 : LAYOUT_SW64;
   static constexpr uint32_t SBO = 8 * ROWB;            // stride of 8-row core-matrix groups
   static constexpr int NO = D + 16;                    // O columns: D values + 16 copies of the sum
-  // TMEM columns: S at 0 (fp32 scores), P at T (bf16 pairs), O at 3T/2
-  static constexpr uint32_t COL_S = 0, COL_P = T, COL_O = T + T / 2;
+  // TMEM columns: score buffers at 0 and T (each later holds its P), O at 2T
+  static constexpr uint32_t COL_O = 2 * T;
   static constexpr uint32_t TMEM_COLS = (COL_O + NO <= 128) ? 128 : 256;
+  // Each V stage is followed by its own block of ones, so that [V | 1] has
+  // the same leading byte offset (TILE_B) in every stage.
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_B;
-  static constexpr int OFF_V = OFF_K + NST * TILE_B;
-  static constexpr int OFF_ONES = OFF_V + NST * TILE_B;
-  static constexpr int OFF_BAR = OFF_ONES + TILE_B;
+  static constexpr int OFF_V = OFF_K + NST * TILE_B;   // NST x [V tile | ones]
+  static constexpr int OFF_BAR = OFF_V + NST * 2 * TILE_B;
   static constexpr int OFF_MISC = OFF_BAR + 8 * 32;
-  static constexpr int BYTES = OFF_MISC + 64;
+  static constexpr int BYTES = OFF_MISC + 64 + NST * 4;
   static constexpr int THREADS = 160;
   static constexpr int CTAS_PER_SM = enc_ctas_per_sm(D);
+  static_assert(TMEM_COLS <= 512 / CTAS_PER_SM, "TMEM columns of the co-resident CTAs exceed 512");
+  static_assert(T % 16 == 0 && TILE_B % 256 == 0, "tile must hold whole swizzle atoms");
 };
 
 template <int D>
@@ -61,19 +74,17 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
   uint8_t* sq = sm + Cfg::OFF_Q;
   uint8_t* sk = sm + Cfg::OFF_K;
   uint8_t* sv = sm + Cfg::OFF_V;
-  uint8_t* sones = sm + Cfg::OFF_ONES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Cfg::OFF_BAR);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = bars + 1 + NST;
-  uint64_t* s_full = bars + 1 + 2 * NST;  // S computed
-  uint64_t* s_free = s_full + 1;           // S loaded by every softmax warp (one arrive per warp)
-  uint64_t* p_full = s_full + 2;           // P stored by every softmax warp (one arrive per warp)
-  uint64_t* p_free = s_full + 3;           // P consumed by the value MMA
-  uint64_t* o_full = s_full + 4;           // every MMA of the CTA done
+  uint64_t* kv_full = bars + 1;            // [NST] K/V tile landed
+  uint64_t* s_full = bars + 1 + NST;       // [2] score buffer computed
+  uint64_t* pv_done = s_full + 2;          // [2] value MMA done reading the buffer's P
+  uint64_t* p_full = s_full + 4;           // [2] P stored by every softmax warp (one arrive per warp)
+  uint64_t* o_full = s_full + 6;           // every MMA of the CTA done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(sm + Cfg::OFF_MISC + 4);
   float* red = reinterpret_cast<float*>(sm + Cfg::OFF_MISC + 16);
+  volatile int* last_load = reinterpret_cast<volatile int*>(sm + Cfg::OFF_MISC + 64);  // per stage
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int LB = p.n_lblocks, S = p.n_splits;
@@ -115,18 +126,21 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
     mbar_init(q_full, 1);
     for (int i = 0; i < NST; ++i) {
       mbar_init(kv_full + i, 1);
-      mbar_init(kv_empty + i, 1);
+      last_load[i] = -1;
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 4);
-    mbar_init(p_full, 4);
-    mbar_init(p_free, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full + i, 1);
+      mbar_init(pv_done + i, 1);
+      mbar_init(p_full + i, 4);
+    }
     mbar_init(o_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  for (int i = threadIdx.x; i < Cfg::TILE_B / 4; i += blockDim.x)
-    reinterpret_cast<uint32_t*>(sones)[i] = 0x3F803F80u;  // bf16 1.0 pairs
+  for (int i = threadIdx.x; i < NST * Cfg::TILE_B / 4; i += blockDim.x) {
+    const int st = i / (Cfg::TILE_B / 4), w = i % (Cfg::TILE_B / 4);
+    reinterpret_cast<uint32_t*>(sv + (2 * st + 1) * Cfg::TILE_B)[w] = 0x3F803F80u;  // bf16 1.0 pairs
+  }
   fence_proxy_async_smem();
   if (warp == 0) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
@@ -137,74 +151,65 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{p.err, abort_flag, p.timeout_ns};
+  // K and V of tile n into ring stage n % NST (one thread)
+  auto load_tile = [&](int n) {
+    const int st = n % NST;
+    mbar_arrive_expect_tx(kv_full + st, 2 * Cfg::TILE_B);
+    const int tok = (t0 + n) * T;
+    tma_load_3d(sk + st * Cfg::TILE_B, &tm_k, kv_full + st, 0, tok, bh);
+    tma_load_3d(sv + st * 2 * Cfg::TILE_B, &tm_v, kv_full + st, 0, tok, bh);
+    last_load[st] = n;
+  };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ control thread
+    // ------------------------------------------------------------ MMA thread
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       mbar_arrive_expect_tx(q_full, p.q_rows * Cfg::ROWB);
       tma_load_3d(sq, &tm_q, q_full, 0, lb * kLatBlock, g);
+      for (int n = 0; n < min(NST, ntiles); ++n) load_tile(n);
       const uint32_t idesc_s = idesc_bf16_f32(128, T, false, false);
       const uint32_t idesc_pv = idesc_bf16_f32(128, Cfg::NO, false, true);
-      const uint32_t sq_a = smem_u32(sq), ones_a = smem_u32(sones);
-      int n_load = 0;
-      auto load = [&]() {
-        const int st = n_load % NST;
-        mbar_arrive_expect_tx(kv_full + st, 2 * Cfg::TILE_B);
-        const int tok = (t0 + n_load) * T;
-        tma_load_3d(sk + st * Cfg::TILE_B, &tm_k, kv_full + st, 0, tok, bh);
-        tma_load_3d(sv + st * Cfg::TILE_B, &tm_v, kv_full + st, 0, tok, bh);
-        ++n_load;
-      };
-      // refill every ring stage whose previous tile's value MMA has completed
-      auto refill = [&]() {
-        while (n_load < ntiles && mbar_test(kv_empty + n_load % NST, ((n_load / NST) & 1) ^ 1)) load();
-      };
+      // descriptors of stage 0; a stage's descriptor adds its byte offset >> 4
+      const uint64_t q_desc = umma_desc(smem_u32(sq), 16, Cfg::SBO, Cfg::LAYOUT);
+      const uint64_t k_desc = umma_desc(smem_u32(sk), 16, Cfg::SBO, Cfg::LAYOUT);
+      const uint64_t v_desc = umma_desc(smem_u32(sv), Cfg::TILE_B, Cfg::SBO, Cfg::LAYOUT);
+      // S_i into buffer i % 2, once tile i has landed and P_{i-2} has been consumed
       auto issue_s = [&](int i) -> bool {
-        while (n_load <= i) {  // tile i not requested yet: wait for its stage
-          if (!mbar_wait(kv_empty + n_load % NST, ((n_load / NST) & 1) ^ 1, wc)) return false;
-          load();
-        }
-        if (!mbar_wait(kv_full + i % NST, (i / NST) & 1, wc)) return false;
+        const int st = i % NST, buf = i & 1;
+        if (!mbar_wait(kv_full + st, (i / NST) & 1, wc)) return false;
+        if (i >= 2 && !mbar_wait(pv_done + buf, ((i - 2) >> 1) & 1, wc)) return false;
         tc_fence_after();
-        const uint32_t k_a = smem_u32(sk + (i % NST) * Cfg::TILE_B);
+        const uint64_t kd = k_desc + static_cast<uint64_t>((st * Cfg::TILE_B) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          umma_ss(tmem + Cfg::COL_S, umma_desc(sq_a + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT),
-                  umma_desc(k_a + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT), idesc_s, kk > 0 ? 1u : 0u);
-        umma_commit(s_full);
+          umma_ss(tmem + buf * T, q_desc + 2 * kk, kd + 2 * kk, idesc_s, kk > 0 ? 1u : 0u);
+        umma_commit(s_full + buf);
         return true;
       };
+      // O += P_i [V_i | 1] once every softmax warp has stored P_i
       auto issue_pv = [&](int i) -> bool {
-        if (!mbar_wait(p_full, i & 1, wc)) return false;
+        const int buf = i & 1;
+        if (!mbar_wait(p_full + buf, (i >> 1) & 1, wc)) return false;
         tc_fence_after();
-        const int st = i % NST;
-        const uint32_t v_a = smem_u32(sv + st * Cfg::TILE_B);
-        const uint32_t lbo = ones_a - v_a;  // [V | 1] : second N-atom = ones block
+        const uint64_t vd = v_desc + static_cast<uint64_t>(((i % NST) * 2 * Cfg::TILE_B) >> 4);
 #pragma unroll
-        for (int ks = 0; ks < T / 16; ++ks) {
-          const uint64_t bdesc = umma_desc(v_a + ks * 16 * Cfg::ROWB, lbo, Cfg::SBO, Cfg::LAYOUT);
-          umma_ts(tmem + Cfg::COL_O, tmem + Cfg::COL_P + ks * 8, bdesc, idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
-        }
-        umma_commit(p_free);
-        umma_commit(kv_empty + st);
+        for (int ks = 0; ks < T / 16; ++ks)
+          umma_ts(tmem + Cfg::COL_O, tmem + buf * T + ks * 8, vd + static_cast<uint64_t>((ks * 16 * Cfg::ROWB) >> 4),
+                  idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(pv_done + buf);
         return true;
       };
-      refill();
       bool ok = mbar_wait(q_full, 0, wc) && issue_s(0);
-      for (int i = 1; ok && i < ntiles; ++i) {
-        ok = mbar_wait(s_free, (i - 1) & 1, wc) && issue_s(i);  // S(i-1) loaded -> S(i)
-        if (ok) ok = issue_pv(i - 1);                             // P(i-1) stored -> P(i-1) V(i-1)
-        if (ok) refill();
+      if (ok && ntiles > 1) ok = issue_s(1);
+      for (int i = 0; ok && i < ntiles; ++i) {
+        ok = issue_pv(i);
+        if (ok && i + 2 < ntiles) ok = issue_s(i + 2);
       }
-      if (ok) issue_pv(ntiles - 1);
       umma_commit(o_full);  // completes once every MMA issued above is done
       mbar_wait_drain(o_full, 0, p.timeout_ns);
-      for (int i = max(0, n_load - NST); i < n_load; ++i)  // copies in flight must land
-        mbar_wait_drain(kv_full + (i % NST), (i / NST) & 1, p.timeout_ns);
-      mbar_wait_drain(q_full, 0, p.timeout_ns);
     }
   } else {
     // ------------------------------------------------------------ softmax
@@ -214,11 +219,13 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
     const bool row_ok = m < p.M;
     const bool warp_live = lb * kLatBlock + wq * 32 < p.M;
     const int tid = threadIdx.x - 32;
-    // bound of the key norms over this split
+    // bound of the key norms over this split (the 32-token groups that
+    // overlap its token range)
     float km = 0.f;
     const float* kn = p.knorm + static_cast<size_t>(bh) * p.n_groups32;
-    const int g_end = min(t1 * (T / kNormGroup), p.n_groups32);
-    for (int gi = t0 * (T / kNormGroup) + tid; gi < g_end; gi += 128) km = fmaxf(km, kn[gi]);
+    const int g_beg = (t0 * T) / kNormGroup;
+    const int g_end = min((t1 * T + kNormGroup - 1) / kNormGroup, p.n_groups32);
+    for (int gi = g_beg + tid; gi < g_end; gi += 128) km = fmaxf(km, kn[gi]);
     km = warp_max(km);
     if (lane == 0) red[wq] = km;
     named_bar_sync(1, 128);
@@ -243,42 +250,44 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
-      if (!mbar_wait_warp(s_full, i & 1, wc)) { ok = false; break; }
+      const int buf = i & 1;
+      if (!mbar_wait_warp(s_full + buf, (i >> 1) & 1, wc)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sa[32], sb[32], pk[32];
-      if (warp_live) {
-        tmem_ld32(lane_base + Cfg::COL_S, sa);
-        tmem_ld32(lane_base + Cfg::COL_S + 32, sb);
+      const int valid = L - (t0 + i) * T;
+      if (warp_live && FLARE_ENC_SPLIT_LD && valid >= T) {
+        // first 16 columns, then the rest while the first are exponentiated
+        constexpr int R = T - 16;
+        uint32_t s0[16], s1[R], pk[T / 2];
+        tmem_ld16(lane_base + buf * T, s0);
         tmem_wait_ld();
-      }
-      tc_fence_before();
-      mbar_arrive_warp(s_free);  // the tensor pipe may now write S(i+1)
-      if (warp_live) {
-        const int valid = L - (t0 + i) * T;
+        tmem_ld_cols<R>(lane_base + buf * T + 16, s1);
+        exp2_row<16, FLARE_ENC_POLY_PAIRS>(s0, c, U, *reinterpret_cast<uint32_t(*)[8]>(&pk[0]));
+        tmem_wait_ld();
+        exp2_row<R, FLARE_ENC_POLY_PAIRS>(s1, c, U, *reinterpret_cast<uint32_t(*)[R / 2]>(&pk[8]));
+        tmem_st_cols<T / 2>(lane_base + buf * T, pk);  // P_i over the first T/2 columns of S_i
+        tmem_wait_st();
+      } else if (warp_live) {
+        uint32_t sc[T], pk[T / 2];
+        tmem_ld_cols<T>(lane_base + buf * T, sc);
+        tmem_wait_ld();
         if (valid >= T) {
-          exp2_chunk64<FLARE_ENC_POLY_PAIRS>(sa, sb, c, U, pk);
+          exp2_row<T, FLARE_ENC_POLY_PAIRS>(sc, c, U, pk);
         } else {  // last, partial tile of the valid range: padded tokens get weight 0
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const float e0 = (2 * k < valid) ? ex2_mufu(fmaf(__uint_as_float(sa[2 * k]), c, -U)) : 0.f;
-            const float e1 = (2 * k + 1 < valid) ? ex2_mufu(fmaf(__uint_as_float(sa[2 * k + 1]), c, -U)) : 0.f;
-            const float e2 = (32 + 2 * k < valid) ? ex2_mufu(fmaf(__uint_as_float(sb[2 * k]), c, -U)) : 0.f;
-            const float e3 =
-                (33 + 2 * k < valid) ? ex2_mufu(fmaf(__uint_as_float(sb[2 * k + 1]), c, -U)) : 0.f;
+          for (int k = 0; k < T / 2; ++k) {
+            const float e0 = (2 * k < valid) ? ex2_mufu(fmaf(__uint_as_float(sc[2 * k]), c, -U)) : 0.f;
+            const float e1 = (2 * k + 1 < valid) ? ex2_mufu(fmaf(__uint_as_float(sc[2 * k + 1]), c, -U)) : 0.f;
             pk[k] = pack_bf16x2(e0, e1);
-            pk[16 + k] = pack_bf16x2(e2, e3);
           }
         }
-      }
-      // P was last read by the value MMA of tile i-1
-      if (i >= 1 && !mbar_wait_warp(p_free, (i - 1) & 1, wc)) { ok = false; break; }
-      tc_fence_after();
-      if (warp_live) {
-        tmem_st32(lane_base + Cfg::COL_P, pk);
+        tmem_st_cols<T / 2>(lane_base + buf * T, pk);  // P_i over the first T/2 columns of S_i
         tmem_wait_st();
       }
       tc_fence_before();
-      mbar_arrive_warp(p_full);
+      mbar_arrive_warp(p_full + buf);
+      // S_i complete implies P_{i-2} V_{i-2} complete: its ring stage is free
+      if (i >= 2 && i - 2 + NST < ntiles && wq == (i & 3) && lane == 0) load_tile(i - 2 + NST);
+      __syncwarp();
     }
     if (ok && mbar_wait_warp(o_full, 0, wc)) {
       tc_fence_after();
@@ -308,6 +317,11 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
+    if (lane == 0) {  // copies still in flight (only after an abort) must land before exit
+      for (int st = 0; st < NST; ++st)
+        if (last_load[st] >= 0) mbar_wait_drain(kv_full + st, (last_load[st] / NST) & 1, p.timeout_ns);
+      mbar_wait_drain(q_full, 0, p.timeout_ns);
+    }
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::TMEM_COLS);
   }
@@ -318,8 +332,9 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
 size_t encode_smem_bytes(int D) {
   const size_t need = (D == 16 ? EncCfg<16>::BYTES : EncCfg<32>::BYTES) + 1024;
   // Reserve enough shared memory that at most enc_ctas_per_sm(D) CTAs share
-  // an SM, so that every resident CTA finds its TMEM columns free.
-  const size_t floor = enc_ctas_per_sm(D) >= 3 ? 70 * 1024 : 100 * 1024;
+  // an SM (228 KB each, 1 KB of it reserved per CTA), so that every resident
+  // CTA finds its TMEM columns free.
+  const size_t floor = (228 * 1024) / (enc_ctas_per_sm(D) + 1) + 1024;
   return need > floor ? need : floor;
 }
 

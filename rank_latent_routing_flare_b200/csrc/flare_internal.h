@@ -12,30 +12,44 @@
 namespace flare {
 
 constexpr int kNumSM = 148;        // B200
-constexpr int kEncTile = 64;       // tokens per encode tile
 constexpr int kLatBlock = 128;     // latents per encode CTA (UMMA M)
 constexpr int kDecTile = 128;      // tokens per decode tile (UMMA M)
-constexpr int kDecChunk = 64;      // latents per decode chunk (UMMA N)
 constexpr int kNormGroup = 32;     // tokens per key-norm group
 constexpr int kProjTile = 128;     // tokens per projection tile
 
+// Tokens per encoder tile.  The encoder keeps two score tiles and the
+// output accumulator in TMEM: 2 * 48 + 32 = 128 columns for D = 16, and
+// 2 * 64 + 48 (within 256) for D = 32.
+__host__ __device__ constexpr int enc_tile(int D) { return D == 16 ? 48 : 64; }
 // Co-resident CTAs per SM of the encoder: 128 TMEM columns per CTA for
-// D = 16 (three CTAs), 256 for D = 32 (two).
-__host__ __device__ constexpr int enc_ctas_per_sm(int D) { return D == 16 ? 3 : 2; }
-// Same for the decoder.
+// D = 16 (up to four CTAs), 256 for D = 32 (two).
+#ifndef FLARE_ENC_CTAS_D16
+#define FLARE_ENC_CTAS_D16 4
+#endif
+__host__ __device__ constexpr int enc_ctas_per_sm(int D) { return D == 16 ? FLARE_ENC_CTAS_D16 : 2; }
+// Latents per decoder chunk.  The decoder keeps two score chunks and the
+// output accumulator in TMEM: 2 * 48 + 32 = 128 columns for D = 16, and
+// 2 * 64 + 48 (within 256) for D = 32.
+__host__ __device__ constexpr int dec_chunk(int D) { return D == 16 ? 48 : 64; }
+// Co-resident CTAs per SM of the decoder (TMEM columns as for the encoder).
 #ifndef FLARE_DEC_CTAS_D16
-#define FLARE_DEC_CTAS_D16 3
+#define FLARE_DEC_CTAS_D16 4
 #endif
 __host__ __device__ constexpr int dec_ctas_per_sm(int D) { return D == 16 ? FLARE_DEC_CTAS_D16 : 2; }
 
-// Of the 32 score pairs of each 64-column softmax chunk, how many are
-// exponentiated on the FMA pipe (polynomial) instead of the MUFU; chosen by
-// measurement on B200 (the encoder gains ~2% with 4, the decoder loses).
+// Of every 32 score pairs of a softmax row, how many are exponentiated on
+// the FMA pipe (polynomial) instead of the MUFU; chosen by measurement on
+// B200 (the encoder gains with 4, the decoder loses).
 #ifndef FLARE_ENC_POLY_PAIRS
 #define FLARE_ENC_POLY_PAIRS 4
 #endif
+// Encoder softmax: load the first 16 score columns, start their
+// exponentials while the rest of the tile is read from TMEM.
+#ifndef FLARE_ENC_SPLIT_LD
+#define FLARE_ENC_SPLIT_LD 1
+#endif
 #ifndef FLARE_DEC_POLY_PAIRS
-#define FLARE_DEC_POLY_PAIRS 0
+#define FLARE_DEC_POLY_PAIRS 6
 #endif
 
 // ---------------------------------------------------------------------------
@@ -69,7 +83,7 @@ struct EncodeParams {
   int B, H, N, M, D;
   int q_per_batch;      // queries [B*H][M][D] (1) or [H][M][D] (0)
   int n_splits;         // S
-  int tiles_per_split;  // in kEncTile tiles
+  int tiles_per_split;  // in tiles of enc_tile(D) tokens
   int n_lblocks;        // ceil(M / kLatBlock)
   int n_groups32;
   int q_rows;           // rows of one query box: min(M, kLatBlock)
@@ -107,7 +121,7 @@ struct DecodeParams {
   int q_per_batch;
   int tiles_per_cta;    // in kDecTile tiles
   int ctas_per_head;
-  int chunk_rows;       // rows of one Q/Z box: min(M, kDecChunk)
+  int qz_box_rows;      // rows of one Q/Z box: min(M, 256)
   float scale, c;
   const int32_t* lengths;
   const uint16_t* q;    // bf16 [G][M][D]

@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
   const int b = bh / p.H, h = bh % p.H;
   int L = p.N;
   if (p.lengths) L = min(max(p.lengths[b], 0), p.N);
-  const int ntv = (L + kEncTile - 1) / kEncTile;
+  const int ntv = (L + enc_tile(D) - 1) / enc_tile(D);
   const int S = p.n_splits;
   const size_t stride = static_cast<size_t>(p.M) * (D + 2);
   const float* base = p.part + static_cast<size_t>(bh) * S * stride + static_cast<size_t>(m) * (D + 2);
@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
     if (t1 <= t0) continue;
     const float U = base[s * stride], l = base[s * stride + 1];
     if (l > 0.f) G = fmaxf(G, U + log2f(l));
-    lost = fmaxf(lost, U - 126.f + log2f(static_cast<float>((t1 - t0) * kEncTile)));
+    lost = fmaxf(lost, U - 126.f + log2f(static_cast<float>((t1 - t0) * enc_tile(D))));
   }
   const bool exact = !(G > -INFINITY) || (lost + log2f(static_cast<float>(S)) - G > -27.f);
   float z = 0.f;

@@ -260,6 +260,35 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+// N consecutive columns (N a multiple of 16; st: a multiple of 8) as 32/16/8-column pieces.
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
+  static_assert(N % 16 == 0, "tmem_ld_cols: N must be a multiple of 16");
+  if constexpr (N >= 32) {
+    tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    if constexpr (N > 32) tmem_ld_cols<N - 32>(taddr + 32, *reinterpret_cast<uint32_t(*)[N - 32]>(&r[32]));
+  } else {
+    tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+  }
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[N]) {
+  static_assert(N % 8 == 0, "tmem_st_cols: N must be a multiple of 8");
+  if constexpr (N >= 32) {
+    tmem_st32(taddr, *reinterpret_cast<const uint32_t(*)[32]>(&r[0]));
+    if constexpr (N > 32) tmem_st_cols<N - 32>(taddr + 32, *reinterpret_cast<const uint32_t(*)[N - 32]>(&r[32]));
+  } else if constexpr (N >= 16) {
+    tmem_st16(taddr, *reinterpret_cast<const uint32_t(*)[16]>(&r[0]));
+    if constexpr (N > 16) tmem_st_cols<N - 16>(taddr + 16, *reinterpret_cast<const uint32_t(*)[N - 16]>(&r[16]));
+  } else {
+    tmem_st8(taddr, *reinterpret_cast<const uint32_t(*)[8]>(&r[0]));
+  }
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -303,6 +332,28 @@ __device__ __forceinline__ void exp2_chunk64(const uint32_t (&a)[32], const uint
     const float x0 = fmaf(__uint_as_float(src[2 * k]), c, -shift);
     const float x1 = fmaf(__uint_as_float(src[2 * k + 1]), c, -shift);
     const bool poly = ((q * NPOLY) % 32) < NPOLY;
+    float e0, e1;
+    if (poly) {
+      e0 = ex2_poly(x0);
+      e1 = ex2_poly(x1);
+    } else {
+      e0 = ex2_mufu(x0);
+      e1 = ex2_mufu(x1);
+    }
+    pk[q] = pack_bf16x2(e0, e1);
+  }
+}
+
+// Exponentials of one row of NV scores (raw fp32 bits in s[0..NV)): e =
+// 2^(s * c - shift), packed to bf16 pairs pk[0..NV/2).  NPOLY of every 32
+// pairs use ex2_poly (FMA pipe), spread evenly; the rest use the MUFU.
+template <int NV, int NPOLY>
+__device__ __forceinline__ void exp2_row(const uint32_t (&s)[NV], float c, float shift, uint32_t (&pk)[NV / 2]) {
+#pragma unroll
+  for (int q = 0; q < NV / 2; ++q) {
+    const float x0 = fmaf(__uint_as_float(s[2 * q]), c, -shift);
+    const float x1 = fmaf(__uint_as_float(s[2 * q + 1]), c, -shift);
+    const bool poly = (((q % 32) * NPOLY) % 32) < NPOLY;
     float e0, e1;
     if (poly) {
       e0 = ex2_poly(x0);
