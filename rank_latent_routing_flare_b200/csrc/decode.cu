@@ -283,9 +283,11 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
         const uint64_t step = static_cast<uint64_t>(x.cc) * CH_STEP;
         const uint64_t zd = z_desc + step - (step << 16);
         const int nks = (x.cc == nc - 1 ? last_n : C) / 16;
-        for (int ks = 0; ks < nks; ++ks)
-          umma_ts(tmem + Cfg::COL_Y, tmem + buf * C + ks * 8, zd + static_cast<uint64_t>((ks * 16 * Cfg::ROWB) >> 4),
-                  idesc_y, (x.cc > 0 || ks > 0) ? 1u : 0u);
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks)
+          if (ks < nks)
+            umma_ts(tmem + Cfg::COL_Y, tmem + buf * C + ks * 8,
+                    zd + static_cast<uint64_t>((ks * 16 * Cfg::ROWB) >> 4), idesc_y, (x.cc > 0 || ks > 0) ? 1u : 0u);
         umma_commit(pv_done + buf);
         if (x.cc == nc - 1) umma_commit(y_full);
         return true;

@@ -31,6 +31,8 @@
 // ring stage of tile i-2 is free, and one softmax warp, in rotation, loads
 // tile i-2+NST into it.  A CTA needs 128 TMEM columns for D = 16: three CTAs
 // (three softmax warps per SM sub-partition) share an SM.
+#include <type_traits>
+
 #include "ptx.cuh"
 
 namespace flare {
@@ -248,47 +250,52 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
     const float c = p.c;
     const float U = c * qn * km;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    bool ok = true;
-    for (int i = 0; i < ntiles; ++i) {
-      const int buf = i & 1;
-      if (!mbar_wait_warp(s_full + buf, (i >> 1) & 1, wc)) { ok = false; break; }
-      tc_fence_after();
-      const int valid = L - (t0 + i) * T;
-      if (warp_live && FLARE_ENC_SPLIT_LD && valid >= T) {
-        // first 16 columns, then the rest while the first are exponentiated
-        constexpr int R = T - 16;
-        uint32_t s0[16], s1[R], pk[T / 2];
-        tmem_ld16(lane_base + buf * T, s0);
-        tmem_wait_ld();
-        tmem_ld_cols<R>(lane_base + buf * T + 16, s1);
-        exp2_row<16, FLARE_ENC_POLY_PAIRS>(s0, c, U, *reinterpret_cast<uint32_t(*)[8]>(&pk[0]));
-        tmem_wait_ld();
-        exp2_row<R, FLARE_ENC_POLY_PAIRS>(s1, c, U, *reinterpret_cast<uint32_t(*)[R / 2]>(&pk[8]));
-        tmem_st_cols<T / 2>(lane_base + buf * T, pk);  // P_i over the first T/2 columns of S_i
-        tmem_wait_st();
-      } else if (warp_live) {
-        uint32_t sc[T], pk[T / 2];
-        tmem_ld_cols<T>(lane_base + buf * T, sc);
-        tmem_wait_ld();
-        if (valid >= T) {
-          exp2_row<T, FLARE_ENC_POLY_PAIRS>(sc, c, U, pk);
-        } else {  // last, partial tile of the valid range: padded tokens get weight 0
+    // the tile loop, with NP polynomial exp2 pairs out of every 32
+    auto run_tiles = [&](auto np_tag) -> bool {
+      constexpr int NP = decltype(np_tag)::value;
+      for (int i = 0; i < ntiles; ++i) {
+        const int buf = i & 1;
+        if (!mbar_wait_warp(s_full + buf, (i >> 1) & 1, wc)) return false;
+        tc_fence_after();
+        const int valid = L - (t0 + i) * T;
+        if (warp_live && FLARE_ENC_SPLIT_LD && valid >= T) {
+          // first 16 columns, then the rest while the first are exponentiated
+          constexpr int R = T - 16;
+          uint32_t s0[16], s1[R], pk[T / 2];
+          tmem_ld16(lane_base + buf * T, s0);
+          tmem_wait_ld();
+          tmem_ld_cols<R>(lane_base + buf * T + 16, s1);
+          exp2_row<16, NP>(s0, c, U, *reinterpret_cast<uint32_t(*)[8]>(&pk[0]));
+          tmem_wait_ld();
+          exp2_row<R, NP>(s1, c, U, *reinterpret_cast<uint32_t(*)[R / 2]>(&pk[8]));
+          tmem_st_cols<T / 2>(lane_base + buf * T, pk);  // P_i over the first T/2 columns of S_i
+          tmem_wait_st();
+        } else if (warp_live) {
+          uint32_t sc[T], pk[T / 2];
+          tmem_ld_cols<T>(lane_base + buf * T, sc);
+          tmem_wait_ld();
+          if (valid >= T) {
+            exp2_row<T, NP>(sc, c, U, pk);
+          } else {  // last, partial tile of the valid range: padded tokens get weight 0
 #pragma unroll
-          for (int k = 0; k < T / 2; ++k) {
-            const float e0 = (2 * k < valid) ? ex2_mufu(fmaf(__uint_as_float(sc[2 * k]), c, -U)) : 0.f;
-            const float e1 = (2 * k + 1 < valid) ? ex2_mufu(fmaf(__uint_as_float(sc[2 * k + 1]), c, -U)) : 0.f;
-            pk[k] = pack_bf16x2(e0, e1);
+            for (int k = 0; k < T / 2; ++k) {
+              const float e0 = (2 * k < valid) ? ex2_mufu(fmaf(__uint_as_float(sc[2 * k]), c, -U)) : 0.f;
+              const float e1 = (2 * k + 1 < valid) ? ex2_mufu(fmaf(__uint_as_float(sc[2 * k + 1]), c, -U)) : 0.f;
+              pk[k] = pack_bf16x2(e0, e1);
+            }
           }
+          tmem_st_cols<T / 2>(lane_base + buf * T, pk);  // P_i over the first T/2 columns of S_i
+          tmem_wait_st();
         }
-        tmem_st_cols<T / 2>(lane_base + buf * T, pk);  // P_i over the first T/2 columns of S_i
-        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive_warp(p_full + buf);
+        // S_i complete implies P_{i-2} V_{i-2} complete: its ring stage is free
+        if (i >= 2 && i - 2 + NST < ntiles && wq == (i & 3) && lane == 0) load_tile(i - 2 + NST);
+        __syncwarp();
       }
-      tc_fence_before();
-      mbar_arrive_warp(p_full + buf);
-      // S_i complete implies P_{i-2} V_{i-2} complete: its ring stage is free
-      if (i >= 2 && i - 2 + NST < ntiles && wq == (i & 3) && lane == 0) load_tile(i - 2 + NST);
-      __syncwarp();
-    }
+      return true;
+    };
+    const bool ok = run_tiles(std::integral_constant<int, FLARE_ENC_POLY_PAIRS>{});
     if (ok && mbar_wait_warp(o_full, 0, wc)) {
       tc_fence_after();
       if (warp_live) {

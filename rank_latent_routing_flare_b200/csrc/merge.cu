@@ -69,30 +69,48 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
   const float* base = p.part + static_cast<size_t>(bh) * S * stride + static_cast<size_t>(m) * (D + 2);
 
   // log2 of the total weight: G = max_s (U_s + log2 l_s); bound of the mass
-  // lost to flushed exponentials: sum_s n_s 2^(U_s - 126)
+  // lost to flushed exponentials: sum_s n_s 2^(U_s - 126).  Lanes take the
+  // splits s = lane, lane + 32, ...; the butterfly reductions below have a
+  // fixed order, so the result is bitwise reproducible.
   float G = -INFINITY, lost = -INFINITY;
-  for (int s = 0; s < S; ++s) {
+  for (int s = lane; s < S; s += 32) {
     const int t0 = s * p.tiles_per_split, t1 = min(t0 + p.tiles_per_split, ntv);
     if (t1 <= t0) continue;
-    const float U = base[s * stride], l = base[s * stride + 1];
-    if (l > 0.f) G = fmaxf(G, U + log2f(l));
-    lost = fmaxf(lost, U - 126.f + log2f(static_cast<float>((t1 - t0) * enc_tile(D))));
+    const float2 ul = *reinterpret_cast<const float2*>(base + s * stride);
+    if (ul.y > 0.f) G = fmaxf(G, ul.x + log2f(ul.y));
+    lost = fmaxf(lost, ul.x - 126.f + log2f(static_cast<float>((t1 - t0) * enc_tile(D))));
   }
+  G = warp_max(G);
+  lost = warp_max(lost);
   const bool exact = !(G > -INFINITY) || (lost + log2f(static_cast<float>(S)) - G > -27.f);
   float z = 0.f;
   if (!exact) {
-    float num = 0.f, den = 0.f;
-    for (int s = 0; s < S; ++s) {
+    float num[D], den = 0.f;
+#pragma unroll
+    for (int d = 0; d < D; ++d) num[d] = 0.f;
+    for (int s = lane; s < S; s += 32) {
       const int t0 = s * p.tiles_per_split, t1 = min(t0 + p.tiles_per_split, ntv);
       if (t1 <= t0) continue;
-      const float* e = base + s * stride;
-      const float l = e[1];
-      if (!(l > 0.f)) continue;
-      const float w = exp2f(e[0] - G);
-      den = fmaf(w, l, den);
-      if (lane < D) num = fmaf(w, e[2 + lane], num);
+      const float* e = base + s * stride;  // (U, l, O[D]), 8-byte aligned
+      const float2 ul = *reinterpret_cast<const float2*>(e);
+      if (!(ul.y > 0.f)) continue;
+      const float w = exp2f(ul.x - G);
+      den = fmaf(w, ul.y, den);
+#pragma unroll
+      for (int d = 0; d < D; d += 2) {
+        const float2 o = *reinterpret_cast<const float2*>(e + 2 + d);
+        num[d] = fmaf(w, o.x, num[d]);
+        num[d + 1] = fmaf(w, o.y, num[d + 1]);
+      }
     }
-    z = num / den;
+    den = warp_sum(den);
+    float mine = 0.f;
+#pragma unroll
+    for (int d = 0; d < D; ++d) {
+      const float t = warp_sum(num[d]);
+      if (d == lane) mine = t;
+    }
+    z = mine / den;
   } else {
     const int g = p.q_per_batch ? bh : h;
     z = merge_exact_row<D>(p, p.q + (static_cast<size_t>(g) * p.M + m) * D, p.k + static_cast<size_t>(bh) * p.N * D,
