@@ -19,8 +19,9 @@
  *                        matrix W (section "Full self-attention": H heads of
  *                        width D = C/H).
  *
- * The head concatenation and the output projection W_O are not part of these
- * calls; Y is returned per head.
+ * flarepp_mixer_out_fwd adds the head concatenation and the output projection
+ * of section "Full self-attention" (the heads' outputs side by side, times
+ * the C x C matrix W_O); the other calls return Y per head.
  *
  * Conventions shared by every call
  * --------------------------------
@@ -88,6 +89,7 @@ typedef enum {
 /* Variant selector for flare_workspace_bytes(). */
 #define FLARE_VARIANT_FLARE 0
 #define FLARE_VARIANT_FLAREPP 1
+#define FLARE_VARIANT_FLAREPP_OUT 2 /* flarepp_mixer_out_fwd */
 
 /*
  * Workspace size in bytes for one call with these sizes (C is ignored for
@@ -115,12 +117,32 @@ FLARE_API flare_status flare_mixer_fwd(const flare_bf16* K, const flare_bf16* V,
  *   Qx_out, Z_out           [B][H][M][D] float, written if not NULL (the
  *                           synthesised routing queries Q(X) and the latent
  *                           values Z, for inspection)
+ * Passing the same pointers as Wk_syn/Wv_syn and Wk/Wv selects the shared
+ * projection variant (W~ = W, so K~ = K and V~ = V): the result is the same
+ * as with two copies of the weights, and only two projections are computed.
  */
 FLARE_API flare_status flarepp_mixer_fwd(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
                                const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0,
                                flare_bf16* Y, int B, int N, int C, int H, int M, int D,
                                const int32_t* lengths, float scale, void* workspace, size_t workspace_bytes,
                                void* stream, float* Qx_out, float* Z_out);
+
+/*
+ * FLARE++ mixer forward with the head concatenation and the output
+ * projection (section "Full self-attention"):
+ *   Out[b][n][:] = (Y_1[b][n][:], ..., Y_H[b][n][:]) @ W_O
+ * with Y_h as in flarepp_mixer_fwd.
+ *   X, Wk, Wv, Wk_syn, Wv_syn, Q0   as in flarepp_mixer_fwd
+ *   Wo    [C][C] bf16, read only (W_O, row-vector convention: Out = Ycat @ Wo)
+ *   Out   [B][N][C] bf16, written; rows of padding tokens are zero
+ * Needs flare_workspace_bytes(FLARE_VARIANT_FLAREPP_OUT, ...) bytes of
+ * workspace (the FLARE++ workspace plus Y with the heads side by side).
+ */
+FLARE_API flare_status flarepp_mixer_out_fwd(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                                             const flare_bf16* Wk_syn, const flare_bf16* Wv_syn,
+                                             const flare_bf16* Q0, const flare_bf16* Wo, flare_bf16* Out, int B,
+                                             int N, int C, int H, int M, int D, const int32_t* lengths, float scale,
+                                             void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Profiling variants: identical work, plus cudaEventRecord() of caller-created

@@ -189,10 +189,23 @@ def flarepp_forward(X, Wk, Wv, Wk_syn, Wv_syn, Q0, H: int, lengths=None, scale=N
     return out
 
 
+def output_projection(Y, Wo):
+    """Head concatenation and output projection (section "Full self-attention":
+    the heads' outputs side by side, times W_O): Out[b, n, :] =
+    (Y[b, 0, n, :], ..., Y[b, H-1, n, :]) @ Wo, in float64."""
+    Y = np.asarray(Y, dtype=np.float64)
+    B, H, N, D = Y.shape
+    Ycat = np.ascontiguousarray(np.transpose(Y, (0, 2, 1, 3))).reshape(B, N, H * D)
+    return Ycat @ np.asarray(Wo, dtype=np.float64)
+
+
 def forward_workload(w, rows=None, keep_projections: bool = False) -> dict:
     """Run the oracle on a ``workloads.Workload`` (bf16 bits widened to fp64)."""
     from workloads import bf16_bits_to_f64 as f64
     if w.variant == "flare":
         return flare_forward(f64(w.K), f64(w.V), f64(w.Q), w.lengths, w.scale, rows)
-    return flarepp_forward(f64(w.X), f64(w.Wk), f64(w.Wv), f64(w.Wk_syn), f64(w.Wv_syn),
-                           f64(w.Q0), w.H, w.lengths, w.scale, rows, keep_projections)
+    out = flarepp_forward(f64(w.X), f64(w.Wk), f64(w.Wv), f64(w.Wk_syn), f64(w.Wv_syn),
+                          f64(w.Q0), w.H, w.lengths, w.scale, rows, keep_projections)
+    if w.Wo is not None and rows is None:
+        out["Out"] = output_projection(out["Y"], f64(w.Wo))
+    return out

@@ -9,6 +9,7 @@ CPU fallback: if the library cannot be loaded, every call raises.
 from ._binding import (  # noqa: F401
     FLARE_VARIANT_FLARE,
     FLARE_VARIANT_FLAREPP,
+    FLARE_VARIANT_FLAREPP_OUT,
     FlareError,
     Status,
     flare_last_device_status,
@@ -18,6 +19,7 @@ from ._binding import (  # noqa: F401
     flare_status_string,
     flare_workspace_bytes,
     flarepp_mixer_fwd,
+    flarepp_mixer_out_fwd,
     library_path,
     load_library,
 )

@@ -14,6 +14,7 @@ _lib = None
 
 FLARE_VARIANT_FLARE = 0
 FLARE_VARIANT_FLAREPP = 1
+FLARE_VARIANT_FLAREPP_OUT = 2
 
 
 class Status(enum.IntEnum):
@@ -59,6 +60,8 @@ def load_library(build_if_missing: bool = True):
         lib.flare_mixer_fwd_profiled.argtypes = lib.flare_mixer_fwd.argtypes + [vp]
         lib.flare_mixer_fwd_profiled.restype = i
         lib.flarepp_mixer_fwd_profiled.argtypes = lib.flarepp_mixer_fwd.argtypes + [vp]
+        lib.flarepp_mixer_out_fwd.restype = i
+        lib.flarepp_mixer_out_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, f, vp, sz, vp]
         lib.flarepp_mixer_fwd_profiled.restype = i
         lib.flare_mixer_fwd_static.argtypes = [vp, vp, vp, vp, i, i, i, i, i, vp, f, vp, vp]
         lib.flare_mixer_fwd_static.restype = i
@@ -196,6 +199,32 @@ def flarepp_mixer_fwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, lengths=None, scale: float 
     if st != 0:
         raise FlareError(st, "flarepp_mixer_fwd")
     return Y
+
+
+def flarepp_mixer_out_fwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, Wo, lengths=None, scale: float = 0.0, Out=None,
+                          workspace=None, stream=None, check: bool = True):
+    """FLARE++ forward with the head concatenation and output projection:
+    Out [B,N,C] bf16 = (Y_1 | ... | Y_H) @ Wo.  Passing the same tensors as
+    Wk_syn/Wv_syn and Wk/Wv selects the shared-projection variant."""
+    torch = _torch()
+    B, N, C = X.shape
+    H, M, D = Q0.shape
+    if check:
+        _check_dev("X", X, torch.bfloat16)
+        for nm, w in (("Wk", Wk), ("Wv", Wv), ("Wk_syn", Wk_syn), ("Wv_syn", Wv_syn), ("Wo", Wo)):
+            _check_dev(nm, w, torch.bfloat16, (C, C))
+        _check_dev("Q0", Q0, torch.bfloat16)
+        _check_dev("lengths", lengths, torch.int32, (B,))
+    if Out is None:
+        Out = torch.empty((B, N, C), dtype=torch.bfloat16, device=X.device)
+    nbytes = flare_workspace_bytes(FLARE_VARIANT_FLAREPP_OUT, B, H, N, M, D, C)
+    workspace = _workspace(workspace, nbytes, X.device)
+    st = load_library().flarepp_mixer_out_fwd(
+        _ptr(X), _ptr(Wk), _ptr(Wv), _ptr(Wk_syn), _ptr(Wv_syn), _ptr(Q0), _ptr(Wo), _ptr(Out), B, N, C, H, M, D,
+        _ptr(lengths), float(scale), _ptr(workspace), workspace.numel(), _stream_ptr(stream, X.device))
+    if st != 0:
+        raise FlareError(st, "flarepp_mixer_out_fwd")
+    return Out
 
 
 FLARE_STATIC_SCRATCH_BYTES = 64 << 20

@@ -97,7 +97,7 @@ struct Plan {
   int dec_ctas = 1, dec_tiles = 1;       // decoder CTAs per head, tiles per CTA
   int G32 = 1;
   size_t off_err = 0, off_kt = 0, off_vt = 0, off_kp = 0, off_vp = 0, off_kn_syn = 0, off_kn = 0, off_part = 0,
-         off_qx32 = 0, off_qx16 = 0, off_z32 = 0, off_z16 = 0, off_fb = 0, total = 0;
+         off_qx32 = 0, off_qx16 = 0, off_z32 = 0, off_z16 = 0, off_fb = 0, off_ycat = 0, total = 0;
 };
 
 Plan make_plan(int variant, long B, long H, long N, long M, long D) {
@@ -118,7 +118,8 @@ Plan make_plan(int variant, long B, long H, long N, long M, long D) {
   p.off_err = off;
   off += 256;
   const size_t proj = align256(static_cast<size_t>(BH * N * D) * 2);
-  if (variant == FLARE_VARIANT_FLAREPP) {
+  const bool pp = variant == FLARE_VARIANT_FLAREPP || variant == FLARE_VARIANT_FLAREPP_OUT;
+  if (pp) {
     p.off_kt = off; off += proj;
     p.off_vt = off; off += proj;
     p.off_kp = off; off += proj;
@@ -128,13 +129,16 @@ Plan make_plan(int variant, long B, long H, long N, long M, long D) {
   p.off_kn = off; off += align256(static_cast<size_t>(BH) * p.G32 * 4);
   p.off_part = off; off += align256(static_cast<size_t>(BH) * p.S * M * (D + 2) * 4);
   const size_t lat32 = align256(static_cast<size_t>(BH * M * D) * 4), lat16 = align256(static_cast<size_t>(BH * M * D) * 2);
-  if (variant == FLARE_VARIANT_FLAREPP) {
+  if (pp) {
     p.off_qx32 = off; off += lat32;
     p.off_qx16 = off; off += lat16;
   }
   p.off_z32 = off; off += lat32;
   p.off_z16 = off; off += lat16;
   p.off_fb = off; off += align256(static_cast<size_t>(BH) * N * 8);
+  if (variant == FLARE_VARIANT_FLAREPP_OUT) {  // Y with the heads side by side, [B][N][C]
+    p.off_ycat = off; off += proj;
+  }
   p.total = off;
   return p;
 }
@@ -198,8 +202,8 @@ flare_status run_encode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
 }
 
 flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_batch, const uint16_t* z16,
-                        const void* k, void* y, int B, int H, int N, int M, int D, const int32_t* lengths,
-                        float scale, cudaStream_t st) {
+                        const void* k, void* y, int y_token_major, int B, int H, int N, int M, int D,
+                        const int32_t* lengths, float scale, cudaStream_t st) {
   const long BH = static_cast<long>(B) * H;
   const long G = q_per_batch ? BH : H;
   CUtensorMap tq, tz, tk;
@@ -218,6 +222,7 @@ flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
   dp.z = z16;
   dp.k = static_cast<const uint16_t*>(k);
   dp.y = static_cast<uint16_t*>(y);
+  dp.y_token_major = y_token_major;
   dp.err = reinterpret_cast<uint32_t*>(ws + pl.off_err);
   dp.fb_count = reinterpret_cast<uint32_t*>(ws + pl.off_err) + 1;
   dp.fb_list = reinterpret_cast<uint64_t*>(ws + pl.off_fb);
@@ -263,9 +268,10 @@ using namespace flare;
 extern "C" {
 
 size_t flare_workspace_bytes(int variant, int B, int H, int N, int M, int D, int C) {
-  if (variant != FLARE_VARIANT_FLARE && variant != FLARE_VARIANT_FLAREPP) return 0;
+  if (variant != FLARE_VARIANT_FLARE && variant != FLARE_VARIANT_FLAREPP && variant != FLARE_VARIANT_FLAREPP_OUT)
+    return 0;
   if (check_common(B, H, N, M, D) != FLARE_OK) return 0;
-  if (variant == FLARE_VARIANT_FLAREPP && (C != H * D || C % 64 != 0 || C > 256)) return 0;
+  if (variant != FLARE_VARIANT_FLARE && (C != H * D || C % 64 != 0 || C > 256)) return 0;
   return make_plan(variant, B, H, N, M, D).total;
 }
 
@@ -306,7 +312,7 @@ flare_status flare_mixer_fwd_profiled(const flare_bf16* K, const flare_bf16* V, 
   uint16_t* z16 = reinterpret_cast<uint16_t*>(ws + pl.off_z16);
   st = run_encode(pl, ws, Q, 0, K, V, kp.knorm, z32, z16, B, H, N, M, D, lengths, sc, s, stage_events, 2);
   if (st != FLARE_OK) return st;
-  st = run_decode(pl, ws, Q, 0, z16, K, Y, B, H, N, M, D, lengths, sc, s);
+  st = run_decode(pl, ws, Q, 0, z16, K, Y, 0, B, H, N, M, D, lengths, sc, s);
   if (st != FLARE_OK) return st;
   return record(stage_events, 4, s) ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
@@ -318,12 +324,15 @@ flare_status flare_mixer_fwd(const flare_bf16* K, const flare_bf16* V, const fla
                                   Z_out, nullptr);
 }
 
-flare_status flarepp_mixer_fwd_profiled(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
-                                        const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0,
-                                        flare_bf16* Y, int B, int N, int C, int H, int M, int D,
-                                        const int32_t* lengths, float scale, void* workspace,
-                                        size_t workspace_bytes, void* stream, float* Qx_out, float* Z_out,
-                                        void* const* stage_events) {
+}  // extern "C"
+
+namespace flare {
+namespace {
+
+// Shape, pointer and alignment checks shared by the FLARE++ entry points.
+flare_status check_flarepp(const void* X, const void* Wk, const void* Wv, const void* Wk_syn, const void* Wv_syn,
+                           const void* Q0, const void* Y, int B, int N, int C, int H, int M, int D,
+                           const int32_t* lengths, const void* workspace, const float* Qx_out, const float* Z_out) {
   if (!X || !Wk || !Wv || !Wk_syn || !Wv_syn || !Q0 || !Y || !workspace) return FLARE_ERR_NULL;
   flare_status st = check_common(B, H, N, M, D);
   if (st != FLARE_OK) return st;
@@ -333,40 +342,69 @@ flare_status flarepp_mixer_fwd_profiled(const flare_bf16* X, const flare_bf16* W
       !aligned16(Q0) || !aligned16(Y) || !aligned16(lengths) || !aligned16(Qx_out) || !aligned16(Z_out) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return FLARE_ERR_ALIGN;
-  const Plan pl = make_plan(FLARE_VARIANT_FLAREPP, B, H, N, M, D);
-  if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
-  const float sc = resolve_scale(scale, D);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  if (cudaMemsetAsync(ws + pl.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  return FLARE_OK;
+}
 
-  // eq. 7 and eq. 9: the four per-head projections
+// Projection launch: n_proj weights (tensor maps tw[0..n_proj)) into out[]
+// ([B][H][N][D], or [B][N][C] when token_major), key norms where given.
+flare_status run_project(const Plan& pl, uint8_t* ws, const CUtensorMap& tx, const CUtensorMap (&tw)[4], int n_proj,
+                         int token_major, uint16_t* const (&out)[4], float* const (&knorm)[4], int B, int N, int C,
+                         int H, int D, cudaStream_t s) {
+  ProjParams pp{};
+  pp.B = B; pp.N = N; pp.C = C; pp.H = H; pp.D = D;
+  pp.tiles_per_b = static_cast<int>(cdiv(N, kProjTile));
+  pp.n_tiles = B * pp.tiles_per_b;
+  const int slots = C == 256 ? kNumSM : kNumSM * 2;
+  pp.groups = std::max(1, std::min(pp.n_tiles, slots / n_proj));
+  pp.n_groups32 = pl.G32;
+  pp.n_proj = n_proj;
+  pp.token_major = token_major;
+  for (int i = 0; i < 4; ++i) {
+    pp.out[i] = out[i];
+    pp.knorm[i] = knorm[i];
+  }
+  pp.err = reinterpret_cast<uint32_t*>(ws + pl.off_err);
+  pp.timeout_ns = wait_timeout_ns();
+  return launch_project(tx, tw, pp, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+}
+
+// The FLARE++ pipeline (eq. 7-11) after the argument checks.  Y is written
+// [B][H][N][D], or [B][N][C] when y_token_major.
+flare_status flarepp_run(const Plan& pl, const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                         const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0, void* Y,
+                         int y_token_major, int B, int N, int C, int H, int M, int D, const int32_t* lengths,
+                         float sc, uint8_t* ws, cudaStream_t s, float* Qx_out, float* Z_out,
+                         void* const* stage_events) {
+  if (cudaMemsetAsync(ws + pl.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  // The same weights for synthesis and encode (the shared-projection
+  // variant): K~ = K and V~ = V, so two projections serve both passes.
+  const bool shared = Wk_syn == Wk && Wv_syn == Wv;
+  // eq. 7 and eq. 9: the per-head projections
   CUtensorMap tx, tw[4];
-  if (!map3d(&tx, X, C, N, B, 64, kProjTile, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map2d(&tw[0], Wk_syn, C, C, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map2d(&tw[1], Wv_syn, C, C, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map2d(&tw[2], Wk, C, C, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !map2d(&tw[3], Wv, C, C, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
-    return FLARE_ERR_LAUNCH;
+  const flare_bf16* w[4] = {Wk_syn, Wv_syn, Wk, Wv};
+  if (shared) {
+    w[0] = Wk;
+    w[1] = Wv;
+  }
+  if (!map3d(&tx, X, C, N, B, 64, kProjTile, CU_TENSOR_MAP_SWIZZLE_128B)) return FLARE_ERR_LAUNCH;
+  for (int i = 0; i < 4; ++i)
+    if (!map2d(&tw[i], w[i], C, C, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return FLARE_ERR_LAUNCH;
   uint16_t* kt = reinterpret_cast<uint16_t*>(ws + pl.off_kt);
   uint16_t* vt = reinterpret_cast<uint16_t*>(ws + pl.off_vt);
   uint16_t* kk = reinterpret_cast<uint16_t*>(ws + pl.off_kp);
   uint16_t* vv = reinterpret_cast<uint16_t*>(ws + pl.off_vp);
   float* kn_syn = reinterpret_cast<float*>(ws + pl.off_kn_syn);
   float* kn = reinterpret_cast<float*>(ws + pl.off_kn);
+  if (shared) {
+    kt = kk;
+    vt = vv;
+    kn_syn = kn;
+  }
   if (!record(stage_events, 0, s)) return FLARE_ERR_LAUNCH;
-  ProjParams pp{};
-  pp.B = B; pp.N = N; pp.C = C; pp.H = H; pp.D = D;
-  pp.tiles_per_b = static_cast<int>(cdiv(N, kProjTile));
-  pp.n_tiles = B * pp.tiles_per_b;
-  const int slots = C == 256 ? kNumSM : kNumSM * 2;
-  pp.groups = std::max(1, std::min(pp.n_tiles, slots / 4));
-  pp.n_groups32 = pl.G32;
-  pp.out[0] = kt; pp.out[1] = vt; pp.out[2] = kk; pp.out[3] = vv;
-  pp.knorm[0] = kn_syn; pp.knorm[1] = nullptr; pp.knorm[2] = kn; pp.knorm[3] = nullptr;
-  pp.err = reinterpret_cast<uint32_t*>(ws + pl.off_err);
-  pp.timeout_ns = wait_timeout_ns();
-  if (launch_project(tx, tw, pp, s) != cudaSuccess || !record(stage_events, 1, s)) return FLARE_ERR_LAUNCH;
+  uint16_t* const outs[4] = {kt, vt, kk, vv};
+  float* const norms[4] = {kn_syn, nullptr, kn, nullptr};
+  flare_status st = run_project(pl, ws, tx, tw, shared ? 2 : 4, 0, outs, norms, B, N, C, H, D, s);
+  if (st != FLARE_OK || !record(stage_events, 1, s)) return FLARE_ERR_LAUNCH;
 
   // eq. 8: query synthesis with the learned seeds
   float* qx32 = Qx_out ? Qx_out : reinterpret_cast<float*>(ws + pl.off_qx32);
@@ -379,9 +417,59 @@ flare_status flarepp_mixer_fwd_profiled(const flare_bf16* X, const flare_bf16* W
   st = run_encode(pl, ws, qx16, 1, kk, vv, kn, z32, z16, B, H, N, M, D, lengths, sc, s, stage_events, 4);
   if (st != FLARE_OK) return st;
   // eq. 11: decode
-  st = run_decode(pl, ws, qx16, 1, z16, kk, Y, B, H, N, M, D, lengths, sc, s);
+  st = run_decode(pl, ws, qx16, 1, z16, kk, Y, y_token_major, B, H, N, M, D, lengths, sc, s);
   if (st != FLARE_OK) return st;
   return record(stage_events, 6, s) ? FLARE_OK : FLARE_ERR_LAUNCH;
+}
+
+}  // namespace
+}  // namespace flare
+
+extern "C" {
+
+flare_status flarepp_mixer_fwd_profiled(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                                        const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0,
+                                        flare_bf16* Y, int B, int N, int C, int H, int M, int D,
+                                        const int32_t* lengths, float scale, void* workspace,
+                                        size_t workspace_bytes, void* stream, float* Qx_out, float* Z_out,
+                                        void* const* stage_events) {
+  flare_status st = check_flarepp(X, Wk, Wv, Wk_syn, Wv_syn, Q0, Y, B, N, C, H, M, D, lengths, workspace, Qx_out,
+                                  Z_out);
+  if (st != FLARE_OK) return st;
+  const Plan pl = make_plan(FLARE_VARIANT_FLAREPP, B, H, N, M, D);
+  if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
+  return flarepp_run(pl, X, Wk, Wv, Wk_syn, Wv_syn, Q0, Y, 0, B, N, C, H, M, D, lengths, resolve_scale(scale, D),
+                     static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream), Qx_out, Z_out,
+                     stage_events);
+}
+
+flare_status flarepp_mixer_out_fwd(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                                   const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0,
+                                   const flare_bf16* Wo, flare_bf16* Out, int B, int N, int C, int H, int M, int D,
+                                   const int32_t* lengths, float scale, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  if (!Wo) return FLARE_ERR_NULL;
+  flare_status st = check_flarepp(X, Wk, Wv, Wk_syn, Wv_syn, Q0, Out, B, N, C, H, M, D, lengths, workspace,
+                                  nullptr, nullptr);
+  if (st != FLARE_OK) return st;
+  if (!aligned16(Wo)) return FLARE_ERR_ALIGN;
+  const Plan pl = make_plan(FLARE_VARIANT_FLAREPP_OUT, B, H, N, M, D);
+  if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint16_t* ycat = reinterpret_cast<uint16_t*>(ws + pl.off_ycat);  // [B][N][C], heads side by side
+  st = flarepp_run(pl, X, Wk, Wv, Wk_syn, Wv_syn, Q0, ycat, 1, B, N, C, H, M, D, lengths, resolve_scale(scale, D),
+                   ws, s, nullptr, nullptr, nullptr);
+  if (st != FLARE_OK) return st;
+  // Out = concat_h(Y_h) W_O: the same tcgen05 projection with one weight and
+  // token-major output rows
+  CUtensorMap ty, two[4];
+  if (!map3d(&ty, ycat, C, N, B, 64, kProjTile, CU_TENSOR_MAP_SWIZZLE_128B)) return FLARE_ERR_LAUNCH;
+  for (int i = 0; i < 4; ++i)
+    if (!map2d(&two[i], Wo, C, C, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return FLARE_ERR_LAUNCH;
+  uint16_t* const outs[4] = {Out, nullptr, nullptr, nullptr};
+  float* const norms[4] = {nullptr, nullptr, nullptr, nullptr};
+  return run_project(pl, ws, ty, two, 1, 1, outs, norms, B, N, C, H, D, s);
 }
 
 flare_status flarepp_mixer_fwd(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,

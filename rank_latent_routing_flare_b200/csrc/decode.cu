@@ -62,6 +62,17 @@ struct DecCfg {
   static_assert(OFF_K % 256 == 0, "key tiles must start on a swizzle atom");
 };
 
+// Output row of token n of head bh: [B*H][N][D], or [B][N][H*D] (the heads of
+// a token side by side) when p.y_token_major.
+template <int D>
+__device__ __forceinline__ uint16_t* y_row(const DecodeParams& p, int bh, int n) {
+  if (p.y_token_major) {
+    const int b = bh / p.H, h = bh - b * p.H;
+    return p.y + (static_cast<size_t>(b) * p.N + n) * (static_cast<size_t>(p.H) * D) + static_cast<size_t>(h) * D;
+  }
+  return p.y + (static_cast<size_t>(bh) * p.N + n) * D;
+}
+
 __device__ __forceinline__ float bf16_row_norm2(const uint4* row, int n16) {
   float s = 0.f;
   for (int u = 0; u < n16; ++u) {
@@ -114,7 +125,7 @@ __global__ void __launch_bounds__(128) decode_fallback_kernel(const DecodeParams
       for (int d = 0; d < D; ++d) y[d] = fmaf(w, __uint_as_float(static_cast<uint32_t>(zh[m * D + d]) << 16), y[d]);
     }
     const float inv = 1.f / den;
-    uint4* dst = reinterpret_cast<uint4*>(p.y + (static_cast<size_t>(bh) * p.N + n) * D);
+    uint4* dst = reinterpret_cast<uint4*>(y_row<D>(p, bh, n));
 #pragma unroll
     for (int u = 0; u < D / 8; ++u)
       dst[u] = make_uint4(pack_bf16x2(y[8 * u + 0] * inv, y[8 * u + 1] * inv),
@@ -171,7 +182,6 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
   const int tc_end = min(tb, tiles_valid);            // tiles [ta, tc_end) are computed
   const int ntiles = max(0, tc_end - ta);
   const int nc = (p.M + C - 1) / C;                   // latent chunks
-  uint16_t* yh = p.y + static_cast<size_t>(bh) * p.N * D;
 
   // tiles entirely past the valid length: zero rows
   {
@@ -180,7 +190,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
     const uint4 zero = make_uint4(0, 0, 0, 0);
     for (size_t e = static_cast<size_t>(z0) * (D / 8) + threadIdx.x; e < static_cast<size_t>(z1) * (D / 8);
          e += blockDim.x)
-      reinterpret_cast<uint4*>(yh)[e] = zero;
+      reinterpret_cast<uint4*>(y_row<D>(p, bh, static_cast<int>(e / (D / 8))))[e % (D / 8)] = zero;
   }
   if (ntiles == 0) return;
 
@@ -361,7 +371,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
         const uint32_t e = atomicAdd(p.fb_count, 1u);
         p.fb_list[e] = static_cast<uint64_t>(bh) * p.N + n;
       } else if (n < p.N) {
-        uint4* dst = reinterpret_cast<uint4*>(yh + static_cast<size_t>(n) * D);
+        uint4* dst = reinterpret_cast<uint4*>(y_row<D>(p, bh, n));
 #pragma unroll
         for (int u = 0; u < D / 8; ++u)
           dst[u] = make_uint4(pack_bf16x2(y[8 * u + 0], y[8 * u + 1]), pack_bf16x2(y[8 * u + 2], y[8 * u + 3]),

@@ -48,6 +48,10 @@ __host__ __device__ constexpr int dec_ctas_per_sm(int D) { return D == 16 ? FLAR
 #ifndef FLARE_ENC_SPLIT_LD
 #define FLARE_ENC_SPLIT_LD 1
 #endif
+// Heads whose projection outputs are read from TMEM per wait.
+#ifndef FLARE_PROJ_EPI_HEADS
+#define FLARE_PROJ_EPI_HEADS 4
+#endif
 #ifndef FLARE_DEC_POLY_PAIRS
 #define FLARE_DEC_POLY_PAIRS 6
 #endif
@@ -61,7 +65,9 @@ struct ProjParams {
   int n_tiles;         // B * tiles_per_b
   int groups;          // CTAs per projection
   int n_groups32;      // ceil(N / kNormGroup)
-  uint16_t* out[4];    // [B][H][N][D] bf16
+  int n_proj;          // projections computed: 1, 2 or 4 (weights tm_w0 .. tm_w{n_proj-1})
+  int token_major;     // 0: out [B][H][N][D]; 1: out [B][N][C] (row n = heads side by side)
+  uint16_t* out[4];    // bf16, layout per token_major
   float* knorm[4];     // [B*H][n_groups32] max key norm per group, or nullptr
   uint32_t* err;
   unsigned long long timeout_ns;
@@ -127,7 +133,8 @@ struct DecodeParams {
   const uint16_t* q;    // bf16 [G][M][D]
   const uint16_t* z;    // bf16 [B*H][M][D]
   const uint16_t* k;    // bf16 [B*H][N][D]
-  uint16_t* y;          // bf16 [B*H][N][D]
+  uint16_t* y;          // bf16 [B*H][N][D], or [B][N][H*D] when y_token_major
+  int y_token_major;
   uint32_t* fb_count;   // number of listed tokens (zeroed before the decoder runs)
   uint64_t* fb_list;    // tokens (bh * N + n) whose row sum underflowed, capacity B*H*N
   uint32_t* err;

@@ -55,8 +55,8 @@ __global__ void __launch_bounds__(192, 1)
   int* abort_flag = reinterpret_cast<int*>(sm + Cfg::OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int proj = blockIdx.x & 3;
-  const int grp = blockIdx.x >> 2;
+  const int proj = blockIdx.x % p.n_proj;
+  const int grp = blockIdx.x / p.n_proj;
   const int H = p.H;
   const int my_tiles = (grp < p.n_tiles) ? (p.n_tiles - 1 - grp) / p.groups + 1 : 0;
   if (my_tiles == 0) return;
@@ -164,41 +164,42 @@ __global__ void __launch_bounds__(192, 1)
       const int n = n0 + r;
       if (!mbar_wait_warp(acc_full + ab, (i >> 1) & 1, wc)) break;
       tc_fence_after();
-      for (int hh = 0; hh < H; ++hh) {
-        uint32_t v[32];
-        if constexpr (D == 16) {
-          uint32_t t[16];
-          tmem_ld16(lane_base + ab * C + hh * 16, t);
-          tmem_wait_ld();
+      // G heads per TMEM read (one wait per G heads)
+      constexpr int G = FLARE_PROJ_EPI_HEADS;
+      for (int h0 = 0; h0 < H; h0 += G) {
+        uint32_t v[G][D];
 #pragma unroll
-          for (int d = 0; d < 16; ++d) v[d] = t[d];
-        } else {
-          tmem_ld32(lane_base + ab * C + hh * 32, v);
-          tmem_wait_ld();
-        }
-        uint32_t pk[16];
-        float nrm = 0.f;
+        for (int j = 0; j < G; ++j)
+          if (h0 + j < H) tmem_ld_cols<D>(lane_base + ab * C + (h0 + j) * D, v[j]);
+        tmem_wait_ld();
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          if (2 * k < D) {
-            pk[k] = pack_bf16x2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+        for (int j = 0; j < G; ++j) {
+          const int hh = h0 + j;
+          if (hh >= H) break;
+          uint32_t pk[D / 2];
+          float nrm = 0.f;
+#pragma unroll
+          for (int k = 0; k < D / 2; ++k) {
+            pk[k] = pack_bf16x2(__uint_as_float(v[j][2 * k]), __uint_as_float(v[j][2 * k + 1]));
             const float a = bf16_lo(pk[k]), bb = bf16_hi(pk[k]);
             nrm = fmaf(a, a, fmaf(bb, bb, nrm));
           }
-        }
-        if (n < p.N) {
-          uint4* dst = reinterpret_cast<uint4*>(out + ((static_cast<size_t>(b) * H + hh) * p.N + n) * D);
+          if (n < p.N) {
+            const size_t row = p.token_major ? (static_cast<size_t>(b) * p.N + n) * p.C + hh * D
+                                             : ((static_cast<size_t>(b) * H + hh) * p.N + n) * D;
+            uint4* dst = reinterpret_cast<uint4*>(out + row);
 #pragma unroll
-          for (int u = 0; u < D / 8; ++u)
-            dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-        } else {
-          nrm = 0.f;
-        }
-        if (knorm != nullptr) {
-          const float gm = warp_max(sqrtf(nrm));
-          const int gi = n0 / kNormGroup + wq;
-          if (lane == 0 && gi < p.n_groups32)
-            knorm[(static_cast<size_t>(b) * H + hh) * p.n_groups32 + gi] = gm;
+            for (int u = 0; u < D / 8; ++u)
+              dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+          } else {
+            nrm = 0.f;
+          }
+          if (knorm != nullptr) {
+            const float gm = warp_max(sqrtf(nrm));
+            const int gi = n0 / kNormGroup + wq;
+            if (lane == 0 && gi < p.n_groups32)
+              knorm[(static_cast<size_t>(b) * H + hh) * p.n_groups32 + gi] = gm;
+          }
         }
       }
       tc_fence_before();
@@ -220,7 +221,7 @@ cudaError_t launch_project_cd(const CUtensorMap& tm_x, const CUtensorMap (&tm_w)
   cudaError_t e = cudaFuncSetAttribute(project_kernel<C, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  project_kernel<C, D><<<dim3(4 * p.groups), 192, smem, s>>>(tm_x, tm_w[0], tm_w[1], tm_w[2], tm_w[3], p);
+  project_kernel<C, D><<<dim3(p.n_proj * p.groups), 192, smem, s>>>(tm_x, tm_w[0], tm_w[1], tm_w[2], tm_w[3], p);
   return cudaGetLastError();
 }
 

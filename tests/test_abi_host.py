@@ -29,7 +29,7 @@ def declared_functions():
 
 def test_header_declares_the_abi():
     names = declared_functions()
-    assert names == sorted(["flare_workspace_bytes", "flare_mixer_fwd", "flarepp_mixer_fwd",
+    assert names == sorted(["flare_workspace_bytes", "flare_mixer_fwd", "flarepp_mixer_fwd", "flarepp_mixer_out_fwd",
                             "flare_mixer_fwd_profiled", "flarepp_mixer_fwd_profiled", "flare_mixer_fwd_static",
                             "flare_last_device_status", "flare_status_string",
                             "flare_selftest_wait_timeout"])
@@ -86,8 +86,16 @@ def test_workspace_unsupported_sizes_return_zero():
     assert fl.flare_workspace_bytes(0, 1, 1, 64, 528, 16, 0) == 0      # M > 512
     assert fl.flare_workspace_bytes(1, 1, 2, 64, 32, 16, 48) == 0      # C != H*D
     assert fl.flare_workspace_bytes(1, 1, 3, 64, 32, 16, 48) == 0      # C not a multiple of 64
-    assert fl.flare_workspace_bytes(2, 1, 1, 64, 32, 16, 16) == 0      # bad variant
+    assert fl.flare_workspace_bytes(3, 1, 1, 64, 32, 16, 64) == 0      # bad variant
+    assert fl.flare_workspace_bytes(2, 1, 3, 64, 32, 16, 48) == 0      # C not a multiple of 64
     assert fl.flare_workspace_bytes(0, 0, 1, 64, 32, 16, 0) == 0       # B = 0
+
+
+def test_output_projection_workspace_adds_the_concatenated_heads():
+    for B, H, N, M, D, C in [(1, 4, 1024, 32, 16, 64), (32, 8, 4096, 128, 32, 256), (1, 8, 1 << 20, 512, 16, 128)]:
+        base = fl.flare_workspace_bytes(1, B, H, N, M, D, C)
+        out = fl.flare_workspace_bytes(2, B, H, N, M, D, C)
+        assert out >= base + B * N * C * 2 and out % 256 == 0
 
 
 def flare_call(K=A, V=A, Q=A, Y=A, B=1, H=2, N=100, M=32, D=16, lengths=None, ws=W, ws_bytes=1 << 40,
@@ -101,6 +109,13 @@ def flarepp_call(X=A, Wk=A, Wv=A, Wks=A, Wvs=A, Q0=A, Y=A, B=1, N=100, C=64, H=4
     lib = fl.load_library()
     return lib.flarepp_mixer_fwd(X, Wk, Wv, Wks, Wvs, Q0, Y, B, N, C, H, M, D, lengths, 0.0, ws, ws_bytes,
                                  None, Qx, Z)
+
+
+def flarepp_out_call(X=A, Wk=A, Wv=A, Wks=A, Wvs=A, Q0=A, Wo=A, Out=A, B=1, N=100, C=64, H=4, M=32, D=16,
+                     lengths=None, ws=W, ws_bytes=1 << 40):
+    lib = fl.load_library()
+    return lib.flarepp_mixer_out_fwd(X, Wk, Wv, Wks, Wvs, Q0, Wo, Out, B, N, C, H, M, D, lengths, 0.0, ws, ws_bytes,
+                                     None)
 
 
 def test_flare_argument_errors():
@@ -131,6 +146,17 @@ def test_flarepp_argument_errors():
     assert flarepp_call(ws_bytes=need - 256) == Status.ERR_WORKSPACE
 
 
+def test_flarepp_out_argument_errors():
+    assert flarepp_out_call(Wo=None) == Status.ERR_NULL
+    assert flarepp_out_call(Out=None) == Status.ERR_NULL
+    assert flarepp_out_call(C=128) == Status.ERR_SHAPE
+    assert flarepp_out_call(Wo=A + 2) == Status.ERR_ALIGN
+    assert flarepp_out_call(Out=A + 8) == Status.ERR_ALIGN
+    need = fl.flare_workspace_bytes(2, 1, 4, 100, 32, 16, 64)
+    assert need > fl.flare_workspace_bytes(1, 1, 4, 100, 32, 16, 64)
+    assert flarepp_out_call(ws_bytes=need - 256) == Status.ERR_WORKSPACE
+
+
 def test_valid_call_without_gpu_reports_launch_error():
     """With valid arguments the library reaches CUDA; on a machine without a
     GPU that fails cleanly with ERR_LAUNCH instead of crashing."""
@@ -139,6 +165,7 @@ def test_valid_call_without_gpu_reports_launch_error():
         pytest.skip("a GPU is present")
     assert flare_call() == Status.ERR_LAUNCH
     assert flarepp_call() == Status.ERR_LAUNCH
+    assert flarepp_out_call() == Status.ERR_LAUNCH
     lib = fl.load_library()
     assert lib.flare_selftest_wait_timeout(W, None, 1000) == Status.ERR_LAUNCH
     assert lib.flare_last_device_status(None, None) == Status.ERR_NULL

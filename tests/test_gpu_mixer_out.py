@@ -1,0 +1,77 @@
+"""GPU parity of the two FLARE++ extensions, through the C ABI:
+
+- flarepp_mixer_out_fwd: the head concatenation and output projection of the
+  FLARE++ paper's section "Full self-attention" (Out = (Y_1 | ... | Y_H) W_O),
+  against the fp64 oracle;
+- the shared-projection variant (the same weights for query synthesis and
+  encode, W~ = W), selected by passing the same tensors twice: it must match
+  the oracle, and give bitwise the same result as passing separate copies of
+  those weights (four projections instead of two).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rank_latent_routing_flare_b200 as fl
+from workloads import make_workload
+
+from .gpu_util import MAX_ABS, REL_L2, dev_bf16, host_f64, max_abs, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    ("flarepp_n1k", {}),
+    ("flarepp_n8k_mesh2d", {"N": 2048, "B": 2}),
+    ("flarepp_n1m_mesh3d", {"N": 8192}),
+    ("flarepp_masked_n4k", {"N": 1024, "B": 8}),
+]
+
+
+def device_inputs(w):
+    X = dev_bf16(w.X)
+    Ws = [dev_bf16(a) for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn)]
+    lengths = None if w.lengths is None else torch.from_numpy(w.lengths).cuda()
+    return X, Ws, dev_bf16(w.Q0), dev_bf16(w.Wo), lengths
+
+
+def check(got, want, label):
+    e_rel, e_abs = rel_l2(got, want), max_abs(got, want)
+    print(label, f"rel_l2={e_rel:.3e} max_abs={e_abs:.3e}")
+    assert np.all(np.isfinite(got)), label
+    assert e_rel <= REL_L2 and e_abs <= MAX_ABS, (label, e_rel, e_abs)
+
+
+@pytest.mark.parametrize("name,kw", CASES, ids=[c[0] for c in CASES])
+def test_output_projection_matches_oracle(name, kw):
+    w = make_workload(name, **kw)
+    X, Ws, Q0, Wo, lengths = device_inputs(w)
+    out = fl.flarepp_mixer_out_fwd(X, *Ws, Q0, Wo, lengths=lengths)
+    torch.cuda.synchronize()
+    got = host_f64(out)
+    ref = oracle.forward_workload(w)["Out"]
+    check(got, ref, f"out {name} {kw}")
+    if w.lengths is not None:
+        for b, L in enumerate(w.lengths):
+            assert np.all(got[b, L:] == 0), (b, L)
+
+
+def shared_workload(name, **kw):
+    """The named workload with W~_K = W_K and W~_V = W_V."""
+    w = make_workload(name, **kw)
+    w.Wk_syn, w.Wv_syn = w.Wk.copy(), w.Wv.copy()
+    return w
+
+
+@pytest.mark.parametrize("name,kw", CASES[:2] + CASES[3:], ids=[c[0] for c in CASES[:2] + CASES[3:]])
+def test_shared_projections_match_oracle_and_separate_copies(name, kw):
+    w = shared_workload(name, **kw)
+    X, (Wk, Wv, Wk_copy, Wv_copy), Q0, Wo, lengths = device_inputs(w)
+    Y_shared = fl.flarepp_mixer_fwd(X, Wk, Wv, Wk, Wv, Q0, lengths=lengths)       # same tensors: 2 projections
+    Y_copies = fl.flarepp_mixer_fwd(X, Wk, Wv, Wk_copy, Wv_copy, Q0, lengths=lengths)  # copies: 4 projections
+    out_shared = fl.flarepp_mixer_out_fwd(X, Wk, Wv, Wk, Wv, Q0, Wo, lengths=lengths)
+    torch.cuda.synchronize()
+    assert torch.equal(Y_shared.view(torch.int16), Y_copies.view(torch.int16))
+    ref = oracle.forward_workload(w)
+    check(host_f64(Y_shared), ref["Y"], f"shared Y {name}")
+    check(host_f64(out_shared), ref["Out"], f"shared Out {name}")

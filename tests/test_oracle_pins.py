@@ -318,3 +318,38 @@ def test_workloads_are_deterministic():
     assert not np.array_equal(a.X, c.X)
     m = make_workload("flarepp_masked_n4k", N=512, B=4)
     assert m.lengths.dtype == np.int32 and m.lengths.min() >= 128 and m.lengths.max() <= 512
+
+
+# --------------------------------------------------------------------------
+# head concatenation and output projection ("Full self-attention": the heads'
+# outputs side by side, times W_O; row-vector convention Out = Ycat @ W_O)
+# --------------------------------------------------------------------------
+
+def test_output_projection_closed_form(oracle_mod):
+    a, b = 0.75, -2.5
+    Y = np.array([[[[a]], [[b]]]])                  # B=1, H=2, N=1, D=1
+    Wo = np.array([[1.0, 2.0], [3.0, 4.0]])
+    out = oracle_mod.output_projection(Y, Wo)
+    assert out.shape == (1, 1, 2)
+    assert np.array_equal(out[0, 0], [a * 1.0 + b * 3.0, a * 2.0 + b * 4.0])
+
+
+def test_output_projection_identity_concatenates_heads_in_order(oracle_mod):
+    rng = np.random.default_rng(21)
+    B, H, N, D = 2, 3, 5, 4
+    Y = rng.standard_normal((B, H, N, D))
+    out = oracle_mod.output_projection(Y, np.eye(H * D))
+    for h in range(H):
+        assert np.array_equal(out[:, :, h * D:(h + 1) * D], Y[:, h])
+
+
+def test_output_projection_matches_torch_linear(oracle_mod):
+    rng = np.random.default_rng(22)
+    X, Ws, Q0 = rand_flarepp(rng, 2, 57, 32, 2, 5)
+    Wo = rng.standard_normal((32, 32)) / math.sqrt(32)
+    s = 1.0 / math.sqrt(16)
+    out = oracle_mod.flarepp_forward(X, *Ws, Q0, 2, None, s)
+    _, _, Y = torch_flarepp(X, Ws, Q0, 2, None, s)
+    Ycat = torch.from_numpy(Y).transpose(1, 2).reshape(2, 57, 32)
+    ref = F.linear(Ycat, torch.from_numpy(Wo).t()).numpy()
+    assert rel(oracle_mod.output_projection(out["Y"], Wo), ref) < 1e-12

@@ -10,7 +10,7 @@ bytes are copied to the GPU and widened to float64 for the oracle.
 
 Draw order for one workload (one ``numpy.random.Generator(PCG64(seed))``):
   FLARE++ : X (coordinates P, lift A, noise E for the mesh kinds), W_K, W_V,
-            W~_K, W~_V, Q0, lengths
+            W~_K, W~_V, Q0, lengths, W_O
   FLARE   : K, V, Q, lengths
 
 Rounding: every value is drawn in float32, then rounded to bf16 with
@@ -105,6 +105,7 @@ class Workload:
     Wk_syn: Optional[np.ndarray] = None
     Wv_syn: Optional[np.ndarray] = None
     Q0: Optional[np.ndarray] = None       # [H][M][D]
+    Wo: Optional[np.ndarray] = None       # [C][C] output projection
     # FLARE inputs (bf16 bits)
     K: Optional[np.ndarray] = None        # [B][H][N][D]
     V: Optional[np.ndarray] = None
@@ -177,4 +178,6 @@ def make_workload(name: str, N: Optional[int] = None, B: Optional[int] = None,
         if Nv != n0:  # reduced case: keep the same fraction of valid tokens
             lo, hi = max(1, lo * Nv // n0), max(1, hi * Nv // n0)
         w.lengths = rng.integers(lo, hi + 1, size=Bv, dtype=np.int64).astype(np.int32)
+    if spec["variant"] == "flarepp":  # drawn last, so the draws above do not depend on it
+        w.Wo = to_bf16_bits(rng.standard_normal((C, C), dtype=np.float32) * wstd)
     return w
