@@ -83,7 +83,9 @@ typedef enum {
   FLARE_ERR_ALIGN = 4,       /* a pointer is not 16-byte (workspace: 256) aligned */
   FLARE_ERR_WORKSPACE = 5,   /* workspace smaller than flare_workspace_bytes()    */
   FLARE_ERR_LAUNCH = 6,      /* CUDA error while enqueueing (no sm_100 device...) */
-  FLARE_ERR_TIMEOUT = 7      /* a device-side bounded wait expired                */
+  FLARE_ERR_TIMEOUT = 7,     /* a device-side bounded wait expired                */
+  FLARE_ERR_UNDERFLOW = 8    /* context parallelism: a merged row's sums underflowed
+                                and could not be recomputed exactly             */
 } flare_status;
 
 /* Variant selector for flare_workspace_bytes(). */
@@ -170,13 +172,60 @@ FLARE_API flare_status flarepp_mixer_fwd_profiled(const flare_bf16* X, const fla
 
 /*
  * Synchronises `stream`, reads the device error word of `workspace` and
- * returns FLARE_OK, FLARE_ERR_TIMEOUT or FLARE_ERR_SHAPE (invalid lengths).
+ * returns FLARE_OK, FLARE_ERR_TIMEOUT, FLARE_ERR_SHAPE (invalid lengths) or
+ * FLARE_ERR_UNDERFLOW (context-parallel merges only).
  * The word is cleared at the start of every mixer call.
  */
 FLARE_API flare_status flare_last_device_status(void* workspace, void* stream);
 
 /* Static, human-readable name of a status. */
 FLARE_API const char* flare_status_string(flare_status status);
+
+/*
+ * Context parallelism (section "Multi-GPU context parallelism", eq. 13-14).
+ *
+ * The tokens of every sequence are split into `world` shards of N tokens, one
+ * per rank: rank r holds tokens [r*N, (r+1)*N) of sequences of world*N tokens
+ * (X, K, V and Y are the shard's rows; `lengths`, if given, counts tokens of
+ * the whole sequence).  Each encoder pass produces per-split partial sums
+ * ("partials", flare_cp_partials_bytes() bytes per rank, fp32); the caller
+ * concatenates the partials of all ranks in rank order (an all-gather,
+ * [world][...]) and passes them to the next phase, which merges them with
+ * the log-sum-exp rule in a fixed order, so every rank holds bitwise the
+ * same Q(X) and Z.  The projections and the decoder only touch local rows.
+ *
+ *   FLARE++ : flarepp_cp_begin  -> all-gather -> flarepp_cp_middle
+ *             -> all-gather -> flarepp_cp_end
+ *   FLARE   : flare_cp_begin    -> all-gather -> flare_cp_end
+ *
+ * The phases of one rank share its workspace (flare_workspace_bytes of the
+ * same variant with the shard's N) and stream; the workspace carries the
+ * projections, Q(X) and Z from one phase to the next.  All ranks must call
+ * with the same sizes.  With world == 1 the result equals flare_mixer_fwd /
+ * flarepp_mixer_fwd.  A merged row whose sums underflowed (the case that
+ * flare_mixer_fwd recomputes exactly from all keys) is reported as
+ * FLARE_ERR_UNDERFLOW by flare_last_device_status when world > 1.
+ */
+FLARE_API size_t flare_cp_partials_bytes(int B, int H, int N, int M, int D);
+
+FLARE_API flare_status flarepp_cp_begin(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                                        const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0,
+                                        int B, int N, int C, int H, int M, int D, const int32_t* lengths, int rank,
+                                        int world, float scale, void* workspace, size_t workspace_bytes,
+                                        void* stream, float* partials);
+FLARE_API flare_status flarepp_cp_middle(const float* partials_all, int B, int N, int C, int H, int M, int D,
+                                         const int32_t* lengths, int rank, int world, float scale, void* workspace,
+                                         size_t workspace_bytes, void* stream, float* partials, float* Qx_out);
+FLARE_API flare_status flarepp_cp_end(const float* partials_all, flare_bf16* Y, int B, int N, int C, int H, int M,
+                                      int D, const int32_t* lengths, int rank, int world, float scale,
+                                      void* workspace, size_t workspace_bytes, void* stream, float* Z_out);
+FLARE_API flare_status flare_cp_begin(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, int B, int H,
+                                      int N, int M, int D, const int32_t* lengths, int rank, int world, float scale,
+                                      void* workspace, size_t workspace_bytes, void* stream, float* partials);
+FLARE_API flare_status flare_cp_end(const float* partials_all, const flare_bf16* K, const flare_bf16* Q,
+                                    flare_bf16* Y, int B, int H, int N, int M, int D, const int32_t* lengths,
+                                    int rank, int world, float scale, void* workspace, size_t workspace_bytes,
+                                    void* stream, float* Z_out);
 
 /*
  * FLARE mixer forward for callers that cannot allocate device memory.

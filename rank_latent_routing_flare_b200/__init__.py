@@ -23,3 +23,4 @@ from ._binding import (  # noqa: F401
     library_path,
     load_library,
 )
+from . import cp  # noqa: F401,E402  (context-parallel forward over torch.distributed)

@@ -26,6 +26,7 @@ class Status(enum.IntEnum):
     ERR_WORKSPACE = 5
     ERR_LAUNCH = 6
     ERR_TIMEOUT = 7
+    ERR_UNDERFLOW = 8
 
 
 class FlareError(RuntimeError):
@@ -60,6 +61,17 @@ def load_library(build_if_missing: bool = True):
         lib.flare_mixer_fwd_profiled.argtypes = lib.flare_mixer_fwd.argtypes + [vp]
         lib.flare_mixer_fwd_profiled.restype = i
         lib.flarepp_mixer_fwd_profiled.argtypes = lib.flarepp_mixer_fwd.argtypes + [vp]
+        lib.flare_cp_partials_bytes.restype = sz
+        lib.flare_cp_partials_bytes.argtypes = [i, i, i, i, i]
+        for name, args in (
+                ("flarepp_cp_begin", [vp] * 6 + [i] * 6 + [vp, i, i, f, vp, sz, vp, vp]),
+                ("flarepp_cp_middle", [vp] + [i] * 6 + [vp, i, i, f, vp, sz, vp, vp, vp]),
+                ("flarepp_cp_end", [vp, vp] + [i] * 6 + [vp, i, i, f, vp, sz, vp, vp]),
+                ("flare_cp_begin", [vp] * 3 + [i] * 5 + [vp, i, i, f, vp, sz, vp, vp]),
+                ("flare_cp_end", [vp] * 4 + [i] * 5 + [vp, i, i, f, vp, sz, vp, vp])):
+            fn = getattr(lib, name)
+            fn.restype = i
+            fn.argtypes = args
         lib.flarepp_mixer_out_fwd.restype = i
         lib.flarepp_mixer_out_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, f, vp, sz, vp]
         lib.flarepp_mixer_fwd_profiled.restype = i

@@ -162,10 +162,13 @@ flare_status check_common(int B, int H, int N, int M, int D) {
 
 float resolve_scale(float scale, int D) { return scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(D)); }
 
-// Encoder pass + merge: queries (bf16, [G][M][D]) against keys/values.
-flare_status run_encode(const Plan& pl, uint8_t* ws, const void* q, int q_per_batch, const void* k, const void* v,
-                        const float* knorm, float* out32, uint16_t* out16, int B, int H, int N, int M, int D,
-                        const int32_t* lengths, float scale, cudaStream_t st, void* const* ev, int ev0) {
+// Encoder pass: split partials of queries (bf16, [G][M][D]) against the keys
+// and values of one shard ([B*H][N][D]; tokens [tok_offset, tok_offset + N) of
+// sequences of n_global tokens) into part ([B*H][S][M][D+2] fp32).
+flare_status run_encode_partials(const Plan& pl, uint8_t* ws, const void* q, int q_per_batch, const void* k,
+                                 const void* v, const float* knorm, float* part, int B, int H, int N, int M, int D,
+                                 const int32_t* lengths, int tok_offset, int n_global, float scale, cudaStream_t st,
+                                 void* const* ev, int ev0) {
   const long BH = static_cast<long>(B) * H;
   const long G = q_per_batch ? BH : H;
   CUtensorMap tq, tk, tv;
@@ -177,33 +180,61 @@ flare_status run_encode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
   ep.q_per_batch = q_per_batch;
   ep.n_splits = pl.S; ep.tiles_per_split = pl.tps; ep.n_lblocks = pl.LB; ep.n_groups32 = pl.G32;
   ep.q_rows = std::min(M, kLatBlock);
+  ep.tok_offset = tok_offset; ep.n_global = n_global;
   ep.c = scale * 1.4426950408889634f;
   ep.lengths = lengths;
   ep.knorm = knorm;
   ep.q = static_cast<const uint16_t*>(q);
-  ep.part = reinterpret_cast<float*>(ws + pl.off_part);
+  ep.part = part;
   ep.err = reinterpret_cast<uint32_t*>(ws + pl.off_err);
   ep.timeout_ns = wait_timeout_ns();
   if (launch_encode(tq, tk, tv, ep, st) != cudaSuccess || !record(ev, ev0, st)) return FLARE_ERR_LAUNCH;
+  return FLARE_OK;
+}
+
+// Merge of the partials of R shards ([R][B*H][S][M][D+2], rank-major) into
+// out32/out16 ([B*H][M][D]).  With R == 1, q/k/v serve the exact
+// recomputation of rows whose sums underflowed.
+flare_status run_merge(const Plan& pl, uint8_t* ws, const float* part, int R, const void* q, int q_per_batch,
+                       const void* k, const void* v, float* out32, uint16_t* out16, int B, int H, int N, int M,
+                       int D, const int32_t* lengths, float scale, cudaStream_t st, void* const* ev, int ev_i,
+                       bool allow_exact = true) {
   MergeParams mp{};
   mp.B = B; mp.H = H; mp.N = N; mp.M = M; mp.D = D;
   mp.q_per_batch = q_per_batch;
   mp.n_splits = pl.S; mp.tiles_per_split = pl.tps;
-  mp.scale = scale; mp.c = ep.c;
+  mp.n_ranks = R;
+  mp.allow_exact = allow_exact ? 1 : 0;
+  mp.rank_stride = static_cast<size_t>(B) * H * pl.S * M * (D + 2);
+  mp.err = reinterpret_cast<uint32_t*>(ws + pl.off_err);
+  mp.scale = scale; mp.c = scale * 1.4426950408889634f;
   mp.lengths = lengths;
-  mp.part = ep.part;
-  mp.q = ep.q;
+  mp.part = part;
+  mp.q = static_cast<const uint16_t*>(q);
   mp.k = static_cast<const uint16_t*>(k);
   mp.v = static_cast<const uint16_t*>(v);
   mp.out_f32 = out32;
   mp.out_bf16 = out16;
-  if (launch_merge(mp, st) != cudaSuccess || !record(ev, ev0 + 1, st)) return FLARE_ERR_LAUNCH;
+  if (launch_merge(mp, st) != cudaSuccess || !record(ev, ev_i, st)) return FLARE_ERR_LAUNCH;
   return FLARE_OK;
+}
+
+// Encoder pass + merge on one GPU (the whole sequence).
+flare_status run_encode(const Plan& pl, uint8_t* ws, const void* q, int q_per_batch, const void* k, const void* v,
+                        const float* knorm, float* out32, uint16_t* out16, int B, int H, int N, int M, int D,
+                        const int32_t* lengths, float scale, cudaStream_t st, void* const* ev, int ev0) {
+  float* part = reinterpret_cast<float*>(ws + pl.off_part);
+  flare_status r = run_encode_partials(pl, ws, q, q_per_batch, k, v, knorm, part, B, H, N, M, D, lengths, 0, N,
+                                       scale, st, ev, ev0);
+  if (r != FLARE_OK) return r;
+  return run_merge(pl, ws, part, 1, q, q_per_batch, k, v, out32, out16, B, H, N, M, D, lengths, scale, st, ev,
+                   ev0 + 1);
 }
 
 flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_batch, const uint16_t* z16,
                         const void* k, void* y, int y_token_major, int B, int H, int N, int M, int D,
-                        const int32_t* lengths, float scale, cudaStream_t st) {
+                        const int32_t* lengths, float scale, cudaStream_t st, int tok_offset = 0,
+                        int n_global = -1) {
   const long BH = static_cast<long>(B) * H;
   const long G = q_per_batch ? BH : H;
   CUtensorMap tq, tz, tk;
@@ -223,6 +254,8 @@ flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
   dp.k = static_cast<const uint16_t*>(k);
   dp.y = static_cast<uint16_t*>(y);
   dp.y_token_major = y_token_major;
+  dp.tok_offset = tok_offset;
+  dp.n_global = n_global < 0 ? N : n_global;
   dp.err = reinterpret_cast<uint32_t*>(ws + pl.off_err);
   dp.fb_count = reinterpret_cast<uint32_t*>(ws + pl.off_err) + 1;
   dp.fb_list = reinterpret_cast<uint64_t*>(ws + pl.off_fb);
@@ -285,6 +318,8 @@ const char* flare_status_string(flare_status s) {
     case FLARE_ERR_WORKSPACE: return "FLARE_ERR_WORKSPACE: workspace too small";
     case FLARE_ERR_LAUNCH: return "FLARE_ERR_LAUNCH: CUDA error while enqueueing";
     case FLARE_ERR_TIMEOUT: return "FLARE_ERR_TIMEOUT: a device-side bounded wait expired";
+    case FLARE_ERR_UNDERFLOW:
+      return "FLARE_ERR_UNDERFLOW: a context-parallel merge found sums that underflowed (not recomputed)";
   }
   return "unknown flare_status";
 }
@@ -368,14 +403,17 @@ flare_status run_project(const Plan& pl, uint8_t* ws, const CUtensorMap& tx, con
   return launch_project(tx, tw, pp, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
 
-// The FLARE++ pipeline (eq. 7-11) after the argument checks.  Y is written
-// [B][H][N][D], or [B][N][C] when y_token_major.
-flare_status flarepp_run(const Plan& pl, const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
-                         const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0, void* Y,
-                         int y_token_major, int B, int N, int C, int H, int M, int D, const int32_t* lengths,
-                         float sc, uint8_t* ws, cudaStream_t s, float* Qx_out, float* Z_out,
-                         void* const* stage_events) {
-  if (cudaMemsetAsync(ws + pl.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+// Outputs of the FLARE++ projections in the workspace.
+struct Projected {
+  uint16_t *kt, *vt, *kk, *vv;
+  float *kn_syn, *kn;
+};
+
+// eq. 7 and eq. 9: the per-head projections of X (two when the synthesis
+// and encode weights are the same tensors, else four).
+flare_status flarepp_project(const Plan& pl, const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                             const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, int B, int N, int C, int H, int D,
+                             uint8_t* ws, cudaStream_t s, void* const* stage_events, Projected* pr) {
   // The same weights for synthesis and encode (the shared-projection
   // variant): K~ = K and V~ = V, so two projections serve both passes.
   const bool shared = Wk_syn == Wk && Wv_syn == Wv;
@@ -405,6 +443,23 @@ flare_status flarepp_run(const Plan& pl, const flare_bf16* X, const flare_bf16* 
   float* const norms[4] = {kn_syn, nullptr, kn, nullptr};
   flare_status st = run_project(pl, ws, tx, tw, shared ? 2 : 4, 0, outs, norms, B, N, C, H, D, s);
   if (st != FLARE_OK || !record(stage_events, 1, s)) return FLARE_ERR_LAUNCH;
+  *pr = Projected{kt, vt, kk, vv, kn_syn, kn};
+  return FLARE_OK;
+}
+
+// The FLARE++ pipeline (eq. 7-11) after the argument checks.  Y is written
+// [B][H][N][D], or [B][N][C] when y_token_major.
+flare_status flarepp_run(const Plan& pl, const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                         const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0, void* Y,
+                         int y_token_major, int B, int N, int C, int H, int M, int D, const int32_t* lengths,
+                         float sc, uint8_t* ws, cudaStream_t s, float* Qx_out, float* Z_out,
+                         void* const* stage_events) {
+  if (cudaMemsetAsync(ws + pl.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  Projected pr;
+  flare_status st = flarepp_project(pl, X, Wk, Wv, Wk_syn, Wv_syn, B, N, C, H, D, ws, s, stage_events, &pr);
+  if (st != FLARE_OK) return st;
+  uint16_t *kt = pr.kt, *vt = pr.vt, *kk = pr.kk, *vv = pr.vv;
+  float *kn_syn = pr.kn_syn, *kn = pr.kn;
 
   // eq. 8: query synthesis with the learned seeds
   float* qx32 = Qx_out ? Qx_out : reinterpret_cast<float*>(ws + pl.off_qx32);
@@ -481,6 +536,146 @@ flare_status flarepp_mixer_fwd(const flare_bf16* X, const flare_bf16* Wk, const 
                                     workspace_bytes, stream, Qx_out, Z_out, nullptr);
 }
 
+// ---------------------------------------------------------------------------
+// Context parallelism (eq. 13-14): phases of one rank over its token shard
+// ---------------------------------------------------------------------------
+
+size_t flare_cp_partials_bytes(int B, int H, int N, int M, int D) {
+  if (check_common(B, H, N, M, D) != FLARE_OK) return 0;
+  const Plan pl = make_plan(FLARE_VARIANT_FLARE, B, H, N, M, D);
+  return static_cast<size_t>(B) * H * pl.S * M * (D + 2) * sizeof(float);
+}
+
+}  // extern "C"
+
+namespace flare {
+namespace {
+
+flare_status check_cp(int N, int rank, int world, const void* part) {
+  if (!part) return FLARE_ERR_NULL;
+  if (world < 1 || rank < 0 || rank >= world) return FLARE_ERR_SHAPE;
+  if (static_cast<long>(N) * world >= (1L << 31)) return FLARE_ERR_UNSUPPORTED;
+  if (!aligned16(part)) return FLARE_ERR_ALIGN;
+  return FLARE_OK;
+}
+
+}  // namespace
+}  // namespace flare
+
+extern "C" {
+
+flare_status flarepp_cp_begin(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                              const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0, int B, int N,
+                              int C, int H, int M, int D, const int32_t* lengths, int rank, int world, float scale,
+                              void* workspace, size_t workspace_bytes, void* stream, float* partials) {
+  flare_status st = check_flarepp(X, Wk, Wv, Wk_syn, Wv_syn, Q0, X, B, N, C, H, M, D, lengths, workspace, nullptr,
+                                  nullptr);
+  if (st != FLARE_OK) return st;
+  if ((st = check_cp(N, rank, world, partials)) != FLARE_OK) return st;
+  const Plan pl = make_plan(FLARE_VARIANT_FLAREPP, B, H, N, M, D);
+  if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws + pl.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  Projected pr;
+  if ((st = flarepp_project(pl, X, Wk, Wv, Wk_syn, Wv_syn, B, N, C, H, D, ws, s, nullptr, &pr)) != FLARE_OK)
+    return st;
+  // eq. 8 on the local shard: the synthesis partials
+  return run_encode_partials(pl, ws, Q0, 0, pr.kt, pr.vt, pr.kn_syn, partials, B, H, N, M, D, lengths, rank * N,
+                             world * N, resolve_scale(scale, D), s, nullptr, 0);
+}
+
+flare_status flarepp_cp_middle(const float* partials_all, int B, int N, int C, int H, int M, int D,
+                               const int32_t* lengths, int rank, int world, float scale, void* workspace,
+                               size_t workspace_bytes, void* stream, float* partials, float* Qx_out) {
+  if (!partials_all || !workspace) return FLARE_ERR_NULL;
+  flare_status st = check_common(B, H, N, M, D);
+  if (st != FLARE_OK) return st;
+  if (C != H * D || C % 64 != 0 || C > 256) return C != H * D ? FLARE_ERR_SHAPE : FLARE_ERR_UNSUPPORTED;
+  if ((st = check_cp(N, rank, world, partials)) != FLARE_OK) return st;
+  if (!aligned16(partials_all) || !aligned16(lengths) || !aligned16(Qx_out)) return FLARE_ERR_ALIGN;
+  const Plan pl = make_plan(FLARE_VARIANT_FLAREPP, B, H, N, M, D);
+  if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const float sc = resolve_scale(scale, D);
+  float* qx32 = Qx_out ? Qx_out : reinterpret_cast<float*>(ws + pl.off_qx32);
+  uint16_t* qx16 = reinterpret_cast<uint16_t*>(ws + pl.off_qx16);
+  // Q(X): every rank merges the same partials in the same order
+  st = run_merge(pl, ws, partials_all, world, nullptr, 0, nullptr, nullptr, qx32, qx16, B, H, N, M, D, lengths, sc, s,
+                 nullptr, 0, false);
+  if (st != FLARE_OK) return st;
+  // eq. 10 on the local shard: the encode partials
+  return run_encode_partials(pl, ws, qx16, 1, ws + pl.off_kp, ws + pl.off_vp, reinterpret_cast<float*>(ws + pl.off_kn),
+                             partials, B, H, N, M, D, lengths, rank * N, world * N, sc, s, nullptr, 0);
+}
+
+flare_status flarepp_cp_end(const float* partials_all, flare_bf16* Y, int B, int N, int C, int H, int M, int D,
+                            const int32_t* lengths, int rank, int world, float scale, void* workspace,
+                            size_t workspace_bytes, void* stream, float* Z_out) {
+  if (!partials_all || !Y || !workspace) return FLARE_ERR_NULL;
+  flare_status st = check_common(B, H, N, M, D);
+  if (st != FLARE_OK) return st;
+  if (C != H * D || C % 64 != 0 || C > 256) return C != H * D ? FLARE_ERR_SHAPE : FLARE_ERR_UNSUPPORTED;
+  if ((st = check_cp(N, rank, world, partials_all)) != FLARE_OK) return st;
+  if (!aligned16(Y) || !aligned16(lengths) || !aligned16(Z_out)) return FLARE_ERR_ALIGN;
+  const Plan pl = make_plan(FLARE_VARIANT_FLAREPP, B, H, N, M, D);
+  if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const float sc = resolve_scale(scale, D);
+  float* z32 = Z_out ? Z_out : reinterpret_cast<float*>(ws + pl.off_z32);
+  uint16_t* z16 = reinterpret_cast<uint16_t*>(ws + pl.off_z16);
+  st = run_merge(pl, ws, partials_all, world, nullptr, 0, nullptr, nullptr, z32, z16, B, H, N, M, D, lengths, sc, s,
+                 nullptr, 0, false);
+  if (st != FLARE_OK) return st;
+  // eq. 11 on the local shard
+  return run_decode(pl, ws, ws + pl.off_qx16, 1, z16, ws + pl.off_kp, Y, 0, B, H, N, M, D, lengths, sc, s, rank * N,
+                    world * N);
+}
+
+flare_status flare_cp_begin(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, int B, int H, int N, int M,
+                            int D, const int32_t* lengths, int rank, int world, float scale, void* workspace,
+                            size_t workspace_bytes, void* stream, float* partials) {
+  if (!K || !V || !Q || !workspace) return FLARE_ERR_NULL;
+  flare_status st = check_common(B, H, N, M, D);
+  if (st != FLARE_OK) return st;
+  if ((st = check_cp(N, rank, world, partials)) != FLARE_OK) return st;
+  if (!aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(lengths) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FLARE_ERR_ALIGN;
+  const Plan pl = make_plan(FLARE_VARIANT_FLARE, B, H, N, M, D);
+  if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws + pl.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  KnormParams kp{B * H, N, D, pl.G32, reinterpret_cast<const uint16_t*>(K), reinterpret_cast<float*>(ws + pl.off_kn)};
+  if (launch_knorm(kp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  return run_encode_partials(pl, ws, Q, 0, K, V, kp.knorm, partials, B, H, N, M, D, lengths, rank * N, world * N,
+                             resolve_scale(scale, D), s, nullptr, 0);
+}
+
+flare_status flare_cp_end(const float* partials_all, const flare_bf16* K, const flare_bf16* Q, flare_bf16* Y, int B,
+                          int H, int N, int M, int D, const int32_t* lengths, int rank, int world, float scale,
+                          void* workspace, size_t workspace_bytes, void* stream, float* Z_out) {
+  if (!partials_all || !K || !Q || !Y || !workspace) return FLARE_ERR_NULL;
+  flare_status st = check_common(B, H, N, M, D);
+  if (st != FLARE_OK) return st;
+  if ((st = check_cp(N, rank, world, partials_all)) != FLARE_OK) return st;
+  if (!aligned16(K) || !aligned16(Q) || !aligned16(Y) || !aligned16(lengths) || !aligned16(Z_out)) return FLARE_ERR_ALIGN;
+  const Plan pl = make_plan(FLARE_VARIANT_FLARE, B, H, N, M, D);
+  if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const float sc = resolve_scale(scale, D);
+  float* z32 = Z_out ? Z_out : reinterpret_cast<float*>(ws + pl.off_z32);
+  uint16_t* z16 = reinterpret_cast<uint16_t*>(ws + pl.off_z16);
+  st = run_merge(pl, ws, partials_all, world, nullptr, 0, nullptr, nullptr, z32, z16, B, H, N, M, D, lengths, sc, s,
+                 nullptr, 0, false);
+  if (st != FLARE_OK) return st;
+  return run_decode(pl, ws, Q, 0, z16, K, Y, 0, B, H, N, M, D, lengths, sc, s, rank * N, world * N);
+}
+
 flare_status flare_mixer_fwd_static(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, flare_bf16* Y,
                                     int B, int H, int N, int M, int D, const int32_t* lengths, float scale,
                                     void* stream, float* Z_out) {
@@ -507,6 +702,7 @@ flare_status flare_last_device_status(void* workspace, void* stream) {
   if (cudaMemcpy(&word, workspace, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return FLARE_ERR_LAUNCH;
   if (word & FLARE_DEV_TIMEOUT) return FLARE_ERR_TIMEOUT;
   if (word & FLARE_DEV_BAD_LENGTH) return FLARE_ERR_SHAPE;
+  if (word & FLARE_DEV_UNDERFLOW) return FLARE_ERR_UNDERFLOW;
   return FLARE_OK;
 }
 

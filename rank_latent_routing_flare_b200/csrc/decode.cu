@@ -166,15 +166,9 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
   const int part = blockIdx.x % p.ctas_per_head;
   const int b = bh / p.H, h = bh % p.H;
   const int g = p.q_per_batch ? bh : h;
-  int L = p.N;
-  if (p.lengths) {
-    int l = p.lengths[b];
-    if (l < 1 || l > p.N) {
-      if (threadIdx.x == 0) atomicOr(p.err, FLARE_DEV_BAD_LENGTH);
-      l = min(max(l, 0), p.N);
-    }
-    L = l;
-  }
+  bool bad_len = false;
+  const int L = shard_valid_len(p.lengths, b, p.N, p.tok_offset, p.n_global, &bad_len);
+  if (bad_len && threadIdx.x == 0) atomicOr(p.err, FLARE_DEV_BAD_LENGTH);
   const int tiles_head = (p.N + kDecTile - 1) / kDecTile;
   const int tiles_valid = (L + kDecTile - 1) / kDecTile;
   const int ta = part * p.tiles_per_cta;

@@ -94,15 +94,9 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
   const int s = (blockIdx.x / LB) % S;
   const int bh = blockIdx.x / (LB * S);
   const int b = bh / p.H, h = bh % p.H;
-  int L = p.N;
-  if (p.lengths) {
-    int l = p.lengths[b];
-    if (l < 1 || l > p.N) {
-      if (threadIdx.x == 0) atomicOr(p.err, FLARE_DEV_BAD_LENGTH);
-      l = min(max(l, 0), p.N);
-    }
-    L = l;
-  }
+  bool bad_len = false;
+  const int L = shard_valid_len(p.lengths, b, p.N, p.tok_offset, p.n_global, &bad_len);
+  if (bad_len && threadIdx.x == 0) atomicOr(p.err, FLARE_DEV_BAD_LENGTH);
   const int ntiles_valid = (L + T - 1) / T;
   const int t0 = s * p.tiles_per_split;
   const int t1 = min(t0 + p.tiles_per_split, ntiles_valid);

@@ -8,8 +8,25 @@
 // Device error word bits (first 4 bytes of the workspace).
 #define FLARE_DEV_TIMEOUT 0x1u
 #define FLARE_DEV_BAD_LENGTH 0x2u
+#define FLARE_DEV_UNDERFLOW 0x4u   // a merged row lost mass and could not be recomputed exactly
 
 namespace flare {
+
+// Valid tokens of sequence b within one shard: `lengths` (NULL = all valid)
+// counts tokens of the whole sequence of n_global tokens, and the shard holds
+// tokens [tok_offset, tok_offset + N).  A length outside [1, n_global] is
+// clamped; *bad is set.
+__host__ __device__ inline int shard_valid_len(const int32_t* lengths, int b, int N, int tok_offset, int n_global,
+                                               bool* bad) {
+  if (lengths == nullptr) return N;
+  int l = lengths[b];
+  if (l < 1 || l > n_global) {
+    *bad = true;
+    l = l < 0 ? 0 : (l > n_global ? n_global : l);
+  }
+  l -= tok_offset;
+  return l < 0 ? 0 : (l > N ? N : l);
+}
 
 constexpr int kNumSM = 148;        // B200
 constexpr int kLatBlock = 128;     // latents per encode CTA (UMMA M)
@@ -48,7 +65,8 @@ __host__ __device__ constexpr int dec_ctas_per_sm(int D) { return D == 16 ? FLAR
 #ifndef FLARE_ENC_SPLIT_LD
 #define FLARE_ENC_SPLIT_LD 1
 #endif
-// Heads whose projection outputs are read from TMEM per wait.
+// Heads (D = 16; half as many for D = 32) whose projection outputs are read
+// from TMEM per wait.
 #ifndef FLARE_PROJ_EPI_HEADS
 #define FLARE_PROJ_EPI_HEADS 4
 #endif
@@ -93,6 +111,8 @@ struct EncodeParams {
   int n_lblocks;        // ceil(M / kLatBlock)
   int n_groups32;
   int q_rows;           // rows of one query box: min(M, kLatBlock)
+  int tok_offset;       // first token of this shard (context parallelism; else 0)
+  int n_global;         // tokens of the whole sequence (else N)
   float c;              // scale * log2(e)
   const int32_t* lengths;
   const float* knorm;   // [B*H][n_groups32]
@@ -106,9 +126,13 @@ struct EncodeParams {
 // Merge of the split partials (log-sum-exp combine) + exact fallback rows
 // ---------------------------------------------------------------------------
 struct MergeParams {
-  int B, H, N, M, D;
+  int B, H, N, M, D;    // N: tokens of one shard (of the sequence without context parallelism)
   int q_per_batch;
   int n_splits, tiles_per_split;
+  int n_ranks;          // shards whose partials are merged (1 without context parallelism)
+  int allow_exact;      // rows whose sums underflowed: recompute from q, k, v (1) or report (0)
+  size_t rank_stride;   // floats between the partials of consecutive shards
+  uint32_t* err;
   float scale, c;
   const int32_t* lengths;
   const float* part;
@@ -126,6 +150,8 @@ struct DecodeParams {
   int B, H, N, M, D;
   int q_per_batch;
   int tiles_per_cta;    // in kDecTile tiles
+  int tok_offset;       // first token of this shard (context parallelism; else 0)
+  int n_global;         // tokens of the whole sequence (else N)
   int ctas_per_head;
   int qz_box_rows;      // rows of one Q/Z box: min(M, 256)
   float scale, c;

@@ -61,37 +61,48 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
   if (row >= p.B * p.H * p.M) return;
   const int bh = row / p.M, m = row % p.M;
   const int b = bh / p.H, h = bh % p.H;
-  int L = p.N;
-  if (p.lengths) L = min(max(p.lengths[b], 0), p.N);
-  const int ntv = (L + enc_tile(D) - 1) / enc_tile(D);
-  const int S = p.n_splits;
+  const int S = p.n_splits, R = p.n_ranks;
   const size_t stride = static_cast<size_t>(p.M) * (D + 2);
-  const float* base = p.part + static_cast<size_t>(bh) * S * stride + static_cast<size_t>(m) * (D + 2);
-
-  // log2 of the total weight: G = max_s (U_s + log2 l_s); bound of the mass
-  // lost to flushed exponentials: sum_s n_s 2^(U_s - 126).  Lanes take the
-  // splits s = lane, lane + 32, ...; the butterfly reductions below have a
-  // fixed order, so the result is bitwise reproducible.
-  float G = -INFINITY, lost = -INFINITY;
-  for (int s = lane; s < S; s += 32) {
+  // partials of split s of shard r: (U, l, O[D]) of this row
+  auto part_of = [&](int r, int s) {
+    return p.part + r * p.rank_stride + (static_cast<size_t>(bh) * S + s) * stride + static_cast<size_t>(m) * (D + 2);
+  };
+  // token tiles of split s of shard r that hold valid tokens
+  bool bad = false;
+  auto split_tiles = [&](int r, int s) {
+    const int Lr = shard_valid_len(p.lengths, b, p.N, r * p.N, R * p.N, &bad);
+    const int ntv = (Lr + enc_tile(D) - 1) / enc_tile(D);
     const int t0 = s * p.tiles_per_split, t1 = min(t0 + p.tiles_per_split, ntv);
-    if (t1 <= t0) continue;
-    const float2 ul = *reinterpret_cast<const float2*>(base + s * stride);
+    return max(0, t1 - t0);
+  };
+
+  // log2 of the total weight: G = max (U + log2 l) over all splits of all
+  // shards; bound of the mass lost to flushed exponentials: sum n 2^(U - 126).
+  // Lanes take the splits j = lane, lane + 32, ... (j = r * S + s); the
+  // butterfly reductions below have a fixed order, so the result is bitwise
+  // reproducible.
+  float G = -INFINITY, lost = -INFINITY;
+  for (int j = lane; j < R * S; j += 32) {
+    const int r = j / S, s = j - r * S;
+    const int nt = split_tiles(r, s);
+    if (nt == 0) continue;
+    const float2 ul = *reinterpret_cast<const float2*>(part_of(r, s));
     if (ul.y > 0.f) G = fmaxf(G, ul.x + log2f(ul.y));
-    lost = fmaxf(lost, ul.x - 126.f + log2f(static_cast<float>((t1 - t0) * enc_tile(D))));
+    lost = fmaxf(lost, ul.x - 126.f + log2f(static_cast<float>(nt * enc_tile(D))));
   }
   G = warp_max(G);
   lost = warp_max(lost);
-  const bool exact = !(G > -INFINITY) || (lost + log2f(static_cast<float>(S)) - G > -27.f);
+  const bool exact = !(G > -INFINITY) || (lost + log2f(static_cast<float>(R * S)) - G > -27.f);
   float z = 0.f;
-  if (!exact) {
+  const bool can_exact = R == 1 && p.allow_exact;
+  if ((!exact || !can_exact) && G > -INFINITY) {
     float num[D], den = 0.f;
 #pragma unroll
     for (int d = 0; d < D; ++d) num[d] = 0.f;
-    for (int s = lane; s < S; s += 32) {
-      const int t0 = s * p.tiles_per_split, t1 = min(t0 + p.tiles_per_split, ntv);
-      if (t1 <= t0) continue;
-      const float* e = base + s * stride;  // (U, l, O[D]), 8-byte aligned
+    for (int j = lane; j < R * S; j += 32) {
+      const int r = j / S, s = j - r * S;
+      if (split_tiles(r, s) == 0) continue;
+      const float* e = part_of(r, s);  // (U, l, O[D]), 8-byte aligned
       const float2 ul = *reinterpret_cast<const float2*>(e);
       if (!(ul.y > 0.f)) continue;
       const float w = exp2f(ul.x - G);
@@ -111,8 +122,12 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
       if (d == lane) mine = t;
     }
     z = mine / den;
-  } else {
+    // with several shards the keys and values of the others are not at hand:
+    // a row that would need the exact recomputation is reported instead
+    if (exact && lane == 0) atomicOr(p.err, FLARE_DEV_UNDERFLOW);
+  } else if (can_exact) {
     const int g = p.q_per_batch ? bh : h;
+    const int L = shard_valid_len(p.lengths, b, p.N, 0, p.N, &bad);
     z = merge_exact_row<D>(p, p.q + (static_cast<size_t>(g) * p.M + m) * D, p.k + static_cast<size_t>(bh) * p.N * D,
                            p.v + static_cast<size_t>(bh) * p.N * D, L, lane);
   }

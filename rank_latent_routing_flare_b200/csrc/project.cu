@@ -164,8 +164,8 @@ __global__ void __launch_bounds__(192, 1)
       const int n = n0 + r;
       if (!mbar_wait_warp(acc_full + ab, (i >> 1) & 1, wc)) break;
       tc_fence_after();
-      // G heads per TMEM read (one wait per G heads)
-      constexpr int G = FLARE_PROJ_EPI_HEADS;
+      // G heads per TMEM read (one wait per G heads; G * D columns)
+      constexpr int G = D == 16 ? FLARE_PROJ_EPI_HEADS : (FLARE_PROJ_EPI_HEADS + 1) / 2;
       for (int h0 = 0; h0 < H; h0 += G) {
         uint32_t v[G][D];
 #pragma unroll

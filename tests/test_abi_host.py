@@ -32,7 +32,8 @@ def test_header_declares_the_abi():
     assert names == sorted(["flare_workspace_bytes", "flare_mixer_fwd", "flarepp_mixer_fwd", "flarepp_mixer_out_fwd",
                             "flare_mixer_fwd_profiled", "flarepp_mixer_fwd_profiled", "flare_mixer_fwd_static",
                             "flare_last_device_status", "flare_status_string",
-                            "flare_selftest_wait_timeout"])
+                            "flare_selftest_wait_timeout", "flare_cp_partials_bytes", "flarepp_cp_begin",
+                            "flarepp_cp_middle", "flarepp_cp_end", "flare_cp_begin", "flare_cp_end"])
 
 
 def test_library_loads_and_exports_every_declared_symbol():
@@ -179,3 +180,23 @@ def test_static_scratch_entry_point_rejects_oversized_problems():
     assert st == Status.ERR_WORKSPACE
     assert lib.flare_mixer_fwd_static(None, A, A, A, 1, 1, 64, 16, 16, None, 0.0, None, None) == Status.ERR_NULL
     assert lib.flare_mixer_fwd_static(A, A, A, A + 2, 1, 1, 64, 16, 16, None, 0.0, None, None) == Status.ERR_ALIGN
+
+
+def test_context_parallel_argument_errors():
+    lib = fl.load_library()
+    assert lib.flare_cp_partials_bytes(1, 2, 100, 32, 16) > 0
+    assert lib.flare_cp_partials_bytes(1, 2, 100, 40, 16) == 0                 # M not a multiple of 16
+    args = (1, 100, 64, 4, 32, 16, None)
+    ws = fl.flare_workspace_bytes(1, 1, 4, 100, 32, 16, 64)
+    # rank outside [0, world), missing partials, unaligned partials
+    assert lib.flarepp_cp_begin(A, A, A, A, A, A, *args, 2, 2, 0.0, W, ws, None, A) == Status.ERR_SHAPE
+    assert lib.flarepp_cp_begin(A, A, A, A, A, A, *args, 0, 1, 0.0, W, ws, None, None) == Status.ERR_NULL
+    assert lib.flarepp_cp_begin(A, A, A, A, A, A, *args, 0, 1, 0.0, W, ws, None, A + 4) == Status.ERR_ALIGN
+    assert lib.flarepp_cp_begin(A, A, A, A, A, A, *args, 0, 1, 0.0, W, ws - 256, None, A) == Status.ERR_WORKSPACE
+    assert lib.flarepp_cp_middle(A, *args, 0, 0, 0.0, W, ws, None, A, None) == Status.ERR_SHAPE   # world 0
+    assert lib.flarepp_cp_end(None, A, *args, 0, 1, 0.0, W, ws, None, None) == Status.ERR_NULL
+    fargs = (1, 2, 100, 32, 16, None)
+    fws = fl.flare_workspace_bytes(0, 1, 2, 100, 32, 16)
+    assert lib.flare_cp_begin(A, A, A, *fargs, -1, 2, 0.0, W, fws, None, A) == Status.ERR_SHAPE
+    assert lib.flare_cp_end(A, A, A, None, *fargs, 0, 2, 0.0, W, fws, None, None) == Status.ERR_NULL
+    assert fl.flare_status_string(8).startswith("FLARE_ERR_UNDERFLOW")
