@@ -15,43 +15,49 @@ namespace flare {
 namespace {
 
 // Exact encoder row: z = sum_n softmax_n(<q, k_n> * scale) v_n over n < L,
-// fp32, two passes, lanes stride over tokens, fixed butterfly reductions.
+// fp32, two passes.  lane = (group, d): the 32 / D groups take the tokens
+// n = group, group + 32 / D, ...; a dot product is a butterfly over the D
+// lanes of a group.  Every reduction has a fixed order.  Returns z[d] of this
+// lane's d.
 template <int D>
 __device__ float merge_exact_row(const MergeParams& p, const uint16_t* qrow, const uint16_t* kh,
                                  const uint16_t* vh, int L, int lane) {
   if (L <= 0) return 0.f;
-  float q[D];
+  constexpr int NG = 32 / D;
+  const int d = lane % D, grp = lane / D;
+  const float qd = __uint_as_float(static_cast<uint32_t>(qrow[d]) << 16);
+  auto score = [&](int n) {  // <q, k_n> * c, the same in every lane of the group
+    float t = qd * __uint_as_float(static_cast<uint32_t>(kh[static_cast<size_t>(n) * D + d]) << 16);
 #pragma unroll
-  for (int d = 0; d < D; ++d) q[d] = __uint_as_float(static_cast<uint32_t>(qrow[d]) << 16);
+    for (int o = 1; o < D; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    return t * p.c;
+  };
+  // every lane of the warp runs the same number of iterations (the shuffles
+  // need the whole warp); tokens past L are skipped arithmetically
+  const int iters = (L + NG - 1) / NG;
   float mx = -INFINITY;
-  for (int n = lane; n < L; n += 32) {
-    float s = 0.f;
-#pragma unroll
-    for (int d = 0; d < D; ++d) s = fmaf(q[d], __uint_as_float(static_cast<uint32_t>(kh[static_cast<size_t>(n) * D + d]) << 16), s);
-    mx = fmaxf(mx, s * p.c);
+  for (int it = 0; it < iters; ++it) {
+    const int n = it * NG + grp;
+    const float sc = score(min(n, L - 1));
+    if (n < L) mx = fmaxf(mx, sc);
   }
   mx = warp_max(mx);
-  float acc[D];
-#pragma unroll
-  for (int d = 0; d < D; ++d) acc[d] = 0.f;
-  float den = 0.f;
-  for (int n = lane; n < L; n += 32) {
-    float s = 0.f;
-#pragma unroll
-    for (int d = 0; d < D; ++d) s = fmaf(q[d], __uint_as_float(static_cast<uint32_t>(kh[static_cast<size_t>(n) * D + d]) << 16), s);
-    const float e = exp2f(s * p.c - mx);
-    den += e;
-#pragma unroll
-    for (int d = 0; d < D; ++d) acc[d] = fmaf(e, __uint_as_float(static_cast<uint32_t>(vh[static_cast<size_t>(n) * D + d]) << 16), acc[d]);
+  float acc = 0.f, den = 0.f;
+  for (int it = 0; it < iters; ++it) {
+    const int n = it * NG + grp;
+    const float sc = score(min(n, L - 1));
+    if (n < L) {
+      const float e = exp2f(sc - mx);
+      den += e;
+      acc = fmaf(e, __uint_as_float(static_cast<uint32_t>(vh[static_cast<size_t>(n) * D + d]) << 16), acc);
+    }
   }
-  den = warp_sum(den);
-  float mine = 0.f;
 #pragma unroll
-  for (int d = 0; d < D; ++d) {
-    const float t = warp_sum(acc[d]);
-    if (d == lane) mine = t;
+  for (int o = D; o < 32; o <<= 1) {
+    acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    den += __shfl_xor_sync(0xffffffffu, den, o);
   }
-  return mine / den;
+  return acc / den;
 }
 
 template <int D>
@@ -96,32 +102,29 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
   float z = 0.f;
   const bool can_exact = R == 1 && p.allow_exact;
   if ((!exact || !can_exact) && G > -INFINITY) {
-    float num[D], den = 0.f;
-#pragma unroll
-    for (int d = 0; d < D; ++d) num[d] = 0.f;
-    for (int j = lane; j < R * S; j += 32) {
+    // lane = (group, d): the 32 / D groups take the splits j = group,
+    // group + 32 / D, ... in ascending order; one value of d per lane keeps
+    // the registers (and so the occupancy) independent of D
+    constexpr int NG = 32 / D;
+    const int d = lane % D, grp = lane / D;
+    float num = 0.f, den = 0.f;
+#pragma unroll 4
+    for (int j = grp; j < R * S; j += NG) {
       const int r = j / S, s = j - r * S;
       if (split_tiles(r, s) == 0) continue;
-      const float* e = part_of(r, s);  // (U, l, O[D]), 8-byte aligned
+      const float* e = part_of(r, s);  // (U, l, O[D])
       const float2 ul = *reinterpret_cast<const float2*>(e);
       if (!(ul.y > 0.f)) continue;
       const float w = exp2f(ul.x - G);
       den = fmaf(w, ul.y, den);
-#pragma unroll
-      for (int d = 0; d < D; d += 2) {
-        const float2 o = *reinterpret_cast<const float2*>(e + 2 + d);
-        num[d] = fmaf(w, o.x, num[d]);
-        num[d + 1] = fmaf(w, o.y, num[d + 1]);
-      }
+      num = fmaf(w, e[2 + d], num);
     }
-    den = warp_sum(den);
-    float mine = 0.f;
 #pragma unroll
-    for (int d = 0; d < D; ++d) {
-      const float t = warp_sum(num[d]);
-      if (d == lane) mine = t;
+    for (int o = D; o < 32; o <<= 1) {  // combine the groups (commutative adds: same bits in every lane)
+      num += __shfl_xor_sync(0xffffffffu, num, o);
+      den += __shfl_xor_sync(0xffffffffu, den, o);
     }
-    z = mine / den;
+    z = num / den;
     // with several shards the keys and values of the others are not at hand:
     // a row that would need the exact recomputation is reported instead
     if (exact && lane == 0) atomicOr(p.err, FLARE_DEV_UNDERFLOW);
