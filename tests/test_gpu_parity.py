@@ -93,6 +93,8 @@ def test_zero_queries_give_token_means(D):
     (3, 2, 200, 144, 32),      # a 16-row partial latent block and decode chunk
     (1, 1, 1, 16, 16),         # one token, smallest M
     (1, 1, 65, 48, 16),        # one full tile + 1 token; 48-latent chunk
+    (1, 2, 777, 512, 32),      # D = 32 with the largest M: eight 64-latent decoder chunks
+    (2, 3, 130, 80, 32),       # D = 32, a short last decoder chunk (16 latents)
 ])
 def test_flare_parity(B, H, N, M, D):
     w = flare_case(B, H, N, M, D, seed=B * 1000 + N)
