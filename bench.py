@@ -416,7 +416,7 @@ def main():
         roof = {"kernel": "merge_kernel", "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": None, "traffic": None}
     roof["peak_source"] = peaks["source"]
-    # whole-step roofline of the benchmark spec: max(bytes/HBM, MMA/tensor, exps/MUFU)
+    # whole-step roofline: max(bytes / HBM peak, MMA flops / tensor peak, exps / MUFU peak)
     tot_bytes = 3 * w.B * w.N * w.C * 2 + w.B * w.H * w.N * w.D * 2
     tot_exps = sum(work[s]["exps"] for s in STAGES_PP)
     tot_flops = sum(work[s]["flops"] for s in STAGES_PP)
