@@ -18,6 +18,12 @@
 namespace flare {
 namespace {
 
+// Largest value of a non-negative float across the warp: for v >= 0 the
+// bit patterns order like the values, so one integer max reduction does it.
+__device__ __forceinline__ float warp_max_nonneg(float v) {
+  return __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(v)));
+}
+
 template <int C>
 struct ProjCfg {
   static constexpr int KC = C / 64;                   // 64-wide K chunks
@@ -195,7 +201,7 @@ __global__ void __launch_bounds__(192, 1)
             nrm = 0.f;
           }
           if (knorm != nullptr) {
-            const float gm = warp_max(sqrtf(nrm));
+            const float gm = warp_max_nonneg(sqrtf(nrm));
             const int gi = n0 / kNormGroup + wq;
             if (lane == 0 && gi < p.n_groups32)
               knorm[(static_cast<size_t>(b) * H + hh) * p.n_groups32 + gi] = gm;
