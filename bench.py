@@ -304,6 +304,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="time replays of one step captured as a CUDA graph (no per-launch host cost); the "
+                         "stage times then come from as many eager steps run after the timed region")
     args = ap.parse_args()
     if args.warmup < 3:
         log("warm-up raised to the minimum of 3 steps")
@@ -343,8 +346,8 @@ def main():
     stream = torch.cuda.current_stream(dev)
     stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
 
-    def step(events=None):
-        fl.flarepp_mixer_fwd(X, *Ws, Q0, lengths=lengths, Y=Y, workspace=ws, stream=stream, check=False,
+    def step(events=None, st=None):
+        fl.flarepp_mixer_fwd(X, *Ws, Q0, lengths=lengths, Y=Y, workspace=ws, stream=st or stream, check=False,
                              stage_events=events)
 
     for _ in range(args.warmup):
@@ -354,6 +357,18 @@ def main():
     if st != fl.Status.OK:
         raise RuntimeError(f"device status after warm-up: {st!r}")
 
+    graph = None
+    if args.graph:  # one step captured once and replayed
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.graph(graph, stream=cap):
+            step(None, st=cap)
+        stream.wait_stream(cap)
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize(dev)
+
     # ---------------- timed region (inputs resident in HBM) ----------------
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clocks:
@@ -362,7 +377,10 @@ def main():
         torch.cuda.synchronize(dev)
         ev0.record(stream)
         for i in range(args.steps):
-            step(stage_ev[i])
+            if graph is not None:
+                graph.replay()
+            else:
+                step(stage_ev[i])
         ev1.record(stream)
         torch.cuda.synchronize(dev)
         if world > 1:
@@ -371,7 +389,11 @@ def main():
     th_per_rank = w.B * w.H * (w.valid_tokens() // w.B if w.lengths is not None else w.N)
     value = whole_job_rate(world, th_per_rank, ms)
 
-    # per-stage device times (same timed steps, same stream)
+    # per-stage device times (the timed steps; with --graph, eager steps after them)
+    if graph is not None:
+        for i in range(args.steps):
+            step(stage_ev[i])
+        torch.cuda.synchronize(dev)
     stage_ms = {s: 0.0 for s in STAGES_PP}
     for evs in stage_ev:
         for j, s in enumerate(STAGES_PP):
@@ -503,6 +525,7 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "N": w.N, "C": w.C, "H": w.H, "D": w.D, "M": w.M,
                        "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "launch": "cuda_graph" if args.graph else "eager",
                        "l2": "inputs larger than L2 (X 256 MiB; K~,V~,K,V 1 GiB per step)"},
             "roofline": roof,
             "step_roofline": step_roofline,
@@ -513,6 +536,7 @@ def main():
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": clk,
         }
+    del graph
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
