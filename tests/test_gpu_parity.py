@@ -204,3 +204,35 @@ def test_deterministic_bits():
     b = run_gpu(w)
     assert np.array_equal(a["Y"], b["Y"])
     assert np.array_equal(a["Qx"], b["Qx"]) and np.array_equal(a["Z"], b["Z"])
+
+
+def test_cuda_graph_capture_replays_the_same_bits():
+    """A whole FLARE++ call can be captured into a CUDA graph (it only enqueues
+    kernels and a memset on the given stream) and replayed with new inputs."""
+    w = make_workload("flarepp_n8k_mesh2d", N=2048, B=2)
+    X = dev_bf16(w.X)
+    Ws = [dev_bf16(a) for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn)]
+    Q0 = dev_bf16(w.Q0)
+    nbytes = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLAREPP, w.B, w.H, w.N, w.M, w.D, w.C)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    Y = torch.empty((w.B, w.H, w.N, w.D), dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        fl.flarepp_mixer_fwd(X, *Ws, Q0, Y=Y, workspace=ws)   # first call outside the capture
+        torch.cuda.synchronize()
+        eager = Y.clone()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            fl.flarepp_mixer_fwd(X, *Ws, Q0, Y=Y, workspace=ws, check=False)
+    Y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(Y.view(torch.int16), eager.view(torch.int16))
+    # new inputs in the same buffers
+    w2 = make_workload("flarepp_n8k_mesh2d", N=2048, B=2, seed=77)
+    w2.Wk, w2.Wv, w2.Wk_syn, w2.Wv_syn, w2.Q0 = w.Wk, w.Wv, w.Wk_syn, w.Wv_syn, w.Q0   # only X changes
+    X.copy_(dev_bf16(w2.X))
+    g.replay()
+    torch.cuda.synchronize()
+    compare({"Y": host_f64(Y)}, oracle.forward_workload(w2), label="graph replay")
+    del g
