@@ -1,23 +1,30 @@
-"""Plain fp64 CPU oracle for the FLARE / FLARE++ mixer forward.
+"""Plain fp64 CPU oracle for the FLARE / FLARE++ mixer, forward and backward.
 
 TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
 ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` are the only code
 allowed to import this package.  The CUDA library never calls it and shares no
 code with it.
 
-The arithmetic lives in ``flare_oracle.c`` (plain loops, fp64, two-pass
-softmax in ascending index order, OpenMP over independent rows); this module
-only marshals numpy arrays.  Every function cites the passage of the FLARE++
-paper (arXiv 2608.11519, section "Method") it follows:
+The arithmetic lives in ``flare_oracle.c`` (forward) and
+``flare_oracle_bwd.c`` (gradients: the SDPA backward of every call, written
+out per call) -- plain loops, fp64, two-pass softmax in ascending index
+order, OpenMP over independent rows; this module only marshals numpy arrays.
+Every function cites the passage of the FLARE++ paper (arXiv 2608.11519,
+section "Method") it follows:
 
   project   eq. 7 / eq. 9   K_h = X W_{K,h}, heads = column blocks of width D
   encode    eq. 5 / 8 / 10  Z_h = softmax_n(Q_h K_h^T / sqrt(D)) V_h
   decode    eq. 6 / 11      Y_h = softmax_m(K_h Q_h^T / sqrt(D)) Z_h
+  *_bwd     the gradients of the three above (the pages name the paper's
+            backward equations, eq. 13-40, without printing them)
 
 Pins (tests/test_oracle_pins.py): torch float64 SDPA chain, the materialised
 rank-M mixing matrix, closed forms (two tokens, identical keys, zero queries,
 one latent), token-permutation equivariance, the masked/unmasked identity and
 the shard-combine identity of section "Multi-GPU context parallelism" (eq. 14).
+Gradient pins (tests/test_oracle_bwd_pins.py): central finite differences of
+the forward oracle, torch float64 autograd through the SDPA chain, the
+shift invariances of the softmax and the sum rules of row-stochastic maps.
 """
 from __future__ import annotations
 
@@ -31,6 +38,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "flare_oracle.c")
+_SRC_BWD = os.path.join(_HERE, "flare_oracle_bwd.c")
 _BUILD = os.path.join(_HERE, "_build")
 _LIB_PATH = os.path.join(_BUILD, "libflare_oracle.so")
 _lock = threading.Lock()
@@ -40,12 +48,12 @@ _lib = None
 def build(force: bool = False) -> str:
     """Compile the C oracle with gcc (OpenMP, IEEE semantics, no FMA contraction)."""
     if not force and os.path.exists(_LIB_PATH) and \
-            os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC):
+            os.path.getmtime(_LIB_PATH) >= max(os.path.getmtime(_SRC), os.path.getmtime(_SRC_BWD)):
         return _LIB_PATH
     os.makedirs(_BUILD, exist_ok=True)
     tmp = _LIB_PATH + f".tmp{os.getpid()}"
     cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fPIC",
-           "-shared", "-o", tmp, _SRC, "-lm"]
+           "-shared", "-o", tmp, _SRC, _SRC_BWD, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
@@ -69,6 +77,14 @@ def _load():
         lib.flare_oracle_decode.argtypes = [dp, dp, ctypes.c_int, dp, ip, ctypes.c_double,
                                             L, L, L, L, L, lp, L, dp]
         lib.flare_oracle_decode.restype = None
+        lib.flare_oracle_encode_bwd.argtypes = [dp, ctypes.c_int, dp, dp, ip, ctypes.c_double,
+                                                L, L, L, L, L, dp, dp, dp, dp]
+        lib.flare_oracle_encode_bwd.restype = None
+        lib.flare_oracle_decode_bwd.argtypes = [dp, dp, ctypes.c_int, dp, ip, ctypes.c_double,
+                                                L, L, L, L, L, dp, dp, dp, dp]
+        lib.flare_oracle_decode_bwd.restype = None
+        lib.flare_oracle_project_bwd.argtypes = [dp, dp, dp, L, L, L, L, L, dp, dp]
+        lib.flare_oracle_project_bwd.restype = None
         lib.flare_oracle_num_threads.argtypes = []
         lib.flare_oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -209,3 +225,109 @@ def forward_workload(w, rows=None, keep_projections: bool = False) -> dict:
     if w.Wo is not None and rows is None:
         out["Out"] = output_projection(out["Y"], f64(w.Wo))
     return out
+
+
+# ---------------------------------------------------------------------------
+# backward (gradients of a scalar loss given dY = dLoss/dY)
+# ---------------------------------------------------------------------------
+
+def _qinfo(Q, B, H, D):
+    if Q.ndim == 3:
+        assert Q.shape[0] == H and Q.shape[2] == D
+        return 0, Q.shape[1]
+    assert Q.shape[:2] == (B, H) and Q.shape[3] == D
+    return 1, Q.shape[2]
+
+
+def encode_bwd(Q, K, V, dZ, lengths=None, scale: Optional[float] = None):
+    """Gradients of the encoder (eq. 5 / 8 / 10) given dZ [B][H][M][D]:
+    returns (dQ shaped like Q, dK, dV [B][H][N][D]).  A query set shared over
+    the batch ([H][M][D]) gets the sum of its per-sample gradients."""
+    Q, K, V, dZ = _f64(Q), _f64(K), _f64(V), _f64(dZ)
+    B, H, N, D = K.shape
+    per_batch, M = _qinfo(Q, B, H, D)
+    assert V.shape == K.shape and dZ.shape == (B, H, M, D)
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    lens, lp = _lens(lengths, B)
+    dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+    _load().flare_oracle_encode_bwd(_dptr(Q), per_batch, _dptr(K), _dptr(V), lp, float(scale),
+                                    B, H, N, M, D, _dptr(dZ), _dptr(dQ), _dptr(dK), _dptr(dV))
+    return dQ, dK, dV
+
+
+def decode_bwd(K, Q, Z, dY, lengths=None, scale: Optional[float] = None):
+    """Gradients of the decoder (eq. 6 / 11) given dY [B][H][N][D] (rows of
+    masked tokens are ignored: their outputs are constant zeros): returns
+    (dK [B][H][N][D], dQ shaped like Q, dZ [B][H][M][D])."""
+    K, Q, Z, dY = _f64(K), _f64(Q), _f64(Z), _f64(dY)
+    B, H, N, D = K.shape
+    per_batch, M = _qinfo(Q, B, H, D)
+    assert Z.shape == (B, H, M, D) and dY.shape == K.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    lens, lp = _lens(lengths, B)
+    dK, dQ, dZ = np.zeros_like(K), np.zeros_like(Q), np.zeros_like(Z)
+    _load().flare_oracle_decode_bwd(_dptr(K), _dptr(Q), per_batch, _dptr(Z), lp, float(scale),
+                                    B, H, N, M, D, _dptr(dY), _dptr(dK), _dptr(dQ), _dptr(dZ))
+    return dK, dQ, dZ
+
+
+def project_bwd(X, W, dOut):
+    """Gradients of the per-head projection (eq. 7 / 9) given dOut
+    [B][H][N][D]: returns (dX [B][N][C], dW [C][C])."""
+    X, W, dOut = _f64(X), _f64(W), _f64(dOut)
+    B, N, C = X.shape
+    _, H, _, D = dOut.shape
+    assert W.shape == (C, C) and dOut.shape == (B, H, N, D) and H * D == C
+    dX, dW = np.zeros_like(X), np.zeros_like(W)
+    _load().flare_oracle_project_bwd(_dptr(X), _dptr(W), _dptr(dOut), B, N, C, H, D,
+                                     _dptr(dX), _dptr(dW))
+    return dX, dW
+
+
+def flare_backward(K, V, Q, dY, lengths=None, scale=None) -> dict:
+    """Gradients of the FLARE mixer Y = SDPA(K, Q, SDPA(Q, K, V)) (eq. 5-6):
+    K gets the sum of its decoder and encoder gradients, Q (shared over the
+    batch) the sum over the batch of both."""
+    Z = encode(Q, K, V, lengths, scale)
+    dK, dQ, dZ = decode_bwd(K, Q, Z, dY, lengths, scale)
+    dQe, dKe, dV = encode_bwd(Q, K, V, dZ, lengths, scale)
+    return {"dK": dK + dKe, "dV": dV, "dQ": dQ + dQe, "dZ": dZ}
+
+
+def flarepp_backward(X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, H: int, lengths=None,
+                     scale=None) -> dict:
+    """Gradients of the FLARE++ mixer (eq. 7-11) with respect to X, the four
+    projection weights and the seeds Q0, given dY [B][H][N][D].  The chain:
+    decode -> (dK, dQ(X), dZ); encode with Q(X) -> (dQ(X), dK, dV); synthesis
+    with Q0 -> (dQ0, dK~, dV~); projections -> dX and the weight gradients.
+    The intermediate dQ(X) and dZ are returned as well."""
+    Kt, Vt = project(X, Wk_syn, H), project(X, Wv_syn, H)
+    Qx = encode(Q0, Kt, Vt, lengths, scale)
+    K, V = project(X, Wk, H), project(X, Wv, H)
+    Z = encode(Qx, K, V, lengths, scale)
+    dK, dQx, dZ = decode_bwd(K, Qx, Z, dY, lengths, scale)
+    dQx_e, dK_e, dV = encode_bwd(Qx, K, V, dZ, lengths, scale)
+    dK = dK + dK_e
+    dQx = dQx + dQx_e
+    dQ0, dKt, dVt = encode_bwd(Q0, Kt, Vt, dQx, lengths, scale)
+    dX = np.zeros_like(_f64(X))
+    grads = {}
+    for name, W, dOut in (("dWk", Wk, dK), ("dWv", Wv, dV), ("dWk_syn", Wk_syn, dKt),
+                          ("dWv_syn", Wv_syn, dVt)):
+        dXi, dWi = project_bwd(X, W, dOut)
+        dX += dXi
+        grads[name] = dWi
+    grads.update(dX=dX, dQ0=dQ0, dQx=dQx, dZ=dZ)
+    return grads
+
+
+def backward_workload(w, dY) -> dict:
+    """Run the backward oracle on a ``workloads.Workload`` and an upstream
+    gradient dY [B][H][N][D] (both bf16 bits, widened to fp64)."""
+    from workloads import bf16_bits_to_f64 as f64
+    if w.variant == "flare":
+        return flare_backward(f64(w.K), f64(w.V), f64(w.Q), f64(dY), w.lengths, w.scale)
+    return flarepp_backward(f64(w.X), f64(w.Wk), f64(w.Wv), f64(w.Wk_syn), f64(w.Wv_syn),
+                            f64(w.Q0), f64(dY), w.H, w.lengths, w.scale)
