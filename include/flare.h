@@ -1,5 +1,6 @@
 /*
- * flare.h - C ABI of the B200 (sm_100a) FLARE / FLARE++ mixer forward.
+ * flare.h - C ABI of the B200 (sm_100a) FLARE / FLARE++ mixer, forward and
+ * backward (gradients).
  *
  * What the calls compute (FLARE++ paper, arXiv 2608.11519, section "Method"):
  *
@@ -92,6 +93,8 @@ typedef enum {
 #define FLARE_VARIANT_FLARE 0
 #define FLARE_VARIANT_FLAREPP 1
 #define FLARE_VARIANT_FLAREPP_OUT 2 /* flarepp_mixer_out_fwd */
+#define FLARE_VARIANT_FLARE_BWD 3   /* flare_mixer_bwd */
+#define FLARE_VARIANT_FLAREPP_BWD 4 /* flarepp_mixer_bwd */
 
 /*
  * Workspace size in bytes for one call with these sizes (C is ignored for
@@ -169,6 +172,55 @@ FLARE_API flare_status flarepp_mixer_fwd_profiled(const flare_bf16* X, const fla
                                                   int M, int D, const int32_t* lengths, float scale,
                                                   void* workspace, size_t workspace_bytes, void* stream,
                                                   float* Qx_out, float* Z_out, void* const* stage_events);
+
+/*
+ * Backward (gradients of a scalar loss, given dY = dLoss/dY).
+ *
+ * The pages name the paper's backward equations (eq. 13-40) without
+ * printing them; every step of the mixer is one SDPA call, so these calls
+ * compute the SDPA backward of each step (for O = softmax_rows(s Qa Ka^T) Va:
+ * dVa = P^T dO, dS = P (dO Va^T - rowsum(P (dO Va^T))), dQa = s dS Ka,
+ * dKa = s dS^T Qa), chained through the mixer.  Each call is
+ * self-contained: it recomputes what the forward produced (the projections,
+ * Q(X), Z and the softmax normalisers, all in fp32) from the inputs, so it
+ * takes the forward's inputs and dY, not the forward's outputs.  Outputs are
+ * written (not accumulated).  Rows of dY for padding tokens are ignored;
+ * padding tokens get zero gradients.  Same size limits as the forward, and
+ * B*H <= 65535.  Arithmetic: fp32 on the CUDA cores (bf16 inputs widened),
+ * the FLARE++ projections recomputed on the tensor cores in bf16 as in the
+ * forward; deterministic like the forward.
+ *
+ * flare_mixer_bwd (FLARE, eq. 5-6), workspace variant FLARE_VARIANT_FLARE_BWD:
+ *   K, V, Q, lengths, scale   as in flare_mixer_fwd
+ *   dY    [B][H][N][D] bf16, read only
+ *   dK, dV [B][H][N][D] bf16, written (dK sums the encoder's and the
+ *          decoder's parts)
+ *   dQ    [H][M][D] float, written (summed over the batch)
+ */
+FLARE_API flare_status flare_mixer_bwd(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q,
+                                       const flare_bf16* dY, flare_bf16* dK, flare_bf16* dV, float* dQ, int B, int H,
+                                       int N, int M, int D, const int32_t* lengths, float scale, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
+/*
+ * flarepp_mixer_bwd (FLARE++, eq. 7-11), workspace variant
+ * FLARE_VARIANT_FLAREPP_BWD:
+ *   X, Wk, Wv, Wk_syn, Wv_syn, Q0, lengths, scale   as in flarepp_mixer_fwd
+ *   dY    [B][H][N][D] bf16, read only (gradient of the per-head output Y)
+ *   dX    [B][N][C] bf16, written
+ *   dWk, dWv, dWk_syn, dWv_syn   [C][C] float, written
+ *   dQ0   [H][M][D] float, written (summed over the batch)
+ * With the shared-projection variant (Wk_syn == Wk and Wv_syn == Wv as
+ * pointers) dWk and dWv receive the whole gradient of the shared weights;
+ * dWk_syn and dWv_syn may then be NULL and, if given, receive the same
+ * values.
+ */
+FLARE_API flare_status flarepp_mixer_bwd(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                                         const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0,
+                                         const flare_bf16* dY, flare_bf16* dX, float* dWk, float* dWv,
+                                         float* dWk_syn, float* dWv_syn, float* dQ0, int B, int N, int C, int H,
+                                         int M, int D, const int32_t* lengths, float scale, void* workspace,
+                                         size_t workspace_bytes, void* stream);
 
 /*
  * Synchronises `stream`, reads the device error word of `workspace` and

@@ -1,4 +1,4 @@
-"""B200 (sm_100a) FLARE / FLARE++ mixer forward.
+"""B200 (sm_100a) FLARE / FLARE++ mixer, forward and backward.
 
 The compute lives in ``libflare.so`` (hand-written CUDA kernels behind the C
 ABI of ``include/flare.h``).  This package is a thin ctypes binding: it checks
@@ -10,14 +10,18 @@ from ._binding import (  # noqa: F401
     FLARE_VARIANT_FLARE,
     FLARE_VARIANT_FLAREPP,
     FLARE_VARIANT_FLAREPP_OUT,
+    FLARE_VARIANT_FLARE_BWD,
+    FLARE_VARIANT_FLAREPP_BWD,
     FlareError,
     Status,
     flare_last_device_status,
+    flare_mixer_bwd,
     flare_mixer_fwd,
     flare_mixer_fwd_static,
     flare_selftest_wait_timeout,
     flare_status_string,
     flare_workspace_bytes,
+    flarepp_mixer_bwd,
     flarepp_mixer_fwd,
     flarepp_mixer_out_fwd,
     library_path,

@@ -15,6 +15,8 @@ _lib = None
 FLARE_VARIANT_FLARE = 0
 FLARE_VARIANT_FLAREPP = 1
 FLARE_VARIANT_FLAREPP_OUT = 2
+FLARE_VARIANT_FLARE_BWD = 3
+FLARE_VARIANT_FLAREPP_BWD = 4
 
 
 class Status(enum.IntEnum):
@@ -73,6 +75,10 @@ def load_library(build_if_missing: bool = True):
             fn.restype = i
             fn.argtypes = args
         lib.flarepp_mixer_out_fwd.restype = i
+        lib.flare_mixer_bwd.restype = i
+        lib.flare_mixer_bwd.argtypes = [vp] * 7 + [i] * 5 + [vp, f, vp, sz, vp]
+        lib.flarepp_mixer_bwd.restype = i
+        lib.flarepp_mixer_bwd.argtypes = [vp] * 13 + [i] * 6 + [vp, f, vp, sz, vp]
         lib.flarepp_mixer_out_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, f, vp, sz, vp]
         lib.flarepp_mixer_fwd_profiled.restype = i
         lib.flare_mixer_fwd_static.argtypes = [vp, vp, vp, vp, i, i, i, i, i, vp, f, vp, vp]
@@ -261,6 +267,74 @@ def flare_mixer_fwd_static(K, V, Q, lengths=None, scale: float = 0.0, Y=None, st
     if st != 0:
         raise FlareError(st, "flare_mixer_fwd_static")
     return Y
+
+
+def flare_mixer_bwd(K, V, Q, dY, lengths=None, scale: float = 0.0, workspace=None, stream=None,
+                    dK=None, dV=None, dQ=None, check: bool = True):
+    """FLARE backward (gradients of eq. 5-6 given dY).  K, V, dY: [B,H,N,D] bf16;
+    Q: [H,M,D] bf16 -> (dK, dV) [B,H,N,D] bf16 and dQ [H,M,D] float32."""
+    torch = _torch()
+    B, H, N, D = K.shape
+    M = Q.shape[1]
+    if check:
+        _check_dev("K", K, torch.bfloat16)
+        for nm, t in (("V", V), ("dY", dY), ("dK", dK), ("dV", dV)):
+            _check_dev(nm, t, torch.bfloat16, K.shape)
+        _check_dev("Q", Q, torch.bfloat16, (H, M, D))
+        _check_dev("dQ", dQ, torch.float32, (H, M, D))
+        _check_dev("lengths", lengths, torch.int32, (B,))
+    dK = torch.empty_like(K) if dK is None else dK
+    dV = torch.empty_like(K) if dV is None else dV
+    dQ = torch.empty((H, M, D), dtype=torch.float32, device=K.device) if dQ is None else dQ
+    nbytes = flare_workspace_bytes(FLARE_VARIANT_FLARE_BWD, B, H, N, M, D)
+    workspace = _workspace(workspace, nbytes, K.device)
+    st = load_library().flare_mixer_bwd(_ptr(K), _ptr(V), _ptr(Q), _ptr(dY), _ptr(dK), _ptr(dV), _ptr(dQ),
+                                        B, H, N, M, D, _ptr(lengths), float(scale), _ptr(workspace),
+                                        workspace.numel(), _stream_ptr(stream, K.device))
+    if st != 0:
+        raise FlareError(st, "flare_mixer_bwd")
+    return dK, dV, dQ
+
+
+def flarepp_mixer_bwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, lengths=None, scale: float = 0.0, workspace=None,
+                      stream=None, grads=None, check: bool = True):
+    """FLARE++ backward (gradients of eq. 7-11 given dY [B,H,N,D] bf16).
+    Returns a dict: dX [B,N,C] bf16; dWk, dWv, dWk_syn, dWv_syn [C,C] float32;
+    dQ0 [H,M,D] float32.  ``grads`` may hold preallocated outputs by name."""
+    torch = _torch()
+    B, N, C = X.shape
+    H, M, D = Q0.shape
+    if check:
+        _check_dev("X", X, torch.bfloat16)
+        for nm, w in (("Wk", Wk), ("Wv", Wv), ("Wk_syn", Wk_syn), ("Wv_syn", Wv_syn)):
+            _check_dev(nm, w, torch.bfloat16, (C, C))
+        _check_dev("Q0", Q0, torch.bfloat16)
+        _check_dev("dY", dY, torch.bfloat16, (B, H, N, D))
+        _check_dev("lengths", lengths, torch.int32, (B,))
+    g = dict(grads or {})
+    dev = X.device
+    if g.get("dX") is None:
+        g["dX"] = torch.empty((B, N, C), dtype=torch.bfloat16, device=dev)
+    for nm in ("dWk", "dWv", "dWk_syn", "dWv_syn"):
+        if g.get(nm) is None:
+            g[nm] = torch.empty((C, C), dtype=torch.float32, device=dev)
+    if g.get("dQ0") is None:
+        g["dQ0"] = torch.empty((H, M, D), dtype=torch.float32, device=dev)
+    if check:
+        _check_dev("dX", g["dX"], torch.bfloat16, (B, N, C))
+        for nm in ("dWk", "dWv", "dWk_syn", "dWv_syn"):
+            _check_dev(nm, g[nm], torch.float32, (C, C))
+        _check_dev("dQ0", g["dQ0"], torch.float32, (H, M, D))
+    nbytes = flare_workspace_bytes(FLARE_VARIANT_FLAREPP_BWD, B, H, N, M, D, C)
+    workspace = _workspace(workspace, nbytes, dev)
+    st = load_library().flarepp_mixer_bwd(
+        _ptr(X), _ptr(Wk), _ptr(Wv), _ptr(Wk_syn), _ptr(Wv_syn), _ptr(Q0), _ptr(dY), _ptr(g["dX"]),
+        _ptr(g["dWk"]), _ptr(g["dWv"]), _ptr(g["dWk_syn"]), _ptr(g["dWv_syn"]), _ptr(g["dQ0"]),
+        B, N, C, H, M, D, _ptr(lengths), float(scale), _ptr(workspace), workspace.numel(),
+        _stream_ptr(stream, dev))
+    if st != 0:
+        raise FlareError(st, "flarepp_mixer_bwd")
+    return g
 
 
 def flare_last_device_status(workspace, stream=None) -> Status:

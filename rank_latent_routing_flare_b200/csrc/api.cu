@@ -6,6 +6,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "bwd_internal.h"
 #include "flare.h"
 #include "flare_internal.h"
 
@@ -141,6 +142,62 @@ Plan make_plan(int variant, long B, long H, long N, long M, long D) {
   }
   p.total = off;
   return p;
+}
+
+// Workspace of the backward: the forward's (projection outputs, error word)
+// followed by the fp32 recompute and gradient buffers.
+struct BwdPlan {
+  Plan fwd;
+  int S = 1, tps = 1, rpb = 32, LB = 1, dw_splits = 1;
+  size_t off_q32 = 0, off_qx32 = 0, off_lsyn = 0, off_dqx32 = 0, off_gsyn = 0, off_z32 = 0, off_lenc = 0,
+         off_ltok = 0, off_dtok = 0, off_dz32 = 0, off_gam = 0, off_fpart = 0, off_pa = 0, off_pb = 0, off_pc = 0,
+         off_g32 = 0, off_dwpart = 0, total = 0;
+};
+
+BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C) {
+  BwdPlan bp;
+  bp.fwd = make_plan(pp ? FLARE_VARIANT_FLAREPP : FLARE_VARIANT_FLARE, B, H, N, M, D);
+  const long BH = B * H;
+  bp.rpb = static_cast<int>(std::min(128L, cdiv(M, 32) * 32));
+  bp.LB = static_cast<int>(cdiv(M, bp.rpb));
+  // token splits of the latent-parallel passes: about eight CTAs per SM
+  const long ntiles = cdiv(N, kBwdTokTile);
+  const long S0 = std::max(1L, std::min(ntiles, cdiv(static_cast<long>(kNumSM) * 8, BH * bp.LB)));
+  bp.tps = static_cast<int>(cdiv(ntiles, S0));
+  bp.S = static_cast<int>(cdiv(ntiles, bp.tps));
+  bp.dw_splits = static_cast<int>(cdiv(B * N, kBwdDwRows));
+  size_t off = bp.fwd.total;
+  auto take = [&off](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t lat = static_cast<size_t>(BH * M * D) * 4, row = static_cast<size_t>(BH * M) * 4;
+  const size_t tokv = static_cast<size_t>(BH * N) * 4;
+  const size_t part = static_cast<size_t>(BH) * bp.S * M * D * 4;
+  bp.off_q32 = take(static_cast<size_t>(H * M * D) * 4);
+  if (pp) {
+    bp.off_qx32 = take(lat);
+    bp.off_lsyn = take(row);
+    bp.off_dqx32 = take(lat);
+    bp.off_gsyn = take(row);
+  }
+  bp.off_z32 = take(lat);
+  bp.off_lenc = take(row);
+  bp.off_ltok = take(tokv);
+  bp.off_dtok = take(tokv);
+  bp.off_dz32 = take(lat);
+  bp.off_gam = take(row);
+  bp.off_fpart = take(static_cast<size_t>(BH) * bp.S * M * (D + 2) * 4);
+  bp.off_pa = take(part);
+  bp.off_pb = take(part);
+  bp.off_pc = take(part);
+  if (pp) {
+    bp.off_g32 = take(static_cast<size_t>(B * N) * 4 * C * 4);
+    bp.off_dwpart = take(static_cast<size_t>(bp.dw_splits) * C * 4 * C * 4);
+  }
+  bp.total = off;
+  return bp;
 }
 
 // Records stage event i (a cudaEvent_t passed as void*) when profiling is on.
@@ -301,10 +358,14 @@ using namespace flare;
 extern "C" {
 
 size_t flare_workspace_bytes(int variant, int B, int H, int N, int M, int D, int C) {
-  if (variant != FLARE_VARIANT_FLARE && variant != FLARE_VARIANT_FLAREPP && variant != FLARE_VARIANT_FLAREPP_OUT)
-    return 0;
+  if (variant < FLARE_VARIANT_FLARE || variant > FLARE_VARIANT_FLAREPP_BWD) return 0;
   if (check_common(B, H, N, M, D) != FLARE_OK) return 0;
-  if (variant != FLARE_VARIANT_FLARE && (C != H * D || C % 64 != 0 || C > 256)) return 0;
+  const bool pp = variant != FLARE_VARIANT_FLARE && variant != FLARE_VARIANT_FLARE_BWD;
+  if (pp && (C != H * D || C % 64 != 0 || C > 256)) return 0;
+  if (variant == FLARE_VARIANT_FLARE_BWD || variant == FLARE_VARIANT_FLAREPP_BWD) {
+    if (static_cast<long>(B) * H > 65535) return 0;
+    return make_bwd_plan(pp, B, H, N, M, D, C).total;
+  }
   return make_plan(variant, B, H, N, M, D).total;
 }
 
@@ -715,6 +776,220 @@ flare_status flare_selftest_wait_timeout(void* workspace, void* stream, unsigned
   if (cudaMemsetAsync(workspace, 0, 4, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   if (launch_wait_selftest(static_cast<uint32_t*>(workspace), timeout_ns, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   return FLARE_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward (gradients)
+// ---------------------------------------------------------------------------
+
+namespace flare {
+namespace {
+
+// Where the token-parallel pass writes dK and dV: token-major fp32 rows of
+// the projection-gradient matrix, or bf16 [B][H][N][D] outputs.
+struct TokOut {
+  float* g32;
+  int g_ld, col_k, col_v;
+  uint16_t *dk16, *dv16;
+};
+
+LatParams lat_params(const BwdPlan& bp, uint8_t* ws, const float* q, int q_per_batch, const void* k, int B, int H,
+                     int N, int M, int D, const int32_t* lengths, float sc) {
+  LatParams lp{};
+  lp.B = B; lp.H = H; lp.N = N; lp.M = M; lp.D = D;
+  lp.q_per_batch = q_per_batch;
+  lp.n_splits = bp.S; lp.tiles_per_split = bp.tps; lp.rows_per_block = bp.rpb;
+  lp.c = sc * 1.4426950408889634f;
+  lp.lengths = lengths;
+  lp.q = q;
+  lp.k = static_cast<const uint16_t*>(k);
+  lp.err = reinterpret_cast<uint32_t*>(ws + bp.fwd.off_err);
+  return lp;
+}
+
+// Encoder recompute: Z (fp32) and the row log2-normalisers of
+// softmax_n(s Q K^T) V.
+flare_status bwd_encode(const BwdPlan& bp, uint8_t* ws, const float* q, int q_per_batch, const void* k, const void* v,
+                        float* z, float* lse, int B, int H, int N, int M, int D, const int32_t* lengths, float sc,
+                        cudaStream_t s) {
+  LatParams lp = lat_params(bp, ws, q, q_per_batch, k, B, H, N, M, D, lengths, sc);
+  lp.v = static_cast<const uint16_t*>(v);
+  lp.part_a = reinterpret_cast<float*>(ws + bp.off_fpart);
+  if (launch_lat(kLatForward, lp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  const LatMergeParams mp{B * H, M, D, bp.S, lp.part_a, z, lse};
+  return launch_lat_merge(mp, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+}
+
+// Backward of Y = SDPA(K, Q, SDPA(Q, K, V)) for queries q (fp32, log2 scaling
+// applied in the kernels): dK and dV go to `out`; the split partials of the
+// decoder's and the encoder's dQ are left in pb and pc.
+flare_status bwd_core(const BwdPlan& bp, uint8_t* ws, const float* q, int q_per_batch, const void* k, const void* v,
+                      const void* dy, int B, int H, int N, int M, int D, const int32_t* lengths, float sc,
+                      cudaStream_t s, const TokOut& out) {
+  float* z32 = reinterpret_cast<float*>(ws + bp.off_z32);
+  float* lenc = reinterpret_cast<float*>(ws + bp.off_lenc);
+  float* ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
+  float* dtok = reinterpret_cast<float*>(ws + bp.off_dtok);
+  float* dz32 = reinterpret_cast<float*>(ws + bp.off_dz32);
+  float* gam = reinterpret_cast<float*>(ws + bp.off_gam);
+  float* pa = reinterpret_cast<float*>(ws + bp.off_pa);
+  float* pb = reinterpret_cast<float*>(ws + bp.off_pb);
+  float* pc = reinterpret_cast<float*>(ws + bp.off_pc);
+  // forward recompute: Z, the encoder's row normalisers, the decoder's
+  // per-token normalisers and delta_n = <dY_n, Y_n>
+  flare_status st = bwd_encode(bp, ws, q, q_per_batch, k, v, z32, lenc, B, H, N, M, D, lengths, sc, s);
+  if (st != FLARE_OK) return st;
+  TokParams tp{};
+  tp.B = B; tp.H = H; tp.N = N; tp.M = M; tp.D = D;
+  tp.q_per_batch = q_per_batch;
+  tp.c = sc * 1.4426950408889634f;
+  tp.lengths = lengths;
+  tp.q = q; tp.z = z32; tp.dz = dz32; tp.lm = lenc; tp.gam = gam;
+  tp.k = static_cast<const uint16_t*>(k);
+  tp.v = static_cast<const uint16_t*>(v);
+  tp.dy = static_cast<const uint16_t*>(dy);
+  tp.ltok = ltok; tp.dtok = dtok;
+  tp.g32 = out.g32; tp.g_ld = out.g_ld; tp.g_col_k = out.col_k; tp.g_col_v = out.col_v;
+  tp.dk16 = out.dk16; tp.dv16 = out.dv16;
+  tp.err = reinterpret_cast<uint32_t*>(ws + bp.fwd.off_err);
+  if (launch_tok(kTokStats, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  // decoder backward, reductions over tokens: dZ and the decoder's dQ
+  LatParams lp = lat_params(bp, ws, q, q_per_batch, k, B, H, N, M, D, lengths, sc);
+  lp.zrow = z32; lp.dy = static_cast<const uint16_t*>(dy); lp.ltok = ltok; lp.dtok = dtok;
+  lp.part_a = pa; lp.part_b = pb;
+  if (launch_lat(kLatDecoder, lp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  const LatSumParams sz{B, H, M, D, bp.S, 0, 1.f, pa, nullptr, z32, gam, dz32};
+  if (launch_lat_sum(sz, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  // dK (both parts) and dV
+  if (launch_tok(kTokFull, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  // encoder backward, reduction over tokens: the encoder's dQ
+  LatParams le = lat_params(bp, ws, q, q_per_batch, k, B, H, N, M, D, lengths, sc);
+  le.zrow = dz32; le.lrow = lenc; le.grow = gam; le.v = static_cast<const uint16_t*>(v);
+  le.part_b = pc;
+  return launch_lat(kLatEncoder, le, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+}
+
+flare_status check_bwd_sizes(int B, int H, int N, int M, int D) {
+  flare_status st = check_common(B, H, N, M, D);
+  if (st != FLARE_OK) return st;
+  return static_cast<long>(B) * H > 65535 ? FLARE_ERR_UNSUPPORTED : FLARE_OK;
+}
+
+}  // namespace
+}  // namespace flare
+
+extern "C" {
+
+flare_status flare_mixer_bwd(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, const flare_bf16* dY,
+                             flare_bf16* dK, flare_bf16* dV, float* dQ, int B, int H, int N, int M, int D,
+                             const int32_t* lengths, float scale, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  if (!K || !V || !Q || !dY || !dK || !dV || !dQ || !workspace) return FLARE_ERR_NULL;
+  flare_status st = check_bwd_sizes(B, H, N, M, D);
+  if (st != FLARE_OK) return st;
+  if (!aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(dY) || !aligned16(dK) || !aligned16(dV) ||
+      !aligned16(dQ) || !aligned16(lengths) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FLARE_ERR_ALIGN;
+  const BwdPlan bp = make_bwd_plan(false, B, H, N, M, D, 0);
+  if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
+  const float sc = resolve_scale(scale, D);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(ws + bp.fwd.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  float* q32 = reinterpret_cast<float*>(ws + bp.off_q32);
+  const CvtParams cv{static_cast<long>(H) * M * D, reinterpret_cast<const uint16_t*>(Q), q32};
+  if (launch_cvt(cv, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  const TokOut out{nullptr, 0, 0, 0, reinterpret_cast<uint16_t*>(dK), reinterpret_cast<uint16_t*>(dV)};
+  st = bwd_core(bp, ws, q32, 0, K, V, dY, B, H, N, M, D, lengths, sc, s, out);
+  if (st != FLARE_OK) return st;
+  // dQ = scale * sum over the batch and the splits of both parts
+  const LatSumParams sq{B, H, M, D, bp.S, 1, sc, reinterpret_cast<float*>(ws + bp.off_pb),
+                        reinterpret_cast<float*>(ws + bp.off_pc), nullptr, nullptr, dQ};
+  return launch_lat_sum(sq, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+}
+
+flare_status flarepp_mixer_bwd(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                               const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0,
+                               const flare_bf16* dY, flare_bf16* dX, float* dWk, float* dWv, float* dWk_syn,
+                               float* dWv_syn, float* dQ0, int B, int N, int C, int H, int M, int D,
+                               const int32_t* lengths, float scale, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  flare_status st = check_flarepp(X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, B, N, C, H, M, D, lengths, workspace, nullptr,
+                                  nullptr);
+  if (st != FLARE_OK) return st;
+  const bool shared = Wk_syn == Wk && Wv_syn == Wv;
+  if (!dX || !dWk || !dWv || !dQ0 || (!shared && (!dWk_syn || !dWv_syn))) return FLARE_ERR_NULL;
+  if ((st = check_bwd_sizes(B, H, N, M, D)) != FLARE_OK) return st;
+  if (static_cast<long>(B) * N > 65535L * kBwdDwRows) return FLARE_ERR_UNSUPPORTED;
+  if (!aligned16(dX) || !aligned16(dWk) || !aligned16(dWv) || !aligned16(dWk_syn) || !aligned16(dWv_syn) ||
+      !aligned16(dQ0))
+    return FLARE_ERR_ALIGN;
+  const BwdPlan bp = make_bwd_plan(true, B, H, N, M, D, C);
+  if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
+  const float sc = resolve_scale(scale, D);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(ws + bp.fwd.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  // eq. 7 and 9: the projections, recomputed (tcgen05, as in the forward)
+  Projected pr;
+  if ((st = flarepp_project(bp.fwd, X, Wk, Wv, Wk_syn, Wv_syn, B, N, C, H, D, ws, s, nullptr, &pr)) != FLARE_OK)
+    return st;
+  float* q32 = reinterpret_cast<float*>(ws + bp.off_q32);
+  const CvtParams cv{static_cast<long>(H) * M * D, reinterpret_cast<const uint16_t*>(Q0), q32};
+  if (launch_cvt(cv, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  // eq. 8 recomputed: Q(X) and the synthesis row normalisers
+  float* qx32 = reinterpret_cast<float*>(ws + bp.off_qx32);
+  float* lsyn = reinterpret_cast<float*>(ws + bp.off_lsyn);
+  if ((st = bwd_encode(bp, ws, q32, 0, pr.kt, pr.vt, qx32, lsyn, B, H, N, M, D, lengths, sc, s)) != FLARE_OK)
+    return st;
+  // eq. 10-11 backward with the queries Q(X): dK, dV into the gradient rows
+  float* g32 = reinterpret_cast<float*>(ws + bp.off_g32);
+  const TokOut main_out{g32, 4 * C, 0, C, nullptr, nullptr};
+  st = bwd_core(bp, ws, qx32, 1, pr.kk, pr.vv, dY, B, H, N, M, D, lengths, sc, s, main_out);
+  if (st != FLARE_OK) return st;
+  // dQ(X) = scale * (decoder part + encoder part); gamma of the synthesis
+  float* dqx32 = reinterpret_cast<float*>(ws + bp.off_dqx32);
+  float* gsyn = reinterpret_cast<float*>(ws + bp.off_gsyn);
+  float* pc = reinterpret_cast<float*>(ws + bp.off_pc);
+  const LatSumParams sq{B, H, M, D, bp.S, 0, sc, reinterpret_cast<float*>(ws + bp.off_pb), pc, qx32, gsyn, dqx32};
+  if (launch_lat_sum(sq, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  // eq. 8 backward with dQ(X) as the upstream gradient: dK~, dV~ ...
+  TokParams tp{};
+  tp.B = B; tp.H = H; tp.N = N; tp.M = M; tp.D = D;
+  tp.q_per_batch = 0;
+  tp.c = sc * 1.4426950408889634f;
+  tp.lengths = lengths;
+  tp.q = q32; tp.dz = dqx32; tp.lm = lsyn; tp.gam = gsyn;
+  tp.k = pr.kt; tp.v = pr.vt;
+  tp.g32 = g32; tp.g_ld = 4 * C; tp.g_col_k = 2 * C; tp.g_col_v = 3 * C;
+  tp.err = reinterpret_cast<uint32_t*>(ws + bp.fwd.off_err);
+  if (launch_tok(kTokEncoder, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  // ... and dQ0 (summed over the batch)
+  LatParams le = lat_params(bp, ws, q32, 0, pr.kt, B, H, N, M, D, lengths, sc);
+  le.zrow = dqx32; le.lrow = lsyn; le.grow = gsyn; le.v = pr.vt;
+  le.part_b = pc;
+  if (launch_lat(kLatEncoder, le, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  const LatSumParams s0{B, H, M, D, bp.S, 1, sc, pc, nullptr, nullptr, nullptr, dQ0};
+  if (launch_lat_sum(s0, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  // projections backward: dX = G [Wk | Wv | Wk~ | Wv~]^T and dW = X^T G
+  const long R = static_cast<long>(B) * N;
+  DxParams dx{};
+  dx.R = static_cast<int>(R); dx.C = C; dx.nw = 4;
+  dx.g = g32;
+  const flare_bf16* ws4[4] = {Wk, Wv, Wk_syn, Wv_syn};
+  for (int i = 0; i < 4; ++i) dx.w[i] = reinterpret_cast<const uint16_t*>(ws4[i]);
+  dx.dx = reinterpret_cast<uint16_t*>(dX);
+  if (launch_dx(dx, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  float* dwpart = reinterpret_cast<float*>(ws + bp.off_dwpart);
+  const DwParams dw{static_cast<int>(R), C, 4 * C, bp.dw_splits, reinterpret_cast<const uint16_t*>(X), g32, dwpart};
+  if (launch_dw(dw, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  DwReduceParams dr{};
+  dr.C = C; dr.J = 4 * C; dr.n_splits = bp.dw_splits; dr.shared = shared ? 1 : 0;
+  dr.part = dwpart;
+  dr.dw[0] = dWk; dr.dw[1] = dWv; dr.dw[2] = dWk_syn; dr.dw[3] = dWv_syn;
+  return launch_dw_reduce(dr, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
 
 }  // extern "C"

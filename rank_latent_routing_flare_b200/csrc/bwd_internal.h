@@ -1,0 +1,129 @@
+// Internal definitions of the backward (gradient) kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace flare {
+
+constexpr int kBwdTokTile = 64;     // tokens per shared-memory tile of the latent-parallel kernels
+constexpr int kBwdTokBlock = 128;   // tokens per CTA of the token-parallel kernels
+constexpr int kBwdLatChunk = 64;    // latents per shared-memory chunk of the token-parallel kernels
+constexpr int kBwdGemmTile = 64;    // output tile (rows and columns) of the projection-gradient GEMMs
+constexpr int kBwdDwRows = 2048;    // token rows per split of the weight-gradient GEMM
+
+// Modes of the latent-parallel kernel (one CTA = a block of latents of one
+// head and one token split; a thread = one latent row, or half of one for
+// D = 32).
+enum LatMode : int {
+  kLatForward = 0,   // encoder recompute: per split (max, sum, sum w v) in log2 units
+  kLatDecoder = 1,   // decoder backward, reductions over tokens: dZ and dQ
+  kLatEncoder = 2,   // encoder backward, reduction over tokens: dQ
+};
+
+struct LatParams {
+  int B, H, N, M, D;
+  int q_per_batch;              // queries [G][M][D] with G = B*H (1) or H (0)
+  int n_splits, tiles_per_split, rows_per_block;
+  float c;                      // scale * log2(e)
+  const int32_t* lengths;
+  const float* q;               // fp32 queries [G][M][D]
+  const float* zrow;            // decoder: Z [B*H][M][D]; encoder: dZ [B*H][M][D]
+  const float* lrow;            // encoder: row log2-normaliser [B*H][M]
+  const float* grow;            // encoder: gamma = <dZ, Z> [B*H][M]
+  const uint16_t* k;            // bf16 [B*H][N][D]
+  const uint16_t* v;            // bf16 [B*H][N][D] (forward, encoder)
+  const uint16_t* dy;           // bf16 [B*H][N][D] (decoder)
+  const float* ltok;            // decoder: per-token log2-normaliser [B*H][N]
+  const float* dtok;            // decoder: delta = <dY, Y> [B*H][N]
+  float* part_a;                // forward: [B*H][S][M][D+2]; decoder: dZ partials [B*H][S][M][D]
+  float* part_b;                // decoder / encoder: dQ partials [B*H][S][M][D]
+  uint32_t* err;
+};
+
+struct LatMergeParams {
+  int BH, M, D, S;
+  const float* part;            // [B*H][S][M][D+2]
+  float* z;                     // [B*H][M][D]
+  float* lse;                   // [B*H][M], log2 units
+};
+
+struct LatSumParams {
+  int B, H, M, D, S;
+  int fold_batch;               // 1: out [H][M][D] sums the batch; 0: out [B*H][M][D]
+  float mult;
+  const float* part0;           // [B*H][S][M][D]
+  const float* part1;           // same shape or NULL
+  const float* zref;            // [B*H][M][D] or NULL: gamma = <out, zref> per row
+  float* gamma;                 // [B*H][M]
+  float* out;                   // fp32
+};
+
+// Modes of the token-parallel kernel (one CTA = kBwdTokBlock tokens of one
+// head; a thread = one token row, or half of one for D = 32).
+enum TokMode : int {
+  kTokStats = 0,     // decoder recompute: per-token log2-normaliser and delta = <dY, Y>
+  kTokFull = 1,      // dK (decoder + encoder parts) and dV
+  kTokEncoder = 2,   // dK and dV of an encoder alone (the query synthesis)
+};
+
+struct TokParams {
+  int B, H, N, M, D;
+  int q_per_batch;
+  float c;
+  const int32_t* lengths;
+  const float* q;               // fp32 queries [G][M][D]
+  const float* z;               // Z [B*H][M][D] (stats, full)
+  const float* dz;              // dZ [B*H][M][D] (full, encoder)
+  const float* lm;              // encoder row log2-normaliser [B*H][M]
+  const float* gam;             // gamma [B*H][M]
+  const uint16_t *k, *v, *dy;   // bf16 [B*H][N][D]
+  float* ltok;                  // [B*H][N]: written (stats), read (full)
+  float* dtok;                  // [B*H][N]: written (stats), read (full)
+  float* g32;                   // token-major fp32 gradient rows [B][N][g_ld] or NULL
+  int g_ld, g_col_k, g_col_v;   // row stride and column offsets of dK and dV (head h adds h*D)
+  uint16_t* dk16;               // or bf16 [B*H][N][D] outputs
+  uint16_t* dv16;
+  uint32_t* err;
+};
+
+// dX[r][c] = sum_q sum_j G[r][q*C + j] W_q[c][j]   (r < R = B*N, q < nw)
+struct DxParams {
+  int R, C, nw;
+  const float* g;               // [R][nw*C]
+  const uint16_t* w[4];         // bf16 [C][C]
+  uint16_t* dx;                 // bf16 [R][C]
+};
+
+// Partial weight gradients dWcat[c][j] = sum_{r in split} X[r][c] G[r][j].
+struct DwParams {
+  int R, C, J, n_splits;
+  const uint16_t* x;            // bf16 [R][C]
+  const float* g;               // [R][J]
+  float* part;                  // [n_splits][C][J]
+};
+
+// dW_q[c][j] = sum_splits part[.][c][q*C + j] (+ part[.][c][(q+2)*C + j]
+// when the synthesis weights are the encode weights).
+struct DwReduceParams {
+  int C, J, n_splits, shared;
+  const float* part;
+  float* dw[4];                 // [C][C] fp32 each (dWk, dWv, dWk_syn, dWv_syn); NULL = not written
+};
+
+struct CvtParams {
+  long n;
+  const uint16_t* src;
+  float* dst;
+};
+
+cudaError_t launch_lat(int mode, const LatParams& p, cudaStream_t s);
+cudaError_t launch_lat_merge(const LatMergeParams& p, cudaStream_t s);
+cudaError_t launch_lat_sum(const LatSumParams& p, cudaStream_t s);
+cudaError_t launch_tok(int mode, const TokParams& p, cudaStream_t s);
+cudaError_t launch_dx(const DxParams& p, cudaStream_t s);
+cudaError_t launch_dw(const DwParams& p, cudaStream_t s);
+cudaError_t launch_dw_reduce(const DwReduceParams& p, cudaStream_t s);
+cudaError_t launch_cvt(const CvtParams& p, cudaStream_t s);
+
+}  // namespace flare

@@ -33,7 +33,8 @@ def test_header_declares_the_abi():
                             "flare_mixer_fwd_profiled", "flarepp_mixer_fwd_profiled", "flare_mixer_fwd_static",
                             "flare_last_device_status", "flare_status_string",
                             "flare_selftest_wait_timeout", "flare_cp_partials_bytes", "flarepp_cp_begin",
-                            "flarepp_cp_middle", "flarepp_cp_end", "flare_cp_begin", "flare_cp_end"])
+                            "flarepp_cp_middle", "flarepp_cp_end", "flare_cp_begin", "flare_cp_end",
+                            "flare_mixer_bwd", "flarepp_mixer_bwd"])
 
 
 def test_library_loads_and_exports_every_declared_symbol():
@@ -87,7 +88,8 @@ def test_workspace_unsupported_sizes_return_zero():
     assert fl.flare_workspace_bytes(0, 1, 1, 64, 528, 16, 0) == 0      # M > 512
     assert fl.flare_workspace_bytes(1, 1, 2, 64, 32, 16, 48) == 0      # C != H*D
     assert fl.flare_workspace_bytes(1, 1, 3, 64, 32, 16, 48) == 0      # C not a multiple of 64
-    assert fl.flare_workspace_bytes(3, 1, 1, 64, 32, 16, 64) == 0      # bad variant
+    assert fl.flare_workspace_bytes(5, 1, 1, 64, 32, 16, 64) == 0      # bad variant
+    assert fl.flare_workspace_bytes(-1, 1, 1, 64, 32, 16, 64) == 0     # bad variant
     assert fl.flare_workspace_bytes(2, 1, 3, 64, 32, 16, 48) == 0      # C not a multiple of 64
     assert fl.flare_workspace_bytes(0, 0, 1, 64, 32, 16, 0) == 0       # B = 0
 
@@ -200,3 +202,71 @@ def test_context_parallel_argument_errors():
     assert lib.flare_cp_begin(A, A, A, *fargs, -1, 2, 0.0, W, fws, None, A) == Status.ERR_SHAPE
     assert lib.flare_cp_end(A, A, A, None, *fargs, 0, 2, 0.0, W, fws, None, None) == Status.ERR_NULL
     assert fl.flare_status_string(8).startswith("FLARE_ERR_UNDERFLOW")
+
+
+# ---------------------------------------------------------------------------
+# backward entry points
+# ---------------------------------------------------------------------------
+
+def flare_bwd_call(K=A, V=A, Q=A, dY=A, dK=A, dV=A, dQ=A, B=1, H=2, N=100, M=32, D=16, lengths=None,
+                   ws=W, ws_bytes=None):
+    lib = fl.load_library()
+    if ws_bytes is None:
+        ws_bytes = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLARE_BWD, B, H, N, M, D) or (1 << 40)
+    return lib.flare_mixer_bwd(K, V, Q, dY, dK, dV, dQ, B, H, N, M, D, lengths, 0.0, ws, ws_bytes, None)
+
+
+def flarepp_bwd_call(X=A, Wk=A, Wv=A, Wks=A + 0x100, Wvs=A + 0x200, Q0=A, dY=A, dX=A, dWk=A, dWv=A, dWks=A,
+                     dWvs=A, dQ0=A, B=1, N=100, C=64, H=4, M=32, D=16, lengths=None, ws=W, ws_bytes=None):
+    lib = fl.load_library()
+    if ws_bytes is None:
+        ws_bytes = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLAREPP_BWD, B, H, N, M, D, C) or (1 << 40)
+    return lib.flarepp_mixer_bwd(X, Wk, Wv, Wks, Wvs, Q0, dY, dX, dWk, dWv, dWks, dWvs, dQ0, B, N, C, H, M, D,
+                                 lengths, 0.0, ws, ws_bytes, None)
+
+
+def test_backward_workspace_sizes():
+    f_fwd = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLARE, 2, 4, 5000, 64, 16)
+    f_bwd = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLARE_BWD, 2, 4, 5000, 64, 16)
+    assert f_bwd > f_fwd > 0 and f_bwd % 256 == 0
+    p_fwd = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLAREPP, 2, 4, 5000, 64, 16, 64)
+    p_bwd = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLAREPP_BWD, 2, 4, 5000, 64, 16, 64)
+    # the FLARE++ backward holds fp32 gradient rows of the four projections
+    assert p_bwd > p_fwd + 2 * 5000 * 4 * 64 * 4
+    assert fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLAREPP_BWD, 2, 4, 5000, 64, 16, 128) == 0   # C != H*D
+    assert fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLARE_BWD, 65536, 1, 64, 16, 16) == 0      # B*H > 65535
+    assert fl.flare_workspace_bytes(5, 1, 4, 100, 32, 16, 64) == 0
+
+
+def test_flare_backward_argument_errors():
+    assert flare_bwd_call(dY=None) == Status.ERR_NULL
+    assert flare_bwd_call(dQ=None) == Status.ERR_NULL
+    assert flare_bwd_call(ws=None) == Status.ERR_NULL
+    assert flare_bwd_call(N=0) == Status.ERR_SHAPE
+    assert flare_bwd_call(D=64) == Status.ERR_UNSUPPORTED
+    assert flare_bwd_call(B=70000, H=1) == Status.ERR_UNSUPPORTED
+    assert flare_bwd_call(dK=A + 8) == Status.ERR_ALIGN
+    assert flare_bwd_call(dQ=A + 4) == Status.ERR_ALIGN
+    need = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLARE_BWD, 1, 2, 100, 32, 16)
+    assert flare_bwd_call(ws_bytes=need - 256) == Status.ERR_WORKSPACE
+
+
+def test_flarepp_backward_argument_errors():
+    assert flarepp_bwd_call(dX=None) == Status.ERR_NULL
+    assert flarepp_bwd_call(dQ0=None) == Status.ERR_NULL
+    assert flarepp_bwd_call(dWks=None) == Status.ERR_NULL           # separate synthesis weights need it
+    assert flarepp_bwd_call(C=128) == Status.ERR_SHAPE
+    assert flarepp_bwd_call(dWv=A + 4) == Status.ERR_ALIGN
+    assert flarepp_bwd_call(dY=A + 2) == Status.ERR_ALIGN
+    need = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLAREPP_BWD, 1, 4, 100, 32, 16, 64)
+    assert flarepp_bwd_call(ws_bytes=need - 256) == Status.ERR_WORKSPACE
+
+
+def test_backward_valid_calls_without_gpu_report_launch_error():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert flare_bwd_call() == Status.ERR_LAUNCH
+    assert flarepp_bwd_call() == Status.ERR_LAUNCH
+    # shared projections: the synthesis weight gradients may be NULL
+    assert flarepp_bwd_call(Wks=A, Wvs=A, dWks=None, dWvs=None) == Status.ERR_LAUNCH

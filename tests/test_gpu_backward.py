@@ -1,0 +1,173 @@
+"""GPU parity of the backward (gradients) against the fp64 oracle.
+
+The CUDA path (flare_mixer_bwd / flarepp_mixer_bwd through the C ABI) and
+the oracle (oracle.flare_backward / flarepp_backward) get the same bf16
+inputs and the same upstream gradient dY.  Tolerance per gradient tensor:
+rel-L2 <= 5e-3 and max |error| <= 3e-2 * max |reference| (the forward's
+bounds, the absolute one taken relative to the tensor's scale because
+gradients of different tensors differ by orders of magnitude).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rank_latent_routing_flare_b200 as fl
+from tests.gpu_util import dev_bf16, host_f64, rel_l2
+from workloads import make_upstream_grad, make_workload
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 5e-3
+MAX_REL = 3e-2
+
+
+def check(got, ref, label):
+    r = rel_l2(got, ref)
+    m = float(np.max(np.abs(got - ref)) / max(np.max(np.abs(ref)), 1e-30))
+    print(f"{label}: rel_l2={r:.3e} max_err/max_ref={m:.3e}")
+    assert r <= REL_L2 and m <= MAX_REL, (label, r, m)
+
+
+def lengths_dev(w):
+    return None if w.lengths is None else torch.from_numpy(w.lengths).cuda()
+
+
+def run_flare_bwd(w, dY):
+    dK, dV, dQ = fl.flare_mixer_bwd(dev_bf16(w.K), dev_bf16(w.V), dev_bf16(w.Q), dev_bf16(dY),
+                                    lengths=lengths_dev(w))
+    torch.cuda.synchronize()
+    return {"dK": host_f64(dK), "dV": host_f64(dV), "dQ": host_f64(dQ)}
+
+
+def run_flarepp_bwd(w, dY, shared=False):
+    X = dev_bf16(w.X)
+    Wk, Wv = dev_bf16(w.Wk), dev_bf16(w.Wv)
+    Wks, Wvs = (Wk, Wv) if shared else (dev_bf16(w.Wk_syn), dev_bf16(w.Wv_syn))
+    g = fl.flarepp_mixer_bwd(X, Wk, Wv, Wks, Wvs, dev_bf16(w.Q0), dev_bf16(dY), lengths=lengths_dev(w))
+    torch.cuda.synchronize()
+    return {k: host_f64(v) for k, v in g.items()}
+
+
+def flare_case(B, H, N, M, D, lengths=None, seed=5):
+    rng = np.random.default_rng(seed)
+    from workloads import to_bf16_bits
+    w = make_workload("flare_n64k", N=N, B=B, M=M, seed=seed)
+    if D != w.D or H != w.H:
+        w.H, w.D, w.C = H, D, H * D
+        w.K = to_bf16_bits(rng.standard_normal((B, H, N, D), dtype=np.float32))
+        w.V = to_bf16_bits(rng.standard_normal((B, H, N, D), dtype=np.float32))
+        w.Q = to_bf16_bits(rng.standard_normal((H, M, D), dtype=np.float32))
+    if lengths is not None:
+        w.lengths = np.asarray(lengths, dtype=np.int32)
+    return w
+
+
+@pytest.mark.parametrize("B,H,N,M,D,lengths", [
+    (2, 2, 777, 64, 16, None),
+    (2, 2, 777, 64, 16, [777, 300]),
+    (1, 3, 1000, 48, 32, None),
+    (3, 2, 200, 16, 16, [1, 200, 129]),
+])
+def test_flare_backward_matches_oracle(B, H, N, M, D, lengths):
+    w = flare_case(B, H, N, M, D, lengths)
+    dY = make_upstream_grad(w)
+    got = run_flare_bwd(w, dY)
+    ref = oracle.backward_workload(w, dY)
+    for k in ("dK", "dV", "dQ"):
+        check(got[k], ref[k], f"FLARE {k} B{B} H{H} N{N} M{M} D{D} L{lengths}")
+    if lengths is not None:
+        for b, L in enumerate(lengths):
+            assert np.all(got["dK"][b, :, L:] == 0) and np.all(got["dV"][b, :, L:] == 0)
+
+
+@pytest.mark.parametrize("name,N,B", [
+    ("flarepp_n1k", None, None),
+    ("flarepp_n8k_mesh2d", 1500, 2),
+    ("flarepp_masked_n4k", 640, 3),
+])
+def test_flarepp_backward_matches_oracle(name, N, B):
+    w = make_workload(name, N=N, B=B)
+    dY = make_upstream_grad(w)
+    got = run_flarepp_bwd(w, dY)
+    ref = oracle.backward_workload(w, dY)
+    for k in ("dX", "dWk", "dWv", "dWk_syn", "dWv_syn", "dQ0"):
+        check(got[k], ref[k], f"{name} N{w.N} B{w.B} {k}")
+    if w.lengths is not None:
+        for b, L in enumerate(w.lengths):
+            assert np.all(got["dX"][b, L:] == 0)
+
+
+def storage_model_bwd(w, dY):
+    """The oracle's FLARE++ backward in fp64 on the bf16-rounded projections
+    K~, V~, K, V (the only rounding inside the GPU backward: the projections
+    are recomputed on the tensor cores and stored as bf16, exactly as in the
+    forward; everything after them is fp32)."""
+    from workloads import bf16_bits_to_f64 as f64, to_bf16_bits
+    r = lambda a: f64(to_bf16_bits(a.astype(np.float32)))
+    X, Q0, dy = f64(w.X), f64(w.Q0), f64(dY)
+    Wk, Wv, Wks, Wvs = (f64(a) for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn))
+    Kt, Vt = r(oracle.project(X, Wks, w.H)), r(oracle.project(X, Wvs, w.H))
+    K, V = r(oracle.project(X, Wk, w.H)), r(oracle.project(X, Wv, w.H))
+    Qx = oracle.encode(Q0, Kt, Vt, w.lengths)
+    Z = oracle.encode(Qx, K, V, w.lengths)
+    dK, dQx, dZ = oracle.decode_bwd(K, Qx, Z, dy, w.lengths)
+    dQx_e, dK_e, dV = oracle.encode_bwd(Qx, K, V, dZ, w.lengths)
+    dQ0, dKt, dVt = oracle.encode_bwd(Q0, Kt, Vt, dQx + dQx_e, w.lengths)
+    out = {"dQ0": dQ0, "dX": np.zeros_like(X)}
+    for nm, W, d in (("dWk", Wk, dK + dK_e), ("dWv", Wv, dV), ("dWk_syn", Wks, dKt), ("dWv_syn", Wvs, dVt)):
+        dXi, out[nm] = oracle.project_bwd(X, W, d)
+        out["dX"] += dXi
+    return out
+
+
+def test_flarepp_backward_sharp_matches_bf16_storage_model():
+    """Diagnostic with all weights ~ N(0, 16/C) (not a graded workload): the
+    sharp softmaxes make the gradients sensitive to the bf16 storage of the
+    projections, which alone moves them by several percent from the exact
+    fp64 values.  The GPU must match the storage model to the standard
+    tolerance; its distance to the exact gradients is reported."""
+    w = make_workload("flarepp_n8k_sharp", N=1200, B=2)
+    dY = make_upstream_grad(w)
+    got = run_flarepp_bwd(w, dY)
+    model = storage_model_bwd(w, dY)
+    exact = oracle.backward_workload(w, dY)
+    for k in ("dX", "dWk", "dWv", "dWk_syn", "dWv_syn", "dQ0"):
+        print(f"sharp {k}: storage model vs exact {rel_l2(model[k], exact[k]):.3e}, "
+              f"gpu vs exact {rel_l2(got[k], exact[k]):.3e}")
+        check(got[k], model[k], f"sharp {k} vs storage model")
+
+
+def test_flarepp_backward_shared_projections():
+    """Wk_syn is Wk and Wv_syn is Wv: the shared weights get the sum of both
+    uses; the oracle with two identical copies gives the reference."""
+    w = make_workload("flarepp_n1k", N=700)
+    w.Wk_syn, w.Wv_syn = w.Wk.copy(), w.Wv.copy()
+    dY = make_upstream_grad(w)
+    got = run_flarepp_bwd(w, dY, shared=True)
+    ref = oracle.backward_workload(w, dY)
+    check(got["dWk"], ref["dWk"] + ref["dWk_syn"], "shared dWk")
+    check(got["dWv"], ref["dWv"] + ref["dWv_syn"], "shared dWv")
+    assert np.array_equal(got["dWk"], got["dWk_syn"]) and np.array_equal(got["dWv"], got["dWv_syn"])
+    check(got["dX"], ref["dX"], "shared dX")
+    check(got["dQ0"], ref["dQ0"], "shared dQ0")
+
+
+def test_backward_is_deterministic():
+    w = make_workload("flarepp_n8k_mesh2d", N=2048, B=2)
+    dY = make_upstream_grad(w)
+    a = run_flarepp_bwd(w, dY)
+    b = run_flarepp_bwd(w, dY)
+    for k in a:
+        assert np.array_equal(a[k], b[k]), k
+
+
+def test_backward_reports_bad_lengths():
+    w = make_workload("flarepp_n1k", N=256)
+    w.lengths = np.array([300], dtype=np.int32)     # > N: clamped, reported
+    dY = make_upstream_grad(w)
+    ws = torch.empty(fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLAREPP_BWD, w.B, w.H, w.N, w.M, w.D, w.C),
+                     dtype=torch.uint8, device="cuda")
+    fl.flarepp_mixer_bwd(dev_bf16(w.X), dev_bf16(w.Wk), dev_bf16(w.Wv), dev_bf16(w.Wk_syn), dev_bf16(w.Wv_syn),
+                         dev_bf16(w.Q0), dev_bf16(dY), lengths=lengths_dev(w), workspace=ws)
+    assert fl.flare_last_device_status(ws) == fl.Status.ERR_SHAPE

@@ -34,6 +34,7 @@ __all__ = [
     "WORKLOADS",
     "Workload",
     "make_workload",
+    "make_upstream_grad",
     "to_bf16_bits",
     "bf16_bits_to_f64",
     "bf16_bits_to_f32",
@@ -181,3 +182,13 @@ def make_workload(name: str, N: Optional[int] = None, B: Optional[int] = None,
     if spec["variant"] == "flarepp":  # drawn last, so the draws above do not depend on it
         w.Wo = to_bf16_bits(rng.standard_normal((C, C), dtype=np.float32) * wstd)
     return w
+
+
+def make_upstream_grad(w: Workload, seed: Optional[int] = None) -> np.ndarray:
+    """Upstream gradient dY = dLoss/dY [B][H][N][D] for the backward, N(0,1)
+    in bf16 bits, from its own generator (seed: the workload's seed + 7919,
+    unless given), so the workload's draws are unchanged.  Rows of padding
+    tokens are drawn too: the backward must ignore them."""
+    s = w.seed + 7919 if seed is None else int(seed)
+    rng = np.random.Generator(np.random.PCG64(s))
+    return to_bf16_bits(rng.standard_normal((w.B, w.H, w.N, w.D), dtype=np.float32))
