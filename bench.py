@@ -250,6 +250,169 @@ def cpu_model():
 
 
 # ---------------------------------------------------------------------------
+# backward (gradients): a separate line, not the headline
+# ---------------------------------------------------------------------------
+
+BWD_METRIC = "mixer bwd token·heads/s at N=1M (1×B200) and % of roofline (HBM/MMA/MUFU)"
+BWD_LAUNCHES = 23   # kernels per FLARE++ backward call (projections, recompute, gradients, GEMMs)
+TF32_PER_BF16 = 0.5  # nominal dense tf32 : bf16 tensor throughput
+
+
+def backward_work(w):
+    """Algorithmic work of the FLARE++ backward per call: one exponential per
+    score of each of the three SDPA calls; per call the score recompute and
+    the four gradient products (5 x 2MD flop per token·head), the projection
+    gradients dX and dW (2 x 4 x 2 C D flop per token·head); HBM: read X and
+    dY, write dX."""
+    th = w.B * w.H * w.N
+    return {"exps": 3 * w.M * th, "flops": (3 * 5 * 2 * w.M * w.D + 16 * w.C * w.D) * th,
+            "bytes": 3 * w.B * w.N * w.C * 2}
+
+
+def oracle_backward_rate(w, dY, target_s: float):
+    import oracle
+    from workloads import bf16_bits_to_f64 as f64
+    oracle.build()
+    W = [f64(a) for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn)]
+    Q0 = f64(w.Q0)
+
+    def run(ns):
+        t0 = time.perf_counter()
+        oracle.flarepp_backward(f64(w.X[:, :ns]), *W, Q0, f64(dY[:, :, :ns]), w.H, None, w.scale)
+        return time.perf_counter() - t0
+
+    ns = min(2048, w.N)
+    t = run(ns)
+    while t < target_s / 4 and ns < w.N:
+        ns = min(w.N, int(ns * min(8.0, max(2.0, target_s / max(t, 1e-3)))))
+        t = run(ns)
+    return w.B * w.H * ns / t, ns, t, oracle.num_threads()
+
+
+def run_backward(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import rank_latent_routing_flare_b200 as fl
+    from workloads import make_upstream_grad
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    fl.load_library()
+    w = make_workload(args.workload, N=args.tokens, seed=rank_seed(rank))
+    assert w.variant == "flarepp"
+    dY_bits = make_upstream_grad(w)
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    X, Q0, dY = to_dev(w.X), to_dev(w.Q0), to_dev(dY_bits)
+    Ws = [to_dev(a) for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn)]
+    lengths = None if w.lengths is None else torch.from_numpy(w.lengths).to(dev)
+    nbytes = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLAREPP_BWD, w.B, w.H, w.N, w.M, w.D, w.C)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    grads = None
+
+    def step():
+        nonlocal grads
+        grads = fl.flarepp_mixer_bwd(X, *Ws, Q0, dY, lengths=lengths, workspace=ws, stream=stream, grads=grads,
+                                     check=False)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st = fl.flare_last_device_status(ws)
+    if st != fl.Status.OK:
+        raise RuntimeError(f"device status after warm-up: {st!r}")
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world, dev)
+    th_per_rank = w.B * w.H * (w.valid_tokens() // w.B if w.lengths is not None else w.N)
+    value = whole_job_rate(world, th_per_rank, ms)
+
+    peaks = load_peaks()
+    mufu_peak = MUFU_PER_CLK_PER_SM * NUM_SM * peaks["sm_max_mhz"] * 1e6
+    tf32_peak = peaks["bf16_tflops"] * 1e12 * TF32_PER_BF16
+    wk = backward_work(w)
+    terms = {"hbm": wk["bytes"] / (peaks["hbm_gbs"] * 1e9), "mma_tf32": wk["flops"] / tf32_peak,
+             "mufu": wk["exps"] / mufu_peak}
+    t_roof = max(terms.values())
+    bound = {"hbm": "hbm", "mma_tf32": "tensor", "mufu": "alu"}[max(terms, key=terms.get)]
+
+    # end to end: inputs and dY in from pinned host memory, gradients back out,
+    # all inside the timed region on the call's stream
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).pin_memory()  # noqa: E731
+    h_in = [pin(a) for a in (w.X, w.Wk, w.Wv, w.Wk_syn, w.Wv_syn, w.Q0, dY_bits)]
+    d_in = [t.view(torch.int16) for t in (X, *Ws, Q0, dY)]
+    h_out = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in grads.items()}
+    h2d = sum(a.numel() * 2 for a in h_in)
+    d2h = sum(v.numel() * v.element_size() for v in grads.values())
+
+    def e2e_step():
+        for d, h in zip(d_in, h_in):
+            d.copy_(h, non_blocking=True)
+        step()
+        for k, v in grads.items():
+            h_out[k].copy_(v, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(max(1, args.e2e_steps)):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / max(1, args.e2e_steps), world, dev)
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            rate, ns, t, threads = oracle_backward_rate(w, dY_bits, args.cpu_seconds)
+            cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+                   "sample": f"fp64 oracle, full FLARE++ backward on the first {ns} of {w.N} tokens "
+                             f"(B={w.B} H={w.H} M={w.M} D={w.D} C={w.C}) in {t:.1f} s; {cpu_model()}"}
+        line = {
+            "metric": BWD_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "tf32", "data": "synthetic",
+            "config": {"workload": w.name, "pass": "backward", "B": w.B, "N": w.N, "C": w.C, "H": w.H,
+                       "D": w.D, "M": w.M, "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": "inputs larger than L2 (X 256 MiB, dY 256 MiB, fp32 gradient rows 2 GiB)"},
+            "step_roofline": {"t_roof_ms": round(t_roof * 1e3, 4), "frac": round(t_roof / (ms * 1e-3), 4),
+                              "bound": bound, "terms_ms": {k: round(v * 1e3, 4) for k, v in terms.items()},
+                              "peak_basis": f"MUFU {MUFU_PER_CLK_PER_SM} ex2/clk/SM x {NUM_SM} x "
+                                            f"{peaks['sm_max_mhz']:.0f} MHz; tf32 = {TF32_PER_BF16} x measured "
+                                            f"bf16 {peaks['bf16_tflops']} TFLOP/s; HBM {peaks['hbm_gbs']} GB/s "
+                                            f"({peaks['source']})"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": whole_job_rate(world, th_per_rank, e2e_ms), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": BWD_LAUNCHES * args.steps,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+# ---------------------------------------------------------------------------
 # reference arm: the oracle timed as it stands
 # ---------------------------------------------------------------------------
 
@@ -304,6 +467,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the FLARE++ backward (gradients) instead of the forward; its own JSON line")
     ap.add_argument("--graph", action="store_true",
                     help="time replays of one step captured as a CUDA graph (no per-launch host cost); the "
                          "stage times then come from as many eager steps run after the timed region")
@@ -317,6 +482,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.backward:
+        return run_backward(args, rank, world, local_rank)
 
     import torch
     import torch.distributed as dist

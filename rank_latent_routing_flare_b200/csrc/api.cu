@@ -151,19 +151,22 @@ struct BwdPlan {
   int S = 1, tps = 1, rpb = 32, LB = 1, dw_splits = 1;
   size_t off_q32 = 0, off_qx32 = 0, off_lsyn = 0, off_dqx32 = 0, off_gsyn = 0, off_z32 = 0, off_lenc = 0,
          off_ltok = 0, off_dtok = 0, off_dz32 = 0, off_gam = 0, off_fpart = 0, off_pa = 0, off_pb = 0, off_pc = 0,
-         off_g32 = 0, off_dwpart = 0, total = 0;
+         off_g32 = 0, off_dwpart = 0, off_qpad = 0, off_q0pad = 0, off_zpad = 0, off_dzpad = 0, off_dqxpad = 0,
+         total = 0;
 };
 
 BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C) {
   BwdPlan bp;
   bp.fwd = make_plan(pp ? FLARE_VARIANT_FLAREPP : FLARE_VARIANT_FLARE, B, H, N, M, D);
   const long BH = B * H;
-  bp.rpb = static_cast<int>(std::min(128L, cdiv(M, 32) * 32));
+  // latent-parallel passes: a warp per 16 latent rows, 2 to 8 warps per CTA
+  bp.rpb = static_cast<int>(std::min(128L, std::max(32L, cdiv(M, 16) * 16)));
   bp.LB = static_cast<int>(cdiv(M, bp.rpb));
-  // token splits of the latent-parallel passes: about eight CTAs per SM
+  // token splits: whole waves of CTAs (about 128 registers per thread, so
+  // 256 / rows_per_block CTAs per SM), by the encoder's cost model
   const long ntiles = cdiv(N, kBwdTokTile);
-  const long S0 = std::max(1L, std::min(ntiles, cdiv(static_cast<long>(kNumSM) * 8, BH * bp.LB)));
-  bp.tps = static_cast<int>(cdiv(ntiles, S0));
+  bp.S = choose_splits(BH * bp.LB, ntiles, static_cast<long>(kNumSM) * std::max(1, 256 / bp.rpb));
+  bp.tps = static_cast<int>(cdiv(ntiles, bp.S));
   bp.S = static_cast<int>(cdiv(ntiles, bp.tps));
   bp.dw_splits = static_cast<int>(cdiv(B * N, kBwdDwRows));
   size_t off = bp.fwd.total;
@@ -192,6 +195,15 @@ BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C) {
   bp.off_pa = take(part);
   bp.off_pb = take(part);
   bp.off_pc = take(part);
+  // padded tf32 images ([rows][D + 4]) read by the token-parallel pass
+  const size_t padded = static_cast<size_t>(BH * M * (D + 4)) * 4;
+  bp.off_qpad = take(padded);
+  bp.off_zpad = take(padded);
+  bp.off_dzpad = take(padded);
+  if (pp) {
+    bp.off_q0pad = take(static_cast<size_t>(H * M * (D + 4)) * 4);
+    bp.off_dqxpad = take(padded);
+  }
   if (pp) {
     bp.off_g32 = take(static_cast<size_t>(B * N) * 4 * C * 4);
     bp.off_dwpart = take(static_cast<size_t>(bp.dw_splits) * C * 4 * C * 4);
@@ -809,6 +821,11 @@ LatParams lat_params(const BwdPlan& bp, uint8_t* ws, const float* q, int q_per_b
   return lp;
 }
 
+flare_status pad(const float* src, float* dst, long rows, int D, float mul, cudaStream_t s) {
+  const PadParams pp{rows, D, mul, src, dst};
+  return launch_pad(pp, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+}
+
 // Encoder recompute: Z (fp32) and the row log2-normalisers of
 // softmax_n(s Q K^T) V.
 flare_status bwd_encode(const BwdPlan& bp, uint8_t* ws, const float* q, int q_per_batch, const void* k, const void* v,
@@ -841,12 +858,19 @@ flare_status bwd_core(const BwdPlan& bp, uint8_t* ws, const float* q, int q_per_
   // per-token normalisers and delta_n = <dY_n, Y_n>
   flare_status st = bwd_encode(bp, ws, q, q_per_batch, k, v, z32, lenc, B, H, N, M, D, lengths, sc, s);
   if (st != FLARE_OK) return st;
+  const float c = sc * 1.4426950408889634f;
+  float* qpad = reinterpret_cast<float*>(ws + bp.off_qpad);
+  float* zpad = reinterpret_cast<float*>(ws + bp.off_zpad);
+  float* dzpad = reinterpret_cast<float*>(ws + bp.off_dzpad);
+  const long G = q_per_batch ? static_cast<long>(B) * H : H;
+  if ((st = pad(q, qpad, G * M, D, c, s)) != FLARE_OK || (st = pad(z32, zpad, static_cast<long>(B) * H * M, D, 1.f, s)) != FLARE_OK)
+    return st;
   TokParams tp{};
   tp.B = B; tp.H = H; tp.N = N; tp.M = M; tp.D = D;
   tp.q_per_batch = q_per_batch;
   tp.c = sc * 1.4426950408889634f;
   tp.lengths = lengths;
-  tp.q = q; tp.z = z32; tp.dz = dz32; tp.lm = lenc; tp.gam = gam;
+  tp.qpad = qpad; tp.zpad = zpad; tp.dzpad = dzpad; tp.lm = lenc; tp.gam = gam;
   tp.k = static_cast<const uint16_t*>(k);
   tp.v = static_cast<const uint16_t*>(v);
   tp.dy = static_cast<const uint16_t*>(dy);
@@ -862,6 +886,7 @@ flare_status bwd_core(const BwdPlan& bp, uint8_t* ws, const float* q, int q_per_
   if (launch_lat(kLatDecoder, lp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   const LatSumParams sz{B, H, M, D, bp.S, 0, 1.f, pa, nullptr, z32, gam, dz32};
   if (launch_lat_sum(sz, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  if ((st = pad(dz32, dzpad, static_cast<long>(B) * H * M, D, 1.f, s)) != FLARE_OK) return st;
   // dK (both parts) and dV
   if (launch_tok(kTokFull, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   // encoder backward, reduction over tokens: the encoder's dQ
@@ -956,12 +981,17 @@ flare_status flarepp_mixer_bwd(const flare_bf16* X, const flare_bf16* Wk, const 
   const LatSumParams sq{B, H, M, D, bp.S, 0, sc, reinterpret_cast<float*>(ws + bp.off_pb), pc, qx32, gsyn, dqx32};
   if (launch_lat_sum(sq, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   // eq. 8 backward with dQ(X) as the upstream gradient: dK~, dV~ ...
+  float* q0pad = reinterpret_cast<float*>(ws + bp.off_q0pad);
+  float* dqxpad = reinterpret_cast<float*>(ws + bp.off_dqxpad);
+  if ((st = pad(q32, q0pad, static_cast<long>(H) * M, D, sc * 1.4426950408889634f, s)) != FLARE_OK ||
+      (st = pad(dqx32, dqxpad, static_cast<long>(B) * H * M, D, 1.f, s)) != FLARE_OK)
+    return st;
   TokParams tp{};
   tp.B = B; tp.H = H; tp.N = N; tp.M = M; tp.D = D;
   tp.q_per_batch = 0;
   tp.c = sc * 1.4426950408889634f;
   tp.lengths = lengths;
-  tp.q = q32; tp.dz = dqx32; tp.lm = lsyn; tp.gam = gsyn;
+  tp.qpad = q0pad; tp.dzpad = dqxpad; tp.lm = lsyn; tp.gam = gsyn;
   tp.k = pr.kt; tp.v = pr.vt;
   tp.g32 = g32; tp.g_ld = 4 * C; tp.g_col_k = 2 * C; tp.g_col_v = 3 * C;
   tp.err = reinterpret_cast<uint32_t*>(ws + bp.fwd.off_err);

@@ -1,4 +1,6 @@
-// Gradient kernels of the FLARE / FLARE++ mixer, fp32 on the CUDA cores.
+// Gradient kernels of the FLARE / FLARE++ mixer: the score and gradient
+// products on the tensor cores (mma.sync, tf32 operands, fp32 accumulation),
+// softmax weights, normalisers and every reduction in fp32.
 //
 // Every step of the mixer is one SDPA call (FLARE++ paper, arXiv
 // 2608.11519, section "FLARE++: dynamic token routing", eq. 8, 10, 11); the
@@ -31,179 +33,323 @@
 namespace flare {
 namespace {
 
-constexpr int kDH = 16;  // feature dimensions held per thread
 constexpr unsigned kAll = 0xffffffffu;
 constexpr float kLn2 = 0.6931471805599453f;
 
 __device__ __forceinline__ float bf(uint16_t x) { return __uint_as_float(static_cast<uint32_t>(x) << 16); }
 
-__device__ __forceinline__ uint16_t to_bf16(float x) { return static_cast<uint16_t>(pack_bf16x2(x, 0.f) & 0xFFFFu); }
-
-// Sum over the TPR threads of one row (adjacent lanes).
-template <int TPR>
-__device__ __forceinline__ float row_sum(float x) {
-  if (TPR == 2) x += __shfl_xor_sync(kAll, x, 1);
-  return x;
+// ---------------------------------------------------------------------------
+// Tensor-core fragments: mma.sync m16n8k8 with tf32 operands and fp32
+// accumulation.  lane = 4 g + t.  A (16 x 8): a0 (g, t), a1 (g+8, t),
+// a2 (g, t+4), a3 (g+8, t+4).  B (8 x 8): b0 (k t, n g), b1 (k t+4, n g).
+// C (16 x 8): c0 (g, 2t), c1 (g, 2t+1), c2 (g+8, 2t), c3 (g+8, 2t+1).
+// A C tile is reused as the A operand of a second product (over its 8
+// columns) with the k order permuted: A'[.][t] = C[.][2t] and
+// A'[.][t+4] = C[.][2t+1]; the B operand then takes rows 2t and 2t+1.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
 }
 
-__device__ __forceinline__ float dot16(const float (&a)[kDH], const float (&b)[kDH]) {
-  float s = 0.f;
-#pragma unroll
-  for (int i = 0; i < kDH; ++i) s = fmaf(a[i], b[i], s);
-  return s;
+__device__ __forceinline__ void mma8(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// 16 floats from shared memory (16-byte aligned).
-__device__ __forceinline__ void lds16(float (&r)[kDH], const float* p) {
-  const float4* q = reinterpret_cast<const float4*>(p);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float4 t = q[i];
-    r[4 * i] = t.x;
-    r[4 * i + 1] = t.y;
-    r[4 * i + 2] = t.z;
-    r[4 * i + 3] = t.w;
+// A operand from a C tile (k order permuted as above), rounded to tf32.
+__device__ __forceinline__ void c_as_a(uint32_t (&a)[4], float c0, float c1, float c2, float c3) {
+  a[0] = tf32(c0);
+  a[1] = tf32(c2);
+  a[2] = tf32(c1);
+  a[3] = tf32(c3);
+}
+
+__device__ __forceinline__ uint32_t fbits(const float* p) { return __float_as_uint(*p); }
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Quad (the 4 lanes of one fragment row) reductions.
+__device__ __forceinline__ float quad_max(float x) {
+  x = fmaxf(x, __shfl_xor_sync(kAll, x, 1));
+  return fmaxf(x, __shfl_xor_sync(kAll, x, 2));
+}
+__device__ __forceinline__ float quad_sum(float x) {
+  x += __shfl_xor_sync(kAll, x, 1);
+  return x + __shfl_xor_sync(kAll, x, 2);
+}
+
+// Stages rows [0, rows) of a [rows][D] operand into shared memory (row
+// stride LD floats), tf32-rounded, scaled by `mul`; rows >= valid are zero.
+template <int D, int LD>
+__device__ __forceinline__ void stage_f32(float* dst, const float* src, int rows, int valid, float mul) {
+  for (int i = threadIdx.x; i < rows * D; i += blockDim.x) {
+    const int r = i / D, c = i - r * D;
+    dst[r * LD + c] = r < valid ? __uint_as_float(tf32(mul * src[i])) : 0.f;
   }
 }
-
-// 16 bf16 values from global memory (32-byte aligned), widened.
-__device__ __forceinline__ void ldg16_bf16(float (&r)[kDH], const uint16_t* p) {
-  const uint4* q = reinterpret_cast<const uint4*>(p);
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const uint4 t = q[i];
-    const uint32_t w[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      r[8 * i + 2 * j] = bf16_lo(w[j]);
-      r[8 * i + 2 * j + 1] = bf16_hi(w[j]);
-    }
+template <int D, int LD>
+__device__ __forceinline__ void stage_bf16(float* dst, const uint16_t* src, int rows, int valid) {
+  for (int i = threadIdx.x; i < rows * D; i += blockDim.x) {
+    const int r = i / D, c = i - r * D;
+    dst[r * LD + c] = r < valid ? bf(src[i]) : 0.f;  // bf16 values are exact in tf32
   }
 }
 
 // ---------------------------------------------------------------------------
-// Latent-parallel pass: a thread owns one latent row m (D = 32: two threads,
-// 16 dimensions each) and walks the valid tokens of its split in tiles that
-// the CTA stages in shared memory as fp32.
+// Latent-parallel pass: a warp owns 16 latent rows (a CTA 16 per warp) of one
+// head and one token split, and walks the split's valid tokens in tiles of 64
+// that the CTA stages in shared memory.  Per tile and 8-token column block:
+// scores S = (c Q) K^T on the tensor cores, then
+//   forward:  online softmax over tokens, O += 2^(S - max) V
+//   decoder:  W = 2^(S - L_n), dS = W (Z dY^T - delta_n), dZ += W dY, dQ += dS K
+//   encoder:  W = 2^(S - L_m), dS = W (dZ V^T - gamma_m), dQ += dS K
 // ---------------------------------------------------------------------------
 template <int D, int MODE>
 __global__ void __launch_bounds__(256) lat_kernel(const LatParams p) {
-  constexpr int TPR = D / kDH;
-  constexpr int T = kBwdTokTile;
-  __shared__ __align__(16) float sK[T * D];
-  __shared__ __align__(16) float sX[T * D];  // V (forward, encoder) or dY (decoder)
-  __shared__ float sL[T], sDl[T];
+  constexpr int KS = D / 8, LD = D + 4, T = kBwdTokTile, NT = T / 8;
+  // two buffers: the next tile is loaded into registers while this one is
+  // used, and stored after it (one barrier per tile)
+  constexpr int PV = (T * D / 8 + 63) / 64;  // 16-byte words per thread and operand (>= 64 threads)
+  __shared__ __align__(16) float sKb[2][T * LD];
+  __shared__ __align__(16) float sXb[2][T * LD];  // V (forward, encoder) or dY (decoder)
+  __shared__ float sLb[2][T], sDlb[2][T];
 
-  const int tid = threadIdx.x;
-  const int row = tid / TPR, part = tid % TPR;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int split = blockIdx.x, bh = blockIdx.z;
-  const int m = blockIdx.y * p.rows_per_block + row;
-  const bool active = m < p.M;
+  const int m0 = blockIdx.y * p.rows_per_block + warp * 16 + g, m1 = m0 + 8;
+  const bool act0 = m0 < p.M, act1 = m1 < p.M;
   const int b = bh / p.H, h = bh % p.H;
-  const int g = p.q_per_batch ? bh : h;
+  const int gq = p.q_per_batch ? bh : h;
   bool bad = false;
   const int L = shard_valid_len(p.lengths, b, p.N, 0, p.N, &bad);
-  if (bad && tid == 0 && split == 0 && blockIdx.y == 0) atomicOr(p.err, FLARE_DEV_BAD_LENGTH);
+  if (bad && threadIdx.x == 0 && split == 0 && blockIdx.y == 0) atomicOr(p.err, FLARE_DEV_BAD_LENGTH);
   const int ntv = (L + T - 1) / T;
   const int t_begin = split * p.tiles_per_split;
   const int t_end = min(t_begin + p.tiles_per_split, ntv);
 
-  // this thread's query (log2-scaled) and row vector; inactive rows compute
-  // on zeros (every thread takes part in the shuffles) and write nothing
-  float qv[kDH], zv[kDH], accA[kDH], accB[kDH];
-  const size_t qoff = (static_cast<size_t>(g) * p.M + (active ? m : 0)) * D + part * kDH;
-  const size_t roff = (static_cast<size_t>(bh) * p.M + (active ? m : 0)) * D + part * kDH;
+  // A fragments of this warp's rows: log2-scaled queries, and Z (decoder) or
+  // dZ (encoder); rows past M are zero and write nothing
+  uint32_t qa[KS][4], za[KS][4];
+  {
+    const float* q0 = p.q + (static_cast<size_t>(gq) * p.M + (act0 ? m0 : 0)) * D;
+    const float* q1 = p.q + (static_cast<size_t>(gq) * p.M + (act1 ? m1 : 0)) * D;
+    const float* z0 = p.zrow + (static_cast<size_t>(bh) * p.M + (act0 ? m0 : 0)) * D;
+    const float* z1 = p.zrow + (static_cast<size_t>(bh) * p.M + (act1 ? m1 : 0)) * D;
 #pragma unroll
-  for (int i = 0; i < kDH; ++i) {
-    qv[i] = active ? p.c * p.q[qoff + i] : 0.f;
-    zv[i] = (MODE != kLatForward && active) ? p.zrow[roff + i] : 0.f;
-    accA[i] = 0.f;
-    accB[i] = 0.f;
+    for (int ks = 0; ks < KS; ++ks) {
+      const int c = ks * 8 + t;
+      qa[ks][0] = act0 ? tf32(p.c * q0[c]) : 0u;
+      qa[ks][1] = act1 ? tf32(p.c * q1[c]) : 0u;
+      qa[ks][2] = act0 ? tf32(p.c * q0[c + 4]) : 0u;
+      qa[ks][3] = act1 ? tf32(p.c * q1[c + 4]) : 0u;
+      if (MODE != kLatForward) {
+        za[ks][0] = act0 ? tf32(z0[c]) : 0u;
+        za[ks][1] = act1 ? tf32(z1[c]) : 0u;
+        za[ks][2] = act0 ? tf32(z0[c + 4]) : 0u;
+        za[ks][3] = act1 ? tf32(z1[c + 4]) : 0u;
+      }
+    }
   }
-  float mx = -INFINITY, l = 0.f, lrow = 0.f, grow = 0.f;
-  if (MODE == kLatEncoder && active) {
-    lrow = p.lrow[static_cast<size_t>(bh) * p.M + m];
-    grow = p.grow[static_cast<size_t>(bh) * p.M + m];
+  float lr0 = 0.f, lr1 = 0.f, gr0 = 0.f, gr1 = 0.f;
+  if (MODE == kLatEncoder) {
+    const size_t rb = static_cast<size_t>(bh) * p.M;
+    if (act0) { lr0 = p.lrow[rb + m0]; gr0 = p.grow[rb + m0]; }
+    if (act1) { lr1 = p.lrow[rb + m1]; gr1 = p.grow[rb + m1]; }
   }
+  float oa[KS][4], ob[KS][4];  // forward: O; decoder: dZ (oa), dQ (ob); encoder: dQ (ob)
+#pragma unroll
+  for (int nd = 0; nd < KS; ++nd)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) oa[nd][i] = ob[nd][i] = 0.f;
+  float mx0 = -INFINITY, mx1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
   const uint16_t* kh = p.k + static_cast<size_t>(bh) * p.N * D;
   const uint16_t* xh = (MODE == kLatDecoder ? p.dy : p.v) + static_cast<size_t>(bh) * p.N * D;
-  for (int t = t_begin; t < t_end; ++t) {
-    const int n0 = t * T;
-    const int nt = min(T, L - n0);
-    __syncthreads();  // the previous tile has been consumed
-    const uint32_t* k32 = reinterpret_cast<const uint32_t*>(kh + static_cast<size_t>(n0) * D);
-    const uint32_t* x32 = reinterpret_cast<const uint32_t*>(xh + static_cast<size_t>(n0) * D);
-    for (int i = tid; i < T * D / 2; i += blockDim.x) {
-      const bool in = (2 * i) / D < nt;
-      const uint32_t wk = in ? k32[i] : 0u, wx = in ? x32[i] : 0u;
-      reinterpret_cast<float2*>(sK)[i] = make_float2(bf16_lo(wk), bf16_hi(wk));
-      reinterpret_cast<float2*>(sX)[i] = make_float2(bf16_lo(wx), bf16_hi(wx));
+  uint4 pk[PV], px[PV];
+  float pl = 0.f, pd = 0.f;
+  auto fetch = [&](int tile) {  // global -> registers; tokens past L are zero
+    const int n0 = tile * T, nv = min(T, L - n0);
+    const uint4* k16 = reinterpret_cast<const uint4*>(kh + static_cast<size_t>(n0) * D);
+    const uint4* x16 = reinterpret_cast<const uint4*>(xh + static_cast<size_t>(n0) * D);
+#pragma unroll
+    for (int u = 0; u < PV; ++u) {
+      const int i = threadIdx.x + u * blockDim.x;
+      const bool in = i < T * D / 8 && (i * 8) / D < nv;
+      pk[u] = in ? k16[i] : make_uint4(0u, 0u, 0u, 0u);
+      px[u] = in ? x16[i] : make_uint4(0u, 0u, 0u, 0u);
     }
-    if (MODE == kLatDecoder) {
-      for (int j = tid; j < T; j += blockDim.x) {
-        const size_t o = static_cast<size_t>(bh) * p.N + n0 + j;
-        sL[j] = j < nt ? p.ltok[o] : 0.f;
-        sDl[j] = j < nt ? p.dtok[o] : 0.f;
-      }
+    if (MODE == kLatDecoder && threadIdx.x < T) {
+      const size_t o = static_cast<size_t>(bh) * p.N + n0 + threadIdx.x;
+      pl = static_cast<int>(threadIdx.x) < nv ? p.ltok[o] : 0.f;
+      pd = static_cast<int>(threadIdx.x) < nv ? p.dtok[o] : 0.f;
     }
-    __syncthreads();
-    for (int j = 0; j < nt; ++j) {
-      float kj[kDH], xj[kDH];
-      lds16(kj, sK + j * D + part * kDH);
-      lds16(xj, sX + j * D + part * kDH);
-      const float s = row_sum<TPR>(dot16(qv, kj));
-      if (MODE == kLatForward) {
-        // online softmax in log2 units; both threads of a row see the same s
-        if (s > mx) {
-          const float r = ex2_mufu(mx - s);
-          l = fmaf(l, r, 1.f);
+  };
+  auto commit = [&](int buf) {  // registers -> shared memory (fp32; bf16 values are exact in tf32)
 #pragma unroll
-          for (int i = 0; i < kDH; ++i) accA[i] = fmaf(accA[i], r, xj[i]);
-          mx = s;
-        } else {
-          const float w = ex2_mufu(s - mx);
-          l += w;
-#pragma unroll
-          for (int i = 0; i < kDH; ++i) accA[i] = fmaf(w, xj[i], accA[i]);
-        }
-      } else if (MODE == kLatDecoder) {
-        // P[n][m] = 2^(t - L_n); dS = P (<dY_n, Z_m> - delta_n)
-        const float w = ex2_mufu(s - sL[j]);
-        const float ds = w * (row_sum<TPR>(dot16(zv, xj)) - sDl[j]);
-#pragma unroll
-        for (int i = 0; i < kDH; ++i) {
-          accA[i] = fmaf(w, xj[i], accA[i]);
-          accB[i] = fmaf(ds, kj[i], accB[i]);
-        }
-      } else {
-        // A[m][n] = 2^(t - L_m); dS = A (<dZ_m, V_n> - gamma_m)
-        const float w = ex2_mufu(s - lrow);
-        const float ds = w * (row_sum<TPR>(dot16(zv, xj)) - grow);
-#pragma unroll
-        for (int i = 0; i < kDH; ++i) accB[i] = fmaf(ds, kj[i], accB[i]);
-      }
+    for (int u = 0; u < PV; ++u) {
+      const int i = threadIdx.x + u * blockDim.x;
+      if (i >= T * D / 8) continue;
+      const int e = i * 8, r = e / D, c = e - r * D;
+      const uint32_t wk[4] = {pk[u].x, pk[u].y, pk[u].z, pk[u].w};
+      const uint32_t wx[4] = {px[u].x, px[u].y, px[u].z, px[u].w};
+      float4* dk = reinterpret_cast<float4*>(&sKb[buf][r * LD + c]);
+      float4* dx = reinterpret_cast<float4*>(&sXb[buf][r * LD + c]);
+      dk[0] = make_float4(bf16_lo(wk[0]), bf16_hi(wk[0]), bf16_lo(wk[1]), bf16_hi(wk[1]));
+      dk[1] = make_float4(bf16_lo(wk[2]), bf16_hi(wk[2]), bf16_lo(wk[3]), bf16_hi(wk[3]));
+      dx[0] = make_float4(bf16_lo(wx[0]), bf16_hi(wx[0]), bf16_lo(wx[1]), bf16_hi(wx[1]));
+      dx[1] = make_float4(bf16_lo(wx[2]), bf16_hi(wx[2]), bf16_lo(wx[3]), bf16_hi(wx[3]));
     }
+    if (MODE == kLatDecoder && threadIdx.x < T) {
+      sLb[buf][threadIdx.x] = pl;
+      sDlb[buf][threadIdx.x] = pd;
+    }
+  };
+  if (t_begin < t_end) {
+    fetch(t_begin);
+    commit(0);
   }
-  if (!active) return;
-  const size_t base = (static_cast<size_t>(bh) * p.n_splits + split) * p.M + m;
+  __syncthreads();
+  for (int tile = t_begin; tile < t_end; ++tile) {
+    const int buf = (tile - t_begin) & 1;
+    const int n0 = tile * T;
+    const int nv = min(T, L - n0);
+    const bool more = tile + 1 < t_end;
+    if (more) fetch(tile + 1);
+    const float* sK = sKb[buf];
+    const float* sX = sXb[buf];
+    const float* sL = sLb[buf];
+    const float* sDl = sDlb[buf];
+
+    float s[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) s[nt][i] = 0.f;
+      const float* kr = sK + (nt * 8 + g) * LD;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) mma8(s[nt], qa[ks], fbits(kr + ks * 8 + t), fbits(kr + ks * 8 + t + 4));
+    }
+    if (MODE == kLatForward) {
+      float tm0 = -INFINITY, tm1 = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int ca = nt * 8 + 2 * t;
+        if (ca >= nv) { s[nt][0] = -INFINITY; s[nt][2] = -INFINITY; }
+        if (ca + 1 >= nv) { s[nt][1] = -INFINITY; s[nt][3] = -INFINITY; }
+        tm0 = fmaxf(tm0, fmaxf(s[nt][0], s[nt][1]));
+        tm1 = fmaxf(tm1, fmaxf(s[nt][2], s[nt][3]));
+      }
+      tm0 = quad_max(tm0);
+      tm1 = quad_max(tm1);
+      const float nm0 = fmaxf(mx0, tm0), nm1 = fmaxf(mx1, tm1);  // finite: the tile holds a valid token
+      const float r0 = ex2_mufu(mx0 - nm0), r1 = ex2_mufu(mx1 - nm1);
+      mx0 = nm0;
+      mx1 = nm1;
+      l0 *= r0;
+      l1 *= r1;
+#pragma unroll
+      for (int nd = 0; nd < KS; ++nd) {
+        oa[nd][0] *= r0; oa[nd][1] *= r0;
+        oa[nd][2] *= r1; oa[nd][3] *= r1;
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const float p0 = ex2_mufu(s[nt][0] - nm0), p1 = ex2_mufu(s[nt][1] - nm0);
+        const float p2 = ex2_mufu(s[nt][2] - nm1), p3 = ex2_mufu(s[nt][3] - nm1);
+        l0 += p0 + p1;
+        l1 += p2 + p3;
+        uint32_t pa[4];
+        c_as_a(pa, p0, p1, p2, p3);
+        const float* v0 = sX + (nt * 8 + 2 * t) * LD + g;
+#pragma unroll
+        for (int nd = 0; nd < KS; ++nd) mma8(oa[nd], pa, fbits(v0 + nd * 8), fbits(v0 + LD + nd * 8));
+      }
+    } else {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float gg[4] = {0.f, 0.f, 0.f, 0.f};
+        const float* xr = sX + (nt * 8 + g) * LD;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) mma8(gg, za[ks], fbits(xr + ks * 8 + t), fbits(xr + ks * 8 + t + 4));
+        const int ca = nt * 8 + 2 * t;
+        const bool va = ca < nv, vb = ca + 1 < nv;
+        float w[4], ds[4];
+        if (MODE == kLatDecoder) {
+          // W = 2^(S - L_n) per token column, dS = W (<Z_m, dY_n> - delta_n)
+          const float la = sL[ca], lb = sL[ca + 1], da = sDl[ca], db = sDl[ca + 1];
+          w[0] = va ? ex2_mufu(s[nt][0] - la) : 0.f;
+          w[1] = vb ? ex2_mufu(s[nt][1] - lb) : 0.f;
+          w[2] = va ? ex2_mufu(s[nt][2] - la) : 0.f;
+          w[3] = vb ? ex2_mufu(s[nt][3] - lb) : 0.f;
+          ds[0] = w[0] * (gg[0] - da);
+          ds[1] = w[1] * (gg[1] - db);
+          ds[2] = w[2] * (gg[2] - da);
+          ds[3] = w[3] * (gg[3] - db);
+          uint32_t wa[4];
+          c_as_a(wa, w[0], w[1], w[2], w[3]);
+          const float* y0 = sX + (nt * 8 + 2 * t) * LD + g;
+#pragma unroll
+          for (int nd = 0; nd < KS; ++nd) mma8(oa[nd], wa, fbits(y0 + nd * 8), fbits(y0 + LD + nd * 8));
+        } else {
+          // W = 2^(S - L_m) per latent row, dS = W (<dZ_m, V_n> - gamma_m)
+          w[0] = va ? ex2_mufu(s[nt][0] - lr0) : 0.f;
+          w[1] = vb ? ex2_mufu(s[nt][1] - lr0) : 0.f;
+          w[2] = va ? ex2_mufu(s[nt][2] - lr1) : 0.f;
+          w[3] = vb ? ex2_mufu(s[nt][3] - lr1) : 0.f;
+          ds[0] = w[0] * (gg[0] - gr0);
+          ds[1] = w[1] * (gg[1] - gr0);
+          ds[2] = w[2] * (gg[2] - gr1);
+          ds[3] = w[3] * (gg[3] - gr1);
+        }
+        uint32_t da4[4];
+        c_as_a(da4, ds[0], ds[1], ds[2], ds[3]);
+        const float* k0 = sK + (nt * 8 + 2 * t) * LD + g;
+#pragma unroll
+        for (int nd = 0; nd < KS; ++nd) mma8(ob[nd], da4, fbits(k0 + nd * 8), fbits(k0 + LD + nd * 8));
+      }
+    }
+    if (more) commit(buf ^ 1);
+    __syncthreads();
+  }
+
+  // partials of rows m0 (c0, c1) and m1 (c2, c3)
+  const size_t base0 = (static_cast<size_t>(bh) * p.n_splits + split) * p.M + m0;
+  const size_t base1 = base0 + 8;
   if (MODE == kLatForward) {
-    float* o = p.part_a + base * (D + 2);
-    if (part == 0) {
-      o[0] = mx;
-      o[1] = l;
+    l0 = quad_sum(l0);
+    l1 = quad_sum(l1);
+    float* o0 = p.part_a + base0 * (D + 2);
+    float* o1 = p.part_a + base1 * (D + 2);
+    if (t == 0) {
+      if (act0) { o0[0] = mx0; o0[1] = l0; }
+      if (act1) { o1[0] = mx1; o1[1] = l1; }
     }
 #pragma unroll
-    for (int i = 0; i < kDH; ++i) o[2 + part * kDH + i] = accA[i];
+    for (int nd = 0; nd < KS; ++nd) {
+      const int c = 2 + nd * 8 + 2 * t;
+      if (act0) { o0[c] = oa[nd][0]; o0[c + 1] = oa[nd][1]; }
+      if (act1) { o1[c] = oa[nd][2]; o1[c + 1] = oa[nd][3]; }
+    }
   } else {
-    if (MODE == kLatDecoder) {
-      float4* oa = reinterpret_cast<float4*>(p.part_a + base * D + part * kDH);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) oa[i] = make_float4(accA[4 * i], accA[4 * i + 1], accA[4 * i + 2], accA[4 * i + 3]);
+    for (int nd = 0; nd < KS; ++nd) {
+      const int c = nd * 8 + 2 * t;
+      if (MODE == kLatDecoder) {
+        if (act0) *reinterpret_cast<float2*>(p.part_a + base0 * D + c) = make_float2(oa[nd][0], oa[nd][1]);
+        if (act1) *reinterpret_cast<float2*>(p.part_a + base1 * D + c) = make_float2(oa[nd][2], oa[nd][3]);
+      }
+      if (act0) *reinterpret_cast<float2*>(p.part_b + base0 * D + c) = make_float2(ob[nd][0], ob[nd][1]);
+      if (act1) *reinterpret_cast<float2*>(p.part_b + base1 * D + c) = make_float2(ob[nd][2], ob[nd][3]);
     }
-    float4* ob = reinterpret_cast<float4*>(p.part_b + base * D + part * kDH);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) ob[i] = make_float4(accB[4 * i], accB[4 * i + 1], accB[4 * i + 2], accB[4 * i + 3]);
   }
 }
 
@@ -278,249 +424,363 @@ __global__ void __launch_bounds__(256) lat_sum_kernel(const LatSumParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// Token-parallel pass: a thread owns one token row (D = 32: two threads) and
-// walks all latents in chunks that the CTA stages in shared memory.
+// Token-parallel pass: a warp owns 16 token rows (a CTA 128) of one head and
+// walks all latents in chunks of 64 that the CTA stages in shared memory.
+// Per 8-latent column block, on the tensor cores: S = K (c Q)^T, and
+//   stats:    online softmax over latents, Y += 2^(S - max) Z; at the end
+//             L_n = log2 sum 2^S and delta_n = <dY_n, Y_n>
+//   full:     A = 2^(S - L_m), P = 2^(S - L_n), dA = V dZ^T, dP = dY Z^T,
+//             dS = A (dA - gamma_m) + P (dP - delta_n), dK += dS (c Q),
+//             dV += A dZ
+//   encoder:  the A terms alone (query synthesis: no decoder)
 // ---------------------------------------------------------------------------
 template <int D, int MODE>
 __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
-  constexpr int TPR = D / kDH;
-  constexpr int MC = kBwdLatChunk;
-  __shared__ __align__(16) float sQ[MC * D];   // log2-scaled queries
-  __shared__ __align__(16) float sA[MC * D];   // Z (stats) or dZ
-  __shared__ __align__(16) float sZ[MC * D];   // Z (full)
-  __shared__ float sLm[MC], sG[MC];
+  constexpr int KS = D / 8, LD = D + 4, MC = tok_chunk(D);
+  // two chunk buffers, filled by cp.async from the padded tf32 copies while
+  // the other chunk is used (one barrier per chunk)
+  __shared__ __align__(16) float sQb[2][MC * LD];  // log2-scaled queries
+  __shared__ __align__(16) float sAb[2][MC * LD];  // Z (stats) or dZ
+  __shared__ __align__(16) float sZb[2][MC * LD];  // Z (full)
+  __shared__ __align__(16) float sLmb[2][MC], sGb[2][MC];
 
-  const int tid = threadIdx.x, row = tid / TPR, part = tid % TPR;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
-  const int g = p.q_per_batch ? bh : h;
-  const int n = blockIdx.x * kBwdTokBlock + row;
+  const int gq = p.q_per_batch ? bh : h;
+  const int r0 = blockIdx.x * kBwdTokBlock + warp * 16 + g, r1 = r0 + 8;
   bool bad = false;
   const int L = shard_valid_len(p.lengths, b, p.N, 0, p.N, &bad);
-  const bool in_range = n < p.N;
-  const bool valid = n < L;
-  const size_t tok = static_cast<size_t>(bh) * p.N + (in_range ? n : 0);
+  const bool in0 = r0 < p.N, in1 = r1 < p.N;
+  const size_t tok0 = static_cast<size_t>(bh) * p.N + (in0 ? r0 : 0);
+  const size_t tok1 = static_cast<size_t>(bh) * p.N + (in1 ? r1 : 0);
 
-  float kv[kDH], vv[kDH], dyv[kDH], accA[kDH], accB[kDH];
-#pragma unroll
-  for (int i = 0; i < kDH; ++i) {
-    kv[i] = vv[i] = dyv[i] = 0.f;
-    accA[i] = accB[i] = 0.f;
-  }
-  if (in_range) {
-    ldg16_bf16(kv, p.k + tok * D + part * kDH);
-    if (MODE != kTokStats) ldg16_bf16(vv, p.v + tok * D + part * kDH);
-    if (MODE != kTokEncoder) ldg16_bf16(dyv, p.dy + tok * D + part * kDH);
-  }
-  float ln = 0.f, dl = 0.f;
-  if (MODE == kTokFull && in_range) {
-    ln = p.ltok[tok];
-    dl = p.dtok[tok];
-  }
-  float mx = -INFINITY, l = 0.f;
-
-  const float* qg = p.q + static_cast<size_t>(g) * p.M * D;
-  const float* zb = p.z + static_cast<size_t>(bh) * p.M * D;
-  const float* dzb = p.dz + static_cast<size_t>(bh) * p.M * D;
-  for (int m0 = 0; m0 < p.M; m0 += MC) {
-    const int mc = min(MC, p.M - m0);
-    __syncthreads();  // the previous chunk has been consumed
-    for (int i = tid; i < mc * D; i += blockDim.x) {
-      sQ[i] = p.c * qg[static_cast<size_t>(m0) * D + i];
-      if (MODE == kTokStats) {
-        sA[i] = zb[static_cast<size_t>(m0) * D + i];
-      } else {
-        sA[i] = dzb[static_cast<size_t>(m0) * D + i];
-        if (MODE == kTokFull) sZ[i] = zb[static_cast<size_t>(m0) * D + i];
-      }
+  const float* qpad = p.qpad + static_cast<size_t>(gq) * p.M * LD;
+  const float* apad = (MODE == kTokStats ? p.zpad : p.dzpad) + static_cast<size_t>(bh) * p.M * LD;
+  const float* zpad = p.zpad + static_cast<size_t>(bh) * p.M * LD;
+  const float* lmh = p.lm + static_cast<size_t>(bh) * p.M;
+  const float* gmh = p.gam + static_cast<size_t>(bh) * p.M;
+  auto issue = [&](int mb, int buf) {
+    const int n16 = min(MC, p.M - mb) * LD / 4;
+    for (int i = threadIdx.x; i < n16; i += blockDim.x) {
+      cp_async16(&sQb[buf][4 * i], qpad + static_cast<size_t>(mb) * LD + 4 * i);
+      cp_async16(&sAb[buf][4 * i], apad + static_cast<size_t>(mb) * LD + 4 * i);
+      if (MODE == kTokFull) cp_async16(&sZb[buf][4 * i], zpad + static_cast<size_t>(mb) * LD + 4 * i);
     }
     if (MODE != kTokStats) {
-      for (int i = tid; i < mc; i += blockDim.x) {
-        sLm[i] = p.lm[static_cast<size_t>(bh) * p.M + m0 + i];
-        sG[i] = p.gam[static_cast<size_t>(bh) * p.M + m0 + i];
+      for (int i = threadIdx.x; i < min(MC, p.M - mb) / 4; i += blockDim.x) {
+        cp_async16(&sLmb[buf][4 * i], lmh + mb + 4 * i);
+        cp_async16(&sGb[buf][4 * i], gmh + mb + 4 * i);
       }
     }
-    __syncthreads();
-    for (int j = 0; j < mc; ++j) {
-      float qj[kDH], aj[kDH];
-      lds16(qj, sQ + j * D + part * kDH);
-      lds16(aj, sA + j * D + part * kDH);
-      const float s = row_sum<TPR>(dot16(kv, qj));
-      if (MODE == kTokStats) {
-        if (s > mx) {
-          const float r = ex2_mufu(mx - s);
-          l = fmaf(l, r, 1.f);
+    cp_async_commit();
+  };
+  issue(0, 0);
+
+  // A fragments of this warp's token rows (bf16 values are exact in tf32)
+  uint32_t ka[KS][4], va[KS][4], ya[KS][4];
+  auto frag = [&](const uint16_t* src, uint32_t (&f)[KS][4]) {
 #pragma unroll
-          for (int i = 0; i < kDH; ++i) accA[i] = fmaf(accA[i], r, aj[i]);
-          mx = s;
-        } else {
-          const float w = ex2_mufu(s - mx);
-          l += w;
+    for (int ks = 0; ks < KS; ++ks) {
+      const int c = ks * 8 + t;
+      f[ks][0] = in0 ? static_cast<uint32_t>(src[tok0 * D + c]) << 16 : 0u;
+      f[ks][1] = in1 ? static_cast<uint32_t>(src[tok1 * D + c]) << 16 : 0u;
+      f[ks][2] = in0 ? static_cast<uint32_t>(src[tok0 * D + c + 4]) << 16 : 0u;
+      f[ks][3] = in1 ? static_cast<uint32_t>(src[tok1 * D + c + 4]) << 16 : 0u;
+    }
+  };
+  frag(p.k, ka);
+  if (MODE != kTokStats) frag(p.v, va);
+  if (MODE == kTokFull) frag(p.dy, ya);
+  float ln0 = 0.f, ln1 = 0.f, dl0 = 0.f, dl1 = 0.f;
+  if (MODE == kTokFull) {
+    if (in0) { ln0 = p.ltok[tok0]; dl0 = p.dtok[tok0]; }
+    if (in1) { ln1 = p.ltok[tok1]; dl1 = p.dtok[tok1]; }
+  }
+  float oa[KS][4], ob[KS][4];  // stats: Y (oa); full, encoder: dK (oa), dV (ob)
 #pragma unroll
-          for (int i = 0; i < kDH; ++i) accA[i] = fmaf(w, aj[i], accA[i]);
+  for (int nd = 0; nd < KS; ++nd)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) oa[nd][i] = ob[nd][i] = 0.f;
+  float mx0 = -INFINITY, mx1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+  for (int mb = 0, it = 0; mb < p.M; mb += MC, ++it) {
+    const int buf = it & 1;
+    const int mc = min(MC, p.M - mb);  // a multiple of 16
+    cp_async_wait_all();
+    __syncthreads();  // chunk `it` has landed; chunk it-1 has been consumed
+    if (mb + MC < p.M) issue(mb + MC, buf ^ 1);
+    const float* sQ = sQb[buf];
+    const float* sA = sAb[buf];
+    const float* sZ = sZb[buf];
+    const float* sLm = sLmb[buf];
+    const float* sG = sGb[buf];
+    const int ntl = mc / 8;
+
+    if (MODE == kTokStats) {
+      float s[MC / 8][4];
+      float tm0 = -INFINITY, tm1 = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < MC / 8; ++nt) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) s[nt][i] = -INFINITY;
+        if (nt < ntl) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) s[nt][i] = 0.f;
+          const float* qr = sQ + (nt * 8 + g) * LD;
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) mma8(s[nt], ka[ks], fbits(qr + ks * 8 + t), fbits(qr + ks * 8 + t + 4));
         }
-      } else {
-        // encoder part: A = 2^(t - L_m), dS = A (<dZ_m, V_n> - gamma_m), dV += A dZ_m
-        const float a = ex2_mufu(s - sLm[j]);
-        float ds = a * (row_sum<TPR>(dot16(vv, aj)) - sG[j]);
+        tm0 = fmaxf(tm0, fmaxf(s[nt][0], s[nt][1]));
+        tm1 = fmaxf(tm1, fmaxf(s[nt][2], s[nt][3]));
+      }
+      tm0 = quad_max(tm0);
+      tm1 = quad_max(tm1);
+      const float nm0 = fmaxf(mx0, tm0), nm1 = fmaxf(mx1, tm1);
+      const float q0 = ex2_mufu(mx0 - nm0), q1 = ex2_mufu(mx1 - nm1);
+      mx0 = nm0;
+      mx1 = nm1;
+      l0 *= q0;
+      l1 *= q1;
 #pragma unroll
-        for (int i = 0; i < kDH; ++i) accB[i] = fmaf(a, aj[i], accB[i]);
+      for (int nd = 0; nd < KS; ++nd) {
+        oa[nd][0] *= q0; oa[nd][1] *= q0;
+        oa[nd][2] *= q1; oa[nd][3] *= q1;
+      }
+#pragma unroll
+      for (int nt = 0; nt < MC / 8; ++nt) {
+        if (nt < ntl) {
+          const float p0 = ex2_mufu(s[nt][0] - nm0), p1 = ex2_mufu(s[nt][1] - nm0);
+          const float p2 = ex2_mufu(s[nt][2] - nm1), p3 = ex2_mufu(s[nt][3] - nm1);
+          l0 += p0 + p1;
+          l1 += p2 + p3;
+          uint32_t pa[4];
+          c_as_a(pa, p0, p1, p2, p3);
+          const float* z0 = sA + (nt * 8 + 2 * t) * LD + g;
+#pragma unroll
+          for (int nd = 0; nd < KS; ++nd) mma8(oa[nd], pa, fbits(z0 + nd * 8), fbits(z0 + LD + nd * 8));
+        }
+      }
+    } else {
+#pragma unroll
+      for (int nt = 0; nt < MC / 8; ++nt) {
+        if (nt >= ntl) continue;
+        float s[4] = {0.f, 0.f, 0.f, 0.f}, da[4] = {0.f, 0.f, 0.f, 0.f};
+        const float* qr = sQ + (nt * 8 + g) * LD;
+        const float* dzr = sA + (nt * 8 + g) * LD;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          mma8(s, ka[ks], fbits(qr + ks * 8 + t), fbits(qr + ks * 8 + t + 4));
+          mma8(da, va[ks], fbits(dzr + ks * 8 + t), fbits(dzr + ks * 8 + t + 4));
+        }
+        const int ca = nt * 8 + 2 * t;
+        const float lma = sLm[ca], lmb = sLm[ca + 1], ga = sG[ca], gb = sG[ca + 1];
+        float a[4], ds[4];
+        a[0] = ex2_mufu(s[0] - lma);
+        a[1] = ex2_mufu(s[1] - lmb);
+        a[2] = ex2_mufu(s[2] - lma);
+        a[3] = ex2_mufu(s[3] - lmb);
+        ds[0] = a[0] * (da[0] - ga);
+        ds[1] = a[1] * (da[1] - gb);
+        ds[2] = a[2] * (da[2] - ga);
+        ds[3] = a[3] * (da[3] - gb);
         if (MODE == kTokFull) {
-          // decoder part: P = 2^(t - L_n), dS += P (<dY_n, Z_m> - delta_n)
-          float zj[kDH];
-          lds16(zj, sZ + j * D + part * kDH);
-          const float pw = ex2_mufu(s - ln);
-          ds = fmaf(pw, row_sum<TPR>(dot16(dyv, zj)) - dl, ds);
-        }
+          float dp[4] = {0.f, 0.f, 0.f, 0.f};
+          const float* zr = sZ + (nt * 8 + g) * LD;
 #pragma unroll
-        for (int i = 0; i < kDH; ++i) accA[i] = fmaf(ds, qj[i], accA[i]);
+          for (int ks = 0; ks < KS; ++ks) mma8(dp, ya[ks], fbits(zr + ks * 8 + t), fbits(zr + ks * 8 + t + 4));
+          ds[0] = fmaf(ex2_mufu(s[0] - ln0), dp[0] - dl0, ds[0]);
+          ds[1] = fmaf(ex2_mufu(s[1] - ln0), dp[1] - dl0, ds[1]);
+          ds[2] = fmaf(ex2_mufu(s[2] - ln1), dp[2] - dl1, ds[2]);
+          ds[3] = fmaf(ex2_mufu(s[3] - ln1), dp[3] - dl1, ds[3]);
+        }
+        uint32_t sa4[4], aa4[4];
+        c_as_a(sa4, ds[0], ds[1], ds[2], ds[3]);
+        c_as_a(aa4, a[0], a[1], a[2], a[3]);
+        const float* q0 = sQ + (nt * 8 + 2 * t) * LD + g;
+        const float* z0 = sA + (nt * 8 + 2 * t) * LD + g;
+#pragma unroll
+        for (int nd = 0; nd < KS; ++nd) {
+          mma8(oa[nd], sa4, fbits(q0 + nd * 8), fbits(q0 + LD + nd * 8));
+          mma8(ob[nd], aa4, fbits(z0 + nd * 8), fbits(z0 + LD + nd * 8));
+        }
       }
     }
   }
 
   if (MODE == kTokStats) {
-    // every thread (also past N) reaches the shuffle; l >= 1 here
-    const float inv = 1.f / l;
-    float y[kDH];
+    // every lane reaches the shuffles; l >= 1 for every row here
+    l0 = quad_sum(l0);
+    l1 = quad_sum(l1);
+    const float i0 = 1.f / l0, i1 = 1.f / l1;
+    float d0 = 0.f, d1 = 0.f;
 #pragma unroll
-    for (int i = 0; i < kDH; ++i) y[i] = accA[i] * inv;
-    const float delta = row_sum<TPR>(dot16(dyv, y));
-    if (in_range && part == 0) {
-      p.ltok[tok] = valid ? mx + __log2f(l) : 0.f;
-      p.dtok[tok] = valid ? delta : 0.f;
+    for (int nd = 0; nd < KS; ++nd) {
+      const int c = nd * 8 + 2 * t;
+      if (in0) d0 += bf(p.dy[tok0 * D + c]) * (oa[nd][0] * i0) + bf(p.dy[tok0 * D + c + 1]) * (oa[nd][1] * i0);
+      if (in1) d1 += bf(p.dy[tok1 * D + c]) * (oa[nd][2] * i1) + bf(p.dy[tok1 * D + c + 1]) * (oa[nd][3] * i1);
+    }
+    d0 = quad_sum(d0);
+    d1 = quad_sum(d1);
+    if (t == 0) {
+      if (in0) { p.ltok[tok0] = r0 < L ? mx0 + __log2f(l0) : 0.f; p.dtok[tok0] = r0 < L ? d0 : 0.f; }
+      if (in1) { p.ltok[tok1] = r1 < L ? mx1 + __log2f(l1) : 0.f; p.dtok[tok1] = r1 < L ? d1 : 0.f; }
     }
     return;
   }
-  if (!in_range) return;
-  // dK = scale sum dS q = ln2 sum dS (scale log2(e) q); masked tokens get zeros
+  // dK = scale sum dS q = ln2 sum dS (scale log2(e) q); padding tokens get zeros
+  const bool v0 = r0 < L, v1 = r1 < L;
 #pragma unroll
-  for (int i = 0; i < kDH; ++i) {
-    accA[i] = valid ? accA[i] * kLn2 : 0.f;
-    accB[i] = valid ? accB[i] : 0.f;
-  }
-  if (p.g32 != nullptr) {
-    float* o = p.g32 + (static_cast<size_t>(b) * p.N + n) * p.g_ld + h * D + part * kDH;
-    float4* ok = reinterpret_cast<float4*>(o + p.g_col_k);
-    float4* ov = reinterpret_cast<float4*>(o + p.g_col_v);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      ok[i] = make_float4(accA[4 * i], accA[4 * i + 1], accA[4 * i + 2], accA[4 * i + 3]);
-      ov[i] = make_float4(accB[4 * i], accB[4 * i + 1], accB[4 * i + 2], accB[4 * i + 3]);
-    }
-  } else {
-    uint4* ok = reinterpret_cast<uint4*>(p.dk16 + tok * D + part * kDH);
-    uint4* ov = reinterpret_cast<uint4*>(p.dv16 + tok * D + part * kDH);
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      ok[i] = make_uint4(pack_bf16x2(accA[8 * i], accA[8 * i + 1]), pack_bf16x2(accA[8 * i + 2], accA[8 * i + 3]),
-                         pack_bf16x2(accA[8 * i + 4], accA[8 * i + 5]), pack_bf16x2(accA[8 * i + 6], accA[8 * i + 7]));
-      ov[i] = make_uint4(pack_bf16x2(accB[8 * i], accB[8 * i + 1]), pack_bf16x2(accB[8 * i + 2], accB[8 * i + 3]),
-                         pack_bf16x2(accB[8 * i + 4], accB[8 * i + 5]), pack_bf16x2(accB[8 * i + 6], accB[8 * i + 7]));
+  for (int nd = 0; nd < KS; ++nd) {
+    const int c = nd * 8 + 2 * t;
+    const float2 k0 = v0 ? make_float2(oa[nd][0] * kLn2, oa[nd][1] * kLn2) : make_float2(0.f, 0.f);
+    const float2 k1 = v1 ? make_float2(oa[nd][2] * kLn2, oa[nd][3] * kLn2) : make_float2(0.f, 0.f);
+    const float2 w0 = v0 ? make_float2(ob[nd][0], ob[nd][1]) : make_float2(0.f, 0.f);
+    const float2 w1 = v1 ? make_float2(ob[nd][2], ob[nd][3]) : make_float2(0.f, 0.f);
+    if (p.g32 != nullptr) {
+      if (in0) {
+        float* o = p.g32 + (static_cast<size_t>(b) * p.N + r0) * p.g_ld + h * D + c;
+        *reinterpret_cast<float2*>(o + p.g_col_k) = k0;
+        *reinterpret_cast<float2*>(o + p.g_col_v) = w0;
+      }
+      if (in1) {
+        float* o = p.g32 + (static_cast<size_t>(b) * p.N + r1) * p.g_ld + h * D + c;
+        *reinterpret_cast<float2*>(o + p.g_col_k) = k1;
+        *reinterpret_cast<float2*>(o + p.g_col_v) = w1;
+      }
+    } else {
+      if (in0) {
+        *reinterpret_cast<uint32_t*>(p.dk16 + tok0 * D + c) = pack_bf16x2(k0.x, k0.y);
+        *reinterpret_cast<uint32_t*>(p.dv16 + tok0 * D + c) = pack_bf16x2(w0.x, w0.y);
+      }
+      if (in1) {
+        *reinterpret_cast<uint32_t*>(p.dk16 + tok1 * D + c) = pack_bf16x2(k1.x, k1.y);
+        *reinterpret_cast<uint32_t*>(p.dv16 + tok1 * D + c) = pack_bf16x2(w1.x, w1.y);
+      }
     }
   }
 }
 
 // ---------------------------------------------------------------------------
-// Projection gradients (eq. 7 and 9 run backwards): 64 x 64 output tiles,
-// 16-deep shared-memory k-steps, 4 x 4 outputs per thread.
+// Projection gradients (eq. 7 and 9 run backwards) on the tensor cores: a CTA
+// of 8 warps computes a 128 x 128 output tile, a warp 16 rows of it, over
+// k-steps of 32 staged in shared memory (fp32, tf32-rounded; bf16 values are
+// exact in tf32).
 // ---------------------------------------------------------------------------
-constexpr int kTK = 16;
-constexpr int kPad = 4;
+constexpr int kGT = 128;       // output tile rows and columns
+constexpr int kGK = 32;        // k-step
+constexpr int kGLD = kGK + 4;  // padded row of a [row][k] tile (conflict-free fragments)
+constexpr int kGLT = kGT + 8;  // padded row of a [k][col] tile
 
 // dX[r][c] = sum_j G[r][j] Wcat[c][j], Wcat = [W_0 | W_1 | ...] (each [C][C]).
+// A = G rows ([row][k] tile), B[k][n] = W_q[c][j] ([c][k] tile).
 __global__ void __launch_bounds__(256) dx_kernel(const DxParams p) {
-  constexpr int TM = kBwdGemmTile, TN = kBwdGemmTile;
-  __shared__ float sG[kTK][TM + kPad];
-  __shared__ float sW[kTK][TN + kPad];
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  const long r0 = static_cast<long>(blockIdx.x) * TM;
-  const int c0 = blockIdx.y * TN;
+  __shared__ __align__(16) float sG[kGT * kGLD];
+  __shared__ __align__(16) float sW[kGT * kGLD];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const long r0 = static_cast<long>(blockIdx.x) * kGT;
+  const int c0 = blockIdx.y * kGT;
   const int J = p.nw * p.C;
-  float acc[4][4] = {};
-  for (int j0 = 0; j0 < J; j0 += kTK) {
-    const int q = j0 / p.C, jj0 = j0 % p.C;
-    for (int e = threadIdx.x; e < TM * kTK; e += blockDim.x) {
-      const int r = e / kTK, k = e % kTK;
-      const long gr = r0 + r;
-      sG[k][r] = gr < p.R ? p.g[gr * J + j0 + k] : 0.f;
+  float acc[kGT / 8][4];
+#pragma unroll
+  for (int nt = 0; nt < kGT / 8; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
+  for (int j0 = 0; j0 < J; j0 += kGK) {
+    const int q = j0 / p.C, jj0 = j0 - q * p.C;
+    __syncthreads();
+    for (int i = threadIdx.x; i < kGT * kGK / 4; i += blockDim.x) {
+      const int row = i / (kGK / 4), c4 = (i - row * (kGK / 4)) * 4;
+      const long gr = r0 + row;
+      float4 v = gr < p.R ? *reinterpret_cast<const float4*>(p.g + gr * J + j0 + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      v = make_float4(__uint_as_float(tf32(v.x)), __uint_as_float(tf32(v.y)), __uint_as_float(tf32(v.z)),
+                      __uint_as_float(tf32(v.w)));
+      *reinterpret_cast<float4*>(&sG[row * kGLD + c4]) = v;
     }
-    for (int e = threadIdx.x; e < TN * kTK; e += blockDim.x) {
-      const int c = e / kTK, k = e % kTK;
-      sW[k][c] = c0 + c < p.C ? bf(p.w[q][static_cast<size_t>(c0 + c) * p.C + jj0 + k]) : 0.f;
+    for (int i = threadIdx.x; i < kGT * kGK / 8; i += blockDim.x) {
+      const int c = i / (kGK / 8), k8 = (i - c * (kGK / 8)) * 8;
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (c0 + c < p.C) w = *reinterpret_cast<const uint4*>(p.w[q] + static_cast<size_t>(c0 + c) * p.C + jj0 + k8);
+      float4* d = reinterpret_cast<float4*>(&sW[c * kGLD + k8]);
+      d[0] = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
+      d[1] = make_float4(bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w));
     }
     __syncthreads();
 #pragma unroll
-    for (int k = 0; k < kTK; ++k) {
-      float a[4], w[4];
+    for (int ks = 0; ks < kGK / 8; ++ks) {
+      const float* ar = sG + (warp * 16 + g) * kGLD + ks * 8 + t;
+      const uint32_t a[4] = {fbits(ar), fbits(ar + 8 * kGLD), fbits(ar + 4), fbits(ar + 8 * kGLD + 4)};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        a[i] = sG[k][ty + 16 * i];
-        w[i] = sW[k][tx + 16 * i];
+      for (int nt = 0; nt < kGT / 8; ++nt) {
+        const float* br = sW + (nt * 8 + g) * kGLD + ks * 8 + t;
+        mma8(acc[nt], a, fbits(br), fbits(br + 4));
       }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], w[j], acc[i][j]);
     }
-    __syncthreads();
   }
+  const long ra = r0 + warp * 16 + g, rb = ra + 8;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const long r = r0 + ty + 16 * i;
-    if (r >= p.R) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = c0 + tx + 16 * j;
-      if (c < p.C) p.dx[r * p.C + c] = to_bf16(acc[i][j]);
-    }
+  for (int nt = 0; nt < kGT / 8; ++nt) {
+    const int c = c0 + nt * 8 + 2 * t;
+    if (c >= p.C) continue;
+    if (ra < p.R) *reinterpret_cast<uint32_t*>(p.dx + ra * p.C + c) = pack_bf16x2(acc[nt][0], acc[nt][1]);
+    if (rb < p.R) *reinterpret_cast<uint32_t*>(p.dx + rb * p.C + c) = pack_bf16x2(acc[nt][2], acc[nt][3]);
   }
 }
 
 // part[split][c][j] = sum over the split's rows r of X[r][c] G[r][j].
+// A[c][k = r] = X[r][c] and B[k = r][j] = G[r][j], both from [k][col] tiles.
 __global__ void __launch_bounds__(256) dw_kernel(const DwParams p) {
-  constexpr int TM = kBwdGemmTile, TN = kBwdGemmTile;
-  __shared__ float sX[kTK][TM + kPad];
-  __shared__ float sG[kTK][TN + kPad];
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  const int c0 = blockIdx.x * TM, j0 = blockIdx.y * TN, split = blockIdx.z;
+  __shared__ __align__(16) float sX[kGK * kGLT];
+  __shared__ __align__(16) float sG[kGK * kGLT];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int c0 = blockIdx.x * kGT, j0 = blockIdx.y * kGT, split = blockIdx.z;
   const long rs = static_cast<long>(split) * kBwdDwRows;
   const long re = min(rs + kBwdDwRows, static_cast<long>(p.R));
-  float acc[4][4] = {};
-  for (long r = rs; r < re; r += kTK) {
-    for (int e = threadIdx.x; e < kTK * TM; e += blockDim.x) {
-      const int k = e / TM, c = e % TM;
-      const long rr = r + k;
-      sX[k][c] = (rr < re && c0 + c < p.C) ? bf(p.x[rr * p.C + c0 + c]) : 0.f;
+  float acc[kGT / 8][4];
+#pragma unroll
+  for (int nt = 0; nt < kGT / 8; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
+  for (long r = rs; r < re; r += kGK) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < kGK * kGT / 8; i += blockDim.x) {
+      const int k = i / (kGT / 8), c8 = (i - k * (kGT / 8)) * 8;
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (r + k < re && c0 + c8 < p.C) w = *reinterpret_cast<const uint4*>(p.x + (r + k) * p.C + c0 + c8);
+      float4* d = reinterpret_cast<float4*>(&sX[k * kGLT + c8]);
+      d[0] = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
+      d[1] = make_float4(bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w));
     }
-    for (int e = threadIdx.x; e < kTK * TN; e += blockDim.x) {
-      const int k = e / TN, j = e % TN;
-      const long rr = r + k;
-      sG[k][j] = (rr < re && j0 + j < p.J) ? p.g[rr * p.J + j0 + j] : 0.f;
+    for (int i = threadIdx.x; i < kGK * kGT / 4; i += blockDim.x) {
+      const int k = i / (kGT / 4), j4 = (i - k * (kGT / 4)) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r + k < re && j0 + j4 < p.J) v = *reinterpret_cast<const float4*>(p.g + (r + k) * p.J + j0 + j4);
+      v = make_float4(__uint_as_float(tf32(v.x)), __uint_as_float(tf32(v.y)), __uint_as_float(tf32(v.z)),
+                      __uint_as_float(tf32(v.w)));
+      *reinterpret_cast<float4*>(&sG[k * kGLT + j4]) = v;
     }
     __syncthreads();
 #pragma unroll
-    for (int k = 0; k < kTK; ++k) {
-      float a[4], w[4];
+    for (int ks = 0; ks < kGK / 8; ++ks) {
+      const float* ar = sX + (ks * 8 + t) * kGLT + warp * 16 + g;
+      const uint32_t a[4] = {fbits(ar), fbits(ar + 8), fbits(ar + 4 * kGLT), fbits(ar + 4 * kGLT + 8)};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        a[i] = sX[k][ty + 16 * i];
-        w[i] = sG[k][tx + 16 * i];
+      for (int nt = 0; nt < kGT / 8; ++nt) {
+        const float* br = sG + (ks * 8 + t) * kGLT + nt * 8 + g;
+        mma8(acc[nt], a, fbits(br), fbits(br + 4 * kGLT));
       }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], w[j], acc[i][j]);
     }
-    __syncthreads();
   }
+  const int ca = c0 + warp * 16 + g, cb = ca + 8;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int c = c0 + ty + 16 * i;
-    if (c >= p.C) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int jj = j0 + tx + 16 * j;
-      if (jj < p.J) p.part[(static_cast<size_t>(split) * p.C + c) * p.J + jj] = acc[i][j];
-    }
+  for (int nt = 0; nt < kGT / 8; ++nt) {
+    const int j = j0 + nt * 8 + 2 * t;
+    if (j >= p.J) continue;
+    if (ca < p.C)
+      *reinterpret_cast<float2*>(p.part + (static_cast<size_t>(split) * p.C + ca) * p.J + j) =
+          make_float2(acc[nt][0], acc[nt][1]);
+    if (cb < p.C)
+      *reinterpret_cast<float2*>(p.part + (static_cast<size_t>(split) * p.C + cb) * p.J + j) =
+          make_float2(acc[nt][2], acc[nt][3]);
   }
 }
 
@@ -540,6 +800,17 @@ __global__ void __launch_bounds__(256) dw_reduce_kernel(const DwReduceParams p) 
   if (p.shared && p.dw[q + 2]) p.dw[q + 2][static_cast<size_t>(c) * p.C + jj] = s;
 }
 
+// dst[r][0..LD) = (tf32(mul * src[r][c]) for c < D, then zeros): the padded
+// shared-memory image of a chunk of rows, copied by the token-parallel pass.
+__global__ void __launch_bounds__(256) pad_kernel(const PadParams p) {
+  const long i = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int ld = p.D + 4;
+  if (i >= p.rows * ld) return;
+  const long r = i / ld;
+  const int c = static_cast<int>(i - r * ld);
+  p.dst[i] = c < p.D ? __uint_as_float(tf32(p.mul * p.src[r * p.D + c])) : 0.f;
+}
+
 __global__ void __launch_bounds__(256) cvt_kernel(const CvtParams p) {
   const long i = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i < p.n) p.dst[i] = bf(p.src[i]);
@@ -551,7 +822,7 @@ unsigned blocks_for(long n, int threads) { return static_cast<unsigned>((n + thr
 
 cudaError_t launch_lat(int mode, const LatParams& p, cudaStream_t s) {
   const dim3 grid(p.n_splits, (p.M + p.rows_per_block - 1) / p.rows_per_block, p.B * p.H);
-  const int threads = p.rows_per_block * (p.D / kDH);
+  const int threads = 2 * p.rows_per_block;  // a warp per 16 latent rows
 #define FLARE_LAT(DD, MM) lat_kernel<DD, MM><<<grid, threads, 0, s>>>(p)
   if (p.D == 16) {
     if (mode == kLatForward) FLARE_LAT(16, kLatForward);
@@ -583,7 +854,7 @@ cudaError_t launch_lat_sum(const LatSumParams& p, cudaStream_t s) {
 
 cudaError_t launch_tok(int mode, const TokParams& p, cudaStream_t s) {
   const dim3 grid((p.N + kBwdTokBlock - 1) / kBwdTokBlock, p.B * p.H);
-  const int threads = kBwdTokBlock * (p.D / kDH);
+  const int threads = 2 * kBwdTokBlock;  // a warp per 16 token rows
 #define FLARE_TOK(DD, MM) tok_kernel<DD, MM><<<grid, threads, 0, s>>>(p)
   if (p.D == 16) {
     if (mode == kTokStats) FLARE_TOK(16, kTokStats);
@@ -599,13 +870,13 @@ cudaError_t launch_tok(int mode, const TokParams& p, cudaStream_t s) {
 }
 
 cudaError_t launch_dx(const DxParams& p, cudaStream_t s) {
-  const dim3 grid(blocks_for(p.R, kBwdGemmTile), blocks_for(p.C, kBwdGemmTile));
+  const dim3 grid(blocks_for(p.R, kGT), blocks_for(p.C, kGT));
   dx_kernel<<<grid, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dw(const DwParams& p, cudaStream_t s) {
-  const dim3 grid(blocks_for(p.C, kBwdGemmTile), blocks_for(p.J, kBwdGemmTile), p.n_splits);
+  const dim3 grid(blocks_for(p.C, kGT), blocks_for(p.J, kGT), p.n_splits);
   dw_kernel<<<grid, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
@@ -613,6 +884,11 @@ cudaError_t launch_dw(const DwParams& p, cudaStream_t s) {
 cudaError_t launch_dw_reduce(const DwReduceParams& p, cudaStream_t s) {
   const long n = static_cast<long>(p.C) * (p.shared ? 2 * p.C : p.J);
   dw_reduce_kernel<<<blocks_for(n, 256), 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pad(const PadParams& p, cudaStream_t s) {
+  pad_kernel<<<blocks_for(p.rows * (p.D + 4), 256), 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 

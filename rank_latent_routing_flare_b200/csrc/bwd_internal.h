@@ -8,13 +8,13 @@ namespace flare {
 
 constexpr int kBwdTokTile = 64;     // tokens per shared-memory tile of the latent-parallel kernels
 constexpr int kBwdTokBlock = 128;   // tokens per CTA of the token-parallel kernels
-constexpr int kBwdLatChunk = 64;    // latents per shared-memory chunk of the token-parallel kernels
-constexpr int kBwdGemmTile = 64;    // output tile (rows and columns) of the projection-gradient GEMMs
+// Latents per shared-memory chunk of the token-parallel kernels (two
+// buffers of three [chunk][D + 4] fp32 operands stay within 48 KB).
+__host__ __device__ constexpr int tok_chunk(int D) { return D == 16 ? 64 : 32; }
 constexpr int kBwdDwRows = 2048;    // token rows per split of the weight-gradient GEMM
 
 // Modes of the latent-parallel kernel (one CTA = a block of latents of one
-// head and one token split; a thread = one latent row, or half of one for
-// D = 32).
+// head and one token split; a warp = 16 latent rows).
 enum LatMode : int {
   kLatForward = 0,   // encoder recompute: per split (max, sum, sum w v) in log2 units
   kLatDecoder = 1,   // decoder backward, reductions over tokens: dZ and dQ
@@ -24,7 +24,7 @@ enum LatMode : int {
 struct LatParams {
   int B, H, N, M, D;
   int q_per_batch;              // queries [G][M][D] with G = B*H (1) or H (0)
-  int n_splits, tiles_per_split, rows_per_block;
+  int n_splits, tiles_per_split, rows_per_block;   // rows_per_block: 16 per warp, at most 128
   float c;                      // scale * log2(e)
   const int32_t* lengths;
   const float* q;               // fp32 queries [G][M][D]
@@ -60,7 +60,7 @@ struct LatSumParams {
 };
 
 // Modes of the token-parallel kernel (one CTA = kBwdTokBlock tokens of one
-// head; a thread = one token row, or half of one for D = 32).
+// head; a warp = 16 token rows).
 enum TokMode : int {
   kTokStats = 0,     // decoder recompute: per-token log2-normaliser and delta = <dY, Y>
   kTokFull = 1,      // dK (decoder + encoder parts) and dV
@@ -72,9 +72,10 @@ struct TokParams {
   int q_per_batch;
   float c;
   const int32_t* lengths;
-  const float* q;               // fp32 queries [G][M][D]
-  const float* z;               // Z [B*H][M][D] (stats, full)
-  const float* dz;              // dZ [B*H][M][D] (full, encoder)
+  // padded tf32 images ([rows][D + 4], see PadParams)
+  const float* qpad;            // log2-scaled queries [G][M][D + 4]
+  const float* zpad;            // Z [B*H][M][D + 4] (stats, full)
+  const float* dzpad;           // dZ [B*H][M][D + 4] (full, encoder)
   const float* lm;              // encoder row log2-normaliser [B*H][M]
   const float* gam;             // gamma [B*H][M]
   const uint16_t *k, *v, *dy;   // bf16 [B*H][N][D]
@@ -111,6 +112,15 @@ struct DwReduceParams {
   float* dw[4];                 // [C][C] fp32 each (dWk, dWv, dWk_syn, dWv_syn); NULL = not written
 };
 
+// dst [rows][D + 4] = tf32(mul * src [rows][D]), the four pad columns zero.
+struct PadParams {
+  long rows;
+  int D;
+  float mul;
+  const float* src;
+  float* dst;
+};
+
 struct CvtParams {
   long n;
   const uint16_t* src;
@@ -124,6 +134,7 @@ cudaError_t launch_tok(int mode, const TokParams& p, cudaStream_t s);
 cudaError_t launch_dx(const DxParams& p, cudaStream_t s);
 cudaError_t launch_dw(const DwParams& p, cudaStream_t s);
 cudaError_t launch_dw_reduce(const DwReduceParams& p, cudaStream_t s);
+cudaError_t launch_pad(const PadParams& p, cudaStream_t s);
 cudaError_t launch_cvt(const CvtParams& p, cudaStream_t s);
 
 }  // namespace flare
