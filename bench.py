@@ -369,15 +369,18 @@ def run_backward(args, rank, world, local_rank):
         for k, v in grads.items():
             h_out[k].copy_(v, non_blocking=True)
 
-    e2e_step()
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(max(1, args.e2e_steps)):
+    e2e_ms = float("nan")
+    if args.e2e_steps > 0:
         e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / max(1, args.e2e_steps), world, dev)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
 
     if rank == 0:
         cpu = None
