@@ -113,8 +113,9 @@ __device__ __forceinline__ void stage_bf16(float* dst, const uint16_t* src, int 
 //   decoder:  W = 2^(S - L_n), dS = W (Z dY^T - delta_n), dZ += W dY, dQ += dS K
 //   encoder:  W = 2^(S - L_m), dS = W (dZ V^T - gamma_m), dQ += dS K
 // ---------------------------------------------------------------------------
-template <int D, int MODE>
+template <int D, int MODE, int MT>
 __global__ void __launch_bounds__(256) lat_kernel(const LatParams p) {
+  static_assert(MODE != kLatForward || MT == 1, "the online softmax keeps one m-tile per warp");
   constexpr int KS = D / 8, LD = D + 4, T = kBwdTokTile, NT = T / 8;
   // two buffers: the next tile is loaded into registers while this one is
   // used, and stored after it (one barrier per tile)
@@ -125,8 +126,6 @@ __global__ void __launch_bounds__(256) lat_kernel(const LatParams p) {
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int split = blockIdx.x, bh = blockIdx.z;
-  const int m0 = blockIdx.y * p.rows_per_block + warp * 16 + g, m1 = m0 + 8;
-  const bool act0 = m0 < p.M, act1 = m1 < p.M;
   const int b = bh / p.H, h = bh % p.H;
   const int gq = p.q_per_batch ? bh : h;
   bool bad = false;
@@ -136,41 +135,55 @@ __global__ void __launch_bounds__(256) lat_kernel(const LatParams p) {
   const int t_begin = split * p.tiles_per_split;
   const int t_end = min(t_begin + p.tiles_per_split, ntv);
 
-  // A fragments of this warp's rows: log2-scaled queries, and Z (decoder) or
-  // dZ (encoder); rows past M are zero and write nothing
-  uint32_t qa[KS][4], za[KS][4];
-  {
-    const float* q0 = p.q + (static_cast<size_t>(gq) * p.M + (act0 ? m0 : 0)) * D;
-    const float* q1 = p.q + (static_cast<size_t>(gq) * p.M + (act1 ? m1 : 0)) * D;
-    const float* z0 = p.zrow + (static_cast<size_t>(bh) * p.M + (act0 ? m0 : 0)) * D;
-    const float* z1 = p.zrow + (static_cast<size_t>(bh) * p.M + (act1 ? m1 : 0)) * D;
+  // this thread's latent rows: m-tile mt of the warp, rows g (i = 0), g + 8 (i = 1)
+  int mr[MT][2];
+  bool act[MT][2];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      mr[mt][i] = blockIdx.y * p.rows_per_block + (warp * MT + mt) * 16 + g + 8 * i;
+      act[mt][i] = mr[mt][i] < p.M;
+    }
+  // A fragments: log2-scaled queries, and Z (decoder) or dZ (encoder); rows
+  // past M are zero and write nothing
+  uint32_t qa[MT][KS][4], za[MT][KS][4];
+  float lr[MT][2], gr[MT][2];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    const float* qrow[2];
+    const float* zrow[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int m = act[mt][i] ? mr[mt][i] : 0;
+      qrow[i] = p.q + (static_cast<size_t>(gq) * p.M + m) * D;
+      zrow[i] = p.zrow + (static_cast<size_t>(bh) * p.M + m) * D;
+      lr[mt][i] = (MODE == kLatEncoder && act[mt][i]) ? p.lrow[static_cast<size_t>(bh) * p.M + m] : 0.f;
+      gr[mt][i] = (MODE == kLatEncoder && act[mt][i]) ? p.grow[static_cast<size_t>(bh) * p.M + m] : 0.f;
+    }
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
       const int c = ks * 8 + t;
-      qa[ks][0] = act0 ? tf32(p.c * q0[c]) : 0u;
-      qa[ks][1] = act1 ? tf32(p.c * q1[c]) : 0u;
-      qa[ks][2] = act0 ? tf32(p.c * q0[c + 4]) : 0u;
-      qa[ks][3] = act1 ? tf32(p.c * q1[c + 4]) : 0u;
+      qa[mt][ks][0] = act[mt][0] ? tf32(p.c * qrow[0][c]) : 0u;
+      qa[mt][ks][1] = act[mt][1] ? tf32(p.c * qrow[1][c]) : 0u;
+      qa[mt][ks][2] = act[mt][0] ? tf32(p.c * qrow[0][c + 4]) : 0u;
+      qa[mt][ks][3] = act[mt][1] ? tf32(p.c * qrow[1][c + 4]) : 0u;
       if (MODE != kLatForward) {
-        za[ks][0] = act0 ? tf32(z0[c]) : 0u;
-        za[ks][1] = act1 ? tf32(z1[c]) : 0u;
-        za[ks][2] = act0 ? tf32(z0[c + 4]) : 0u;
-        za[ks][3] = act1 ? tf32(z1[c + 4]) : 0u;
+        za[mt][ks][0] = act[mt][0] ? tf32(zrow[0][c]) : 0u;
+        za[mt][ks][1] = act[mt][1] ? tf32(zrow[1][c]) : 0u;
+        za[mt][ks][2] = act[mt][0] ? tf32(zrow[0][c + 4]) : 0u;
+        za[mt][ks][3] = act[mt][1] ? tf32(zrow[1][c + 4]) : 0u;
       }
     }
   }
-  float lr0 = 0.f, lr1 = 0.f, gr0 = 0.f, gr1 = 0.f;
-  if (MODE == kLatEncoder) {
-    const size_t rb = static_cast<size_t>(bh) * p.M;
-    if (act0) { lr0 = p.lrow[rb + m0]; gr0 = p.grow[rb + m0]; }
-    if (act1) { lr1 = p.lrow[rb + m1]; gr1 = p.grow[rb + m1]; }
-  }
-  float oa[KS][4], ob[KS][4];  // forward: O; decoder: dZ (oa), dQ (ob); encoder: dQ (ob)
+  float oa[MT][KS][4], ob[MT][KS][4];  // forward: O; decoder: dZ (oa), dQ (ob); encoder: dQ (ob)
 #pragma unroll
-  for (int nd = 0; nd < KS; ++nd)
+  for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) oa[nd][i] = ob[nd][i] = 0.f;
-  float mx0 = -INFINITY, mx1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    for (int nd = 0; nd < KS; ++nd)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) oa[mt][nd][i] = ob[mt][nd][i] = 0.f;
+  float mx0 = -INFINITY, mx1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // forward (MT == 1)
 
   const uint16_t* kh = p.k + static_cast<size_t>(bh) * p.N * D;
   const uint16_t* xh = (MODE == kLatDecoder ? p.dy : p.v) + static_cast<size_t>(bh) * p.N * D;
@@ -229,16 +242,16 @@ __global__ void __launch_bounds__(256) lat_kernel(const LatParams p) {
     const float* sL = sLb[buf];
     const float* sDl = sDlb[buf];
 
-    float s[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) s[nt][i] = 0.f;
-      const float* kr = sK + (nt * 8 + g) * LD;
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) mma8(s[nt], qa[ks], fbits(kr + ks * 8 + t), fbits(kr + ks * 8 + t + 4));
-    }
     if (MODE == kLatForward) {
+      float s[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) s[nt][i] = 0.f;
+        const float* kr = sK + (nt * 8 + g) * LD;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) mma8(s[nt], qa[0][ks], fbits(kr + ks * 8 + t), fbits(kr + ks * 8 + t + 4));
+      }
       float tm0 = -INFINITY, tm1 = -INFINITY;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -258,8 +271,8 @@ __global__ void __launch_bounds__(256) lat_kernel(const LatParams p) {
       l1 *= r1;
 #pragma unroll
       for (int nd = 0; nd < KS; ++nd) {
-        oa[nd][0] *= r0; oa[nd][1] *= r0;
-        oa[nd][2] *= r1; oa[nd][3] *= r1;
+        oa[0][nd][0] *= r0; oa[0][nd][1] *= r0;
+        oa[0][nd][2] *= r1; oa[0][nd][3] *= r1;
       }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -271,85 +284,119 @@ __global__ void __launch_bounds__(256) lat_kernel(const LatParams p) {
         c_as_a(pa, p0, p1, p2, p3);
         const float* v0 = sX + (nt * 8 + 2 * t) * LD + g;
 #pragma unroll
-        for (int nd = 0; nd < KS; ++nd) mma8(oa[nd], pa, fbits(v0 + nd * 8), fbits(v0 + LD + nd * 8));
+        for (int nd = 0; nd < KS; ++nd) mma8(oa[0][nd], pa, fbits(v0 + nd * 8), fbits(v0 + LD + nd * 8));
       }
     } else {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        float gg[4] = {0.f, 0.f, 0.f, 0.f};
+        // B fragments of this 8-token block, shared by the warp's m-tiles
+        uint32_t bs[KS][2], bg[KS][2], bk[KS][2], by[KS][2];
+        const float* kr = sK + (nt * 8 + g) * LD;
         const float* xr = sX + (nt * 8 + g) * LD;
+        const float* k0 = sK + (nt * 8 + 2 * t) * LD + g;
+        const float* y0 = sX + (nt * 8 + 2 * t) * LD + g;
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) mma8(gg, za[ks], fbits(xr + ks * 8 + t), fbits(xr + ks * 8 + t + 4));
+        for (int ks = 0; ks < KS; ++ks) {
+          bs[ks][0] = fbits(kr + ks * 8 + t);
+          bs[ks][1] = fbits(kr + ks * 8 + t + 4);
+          bg[ks][0] = fbits(xr + ks * 8 + t);
+          bg[ks][1] = fbits(xr + ks * 8 + t + 4);
+          bk[ks][0] = fbits(k0 + ks * 8);
+          bk[ks][1] = fbits(k0 + LD + ks * 8);
+          if (MODE == kLatDecoder) {
+            by[ks][0] = fbits(y0 + ks * 8);
+            by[ks][1] = fbits(y0 + LD + ks * 8);
+          }
+        }
         const int ca = nt * 8 + 2 * t;
         const bool va = ca < nv, vb = ca + 1 < nv;
-        float w[4], ds[4];
+        float la = 0.f, lb = 0.f, da = 0.f, db = 0.f;
         if (MODE == kLatDecoder) {
-          // W = 2^(S - L_n) per token column, dS = W (<Z_m, dY_n> - delta_n)
-          const float la = sL[ca], lb = sL[ca + 1], da = sDl[ca], db = sDl[ca + 1];
-          w[0] = va ? ex2_mufu(s[nt][0] - la) : 0.f;
-          w[1] = vb ? ex2_mufu(s[nt][1] - lb) : 0.f;
-          w[2] = va ? ex2_mufu(s[nt][2] - la) : 0.f;
-          w[3] = vb ? ex2_mufu(s[nt][3] - lb) : 0.f;
-          ds[0] = w[0] * (gg[0] - da);
-          ds[1] = w[1] * (gg[1] - db);
-          ds[2] = w[2] * (gg[2] - da);
-          ds[3] = w[3] * (gg[3] - db);
-          uint32_t wa[4];
-          c_as_a(wa, w[0], w[1], w[2], w[3]);
-          const float* y0 = sX + (nt * 8 + 2 * t) * LD + g;
-#pragma unroll
-          for (int nd = 0; nd < KS; ++nd) mma8(oa[nd], wa, fbits(y0 + nd * 8), fbits(y0 + LD + nd * 8));
-        } else {
-          // W = 2^(S - L_m) per latent row, dS = W (<dZ_m, V_n> - gamma_m)
-          w[0] = va ? ex2_mufu(s[nt][0] - lr0) : 0.f;
-          w[1] = vb ? ex2_mufu(s[nt][1] - lr0) : 0.f;
-          w[2] = va ? ex2_mufu(s[nt][2] - lr1) : 0.f;
-          w[3] = vb ? ex2_mufu(s[nt][3] - lr1) : 0.f;
-          ds[0] = w[0] * (gg[0] - gr0);
-          ds[1] = w[1] * (gg[1] - gr0);
-          ds[2] = w[2] * (gg[2] - gr1);
-          ds[3] = w[3] * (gg[3] - gr1);
+          la = sL[ca];
+          lb = sL[ca + 1];
+          da = sDl[ca];
+          db = sDl[ca + 1];
         }
-        uint32_t da4[4];
-        c_as_a(da4, ds[0], ds[1], ds[2], ds[3]);
-        const float* k0 = sK + (nt * 8 + 2 * t) * LD + g;
 #pragma unroll
-        for (int nd = 0; nd < KS; ++nd) mma8(ob[nd], da4, fbits(k0 + nd * 8), fbits(k0 + LD + nd * 8));
+        for (int mt = 0; mt < MT; ++mt) {
+          float s[4] = {0.f, 0.f, 0.f, 0.f}, gg[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            mma8(s, qa[mt][ks], bs[ks][0], bs[ks][1]);
+            mma8(gg, za[mt][ks], bg[ks][0], bg[ks][1]);
+          }
+          float w[4], ds[4];
+          if (MODE == kLatDecoder) {
+            // W = 2^(S - L_n) per token column, dS = W (<Z_m, dY_n> - delta_n)
+            w[0] = va ? ex2_mufu(s[0] - la) : 0.f;
+            w[1] = vb ? ex2_mufu(s[1] - lb) : 0.f;
+            w[2] = va ? ex2_mufu(s[2] - la) : 0.f;
+            w[3] = vb ? ex2_mufu(s[3] - lb) : 0.f;
+            ds[0] = w[0] * (gg[0] - da);
+            ds[1] = w[1] * (gg[1] - db);
+            ds[2] = w[2] * (gg[2] - da);
+            ds[3] = w[3] * (gg[3] - db);
+            uint32_t wa[4];
+            c_as_a(wa, w[0], w[1], w[2], w[3]);
+#pragma unroll
+            for (int nd = 0; nd < KS; ++nd) mma8(oa[mt][nd], wa, by[nd][0], by[nd][1]);
+          } else {
+            // W = 2^(S - L_m) per latent row, dS = W (<dZ_m, V_n> - gamma_m)
+            w[0] = va ? ex2_mufu(s[0] - lr[mt][0]) : 0.f;
+            w[1] = vb ? ex2_mufu(s[1] - lr[mt][0]) : 0.f;
+            w[2] = va ? ex2_mufu(s[2] - lr[mt][1]) : 0.f;
+            w[3] = vb ? ex2_mufu(s[3] - lr[mt][1]) : 0.f;
+            ds[0] = w[0] * (gg[0] - gr[mt][0]);
+            ds[1] = w[1] * (gg[1] - gr[mt][0]);
+            ds[2] = w[2] * (gg[2] - gr[mt][1]);
+            ds[3] = w[3] * (gg[3] - gr[mt][1]);
+          }
+          uint32_t da4[4];
+          c_as_a(da4, ds[0], ds[1], ds[2], ds[3]);
+#pragma unroll
+          for (int nd = 0; nd < KS; ++nd) mma8(ob[mt][nd], da4, bk[nd][0], bk[nd][1]);
+        }
       }
     }
     if (more) commit(buf ^ 1);
     __syncthreads();
   }
 
-  // partials of rows m0 (c0, c1) and m1 (c2, c3)
-  const size_t base0 = (static_cast<size_t>(bh) * p.n_splits + split) * p.M + m0;
-  const size_t base1 = base0 + 8;
+  // partials of rows mr[mt][0] (c0, c1) and mr[mt][1] (c2, c3)
   if (MODE == kLatForward) {
     l0 = quad_sum(l0);
     l1 = quad_sum(l1);
-    float* o0 = p.part_a + base0 * (D + 2);
-    float* o1 = p.part_a + base1 * (D + 2);
-    if (t == 0) {
-      if (act0) { o0[0] = mx0; o0[1] = l0; }
-      if (act1) { o1[0] = mx1; o1[1] = l1; }
-    }
+    const float mx[2] = {mx0, mx1}, ll[2] = {l0, l1};
 #pragma unroll
-    for (int nd = 0; nd < KS; ++nd) {
-      const int c = 2 + nd * 8 + 2 * t;
-      if (act0) { o0[c] = oa[nd][0]; o0[c + 1] = oa[nd][1]; }
-      if (act1) { o1[c] = oa[nd][2]; o1[c + 1] = oa[nd][3]; }
+    for (int i = 0; i < 2; ++i) {
+      if (!act[0][i]) continue;
+      float* o = p.part_a + ((static_cast<size_t>(bh) * p.n_splits + split) * p.M + mr[0][i]) * (D + 2);
+      if (t == 0) {
+        o[0] = mx[i];
+        o[1] = ll[i];
+      }
+#pragma unroll
+      for (int nd = 0; nd < KS; ++nd) {
+        const int c = 2 + nd * 8 + 2 * t;
+        o[c] = oa[0][nd][2 * i];
+        o[c + 1] = oa[0][nd][2 * i + 1];
+      }
     }
   } else {
 #pragma unroll
-    for (int nd = 0; nd < KS; ++nd) {
-      const int c = nd * 8 + 2 * t;
-      if (MODE == kLatDecoder) {
-        if (act0) *reinterpret_cast<float2*>(p.part_a + base0 * D + c) = make_float2(oa[nd][0], oa[nd][1]);
-        if (act1) *reinterpret_cast<float2*>(p.part_a + base1 * D + c) = make_float2(oa[nd][2], oa[nd][3]);
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        if (!act[mt][i]) continue;
+        const size_t base = (static_cast<size_t>(bh) * p.n_splits + split) * p.M + mr[mt][i];
+#pragma unroll
+        for (int nd = 0; nd < KS; ++nd) {
+          const int c = nd * 8 + 2 * t;
+          if (MODE == kLatDecoder)
+            *reinterpret_cast<float2*>(p.part_a + base * D + c) = make_float2(oa[mt][nd][2 * i], oa[mt][nd][2 * i + 1]);
+          *reinterpret_cast<float2*>(p.part_b + base * D + c) = make_float2(ob[mt][nd][2 * i], ob[mt][nd][2 * i + 1]);
+        }
       }
-      if (act0) *reinterpret_cast<float2*>(p.part_b + base0 * D + c) = make_float2(ob[nd][0], ob[nd][1]);
-      if (act1) *reinterpret_cast<float2*>(p.part_b + base1 * D + c) = make_float2(ob[nd][2], ob[nd][3]);
-    }
   }
 }
 
@@ -434,7 +481,7 @@ __global__ void __launch_bounds__(256) lat_sum_kernel(const LatSumParams p) {
 //             dV += A dZ
 //   encoder:  the A terms alone (query synthesis: no decoder)
 // ---------------------------------------------------------------------------
-template <int D, int MODE>
+template <int D, int MODE, int MT>
 __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
   constexpr int KS = D / 8, LD = D + 4, MC = tok_chunk(D);
   // two chunk buffers, filled by cp.async from the padded tf32 copies while
@@ -447,12 +494,20 @@ __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
   const int gq = p.q_per_batch ? bh : h;
-  const int r0 = blockIdx.x * kBwdTokBlock + warp * 16 + g, r1 = r0 + 8;
   bool bad = false;
   const int L = shard_valid_len(p.lengths, b, p.N, 0, p.N, &bad);
-  const bool in0 = r0 < p.N, in1 = r1 < p.N;
-  const size_t tok0 = static_cast<size_t>(bh) * p.N + (in0 ? r0 : 0);
-  const size_t tok1 = static_cast<size_t>(bh) * p.N + (in1 ? r1 : 0);
+  // this thread's token rows: m-tile mt of the warp, rows g (i = 0) and g + 8 (i = 1)
+  int rr[MT][2];
+  bool in[MT][2];
+  size_t tk[MT][2];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      rr[mt][i] = blockIdx.x * kBwdTokBlock + (warp * MT + mt) * 16 + g + 8 * i;
+      in[mt][i] = rr[mt][i] < p.N;
+      tk[mt][i] = static_cast<size_t>(bh) * p.N + (in[mt][i] ? rr[mt][i] : 0);
+    }
 
   const float* qpad = p.qpad + static_cast<size_t>(gq) * p.M * LD;
   const float* apad = (MODE == kTokStats ? p.zpad : p.dzpad) + static_cast<size_t>(bh) * p.M * LD;
@@ -477,31 +532,38 @@ __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
   issue(0, 0);
 
   // A fragments of this warp's token rows (bf16 values are exact in tf32)
-  uint32_t ka[KS][4], va[KS][4], ya[KS][4];
-  auto frag = [&](const uint16_t* src, uint32_t (&f)[KS][4]) {
+  uint32_t ka[MT][KS][4], va[MT][KS][4], ya[MT][KS][4];
+  auto frag = [&](const uint16_t* src, uint32_t (&f)[MT][KS][4]) {
 #pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      const int c = ks * 8 + t;
-      f[ks][0] = in0 ? static_cast<uint32_t>(src[tok0 * D + c]) << 16 : 0u;
-      f[ks][1] = in1 ? static_cast<uint32_t>(src[tok1 * D + c]) << 16 : 0u;
-      f[ks][2] = in0 ? static_cast<uint32_t>(src[tok0 * D + c + 4]) << 16 : 0u;
-      f[ks][3] = in1 ? static_cast<uint32_t>(src[tok1 * D + c + 4]) << 16 : 0u;
-    }
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const int c = ks * 8 + t;
+        f[mt][ks][0] = in[mt][0] ? static_cast<uint32_t>(src[tk[mt][0] * D + c]) << 16 : 0u;
+        f[mt][ks][1] = in[mt][1] ? static_cast<uint32_t>(src[tk[mt][1] * D + c]) << 16 : 0u;
+        f[mt][ks][2] = in[mt][0] ? static_cast<uint32_t>(src[tk[mt][0] * D + c + 4]) << 16 : 0u;
+        f[mt][ks][3] = in[mt][1] ? static_cast<uint32_t>(src[tk[mt][1] * D + c + 4]) << 16 : 0u;
+      }
   };
   frag(p.k, ka);
   if (MODE != kTokStats) frag(p.v, va);
   if (MODE == kTokFull) frag(p.dy, ya);
-  float ln0 = 0.f, ln1 = 0.f, dl0 = 0.f, dl1 = 0.f;
-  if (MODE == kTokFull) {
-    if (in0) { ln0 = p.ltok[tok0]; dl0 = p.dtok[tok0]; }
-    if (in1) { ln1 = p.ltok[tok1]; dl1 = p.dtok[tok1]; }
-  }
-  float oa[KS][4], ob[KS][4];  // stats: Y (oa); full, encoder: dK (oa), dV (ob)
+  float ln[MT][2], dl[MT][2];
 #pragma unroll
-  for (int nd = 0; nd < KS; ++nd)
+  for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) oa[nd][i] = ob[nd][i] = 0.f;
-  float mx0 = -INFINITY, mx1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    for (int i = 0; i < 2; ++i) {
+      ln[mt][i] = (MODE == kTokFull && in[mt][i]) ? p.ltok[tk[mt][i]] : 0.f;
+      dl[mt][i] = (MODE == kTokFull && in[mt][i]) ? p.dtok[tk[mt][i]] : 0.f;
+    }
+  float oa[MT][KS][4], ob[MT][KS][4];  // stats: Y (oa); full, encoder: dK (oa), dV (ob)
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nd = 0; nd < KS; ++nd)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) oa[mt][nd][i] = ob[mt][nd][i] = 0.f;
+  float mx0 = -INFINITY, mx1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // stats (MT == 1)
 
   for (int mb = 0, it = 0; mb < p.M; mb += MC, ++it) {
     const int buf = it & 1;
@@ -517,6 +579,7 @@ __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
     const int ntl = mc / 8;
 
     if (MODE == kTokStats) {
+      static_assert(MODE != kTokStats || MT == 1, "the statistics pass keeps one m-tile per warp");
       float s[MC / 8][4];
       float tm0 = -INFINITY, tm1 = -INFINITY;
 #pragma unroll
@@ -528,7 +591,7 @@ __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
           for (int i = 0; i < 4; ++i) s[nt][i] = 0.f;
           const float* qr = sQ + (nt * 8 + g) * LD;
 #pragma unroll
-          for (int ks = 0; ks < KS; ++ks) mma8(s[nt], ka[ks], fbits(qr + ks * 8 + t), fbits(qr + ks * 8 + t + 4));
+          for (int ks = 0; ks < KS; ++ks) mma8(s[nt], ka[0][ks], fbits(qr + ks * 8 + t), fbits(qr + ks * 8 + t + 4));
         }
         tm0 = fmaxf(tm0, fmaxf(s[nt][0], s[nt][1]));
         tm1 = fmaxf(tm1, fmaxf(s[nt][2], s[nt][3]));
@@ -543,8 +606,8 @@ __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
       l1 *= q1;
 #pragma unroll
       for (int nd = 0; nd < KS; ++nd) {
-        oa[nd][0] *= q0; oa[nd][1] *= q0;
-        oa[nd][2] *= q1; oa[nd][3] *= q1;
+        oa[0][nd][0] *= q0; oa[0][nd][1] *= q0;
+        oa[0][nd][2] *= q1; oa[0][nd][3] *= q1;
       }
 #pragma unroll
       for (int nt = 0; nt < MC / 8; ++nt) {
@@ -557,51 +620,71 @@ __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
           c_as_a(pa, p0, p1, p2, p3);
           const float* z0 = sA + (nt * 8 + 2 * t) * LD + g;
 #pragma unroll
-          for (int nd = 0; nd < KS; ++nd) mma8(oa[nd], pa, fbits(z0 + nd * 8), fbits(z0 + LD + nd * 8));
+          for (int nd = 0; nd < KS; ++nd) mma8(oa[0][nd], pa, fbits(z0 + nd * 8), fbits(z0 + LD + nd * 8));
         }
       }
     } else {
 #pragma unroll
       for (int nt = 0; nt < MC / 8; ++nt) {
         if (nt >= ntl) continue;
-        float s[4] = {0.f, 0.f, 0.f, 0.f}, da[4] = {0.f, 0.f, 0.f, 0.f};
+        // B fragments of this 8-latent block, shared by the warp's m-tiles
+        uint32_t bq[KS][2], bz[KS][2], bzz[KS][2], bk[KS][2], bv[KS][2];
         const float* qr = sQ + (nt * 8 + g) * LD;
         const float* dzr = sA + (nt * 8 + g) * LD;
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          mma8(s, ka[ks], fbits(qr + ks * 8 + t), fbits(qr + ks * 8 + t + 4));
-          mma8(da, va[ks], fbits(dzr + ks * 8 + t), fbits(dzr + ks * 8 + t + 4));
-        }
-        const int ca = nt * 8 + 2 * t;
-        const float lma = sLm[ca], lmb = sLm[ca + 1], ga = sG[ca], gb = sG[ca + 1];
-        float a[4], ds[4];
-        a[0] = ex2_mufu(s[0] - lma);
-        a[1] = ex2_mufu(s[1] - lmb);
-        a[2] = ex2_mufu(s[2] - lma);
-        a[3] = ex2_mufu(s[3] - lmb);
-        ds[0] = a[0] * (da[0] - ga);
-        ds[1] = a[1] * (da[1] - gb);
-        ds[2] = a[2] * (da[2] - ga);
-        ds[3] = a[3] * (da[3] - gb);
-        if (MODE == kTokFull) {
-          float dp[4] = {0.f, 0.f, 0.f, 0.f};
-          const float* zr = sZ + (nt * 8 + g) * LD;
-#pragma unroll
-          for (int ks = 0; ks < KS; ++ks) mma8(dp, ya[ks], fbits(zr + ks * 8 + t), fbits(zr + ks * 8 + t + 4));
-          ds[0] = fmaf(ex2_mufu(s[0] - ln0), dp[0] - dl0, ds[0]);
-          ds[1] = fmaf(ex2_mufu(s[1] - ln0), dp[1] - dl0, ds[1]);
-          ds[2] = fmaf(ex2_mufu(s[2] - ln1), dp[2] - dl1, ds[2]);
-          ds[3] = fmaf(ex2_mufu(s[3] - ln1), dp[3] - dl1, ds[3]);
-        }
-        uint32_t sa4[4], aa4[4];
-        c_as_a(sa4, ds[0], ds[1], ds[2], ds[3]);
-        c_as_a(aa4, a[0], a[1], a[2], a[3]);
+        const float* zr = sZ + (nt * 8 + g) * LD;
         const float* q0 = sQ + (nt * 8 + 2 * t) * LD + g;
         const float* z0 = sA + (nt * 8 + 2 * t) * LD + g;
 #pragma unroll
-        for (int nd = 0; nd < KS; ++nd) {
-          mma8(oa[nd], sa4, fbits(q0 + nd * 8), fbits(q0 + LD + nd * 8));
-          mma8(ob[nd], aa4, fbits(z0 + nd * 8), fbits(z0 + LD + nd * 8));
+        for (int ks = 0; ks < KS; ++ks) {
+          bq[ks][0] = fbits(qr + ks * 8 + t);
+          bq[ks][1] = fbits(qr + ks * 8 + t + 4);
+          bz[ks][0] = fbits(dzr + ks * 8 + t);
+          bz[ks][1] = fbits(dzr + ks * 8 + t + 4);
+          if (MODE == kTokFull) {
+            bzz[ks][0] = fbits(zr + ks * 8 + t);
+            bzz[ks][1] = fbits(zr + ks * 8 + t + 4);
+          }
+          bk[ks][0] = fbits(q0 + ks * 8);
+          bk[ks][1] = fbits(q0 + LD + ks * 8);
+          bv[ks][0] = fbits(z0 + ks * 8);
+          bv[ks][1] = fbits(z0 + LD + ks * 8);
+        }
+        const int ca = nt * 8 + 2 * t;
+        const float lma = sLm[ca], lmb = sLm[ca + 1], ga = sG[ca], gb = sG[ca + 1];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          float s[4] = {0.f, 0.f, 0.f, 0.f}, da[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            mma8(s, ka[mt][ks], bq[ks][0], bq[ks][1]);
+            mma8(da, va[mt][ks], bz[ks][0], bz[ks][1]);
+          }
+          float a[4], ds[4];
+          a[0] = ex2_mufu(s[0] - lma);
+          a[1] = ex2_mufu(s[1] - lmb);
+          a[2] = ex2_mufu(s[2] - lma);
+          a[3] = ex2_mufu(s[3] - lmb);
+          ds[0] = a[0] * (da[0] - ga);
+          ds[1] = a[1] * (da[1] - gb);
+          ds[2] = a[2] * (da[2] - ga);
+          ds[3] = a[3] * (da[3] - gb);
+          if (MODE == kTokFull) {
+            float dp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) mma8(dp, ya[mt][ks], bzz[ks][0], bzz[ks][1]);
+            ds[0] = fmaf(ex2_mufu(s[0] - ln[mt][0]), dp[0] - dl[mt][0], ds[0]);
+            ds[1] = fmaf(ex2_mufu(s[1] - ln[mt][0]), dp[1] - dl[mt][0], ds[1]);
+            ds[2] = fmaf(ex2_mufu(s[2] - ln[mt][1]), dp[2] - dl[mt][1], ds[2]);
+            ds[3] = fmaf(ex2_mufu(s[3] - ln[mt][1]), dp[3] - dl[mt][1], ds[3]);
+          }
+          uint32_t sa4[4], aa4[4];
+          c_as_a(sa4, ds[0], ds[1], ds[2], ds[3]);
+          c_as_a(aa4, a[0], a[1], a[2], a[3]);
+#pragma unroll
+          for (int nd = 0; nd < KS; ++nd) {
+            mma8(oa[mt][nd], sa4, bk[nd][0], bk[nd][1]);
+            mma8(ob[mt][nd], aa4, bv[nd][0], bv[nd][1]);
+          }
         }
       }
     }
@@ -609,6 +692,8 @@ __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
 
   if (MODE == kTokStats) {
     // every lane reaches the shuffles; l >= 1 for every row here
+    const size_t tok0 = tk[0][0], tok1 = tk[0][1];
+    const bool in0 = in[0][0], in1 = in[0][1];
     l0 = quad_sum(l0);
     l1 = quad_sum(l1);
     const float i0 = 1.f / l0, i1 = 1.f / l1;
@@ -616,48 +701,40 @@ __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
 #pragma unroll
     for (int nd = 0; nd < KS; ++nd) {
       const int c = nd * 8 + 2 * t;
-      if (in0) d0 += bf(p.dy[tok0 * D + c]) * (oa[nd][0] * i0) + bf(p.dy[tok0 * D + c + 1]) * (oa[nd][1] * i0);
-      if (in1) d1 += bf(p.dy[tok1 * D + c]) * (oa[nd][2] * i1) + bf(p.dy[tok1 * D + c + 1]) * (oa[nd][3] * i1);
+      if (in0) d0 += bf(p.dy[tok0 * D + c]) * (oa[0][nd][0] * i0) + bf(p.dy[tok0 * D + c + 1]) * (oa[0][nd][1] * i0);
+      if (in1) d1 += bf(p.dy[tok1 * D + c]) * (oa[0][nd][2] * i1) + bf(p.dy[tok1 * D + c + 1]) * (oa[0][nd][3] * i1);
     }
     d0 = quad_sum(d0);
     d1 = quad_sum(d1);
     if (t == 0) {
-      if (in0) { p.ltok[tok0] = r0 < L ? mx0 + __log2f(l0) : 0.f; p.dtok[tok0] = r0 < L ? d0 : 0.f; }
-      if (in1) { p.ltok[tok1] = r1 < L ? mx1 + __log2f(l1) : 0.f; p.dtok[tok1] = r1 < L ? d1 : 0.f; }
+      if (in0) { p.ltok[tok0] = rr[0][0] < L ? mx0 + __log2f(l0) : 0.f; p.dtok[tok0] = rr[0][0] < L ? d0 : 0.f; }
+      if (in1) { p.ltok[tok1] = rr[0][1] < L ? mx1 + __log2f(l1) : 0.f; p.dtok[tok1] = rr[0][1] < L ? d1 : 0.f; }
     }
     return;
   }
   // dK = scale sum dS q = ln2 sum dS (scale log2(e) q); padding tokens get zeros
-  const bool v0 = r0 < L, v1 = r1 < L;
 #pragma unroll
-  for (int nd = 0; nd < KS; ++nd) {
-    const int c = nd * 8 + 2 * t;
-    const float2 k0 = v0 ? make_float2(oa[nd][0] * kLn2, oa[nd][1] * kLn2) : make_float2(0.f, 0.f);
-    const float2 k1 = v1 ? make_float2(oa[nd][2] * kLn2, oa[nd][3] * kLn2) : make_float2(0.f, 0.f);
-    const float2 w0 = v0 ? make_float2(ob[nd][0], ob[nd][1]) : make_float2(0.f, 0.f);
-    const float2 w1 = v1 ? make_float2(ob[nd][2], ob[nd][3]) : make_float2(0.f, 0.f);
-    if (p.g32 != nullptr) {
-      if (in0) {
-        float* o = p.g32 + (static_cast<size_t>(b) * p.N + r0) * p.g_ld + h * D + c;
-        *reinterpret_cast<float2*>(o + p.g_col_k) = k0;
-        *reinterpret_cast<float2*>(o + p.g_col_v) = w0;
-      }
-      if (in1) {
-        float* o = p.g32 + (static_cast<size_t>(b) * p.N + r1) * p.g_ld + h * D + c;
-        *reinterpret_cast<float2*>(o + p.g_col_k) = k1;
-        *reinterpret_cast<float2*>(o + p.g_col_v) = w1;
-      }
-    } else {
-      if (in0) {
-        *reinterpret_cast<uint32_t*>(p.dk16 + tok0 * D + c) = pack_bf16x2(k0.x, k0.y);
-        *reinterpret_cast<uint32_t*>(p.dv16 + tok0 * D + c) = pack_bf16x2(w0.x, w0.y);
-      }
-      if (in1) {
-        *reinterpret_cast<uint32_t*>(p.dk16 + tok1 * D + c) = pack_bf16x2(k1.x, k1.y);
-        *reinterpret_cast<uint32_t*>(p.dv16 + tok1 * D + c) = pack_bf16x2(w1.x, w1.y);
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      if (!in[mt][i]) continue;
+      const bool v = rr[mt][i] < L;
+#pragma unroll
+      for (int nd = 0; nd < KS; ++nd) {
+        const int c = nd * 8 + 2 * t;
+        const float2 kk = v ? make_float2(oa[mt][nd][2 * i] * kLn2, oa[mt][nd][2 * i + 1] * kLn2)
+                            : make_float2(0.f, 0.f);
+        const float2 vv = v ? make_float2(ob[mt][nd][2 * i], ob[mt][nd][2 * i + 1]) : make_float2(0.f, 0.f);
+        if (p.g32 != nullptr) {
+          float* o = p.g32 + (static_cast<size_t>(b) * p.N + rr[mt][i]) * p.g_ld + h * D + c;
+          *reinterpret_cast<float2*>(o + p.g_col_k) = kk;
+          *reinterpret_cast<float2*>(o + p.g_col_v) = vv;
+        } else {
+          *reinterpret_cast<uint32_t*>(p.dk16 + tk[mt][i] * D + c) = pack_bf16x2(kk.x, kk.y);
+          *reinterpret_cast<uint32_t*>(p.dv16 + tk[mt][i] * D + c) = pack_bf16x2(vv.x, vv.y);
+        }
       }
     }
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -821,17 +898,20 @@ unsigned blocks_for(long n, int threads) { return static_cast<unsigned>((n + thr
 }  // namespace
 
 cudaError_t launch_lat(int mode, const LatParams& p, cudaStream_t s) {
+  // a warp per 16 latent rows (forward) or per 32 (two m-tiles sharing the B
+  // fragments: the gradient modes, when the CTA keeps at least two warps)
   const dim3 grid(p.n_splits, (p.M + p.rows_per_block - 1) / p.rows_per_block, p.B * p.H);
-  const int threads = 2 * p.rows_per_block;  // a warp per 16 latent rows
-#define FLARE_LAT(DD, MM) lat_kernel<DD, MM><<<grid, threads, 0, s>>>(p)
+  const bool two = mode != kLatForward && p.rows_per_block >= 64 && p.D == 16;  // D = 32 would spill
+  const int threads = two ? p.rows_per_block : 2 * p.rows_per_block;
+#define FLARE_LAT(DD, MM, MT) lat_kernel<DD, MM, MT><<<grid, threads, 0, s>>>(p)
   if (p.D == 16) {
-    if (mode == kLatForward) FLARE_LAT(16, kLatForward);
-    else if (mode == kLatDecoder) FLARE_LAT(16, kLatDecoder);
-    else FLARE_LAT(16, kLatEncoder);
+    if (mode == kLatForward) FLARE_LAT(16, kLatForward, 1);
+    else if (mode == kLatDecoder) { if (two) FLARE_LAT(16, kLatDecoder, 2); else FLARE_LAT(16, kLatDecoder, 1); }
+    else { if (two) FLARE_LAT(16, kLatEncoder, 2); else FLARE_LAT(16, kLatEncoder, 1); }
   } else {
-    if (mode == kLatForward) FLARE_LAT(32, kLatForward);
-    else if (mode == kLatDecoder) FLARE_LAT(32, kLatDecoder);
-    else FLARE_LAT(32, kLatEncoder);
+    if (mode == kLatForward) FLARE_LAT(32, kLatForward, 1);
+    else if (mode == kLatDecoder) { if (two) FLARE_LAT(32, kLatDecoder, 2); else FLARE_LAT(32, kLatDecoder, 1); }
+    else { if (two) FLARE_LAT(32, kLatEncoder, 2); else FLARE_LAT(32, kLatEncoder, 1); }
   }
 #undef FLARE_LAT
   return cudaGetLastError();
@@ -853,17 +933,19 @@ cudaError_t launch_lat_sum(const LatSumParams& p, cudaStream_t s) {
 }
 
 cudaError_t launch_tok(int mode, const TokParams& p, cudaStream_t s) {
+  // a warp per 16 token rows (statistics, D = 32) or per 32 (two m-tiles
+  // sharing the B fragments: the gradient modes at D = 16)
   const dim3 grid((p.N + kBwdTokBlock - 1) / kBwdTokBlock, p.B * p.H);
-  const int threads = 2 * kBwdTokBlock;  // a warp per 16 token rows
-#define FLARE_TOK(DD, MM) tok_kernel<DD, MM><<<grid, threads, 0, s>>>(p)
+  const int t1 = 2 * kBwdTokBlock, t2 = kBwdTokBlock;
+#define FLARE_TOK(DD, MM, MT) tok_kernel<DD, MM, MT><<<grid, (MT == 1 ? t1 : t2), 0, s>>>(p)
   if (p.D == 16) {
-    if (mode == kTokStats) FLARE_TOK(16, kTokStats);
-    else if (mode == kTokFull) FLARE_TOK(16, kTokFull);
-    else FLARE_TOK(16, kTokEncoder);
+    if (mode == kTokStats) FLARE_TOK(16, kTokStats, 1);
+    else if (mode == kTokFull) FLARE_TOK(16, kTokFull, 2);
+    else FLARE_TOK(16, kTokEncoder, 2);
   } else {
-    if (mode == kTokStats) FLARE_TOK(32, kTokStats);
-    else if (mode == kTokFull) FLARE_TOK(32, kTokFull);
-    else FLARE_TOK(32, kTokEncoder);
+    if (mode == kTokStats) FLARE_TOK(32, kTokStats, 1);
+    else if (mode == kTokFull) FLARE_TOK(32, kTokFull, 1);   // two m-tiles would need ~240 registers
+    else FLARE_TOK(32, kTokEncoder, 1);
   }
 #undef FLARE_TOK
   return cudaGetLastError();
