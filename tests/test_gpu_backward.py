@@ -68,6 +68,7 @@ def flare_case(B, H, N, M, D, lengths=None, seed=5):
     (2, 2, 777, 64, 16, [777, 300]),
     (1, 3, 1000, 48, 32, None),
     (3, 2, 200, 16, 16, [1, 200, 129]),
+    (2, 2, 2000, 256, 32, [2000, 1537]),
 ])
 def test_flare_backward_matches_oracle(B, H, N, M, D, lengths):
     w = flare_case(B, H, N, M, D, lengths)
@@ -85,6 +86,7 @@ def test_flare_backward_matches_oracle(B, H, N, M, D, lengths):
     ("flarepp_n1k", None, None),
     ("flarepp_n8k_mesh2d", 1500, 2),
     ("flarepp_masked_n4k", 640, 3),
+    ("flarepp_n1m_mesh3d", 3000, None),   # the million-token shape's M = 512: 8 chunks, 4 latent blocks
 ])
 def test_flarepp_backward_matches_oracle(name, N, B):
     w = make_workload(name, N=N, B=B)
@@ -176,3 +178,30 @@ def test_backward_reports_bad_lengths():
     fl.flarepp_mixer_bwd(dev_bf16(w.X), dev_bf16(w.Wk), dev_bf16(w.Wv), dev_bf16(w.Wk_syn), dev_bf16(w.Wv_syn),
                          dev_bf16(w.Q0), dev_bf16(dY), lengths=lengths_dev(w), workspace=ws)
     assert fl.flare_last_device_status(ws) == fl.Status.ERR_SHAPE
+
+
+def test_backward_cuda_graph_replays_the_same_bits():
+    """The backward call only enqueues kernels and a memset on its stream, so
+    it can be captured into a CUDA graph; a replay gives the eager bits."""
+    w = make_workload("flarepp_n8k_mesh2d", N=1024, B=2)
+    dY = dev_bf16(make_upstream_grad(w))
+    X, Q0 = dev_bf16(w.X), dev_bf16(w.Q0)
+    Ws = [dev_bf16(a) for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn)]
+    nbytes = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLAREPP_BWD, w.B, w.H, w.N, w.M, w.D, w.C)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        g = fl.flarepp_mixer_bwd(X, *Ws, Q0, dY, workspace=ws, stream=s)
+        torch.cuda.synchronize()
+        eager = {k: v.clone() for k, v in g.items()}
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            fl.flarepp_mixer_bwd(X, *Ws, Q0, dY, workspace=ws, stream=s, grads=g, check=False)
+    for v in g.values():
+        v.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    for k in g:
+        assert torch.equal(g[k].view(torch.int16) if g[k].dtype == torch.bfloat16 else g[k],
+                           eager[k].view(torch.int16) if eager[k].dtype == torch.bfloat16 else eager[k]), k
+    del graph
