@@ -877,7 +877,6 @@ flare_status bwd_core(const BwdPlan& bp, uint8_t* ws, const float* q, int q_per_
   tp.ltok = ltok; tp.dtok = dtok;
   tp.g32 = out.g32; tp.g_ld = out.g_ld; tp.g_col_k = out.col_k; tp.g_col_v = out.col_v;
   tp.dk16 = out.dk16; tp.dv16 = out.dv16;
-  tp.err = reinterpret_cast<uint32_t*>(ws + bp.fwd.off_err);
   if (launch_tok(kTokStats, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   // decoder backward, reductions over tokens: dZ and the decoder's dQ
   LatParams lp = lat_params(bp, ws, q, q_per_batch, k, B, H, N, M, D, lengths, sc);
@@ -994,7 +993,6 @@ flare_status flarepp_mixer_bwd(const flare_bf16* X, const flare_bf16* Wk, const 
   tp.qpad = q0pad; tp.dzpad = dqxpad; tp.lm = lsyn; tp.gam = gsyn;
   tp.k = pr.kt; tp.v = pr.vt;
   tp.g32 = g32; tp.g_ld = 4 * C; tp.g_col_k = 2 * C; tp.g_col_v = 3 * C;
-  tp.err = reinterpret_cast<uint32_t*>(ws + bp.fwd.off_err);
   if (launch_tok(kTokEncoder, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   // ... and dQ0 (summed over the batch)
   LatParams le = lat_params(bp, ws, q32, 0, pr.kt, B, H, N, M, D, lengths, sc);

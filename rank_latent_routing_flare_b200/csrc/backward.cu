@@ -15,17 +15,19 @@
 // (latent-parallel pass, split over tokens, merged in a fixed order) and the
 // decoder's per token (token-parallel pass over all latents).
 //
-// Kernels:
-//   lat_kernel<kLatForward>  encoder recompute partials (max, sum, sum w v)
-//   lat_merge_kernel         Z and the encoder row log-normalisers
-//   tok_kernel<kTokStats>    decoder per-token log-normaliser and delta
-//   lat_kernel<kLatDecoder>  dZ = P^T dY and the decoder's dQ (per split)
-//   lat_sum_kernel           fixed-order sums of split partials (+ gamma)
-//   tok_kernel<kTokFull>     dK (decoder + encoder) and dV
-//   lat_kernel<kLatEncoder>  the encoder's dQ (per split)
-//   tok_kernel<kTokEncoder>  dK, dV of the query synthesis
+// Kernels (template arguments <D, mode, 16-row tiles per warp>):
+//   lat_kernel<., kLatForward, 1>    encoder recompute partials (max, sum, sum w v)
+//   lat_merge_kernel                 Z and the encoder row log-normalisers
+//   tok_kernel<., kTokStats, 1>      decoder per-token log-normaliser and delta
+//   lat_kernel<., kLatDecoder, .>    dZ = P^T dY and the decoder's dQ (per split)
+//   lat_sum_kernel                   fixed-order sums of split partials (+ gamma)
+//   pad_kernel                       padded tf32 images of Q, Z, dZ for the token pass
+//   tok_kernel<., kTokFull, .>       dK (decoder + encoder) and dV
+//   lat_kernel<., kLatEncoder, .>    the encoder's dQ (per split)
+//   tok_kernel<., kTokEncoder, .>    dK, dV of the query synthesis
 //   dx_kernel / dw_kernel / dw_reduce_kernel   projection gradients
 // Every reduction has a fixed order: the results are bitwise reproducible.
+// No kernel waits on another CTA or on a flag: there are no spin loops.
 #include "bwd_internal.h"
 #include "flare_internal.h"
 #include "ptx.cuh"

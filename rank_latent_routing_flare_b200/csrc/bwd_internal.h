@@ -85,7 +85,6 @@ struct TokParams {
   int g_ld, g_col_k, g_col_v;   // row stride and column offsets of dK and dV (head h adds h*D)
   uint16_t* dk16;               // or bf16 [B*H][N][D] outputs
   uint16_t* dv16;
-  uint32_t* err;
 };
 
 // dX[r][c] = sum_q sum_j G[r][q*C + j] W_q[c][j]   (r < R = B*N, q < nw)

@@ -73,3 +73,19 @@ def test_reference_arm_works_on_rank_zero_only(capsys):
         workload, steps, warmup = bench.WORKLOAD, 1, 3
     assert bench.run_reference(Args, rank=1, world=2) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_backward_work_counts():
+    """Algorithmic work of one FLARE++ backward call: three exponentials per
+    token-head-latent (one per score of each SDPA call), per SDPA call the
+    score recompute and four gradient products (5 x 2 M D flops per
+    token-head), the projection gradients dX and dW of four C x C weights
+    (2 x 4 x 2 C D per token-head); HBM: X and dY read, dX written."""
+    import bench
+    from workloads import make_workload
+    w = make_workload("flarepp_n1k", N=256)
+    wk = bench.backward_work(w)
+    th = w.B * w.H * w.N
+    assert wk["exps"] == 3 * w.M * th
+    assert wk["flops"] == (30 * w.M * w.D + 16 * w.C * w.D) * th
+    assert wk["bytes"] == 3 * w.B * w.N * w.C * 2
