@@ -254,31 +254,40 @@ def cpu_model():
 # ---------------------------------------------------------------------------
 
 BWD_METRIC = "mixer bwd token·heads/s at N=1M (1×B200) and % of roofline (HBM/MMA/MUFU)"
-BWD_LAUNCHES = 23   # kernels per FLARE++ backward call (projections, recompute, gradients, GEMMs)
+BWD_LAUNCHES = 23        # kernels per FLARE++ backward call (projections, recompute, gradients, GEMMs)
+BWD_LAUNCHES_FLARE = 12  # kernels per FLARE backward call (recompute, gradients, merges, pads)
 TF32_PER_BF16 = 0.5  # nominal dense tf32 : bf16 tensor throughput
 
 
 def backward_work(w):
-    """Algorithmic work of the FLARE++ backward per call: one exponential per
-    score of each of the three SDPA calls; per call the score recompute and
-    the four gradient products (5 x 2MD flop per token·head), the projection
-    gradients dX and dW (2 x 4 x 2 C D flop per token·head); HBM: read X and
-    dY, write dX."""
-    th = w.B * w.H * w.N
+    """Algorithmic work of one backward call: one exponential per score of
+    each SDPA call (three for FLARE++, two for FLARE); per call the score
+    recompute and the four gradient products (5 x 2MD flop per token·head);
+    FLARE++ adds the projection gradients dX and dW (2 x 4 x 2 C D flop per
+    token·head).  HBM: FLARE++ reads X and dY and writes dX; FLARE reads K, V
+    and dY and writes dK and dV.  Token counts are valid (unpadded) tokens,
+    as in the forward's work model."""
+    th = w.H * w.valid_tokens()
+    if w.variant == "flare":
+        return {"exps": 2 * w.M * th, "flops": 2 * 5 * 2 * w.M * w.D * th, "bytes": 5 * th * w.D * 2}
     return {"exps": 3 * w.M * th, "flops": (3 * 5 * 2 * w.M * w.D + 16 * w.C * w.D) * th,
-            "bytes": 3 * w.B * w.N * w.C * 2}
+            "bytes": 3 * w.valid_tokens() * w.C * 2}
 
 
 def oracle_backward_rate(w, dY, target_s: float):
     import oracle
     from workloads import bf16_bits_to_f64 as f64
     oracle.build()
-    W = [f64(a) for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn)]
-    Q0 = f64(w.Q0)
+    W = [f64(a) for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn)] if w.variant != "flare" else None
+    Q0 = f64(w.Q0) if w.variant != "flare" else None
 
     def run(ns):
         t0 = time.perf_counter()
-        oracle.flarepp_backward(f64(w.X[:, :ns]), *W, Q0, f64(dY[:, :, :ns]), w.H, None, w.scale)
+        if w.variant == "flare":
+            oracle.flare_backward(f64(w.K[:, :, :ns]), f64(w.V[:, :, :ns]), f64(w.Q), f64(dY[:, :, :ns]), None,
+                                  w.scale)
+        else:
+            oracle.flarepp_backward(f64(w.X[:, :ns]), *W, Q0, f64(dY[:, :, :ns]), w.H, None, w.scale)
         return time.perf_counter() - t0
 
     ns = min(2048, w.N)
@@ -302,24 +311,37 @@ def run_backward(args, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     fl.load_library()
     w = make_workload(args.workload, N=args.tokens, seed=rank_seed(rank))
-    assert w.variant == "flarepp"
     dY_bits = make_upstream_grad(w)
 
     def to_dev(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    X, Q0, dY = to_dev(w.X), to_dev(w.Q0), to_dev(dY_bits)
-    Ws = [to_dev(a) for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn)]
+    flare = w.variant == "flare"
+    dY = to_dev(dY_bits)
+    if flare:
+        host_inputs = (w.K, w.V, w.Q)
+        K, V, Q = (to_dev(a) for a in host_inputs)
+        dev_inputs = (K, V, Q)
+        nbytes = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLARE_BWD, w.B, w.H, w.N, w.M, w.D)
+    else:
+        host_inputs = (w.X, w.Wk, w.Wv, w.Wk_syn, w.Wv_syn, w.Q0)
+        dev_inputs = tuple(to_dev(a) for a in host_inputs)
+        nbytes = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLAREPP_BWD, w.B, w.H, w.N, w.M, w.D, w.C)
     lengths = None if w.lengths is None else torch.from_numpy(w.lengths).to(dev)
-    nbytes = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLAREPP_BWD, w.B, w.H, w.N, w.M, w.D, w.C)
     ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     grads = None
 
     def step():
         nonlocal grads
-        grads = fl.flarepp_mixer_bwd(X, *Ws, Q0, dY, lengths=lengths, workspace=ws, stream=stream, grads=grads,
-                                     check=False)
+        if flare:
+            out = (None, None, None) if grads is None else (grads["dK"], grads["dV"], grads["dQ"])
+            dK, dV, dQ = fl.flare_mixer_bwd(*dev_inputs, dY, lengths=lengths, workspace=ws, stream=stream,
+                                            dK=out[0], dV=out[1], dQ=out[2], check=False)
+            grads = {"dK": dK, "dV": dV, "dQ": dQ}
+        else:
+            grads = fl.flarepp_mixer_bwd(*dev_inputs, dY, lengths=lengths, workspace=ws, stream=stream,
+                                         grads=grads, check=False)
 
     for _ in range(args.warmup):
         step()
@@ -356,8 +378,8 @@ def run_backward(args, rank, world, local_rank):
     # end to end: inputs and dY in from pinned host memory, gradients back out,
     # all inside the timed region on the call's stream
     pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).pin_memory()  # noqa: E731
-    h_in = [pin(a) for a in (w.X, w.Wk, w.Wv, w.Wk_syn, w.Wv_syn, w.Q0, dY_bits)]
-    d_in = [t.view(torch.int16) for t in (X, *Ws, Q0, dY)]
+    h_in = [pin(a) for a in (*host_inputs, dY_bits)]
+    d_in = [t.view(torch.int16) for t in (*dev_inputs, dY)]
     h_out = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in grads.items()}
     h2d = sum(a.numel() * 2 for a in h_in)
     d2h = sum(v.numel() * v.element_size() for v in grads.values())
@@ -387,15 +409,18 @@ def run_backward(args, rank, world, local_rank):
         if world == 1 and not args.no_cpu_baseline:
             rate, ns, t, threads = oracle_backward_rate(w, dY_bits, args.cpu_seconds)
             cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
-                   "sample": f"fp64 oracle, full FLARE++ backward on the first {ns} of {w.N} tokens "
-                             f"(B={w.B} H={w.H} M={w.M} D={w.D} C={w.C}) in {t:.1f} s; {cpu_model()}"}
+                   "sample": f"fp64 oracle, full {'FLARE' if flare else 'FLARE++'} backward on the first {ns} "
+                             f"of {w.N} tokens (B={w.B} H={w.H} M={w.M} D={w.D} C={w.C}) in {t:.1f} s; "
+                             f"{cpu_model()}"}
         line = {
             "metric": BWD_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "tf32", "data": "synthetic",
             "config": {"workload": w.name, "pass": "backward", "B": w.B, "N": w.N, "C": w.C, "H": w.H,
                        "D": w.D, "M": w.M, "parallelism": f"replicas{world}" if world > 1 else "single",
-                       "l2": "inputs larger than L2 (X 256 MiB, dY 256 MiB, fp32 gradient rows 2 GiB)"},
+                       "l2": ("inputs larger than L2 (K, V, dY: " +
+                              f"{3 * w.B * w.H * w.N * w.D * 2 / 2**20:.0f} MiB together)" if flare else
+                              "inputs larger than L2 (X 256 MiB, dY 256 MiB, fp32 gradient rows 2 GiB)")},
             "step_roofline": {"t_roof_ms": round(t_roof * 1e3, 4), "frac": round(t_roof / (ms * 1e-3), 4),
                               "bound": bound, "terms_ms": {k: round(v * 1e3, 4) for k, v in terms.items()},
                               "peak_basis": f"MUFU {MUFU_PER_CLK_PER_SM} ex2/clk/SM x {NUM_SM} x "
@@ -405,7 +430,7 @@ def run_backward(args, rank, world, local_rank):
             "cpu_baseline": cpu,
             "e2e": {"value": whole_job_rate(world, th_per_rank, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": BWD_LAUNCHES * args.steps,
+            "gpu_launches": (BWD_LAUNCHES_FLARE if flare else BWD_LAUNCHES) * args.steps,
             "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)

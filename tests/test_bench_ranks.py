@@ -89,3 +89,13 @@ def test_backward_work_counts():
     assert wk["exps"] == 3 * w.M * th
     assert wk["flops"] == (30 * w.M * w.D + 16 * w.C * w.D) * th
     assert wk["bytes"] == 3 * w.B * w.N * w.C * 2
+
+
+def test_backward_work_counts_flare():
+    import bench
+    from workloads import make_workload
+    w = make_workload("flare_n64k", N=512, B=1)
+    wk = bench.backward_work(w)
+    th = w.B * w.H * w.N
+    assert wk["exps"] == 2 * w.M * th and wk["flops"] == 20 * w.M * w.D * th
+    assert wk["bytes"] == 5 * th * w.D * 2
