@@ -186,9 +186,11 @@ FLARE_API flare_status flarepp_mixer_fwd_profiled(const flare_bf16* X, const fla
  * takes the forward's inputs and dY, not the forward's outputs.  Outputs are
  * written (not accumulated).  Rows of dY for padding tokens are ignored;
  * padding tokens get zero gradients.  Same size limits as the forward, and
- * B*H <= 65535.  Arithmetic: fp32 on the CUDA cores (bf16 inputs widened),
- * the FLARE++ projections recomputed on the tensor cores in bf16 as in the
- * forward; deterministic like the forward.
+ * B*H <= 65535.  Arithmetic: the score and gradient products on the tensor
+ * cores with tf32 operands (bf16 inputs are exact in tf32) and fp32
+ * accumulation; softmax weights, normalisers and every reduction in fp32;
+ * the FLARE++ projections recomputed in bf16 as in the forward.
+ * Deterministic like the forward.
  *
  * flare_mixer_bwd (FLARE, eq. 5-6), workspace variant FLARE_VARIANT_FLARE_BWD:
  *   K, V, Q, lengths, scale   as in flare_mixer_fwd
