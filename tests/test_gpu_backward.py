@@ -205,3 +205,17 @@ def test_backward_cuda_graph_replays_the_same_bits():
         assert torch.equal(g[k].view(torch.int16) if g[k].dtype == torch.bfloat16 else g[k],
                            eager[k].view(torch.int16) if eager[k].dtype == torch.bfloat16 else eager[k]), k
     del graph
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["flare_n64k", "flarepp_n64k"])
+def test_backward_full_size(name):
+    """The 64K-token configurations at full size (B=4, N=65536, M=256): every
+    gradient against the fp64 oracle (15-60 s of host time)."""
+    w = make_workload(name)
+    dY = make_upstream_grad(w)
+    got = run_flare_bwd(w, dY) if w.variant == "flare" else run_flarepp_bwd(w, dY)
+    ref = oracle.backward_workload(w, dY)
+    keys = ("dK", "dV", "dQ") if w.variant == "flare" else ("dX", "dWk", "dWv", "dWk_syn", "dWv_syn", "dQ0")
+    for k in keys:
+        check(got[k], ref[k], f"{name} full {k}")
