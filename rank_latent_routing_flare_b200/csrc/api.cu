@@ -159,8 +159,9 @@ BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C) {
   BwdPlan bp;
   bp.fwd = make_plan(pp ? FLARE_VARIANT_FLAREPP : FLARE_VARIANT_FLARE, B, H, N, M, D);
   const long BH = B * H;
-  // latent-parallel passes: a warp per 16 latent rows, 2 to 8 warps per CTA
-  bp.rpb = static_cast<int>(std::min(128L, std::max(32L, cdiv(M, 16) * 16)));
+  // latent-parallel passes: 32, 64, 96 or 128 latent rows per CTA, so that
+  // both a warp per 16 rows and a warp per 32 rows give whole warps
+  bp.rpb = static_cast<int>(std::min(128L, cdiv(M, 32) * 32));
   bp.LB = static_cast<int>(cdiv(M, bp.rpb));
   // token splits: whole waves of CTAs (about 128 registers per thread, so
   // 256 / rows_per_block CTAs per SM), by the encoder's cost model

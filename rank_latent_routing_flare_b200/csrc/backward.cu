@@ -900,10 +900,13 @@ unsigned blocks_for(long n, int threads) { return static_cast<unsigned>((n + thr
 }  // namespace
 
 cudaError_t launch_lat(int mode, const LatParams& p, cudaStream_t s) {
+  if (p.rows_per_block % 32 != 0 || p.rows_per_block < 32 || p.rows_per_block > 128) return cudaErrorInvalidValue;
   // a warp per 16 latent rows (forward) or per 32 (two m-tiles sharing the B
   // fragments: the gradient modes, when the CTA keeps at least two warps)
   const dim3 grid(p.n_splits, (p.M + p.rows_per_block - 1) / p.rows_per_block, p.B * p.H);
-  const bool two = mode != kLatForward && p.rows_per_block >= 64 && p.D == 16;  // D = 32 would spill
+  // two m-tiles need rows_per_block / 32 whole warps, and at least two of them
+  // (the tile loads assume 64 threads); D = 32 would spill
+  const bool two = mode != kLatForward && p.rows_per_block >= 64 && p.rows_per_block % 32 == 0 && p.D == 16;
   const int threads = two ? p.rows_per_block : 2 * p.rows_per_block;
 #define FLARE_LAT(DD, MM, MT) lat_kernel<DD, MM, MT><<<grid, threads, 0, s>>>(p)
   if (p.D == 16) {

@@ -69,6 +69,8 @@ def flare_case(B, H, N, M, D, lengths=None, seed=5):
     (1, 3, 1000, 48, 32, None),
     (3, 2, 200, 16, 16, [1, 200, 129]),
     (2, 2, 2000, 256, 32, [2000, 1537]),
+    (1, 2, 700, 80, 16, None),        # M = 80: 96 latent rows per CTA, the last 16 idle
+    (1, 2, 500, 112, 16, [433]),      # M = 112
 ])
 def test_flare_backward_matches_oracle(B, H, N, M, D, lengths):
     w = flare_case(B, H, N, M, D, lengths)
