@@ -254,7 +254,7 @@ def cpu_model():
 # ---------------------------------------------------------------------------
 
 BWD_METRIC = "mixer bwd token·heads/s at N=1M (1×B200) and % of roofline (HBM/MMA/MUFU)"
-BWD_LAUNCHES = 23        # kernels per FLARE++ backward call (projections, recompute, gradients, GEMMs)
+BWD_LAUNCHES = 24        # kernels per FLARE++ backward call (projections, recompute, gradients, GEMMs)
 BWD_LAUNCHES_FLARE = 12  # kernels per FLARE backward call (recompute, gradients, merges, pads)
 TF32_PER_BF16 = 0.5  # nominal dense tf32 : bf16 tensor throughput
 

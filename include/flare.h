@@ -225,6 +225,43 @@ FLARE_API flare_status flarepp_mixer_bwd(const flare_bf16* X, const flare_bf16* 
                                          size_t workspace_bytes, void* stream);
 
 /*
+ * Context-parallel FLARE++ backward (the token-sharded encoder of section
+ * "Multi-GPU context parallelism", eq. 13-14, with its backward).
+ *
+ * Token sharding as for the forward phases (rank r holds tokens
+ * [r*N, (r+1)*N) of sequences of world*N tokens; X, dY and dX are the shard's
+ * rows; `lengths` counts tokens of the whole sequences).  The backward runs in
+ * FLARE_CP_BWD_PHASES phases, all with the same arguments except `phase`,
+ * `gathered` and `exchange`:
+ *
+ *   for phase = 0 .. FLARE_CP_BWD_PHASES - 1:
+ *     flarepp_cp_bwd_phase(phase, ..., gathered, exchange, ...)
+ *     gathered = all-gather of every rank's `exchange`, in rank order
+ *
+ * Phase p (< FLARE_CP_BWD_PHASES - 1) writes flarepp_cp_bwd_exchange_bytes(p,
+ * ...) bytes (fp32) to `exchange`; phase p > 0 reads `gathered` = world of
+ * those buffers of phase p - 1, rank-major (NULL for phase 0; `exchange` is
+ * NULL for the last phase).  Every rank merges the gathered buffers in the
+ * same ascending (rank, split) order, so every rank ends with bitwise the
+ * same dW_K, dW_V, dW~_K, dW~_V and dQ0 (written by the last two phases);
+ * dX holds the shard's rows.  With world == 1 the result equals
+ * flarepp_mixer_bwd bit for bit.  The phases of one rank share its workspace
+ * (flare_workspace_bytes(FLARE_VARIANT_FLAREPP_BWD, ...) with the shard's N)
+ * and carry the shard's state in it; the other arguments are as for
+ * flarepp_mixer_bwd.  An out-of-range phase returns FLARE_ERR_SHAPE.
+ */
+#define FLARE_CP_BWD_PHASES 7
+FLARE_API size_t flarepp_cp_bwd_exchange_bytes(int phase, int B, int N, int C, int H, int M, int D);
+FLARE_API flare_status flarepp_cp_bwd_phase(int phase, const flare_bf16* X, const flare_bf16* Wk,
+                                            const flare_bf16* Wv, const flare_bf16* Wk_syn,
+                                            const flare_bf16* Wv_syn, const flare_bf16* Q0, const flare_bf16* dY,
+                                            const float* gathered, float* exchange, flare_bf16* dX, float* dWk,
+                                            float* dWv, float* dWk_syn, float* dWv_syn, float* dQ0, int B, int N,
+                                            int C, int H, int M, int D, const int32_t* lengths, int rank,
+                                            int world, float scale, void* workspace, size_t workspace_bytes,
+                                            void* stream);
+
+/*
  * Synchronises `stream`, reads the device error word of `workspace` and
  * returns FLARE_OK, FLARE_ERR_TIMEOUT, FLARE_ERR_SHAPE (invalid lengths) or
  * FLARE_ERR_UNDERFLOW (context-parallel merges only).

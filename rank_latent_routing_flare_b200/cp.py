@@ -1,4 +1,5 @@
-"""Context-parallel FLARE / FLARE++ forward over torch.distributed.
+"""Context-parallel FLARE / FLARE++ forward (and FLARE++ backward) over
+torch.distributed.
 
 The FLARE++ paper (arXiv 2608.11519, section "Multi-GPU context parallelism",
 eq. 13-14) shards the tokens of every sequence across ranks.  The projections
@@ -97,3 +98,48 @@ def flare_mixer_cp_fwd(K, V, Q, lengths=None, group=None, scale: float = 0.0, Y=
     _status(lib.flare_cp_end(b._ptr(gathered), b._ptr(K), b._ptr(Q), b._ptr(Y), *common, b._ptr(Z_out)),
             "flare_cp_end")
     return Y
+
+
+FLARE_CP_BWD_PHASES = 7
+
+
+def flarepp_mixer_cp_bwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, lengths=None, group=None, scale: float = 0.0,
+                         workspace=None, stream=None, grads=None):
+    """FLARE++ backward of this rank's token shard (the same sharding as
+    flarepp_mixer_cp_fwd; dY [B, H, N, D] holds the shard's rows).  Returns a
+    dict: dX [B, N, C] (the shard's rows), dWk, dWv, dWk_syn, dWv_syn, dQ0
+    (bitwise the same on every rank).  Seven phases with one all-gather of a
+    small fp32 buffer between two of them."""
+    torch = b._torch()
+    rank, world = _group_info(group)
+    B, N, C = X.shape
+    H, M, D = Q0.shape
+    dev = X.device
+    lib = b.load_library()
+    g = dict(grads or {})
+    if g.get("dX") is None:
+        g["dX"] = torch.empty((B, N, C), dtype=torch.bfloat16, device=dev)
+    for nm in ("dWk", "dWv", "dWk_syn", "dWv_syn"):
+        if g.get(nm) is None:
+            g[nm] = torch.empty((C, C), dtype=torch.float32, device=dev)
+    if g.get("dQ0") is None:
+        g["dQ0"] = torch.empty((H, M, D), dtype=torch.float32, device=dev)
+    nbytes = b.flare_workspace_bytes(b.FLARE_VARIANT_FLAREPP_BWD, B, H, N, M, D, C)
+    ws = b._workspace(workspace, nbytes, dev)
+    st = b._stream_ptr(stream, dev)
+    ins = [b._ptr(t) for t in (X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY)]
+    outs = [b._ptr(g[k]) for k in ("dX", "dWk", "dWv", "dWk_syn", "dWv_syn", "dQ0")]
+    gathered = None
+    for phase in range(FLARE_CP_BWD_PHASES):
+        exch = None
+        if phase < FLARE_CP_BWD_PHASES - 1:
+            nb = lib.flarepp_cp_bwd_exchange_bytes(phase, B, N, C, H, M, D)
+            if nb == 0:
+                raise ValueError("unsupported sizes")
+            exch = torch.empty(nb // 4, dtype=torch.float32, device=dev)
+        _status(lib.flarepp_cp_bwd_phase(phase, *ins, b._ptr(gathered), b._ptr(exch), *outs, B, N, C, H, M, D,
+                                         b._ptr(lengths), rank, world, float(scale), b._ptr(ws), ws.numel(), st),
+                f"flarepp_cp_bwd_phase({phase})")
+        if exch is not None:
+            gathered = allgather_partials(exch, world, group)
+    return g

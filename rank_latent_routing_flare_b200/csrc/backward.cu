@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(256) lat_kernel(const LatParams p) {
   const int b = bh / p.H, h = bh % p.H;
   const int gq = p.q_per_batch ? bh : h;
   bool bad = false;
-  const int L = shard_valid_len(p.lengths, b, p.N, 0, p.N, &bad);
+  const int L = shard_valid_len(p.lengths, b, p.N, p.tok_offset, p.n_global, &bad);
   if (bad && threadIdx.x == 0 && split == 0 && blockIdx.y == 0) atomicOr(p.err, FLARE_DEV_BAD_LENGTH);
   const int ntv = (L + T - 1) / T;
   const int t_begin = split * p.tiles_per_split;
@@ -411,16 +411,17 @@ __global__ void __launch_bounds__(256) lat_merge_kernel(const LatMergeParams p) 
   const long bh = r / p.M, m = r % p.M;
   const size_t sstride = static_cast<size_t>(p.M) * (D + 2);
   const float* base = p.part + (static_cast<size_t>(bh) * p.S * p.M + m) * (D + 2);
+  // splits in ascending (rank, split) order
   float G = -INFINITY;
-  for (int s = 0; s < p.S; ++s) {
-    const float* e = base + s * sstride;
+  for (int j = 0; j < p.R * p.S; ++j) {
+    const float* e = base + (j / p.S) * p.rank_stride + (j % p.S) * sstride;
     if (e[1] > 0.f) G = fmaxf(G, e[0]);
   }
   float den = 0.f, acc[D];
 #pragma unroll
   for (int d = 0; d < D; ++d) acc[d] = 0.f;
-  for (int s = 0; s < p.S; ++s) {
-    const float* e = base + s * sstride;
+  for (int j = 0; j < p.R * p.S; ++j) {
+    const float* e = base + (j / p.S) * p.rank_stride + (j % p.S) * sstride;
     if (!(e[1] > 0.f)) continue;
     const float w = ex2_mufu(e[0] - G);
     den = fmaf(w, e[1], den);
@@ -449,8 +450,10 @@ __global__ void __launch_bounds__(256) lat_sum_kernel(const LatSumParams p) {
     for (int pi = 0; pi < 2; ++pi) {
       const float* part = pi == 0 ? p.part0 : p.part1;
       if (part == nullptr) continue;
-      for (int s = 0; s < p.S; ++s) {
-        const float4* e = reinterpret_cast<const float4*>(part + ((static_cast<size_t>(bh) * p.S + s) * p.M + m) * D);
+      for (int j = 0; j < p.R * p.S; ++j) {  // ascending (rank, split)
+        const int s = j % p.S;
+        const float4* e = reinterpret_cast<const float4*>(part + (j / p.S) * p.rank_stride +
+                                                          ((static_cast<size_t>(bh) * p.S + s) * p.M + m) * D);
 #pragma unroll
         for (int u = 0; u < D / 4; ++u) {
           const float4 t = e[u];
@@ -466,6 +469,7 @@ __global__ void __launch_bounds__(256) lat_sum_kernel(const LatSumParams p) {
 #pragma unroll
   for (int d = 0; d < D; ++d) {
     acc[d] *= p.mult;
+    if (p.addend) acc[d] += p.addend[static_cast<size_t>(r) * D + d];
     p.out[static_cast<size_t>(r) * D + d] = acc[d];
     if (p.zref) gsum = fmaf(acc[d], p.zref[static_cast<size_t>(r) * D + d], gsum);
   }
@@ -497,7 +501,7 @@ __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
   const int bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
   const int gq = p.q_per_batch ? bh : h;
   bool bad = false;
-  const int L = shard_valid_len(p.lengths, b, p.N, 0, p.N, &bad);
+  const int L = shard_valid_len(p.lengths, b, p.N, p.tok_offset, p.n_global, &bad);
   // this thread's token rows: m-tile mt of the warp, rows g (i = 0) and g + 8 (i = 1)
   int rr[MT][2];
   bool in[MT][2];

@@ -23,6 +23,7 @@ enum LatMode : int {
 
 struct LatParams {
   int B, H, N, M, D;
+  int tok_offset, n_global;     // this shard holds tokens [tok_offset, tok_offset + N) of n_global
   int q_per_batch;              // queries [G][M][D] with G = B*H (1) or H (0)
   int n_splits, tiles_per_split, rows_per_block;   // rows_per_block: 16 per warp, at most 128
   float c;                      // scale * log2(e)
@@ -43,7 +44,9 @@ struct LatParams {
 
 struct LatMergeParams {
   int BH, M, D, S;
-  const float* part;            // [B*H][S][M][D+2]
+  int R;                        // shards (ranks), partials rank-major
+  size_t rank_stride;           // floats between two ranks' partials
+  const float* part;            // [R][B*H][S][M][D+2]
   float* z;                     // [B*H][M][D]
   float* lse;                   // [B*H][M], log2 units
 };
@@ -52,11 +55,14 @@ struct LatSumParams {
   int B, H, M, D, S;
   int fold_batch;               // 1: out [H][M][D] sums the batch; 0: out [B*H][M][D]
   float mult;
-  const float* part0;           // [B*H][S][M][D]
+  const float* part0;           // [R][B*H][S][M][D] (rank-major)
   const float* part1;           // same shape or NULL
   const float* zref;            // [B*H][M][D] or NULL: gamma = <out, zref> per row
   float* gamma;                 // [B*H][M]
-  float* out;                   // fp32
+  float* out;                   // fp32: out = addend + mult * sum
+  int R;                        // shards (ranks)
+  size_t rank_stride;           // floats between two ranks' partials
+  const float* addend;          // same shape as out, or NULL
 };
 
 // Modes of the token-parallel kernel (one CTA = kBwdTokBlock tokens of one
@@ -69,6 +75,7 @@ enum TokMode : int {
 
 struct TokParams {
   int B, H, N, M, D;
+  int tok_offset, n_global;     // this shard holds tokens [tok_offset, tok_offset + N) of n_global
   int q_per_batch;
   float c;
   const int32_t* lengths;

@@ -34,7 +34,8 @@ def test_header_declares_the_abi():
                             "flare_last_device_status", "flare_status_string",
                             "flare_selftest_wait_timeout", "flare_cp_partials_bytes", "flarepp_cp_begin",
                             "flarepp_cp_middle", "flarepp_cp_end", "flare_cp_begin", "flare_cp_end",
-                            "flare_mixer_bwd", "flarepp_mixer_bwd"])
+                            "flare_mixer_bwd", "flarepp_mixer_bwd", "flarepp_cp_bwd_exchange_bytes",
+                            "flarepp_cp_bwd_phase"])
 
 
 def test_library_loads_and_exports_every_declared_symbol():
@@ -270,3 +271,42 @@ def test_backward_valid_calls_without_gpu_report_launch_error():
     assert flarepp_bwd_call() == Status.ERR_LAUNCH
     # shared projections: the synthesis weight gradients may be NULL
     assert flarepp_bwd_call(Wks=A, Wvs=A, dWks=None, dWvs=None) == Status.ERR_LAUNCH
+
+
+def cp_bwd_call(phase=0, gathered=None, exchange=A, rank=0, world=2, B=1, N=100, C=64, H=4, M=32, D=16, ws=W,
+                ws_bytes=None, dX=A):
+    lib = fl.load_library()
+    if ws_bytes is None:
+        ws_bytes = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLAREPP_BWD, B, H, N, M, D, C) or (1 << 40)
+    return lib.flarepp_cp_bwd_phase(phase, A, A, A, A + 0x100, A + 0x200, A, A, gathered, exchange, dX, A, A, A, A,
+                                    A, B, N, C, H, M, D, None, rank, world, 0.0, ws, ws_bytes, None)
+
+
+def test_cp_backward_exchange_sizes():
+    lib = fl.load_library()
+    sizes = [lib.flarepp_cp_bwd_exchange_bytes(p, 1, 1000, 64, 4, 32, 16) for p in range(8)]
+    assert all(x > 0 and x % 16 == 0 for x in sizes[:6]) and sizes[6] == 0 and sizes[7] == 0
+    assert sizes[0] == sizes[1] and sizes[3] == sizes[4]
+    assert sizes[2] == 2 * sizes[3]                       # [dZ | dQ] partials
+    assert lib.flarepp_cp_bwd_exchange_bytes(0, 1, 1000, 128, 4, 32, 16) == 0   # C != H*D
+    assert lib.flarepp_cp_bwd_exchange_bytes(-1, 1, 1000, 64, 4, 32, 16) == 0
+
+
+def test_cp_backward_argument_errors():
+    assert cp_bwd_call(phase=7) == Status.ERR_SHAPE
+    assert cp_bwd_call(phase=-1) == Status.ERR_SHAPE
+    assert cp_bwd_call(rank=2, world=2) == Status.ERR_SHAPE
+    assert cp_bwd_call(phase=1, gathered=None) == Status.ERR_NULL   # phases after the first read the gather
+    assert cp_bwd_call(phase=0, exchange=None) == Status.ERR_NULL
+    assert cp_bwd_call(phase=6, gathered=A, exchange=None, dX=None) == Status.ERR_NULL
+    assert cp_bwd_call(phase=2, gathered=A + 4) == Status.ERR_ALIGN
+    need = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLAREPP_BWD, 1, 4, 100, 32, 16, 64)
+    assert cp_bwd_call(ws_bytes=need - 256) == Status.ERR_WORKSPACE
+
+
+def test_cp_backward_valid_call_without_gpu_reports_launch_error():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert cp_bwd_call() == Status.ERR_LAUNCH
+    assert cp_bwd_call(phase=6, gathered=A, exchange=None) == Status.ERR_LAUNCH

@@ -1,0 +1,108 @@
+"""GPU parity of the context-parallel FLARE++ backward (FLARE++ paper,
+section "Multi-GPU context parallelism", eq. 13-14: the token-sharded encoder
+and its backward).
+
+One GPU plays R ranks: each rank runs the seven phases of
+flarepp_cp_bwd_phase through the C ABI on its own token shard and workspace,
+and the all-gather between two phases is a concatenation in rank order.
+Checked: with one rank the phases reproduce flarepp_mixer_bwd bit for bit;
+with several ranks every rank holds bitwise the same weight and seed
+gradients, and the gradients (dX from the shards' rows) match the fp64
+oracle on the whole sequences, including a rank whose shard has no valid
+token of a sample.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rank_latent_routing_flare_b200 as fl
+from workloads import make_upstream_grad, make_workload
+
+from .gpu_util import dev_bf16, host_f64, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+PHASES = 7
+KEYS = ("dX", "dWk", "dWv", "dWk_syn", "dWv_syn", "dQ0")
+
+
+def check(got, ref, label, bound=5e-3):
+    r = rel_l2(got, ref)
+    m = float(np.max(np.abs(got - ref)) / max(np.max(np.abs(ref)), 1e-30))
+    print(f"{label}: rel_l2={r:.3e} max_err/max_ref={m:.3e}")
+    assert r <= bound and m <= 3e-2, (label, r, m)
+
+
+def emulate(w, dY, R):
+    lib = fl.load_library()
+    B, N, C, H, M, D = w.B, w.N // R, w.C, w.H, w.M, w.D
+    X, dYd = dev_bf16(w.X), dev_bf16(dY)
+    Ws = [dev_bf16(a) for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn)]
+    Q0 = dev_bf16(w.Q0)
+    lengths = None if w.lengths is None else torch.from_numpy(w.lengths).cuda()
+    lp = None if lengths is None else lengths.data_ptr()
+    nbytes = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLAREPP_BWD, B, H, N, M, D, C)
+    st = torch.cuda.current_stream().cuda_stream
+    Xs = [X[:, r * N:(r + 1) * N].contiguous() for r in range(R)]
+    dYs = [dYd[:, :, r * N:(r + 1) * N].contiguous() for r in range(R)]
+    wss = [torch.empty(nbytes, dtype=torch.uint8, device="cuda") for _ in range(R)]
+    outs = [{"dX": torch.empty((B, N, C), dtype=torch.bfloat16, device="cuda"),
+             **{k: torch.empty((C, C), dtype=torch.float32, device="cuda") for k in KEYS[1:5]},
+             "dQ0": torch.empty((H, M, D), dtype=torch.float32, device="cuda")} for _ in range(R)]
+    gathered = None
+    for phase in range(PHASES):
+        exch = [None] * R
+        if phase < PHASES - 1:
+            nb = lib.flarepp_cp_bwd_exchange_bytes(phase, B, N, C, H, M, D)
+            assert nb > 0
+            exch = [torch.empty(nb // 4, dtype=torch.float32, device="cuda") for _ in range(R)]
+        for r in range(R):
+            rc = lib.flarepp_cp_bwd_phase(
+                phase, Xs[r].data_ptr(), *[a.data_ptr() for a in Ws], Q0.data_ptr(), dYs[r].data_ptr(),
+                None if gathered is None else gathered.data_ptr(), None if exch[r] is None else exch[r].data_ptr(),
+                *[outs[r][k].data_ptr() for k in KEYS], B, N, C, H, M, D, lp, r, R, 0.0, wss[r].data_ptr(), nbytes,
+                st)
+            assert rc == 0, (phase, r, rc)
+        if phase < PHASES - 1:
+            gathered = torch.cat(exch)
+    torch.cuda.synchronize()
+    for r in range(R):
+        assert fl.flare_last_device_status(wss[r]) == fl.Status.OK
+    return outs
+
+
+def test_one_rank_reproduces_the_single_gpu_backward():
+    w = make_workload("flarepp_n1k", N=900)
+    dY = make_upstream_grad(w)
+    outs = emulate(w, dY, 1)[0]
+    g = fl.flarepp_mixer_bwd(dev_bf16(w.X), dev_bf16(w.Wk), dev_bf16(w.Wv), dev_bf16(w.Wk_syn),
+                             dev_bf16(w.Wv_syn), dev_bf16(w.Q0), dev_bf16(dY))
+    torch.cuda.synchronize()
+    for k in KEYS:
+        a, b = outs[k], g[k]
+        if a.dtype == torch.bfloat16:
+            a, b = a.view(torch.int16), b.view(torch.int16)
+        assert torch.equal(a, b), k
+
+
+@pytest.mark.parametrize("name,N,B,R,lengths", [
+    ("flarepp_n1k", 1024, 1, 2, None),
+    ("flarepp_n8k_mesh2d", 1536, 2, 3, [1536, 700]),      # rank 2 holds no valid token of sample 1
+    ("flarepp_masked_n4k", 512, 2, 4, [512, 77]),         # D = 32; ranks 1-3 empty for sample 1
+])
+def test_sharded_backward_matches_oracle(name, N, B, R, lengths):
+    w = make_workload(name, N=N, B=B, lengths=None if lengths is None else np.array(lengths, dtype=np.int32))
+    dY = make_upstream_grad(w)
+    outs = emulate(w, dY, R)
+    for r in range(1, R):
+        for k in KEYS[1:]:
+            assert torch.equal(outs[r][k], outs[0][k]), (r, k)
+    got = {k: host_f64(outs[0][k]) for k in KEYS[1:]}
+    got["dX"] = np.concatenate([host_f64(outs[r]["dX"]) for r in range(R)], axis=1)
+    ref = oracle.backward_workload(w, dY)
+    for k in KEYS:
+        check(got[k], ref[k], f"{name} R={R} {k}")
+    if lengths is not None:
+        for b, L in enumerate(lengths):
+            assert np.all(got["dX"][b, L:] == 0)
