@@ -52,3 +52,81 @@ def test_single_rank_without_process_group():
     part = torch.ones(3)
     assert cp._group_info(None) == (0, 1)
     assert cp.allgather_partials(part, 1) is part
+
+
+class _FakeLib:
+    """Stands in for libflare.so: records the backward phases and fills each
+    exchange buffer with (rank, phase) markers, and records what each phase
+    was handed as `gathered`."""
+
+    def __init__(self, rank):
+        self.rank = rank
+        self.calls = []
+
+    def flarepp_cp_bwd_exchange_bytes(self, phase, B, N, C, H, M, D):
+        return 4 * (3 + phase) if 0 <= phase < 6 else 0
+
+    def flarepp_cp_bwd_phase(self, phase, *args):
+        import ctypes
+        gathered, exchange = args[7], args[8]
+        rank_arg, world_arg = args[22], args[23]   # after B, N, C, H, M, D and lengths
+        seen = None
+        if gathered:
+            n = 2 * (3 + phase - 1)
+            seen = list((ctypes.c_float * n).from_address(gathered))
+        if exchange:
+            n = 3 + phase
+            buf = (ctypes.c_float * n).from_address(exchange)
+            for i in range(n):
+                buf[i] = 100 * self.rank + 10 * phase + i
+        self.calls.append((phase, rank_arg, world_arg, seen, bool(exchange)))
+        return 0
+
+
+def _bwd_rank_main(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import torch.distributed as dist
+    from rank_latent_routing_flare_b200 import _binding, cp
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        fake = _FakeLib(rank)
+        _binding.load_library = lambda *a, **k: fake
+        _binding.flare_workspace_bytes = lambda *a, **k: 256
+
+        class _Stream:
+            cuda_stream = 0
+        B, N, C, H, M, D = 1, 4, 64, 4, 2, 16
+        X = torch.zeros((B, N, C), dtype=torch.bfloat16)
+        W = torch.zeros((C, C), dtype=torch.bfloat16)
+        Q0 = torch.zeros((H, M, D), dtype=torch.bfloat16)
+        dY = torch.zeros((B, H, N, D), dtype=torch.bfloat16)
+        cp.flarepp_mixer_cp_bwd(X, W, W, W, W, Q0, dY, stream=_Stream())
+        out.put((rank, fake.calls))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_backward_phases_run_in_order_with_rank_ordered_gathers():
+    world = 2
+    ctx = multiprocessing.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bwd_rank_main, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = sorted(out.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, calls in results:
+        assert [c[0] for c in calls] == list(range(7))
+        assert all(c[1] == rank and c[2] == world for c in calls)
+        assert calls[0][3] is None                       # nothing gathered before phase 0
+        assert [c[4] for c in calls] == [True] * 6 + [False]   # no exchange after the last phase
+        for phase in range(1, 7):
+            n = 3 + phase - 1
+            want = [float(10 * (phase - 1) + i) for i in range(n)] + \
+                   [float(100 + 10 * (phase - 1) + i) for i in range(n)]
+            assert calls[phase][3] == want, (rank, phase)
