@@ -1,6 +1,8 @@
-// Host entry points of the C ABI declared in include/flare.h: argument
-// validation (before anything is enqueued), workspace layout, TMA tensor maps
-// and the launch sequence of the FLARE / FLARE++ forward.
+// Host entry points of the C ABI declared in include/flare.h, forward side:
+// argument validation (before anything is enqueued), workspace layout, TMA
+// tensor maps and the launch sequences of the FLARE / FLARE++ forward and of
+// its context-parallel phases.  The backward's entry points are in
+// api_bwd.cu; host_internal.h declares what the two share.
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -9,9 +11,9 @@
 #include "bwd_internal.h"
 #include "flare.h"
 #include "flare_internal.h"
+#include "host_internal.h"
 
 namespace flare {
-namespace {
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -68,8 +70,6 @@ bool map2d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint32_t 
 
 CUtensorMapSwizzle row_swizzle(int D) { return D == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B; }
 
-size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-long cdiv(long a, long b) { return (a + b - 1) / b; }
 
 // Number of token splits of the encoder.  Cost model: the CTAs run in
 // waves of `slots` (CTAs resident on the whole GPU); a wave lasts as long as
@@ -93,13 +93,6 @@ int choose_splits(long units, long ntiles, long slots) {
   return best;
 }
 
-struct Plan {
-  int S = 1, tps = 1, LB = 1;            // encoder splits, tiles per split, latent blocks
-  int dec_ctas = 1, dec_tiles = 1;       // decoder CTAs per head, tiles per CTA
-  int G32 = 1;
-  size_t off_err = 0, off_kt = 0, off_vt = 0, off_kp = 0, off_vp = 0, off_kn_syn = 0, off_kn = 0, off_part = 0,
-         off_qx32 = 0, off_qx16 = 0, off_z32 = 0, off_z16 = 0, off_fb = 0, off_ycat = 0, total = 0;
-};
 
 Plan make_plan(int variant, long B, long H, long N, long M, long D) {
   Plan p;
@@ -144,82 +137,12 @@ Plan make_plan(int variant, long B, long H, long N, long M, long D) {
   return p;
 }
 
-// Workspace of the backward: the forward's (projection outputs, error word)
-// followed by the fp32 recompute and gradient buffers.
-struct BwdPlan {
-  Plan fwd;
-  int S = 1, tps = 1, rpb = 32, LB = 1, dw_splits = 1;
-  size_t off_q32 = 0, off_qx32 = 0, off_lsyn = 0, off_dqx32 = 0, off_gsyn = 0, off_z32 = 0, off_lenc = 0,
-         off_ltok = 0, off_dtok = 0, off_dz32 = 0, off_gam = 0, off_fpart = 0, off_pa = 0, off_pc = 0,
-         off_g32 = 0, off_dwpart = 0, off_qpad = 0, off_q0pad = 0, off_zpad = 0, off_dzpad = 0, off_dqxpad = 0,
-         off_dqxdec = 0, total = 0;
-};
-
-BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C) {
-  BwdPlan bp;
-  bp.fwd = make_plan(pp ? FLARE_VARIANT_FLAREPP : FLARE_VARIANT_FLARE, B, H, N, M, D);
-  const long BH = B * H;
-  // latent-parallel passes: 32, 64, 96 or 128 latent rows per CTA, so that
-  // both a warp per 16 rows and a warp per 32 rows give whole warps
-  bp.rpb = static_cast<int>(std::min(128L, cdiv(M, 32) * 32));
-  bp.LB = static_cast<int>(cdiv(M, bp.rpb));
-  // token splits: whole waves of CTAs (about 128 registers per thread, so
-  // 256 / rows_per_block CTAs per SM), by the encoder's cost model
-  const long ntiles = cdiv(N, kBwdTokTile);
-  bp.S = choose_splits(BH * bp.LB, ntiles, static_cast<long>(kNumSM) * std::max(1, 256 / bp.rpb));
-  bp.tps = static_cast<int>(cdiv(ntiles, bp.S));
-  bp.S = static_cast<int>(cdiv(ntiles, bp.tps));
-  bp.dw_splits = static_cast<int>(cdiv(B * N, kBwdDwRows));
-  size_t off = bp.fwd.total;
-  auto take = [&off](size_t bytes) {
-    const size_t o = off;
-    off += align256(bytes);
-    return o;
-  };
-  const size_t lat = static_cast<size_t>(BH * M * D) * 4, row = static_cast<size_t>(BH * M) * 4;
-  const size_t tokv = static_cast<size_t>(BH * N) * 4;
-  const size_t part = static_cast<size_t>(BH) * bp.S * M * D * 4;
-  bp.off_q32 = take(static_cast<size_t>(H * M * D) * 4);
-  if (pp) {
-    bp.off_qx32 = take(lat);
-    bp.off_lsyn = take(row);
-    bp.off_dqx32 = take(lat);
-    bp.off_gsyn = take(row);
-  }
-  bp.off_z32 = take(lat);
-  bp.off_lenc = take(row);
-  bp.off_ltok = take(tokv);
-  bp.off_dtok = take(tokv);
-  bp.off_dz32 = take(lat);
-  bp.off_gam = take(row);
-  bp.off_fpart = take(static_cast<size_t>(BH) * bp.S * M * (D + 2) * 4);
-  bp.off_pa = take(2 * part);  // [dZ partials | dQ partials] of the decoder backward
-  bp.off_pc = take(part);
-  // padded tf32 images ([rows][D + 4]) read by the token-parallel pass
-  const size_t padded = static_cast<size_t>(BH * M * (D + 4)) * 4;
-  bp.off_qpad = take(padded);
-  bp.off_zpad = take(padded);
-  bp.off_dzpad = take(padded);
-  if (pp) {
-    bp.off_q0pad = take(static_cast<size_t>(H * M * (D + 4)) * 4);
-    bp.off_dqxpad = take(padded);
-    bp.off_dqxdec = take(lat);
-  }
-  if (pp) {
-    bp.off_g32 = take(static_cast<size_t>(B * N) * 4 * C * 4);
-    bp.off_dwpart = take(static_cast<size_t>(bp.dw_splits) * C * 4 * C * 4);
-  }
-  bp.total = off;
-  return bp;
-}
-
 // Records stage event i (a cudaEvent_t passed as void*) when profiling is on.
 bool record(void* const* ev, int i, cudaStream_t s) {
   if (ev == nullptr || ev[i] == nullptr) return true;
   return cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) == cudaSuccess;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 flare_status check_common(int B, int H, int N, int M, int D) {
   if (B < 1 || H < 1 || N < 1 || M < 1 || D < 1) return FLARE_ERR_SHAPE;
@@ -334,11 +257,9 @@ flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
   return FLARE_OK;
 }
 
-}  // namespace
 }  // namespace flare
 
 namespace flare {
-namespace {
 
 // Scratch for callers that cannot allocate device memory (see
 // flare_mixer_fwd_static): a fixed array in the library's device image.
@@ -363,7 +284,6 @@ flare_status static_scratch_address(void** out) {
   return FLARE_OK;
 }
 
-}  // namespace
 }  // namespace flare
 
 using namespace flare;
@@ -436,7 +356,6 @@ flare_status flare_mixer_fwd(const flare_bf16* K, const flare_bf16* V, const fla
 }  // extern "C"
 
 namespace flare {
-namespace {
 
 // Shape, pointer and alignment checks shared by the FLARE++ entry points.
 flare_status check_flarepp(const void* X, const void* Wk, const void* Wv, const void* Wk_syn, const void* Wv_syn,
@@ -477,11 +396,6 @@ flare_status run_project(const Plan& pl, uint8_t* ws, const CUtensorMap& tx, con
   return launch_project(tx, tw, pp, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
 
-// Outputs of the FLARE++ projections in the workspace.
-struct Projected {
-  uint16_t *kt, *vt, *kk, *vv;
-  float *kn_syn, *kn;
-};
 
 // eq. 7 and eq. 9: the per-head projections of X (two when the synthesis
 // and encode weights are the same tensors, else four).
@@ -551,7 +465,6 @@ flare_status flarepp_run(const Plan& pl, const flare_bf16* X, const flare_bf16* 
   return record(stage_events, 6, s) ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
 
-}  // namespace
 }  // namespace flare
 
 extern "C" {
@@ -623,7 +536,6 @@ size_t flare_cp_partials_bytes(int B, int H, int N, int M, int D) {
 }  // extern "C"
 
 namespace flare {
-namespace {
 
 flare_status check_cp(int N, int rank, int world, const void* part) {
   if (!part) return FLARE_ERR_NULL;
@@ -633,7 +545,6 @@ flare_status check_cp(int N, int rank, int world, const void* part) {
   return FLARE_OK;
 }
 
-}  // namespace
 }  // namespace flare
 
 extern "C" {
@@ -789,433 +700,6 @@ flare_status flare_selftest_wait_timeout(void* workspace, void* stream, unsigned
   if (cudaMemsetAsync(workspace, 0, 4, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   if (launch_wait_selftest(static_cast<uint32_t*>(workspace), timeout_ns, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   return FLARE_OK;
-}
-
-}  // extern "C"
-
-// ---------------------------------------------------------------------------
-// Backward (gradients)
-// ---------------------------------------------------------------------------
-
-namespace flare {
-namespace {
-
-constexpr float kLog2e = 1.4426950408889634f;
-
-// Where the token-parallel pass writes dK and dV: token-major fp32 rows of
-// the projection-gradient matrix, or bf16 [B][H][N][D] outputs.
-struct TokOut {
-  float* g32;
-  int g_ld, col_k, col_v;
-  uint16_t *dk16, *dv16;
-};
-
-// This GPU's token shard: tokens [tok_offset, tok_offset + N) of sequences
-// of n_global tokens, one of R shards (R = 1: the whole sequence).
-struct Shard {
-  int tok_offset, n_global, R;
-};
-
-LatParams lat_params(const BwdPlan& bp, uint8_t* ws, const float* q, int q_per_batch, const void* k, int B, int H,
-                     int N, int M, int D, const int32_t* lengths, float sc, const Shard& sh) {
-  LatParams lp{};
-  lp.B = B; lp.H = H; lp.N = N; lp.M = M; lp.D = D;
-  lp.tok_offset = sh.tok_offset; lp.n_global = sh.n_global;
-  lp.q_per_batch = q_per_batch;
-  lp.n_splits = bp.S; lp.tiles_per_split = bp.tps; lp.rows_per_block = bp.rpb;
-  lp.c = sc * kLog2e;
-  lp.lengths = lengths;
-  lp.q = q;
-  lp.k = static_cast<const uint16_t*>(k);
-  lp.err = reinterpret_cast<uint32_t*>(ws + bp.fwd.off_err);
-  return lp;
-}
-
-TokParams tok_params(int B, int H, int N, int M, int D, int q_per_batch, const int32_t* lengths, float sc,
-                     const Shard& sh) {
-  TokParams tp{};
-  tp.B = B; tp.H = H; tp.N = N; tp.M = M; tp.D = D;
-  tp.tok_offset = sh.tok_offset; tp.n_global = sh.n_global;
-  tp.q_per_batch = q_per_batch;
-  tp.c = sc * kLog2e;
-  tp.lengths = lengths;
-  return tp;
-}
-
-// out = addend + mult * (sum over R shards and S splits of part0 (+ part1)),
-// gamma = <out, zref> per row when zref is given.
-flare_status lat_sum(int B, int H, int M, int D, int S, int fold_batch, float mult, const float* part0,
-                     const float* part1, int R, size_t rank_stride, const float* addend, const float* zref,
-                     float* gamma, float* out, cudaStream_t s) {
-  LatSumParams p{};
-  p.B = B; p.H = H; p.M = M; p.D = D; p.S = S;
-  p.fold_batch = fold_batch; p.mult = mult;
-  p.part0 = part0; p.part1 = part1; p.zref = zref; p.gamma = gamma; p.out = out;
-  p.R = R; p.rank_stride = rank_stride; p.addend = addend;
-  return launch_lat_sum(p, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
-}
-
-// Merge of the recompute partials of R shards: Z (or Q(X)) and L_m.
-flare_status lat_merge(const float* part, int R, size_t rank_stride, int BH, int M, int D, int S, float* z,
-                       float* lse, cudaStream_t s) {
-  LatMergeParams mp{};
-  mp.BH = BH; mp.M = M; mp.D = D; mp.S = S;
-  mp.R = R; mp.rank_stride = rank_stride;
-  mp.part = part; mp.z = z; mp.lse = lse;
-  return launch_lat_merge(mp, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
-}
-
-flare_status pad(const float* src, float* dst, long rows, int D, float mul, cudaStream_t s) {
-  const PadParams pp{rows, D, mul, src, dst};
-  return launch_pad(pp, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
-}
-
-// fp32 elements of one split-partials buffer [B*H][S][M][D] (+2 per row for
-// the recompute partials).
-size_t part_floats(const BwdPlan& bp, int B, int H, int M, int D, bool recompute) {
-  return static_cast<size_t>(B) * H * bp.S * M * (D + (recompute ? 2 : 0));
-}
-
-// FLARE (eq. 5-6) backward on one GPU: dK, dV to bf16 outputs, dQ summed
-// over the batch.
-flare_status flare_bwd_run(const BwdPlan& bp, uint8_t* ws, const float* q, const void* k, const void* v,
-                           const void* dy, uint16_t* dk, uint16_t* dv, float* dq, int B, int H, int N, int M, int D,
-                           const int32_t* lengths, float sc, cudaStream_t s) {
-  const Shard sh{0, N, 1};
-  const long BH = static_cast<long>(B) * H;
-  float* z32 = reinterpret_cast<float*>(ws + bp.off_z32);
-  float* lenc = reinterpret_cast<float*>(ws + bp.off_lenc);
-  float* dz32 = reinterpret_cast<float*>(ws + bp.off_dz32);
-  float* gam = reinterpret_cast<float*>(ws + bp.off_gam);
-  float* pa = reinterpret_cast<float*>(ws + bp.off_pa);
-  float* pb = pa + part_floats(bp, B, H, M, D, false);
-  float* pc = reinterpret_cast<float*>(ws + bp.off_pc);
-  float* qpad = reinterpret_cast<float*>(ws + bp.off_qpad);
-  float* zpad = reinterpret_cast<float*>(ws + bp.off_zpad);
-  float* dzpad = reinterpret_cast<float*>(ws + bp.off_dzpad);
-  // encoder recompute: Z and the row normalisers
-  LatParams lf = lat_params(bp, ws, q, 0, k, B, H, N, M, D, lengths, sc, sh);
-  lf.v = static_cast<const uint16_t*>(v);
-  lf.part_a = reinterpret_cast<float*>(ws + bp.off_fpart);
-  if (launch_lat(kLatForward, lf, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  flare_status st = lat_merge(lf.part_a, 1, 0, static_cast<int>(BH), M, D, bp.S, z32, lenc, s);
-  if (st != FLARE_OK) return st;
-  if ((st = pad(q, qpad, static_cast<long>(H) * M, D, sc * kLog2e, s)) != FLARE_OK ||
-      (st = pad(z32, zpad, BH * M, D, 1.f, s)) != FLARE_OK)
-    return st;
-  // decoder recompute: L_n and delta_n
-  TokParams tp = tok_params(B, H, N, M, D, 0, lengths, sc, sh);
-  tp.qpad = qpad; tp.zpad = zpad; tp.dzpad = dzpad; tp.lm = lenc; tp.gam = gam;
-  tp.k = static_cast<const uint16_t*>(k);
-  tp.v = static_cast<const uint16_t*>(v);
-  tp.dy = static_cast<const uint16_t*>(dy);
-  tp.ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
-  tp.dtok = reinterpret_cast<float*>(ws + bp.off_dtok);
-  tp.dk16 = dk; tp.dv16 = dv;
-  if (launch_tok(kTokStats, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  // decoder backward, reductions over tokens: dZ and the decoder's dQ
-  LatParams ld = lat_params(bp, ws, q, 0, k, B, H, N, M, D, lengths, sc, sh);
-  ld.zrow = z32; ld.dy = tp.dy; ld.ltok = tp.ltok; ld.dtok = tp.dtok;
-  ld.part_a = pa; ld.part_b = pb;
-  if (launch_lat(kLatDecoder, ld, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  if ((st = lat_sum(B, H, M, D, bp.S, 0, 1.f, pa, nullptr, 1, 0, nullptr, z32, gam, dz32, s)) != FLARE_OK ||
-      (st = pad(dz32, dzpad, BH * M, D, 1.f, s)) != FLARE_OK)
-    return st;
-  // dK (both parts) and dV
-  if (launch_tok(kTokFull, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  // encoder backward: its dQ; dQ = scale * (decoder + encoder parts), summed over the batch
-  LatParams le = lat_params(bp, ws, q, 0, k, B, H, N, M, D, lengths, sc, sh);
-  le.zrow = dz32; le.lrow = lenc; le.grow = gam; le.v = tp.v;
-  le.part_b = pc;
-  if (launch_lat(kLatEncoder, le, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  return lat_sum(B, H, M, D, bp.S, 1, sc, pb, pc, 1, 0, nullptr, nullptr, nullptr, dq, s);
-}
-
-// ---------------------------------------------------------------------------
-// FLARE++ (eq. 7-11) backward in seven phases.  Between two phases every
-// shard's exchange buffer is all-gathered in rank order; the next phase reads
-// the gathered buffers (R shards, `stride` floats apart) and merges them in
-// ascending (rank, split) order, so every rank holds bitwise the same Q(X),
-// Z, dZ, dQ(X), dQ0 and dW.  On one GPU the phases run back to back with the
-// exchanges in the workspace.  The workspace carries the shard's state
-// (projections, Q(X), Z, normalisers, gradient rows) from phase to phase.
-//   0: projections; synthesis recompute partials                 -> E0
-//   1: merge E0 -> Q(X), L~_m; encode recompute partials         -> E1
-//   2: merge E1 -> Z, L_m; decoder stats; decoder backward       -> E2 = [dZ | dQ_dec partials]
-//   3: dZ, gamma, scale * dQ_dec; dK, dV rows; encoder dQ        -> E3
-//   4: dQ(X), gamma~; dK~, dV~ rows; synthesis dQ0 partials      -> E4
-//   5: dQ0; dX (local rows); dW partials of the local rows       -> E5
-//   6: dW
-// ---------------------------------------------------------------------------
-constexpr int kPpPhases = 7;
-
-struct PpArgs {
-  const flare_bf16 *X, *Wk, *Wv, *Wk_syn, *Wv_syn, *Q0, *dY;
-  flare_bf16* dX;
-  float *dWk, *dWv, *dWk_syn, *dWv_syn, *dQ0;
-  int B, N, C, H, M, D;
-  const int32_t* lengths;
-  float sc;
-  Shard sh;
-};
-
-size_t pp_exchange_floats(const BwdPlan& bp, int phase, int B, int H, int M, int D, int C) {
-  switch (phase) {
-    case 0:
-    case 1: return part_floats(bp, B, H, M, D, true);
-    case 2: return 2 * part_floats(bp, B, H, M, D, false);
-    case 3:
-    case 4: return part_floats(bp, B, H, M, D, false);
-    case 5: return static_cast<size_t>(bp.dw_splits) * C * 4 * C;
-    default: return 0;
-  }
-}
-
-flare_status pp_phase(int phase, const BwdPlan& bp, uint8_t* ws, const PpArgs& a, const float* gathered,
-                      float* exch, cudaStream_t s) {
-  const int B = a.B, N = a.N, C = a.C, H = a.H, M = a.M, D = a.D;
-  const long BH = static_cast<long>(B) * H;
-  const float sc = a.sc, c = sc * kLog2e;
-  const int R = a.sh.R;
-  const bool shared = a.Wk_syn == a.Wk && a.Wv_syn == a.Wv;
-  uint16_t* kk = reinterpret_cast<uint16_t*>(ws + bp.fwd.off_kp);
-  uint16_t* vv = reinterpret_cast<uint16_t*>(ws + bp.fwd.off_vp);
-  uint16_t* kt = shared ? kk : reinterpret_cast<uint16_t*>(ws + bp.fwd.off_kt);
-  uint16_t* vt = shared ? vv : reinterpret_cast<uint16_t*>(ws + bp.fwd.off_vt);
-  float* q32 = reinterpret_cast<float*>(ws + bp.off_q32);
-  float* qx32 = reinterpret_cast<float*>(ws + bp.off_qx32);
-  float* lsyn = reinterpret_cast<float*>(ws + bp.off_lsyn);
-  float* z32 = reinterpret_cast<float*>(ws + bp.off_z32);
-  float* lenc = reinterpret_cast<float*>(ws + bp.off_lenc);
-  float* ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
-  float* dtok = reinterpret_cast<float*>(ws + bp.off_dtok);
-  float* dz32 = reinterpret_cast<float*>(ws + bp.off_dz32);
-  float* gam = reinterpret_cast<float*>(ws + bp.off_gam);
-  float* dqx32 = reinterpret_cast<float*>(ws + bp.off_dqx32);
-  float* dqxdec = reinterpret_cast<float*>(ws + bp.off_dqxdec);
-  float* gsyn = reinterpret_cast<float*>(ws + bp.off_gsyn);
-  float* qpad = reinterpret_cast<float*>(ws + bp.off_qpad);
-  float* zpad = reinterpret_cast<float*>(ws + bp.off_zpad);
-  float* dzpad = reinterpret_cast<float*>(ws + bp.off_dzpad);
-  float* q0pad = reinterpret_cast<float*>(ws + bp.off_q0pad);
-  float* dqxpad = reinterpret_cast<float*>(ws + bp.off_dqxpad);
-  float* g32 = reinterpret_cast<float*>(ws + bp.off_g32);
-  const size_t P = part_floats(bp, B, H, M, D, false);
-  const size_t stride = pp_exchange_floats(bp, phase - 1, B, H, M, D, C);  // of the gathered buffers
-  flare_status st = FLARE_OK;
-  switch (phase) {
-    case 0: {
-      if (cudaMemsetAsync(ws + bp.fwd.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-      // eq. 7 and 9: the projections, recomputed (tcgen05, as in the forward)
-      Projected pr;
-      if ((st = flarepp_project(bp.fwd, a.X, a.Wk, a.Wv, a.Wk_syn, a.Wv_syn, B, N, C, H, D, ws, s, nullptr, &pr)) !=
-          FLARE_OK)
-        return st;
-      const CvtParams cv{static_cast<long>(H) * M * D, reinterpret_cast<const uint16_t*>(a.Q0), q32};
-      if (launch_cvt(cv, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-      // eq. 8 recomputed: the synthesis partials of this shard
-      LatParams lf = lat_params(bp, ws, q32, 0, kt, B, H, N, M, D, a.lengths, sc, a.sh);
-      lf.v = vt;
-      lf.part_a = exch;
-      return launch_lat(kLatForward, lf, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
-    }
-    case 1: {
-      if ((st = lat_merge(gathered, R, stride, static_cast<int>(BH), M, D, bp.S, qx32, lsyn, s)) != FLARE_OK)
-        return st;
-      // eq. 10 recomputed: the encode partials of this shard
-      LatParams lf = lat_params(bp, ws, qx32, 1, kk, B, H, N, M, D, a.lengths, sc, a.sh);
-      lf.v = vv;
-      lf.part_a = exch;
-      return launch_lat(kLatForward, lf, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
-    }
-    case 2: {
-      if ((st = lat_merge(gathered, R, stride, static_cast<int>(BH), M, D, bp.S, z32, lenc, s)) != FLARE_OK ||
-          (st = pad(qx32, qpad, BH * M, D, c, s)) != FLARE_OK || (st = pad(z32, zpad, BH * M, D, 1.f, s)) != FLARE_OK)
-        return st;
-      // eq. 11: the decoder's per-token normalisers and delta_n
-      TokParams tp = tok_params(B, H, N, M, D, 1, a.lengths, sc, a.sh);
-      tp.qpad = qpad; tp.zpad = zpad;
-      tp.k = kk; tp.dy = reinterpret_cast<const uint16_t*>(a.dY);
-      tp.ltok = ltok; tp.dtok = dtok;
-      if (launch_tok(kTokStats, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-      // decoder backward, reductions over this shard's tokens: dZ and dQ(X) partials
-      LatParams ld = lat_params(bp, ws, qx32, 1, kk, B, H, N, M, D, a.lengths, sc, a.sh);
-      ld.zrow = z32; ld.dy = tp.dy; ld.ltok = ltok; ld.dtok = dtok;
-      ld.part_a = exch; ld.part_b = exch + P;
-      return launch_lat(kLatDecoder, ld, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
-    }
-    case 3: {
-      // dZ and gamma; the decoder's part of dQ(X)
-      if ((st = lat_sum(B, H, M, D, bp.S, 0, 1.f, gathered, nullptr, R, stride, nullptr, z32, gam, dz32, s)) !=
-              FLARE_OK ||
-          (st = lat_sum(B, H, M, D, bp.S, 0, sc, gathered + P, nullptr, R, stride, nullptr, nullptr, nullptr,
-                        dqxdec, s)) != FLARE_OK ||
-          (st = pad(dz32, dzpad, BH * M, D, 1.f, s)) != FLARE_OK)
-        return st;
-      // dK (both parts) and dV of this shard's tokens, into the gradient rows
-      TokParams tp = tok_params(B, H, N, M, D, 1, a.lengths, sc, a.sh);
-      tp.qpad = qpad; tp.zpad = zpad; tp.dzpad = dzpad; tp.lm = lenc; tp.gam = gam;
-      tp.k = kk; tp.v = vv; tp.dy = reinterpret_cast<const uint16_t*>(a.dY);
-      tp.ltok = ltok; tp.dtok = dtok;
-      tp.g32 = g32; tp.g_ld = 4 * C; tp.g_col_k = 0; tp.g_col_v = C;
-      if (launch_tok(kTokFull, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-      // encoder backward: its dQ(X) partials
-      LatParams le = lat_params(bp, ws, qx32, 1, kk, B, H, N, M, D, a.lengths, sc, a.sh);
-      le.zrow = dz32; le.lrow = lenc; le.grow = gam; le.v = vv;
-      le.part_b = exch;
-      return launch_lat(kLatEncoder, le, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
-    }
-    case 4: {
-      // dQ(X) = scale * (decoder + encoder parts); gamma of the synthesis
-      if ((st = lat_sum(B, H, M, D, bp.S, 0, sc, gathered, nullptr, R, stride, dqxdec, qx32, gsyn, dqx32, s)) !=
-              FLARE_OK ||
-          (st = pad(q32, q0pad, static_cast<long>(H) * M, D, c, s)) != FLARE_OK ||
-          (st = pad(dqx32, dqxpad, BH * M, D, 1.f, s)) != FLARE_OK)
-        return st;
-      // eq. 8 backward with dQ(X) as the upstream gradient: dK~, dV~ rows ...
-      TokParams tp = tok_params(B, H, N, M, D, 0, a.lengths, sc, a.sh);
-      tp.qpad = q0pad; tp.dzpad = dqxpad; tp.lm = lsyn; tp.gam = gsyn;
-      tp.k = kt; tp.v = vt;
-      tp.g32 = g32; tp.g_ld = 4 * C; tp.g_col_k = 2 * C; tp.g_col_v = 3 * C;
-      if (launch_tok(kTokEncoder, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-      // ... and the partials of dQ0
-      LatParams le = lat_params(bp, ws, q32, 0, kt, B, H, N, M, D, a.lengths, sc, a.sh);
-      le.zrow = dqx32; le.lrow = lsyn; le.grow = gsyn; le.v = vt;
-      le.part_b = exch;
-      return launch_lat(kLatEncoder, le, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
-    }
-    case 5: {
-      // dQ0, summed over the batch and the shards
-      if ((st = lat_sum(B, H, M, D, bp.S, 1, sc, gathered, nullptr, R, stride, nullptr, nullptr, nullptr, a.dQ0, s)) !=
-          FLARE_OK)
-        return st;
-      // projections backward on this shard's rows: dX = G [Wk | Wv | Wk~ | Wv~]^T, partials of X^T G
-      const long rows = static_cast<long>(B) * N;
-      DxParams dx{};
-      dx.R = static_cast<int>(rows); dx.C = C; dx.nw = 4;
-      dx.g = g32;
-      const flare_bf16* w4[4] = {a.Wk, a.Wv, a.Wk_syn, a.Wv_syn};
-      for (int i = 0; i < 4; ++i) dx.w[i] = reinterpret_cast<const uint16_t*>(w4[i]);
-      dx.dx = reinterpret_cast<uint16_t*>(a.dX);
-      if (launch_dx(dx, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-      const DwParams dw{static_cast<int>(rows), C, 4 * C, bp.dw_splits, reinterpret_cast<const uint16_t*>(a.X), g32,
-                        exch};
-      return launch_dw(dw, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
-    }
-    case 6: {
-      // dW: the partials of every shard's rows (rank-major, so the splits of all
-      // shards form one ascending sequence)
-      DwReduceParams dr{};
-      dr.C = C; dr.J = 4 * C; dr.n_splits = R * bp.dw_splits; dr.shared = shared ? 1 : 0;
-      dr.part = gathered;
-      dr.dw[0] = a.dWk; dr.dw[1] = a.dWv; dr.dw[2] = a.dWk_syn; dr.dw[3] = a.dWv_syn;
-      return launch_dw_reduce(dr, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
-    }
-    default:
-      return FLARE_ERR_SHAPE;
-  }
-}
-
-flare_status check_bwd_sizes(int B, int H, int N, int M, int D) {
-  flare_status st = check_common(B, H, N, M, D);
-  if (st != FLARE_OK) return st;
-  return static_cast<long>(B) * H > 65535 ? FLARE_ERR_UNSUPPORTED : FLARE_OK;
-}
-
-// Checks shared by the FLARE++ backward entry points.
-flare_status check_pp_bwd(const PpArgs& a, const void* workspace) {
-  flare_status st = check_flarepp(a.X, a.Wk, a.Wv, a.Wk_syn, a.Wv_syn, a.Q0, a.dY, a.B, a.N, a.C, a.H, a.M, a.D,
-                                  a.lengths, workspace, nullptr, nullptr);
-  if (st != FLARE_OK) return st;
-  const bool shared = a.Wk_syn == a.Wk && a.Wv_syn == a.Wv;
-  if (!a.dX || !a.dWk || !a.dWv || !a.dQ0 || (!shared && (!a.dWk_syn || !a.dWv_syn))) return FLARE_ERR_NULL;
-  if ((st = check_bwd_sizes(a.B, a.H, a.N, a.M, a.D)) != FLARE_OK) return st;
-  if (static_cast<long>(a.B) * a.N > 65535L * kBwdDwRows) return FLARE_ERR_UNSUPPORTED;
-  if (!aligned16(a.dX) || !aligned16(a.dWk) || !aligned16(a.dWv) || !aligned16(a.dWk_syn) || !aligned16(a.dWv_syn) ||
-      !aligned16(a.dQ0))
-    return FLARE_ERR_ALIGN;
-  return FLARE_OK;
-}
-
-}  // namespace
-}  // namespace flare
-
-extern "C" {
-
-flare_status flare_mixer_bwd(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, const flare_bf16* dY,
-                             flare_bf16* dK, flare_bf16* dV, float* dQ, int B, int H, int N, int M, int D,
-                             const int32_t* lengths, float scale, void* workspace, size_t workspace_bytes,
-                             void* stream) {
-  if (!K || !V || !Q || !dY || !dK || !dV || !dQ || !workspace) return FLARE_ERR_NULL;
-  flare_status st = check_bwd_sizes(B, H, N, M, D);
-  if (st != FLARE_OK) return st;
-  if (!aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(dY) || !aligned16(dK) || !aligned16(dV) ||
-      !aligned16(dQ) || !aligned16(lengths) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return FLARE_ERR_ALIGN;
-  const BwdPlan bp = make_bwd_plan(false, B, H, N, M, D, 0);
-  if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  if (cudaMemsetAsync(ws + bp.fwd.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  float* q32 = reinterpret_cast<float*>(ws + bp.off_q32);
-  const CvtParams cv{static_cast<long>(H) * M * D, reinterpret_cast<const uint16_t*>(Q), q32};
-  if (launch_cvt(cv, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  return flare_bwd_run(bp, ws, q32, K, V, dY, reinterpret_cast<uint16_t*>(dK), reinterpret_cast<uint16_t*>(dV), dQ, B,
-                       H, N, M, D, lengths, resolve_scale(scale, D), s);
-}
-
-flare_status flarepp_mixer_bwd(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
-                               const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0,
-                               const flare_bf16* dY, flare_bf16* dX, float* dWk, float* dWv, float* dWk_syn,
-                               float* dWv_syn, float* dQ0, int B, int N, int C, int H, int M, int D,
-                               const int32_t* lengths, float scale, void* workspace, size_t workspace_bytes,
-                               void* stream) {
-  const PpArgs a{X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, dX, dWk, dWv, dWk_syn, dWv_syn, dQ0,
-                 B, N, C, H, M, D, lengths, resolve_scale(scale, D), Shard{0, N, 1}};
-  flare_status st = check_pp_bwd(a, workspace);
-  if (st != FLARE_OK) return st;
-  const BwdPlan bp = make_bwd_plan(true, B, H, N, M, D, C);
-  if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  // one shard: the exchanges stay in the workspace (stream order makes every
-  // reuse safe: a buffer is read by the next phase's first launches before
-  // that phase writes its own exchange)
-  float* ex[kPpPhases - 1] = {reinterpret_cast<float*>(ws + bp.off_fpart), reinterpret_cast<float*>(ws + bp.off_fpart),
-                              reinterpret_cast<float*>(ws + bp.off_pa),    reinterpret_cast<float*>(ws + bp.off_pc),
-                              reinterpret_cast<float*>(ws + bp.off_pc),    reinterpret_cast<float*>(ws + bp.off_dwpart)};
-  for (int ph = 0; ph < kPpPhases; ++ph) {
-    st = pp_phase(ph, bp, ws, a, ph > 0 ? ex[ph - 1] : nullptr, ph < kPpPhases - 1 ? ex[ph] : nullptr, s);
-    if (st != FLARE_OK) return st;
-  }
-  return FLARE_OK;
-}
-
-size_t flarepp_cp_bwd_exchange_bytes(int phase, int B, int N, int C, int H, int M, int D) {
-  if (phase < 0 || phase >= kPpPhases - 1) return 0;
-  if (check_bwd_sizes(B, H, N, M, D) != FLARE_OK || C != H * D || C % 64 != 0 || C > 256) return 0;
-  return pp_exchange_floats(make_bwd_plan(true, B, H, N, M, D, C), phase, B, H, M, D, C) * sizeof(float);
-}
-
-flare_status flarepp_cp_bwd_phase(int phase, const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
-                                  const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0,
-                                  const flare_bf16* dY, const float* gathered, float* exchange, flare_bf16* dX,
-                                  float* dWk, float* dWv, float* dWk_syn, float* dWv_syn, float* dQ0, int B, int N,
-                                  int C, int H, int M, int D, const int32_t* lengths, int rank, int world,
-                                  float scale, void* workspace, size_t workspace_bytes, void* stream) {
-  if (phase < 0 || phase >= kPpPhases) return FLARE_ERR_SHAPE;
-  if (world < 1 || rank < 0 || rank >= world) return FLARE_ERR_SHAPE;
-  if (static_cast<long>(N) * world >= (1L << 31)) return FLARE_ERR_UNSUPPORTED;
-  if ((phase > 0 && !gathered) || (phase < kPpPhases - 1 && !exchange)) return FLARE_ERR_NULL;
-  if (!aligned16(gathered) || !aligned16(exchange)) return FLARE_ERR_ALIGN;
-  const PpArgs a{X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, dX, dWk, dWv, dWk_syn, dWv_syn, dQ0,
-                 B, N, C, H, M, D, lengths, resolve_scale(scale, D), Shard{rank * N, world * N, world}};
-  flare_status st = check_pp_bwd(a, workspace);
-  if (st != FLARE_OK) return st;
-  const BwdPlan bp = make_bwd_plan(true, B, H, N, M, D, C);
-  if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
-  return pp_phase(phase, bp, static_cast<uint8_t*>(workspace), a, gathered, exchange,
-                  static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
