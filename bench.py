@@ -7,14 +7,15 @@ the four per-head projections, the query-synthesis encode, the encode with
 the synthesised queries, both log-sum-exp merges and the decode.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --backward [--workload NAME] ...   # the backward: its own JSON line
 
 Prints one JSON line (rank 0).  ``value`` is whole-job token*heads/s with the
 inputs resident in HBM, timed with CUDA events on the launching stream over
 exactly K steps (max over ranks).  ``e2e`` is the same metric with every
 step's host->device copy of its inputs (pinned memory) and device->host copy
 of Y inside the timed region; the copies run on their own streams into double
-buffers, so those of neighbouring steps overlap the current step's compute.  ``roofline`` reports the dominant kernel
-against the exp-unit (MUFU) peak, ``cpu_baseline`` the fp64 oracle on a
+buffers, so those of neighbouring steps overlap the current step's compute.
+``roofline`` reports the dominant kernel against the exp-unit (MUFU) peak, ``cpu_baseline`` the fp64 oracle on a
 bounded sample of the same workload on this host's cores.  ``--impl
 reference`` times the oracle itself as the reference arm.
 
@@ -22,6 +23,11 @@ With ``--gpus N`` (launched through torch.distributed.run) every rank runs an
 independent copy of the workload on its own synthetic input (weak scaling; the
 heads and samples of the mixer are independent, so there is no data-path
 collective).
+
+``--backward`` times one ``flarepp_mixer_bwd`` call (``flare_mixer_bwd`` for a
+FLARE workload) per step with a seeded upstream gradient dY, against the
+backward's own roofline (three exponentials per score, the tf32 tensor term,
+HBM); ``e2e`` then copies the inputs and dY in and every gradient out.
 """
 from __future__ import annotations
 
