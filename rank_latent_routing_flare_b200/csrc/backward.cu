@@ -107,9 +107,11 @@ __device__ __forceinline__ void stage_bf16(float* dst, const uint16_t* src, int 
 }
 
 // ---------------------------------------------------------------------------
-// Latent-parallel pass: a warp owns 16 latent rows (a CTA 16 per warp) of one
-// head and one token split, and walks the split's valid tokens in tiles of 64
-// that the CTA stages in shared memory.  Per tile and 8-token column block:
+// Latent-parallel pass: a warp owns MT tiles of 16 latent rows of one head and
+// one token split (MT = 2 shares every B fragment between two MMAs; the
+// forward mode keeps MT = 1 for its online softmax), and walks the split's
+// valid tokens in tiles of 64 that the CTA stages in shared memory (double
+// buffered).  Per tile and 8-token column block:
 // scores S = (c Q) K^T on the tensor cores, then
 //   forward:  online softmax over tokens, O += 2^(S - max) V
 //   decoder:  W = 2^(S - L_n), dS = W (Z dY^T - delta_n), dZ += W dY, dQ += dS K
@@ -477,8 +479,9 @@ __global__ void __launch_bounds__(256) lat_sum_kernel(const LatSumParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// Token-parallel pass: a warp owns 16 token rows (a CTA 128) of one head and
-// walks all latents in chunks of 64 that the CTA stages in shared memory.
+// Token-parallel pass: a warp owns MT tiles of 16 token rows (a CTA 128 tokens)
+// of one head and walks all latents in chunks of 64 (32 for D = 32), copied
+// with cp.async from padded tf32 images into two shared-memory buffers.
 // Per 8-latent column block, on the tensor cores: S = K (c Q)^T, and
 //   stats:    online softmax over latents, Y += 2^(S - max) Z; at the end
 //             L_n = log2 sum 2^S and delta_n = <dY_n, Y_n>

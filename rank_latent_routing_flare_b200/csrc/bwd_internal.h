@@ -14,7 +14,7 @@ __host__ __device__ constexpr int tok_chunk(int D) { return D == 16 ? 64 : 32; }
 constexpr int kBwdDwRows = 2048;    // token rows per split of the weight-gradient GEMM
 
 // Modes of the latent-parallel kernel (one CTA = a block of latents of one
-// head and one token split; a warp = 16 latent rows).
+// head and one token split; a warp = one or two tiles of 16 latent rows).
 enum LatMode : int {
   kLatForward = 0,   // encoder recompute: per split (max, sum, sum w v) in log2 units
   kLatDecoder = 1,   // decoder backward, reductions over tokens: dZ and dQ
@@ -66,7 +66,7 @@ struct LatSumParams {
 };
 
 // Modes of the token-parallel kernel (one CTA = kBwdTokBlock tokens of one
-// head; a warp = 16 token rows).
+// head; a warp = one or two tiles of 16 token rows).
 enum TokMode : int {
   kTokStats = 0,     // decoder recompute: per-token log2-normaliser and delta = <dY, Y>
   kTokFull = 1,      // dK (decoder + encoder parts) and dV
