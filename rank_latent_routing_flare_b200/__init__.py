@@ -27,4 +27,5 @@ from ._binding import (  # noqa: F401
     library_path,
     load_library,
 )
-from . import cp  # noqa: F401,E402  (context-parallel forward over torch.distributed)
+from . import cp  # noqa: F401,E402  (context-parallel forward and backward over torch.distributed)
+from .autograd import flare_mixer, flarepp_mixer  # noqa: F401,E402  (torch.autograd wrappers)

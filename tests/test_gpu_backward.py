@@ -221,3 +221,24 @@ def test_backward_full_size(name):
     keys = ("dK", "dV", "dQ") if w.variant == "flare" else ("dX", "dWk", "dWv", "dWk_syn", "dWv_syn", "dQ0")
     for k in keys:
         check(got[k], ref[k], f"{name} full {k}")
+
+
+def test_autograd_wrapper_matches_the_direct_calls():
+    """fl.flarepp_mixer (torch.autograd) gives the bits of flarepp_mixer_fwd and
+    flarepp_mixer_bwd called directly (weight and seed gradients rounded to
+    the parameters' bf16)."""
+    w = make_workload("flarepp_n1k", N=512)
+    X = dev_bf16(w.X).requires_grad_()
+    Ws = [dev_bf16(a).requires_grad_() for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn)]
+    Q0 = dev_bf16(w.Q0).requires_grad_()
+    dY = dev_bf16(make_upstream_grad(w))
+    Y = fl.flarepp_mixer(X, *Ws, Q0)
+    (Y.float() * dY.float()).sum().backward()
+    Y_direct = fl.flarepp_mixer_fwd(X.detach(), *[a.detach() for a in Ws], Q0.detach())
+    g = fl.flarepp_mixer_bwd(X.detach(), *[a.detach() for a in Ws], Q0.detach(), dY)
+    torch.cuda.synchronize()
+    assert torch.equal(Y.detach().view(torch.int16), Y_direct.view(torch.int16))
+    assert torch.equal(X.grad.view(torch.int16), g["dX"].view(torch.int16))
+    for W, k in zip(Ws, ("dWk", "dWv", "dWk_syn", "dWv_syn")):
+        assert torch.equal(W.grad.view(torch.int16), g[k].to(torch.bfloat16).view(torch.int16)), k
+    assert torch.equal(Q0.grad.view(torch.int16), g["dQ0"].to(torch.bfloat16).view(torch.int16))
