@@ -1,4 +1,5 @@
-"""Seeded synthetic inputs for the FLARE / FLARE++ mixer forward.
+"""Seeded synthetic inputs for the FLARE / FLARE++ mixer (forward inputs, and
+the upstream gradient dY of the backward).
 
 This module only draws random numbers and rounds them to bfloat16.  It holds
 none of the mixer's arithmetic, so the fp64 oracle (``oracle/``) and the CUDA
