@@ -50,8 +50,16 @@ from workloads import make_workload  # noqa: E402
 METRIC = "mixer fwd token·heads/s at N=1M (1×B200) and % of roofline (HBM/MMA/MUFU)"
 UNIT = "token·heads/s"
 WORKLOAD = "flarepp_n1m_mesh3d"
-MUFU_PER_CLK_PER_SM = 16          # ex2 results per clock per SM (special-function unit)
+MUFU_PER_CLK_PER_SM = 16          # nominal ex2 results per clock per SM (used only if the probe fails)
+FMA_PER_CLK_PER_SM = 128          # nominal fp32 fma per clock per SM (ditto)
 NUM_SM = 148
+# Issue-slot cost of the softmax's own arithmetic per score (the kernels'
+# exponential step): one FFMA for the scale-and-shift and half a bf16x2 pack,
+# plus the exponential itself -- one MUFU instruction, or the 9 instructions
+# of the FMA-pipe polynomial (clamp, two adds and a subtract for the range
+# reduction, three FFMAs, a shift and an integer add for the exponent).
+SOFTMAX_BASE_OPS = 1.5
+POLY_EXP_OPS = 9.0
 STAGES_PP = ["project", "synth_encode", "synth_merge", "encode", "merge", "decode"]
 KERNEL_SOURCES = {"project": "project.cu", "synth_encode": "encode.cu", "encode": "encode.cu",
                   "synth_merge": "merge.cu", "merge": "merge.cu", "decode": "decode.cu"}
@@ -162,6 +170,37 @@ def stage_work(w):
         "merge": {"bytes": 0, "flops": 0, "exps": 0},
         "decode": {"bytes": dec_bytes, "flops": enc_flops, "exps": enc_exps},
     }
+
+
+def pipe_rates(fl, dev) -> dict:
+    """ex2 (MUFU) and fp32 fma (FMA pipe) results per clock per SM, measured
+    on this device by the library's probe kernels; nominal values if the
+    probe fails (then labelled so)."""
+    try:
+        r = fl.flare_probe_pipe_rates(dev)
+        if r["ex2"] > 0 and r["ffma"] > 0:
+            return {"ex2": r["ex2"], "ffma": r["ffma"], "source": "measured (flare_probe_pipe_rates)"}
+    except Exception as e:  # noqa: BLE001
+        log(f"pipe probe failed: {e}")
+    return {"ex2": float(MUFU_PER_CLK_PER_SM), "ffma": float(FMA_PER_CLK_PER_SM), "source": "nominal"}
+
+
+def exp_unit_bounds(rates: dict) -> dict:
+    """Clocks per score per SM of the softmax's exponential step under two
+    bounds:
+
+    - mufu_only: every exponential on the special-function unit (1 / ex2 rate);
+    - combined: a fraction f of the exponentials on the FMA-pipe polynomial,
+      chosen to balance the MUFU against the issue slots (one instruction per
+      clock per sub-partition, measured as the fma rate), which every
+      instruction of the step takes: t = max((1 - f) / ex2, (base + (1 - f)
+      + poly * f) / issue).  The best any MUFU/polynomial split of this
+      arithmetic can reach."""
+    ex2, issue = rates["ex2"], rates["ffma"]
+    r = issue / ex2
+    f = min(1.0, max(0.0, (r - SOFTMAX_BASE_OPS - 1.0) / (r + POLY_EXP_OPS - 1.0)))
+    t_comb = max((1.0 - f) / ex2, (SOFTMAX_BASE_OPS + (1.0 - f) + POLY_EXP_OPS * f) / issue)
+    return {"mufu_only": 1.0 / ex2, "combined": t_comb, "poly_fraction": f}
 
 
 def kernel_traffic(kernel_file: str, workload: str):
@@ -373,7 +412,8 @@ def run_backward(args, rank, world, local_rank):
     value = whole_job_rate(world, th_per_rank, ms)
 
     peaks = load_peaks()
-    mufu_peak = MUFU_PER_CLK_PER_SM * NUM_SM * peaks["sm_max_mhz"] * 1e6
+    rates = pipe_rates(fl, dev)
+    mufu_peak = rates["ex2"] * NUM_SM * peaks["sm_max_mhz"] * 1e6
     tf32_peak = peaks["bf16_tflops"] * 1e12 * TF32_PER_BF16
     wk = backward_work(w)
     terms = {"hbm": wk["bytes"] / (peaks["hbm_gbs"] * 1e9), "mma_tf32": wk["flops"] / tf32_peak,
@@ -429,7 +469,7 @@ def run_backward(args, rank, world, local_rank):
                               "inputs larger than L2 (X 256 MiB, dY 256 MiB, fp32 gradient rows 2 GiB)")},
             "step_roofline": {"t_roof_ms": round(t_roof * 1e3, 4), "frac": round(t_roof / (ms * 1e-3), 4),
                               "bound": bound, "terms_ms": {k: round(v * 1e3, 4) for k, v in terms.items()},
-                              "peak_basis": f"MUFU {MUFU_PER_CLK_PER_SM} ex2/clk/SM x {NUM_SM} x "
+                              "peak_basis": f"MUFU {rates['ex2']:.2f} ex2/clk/SM ({rates['source']}) x {NUM_SM} x "
                                             f"{peaks['sm_max_mhz']:.0f} MHz; tf32 = {TF32_PER_BF16} x measured "
                                             f"bf16 {peaks['bf16_tflops']} TFLOP/s; HBM {peaks['hbm_gbs']} GB/s "
                                             f"({peaks['source']})"},
@@ -602,7 +642,11 @@ def main():
     work = stage_work(w)
     peaks = load_peaks()
     clk = clocks.summary()
-    mufu_peak_max = MUFU_PER_CLK_PER_SM * NUM_SM * peaks["sm_max_mhz"] * 1e6
+    rates = pipe_rates(fl, dev)
+    bounds = exp_unit_bounds(rates)
+    sm_hz = NUM_SM * peaks["sm_max_mhz"] * 1e6
+    exp_peak = {k: sm_hz / bounds[k] for k in ("mufu_only", "combined")}   # exps/s at the maximum clock
+    mufu_peak_max = exp_peak["mufu_only"]
     stages = {}
     for s in STAGES_PP:
         t = stage_ms[s] * 1e-3
@@ -621,14 +665,20 @@ def main():
         exps = work["encode" if dom == "encode" else "decode"]["exps"]
         achieved = exps / (per_launch_ms * 1e-3) / 1e9
         roof = {"kernel": f"{dom}_kernel", "bound": "alu", "achieved": round(achieved, 1),
-                "peak": round(mufu_peak_max / 1e9, 1), "unit": "Gexp/s",
-                "frac": round(achieved / (mufu_peak_max / 1e9), 4),
-                "peak_basis": f"{MUFU_PER_CLK_PER_SM} ex2/clk/SM x {NUM_SM} SMs x {peaks['sm_max_mhz']:.0f} MHz",
+                "peak": round(exp_peak["combined"] / 1e9, 1), "unit": "Gexp/s",
+                "frac": round(achieved / (exp_peak["combined"] / 1e9), 4),
+                "frac_combined": round(achieved / (exp_peak["combined"] / 1e9), 4),
+                "frac_mufu_only": round(achieved / (exp_peak["mufu_only"] / 1e9), 4),
+                "peak_mufu_only": round(exp_peak["mufu_only"] / 1e9, 1),
+                "peak_basis": (f"ex2 {rates['ex2']:.2f}/clk/SM and fma (issue) {rates['ffma']:.2f}/clk/SM "
+                               f"({rates['source']}) x {NUM_SM} SMs x {peaks['sm_max_mhz']:.0f} MHz; combined: "
+                               f"{bounds['poly_fraction']:.3f} of the exps on a {POLY_EXP_OPS:g}-instruction "
+                               f"polynomial, {SOFTMAX_BASE_OPS:g} more instructions per score"),
                 "per_launch_ms": round(per_launch_ms, 4),
                 "traffic": kernel_traffic(f"{dom}.cu", w.name)}
         if clk.get("sm_mhz"):
             roof["frac_at_observed_clock"] = round(
-                achieved / (MUFU_PER_CLK_PER_SM * NUM_SM * clk["sm_mhz"] * 1e-3), 4)
+                achieved / (exp_peak["combined"] / 1e9 * clk["sm_mhz"] / peaks["sm_max_mhz"]), 4)
     elif dom == "project":
         per = kern_ms[dom]
         achieved = work["project"]["bytes"] / (per * 1e-3) / 1e9
@@ -638,17 +688,22 @@ def main():
     else:
         roof = {"kernel": "merge_kernel", "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": None, "traffic": None}
-    roof["peak_source"] = peaks["source"]
+    roof["peak_source"] = rates["source"] if roof["bound"] == "alu" else peaks["source"]
     # whole-step roofline: max(bytes / HBM peak, MMA flops / tensor peak, exps / MUFU peak)
     tot_bytes = 3 * w.B * w.N * w.C * 2 + w.B * w.H * w.N * w.D * 2
     tot_exps = sum(work[s]["exps"] for s in STAGES_PP)
     tot_flops = sum(work[s]["flops"] for s in STAGES_PP)
-    t_roof = max(tot_bytes / (peaks["hbm_gbs"] * 1e9), tot_flops / (peaks["bf16_tflops"] * 1e12),
-                 tot_exps / mufu_peak_max)
+    t_hbm, t_mma = tot_bytes / (peaks["hbm_gbs"] * 1e9), tot_flops / (peaks["bf16_tflops"] * 1e12)
+    t_roof = max(t_hbm, t_mma, tot_exps / exp_peak["combined"])
+    t_roof_mufu = max(t_hbm, t_mma, tot_exps / exp_peak["mufu_only"])
     step_roofline = {"t_roof_ms": round(t_roof * 1e3, 4), "frac": round(t_roof / (ms * 1e-3), 4),
-                     "terms_ms": {"hbm": round(tot_bytes / (peaks["hbm_gbs"] * 1e9) * 1e3, 4),
-                                  "mma": round(tot_flops / (peaks["bf16_tflops"] * 1e12) * 1e3, 4),
-                                  "mufu": round(tot_exps / mufu_peak_max * 1e3, 4)}}
+                     "frac_combined": round(t_roof / (ms * 1e-3), 4),
+                     "frac_mufu_only": round(t_roof_mufu / (ms * 1e-3), 4),
+                     "terms_ms": {"hbm": round(t_hbm * 1e3, 4), "mma": round(t_mma * 1e3, 4),
+                                  "exp_combined": round(tot_exps / exp_peak["combined"] * 1e3, 4),
+                                  "exp_mufu_only": round(tot_exps / exp_peak["mufu_only"] * 1e3, 4)},
+                     "pipe_rates": {"ex2_per_clk_sm": round(rates["ex2"], 3),
+                                    "ffma_per_clk_sm": round(rates["ffma"], 3), "source": rates["source"]}}
 
     # ---------------- end to end through the public API ----------------
     # Every step copies its inputs (X, the four weights, Q0) in from pinned host

@@ -174,6 +174,26 @@ FLARE_API flare_status flarepp_mixer_fwd_profiled(const flare_bf16* X, const fla
                                                   float* Qx_out, float* Z_out, void* const* stage_events);
 
 /*
+ * Inspection variants: identical work and outputs, plus Y_f32_out
+ * [B][H][N][D] float (written, required): the fp32 values that the decoder
+ * rounds to the bf16 Y (zeros for padding tokens).  They let a caller check
+ * the token-dependent part of Y (the routing of eq. 6 / eq. 11) more finely
+ * than bf16 resolves it.  Other arguments as in flare_mixer_fwd /
+ * flarepp_mixer_fwd.
+ */
+FLARE_API flare_status flare_mixer_fwd_inspect(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q,
+                                               flare_bf16* Y, int B, int H, int N, int M, int D,
+                                               const int32_t* lengths, float scale, void* workspace,
+                                               size_t workspace_bytes, void* stream, float* Z_out,
+                                               float* Y_f32_out);
+FLARE_API flare_status flarepp_mixer_fwd_inspect(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                                                 const flare_bf16* Wk_syn, const flare_bf16* Wv_syn,
+                                                 const flare_bf16* Q0, flare_bf16* Y, int B, int N, int C, int H,
+                                                 int M, int D, const int32_t* lengths, float scale,
+                                                 void* workspace, size_t workspace_bytes, void* stream,
+                                                 float* Qx_out, float* Z_out, float* Y_f32_out);
+
+/*
  * Backward (gradients of a scalar loss, given dY = dLoss/dY).
  *
  * The pages name the paper's backward equations (eq. 13-40) without
@@ -340,13 +360,36 @@ FLARE_API flare_status flare_cp_end(const float* partials_all, const flare_bf16*
  *     the last call's contents (the words that must start at zero are
  *     cleared by each call).  Calls whose execution overlaps on the GPU race
  *     on the scratch and give wrong results: serialise them.
- *   - The device error word lives in the shared array, so
- *     flare_last_device_status() cannot be used with this call.
+ *   - The device error word (an expired bounded wait, a length outside
+ *     [1, N]) lives at the start of the shared array and is cleared by each
+ *     call; read it with flare_static_last_device_status().
  */
 #define FLARE_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
 FLARE_API flare_status flare_mixer_fwd_static(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q,
                                               flare_bf16* Y, int B, int H, int N, int M, int D,
                                               const int32_t* lengths, float scale, void* stream, float* Z_out);
+
+/*
+ * flare_last_device_status() for flare_mixer_fwd_static: synchronises
+ * `stream` and reads the device error word of the static scratch (the last
+ * static call's, whichever stream it ran on).  Same return values.
+ */
+FLARE_API flare_status flare_static_last_device_status(void* stream);
+
+/*
+ * Pipe-throughput probes (no counterpart in the pages: they measure the
+ * denominators of the exp-unit roofline on the device at hand).  Runs two
+ * short kernels on `stream` -- independent chains of ex2.approx.f32 on the
+ * special-function unit and of fp32 fma on the FMA pipe, one wave of CTAs
+ * on every SM -- synchronises the stream and writes the results per SM
+ * clock (from each SM's own clock64 counter, so independent of the clock
+ * frequency) to *ex2_per_clk_sm and *ffma_per_clk_sm.  `scratch`: caller-
+ * owned DEVICE memory of flare_probe_scratch_bytes() bytes, 256-byte
+ * aligned.  Not for use during stream capture.
+ */
+FLARE_API size_t flare_probe_scratch_bytes(void);
+FLARE_API flare_status flare_probe_pipe_rates(void* scratch, size_t scratch_bytes, void* stream,
+                                              double* ex2_per_clk_sm, double* ffma_per_clk_sm);
 
 /*
  * Self-test of the bounded-wait error path: enqueues one small kernel that

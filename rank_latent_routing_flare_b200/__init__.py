@@ -18,7 +18,9 @@ from ._binding import (  # noqa: F401
     flare_mixer_bwd,
     flare_mixer_fwd,
     flare_mixer_fwd_static,
+    flare_probe_pipe_rates,
     flare_selftest_wait_timeout,
+    flare_static_last_device_status,
     flare_status_string,
     flare_workspace_bytes,
     flarepp_mixer_bwd,

@@ -63,6 +63,17 @@ def load_library(build_if_missing: bool = True):
         lib.flare_mixer_fwd_profiled.argtypes = lib.flare_mixer_fwd.argtypes + [vp]
         lib.flare_mixer_fwd_profiled.restype = i
         lib.flarepp_mixer_fwd_profiled.argtypes = lib.flarepp_mixer_fwd.argtypes + [vp]
+        lib.flare_mixer_fwd_inspect.argtypes = lib.flare_mixer_fwd.argtypes + [vp]
+        lib.flare_mixer_fwd_inspect.restype = i
+        lib.flarepp_mixer_fwd_inspect.argtypes = lib.flarepp_mixer_fwd.argtypes + [vp]
+        lib.flarepp_mixer_fwd_inspect.restype = i
+        lib.flare_probe_scratch_bytes.argtypes = []
+        lib.flare_probe_scratch_bytes.restype = sz
+        lib.flare_probe_pipe_rates.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_double),
+                                               ctypes.POINTER(ctypes.c_double)]
+        lib.flare_probe_pipe_rates.restype = i
+        lib.flare_static_last_device_status.argtypes = [vp]
+        lib.flare_static_last_device_status.restype = i
         lib.flare_cp_partials_bytes.restype = sz
         lib.flare_cp_partials_bytes.argtypes = [i, i, i, i, i]
         for name, args in (
@@ -149,6 +160,21 @@ def _workspace(workspace, nbytes, device):
     return workspace
 
 
+def _device_check(device_check, workspace_given: bool, workspace, stream, where: str) -> None:
+    """Read the device error word (an expired bounded wait, a length outside
+    [1, N], an underflowed context-parallel merge) after the call's work and
+    raise FlareError if it is set.  ``device_check`` None means: check when the
+    workspace was allocated here, since the caller then has no workspace to
+    query.  Checking synchronises the stream."""
+    if device_check is None:
+        device_check = not workspace_given
+    if not device_check:
+        return
+    st = load_library().flare_last_device_status(_ptr(workspace), _stream_ptr(stream, workspace.device))
+    if st != 0:
+        raise FlareError(st, where + " (device status)")
+
+
 def _event_array(events):
     """cudaEvent_t handles of torch.cuda.Event objects (each recorded once so
     that its handle exists) as a ctypes void* array."""
@@ -163,8 +189,11 @@ def _event_array(events):
 
 
 def flare_mixer_fwd(K, V, Q, lengths=None, scale: float = 0.0, Y=None, workspace=None, stream=None,
-                    Z_out=None, check: bool = True, stage_events=None):
-    """FLARE forward (eq. 5-6).  K, V: [B,H,N,D] bf16; Q: [H,M,D] bf16 -> Y [B,H,N,D] bf16."""
+                    Z_out=None, check: bool = True, stage_events=None, Y_f32_out=None, device_check=None):
+    """FLARE forward (eq. 5-6).  K, V: [B,H,N,D] bf16; Q: [H,M,D] bf16 -> Y [B,H,N,D] bf16.
+    ``Y_f32_out`` ([B,H,N,D] float32) selects flare_mixer_fwd_inspect: it also
+    receives the fp32 values Y is rounded from.  ``device_check``: see
+    ``_device_check`` (default: only when no workspace is passed)."""
     torch = _torch()
     B, H, N, D = K.shape
     M = Q.shape[1]
@@ -174,27 +203,34 @@ def flare_mixer_fwd(K, V, Q, lengths=None, scale: float = 0.0, Y=None, workspace
         _check_dev("Q", Q, torch.bfloat16, (H, M, D))
         _check_dev("lengths", lengths, torch.int32, (B,))
         _check_dev("Z_out", Z_out, torch.float32, (B, H, M, D))
+        _check_dev("Y_f32_out", Y_f32_out, torch.float32, (B, H, N, D))
     if Y is None:
         Y = torch.empty_like(K)
     nbytes = flare_workspace_bytes(FLARE_VARIANT_FLARE, B, H, N, M, D)
+    given = workspace is not None
     workspace = _workspace(workspace, nbytes, K.device)
     args = (_ptr(K), _ptr(V), _ptr(Q), _ptr(Y), B, H, N, M, D, _ptr(lengths), float(scale), _ptr(workspace),
             workspace.numel(), _stream_ptr(stream, K.device), _ptr(Z_out))
-    if stage_events is None:
+    if Y_f32_out is not None:
+        assert stage_events is None, "stage events and Y_f32_out are not combined"
+        st = load_library().flare_mixer_fwd_inspect(*args, _ptr(Y_f32_out))
+    elif stage_events is None:
         st = load_library().flare_mixer_fwd(*args)
     else:
         assert len(stage_events) == 5
         st = load_library().flare_mixer_fwd_profiled(*args, _event_array(stage_events))
     if st != 0:
         raise FlareError(st, "flare_mixer_fwd")
+    _device_check(device_check, given, workspace, stream, "flare_mixer_fwd")
     return Y
 
 
 def flarepp_mixer_fwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, lengths=None, scale: float = 0.0, Y=None,
                       workspace=None, stream=None, Qx_out=None, Z_out=None, check: bool = True,
-                      stage_events=None):
+                      stage_events=None, Y_f32_out=None, device_check=None):
     """FLARE++ forward (eq. 7-11).  X: [B,N,C] bf16; W*: [C,C] bf16; Q0: [H,M,D] bf16
-    -> Y [B,H,N,D] bf16."""
+    -> Y [B,H,N,D] bf16.  ``Y_f32_out`` ([B,H,N,D] float32) selects
+    flarepp_mixer_fwd_inspect: it also receives the fp32 values Y is rounded from."""
     torch = _torch()
     B, N, C = X.shape
     H, M, D = Q0.shape
@@ -206,25 +242,31 @@ def flarepp_mixer_fwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, lengths=None, scale: float 
         _check_dev("lengths", lengths, torch.int32, (B,))
         _check_dev("Qx_out", Qx_out, torch.float32, (B, H, M, D))
         _check_dev("Z_out", Z_out, torch.float32, (B, H, M, D))
+        _check_dev("Y_f32_out", Y_f32_out, torch.float32, (B, H, N, D))
     if Y is None:
         Y = torch.empty((B, H, N, D), dtype=torch.bfloat16, device=X.device)
     nbytes = flare_workspace_bytes(FLARE_VARIANT_FLAREPP, B, H, N, M, D, C)
+    given = workspace is not None
     workspace = _workspace(workspace, nbytes, X.device)
     args = (_ptr(X), _ptr(Wk), _ptr(Wv), _ptr(Wk_syn), _ptr(Wv_syn), _ptr(Q0), _ptr(Y), B, N, C, H, M, D,
             _ptr(lengths), float(scale), _ptr(workspace), workspace.numel(), _stream_ptr(stream, X.device),
             _ptr(Qx_out), _ptr(Z_out))
-    if stage_events is None:
+    if Y_f32_out is not None:
+        assert stage_events is None, "stage events and Y_f32_out are not combined"
+        st = load_library().flarepp_mixer_fwd_inspect(*args, _ptr(Y_f32_out))
+    elif stage_events is None:
         st = load_library().flarepp_mixer_fwd(*args)
     else:
         assert len(stage_events) == 7
         st = load_library().flarepp_mixer_fwd_profiled(*args, _event_array(stage_events))
     if st != 0:
         raise FlareError(st, "flarepp_mixer_fwd")
+    _device_check(device_check, given, workspace, stream, "flarepp_mixer_fwd")
     return Y
 
 
 def flarepp_mixer_out_fwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, Wo, lengths=None, scale: float = 0.0, Out=None,
-                          workspace=None, stream=None, check: bool = True):
+                          workspace=None, stream=None, check: bool = True, device_check=None):
     """FLARE++ forward with the head concatenation and output projection:
     Out [B,N,C] bf16 = (Y_1 | ... | Y_H) @ Wo.  Passing the same tensors as
     Wk_syn/Wv_syn and Wk/Wv selects the shared-projection variant."""
@@ -240,22 +282,27 @@ def flarepp_mixer_out_fwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, Wo, lengths=None, scale
     if Out is None:
         Out = torch.empty((B, N, C), dtype=torch.bfloat16, device=X.device)
     nbytes = flare_workspace_bytes(FLARE_VARIANT_FLAREPP_OUT, B, H, N, M, D, C)
+    given = workspace is not None
     workspace = _workspace(workspace, nbytes, X.device)
     st = load_library().flarepp_mixer_out_fwd(
         _ptr(X), _ptr(Wk), _ptr(Wv), _ptr(Wk_syn), _ptr(Wv_syn), _ptr(Q0), _ptr(Wo), _ptr(Out), B, N, C, H, M, D,
         _ptr(lengths), float(scale), _ptr(workspace), workspace.numel(), _stream_ptr(stream, X.device))
     if st != 0:
         raise FlareError(st, "flarepp_mixer_out_fwd")
+    _device_check(device_check, given, workspace, stream, "flarepp_mixer_out_fwd")
     return Out
 
 
 FLARE_STATIC_SCRATCH_BYTES = 64 << 20
 
 
-def flare_mixer_fwd_static(K, V, Q, lengths=None, scale: float = 0.0, Y=None, stream=None, Z_out=None):
+def flare_mixer_fwd_static(K, V, Q, lengths=None, scale: float = 0.0, Y=None, stream=None, Z_out=None,
+                           device_check: bool = True):
     """FLARE forward without a caller-provided workspace (the library's fixed
     device scratch of FLARE_STATIC_SCRATCH_BYTES is used; nothing is
-    allocated by the library).  Calls must not overlap on the GPU."""
+    allocated by the library).  Calls must not overlap on the GPU.  With
+    ``device_check`` the static scratch's error word is read after the call
+    (synchronises the stream) and a set word raises FlareError."""
     torch = _torch()
     B, H, N, D = K.shape
     M = Q.shape[1]
@@ -270,11 +317,15 @@ def flare_mixer_fwd_static(K, V, Q, lengths=None, scale: float = 0.0, Y=None, st
                                                float(scale), _stream_ptr(stream, K.device), _ptr(Z_out))
     if st != 0:
         raise FlareError(st, "flare_mixer_fwd_static")
+    if device_check:
+        st = load_library().flare_static_last_device_status(_stream_ptr(stream, K.device))
+        if st != 0:
+            raise FlareError(st, "flare_mixer_fwd_static (device status)")
     return Y
 
 
 def flare_mixer_bwd(K, V, Q, dY, lengths=None, scale: float = 0.0, workspace=None, stream=None,
-                    dK=None, dV=None, dQ=None, check: bool = True):
+                    dK=None, dV=None, dQ=None, check: bool = True, device_check=None):
     """FLARE backward (gradients of eq. 5-6 given dY).  K, V, dY: [B,H,N,D] bf16;
     Q: [H,M,D] bf16 -> (dK, dV) [B,H,N,D] bf16 and dQ [H,M,D] float32."""
     torch = _torch()
@@ -291,17 +342,19 @@ def flare_mixer_bwd(K, V, Q, dY, lengths=None, scale: float = 0.0, workspace=Non
     dV = torch.empty_like(K) if dV is None else dV
     dQ = torch.empty((H, M, D), dtype=torch.float32, device=K.device) if dQ is None else dQ
     nbytes = flare_workspace_bytes(FLARE_VARIANT_FLARE_BWD, B, H, N, M, D)
+    given = workspace is not None
     workspace = _workspace(workspace, nbytes, K.device)
     st = load_library().flare_mixer_bwd(_ptr(K), _ptr(V), _ptr(Q), _ptr(dY), _ptr(dK), _ptr(dV), _ptr(dQ),
                                         B, H, N, M, D, _ptr(lengths), float(scale), _ptr(workspace),
                                         workspace.numel(), _stream_ptr(stream, K.device))
     if st != 0:
         raise FlareError(st, "flare_mixer_bwd")
+    _device_check(device_check, given, workspace, stream, "flare_mixer_bwd")
     return dK, dV, dQ
 
 
 def flarepp_mixer_bwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, lengths=None, scale: float = 0.0, workspace=None,
-                      stream=None, grads=None, check: bool = True):
+                      stream=None, grads=None, check: bool = True, device_check=None):
     """FLARE++ backward (gradients of eq. 7-11 given dY [B,H,N,D] bf16).
     Returns a dict: dX [B,N,C] bf16; dWk, dWv, dWk_syn, dWv_syn [C,C] float32;
     dQ0 [H,M,D] float32.  ``grads`` may hold preallocated outputs by name."""
@@ -330,6 +383,7 @@ def flarepp_mixer_bwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, lengths=None, scale: fl
             _check_dev(nm, g[nm], torch.float32, (C, C))
         _check_dev("dQ0", g["dQ0"], torch.float32, (H, M, D))
     nbytes = flare_workspace_bytes(FLARE_VARIANT_FLAREPP_BWD, B, H, N, M, D, C)
+    given = workspace is not None
     workspace = _workspace(workspace, nbytes, dev)
     st = load_library().flarepp_mixer_bwd(
         _ptr(X), _ptr(Wk), _ptr(Wv), _ptr(Wk_syn), _ptr(Wv_syn), _ptr(Q0), _ptr(dY), _ptr(g["dX"]),
@@ -338,11 +392,33 @@ def flarepp_mixer_bwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, lengths=None, scale: fl
         _stream_ptr(stream, dev))
     if st != 0:
         raise FlareError(st, "flarepp_mixer_bwd")
+    _device_check(device_check, given, workspace, stream, "flarepp_mixer_bwd")
     return g
 
 
 def flare_last_device_status(workspace, stream=None) -> Status:
     return Status(load_library().flare_last_device_status(_ptr(workspace), _stream_ptr(stream, workspace.device)))
+
+
+def flare_static_last_device_status(stream=None) -> Status:
+    """Device error word of the last flare_mixer_fwd_static call (syncs the stream)."""
+    torch = _torch()
+    return Status(load_library().flare_static_last_device_status(_stream_ptr(stream, torch.device("cuda"))))
+
+
+def flare_probe_pipe_rates(device=None, stream=None) -> dict:
+    """Measured results per SM clock of ex2.approx.f32 (special-function unit)
+    and fp32 fma (FMA pipe) on this device: {"ex2": ..., "ffma": ...}."""
+    torch = _torch()
+    device = torch.device("cuda") if device is None else torch.device(device)
+    lib = load_library()
+    scratch = torch.empty(int(lib.flare_probe_scratch_bytes()), dtype=torch.uint8, device=device)
+    e, f = ctypes.c_double(0.0), ctypes.c_double(0.0)
+    st = lib.flare_probe_pipe_rates(_ptr(scratch), scratch.numel(), _stream_ptr(stream, device), ctypes.byref(e),
+                                    ctypes.byref(f))
+    if st != 0:
+        raise FlareError(st, "flare_probe_pipe_rates")
+    return {"ex2": e.value, "ffma": f.value}
 
 
 def flare_selftest_wait_timeout(workspace, timeout_ns: int, stream=None) -> None:

@@ -27,14 +27,30 @@ def _group_info(group):
     return dist.get_rank(group), dist.get_world_size(group)
 
 
-def allgather_partials(part, world: int, group=None):
-    """Concatenate every rank's partials in rank order: [world * part.numel()]."""
+def allgather_partials(part, world: int, group=None, stream=None):
+    """Concatenate every rank's partials in rank order: [world * part.numel()].
+
+    The library writes ``part`` and reads the result on ``stream`` (None: the
+    current stream), while the collective runs on torch's current stream.
+    When the two differ, the collective first waits for ``stream``, ``stream``
+    then waits for the collective, and both buffers are recorded as used on
+    ``stream`` so that the caching allocator does not hand their memory out
+    while a library kernel may still touch it."""
     torch = b._torch()
+    cur = torch.cuda.current_stream(part.device) if part.is_cuda else None
+    other = part.is_cuda and stream is not None and stream != cur
+    if other:
+        part.record_stream(stream)
     if world == 1:
         return part
     import torch.distributed as dist
+    if other:
+        cur.wait_stream(stream)
     out = torch.empty(world * part.numel(), dtype=part.dtype, device=part.device)
     dist.all_gather_into_tensor(out, part, group=group)
+    if other:
+        stream.wait_stream(cur)
+        out.record_stream(stream)
     return out
 
 
@@ -50,11 +66,27 @@ def _status(st, where):
         raise b.FlareError(st, where)
 
 
+def _device_status(device_check, workspace_given, ws, stream, where):
+    """After the last phase: read the workspace's device error word (a merged
+    row whose sums underflowed, a length outside [1, N], an expired bounded
+    wait) and raise FlareError if it is set; synchronises the stream.  Done by
+    default when the workspace was allocated here (the caller cannot query
+    it)."""
+    if device_check is None:
+        device_check = not workspace_given
+    if device_check:
+        st = b.load_library().flare_last_device_status(b._ptr(ws), b._stream_ptr(stream, ws.device))
+        if st != 0:
+            raise b.FlareError(st, where + " (device status)")
+
+
 def flarepp_mixer_cp_fwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, lengths=None, group=None, scale: float = 0.0,
-                         Y=None, workspace=None, stream=None, Qx_out=None, Z_out=None):
+                         Y=None, workspace=None, stream=None, Qx_out=None, Z_out=None, device_check=None):
     """FLARE++ forward of this rank's token shard X [B, N, C] (tokens
     [rank*N, (rank+1)*N) of sequences of world*N tokens; ``lengths`` counts
-    tokens of the whole sequences).  Returns Y [B, H, N, D] of the shard."""
+    tokens of the whole sequences).  Returns Y [B, H, N, D] of the shard.
+    ``stream``: a torch stream for the library's kernels (None: the current
+    stream).  ``device_check``: see ``_device_status``."""
     torch = b._torch()
     rank, world = _group_info(group)
     B, N, C = X.shape
@@ -64,21 +96,24 @@ def flarepp_mixer_cp_fwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, lengths=None, group=None
         Y = torch.empty((B, H, N, D), dtype=torch.bfloat16, device=X.device)
     nbytes = b.flare_workspace_bytes(b.FLARE_VARIANT_FLAREPP, B, H, N, M, D, C)
     ws = b._workspace(workspace, nbytes, X.device)
+    if stream is not None and X.is_cuda:
+        ws.record_stream(stream)
     st = b._stream_ptr(stream, X.device)
     part = torch.empty(partials_numel(B, H, N, M, D), dtype=torch.float32, device=X.device)
     common = (B, N, C, H, M, D, b._ptr(lengths), rank, world, float(scale), b._ptr(ws), ws.numel(), st)
     _status(lib.flarepp_cp_begin(b._ptr(X), b._ptr(Wk), b._ptr(Wv), b._ptr(Wk_syn), b._ptr(Wv_syn), b._ptr(Q0),
                                  *common, b._ptr(part)), "flarepp_cp_begin")
-    gathered = allgather_partials(part, world, group)
+    gathered = allgather_partials(part, world, group, stream)
     part2 = torch.empty_like(part)
     _status(lib.flarepp_cp_middle(b._ptr(gathered), *common, b._ptr(part2), b._ptr(Qx_out)), "flarepp_cp_middle")
-    gathered = allgather_partials(part2, world, group)
+    gathered = allgather_partials(part2, world, group, stream)
     _status(lib.flarepp_cp_end(b._ptr(gathered), b._ptr(Y), *common, b._ptr(Z_out)), "flarepp_cp_end")
+    _device_status(device_check, workspace is not None, ws, stream, "flarepp_mixer_cp_fwd")
     return Y
 
 
 def flare_mixer_cp_fwd(K, V, Q, lengths=None, group=None, scale: float = 0.0, Y=None, workspace=None,
-                       stream=None, Z_out=None):
+                       stream=None, Z_out=None, device_check=None):
     """FLARE forward of this rank's token shard K, V [B, H, N, D] (see
     flarepp_mixer_cp_fwd).  Returns Y [B, H, N, D] of the shard."""
     torch = b._torch()
@@ -90,13 +125,16 @@ def flare_mixer_cp_fwd(K, V, Q, lengths=None, group=None, scale: float = 0.0, Y=
         Y = torch.empty_like(K)
     nbytes = b.flare_workspace_bytes(b.FLARE_VARIANT_FLARE, B, H, N, M, D)
     ws = b._workspace(workspace, nbytes, K.device)
+    if stream is not None and K.is_cuda:
+        ws.record_stream(stream)
     st = b._stream_ptr(stream, K.device)
     part = torch.empty(partials_numel(B, H, N, M, D), dtype=torch.float32, device=K.device)
     common = (B, H, N, M, D, b._ptr(lengths), rank, world, float(scale), b._ptr(ws), ws.numel(), st)
     _status(lib.flare_cp_begin(b._ptr(K), b._ptr(V), b._ptr(Q), *common, b._ptr(part)), "flare_cp_begin")
-    gathered = allgather_partials(part, world, group)
+    gathered = allgather_partials(part, world, group, stream)
     _status(lib.flare_cp_end(b._ptr(gathered), b._ptr(K), b._ptr(Q), b._ptr(Y), *common, b._ptr(Z_out)),
             "flare_cp_end")
+    _device_status(device_check, workspace is not None, ws, stream, "flare_mixer_cp_fwd")
     return Y
 
 
@@ -104,7 +142,7 @@ FLARE_CP_BWD_PHASES = 7
 
 
 def flarepp_mixer_cp_bwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, lengths=None, group=None, scale: float = 0.0,
-                         workspace=None, stream=None, grads=None):
+                         workspace=None, stream=None, grads=None, device_check=None):
     """FLARE++ backward of this rank's token shard (the same sharding as
     flarepp_mixer_cp_fwd; dY [B, H, N, D] holds the shard's rows).  Returns a
     dict: dX [B, N, C] (the shard's rows), dWk, dWv, dWk_syn, dWv_syn, dQ0
@@ -126,6 +164,8 @@ def flarepp_mixer_cp_bwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, lengths=None, group=
         g["dQ0"] = torch.empty((H, M, D), dtype=torch.float32, device=dev)
     nbytes = b.flare_workspace_bytes(b.FLARE_VARIANT_FLAREPP_BWD, B, H, N, M, D, C)
     ws = b._workspace(workspace, nbytes, dev)
+    if stream is not None and X.is_cuda:
+        ws.record_stream(stream)
     st = b._stream_ptr(stream, dev)
     ins = [b._ptr(t) for t in (X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY)]
     outs = [b._ptr(g[k]) for k in ("dX", "dWk", "dWv", "dWk_syn", "dWv_syn", "dQ0")]
@@ -141,5 +181,6 @@ def flarepp_mixer_cp_bwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, lengths=None, group=
                                          b._ptr(lengths), rank, world, float(scale), b._ptr(ws), ws.numel(), st),
                 f"flarepp_cp_bwd_phase({phase})")
         if exch is not None:
-            gathered = allgather_partials(exch, world, group)
+            gathered = allgather_partials(exch, world, group, stream)
+    _device_status(device_check, workspace is not None, ws, stream, "flarepp_mixer_cp_bwd")
     return g

@@ -227,7 +227,7 @@ flare_status run_encode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
 flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_batch, const uint16_t* z16,
                         const void* k, void* y, int y_token_major, int B, int H, int N, int M, int D,
                         const int32_t* lengths, float scale, cudaStream_t st, int tok_offset = 0,
-                        int n_global = -1) {
+                        int n_global = -1, float* y_f32 = nullptr) {
   const long BH = static_cast<long>(B) * H;
   const long G = q_per_batch ? BH : H;
   CUtensorMap tq, tz, tk;
@@ -247,6 +247,7 @@ flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
   dp.k = static_cast<const uint16_t*>(k);
   dp.y = static_cast<uint16_t*>(y);
   dp.y_token_major = y_token_major;
+  dp.y_f32 = y_f32;
   dp.tok_offset = tok_offset;
   dp.n_global = n_global < 0 ? N : n_global;
   dp.err = reinterpret_cast<uint32_t*>(ws + pl.off_err);
@@ -318,15 +319,21 @@ const char* flare_status_string(flare_status s) {
   return "unknown flare_status";
 }
 
-flare_status flare_mixer_fwd_profiled(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, flare_bf16* Y,
-                                      int B, int H, int N, int M, int D, const int32_t* lengths, float scale,
-                                      void* workspace, size_t workspace_bytes, void* stream, float* Z_out,
-                                      void* const* stage_events) {
+}  // extern "C"
+
+namespace flare {
+
+// The FLARE forward (eq. 5-6) after nothing but the caller's arguments:
+// checks, then key norms | encode | merge | decode on `stream`.
+flare_status flare_fwd(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, flare_bf16* Y, int B, int H,
+                       int N, int M, int D, const int32_t* lengths, float scale, void* workspace,
+                       size_t workspace_bytes, void* stream, float* Z_out, float* Y_f32_out,
+                       void* const* stage_events) {
   if (!K || !V || !Q || !Y || !workspace) return FLARE_ERR_NULL;
   flare_status st = check_common(B, H, N, M, D);
   if (st != FLARE_OK) return st;
   if (!aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(Y) || !aligned16(lengths) || !aligned16(Z_out) ||
-      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      !aligned16(Y_f32_out) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return FLARE_ERR_ALIGN;
   const Plan pl = make_plan(FLARE_VARIANT_FLARE, B, H, N, M, D);
   if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
@@ -341,9 +348,30 @@ flare_status flare_mixer_fwd_profiled(const flare_bf16* K, const flare_bf16* V, 
   uint16_t* z16 = reinterpret_cast<uint16_t*>(ws + pl.off_z16);
   st = run_encode(pl, ws, Q, 0, K, V, kp.knorm, z32, z16, B, H, N, M, D, lengths, sc, s, stage_events, 2);
   if (st != FLARE_OK) return st;
-  st = run_decode(pl, ws, Q, 0, z16, K, Y, 0, B, H, N, M, D, lengths, sc, s);
+  st = run_decode(pl, ws, Q, 0, z16, K, Y, 0, B, H, N, M, D, lengths, sc, s, 0, -1, Y_f32_out);
   if (st != FLARE_OK) return st;
   return record(stage_events, 4, s) ? FLARE_OK : FLARE_ERR_LAUNCH;
+}
+
+}  // namespace flare
+
+extern "C" {
+
+flare_status flare_mixer_fwd_profiled(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, flare_bf16* Y,
+                                      int B, int H, int N, int M, int D, const int32_t* lengths, float scale,
+                                      void* workspace, size_t workspace_bytes, void* stream, float* Z_out,
+                                      void* const* stage_events) {
+  return flare_fwd(K, V, Q, Y, B, H, N, M, D, lengths, scale, workspace, workspace_bytes, stream, Z_out, nullptr,
+                   stage_events);
+}
+
+flare_status flare_mixer_fwd_inspect(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, flare_bf16* Y,
+                                     int B, int H, int N, int M, int D, const int32_t* lengths, float scale,
+                                     void* workspace, size_t workspace_bytes, void* stream, float* Z_out,
+                                     float* Y_f32_out) {
+  if (!Y_f32_out) return FLARE_ERR_NULL;
+  return flare_fwd(K, V, Q, Y, B, H, N, M, D, lengths, scale, workspace, workspace_bytes, stream, Z_out, Y_f32_out,
+                   nullptr);
 }
 
 flare_status flare_mixer_fwd(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, flare_bf16* Y, int B,
@@ -441,7 +469,7 @@ flare_status flarepp_run(const Plan& pl, const flare_bf16* X, const flare_bf16* 
                          const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0, void* Y,
                          int y_token_major, int B, int N, int C, int H, int M, int D, const int32_t* lengths,
                          float sc, uint8_t* ws, cudaStream_t s, float* Qx_out, float* Z_out,
-                         void* const* stage_events) {
+                         void* const* stage_events, float* Y_f32_out = nullptr) {
   if (cudaMemsetAsync(ws + pl.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   Projected pr;
   flare_status st = flarepp_project(pl, X, Wk, Wv, Wk_syn, Wv_syn, B, N, C, H, D, ws, s, stage_events, &pr);
@@ -460,7 +488,7 @@ flare_status flarepp_run(const Plan& pl, const flare_bf16* X, const flare_bf16* 
   st = run_encode(pl, ws, qx16, 1, kk, vv, kn, z32, z16, B, H, N, M, D, lengths, sc, s, stage_events, 4);
   if (st != FLARE_OK) return st;
   // eq. 11: decode
-  st = run_decode(pl, ws, qx16, 1, z16, kk, Y, y_token_major, B, H, N, M, D, lengths, sc, s);
+  st = run_decode(pl, ws, qx16, 1, z16, kk, Y, y_token_major, B, H, N, M, D, lengths, sc, s, 0, -1, Y_f32_out);
   if (st != FLARE_OK) return st;
   return record(stage_events, 6, s) ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
@@ -483,6 +511,23 @@ flare_status flarepp_mixer_fwd_profiled(const flare_bf16* X, const flare_bf16* W
   return flarepp_run(pl, X, Wk, Wv, Wk_syn, Wv_syn, Q0, Y, 0, B, N, C, H, M, D, lengths, resolve_scale(scale, D),
                      static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream), Qx_out, Z_out,
                      stage_events);
+}
+
+flare_status flarepp_mixer_fwd_inspect(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                                       const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0,
+                                       flare_bf16* Y, int B, int N, int C, int H, int M, int D,
+                                       const int32_t* lengths, float scale, void* workspace, size_t workspace_bytes,
+                                       void* stream, float* Qx_out, float* Z_out, float* Y_f32_out) {
+  if (!Y_f32_out) return FLARE_ERR_NULL;
+  flare_status st = check_flarepp(X, Wk, Wv, Wk_syn, Wv_syn, Q0, Y, B, N, C, H, M, D, lengths, workspace, Qx_out,
+                                  Z_out);
+  if (st != FLARE_OK) return st;
+  if (!aligned16(Y_f32_out)) return FLARE_ERR_ALIGN;
+  const Plan pl = make_plan(FLARE_VARIANT_FLAREPP, B, H, N, M, D);
+  if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
+  return flarepp_run(pl, X, Wk, Wv, Wk_syn, Wv_syn, Q0, Y, 0, B, N, C, H, M, D, lengths, resolve_scale(scale, D),
+                     static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream), Qx_out, Z_out, nullptr,
+                     Y_f32_out);
 }
 
 flare_status flarepp_mixer_out_fwd(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
@@ -689,6 +734,15 @@ flare_status flare_last_device_status(void* workspace, void* stream) {
   if (word & FLARE_DEV_BAD_LENGTH) return FLARE_ERR_SHAPE;
   if (word & FLARE_DEV_UNDERFLOW) return FLARE_ERR_UNDERFLOW;
   return FLARE_OK;
+}
+
+flare_status flare_static_last_device_status(void* stream) {
+  // The error word of flare_mixer_fwd_static sits at the start of the static
+  // scratch, exactly where a workspace keeps it.
+  void* scratch = nullptr;
+  const flare_status st = static_scratch_address(&scratch);
+  if (st != FLARE_OK) return st;
+  return flare_last_device_status(scratch, stream);
 }
 
 flare_status flare_selftest_wait_timeout(void* workspace, void* stream, unsigned long long timeout_ns) {

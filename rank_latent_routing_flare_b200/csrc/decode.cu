@@ -125,6 +125,12 @@ __global__ void __launch_bounds__(128) decode_fallback_kernel(const DecodeParams
       for (int d = 0; d < D; ++d) y[d] = fmaf(w, __uint_as_float(static_cast<uint32_t>(zh[m * D + d]) << 16), y[d]);
     }
     const float inv = 1.f / den;
+    if (p.y_f32 != nullptr) {
+      float4* d32 = reinterpret_cast<float4*>(p.y_f32 + (static_cast<size_t>(bh) * p.N + n) * D);
+#pragma unroll
+      for (int u = 0; u < D / 4; ++u)
+        d32[u] = make_float4(y[4 * u] * inv, y[4 * u + 1] * inv, y[4 * u + 2] * inv, y[4 * u + 3] * inv);
+    }
     uint4* dst = reinterpret_cast<uint4*>(y_row<D>(p, bh, n));
 #pragma unroll
     for (int u = 0; u < D / 8; ++u)
@@ -185,6 +191,12 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
     for (size_t e = static_cast<size_t>(z0) * (D / 8) + threadIdx.x; e < static_cast<size_t>(z1) * (D / 8);
          e += blockDim.x)
       reinterpret_cast<uint4*>(y_row<D>(p, bh, static_cast<int>(e / (D / 8))))[e % (D / 8)] = zero;
+    if (p.y_f32 != nullptr) {
+      uint4* d32 = reinterpret_cast<uint4*>(p.y_f32 + static_cast<size_t>(bh) * p.N * D);
+      for (size_t e = static_cast<size_t>(z0) * (D / 4) + threadIdx.x; e < static_cast<size_t>(z1) * (D / 4);
+           e += blockDim.x)
+        d32[e] = zero;
+    }
   }
   if (ntiles == 0) return;
 
@@ -365,6 +377,11 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
         const uint32_t e = atomicAdd(p.fb_count, 1u);
         p.fb_list[e] = static_cast<uint64_t>(bh) * p.N + n;
       } else if (n < p.N) {
+        if (p.y_f32 != nullptr) {
+          float4* d32 = reinterpret_cast<float4*>(p.y_f32 + (static_cast<size_t>(bh) * p.N + n) * D);
+#pragma unroll
+          for (int u = 0; u < D / 4; ++u) d32[u] = make_float4(y[4 * u], y[4 * u + 1], y[4 * u + 2], y[4 * u + 3]);
+        }
         uint4* dst = reinterpret_cast<uint4*>(y_row<D>(p, bh, n));
 #pragma unroll
         for (int u = 0; u < D / 8; ++u)

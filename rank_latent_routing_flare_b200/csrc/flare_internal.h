@@ -161,6 +161,7 @@ struct DecodeParams {
   const uint16_t* k;    // bf16 [B*H][N][D]
   uint16_t* y;          // bf16 [B*H][N][D], or [B][N][H*D] when y_token_major
   int y_token_major;
+  float* y_f32;         // optional fp32 copy of Y ([B*H][N][D], the values Y is rounded from), or nullptr
   uint32_t* fb_count;   // number of listed tokens (zeroed before the decoder runs)
   uint64_t* fb_list;    // tokens (bh * N + n) whose row sum underflowed, capacity B*H*N
   uint32_t* err;

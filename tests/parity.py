@@ -1,0 +1,169 @@
+"""Parity criteria of the CUDA path against the fp64 oracle, in plain numpy.
+
+Used by the GPU tests (through ``gpu_util.compare``) and pinned on the CPU by
+``test_centred_bound.py``, which runs the same checks on the oracle's own
+outputs, on a model of the CUDA path's bf16 storage and on planted wrong
+decoders.
+
+Two criteria on the output Y:
+
+1. The stated tolerance: relative L2 <= 5e-3 and max |error| <= 3e-2.
+2. The token-centred part.  Under the workloads' distributions the FLARE++
+   output is nearly the same for every token: the part of Y that depends on
+   the token, Y_n - mean_n(Y) per (b, h) -- the part that the decoder's
+   routing softmax_m(K_n Q(X)^T) decides (FLARE++ paper, section "FLARE++:
+   dynamic token routing", eq. 11) -- is only 0.3-2 % of ||Y||.  A relative
+   L2 of 5e-3 on Y therefore permits a wrong routing; the centred part is
+   held to its own bound:
+
+   - fp32 Y (the inspection entry points): rel-L2 of the centred part
+     <= CENTRED_F32 = 5e-2.  Derivation: the CUDA path loses accuracy only
+     where it stores an intermediate in bf16 (K~, V~, K, V, Q(X), Z and the
+     softmax weights P as tensor-core operands); the oracle run on exactly
+     those rounded values (``storage_model`` plus bf16 weights) moves the
+     centred part by at most 1.25e-2 on every FLARE++ workload, so 5e-2
+     leaves a factor 4.  A decoder that gives every token the same row has
+     error 1.
+   - bf16 Y: the output's own rounding (half an ulp of each element, about
+     0.2 % of ||Y||) is as large as the centred part itself on the 8K-token
+     workloads.  That rounding error is measured exactly on the oracle's Y
+     (e_r = ||c(bf16(Y_ref)) - c(Y_ref)|| / ||c(Y_ref)||); the GPU's bf16 Y
+     carries one of the same size, independent of the routing error, so the
+     bound is 1.25 * e_r + 5e-2 (1.25 covers the statistical spread of the
+     rounding error's norm, 5e-2 the computation as above).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from workloads import bf16_bits_to_f64, to_bf16_bits
+
+# stated tolerance on the bf16 outputs (fp32 accumulation)
+REL_L2 = 5e-3
+MAX_ABS = 3e-2
+# token-centred part of Y
+CENTRED_F32 = 5e-2
+CENTRED_BF16_SLACK = 1.25
+CENTRED_BF16_ALLOW = 5e-2
+
+
+def rel_l2(a, b) -> float:
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def max_abs(a, b) -> float:
+    return float(np.max(np.abs(np.asarray(a, np.float64) - np.asarray(b, np.float64))))
+
+
+def bf16_round(a) -> np.ndarray:
+    """Round to bf16 as the CUDA path stores (float32, then round to nearest even)."""
+    return bf16_bits_to_f64(to_bf16_bits(a))
+
+
+def centred(Y, lengths=None, rows=None) -> np.ndarray:
+    """Token-centred part of Y [B][H][n][D]: per (b, h), each valid row minus
+    the mean of the valid rows; rows of padding tokens are dropped.  ``rows``
+    gives the token index of each of the n rows (sampled rows; default 0..n-1),
+    the mean is then over the valid sampled rows.  Returns a flat vector."""
+    Y = np.asarray(Y, np.float64)
+    B, H, n, D = Y.shape
+    idx = np.arange(n) if rows is None else np.asarray(rows)
+    out = []
+    for b in range(B):
+        valid = np.ones(n, bool) if lengths is None else idx < int(lengths[b])
+        yb = Y[b][:, valid]
+        if yb.shape[1] == 0:
+            continue
+        out.append((yb - yb.mean(axis=1, keepdims=True)).ravel())
+    return np.concatenate(out) if out else np.zeros(0)
+
+
+def centred_errors(Y_ref, Y=None, Y32=None, lengths=None, rows=None) -> dict:
+    """Relative L2 errors of the token-centred parts of a bf16 output Y and an
+    fp32 output Y32 against the oracle's Y_ref, the oracle's own bf16-rounding
+    error ``e_r`` and the bf16 bound that follows from it.  Empty when the
+    oracle's centred part vanishes (one token, one latent)."""
+    yc = centred(Y_ref, lengths, rows)
+    nrm = float(np.linalg.norm(yc))
+    if yc.size == 0 or nrm <= 1e-12 * max(float(np.linalg.norm(Y_ref)), 1e-300):
+        return {}
+    e_r = float(np.linalg.norm(centred(bf16_round(Y_ref), lengths, rows) - yc)) / nrm
+    errs = {"Yc_round": e_r, "Yc_bound": CENTRED_BF16_SLACK * e_r + CENTRED_BF16_ALLOW}
+    if Y is not None:
+        errs["Yc_rel_l2"] = float(np.linalg.norm(centred(Y, lengths, rows) - yc)) / nrm
+    if Y32 is not None:
+        errs["Yc32_rel_l2"] = float(np.linalg.norm(centred(Y32, lengths, rows) - yc)) / nrm
+    return errs
+
+
+def check(gpu: dict, ref: dict, rows=None, lengths=None, label: str = "") -> dict:
+    """Assert both criteria on ``gpu["Y"]`` (bf16 values as float64) and, if
+    present, ``gpu["Y32"]`` (fp32), plus the standard tolerance on the fp32
+    diagnostics Q(X) and Z; ``rows`` selects sampled rows of the GPU output
+    that ``ref`` holds.  Returns the measured errors."""
+    Yg = gpu["Y"] if rows is None else gpu["Y"][:, :, rows]
+    Y32 = gpu.get("Y32")
+    if Y32 is not None and rows is not None:
+        Y32 = Y32[:, :, rows]
+    errs = {"Y_rel_l2": rel_l2(Yg, ref["Y"]), "Y_max_abs": max_abs(Yg, ref["Y"])}
+    for k in ("Qx", "Z"):
+        if k in gpu and k in ref:
+            errs[f"{k}_rel_l2"] = rel_l2(gpu[k], ref[k])
+    errs.update(centred_errors(ref["Y"], Yg, Y32, lengths, rows))
+    print(label, {k: f"{v:.3e}" for k, v in errs.items()})
+    assert np.all(np.isfinite(Yg)), label
+    assert errs["Y_rel_l2"] <= REL_L2, (label, errs)
+    assert errs["Y_max_abs"] <= MAX_ABS, (label, errs)
+    for k in ("Qx_rel_l2", "Z_rel_l2"):
+        if k in errs:
+            assert errs[k] <= REL_L2, (label, errs)
+    if "Yc_rel_l2" in errs:
+        assert errs["Yc_rel_l2"] <= errs["Yc_bound"], (label, "token-centred Y (bf16)", errs)
+    if "Yc32_rel_l2" in errs:
+        assert np.all(np.isfinite(Y32)), label
+        assert errs["Yc32_rel_l2"] <= CENTRED_F32, (label, "token-centred Y (fp32)", errs)
+    return errs
+
+
+def storage_model(w, oracle, p_round: bool = False) -> dict:
+    """The oracle's own functions composed with the CUDA path's storage format:
+    K~, V~, K, V, Q(X) and Z rounded to bf16 where the kernels store them as
+    tensor-core operands.  Everything else is the fp64 oracle.  With
+    ``p_round`` the softmax weights are rounded to bf16 too (as the value
+    products read them), computed here in numpy.  Returns Qx, Z and Y
+    (unrounded)."""
+    f64 = bf16_bits_to_f64
+    X = f64(w.X)
+    Wk, Wv, Wks, Wvs = (f64(a) for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn))
+    Kt, Vt = bf16_round(oracle.project(X, Wks, w.H)), bf16_round(oracle.project(X, Wvs, w.H))
+    K, V = bf16_round(oracle.project(X, Wk, w.H)), bf16_round(oracle.project(X, Wv, w.H))
+    if not p_round:
+        Qx = oracle.encode(f64(w.Q0), Kt, Vt, w.lengths)
+        Z = oracle.encode(bf16_round(Qx), K, V, w.lengths)
+        return {"Qx": Qx, "Z": Z, "Y": oracle.decode(K, bf16_round(Qx), bf16_round(Z), w.lengths)}
+    s = w.scale
+
+    def softmax_rounded(S):
+        return bf16_round(np.exp(S - S.max(axis=1, keepdims=True)))
+
+    def enc(Qs, Ks, Vs):
+        B, H = Ks.shape[:2]
+        out = np.zeros((B, H, Qs.shape[-2], Ks.shape[3]))
+        for b in range(B):
+            n = Ks.shape[2] if w.lengths is None else int(w.lengths[b])
+            for h in range(H):
+                P = softmax_rounded((Qs[b, h] if Qs.ndim == 4 else Qs[h]) @ Ks[b, h, :n].T * s)
+                out[b, h] = (P @ Vs[b, h, :n]) / P.sum(axis=1, keepdims=True)
+        return out
+
+    Qx = enc(f64(w.Q0), Kt, Vt)
+    Z = enc(bf16_round(Qx), K, V)
+    Qb, Zb = bf16_round(Qx), bf16_round(Z)
+    Y = np.zeros_like(K)
+    for b in range(K.shape[0]):
+        n = K.shape[2] if w.lengths is None else int(w.lengths[b])
+        for h in range(K.shape[1]):
+            P = softmax_rounded(K[b, h, :n] @ Qb[b, h].T * s)
+            Y[b, h, :n] = (P @ Zb[b, h]) / P.sum(axis=1, keepdims=True)
+    return {"Qx": Qx, "Z": Z, "Y": Y}

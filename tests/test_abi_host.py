@@ -35,7 +35,9 @@ def test_header_declares_the_abi():
                             "flare_selftest_wait_timeout", "flare_cp_partials_bytes", "flarepp_cp_begin",
                             "flarepp_cp_middle", "flarepp_cp_end", "flare_cp_begin", "flare_cp_end",
                             "flare_mixer_bwd", "flarepp_mixer_bwd", "flarepp_cp_bwd_exchange_bytes",
-                            "flarepp_cp_bwd_phase"])
+                            "flarepp_cp_bwd_phase", "flare_mixer_fwd_inspect", "flarepp_mixer_fwd_inspect",
+                            "flare_static_last_device_status", "flare_probe_scratch_bytes",
+                            "flare_probe_pipe_rates"])
 
 
 def test_library_loads_and_exports_every_declared_symbol():

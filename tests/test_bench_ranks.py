@@ -99,3 +99,20 @@ def test_backward_work_counts_flare():
     th = w.B * w.H * w.N
     assert wk["exps"] == 2 * w.M * th and wk["flops"] == 20 * w.M * w.D * th
     assert wk["bytes"] == 5 * th * w.D * 2
+
+
+def test_exp_unit_bounds_balance_the_two_pipes():
+    """The combined bound puts the fraction f of exponentials on the
+    polynomial where the special-function unit and the issue slots take
+    equally long; it is never above the MUFU-only bound, and with a MUFU as
+    fast as the issue rate nothing is moved."""
+    b = bench.exp_unit_bounds({"ex2": 16.0, "ffma": 128.0})
+    f = b["poly_fraction"]
+    assert 0.0 < f < 1.0
+    t_mufu = (1 - f) / 16.0
+    t_issue = (bench.SOFTMAX_BASE_OPS + (1 - f) + bench.POLY_EXP_OPS * f) / 128.0
+    assert abs(t_mufu - t_issue) < 1e-12 and abs(b["combined"] - t_mufu) < 1e-12
+    assert b["combined"] < b["mufu_only"] == 1 / 16.0
+    fast = bench.exp_unit_bounds({"ex2": 128.0, "ffma": 128.0})
+    assert fast["poly_fraction"] == 0.0
+    assert fast["combined"] == max(1 / 128.0, (bench.SOFTMAX_BASE_OPS + 1) / 128.0)

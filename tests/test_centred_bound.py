@@ -1,0 +1,134 @@
+"""CPU pins of the parity criteria (``parity.py``), in particular the bound on
+the token-centred part of Y.
+
+Under the workloads' distributions the FLARE++ output is nearly the same for
+every token, so the stated tolerance on Y alone cannot tell a correct decoder
+from one that routes every token the same way.  These tests run the GPU
+tests' own ``check`` on:
+
+- a model of the CUDA path's arithmetic (the oracle on bf16-stored
+  projections, Q(X), Z and softmax weights, the output rounded to bf16):
+  it must pass, on every FLARE++ workload the GPU tests use;
+- planted wrong decoders (every token given its head's token mean; routing
+  with the seeds Q0 instead of the synthesised Q(X); half the routing
+  strength): each must fail, including at the full size of the 8K-token
+  2-D point-cloud workload, where the centred part is 0.27 % of ||Y||.
+
+The planted mistakes live here, on the CPU; no GPU kernel is altered.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from workloads import bf16_bits_to_f64, make_workload
+
+from .parity import CENTRED_F32, bf16_round, centred_errors, check, storage_model
+
+CASES = [
+    ("flarepp_n1k", {}),
+    ("flarepp_n8k_mesh2d", {"N": 2048, "B": 2}),
+    ("flarepp_n64k", {"N": 8192, "B": 1}),
+    ("flarepp_n1m_mesh3d", {"N": 16384}),
+    ("flarepp_masked_n4k", {"N": 1024, "B": 8}),
+    ("flarepp_n8k_mesh2d", {}),
+]
+IDS = [f"{n}-{kw.get('N', 'full')}" for n, kw in CASES]
+
+
+@pytest.fixture(scope="module")
+def cases(oracle_mod):
+    out = {}
+    for (name, kw), cid in zip(CASES, IDS):
+        w = make_workload(name, **kw)
+        ref = oracle.forward_workload(w)
+        model = storage_model(w, oracle, p_round=True)
+        out[cid] = (w, ref, model)
+    return out
+
+
+def token_mean(Y, lengths):
+    """Every valid token of (b, h) gets the mean of the head's valid rows."""
+    out = np.zeros_like(Y)
+    for b in range(Y.shape[0]):
+        L = Y.shape[2] if lengths is None else int(lengths[b])
+        out[b, :, :L] = Y[b, :, :L].mean(axis=1, keepdims=True)
+    return out
+
+
+@pytest.mark.parametrize("cid", IDS)
+def test_model_of_the_cuda_arithmetic_passes(cases, cid):
+    w, ref, model = cases[cid]
+    errs = check({"Y": bf16_round(model["Y"]), "Y32": model["Y"], "Qx": model["Qx"], "Z": model["Z"]}, ref,
+                 lengths=w.lengths, label=f"model {cid}")
+    # the bound keeps a factor of at least 3 over what the stored intermediates cost
+    assert errs["Yc32_rel_l2"] <= CENTRED_F32 / 3
+
+
+@pytest.mark.parametrize("cid", IDS)
+def test_token_mean_decoder_fails(cases, cid):
+    w, ref, model = cases[cid]
+    Ym = token_mean(model["Y"], w.lengths)
+    with pytest.raises(AssertionError):
+        check({"Y": bf16_round(Ym)}, ref, lengths=w.lengths, label=f"token-mean bf16 {cid}")
+    # the centred criterion on bf16 Y rejects it by itself (with no fp32 copy)
+    errs = centred_errors(ref["Y"], bf16_round(Ym), Ym, w.lengths)
+    assert errs["Yc_rel_l2"] > errs["Yc_bound"]
+    assert errs["Yc32_rel_l2"] > CENTRED_F32
+
+
+def test_the_stated_tolerance_alone_misses_the_token_mean_decoder(cases):
+    """What motivated the centred bound: on the full 8K-token 2-D cloud the
+    token-mean decoder is within the stated rel-L2 (5e-3) of the oracle, and
+    its largest error (3.05e-2) exceeds the max-abs bound (3e-2) by 2 % only."""
+    w, ref, model = cases["flarepp_n8k_mesh2d-full"]
+    Ym = bf16_round(token_mean(model["Y"], w.lengths))
+    rel = np.linalg.norm(Ym - ref["Y"]) / np.linalg.norm(ref["Y"])
+    assert rel <= 5e-3 and np.max(np.abs(Ym - ref["Y"])) <= 1.05 * 3e-2
+
+
+@pytest.mark.parametrize("cid", IDS)
+def test_half_strength_routing_fails(cases, cid):
+    """Y = mean + 0.5 * (Y - mean): the routing's effect halved."""
+    w, ref, model = cases[cid]
+    Ym = token_mean(model["Y"], w.lengths)
+    Yh = Ym + 0.5 * (model["Y"] - Ym)
+    with pytest.raises(AssertionError):
+        check({"Y": bf16_round(Yh), "Y32": Yh}, ref, lengths=w.lengths, label=f"half routing {cid}")
+    assert centred_errors(ref["Y"], None, Yh, w.lengths)["Yc32_rel_l2"] > CENTRED_F32
+
+
+@pytest.mark.parametrize("cid", IDS[:3] + IDS[4:5])
+def test_decoder_routed_by_the_seeds_fails(cases, cid):
+    """A plausible slip: the decoder uses the seeds Q0 instead of the
+    synthesised Q(X) as its queries (eq. 11 read as eq. 6 with Q = Q0)."""
+    w, ref, model = cases[cid]
+    f64 = bf16_bits_to_f64
+    K = bf16_round(oracle.project(f64(w.X), f64(w.Wk), w.H))
+    Yq = oracle.decode(K, f64(w.Q0), bf16_round(model["Z"]), w.lengths)
+    with pytest.raises(AssertionError):
+        check({"Y": bf16_round(Yq), "Y32": Yq}, ref, lengths=w.lengths, label=f"seed routing {cid}")
+
+
+def test_flare_workload_rounding_alone_passes():
+    """FLARE (fixed queries ~ N(0,1)) routes strongly: the oracle's own bf16
+    output passes with a small centred error."""
+    w = make_workload("flare_n64k", N=4096, B=1)
+    ref = oracle.forward_workload(w)
+    errs = check({"Y": bf16_round(ref["Y"]), "Y32": ref["Y"]}, ref, label="flare rounding")
+    assert errs["Yc_rel_l2"] < 1e-2
+
+
+def test_sampled_rows_are_centred_over_the_sample():
+    """The million-token GPU test compares sampled rows: centring over the
+    sampled valid rows of both sides still rejects the token-mean decoder."""
+    w = make_workload("flarepp_n8k_mesh2d", N=4096, B=1)
+    ref_full = oracle.forward_workload(w)
+    rows = np.sort(np.random.default_rng(0).choice(w.N, 512, replace=False))
+    ref = {"Y": ref_full["Y"][:, :, rows]}
+    good = {"Y": bf16_round(ref_full["Y"]), "Y32": ref_full["Y"]}
+    check(good, ref, rows=rows, label="sampled exact")
+    Ym = token_mean(ref_full["Y"], None)
+    with pytest.raises(AssertionError):
+        check({"Y": bf16_round(Ym), "Y32": Ym}, ref, rows=rows, label="sampled token-mean")
+    errs = centred_errors(ref["Y"], bf16_round(Ym)[:, :, rows], Ym[:, :, rows], None, rows)
+    assert errs["Yc_rel_l2"] > errs["Yc_bound"] and errs["Yc32_rel_l2"] > CENTRED_F32

@@ -82,6 +82,10 @@ class _FakeLib:
         self.calls.append((phase, rank_arg, world_arg, seen, bool(exchange)))
         return 0
 
+    def flare_last_device_status(self, workspace, stream):
+        self.calls.append(("status",))
+        return 0
+
 
 def _bwd_rank_main(rank, world, port, out):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
@@ -121,6 +125,8 @@ def test_backward_phases_run_in_order_with_rank_ordered_gathers():
         p.join(timeout=60)
         assert p.exitcode == 0
     for rank, calls in results:
+        assert calls[-1] == ("status",)      # the device word is read after the last phase
+        calls = calls[:-1]
         assert [c[0] for c in calls] == list(range(7))
         assert all(c[1] == rank and c[2] == world for c in calls)
         assert calls[0][3] is None                       # nothing gathered before phase 0
@@ -130,3 +136,55 @@ def test_backward_phases_run_in_order_with_rank_ordered_gathers():
             want = [float(10 * (phase - 1) + i) for i in range(n)] + \
                    [float(100 + 10 * (phase - 1) + i) for i in range(n)]
             assert calls[phase][3] == want, (rank, phase)
+
+
+class _StatusLib(_FakeLib):
+    """A fake library whose device error word reports a bad length."""
+
+    def __init__(self, word):
+        super().__init__(0)
+        self.word = word
+
+    def flare_last_device_status(self, workspace, stream):
+        self.calls.append(("status",))
+        return self.word
+
+    def flare_status_string(self, status):
+        return b"FLARE_ERR_SHAPE (fake)"
+
+
+def _run_single_rank_bwd(monkeypatch, fake, workspace=None, device_check=None):
+    from rank_latent_routing_flare_b200 import _binding, cp
+    monkeypatch.setattr(_binding, "load_library", lambda *a, **k: fake)
+    monkeypatch.setattr(_binding, "flare_workspace_bytes", lambda *a, **k: 256)
+    # a CPU tensor stands in for the caller's device workspace
+    monkeypatch.setattr(_binding, "_workspace", lambda ws, n, dev: ws if ws is not None else torch.empty(n, dtype=torch.uint8))
+
+    class _Stream:
+        cuda_stream = 0
+    B, N, C, H, M, D = 1, 4, 64, 4, 2, 16
+    X = torch.zeros((B, N, C), dtype=torch.bfloat16)
+    W = torch.zeros((C, C), dtype=torch.bfloat16)
+    return cp.flarepp_mixer_cp_bwd(X, W, W, W, W, torch.zeros((H, M, D), dtype=torch.bfloat16),
+                                   torch.zeros((B, H, N, D), dtype=torch.bfloat16), stream=_Stream(),
+                                   workspace=workspace, device_check=device_check)
+
+
+def test_device_error_word_raises_when_the_workspace_is_internal(monkeypatch):
+    import pytest
+    from rank_latent_routing_flare_b200 import FlareError, Status
+    fake = _StatusLib(int(Status.ERR_SHAPE))
+    with pytest.raises(FlareError) as e:
+        _run_single_rank_bwd(monkeypatch, fake)
+    assert e.value.status == Status.ERR_SHAPE
+    assert fake.calls[-1] == ("status",)
+
+
+def test_a_caller_workspace_is_left_for_the_caller_to_check(monkeypatch):
+    fake = _StatusLib(2)
+    ws = torch.empty(256, dtype=torch.uint8)
+    _run_single_rank_bwd(monkeypatch, fake, workspace=ws)
+    assert ("status",) not in fake.calls
+    fake2 = _StatusLib(0)
+    _run_single_rank_bwd(monkeypatch, fake2, workspace=ws, device_check=True)
+    assert fake2.calls[-1] == ("status",)

@@ -17,7 +17,7 @@ import rank_latent_routing_flare_b200 as fl
 from rank_latent_routing_flare_b200 import cp
 from workloads import make_workload
 
-from .gpu_util import MAX_ABS, REL_L2, dev_bf16, host_f64, max_abs, rel_l2
+from .gpu_util import MAX_ABS, REL_L2, compare, dev_bf16, host_f64, max_abs, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -80,7 +80,7 @@ def test_emulated_ranks_match_oracle_and_agree(name, kw, R):
     for r in range(1, R):
         assert torch.equal(qxs[r], qxs[0]) and torch.equal(zs[r], zs[0]), r
     ref = oracle.forward_workload(w)
-    check(host_f64(Y), ref["Y"], f"cp Y {name} R={R}")
+    compare({"Y": host_f64(Y)}, {"Y": ref["Y"]}, lengths=w.lengths, label=f"cp Y {name} R={R}")
     check(host_f64(qxs[0]), ref["Qx"], f"cp Qx {name}")
     check(host_f64(zs[0]), ref["Z"], f"cp Z {name}")
 
@@ -117,4 +117,5 @@ def test_flare_emulated_ranks():
         assert lib.flare_cp_end(gathered.data_ptr(), Ks[r].data_ptr(), Q.data_ptr(), Ys[r].data_ptr(), B, H, N, M, D,
                                 None, r, R, 0.0, wss[r].data_ptr(), nbytes, st, None) == 0
     torch.cuda.synchronize()
-    check(host_f64(torch.cat(Ys, dim=2)), oracle.forward_workload(w)["Y"], "cp flare")
+    compare({"Y": host_f64(torch.cat(Ys, dim=2))}, {"Y": oracle.forward_workload(w)["Y"]}, lengths=w.lengths,
+            label="cp flare")

@@ -16,7 +16,7 @@ import oracle
 import rank_latent_routing_flare_b200 as fl
 from workloads import make_workload
 
-from .gpu_util import MAX_ABS, REL_L2, dev_bf16, host_f64, max_abs, rel_l2
+from .gpu_util import MAX_ABS, REL_L2, compare, dev_bf16, host_f64, max_abs, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -51,6 +51,8 @@ def test_output_projection_matches_oracle(name, kw):
     got = host_f64(out)
     ref = oracle.forward_workload(w)["Out"]
     check(got, ref, f"out {name} {kw}")
+    # token-centred part of Out = (Y_1 | ... | Y_H) W_O, as for Y (Out viewed as one head of width C)
+    compare({"Y": got[:, None]}, {"Y": ref[:, None]}, lengths=w.lengths, label=f"out {name} {kw} (centred)")
     if w.lengths is not None:
         for b, L in enumerate(w.lengths):
             assert np.all(got[b, L:] == 0), (b, L)
@@ -73,5 +75,5 @@ def test_shared_projections_match_oracle_and_separate_copies(name, kw):
     torch.cuda.synchronize()
     assert torch.equal(Y_shared.view(torch.int16), Y_copies.view(torch.int16))
     ref = oracle.forward_workload(w)
-    check(host_f64(Y_shared), ref["Y"], f"shared Y {name}")
+    compare({"Y": host_f64(Y_shared)}, {"Y": ref["Y"]}, lengths=w.lengths, label=f"shared Y {name}")
     check(host_f64(out_shared), ref["Out"], f"shared Out {name}")

@@ -17,6 +17,7 @@ from rank_latent_routing_flare_b200 import Status
 from workloads import Workload, bf16_bits_to_f64, make_workload, to_bf16_bits
 
 from .gpu_util import compare, dev_bf16, host_f64, run_gpu
+from .parity import storage_model
 
 pytestmark = pytest.mark.gpu
 
@@ -140,21 +141,6 @@ def test_workload_reduced(name, kw):
     compare(run_gpu(w), oracle.forward_workload(w), label=f"{name} {kw}")
 
 
-def storage_model(w):
-    """The oracle's own functions composed with the CUDA path's storage format:
-    K~, V~, K, V, Q(X) and Z rounded to bf16 where the kernels store them.
-    Everything else is the fp64 oracle."""
-    from workloads import bf16_bits_to_f64 as f64
-    r = lambda a: f64(to_bf16_bits(a))  # noqa: E731
-    X = f64(w.X)
-    Wk, Wv, Wks, Wvs = (f64(a) for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn))
-    Kt, Vt = r(oracle.project(X, Wks, w.H)), r(oracle.project(X, Wvs, w.H))
-    Qx = oracle.encode(f64(w.Q0), Kt, Vt, w.lengths)
-    K, V = r(oracle.project(X, Wk, w.H)), r(oracle.project(X, Wv, w.H))
-    Z = oracle.encode(r(Qx), K, V, w.lengths)
-    return {"Qx": Qx, "Z": Z, "Y": oracle.decode(K, r(Qx), r(Z), w.lengths)}
-
-
 def test_sharp_scores_match_bf16_storage_model():
     """Diagnostic with all weights ~ N(0, 16/C): encode/decode scores spread
     over tens of units and many tokens sit near ties between latents with very
@@ -168,7 +154,7 @@ def test_sharp_scores_match_bf16_storage_model():
     from .gpu_util import REL_L2, rel_l2
     w = make_workload("flarepp_n8k_sharp", N=2048, B=2)
     g = run_gpu(w)
-    model = storage_model(w)
+    model = storage_model(w, oracle)
     exact = oracle.forward_workload(w)
     assert rel_l2(g["Qx"], model["Qx"]) <= REL_L2
     storage_err = rel_l2(model["Y"], exact["Y"])
