@@ -54,10 +54,10 @@ def run_gpu(w, debug: bool = True):
     return out
 
 
-def compare(gpu: dict, ref: dict, rows=None, label="", lengths=None):
+def compare(gpu: dict, ref: dict, rows=None, label="", lengths=None, extra_rounding=None):
     """Assert the stated tolerance on Y, the bound on its token-centred part
     (bf16 and, when present, fp32) and the tolerance on the Q(X) / Z
     diagnostics; returns the measured errors."""
     if lengths is None:
         lengths = gpu.get("lengths")
-    return check(gpu, ref, rows=rows, lengths=lengths, label=label)
+    return check(gpu, ref, rows=rows, lengths=lengths, label=label, extra_rounding=extra_rounding)

@@ -132,3 +132,25 @@ def test_sampled_rows_are_centred_over_the_sample():
         check({"Y": bf16_round(Ym), "Y32": Ym}, ref, rows=rows, label="sampled token-mean")
     errs = centred_errors(ref["Y"], bf16_round(Ym)[:, :, rows], Ym[:, :, rows], None, rows)
     assert errs["Yc_rel_l2"] > errs["Yc_bound"] and errs["Yc32_rel_l2"] > CENTRED_F32
+
+
+@pytest.mark.parametrize("cid", IDS[:2] + IDS[4:5])
+def test_output_projection_bound_counts_the_intermediate_rounding(cases, cid):
+    """Out = (Y_1 | ... | Y_H) W_O from a bf16-stored Ycat: the model of the
+    CUDA path (two roundings) passes once the first rounding is counted; the
+    token-mean decoder still fails."""
+    w, ref, model = cases[cid]
+    f64 = bf16_bits_to_f64
+    Wo = f64(w.Wo)
+
+    def cat(Y):
+        return np.transpose(Y, (0, 2, 1, 3)).reshape(w.B, w.N, w.C)
+
+    out_ref = cat(ref["Y"]) @ Wo
+    extra = ((bf16_round(cat(ref["Y"])) - cat(ref["Y"])) @ Wo)[:, None]
+    out_model = bf16_round(bf16_round(cat(model["Y"])) @ Wo)
+    check({"Y": out_model[:, None]}, {"Y": out_ref[:, None]}, lengths=w.lengths, label=f"Out model {cid}",
+          extra_rounding=extra)
+    out_mean = bf16_round(bf16_round(cat(token_mean(model["Y"], w.lengths))) @ Wo)
+    errs = centred_errors(out_ref[:, None], out_mean[:, None], None, w.lengths, None, extra)
+    assert errs["Yc_rel_l2"] > errs["Yc_bound"]
