@@ -15,7 +15,13 @@ exactly K steps (max over ranks).  ``e2e`` is the same metric with every
 step's host->device copy of its inputs (pinned memory) and device->host copy
 of Y inside the timed region; the copies run on their own streams into double
 buffers, so those of neighbouring steps overlap the current step's compute.
-``roofline`` reports the dominant kernel against the exp-unit (MUFU) peak, ``cpu_baseline`` the fp64 oracle on a
+The timed steps run without events between the kernels; the per-stage times
+come from as many steps with stage events, run after the timed region.
+``roofline`` reports the dominant kernel against the exp-unit bound, from the
+ex2 and fp32-fma rates measured on the device by the library's probe: ``frac``
+(= ``frac_combined``) against the best split of the exponentials between the
+special-function unit and an FMA-pipe polynomial, ``frac_mufu_only`` against
+the special-function unit alone.  ``cpu_baseline`` is the fp64 oracle on a
 bounded sample of the same workload on this host's cores.  ``--impl
 reference`` times the oracle itself as the reference arm.
 
@@ -545,7 +551,7 @@ def main():
                     help="time the FLARE++ backward (gradients) instead of the forward; its own JSON line")
     ap.add_argument("--graph", action="store_true",
                     help="time replays of one step captured as a CUDA graph (no per-launch host cost); the "
-                         "stage times then come from as many eager steps run after the timed region")
+                         "stage times come from as many eager steps with stage events after the timed region")
     args = ap.parse_args()
     if args.warmup < 3:
         log("warm-up raised to the minimum of 3 steps")
@@ -621,7 +627,7 @@ def main():
             if graph is not None:
                 graph.replay()
             else:
-                step(stage_ev[i])
+                step()
         ev1.record(stream)
         torch.cuda.synchronize(dev)
         if world > 1:
@@ -630,11 +636,12 @@ def main():
     th_per_rank = w.B * w.H * (w.valid_tokens() // w.B if w.lengths is not None else w.N)
     value = whole_job_rate(world, th_per_rank, ms)
 
-    # per-stage device times (the timed steps; with --graph, eager steps after them)
-    if graph is not None:
-        for i in range(args.steps):
-            step(stage_ev[i])
-        torch.cuda.synchronize(dev)
+    # per-stage device times: as many steps again, after the timed region,
+    # with CUDA events between the stages (the timed steps run without them:
+    # an event between two kernels keeps the second from starting early)
+    for i in range(args.steps):
+        step(stage_ev[i])
+    torch.cuda.synchronize(dev)
     stage_ms = {s: 0.0 for s in STAGES_PP}
     for evs in stage_ev:
         for j, s in enumerate(STAGES_PP):

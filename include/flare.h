@@ -85,8 +85,8 @@ typedef enum {
   FLARE_ERR_WORKSPACE = 5,   /* workspace smaller than flare_workspace_bytes()    */
   FLARE_ERR_LAUNCH = 6,      /* CUDA error while enqueueing (no sm_100 device...) */
   FLARE_ERR_TIMEOUT = 7,     /* a device-side bounded wait expired                */
-  FLARE_ERR_UNDERFLOW = 8    /* context parallelism: a merged row's sums underflowed
-                                and could not be recomputed exactly             */
+  FLARE_ERR_UNDERFLOW = 8    /* context parallelism without the exact step: a merged
+                                row's sums underflowed and were not recomputed  */
 } flare_status;
 
 /* Variant selector for flare_workspace_bytes(). */
@@ -305,38 +305,69 @@ FLARE_API const char* flare_status_string(flare_status status);
  * the log-sum-exp rule in a fixed order, so every rank holds bitwise the
  * same Q(X) and Z.  The projections and the decoder only touch local rows.
  *
- *   FLARE++ : flarepp_cp_begin  -> all-gather -> flarepp_cp_middle
- *             -> all-gather -> flarepp_cp_end
- *   FLARE   : flare_cp_begin    -> all-gather -> flare_cp_end
+ *   FLARE++ : flarepp_cp_begin -> all-gather (P1) -> flarepp_cp_exact(0, P1)
+ *             -> all-gather (E1) -> flarepp_cp_middle(P1, E1)
+ *             -> all-gather (P2) -> flarepp_cp_exact(1, P2)
+ *             -> all-gather (E2) -> flarepp_cp_end(P2, E2)
+ *   FLARE   : flare_cp_begin -> all-gather (P) -> flare_cp_exact(P)
+ *             -> all-gather (E) -> flare_cp_end(P, E)
+ *
+ * The exact step: a row of an encoder whose fast-path sums may have lost
+ * mass to underflow (the encoder shifts each split by a norm bound, which
+ * can be far above the row's largest score) is recomputed exactly on one
+ * GPU from all keys.  Across shards no rank holds all keys, so every rank
+ * finds the same such rows in the gathered partials (the merge's own test)
+ * and writes, for them, the exact partial sums of its own tokens (max,
+ * sum, weighted values; two passes in fp32) to `exact_out`
+ * (flare_cp_exact_bytes() bytes, fp32; other rows are marked empty).  The
+ * all-gathered exact partials (E, [world][...] rank-major) let every rank's
+ * merge combine those rows exactly with the same log-sum-exp rule, so the
+ * result is exact for any split of the tokens.  The exact step does real
+ * work only for rows that need it.  Passing NULL as exact_all skips it: a
+ * row that needs it is then reported as FLARE_ERR_UNDERFLOW by
+ * flare_last_device_status.
  *
  * The phases of one rank share its workspace (flare_workspace_bytes of the
  * same variant with the shard's N) and stream; the workspace carries the
  * projections, Q(X) and Z from one phase to the next.  All ranks must call
  * with the same sizes.  With world == 1 the result equals flare_mixer_fwd /
- * flarepp_mixer_fwd.  A merged row whose sums underflowed (the case that
- * flare_mixer_fwd recomputes exactly from all keys) is reported as
- * FLARE_ERR_UNDERFLOW by flare_last_device_status when world > 1.
+ * flarepp_mixer_fwd.
  */
 FLARE_API size_t flare_cp_partials_bytes(int B, int H, int N, int M, int D);
+FLARE_API size_t flare_cp_exact_bytes(int B, int H, int M, int D);
 
 FLARE_API flare_status flarepp_cp_begin(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
                                         const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0,
                                         int B, int N, int C, int H, int M, int D, const int32_t* lengths, int rank,
                                         int world, float scale, void* workspace, size_t workspace_bytes,
                                         void* stream, float* partials);
-FLARE_API flare_status flarepp_cp_middle(const float* partials_all, int B, int N, int C, int H, int M, int D,
-                                         const int32_t* lengths, int rank, int world, float scale, void* workspace,
-                                         size_t workspace_bytes, void* stream, float* partials, float* Qx_out);
-FLARE_API flare_status flarepp_cp_end(const float* partials_all, flare_bf16* Y, int B, int N, int C, int H, int M,
-                                      int D, const int32_t* lengths, int rank, int world, float scale,
-                                      void* workspace, size_t workspace_bytes, void* stream, float* Z_out);
+/* pass 0: the query synthesis (after flarepp_cp_begin); pass 1: the encode
+ * (after flarepp_cp_middle).  The weight pointers only tell the shared-
+ * projection variant apart, as in flarepp_cp_begin; Q0 is read in pass 0. */
+FLARE_API flare_status flarepp_cp_exact(int pass, const float* partials_all, const flare_bf16* Wk,
+                                        const flare_bf16* Wv, const flare_bf16* Wk_syn, const flare_bf16* Wv_syn,
+                                        const flare_bf16* Q0, int B, int N, int C, int H, int M, int D,
+                                        const int32_t* lengths, int rank, int world, float scale, void* workspace,
+                                        size_t workspace_bytes, void* stream, float* exact_out);
+FLARE_API flare_status flarepp_cp_middle(const float* partials_all, const float* exact_all, int B, int N, int C,
+                                         int H, int M, int D, const int32_t* lengths, int rank, int world,
+                                         float scale, void* workspace, size_t workspace_bytes, void* stream,
+                                         float* partials, float* Qx_out);
+FLARE_API flare_status flarepp_cp_end(const float* partials_all, const float* exact_all, flare_bf16* Y, int B,
+                                      int N, int C, int H, int M, int D, const int32_t* lengths, int rank, int world,
+                                      float scale, void* workspace, size_t workspace_bytes, void* stream,
+                                      float* Z_out);
 FLARE_API flare_status flare_cp_begin(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, int B, int H,
                                       int N, int M, int D, const int32_t* lengths, int rank, int world, float scale,
                                       void* workspace, size_t workspace_bytes, void* stream, float* partials);
-FLARE_API flare_status flare_cp_end(const float* partials_all, const flare_bf16* K, const flare_bf16* Q,
-                                    flare_bf16* Y, int B, int H, int N, int M, int D, const int32_t* lengths,
-                                    int rank, int world, float scale, void* workspace, size_t workspace_bytes,
-                                    void* stream, float* Z_out);
+FLARE_API flare_status flare_cp_exact(const float* partials_all, const flare_bf16* K, const flare_bf16* V,
+                                      const flare_bf16* Q, int B, int H, int N, int M, int D,
+                                      const int32_t* lengths, int rank, int world, float scale, void* workspace,
+                                      size_t workspace_bytes, void* stream, float* exact_out);
+FLARE_API flare_status flare_cp_end(const float* partials_all, const float* exact_all, const flare_bf16* K,
+                                    const flare_bf16* Q, flare_bf16* Y, int B, int H, int N, int M, int D,
+                                    const int32_t* lengths, int rank, int world, float scale, void* workspace,
+                                    size_t workspace_bytes, void* stream, float* Z_out);
 
 /*
  * FLARE mixer forward for callers that cannot allocate device memory.

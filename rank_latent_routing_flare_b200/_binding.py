@@ -76,12 +76,16 @@ def load_library(build_if_missing: bool = True):
         lib.flare_static_last_device_status.restype = i
         lib.flare_cp_partials_bytes.restype = sz
         lib.flare_cp_partials_bytes.argtypes = [i, i, i, i, i]
+        lib.flare_cp_exact_bytes.restype = sz
+        lib.flare_cp_exact_bytes.argtypes = [i, i, i, i]
         for name, args in (
                 ("flarepp_cp_begin", [vp] * 6 + [i] * 6 + [vp, i, i, f, vp, sz, vp, vp]),
-                ("flarepp_cp_middle", [vp] + [i] * 6 + [vp, i, i, f, vp, sz, vp, vp, vp]),
-                ("flarepp_cp_end", [vp, vp] + [i] * 6 + [vp, i, i, f, vp, sz, vp, vp]),
+                ("flarepp_cp_exact", [i] + [vp] * 6 + [i] * 6 + [vp, i, i, f, vp, sz, vp, vp]),
+                ("flarepp_cp_middle", [vp, vp] + [i] * 6 + [vp, i, i, f, vp, sz, vp, vp, vp]),
+                ("flarepp_cp_end", [vp, vp, vp] + [i] * 6 + [vp, i, i, f, vp, sz, vp, vp]),
                 ("flare_cp_begin", [vp] * 3 + [i] * 5 + [vp, i, i, f, vp, sz, vp, vp]),
-                ("flare_cp_end", [vp] * 4 + [i] * 5 + [vp, i, i, f, vp, sz, vp, vp])):
+                ("flare_cp_exact", [vp] * 4 + [i] * 5 + [vp, i, i, f, vp, sz, vp, vp]),
+                ("flare_cp_end", [vp] * 5 + [i] * 5 + [vp, i, i, f, vp, sz, vp, vp])):
             fn = getattr(lib, name)
             fn.restype = i
             fn.argtypes = args

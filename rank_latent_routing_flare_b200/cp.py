@@ -8,7 +8,10 @@ and the decoder are pointwise in the tokens and stay local; each encoder pass
 one exchange: every rank computes per-split partial sums of its shard, the
 partials of all ranks are all-gathered, and every rank merges them with the
 log-sum-exp rule in the same fixed order, so all ranks hold bitwise the same
-Q(X) and Z.
+Q(X) and Z.  After each gather a second, small one carries, for the rows
+whose fast-path sums may have lost mass to underflow (none, usually), every
+rank's exact partial sums of its own tokens, so the merge stays exact for any
+split of the tokens.
 
 All arithmetic runs in the CUDA library (the ``*_cp_*`` entry points of
 include/flare.h); this module only allocates the buffers and moves the
@@ -61,6 +64,13 @@ def partials_numel(B: int, H: int, N: int, M: int, D: int) -> int:
     return nbytes // 4
 
 
+def exact_numel(B: int, H: int, M: int, D: int) -> int:
+    nbytes = b.load_library().flare_cp_exact_bytes(B, H, M, D)
+    if nbytes == 0:
+        raise ValueError("unsupported sizes")
+    return nbytes // 4
+
+
 def _status(st, where):
     if st != 0:
         raise b.FlareError(st, where)
@@ -100,14 +110,22 @@ def flarepp_mixer_cp_fwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, lengths=None, group=None
         ws.record_stream(stream)
     st = b._stream_ptr(stream, X.device)
     part = torch.empty(partials_numel(B, H, N, M, D), dtype=torch.float32, device=X.device)
+    exact = torch.empty(exact_numel(B, H, M, D), dtype=torch.float32, device=X.device)
+    weights = [b._ptr(t) for t in (Wk, Wv, Wk_syn, Wv_syn, Q0)]
     common = (B, N, C, H, M, D, b._ptr(lengths), rank, world, float(scale), b._ptr(ws), ws.numel(), st)
-    _status(lib.flarepp_cp_begin(b._ptr(X), b._ptr(Wk), b._ptr(Wv), b._ptr(Wk_syn), b._ptr(Wv_syn), b._ptr(Q0),
-                                 *common, b._ptr(part)), "flarepp_cp_begin")
+    _status(lib.flarepp_cp_begin(b._ptr(X), *weights, *common, b._ptr(part)), "flarepp_cp_begin")
     gathered = allgather_partials(part, world, group, stream)
+    _status(lib.flarepp_cp_exact(0, b._ptr(gathered), *weights, *common, b._ptr(exact)), "flarepp_cp_exact(0)")
+    gathered_exact = allgather_partials(exact, world, group, stream)
     part2 = torch.empty_like(part)
-    _status(lib.flarepp_cp_middle(b._ptr(gathered), *common, b._ptr(part2), b._ptr(Qx_out)), "flarepp_cp_middle")
+    _status(lib.flarepp_cp_middle(b._ptr(gathered), b._ptr(gathered_exact), *common, b._ptr(part2),
+                                  b._ptr(Qx_out)), "flarepp_cp_middle")
     gathered = allgather_partials(part2, world, group, stream)
-    _status(lib.flarepp_cp_end(b._ptr(gathered), b._ptr(Y), *common, b._ptr(Z_out)), "flarepp_cp_end")
+    exact2 = torch.empty_like(exact)
+    _status(lib.flarepp_cp_exact(1, b._ptr(gathered), *weights, *common, b._ptr(exact2)), "flarepp_cp_exact(1)")
+    gathered_exact = allgather_partials(exact2, world, group, stream)
+    _status(lib.flarepp_cp_end(b._ptr(gathered), b._ptr(gathered_exact), b._ptr(Y), *common, b._ptr(Z_out)),
+            "flarepp_cp_end")
     _device_status(device_check, workspace is not None, ws, stream, "flarepp_mixer_cp_fwd")
     return Y
 
@@ -129,11 +147,15 @@ def flare_mixer_cp_fwd(K, V, Q, lengths=None, group=None, scale: float = 0.0, Y=
         ws.record_stream(stream)
     st = b._stream_ptr(stream, K.device)
     part = torch.empty(partials_numel(B, H, N, M, D), dtype=torch.float32, device=K.device)
+    exact = torch.empty(exact_numel(B, H, M, D), dtype=torch.float32, device=K.device)
     common = (B, H, N, M, D, b._ptr(lengths), rank, world, float(scale), b._ptr(ws), ws.numel(), st)
     _status(lib.flare_cp_begin(b._ptr(K), b._ptr(V), b._ptr(Q), *common, b._ptr(part)), "flare_cp_begin")
     gathered = allgather_partials(part, world, group, stream)
-    _status(lib.flare_cp_end(b._ptr(gathered), b._ptr(K), b._ptr(Q), b._ptr(Y), *common, b._ptr(Z_out)),
-            "flare_cp_end")
+    _status(lib.flare_cp_exact(b._ptr(gathered), b._ptr(K), b._ptr(V), b._ptr(Q), *common, b._ptr(exact)),
+            "flare_cp_exact")
+    gathered_exact = allgather_partials(exact, world, group, stream)
+    _status(lib.flare_cp_end(b._ptr(gathered), b._ptr(gathered_exact), b._ptr(K), b._ptr(Q), b._ptr(Y), *common,
+                             b._ptr(Z_out)), "flare_cp_end")
     _device_status(device_check, workspace is not None, ws, stream, "flare_mixer_cp_fwd")
     return Y
 

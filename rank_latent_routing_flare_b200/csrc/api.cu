@@ -73,18 +73,17 @@ CUtensorMapSwizzle row_swizzle(int D) { return D == 16 ? CU_TENSOR_MAP_SWIZZLE_3
 
 // Number of token splits of the encoder.  Cost model: the CTAs run in
 // waves of `slots` (CTAs resident on the whole GPU); a wave lasts as long as
-// one split (its tiles plus a fixed set-up cost worth kSplitSetupTiles
-// tiles).  Depends on the sizes only, so a given problem always uses the same
-// split count (and gives the same bits).
-constexpr long kSplitSetupTiles = 8;
-int choose_splits(long units, long ntiles, long slots) {
+// one split (its tiles plus a fixed set-up cost worth setup_tiles tiles).
+// Depends on the sizes only, so a given problem always uses the same split
+// count (and gives the same bits).
+int choose_splits(long units, long ntiles, long slots, long setup_tiles) {
   const long smax = std::max(1L, std::min(ntiles, 1024L));
   int best = 1;
   long best_cost = -1;
   for (long s = 1; s <= smax; ++s) {
     const long tps = cdiv(ntiles, s);
     if (s > 1 && cdiv(ntiles, tps) < s) continue;  // same tiling as a smaller s
-    const long cost = cdiv(units * s, slots) * (tps + kSplitSetupTiles);
+    const long cost = cdiv(units * s, slots) * (tps + setup_tiles);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best = static_cast<int>(s);
@@ -99,7 +98,10 @@ Plan make_plan(int variant, long B, long H, long N, long M, long D) {
   const long BH = B * H;
   const long ntiles = cdiv(N, enc_tile(static_cast<int>(D)));
   p.LB = static_cast<int>(cdiv(M, kLatBlock));
-  p.S = choose_splits(BH * p.LB, ntiles, static_cast<long>(kNumSM) * enc_ctas_per_sm(static_cast<int>(D)));
+  // an encoder CTA's set-up (TMEM allocation, barriers, the first tiles of
+  // its pipeline) costs about as much as 384 tokens of work
+  p.S = choose_splits(BH * p.LB, ntiles, static_cast<long>(kNumSM) * enc_ctas_per_sm(static_cast<int>(D)),
+                      cdiv(384, enc_tile(static_cast<int>(D))));
   p.tps = static_cast<int>(cdiv(ntiles, p.S));
   p.S = static_cast<int>(cdiv(ntiles, p.tps));
   const long dtiles = cdiv(N, kDecTile);
@@ -161,7 +163,7 @@ float resolve_scale(float scale, int D) { return scale > 0.f ? scale : 1.0f / st
 flare_status run_encode_partials(const Plan& pl, uint8_t* ws, const void* q, int q_per_batch, const void* k,
                                  const void* v, const float* knorm, float* part, int B, int H, int N, int M, int D,
                                  const int32_t* lengths, int tok_offset, int n_global, float scale, cudaStream_t st,
-                                 void* const* ev, int ev0) {
+                                 void* const* ev, int ev0, bool pdl) {
   const long BH = static_cast<long>(B) * H;
   const long G = q_per_batch ? BH : H;
   CUtensorMap tq, tk, tv;
@@ -181,17 +183,18 @@ flare_status run_encode_partials(const Plan& pl, uint8_t* ws, const void* q, int
   ep.part = part;
   ep.err = reinterpret_cast<uint32_t*>(ws + pl.off_err);
   ep.timeout_ns = wait_timeout_ns();
-  if (launch_encode(tq, tk, tv, ep, st) != cudaSuccess || !record(ev, ev0, st)) return FLARE_ERR_LAUNCH;
+  if (launch_encode(tq, tk, tv, ep, st, pdl) != cudaSuccess || !record(ev, ev0, st)) return FLARE_ERR_LAUNCH;
   return FLARE_OK;
 }
 
 // Merge of the partials of R shards ([R][B*H][S][M][D+2], rank-major) into
 // out32/out16 ([B*H][M][D]).  With R == 1, q/k/v serve the exact
 // recomputation of rows whose sums underflowed.
-flare_status run_merge(const Plan& pl, uint8_t* ws, const float* part, int R, const void* q, int q_per_batch,
-                       const void* k, const void* v, float* out32, uint16_t* out16, int B, int H, int N, int M,
-                       int D, const int32_t* lengths, float scale, cudaStream_t st, void* const* ev, int ev_i,
-                       bool allow_exact = true) {
+// exact: every shard's exact partials of the rows that need them
+// ([R][B*H*M][D+2], context parallelism), or nullptr.
+MergeParams merge_params(const Plan& pl, uint8_t* ws, const float* part, int R, const void* q, int q_per_batch,
+                         const void* k, const void* v, float* out32, uint16_t* out16, int B, int H, int N, int M,
+                         int D, const int32_t* lengths, float scale, bool allow_exact, const float* exact) {
   MergeParams mp{};
   mp.B = B; mp.H = H; mp.N = N; mp.M = M; mp.D = D;
   mp.q_per_batch = q_per_batch;
@@ -208,25 +211,46 @@ flare_status run_merge(const Plan& pl, uint8_t* ws, const float* part, int R, co
   mp.v = static_cast<const uint16_t*>(v);
   mp.out_f32 = out32;
   mp.out_bf16 = out16;
-  if (launch_merge(mp, st) != cudaSuccess || !record(ev, ev_i, st)) return FLARE_ERR_LAUNCH;
+  mp.fix = exact;
+  mp.fix_rank_stride = static_cast<size_t>(B) * H * M * (D + 2);
+  return mp;
+}
+
+flare_status run_merge(const Plan& pl, uint8_t* ws, const float* part, int R, const void* q, int q_per_batch,
+                       const void* k, const void* v, float* out32, uint16_t* out16, int B, int H, int N, int M,
+                       int D, const int32_t* lengths, float scale, cudaStream_t st, void* const* ev, int ev_i,
+                       bool pdl, bool allow_exact = true, const float* exact = nullptr) {
+  const MergeParams mp =
+      merge_params(pl, ws, part, R, q, q_per_batch, k, v, out32, out16, B, H, N, M, D, lengths, scale, allow_exact, exact);
+  if (launch_merge(mp, st, pdl) != cudaSuccess || !record(ev, ev_i, st)) return FLARE_ERR_LAUNCH;
   return FLARE_OK;
+}
+
+// Context parallelism: this shard's exact partials (out, [B*H*M][D+2]) of
+// the rows whose merge of the gathered partials `part` needs them.
+flare_status run_cp_exact(const Plan& pl, uint8_t* ws, const float* part, int R, int rank, const void* q,
+                          int q_per_batch, const void* k, const void* v, int B, int H, int N, int M, int D,
+                          const int32_t* lengths, float scale, cudaStream_t st, float* out) {
+  const MergeParams mp = merge_params(pl, ws, part, R, q, q_per_batch, k, v, nullptr, nullptr, B, H, N, M, D,
+                                      lengths, scale, false, nullptr);
+  return launch_cp_exact(mp, rank, out, st) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
 
 // Encoder pass + merge on one GPU (the whole sequence).
 flare_status run_encode(const Plan& pl, uint8_t* ws, const void* q, int q_per_batch, const void* k, const void* v,
                         const float* knorm, float* out32, uint16_t* out16, int B, int H, int N, int M, int D,
-                        const int32_t* lengths, float scale, cudaStream_t st, void* const* ev, int ev0) {
+                        const int32_t* lengths, float scale, cudaStream_t st, void* const* ev, int ev0, bool pdl) {
   float* part = reinterpret_cast<float*>(ws + pl.off_part);
   flare_status r = run_encode_partials(pl, ws, q, q_per_batch, k, v, knorm, part, B, H, N, M, D, lengths, 0, N,
-                                       scale, st, ev, ev0);
+                                       scale, st, ev, ev0, pdl);
   if (r != FLARE_OK) return r;
   return run_merge(pl, ws, part, 1, q, q_per_batch, k, v, out32, out16, B, H, N, M, D, lengths, scale, st, ev,
-                   ev0 + 1);
+                   ev0 + 1, pdl);
 }
 
 flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_batch, const uint16_t* z16,
                         const void* k, void* y, int y_token_major, int B, int H, int N, int M, int D,
-                        const int32_t* lengths, float scale, cudaStream_t st, int tok_offset = 0,
+                        const int32_t* lengths, float scale, cudaStream_t st, bool pdl, int tok_offset = 0,
                         int n_global = -1, float* y_f32 = nullptr) {
   const long BH = static_cast<long>(B) * H;
   const long G = q_per_batch ? BH : H;
@@ -254,7 +278,7 @@ flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
   dp.fb_count = reinterpret_cast<uint32_t*>(ws + pl.off_err) + 1;
   dp.fb_list = reinterpret_cast<uint64_t*>(ws + pl.off_fb);
   dp.timeout_ns = wait_timeout_ns();
-  if (launch_decode(tq, tz, tk, dp, st) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  if (launch_decode(tq, tz, tk, dp, st, pdl) != cudaSuccess) return FLARE_ERR_LAUNCH;
   return FLARE_OK;
 }
 
@@ -346,9 +370,12 @@ flare_status flare_fwd(const flare_bf16* K, const flare_bf16* V, const flare_bf1
   if (launch_knorm(kp, s) != cudaSuccess || !record(stage_events, 1, s)) return FLARE_ERR_LAUNCH;
   float* z32 = Z_out ? Z_out : reinterpret_cast<float*>(ws + pl.off_z32);
   uint16_t* z16 = reinterpret_cast<uint16_t*>(ws + pl.off_z16);
-  st = run_encode(pl, ws, Q, 0, K, V, kp.knorm, z32, z16, B, H, N, M, D, lengths, sc, s, stage_events, 2);
+  // kernels after the first start early (programmatic launch) unless stage
+  // events sit between them
+  const bool pdl = stage_events == nullptr;
+  st = run_encode(pl, ws, Q, 0, K, V, kp.knorm, z32, z16, B, H, N, M, D, lengths, sc, s, stage_events, 2, pdl);
   if (st != FLARE_OK) return st;
-  st = run_decode(pl, ws, Q, 0, z16, K, Y, 0, B, H, N, M, D, lengths, sc, s, 0, -1, Y_f32_out);
+  st = run_decode(pl, ws, Q, 0, z16, K, Y, 0, B, H, N, M, D, lengths, sc, s, pdl, 0, -1, Y_f32_out);
   if (st != FLARE_OK) return st;
   return record(stage_events, 4, s) ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
@@ -405,7 +432,7 @@ flare_status check_flarepp(const void* X, const void* Wk, const void* Wv, const 
 // ([B][H][N][D], or [B][N][C] when token_major), key norms where given.
 flare_status run_project(const Plan& pl, uint8_t* ws, const CUtensorMap& tx, const CUtensorMap (&tw)[4], int n_proj,
                          int token_major, uint16_t* const (&out)[4], float* const (&knorm)[4], int B, int N, int C,
-                         int H, int D, cudaStream_t s) {
+                         int H, int D, cudaStream_t s, bool pdl) {
   ProjParams pp{};
   pp.B = B; pp.N = N; pp.C = C; pp.H = H; pp.D = D;
   pp.tiles_per_b = static_cast<int>(cdiv(N, kProjTile));
@@ -421,7 +448,7 @@ flare_status run_project(const Plan& pl, uint8_t* ws, const CUtensorMap& tx, con
   }
   pp.err = reinterpret_cast<uint32_t*>(ws + pl.off_err);
   pp.timeout_ns = wait_timeout_ns();
-  return launch_project(tx, tw, pp, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+  return launch_project(tx, tw, pp, s, pdl) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
 
 
@@ -457,7 +484,7 @@ flare_status flarepp_project(const Plan& pl, const flare_bf16* X, const flare_bf
   if (!record(stage_events, 0, s)) return FLARE_ERR_LAUNCH;
   uint16_t* const outs[4] = {kt, vt, kk, vv};
   float* const norms[4] = {kn_syn, nullptr, kn, nullptr};
-  flare_status st = run_project(pl, ws, tx, tw, shared ? 2 : 4, 0, outs, norms, B, N, C, H, D, s);
+  flare_status st = run_project(pl, ws, tx, tw, shared ? 2 : 4, 0, outs, norms, B, N, C, H, D, s, false);
   if (st != FLARE_OK || !record(stage_events, 1, s)) return FLARE_ERR_LAUNCH;
   *pr = Projected{kt, vt, kk, vv, kn_syn, kn};
   return FLARE_OK;
@@ -477,18 +504,21 @@ flare_status flarepp_run(const Plan& pl, const flare_bf16* X, const flare_bf16* 
   uint16_t *kt = pr.kt, *vt = pr.vt, *kk = pr.kk, *vv = pr.vv;
   float *kn_syn = pr.kn_syn, *kn = pr.kn;
 
+  // kernels after the first start early (programmatic launch) unless stage
+  // events sit between them
+  const bool pdl = stage_events == nullptr;
   // eq. 8: query synthesis with the learned seeds
   float* qx32 = Qx_out ? Qx_out : reinterpret_cast<float*>(ws + pl.off_qx32);
   uint16_t* qx16 = reinterpret_cast<uint16_t*>(ws + pl.off_qx16);
-  st = run_encode(pl, ws, Q0, 0, kt, vt, kn_syn, qx32, qx16, B, H, N, M, D, lengths, sc, s, stage_events, 2);
+  st = run_encode(pl, ws, Q0, 0, kt, vt, kn_syn, qx32, qx16, B, H, N, M, D, lengths, sc, s, stage_events, 2, pdl);
   if (st != FLARE_OK) return st;
   // eq. 10: encode with the synthesised queries
   float* z32 = Z_out ? Z_out : reinterpret_cast<float*>(ws + pl.off_z32);
   uint16_t* z16 = reinterpret_cast<uint16_t*>(ws + pl.off_z16);
-  st = run_encode(pl, ws, qx16, 1, kk, vv, kn, z32, z16, B, H, N, M, D, lengths, sc, s, stage_events, 4);
+  st = run_encode(pl, ws, qx16, 1, kk, vv, kn, z32, z16, B, H, N, M, D, lengths, sc, s, stage_events, 4, pdl);
   if (st != FLARE_OK) return st;
   // eq. 11: decode
-  st = run_decode(pl, ws, qx16, 1, z16, kk, Y, y_token_major, B, H, N, M, D, lengths, sc, s, 0, -1, Y_f32_out);
+  st = run_decode(pl, ws, qx16, 1, z16, kk, Y, y_token_major, B, H, N, M, D, lengths, sc, s, pdl, 0, -1, Y_f32_out);
   if (st != FLARE_OK) return st;
   return record(stage_events, 6, s) ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
@@ -556,7 +586,7 @@ flare_status flarepp_mixer_out_fwd(const flare_bf16* X, const flare_bf16* Wk, co
     if (!map2d(&two[i], Wo, C, C, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return FLARE_ERR_LAUNCH;
   uint16_t* const outs[4] = {Out, nullptr, nullptr, nullptr};
   float* const norms[4] = {nullptr, nullptr, nullptr, nullptr};
-  return run_project(pl, ws, ty, two, 1, 1, outs, norms, B, N, C, H, D, s);
+  return run_project(pl, ws, ty, two, 1, 1, outs, norms, B, N, C, H, D, s, true);
 }
 
 flare_status flarepp_mixer_fwd(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
@@ -576,6 +606,11 @@ size_t flare_cp_partials_bytes(int B, int H, int N, int M, int D) {
   if (check_common(B, H, N, M, D) != FLARE_OK) return 0;
   const Plan pl = make_plan(FLARE_VARIANT_FLARE, B, H, N, M, D);
   return static_cast<size_t>(B) * H * pl.S * M * (D + 2) * sizeof(float);
+}
+
+size_t flare_cp_exact_bytes(int B, int H, int M, int D) {
+  if (check_common(B, H, 1, M, D) != FLARE_OK) return 0;
+  return static_cast<size_t>(B) * H * M * (D + 2) * sizeof(float);
 }
 
 }  // extern "C"
@@ -612,18 +647,19 @@ flare_status flarepp_cp_begin(const flare_bf16* X, const flare_bf16* Wk, const f
     return st;
   // eq. 8 on the local shard: the synthesis partials
   return run_encode_partials(pl, ws, Q0, 0, pr.kt, pr.vt, pr.kn_syn, partials, B, H, N, M, D, lengths, rank * N,
-                             world * N, resolve_scale(scale, D), s, nullptr, 0);
+                             world * N, resolve_scale(scale, D), s, nullptr, 0, true);
 }
 
-flare_status flarepp_cp_middle(const float* partials_all, int B, int N, int C, int H, int M, int D,
-                               const int32_t* lengths, int rank, int world, float scale, void* workspace,
+flare_status flarepp_cp_middle(const float* partials_all, const float* exact_all, int B, int N, int C, int H, int M,
+                               int D, const int32_t* lengths, int rank, int world, float scale, void* workspace,
                                size_t workspace_bytes, void* stream, float* partials, float* Qx_out) {
   if (!partials_all || !workspace) return FLARE_ERR_NULL;
   flare_status st = check_common(B, H, N, M, D);
   if (st != FLARE_OK) return st;
   if (C != H * D || C % 64 != 0 || C > 256) return C != H * D ? FLARE_ERR_SHAPE : FLARE_ERR_UNSUPPORTED;
   if ((st = check_cp(N, rank, world, partials)) != FLARE_OK) return st;
-  if (!aligned16(partials_all) || !aligned16(lengths) || !aligned16(Qx_out)) return FLARE_ERR_ALIGN;
+  if (!aligned16(partials_all) || !aligned16(exact_all) || !aligned16(lengths) || !aligned16(Qx_out))
+    return FLARE_ERR_ALIGN;
   const Plan pl = make_plan(FLARE_VARIANT_FLAREPP, B, H, N, M, D);
   if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -633,22 +669,22 @@ flare_status flarepp_cp_middle(const float* partials_all, int B, int N, int C, i
   uint16_t* qx16 = reinterpret_cast<uint16_t*>(ws + pl.off_qx16);
   // Q(X): every rank merges the same partials in the same order
   st = run_merge(pl, ws, partials_all, world, nullptr, 0, nullptr, nullptr, qx32, qx16, B, H, N, M, D, lengths, sc, s,
-                 nullptr, 0, false);
+                 nullptr, 0, false, false, exact_all);
   if (st != FLARE_OK) return st;
   // eq. 10 on the local shard: the encode partials
   return run_encode_partials(pl, ws, qx16, 1, ws + pl.off_kp, ws + pl.off_vp, reinterpret_cast<float*>(ws + pl.off_kn),
-                             partials, B, H, N, M, D, lengths, rank * N, world * N, sc, s, nullptr, 0);
+                             partials, B, H, N, M, D, lengths, rank * N, world * N, sc, s, nullptr, 0, true);
 }
 
-flare_status flarepp_cp_end(const float* partials_all, flare_bf16* Y, int B, int N, int C, int H, int M, int D,
-                            const int32_t* lengths, int rank, int world, float scale, void* workspace,
-                            size_t workspace_bytes, void* stream, float* Z_out) {
+flare_status flarepp_cp_end(const float* partials_all, const float* exact_all, flare_bf16* Y, int B, int N, int C,
+                            int H, int M, int D, const int32_t* lengths, int rank, int world, float scale,
+                            void* workspace, size_t workspace_bytes, void* stream, float* Z_out) {
   if (!partials_all || !Y || !workspace) return FLARE_ERR_NULL;
   flare_status st = check_common(B, H, N, M, D);
   if (st != FLARE_OK) return st;
   if (C != H * D || C % 64 != 0 || C > 256) return C != H * D ? FLARE_ERR_SHAPE : FLARE_ERR_UNSUPPORTED;
   if ((st = check_cp(N, rank, world, partials_all)) != FLARE_OK) return st;
-  if (!aligned16(Y) || !aligned16(lengths) || !aligned16(Z_out)) return FLARE_ERR_ALIGN;
+  if (!aligned16(Y) || !aligned16(exact_all) || !aligned16(lengths) || !aligned16(Z_out)) return FLARE_ERR_ALIGN;
   const Plan pl = make_plan(FLARE_VARIANT_FLAREPP, B, H, N, M, D);
   if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -657,11 +693,52 @@ flare_status flarepp_cp_end(const float* partials_all, flare_bf16* Y, int B, int
   float* z32 = Z_out ? Z_out : reinterpret_cast<float*>(ws + pl.off_z32);
   uint16_t* z16 = reinterpret_cast<uint16_t*>(ws + pl.off_z16);
   st = run_merge(pl, ws, partials_all, world, nullptr, 0, nullptr, nullptr, z32, z16, B, H, N, M, D, lengths, sc, s,
-                 nullptr, 0, false);
+                 nullptr, 0, false, false, exact_all);
   if (st != FLARE_OK) return st;
   // eq. 11 on the local shard
-  return run_decode(pl, ws, ws + pl.off_qx16, 1, z16, ws + pl.off_kp, Y, 0, B, H, N, M, D, lengths, sc, s, rank * N,
-                    world * N);
+  return run_decode(pl, ws, ws + pl.off_qx16, 1, z16, ws + pl.off_kp, Y, 0, B, H, N, M, D, lengths, sc, s, true,
+                    rank * N, world * N);
+}
+
+flare_status flarepp_cp_exact(int pass, const float* partials_all, const flare_bf16* Wk, const flare_bf16* Wv,
+                              const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0, int B, int N,
+                              int C, int H, int M, int D, const int32_t* lengths, int rank, int world, float scale,
+                              void* workspace, size_t workspace_bytes, void* stream, float* exact_out) {
+  if (pass != 0 && pass != 1) return FLARE_ERR_SHAPE;
+  if (!partials_all || !exact_out || !workspace || !Wk || !Wv || !Wk_syn || !Wv_syn || !Q0) return FLARE_ERR_NULL;
+  flare_status st = check_common(B, H, N, M, D);
+  if (st != FLARE_OK) return st;
+  if (C != H * D || C % 64 != 0 || C > 256) return C != H * D ? FLARE_ERR_SHAPE : FLARE_ERR_UNSUPPORTED;
+  if ((st = check_cp(N, rank, world, partials_all)) != FLARE_OK) return st;
+  if (!aligned16(exact_out) || !aligned16(lengths) || !aligned16(Q0) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FLARE_ERR_ALIGN;
+  const Plan pl = make_plan(FLARE_VARIANT_FLAREPP, B, H, N, M, D);
+  if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const bool shared = Wk_syn == Wk && Wv_syn == Wv;  // the synthesis used K and V (as in flarepp_cp_begin)
+  if (pass == 0)
+    return run_cp_exact(pl, ws, partials_all, world, rank, Q0, 0, ws + (shared ? pl.off_kp : pl.off_kt),
+                        ws + (shared ? pl.off_vp : pl.off_vt), B, H, N, M, D, lengths, resolve_scale(scale, D),
+                        static_cast<cudaStream_t>(stream), exact_out);
+  return run_cp_exact(pl, ws, partials_all, world, rank, ws + pl.off_qx16, 1, ws + pl.off_kp, ws + pl.off_vp, B, H, N,
+                      M, D, lengths, resolve_scale(scale, D), static_cast<cudaStream_t>(stream), exact_out);
+}
+
+flare_status flare_cp_exact(const float* partials_all, const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q,
+                            int B, int H, int N, int M, int D, const int32_t* lengths, int rank, int world,
+                            float scale, void* workspace, size_t workspace_bytes, void* stream, float* exact_out) {
+  if (!partials_all || !exact_out || !workspace || !K || !V || !Q) return FLARE_ERR_NULL;
+  flare_status st = check_common(B, H, N, M, D);
+  if (st != FLARE_OK) return st;
+  if ((st = check_cp(N, rank, world, partials_all)) != FLARE_OK) return st;
+  if (!aligned16(exact_out) || !aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(lengths) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FLARE_ERR_ALIGN;
+  const Plan pl = make_plan(FLARE_VARIANT_FLARE, B, H, N, M, D);
+  if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
+  return run_cp_exact(pl, static_cast<uint8_t*>(workspace), partials_all, world, rank, Q, 0, K, V, B, H, N, M, D,
+                      lengths, resolve_scale(scale, D), static_cast<cudaStream_t>(stream), exact_out);
 }
 
 flare_status flare_cp_begin(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, int B, int H, int N, int M,
@@ -682,17 +759,19 @@ flare_status flare_cp_begin(const flare_bf16* K, const flare_bf16* V, const flar
   KnormParams kp{B * H, N, D, pl.G32, reinterpret_cast<const uint16_t*>(K), reinterpret_cast<float*>(ws + pl.off_kn)};
   if (launch_knorm(kp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   return run_encode_partials(pl, ws, Q, 0, K, V, kp.knorm, partials, B, H, N, M, D, lengths, rank * N, world * N,
-                             resolve_scale(scale, D), s, nullptr, 0);
+                             resolve_scale(scale, D), s, nullptr, 0, true);
 }
 
-flare_status flare_cp_end(const float* partials_all, const flare_bf16* K, const flare_bf16* Q, flare_bf16* Y, int B,
-                          int H, int N, int M, int D, const int32_t* lengths, int rank, int world, float scale,
-                          void* workspace, size_t workspace_bytes, void* stream, float* Z_out) {
+flare_status flare_cp_end(const float* partials_all, const float* exact_all, const flare_bf16* K, const flare_bf16* Q,
+                          flare_bf16* Y, int B, int H, int N, int M, int D, const int32_t* lengths, int rank, int world,
+                          float scale, void* workspace, size_t workspace_bytes, void* stream, float* Z_out) {
   if (!partials_all || !K || !Q || !Y || !workspace) return FLARE_ERR_NULL;
   flare_status st = check_common(B, H, N, M, D);
   if (st != FLARE_OK) return st;
   if ((st = check_cp(N, rank, world, partials_all)) != FLARE_OK) return st;
-  if (!aligned16(K) || !aligned16(Q) || !aligned16(Y) || !aligned16(lengths) || !aligned16(Z_out)) return FLARE_ERR_ALIGN;
+  if (!aligned16(K) || !aligned16(Q) || !aligned16(Y) || !aligned16(exact_all) || !aligned16(lengths) ||
+      !aligned16(Z_out))
+    return FLARE_ERR_ALIGN;
   const Plan pl = make_plan(FLARE_VARIANT_FLARE, B, H, N, M, D);
   if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -701,9 +780,9 @@ flare_status flare_cp_end(const float* partials_all, const flare_bf16* K, const 
   float* z32 = Z_out ? Z_out : reinterpret_cast<float*>(ws + pl.off_z32);
   uint16_t* z16 = reinterpret_cast<uint16_t*>(ws + pl.off_z16);
   st = run_merge(pl, ws, partials_all, world, nullptr, 0, nullptr, nullptr, z32, z16, B, H, N, M, D, lengths, sc, s,
-                 nullptr, 0, false);
+                 nullptr, 0, false, false, exact_all);
   if (st != FLARE_OK) return st;
-  return run_decode(pl, ws, Q, 0, z16, K, Y, 0, B, H, N, M, D, lengths, sc, s, rank * N, world * N);
+  return run_decode(pl, ws, Q, 0, z16, K, Y, 0, B, H, N, M, D, lengths, sc, s, true, rank * N, world * N);
 }
 
 flare_status flare_mixer_fwd_static(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, flare_bf16* Y,

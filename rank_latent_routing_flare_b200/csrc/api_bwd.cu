@@ -23,7 +23,7 @@ BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C) {
   // token splits: whole waves of CTAs (about 128 registers per thread, so
   // 256 / rows_per_block CTAs per SM), by the encoder's cost model
   const long ntiles = cdiv(N, kBwdTokTile);
-  bp.S = choose_splits(BH * bp.LB, ntiles, static_cast<long>(kNumSM) * std::max(1, 256 / bp.rpb));
+  bp.S = choose_splits(BH * bp.LB, ntiles, static_cast<long>(kNumSM) * std::max(1, 256 / bp.rpb), 8);
   bp.tps = static_cast<int>(cdiv(ntiles, bp.S));
   bp.S = static_cast<int>(cdiv(ntiles, bp.tps));
   bp.dw_splits = static_cast<int>(cdiv(B * N, kBwdDwRows));

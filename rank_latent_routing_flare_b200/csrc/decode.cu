@@ -16,18 +16,21 @@
 // and recomputed exactly by decode_fallback_kernel.
 //
 // The chunks of all tiles form one sequence q = tile * nc + chunk.  TMEM holds
-// two score buffers (chunk q uses buffer q % 2; the softmax threads write P_q
-// over the first C/2 columns of S_q once S_q is in registers) and the Y
-// accumulator.  The MMA thread computes S_{q+1} while the softmax threads work
-// on S_q; S_{q+2} reuses the buffer once the value MMA of chunk q is done.
-// Every barrier reused across chunks exists once per buffer, so no party can
-// run a full phase ahead of the party that waits on it.  The epilogue of a
-// tile (Y / sum, bf16 stores) runs after the first chunk of the next tile.
+// NB score buffers (dec_bufs: two at D = 16, three at D = 32; chunk q uses
+// buffer q % NB; the softmax threads write P_q over the first C/2 columns of
+// S_q once S_q is in registers) and the Y accumulator.  The MMA thread issues
+// S_{q+2} right after P_q [Z_c | 1] (with two buffers, once that value MMA is
+// done; with three, at once, since S_{q+2}'s buffer last held P_{q-1}), so
+// the softmax threads find S_{q+1} ready when they finish chunk q.  Every
+// barrier reused across chunks exists once per buffer, so no party can run a
+// full phase ahead of the party that waits on it.  The epilogue of a tile
+// (Y / sum, bf16 stores) runs after the first chunk of the next tile.
 //
 // Warp roles (5 warps): warp 0 lane 0 is the MMA thread (it also loads Q, Z
 // and the first key tiles).  Warps 1..4 are the softmax warps (thread <->
 // TMEM lane <-> token); one of them, in rotation, refills the key ring.  A
-// CTA needs 128 TMEM columns for D = 16, so four CTAs share an SM.
+// CTA needs 128 TMEM columns for D = 16 (two 48-latent score buffers and Y),
+// so four CTAs share an SM.
 #include <type_traits>
 
 #include "ptx.cuh"
@@ -45,19 +48,21 @@ struct DecCfg {
   static constexpr uint32_t LAYOUT = (D == 16) ? LAYOUT_SW32 : LAYOUT_SW64;
   static constexpr uint32_t SBO = 8 * ROWB;
   static constexpr int NY = D + 16;                     // Y columns: D values + sums
+  static constexpr int NB = dec_bufs(D);                // score buffers
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_Z = OFF_Q + QZ_B;
   static constexpr int OFF_ONES = OFF_Z + QZ_B;         // C x ROWB block of ones
   static constexpr int OFF_K = OFF_ONES + C * ROWB;     // NST * KT_B
   static constexpr int OFF_BAR = OFF_K + NST * KT_B;
-  static constexpr int OFF_MISC = OFF_BAR + 8 * 32;
+  static constexpr int OFF_MISC = OFF_BAR + 8 * (4 + NST + 3 * NB);
   static constexpr int BYTES = OFF_MISC + 64 + NST * 4;
-  // TMEM columns: score buffers at 0 and C (each later holds its P), Y at 2C
-  static constexpr uint32_t COL_Y = 2 * C;
+  // TMEM columns: score buffers at 0, C, 2C (each later holds its P), Y at 3C
+  static constexpr uint32_t COL_Y = NB * C;
   static constexpr uint32_t TMEM_COLS = (COL_Y + NY <= 128) ? 128 : 256;
   static constexpr int THREADS = 160;
   static constexpr int CTAS_PER_SM = dec_ctas_per_sm(D);
   static_assert(TMEM_COLS <= 512 / CTAS_PER_SM, "TMEM columns of the co-resident CTAs exceed 512");
+  static_assert(COL_Y + NY <= TMEM_COLS, "score buffers and Y exceed the allocation");
   static_assert(OFF_K % 512 == 0 || D == 16, "key tiles must start on a swizzle atom");
   static_assert(OFF_K % 256 == 0, "key tiles must start on a swizzle atom");
 };
@@ -93,6 +98,7 @@ __device__ __forceinline__ float bf16_row_norm2(const uint4* row, int n16) {
 // global memory; one thread per listed token.
 template <int D>
 __global__ void __launch_bounds__(128) decode_fallback_kernel(const DecodeParams p) {
+  pdl_wait();
   const uint32_t count = *p.fb_count;
   for (uint32_t e = blockIdx.x * blockDim.x + threadIdx.x; e < count; e += gridDim.x * blockDim.x) {
     const uint64_t tok = p.fb_list[e];
@@ -146,7 +152,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
     decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_z,
                   const __grid_constant__ CUtensorMap tm_k, const DecodeParams p) {
   using Cfg = DecCfg<D>;
-  constexpr int NST = Cfg::NST, C = Cfg::C;
+  constexpr int NST = Cfg::NST, C = Cfg::C, NB = Cfg::NB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sq = sm + Cfg::OFF_Q;
@@ -156,12 +162,12 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Cfg::OFF_BAR);
   uint64_t* qz_full = bars;
   uint64_t* k_full = bars + 1;             // [NST] key tile landed
-  uint64_t* s_full = bars + 1 + NST;       // [2] score buffer computed
-  uint64_t* pv_done = s_full + 2;          // [2] value MMA done reading the buffer's P
-  uint64_t* p_full = s_full + 4;           // [2] P stored by every softmax warp
-  uint64_t* y_full = s_full + 6;           // Y of a tile complete
-  uint64_t* y_free = s_full + 7;           // Y read by every softmax warp
-  uint64_t* mma_done = s_full + 8;
+  uint64_t* s_full = bars + 1 + NST;       // [NB] score buffer computed
+  uint64_t* pv_done = s_full + NB;         // [NB] value MMA done reading the buffer's P
+  uint64_t* p_full = s_full + 2 * NB;      // [NB] P stored by every softmax warp
+  uint64_t* y_full = s_full + 3 * NB;      // Y of a tile complete
+  uint64_t* y_free = y_full + 1;           // Y read by every softmax warp
+  uint64_t* mma_done = y_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(sm + Cfg::OFF_MISC + 4);
   float* red = reinterpret_cast<float*>(sm + Cfg::OFF_MISC + 16);
@@ -182,9 +188,10 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
   const int tc_end = min(tb, tiles_valid);            // tiles [ta, tc_end) are computed
   const int ntiles = max(0, tc_end - ta);
   const int nc = (p.M + C - 1) / C;                   // latent chunks
+  pdl_launch_dependents();
 
   // tiles entirely past the valid length: zero rows
-  {
+  auto zero_rows = [&]() {
     const int z0 = max(ta, tiles_valid) * kDecTile;
     const int z1 = min(tb * kDecTile, p.N);
     const uint4 zero = make_uint4(0, 0, 0, 0);
@@ -197,8 +204,12 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
            e += blockDim.x)
         d32[e] = zero;
     }
+  };
+  if (ntiles == 0) {
+    pdl_wait();
+    zero_rows();
+    return;
   }
-  if (ntiles == 0) return;
 
   if (threadIdx.x == 0) {
     mbar_init(qz_full, 1);
@@ -206,7 +217,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
       mbar_init(k_full + i, 1);
       last_load[i] = -1;
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NB; ++i) {
       mbar_init(s_full + i, 1);
       mbar_init(pv_done + i, 1);
       mbar_init(p_full + i, 4);
@@ -227,6 +238,9 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // set-up done: from here on global memory that the previous kernel writes
+  pdl_wait();
+  zero_rows();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{p.err, abort_flag, p.timeout_ns};
   // key tile n (of this CTA's range) into ring stage n % NST (one thread)
@@ -273,12 +287,12 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
       // [Z_c | 1]: chunk c starts CH_STEP * c further on, and its ones block
       // (leading byte offset) is that much closer
       const uint64_t z_desc = umma_desc(sz_a, ones_a - sz_a, Cfg::SBO, Cfg::LAYOUT);
-      // S_q = K_tile Q_c^T into buffer q % 2, once the key tile has landed and
-      // P_{q-2} has been consumed
+      // S_q = K_tile Q_c^T into buffer q % NB, once the key tile has landed and
+      // P_{q-NB} has been consumed
       auto issue_s = [&](const Cursor& x) -> bool {
-        const int buf = x.q & 1, st = x.tile % NST;
+        const int buf = x.q % NB, st = x.tile % NST;
         if (x.cc == 0 && !mbar_wait(k_full + st, (x.tile / NST) & 1, wc)) return false;
-        if (x.q >= 2 && !mbar_wait(pv_done + buf, ((x.q - 2) >> 1) & 1, wc)) return false;
+        if (x.q >= NB && !mbar_wait(pv_done + buf, ((x.q - NB) / NB) & 1, wc)) return false;
         tc_fence_after();
         const uint32_t idesc_s = x.cc == nc - 1 ? idesc_last : idesc_full;
         const uint64_t kd = k_desc + static_cast<uint64_t>(st) * (Cfg::KT_B >> 4);
@@ -292,8 +306,8 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
       // Y += P_q [Z_c | 1] once every softmax warp has stored P_q (and, for a
       // tile's first chunk, has read the previous tile's Y)
       auto issue_pv = [&](const Cursor& x) -> bool {
-        const int buf = x.q & 1;
-        if (!mbar_wait(p_full + buf, (x.q >> 1) & 1, wc)) return false;
+        const int buf = x.q % NB;
+        if (!mbar_wait(p_full + buf, (x.q / NB) & 1, wc)) return false;
         if (x.cc == 0 && x.tile >= 1 && !mbar_wait(y_free, (x.tile - 1) & 1, wc)) return false;
         tc_fence_after();
         const uint64_t step = static_cast<uint64_t>(x.cc) * CH_STEP;
@@ -402,7 +416,8 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
         tmem_ld_cols<CN - 16>(cb + 16, s1);
         exp2_row<16, FLARE_DEC_POLY_PAIRS>(s0, c, nu, *reinterpret_cast<uint32_t(*)[8]>(&pk[0]));
         tmem_wait_ld();
-        exp2_row<CN - 16, FLARE_DEC_POLY_PAIRS>(s1, c, nu, *reinterpret_cast<uint32_t(*)[(CN - 16) / 2]>(&pk[8]));
+        exp2_row<CN - 16, FLARE_DEC_POLY_PAIRS, 8>(s1, c, nu,
+                                                   *reinterpret_cast<uint32_t(*)[(CN - 16) / 2]>(&pk[8]));
       } else {
         exp2_row<16, FLARE_DEC_POLY_PAIRS>(s0, c, nu, pk);
       }
@@ -411,9 +426,8 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
     };
     bool ok = true;
     float nu = 0.f;
-    for (int q = 0, tile = 0, cc = 0; q < total; ++q) {
-      const int buf = q & 1;
-      if (!mbar_wait_warp(s_full + buf, (q >> 1) & 1, wc)) { ok = false; break; }
+    for (int q = 0, tile = 0, cc = 0, buf = 0, use = 0; q < total; ++q) {
+      if (!mbar_wait_warp(s_full + buf, use & 1, wc)) { ok = false; break; }
       tc_fence_after();
       if (cc == 0) {
         // |k_n| from the key tile in shared memory (the swizzle only permutes
@@ -426,8 +440,8 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
       const int cn = min(C, p.M - cc * C);
       const uint32_t cb = lane_base + buf * C;
       if (cn == C) run_chunk(std::integral_constant<int, C>{}, cb, nu);
-      else if (cn == 48) run_chunk(std::integral_constant<int, 48>{}, cb, nu);
-      else if (cn == 32) run_chunk(std::integral_constant<int, 32>{}, cb, nu);
+      else if (C > 48 && cn == 48) run_chunk(std::integral_constant<int, (C > 48 ? 48 : 16)>{}, cb, nu);
+      else if (C > 32 && cn == 32) run_chunk(std::integral_constant<int, (C > 32 ? 32 : 16)>{}, cb, nu);
       else run_chunk(std::integral_constant<int, 16>{}, cb, nu);
       tc_fence_before();
       mbar_arrive_warp(p_full + buf);
@@ -438,6 +452,10 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
       if (++cc == nc) {
         cc = 0;
         ++tile;
+      }
+      if (++buf == NB) {
+        buf = 0;
+        ++use;
       }
     }
     if (ok) epilogue(ntiles - 1);
@@ -466,25 +484,21 @@ size_t decode_smem_bytes(int D, int /*M*/) {
 }
 
 cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_z, const CUtensorMap& tm_k,
-                          const DecodeParams& p, cudaStream_t s) {
+                          const DecodeParams& p, cudaStream_t s, bool pdl) {
   const size_t smem = decode_smem_bytes(p.D, p.M);
   const dim3 grid(static_cast<unsigned>(p.B * p.H * p.ctas_per_head));
-  if (p.D == 16) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+  auto go = [&](auto kern, int threads) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    decode_kernel<16><<<grid, DecCfg<16>::THREADS, smem, s>>>(tm_q, tm_z, tm_k, p);
-  } else {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    decode_kernel<32><<<grid, DecCfg<32>::THREADS, smem, s>>>(tm_q, tm_z, tm_k, p);
-  }
-  cudaError_t e = cudaGetLastError();
+    LaunchCfg lc(grid, dim3(threads), smem, s, pdl);
+    return cudaLaunchKernelEx(&lc.cfg, kern, tm_q, tm_z, tm_k, p);
+  };
+  cudaError_t e = p.D == 16 ? go(decode_kernel<16>, DecCfg<16>::THREADS) : go(decode_kernel<32>, DecCfg<32>::THREADS);
   if (e != cudaSuccess) return e;
-  if (p.D == 16) decode_fallback_kernel<16><<<kNumSM, 128, 0, s>>>(p);
-  else decode_fallback_kernel<32><<<kNumSM, 128, 0, s>>>(p);
-  return cudaGetLastError();
+  // the fallback follows the decoder on the same stream: always programmatic
+  LaunchCfg fb(dim3(kNumSM), dim3(128), 0, s, true);
+  return p.D == 16 ? cudaLaunchKernelEx(&fb.cfg, decode_fallback_kernel<16>, p)
+                   : cudaLaunchKernelEx(&fb.cfg, decode_fallback_kernel<32>, p);
 }
 
 }  // namespace flare

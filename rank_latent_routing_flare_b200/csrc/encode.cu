@@ -14,11 +14,14 @@
 // (U_m, sum_m, O_m) and the merge kernel combines splits with the exact
 // log-sum-exp rule of section "Multi-GPU context parallelism" (eq. 14).
 //
-// TMEM holds two score buffers; tile i uses buffer i % 2, and the softmax
-// threads write P_i (bf16 pairs) over the first T/2 columns of S_i once they
-// hold S_i in registers.  S_{i+2} reuses the buffer after the value MMA of
-// tile i has completed.  The MMA thread therefore computes S_{i+1} while the
-// softmax threads work on S_i, and the softmax threads wait on a single
+// TMEM holds NB score buffers (enc_bufs: two at D = 16, three at D = 32);
+// tile i uses buffer i % NB, and the softmax threads write P_i (bf16 pairs)
+// over the first T/2 columns of S_i once they hold S_i in registers.
+// S_{i+NB} reuses the buffer after the value MMA of tile i has completed.
+// The MMA thread issues S_{i+2} right after P_i V_i: with two buffers it
+// waits for that value MMA first; with three, S_{i+2}'s buffer last held
+// P_{i-1}, whose value MMA finished a tile earlier.  Either way the softmax
+// threads find S_{i+1} ready when they finish tile i.  They wait on a single
 // barrier per tile (S_i ready); their only other barrier operation is the
 // arrive that hands P_i to the MMA thread.  Every barrier that is reused
 // across tiles exists once per buffer, so no party can run a full phase
@@ -29,8 +32,9 @@
 // warps (thread <-> TMEM lane <-> latent row).  They also refill the K/V
 // ring: S_i was issued after P_{i-2} V_{i-2}, so once S_i is complete the
 // ring stage of tile i-2 is free, and one softmax warp, in rotation, loads
-// tile i-2+NST into it.  A CTA needs 128 TMEM columns for D = 16: three CTAs
-// (three softmax warps per SM sub-partition) share an SM.
+// tile i-2+NST into it.  A CTA needs 128 TMEM columns for D = 16 (two
+// 48-token score buffers and O), so four CTAs (four softmax warps per SM
+// sub-partition) share an SM.
 #include <type_traits>
 
 #include "ptx.cuh"
@@ -48,8 +52,9 @@ struct EncCfg {
   static constexpr uint32_t LAYOUT = (D == 16) ? LAYOUT_SW32 : LAYOUT_SW64;
   static constexpr uint32_t SBO = 8 * ROWB;            // stride of 8-row core-matrix groups
   static constexpr int NO = D + 16;                    // O columns: D values + 16 copies of the sum
-  // TMEM columns: score buffers at 0 and T (each later holds its P), O at 2T
-  static constexpr uint32_t COL_O = 2 * T;
+  static constexpr int NB = enc_bufs(D);               // score buffers
+  // TMEM columns: score buffers at 0, T, 2T (each later holds its P), O at 3T
+  static constexpr uint32_t COL_O = NB * T;
   static constexpr uint32_t TMEM_COLS = (COL_O + NO <= 128) ? 128 : 256;
   // Each V stage is followed by its own block of ones, so that [V | 1] has
   // the same leading byte offset (TILE_B) in every stage.
@@ -57,11 +62,12 @@ struct EncCfg {
   static constexpr int OFF_K = OFF_Q + Q_B;
   static constexpr int OFF_V = OFF_K + NST * TILE_B;   // NST x [V tile | ones]
   static constexpr int OFF_BAR = OFF_V + NST * 2 * TILE_B;
-  static constexpr int OFF_MISC = OFF_BAR + 8 * 32;
+  static constexpr int OFF_MISC = OFF_BAR + 8 * (2 + NST + 3 * NB);
   static constexpr int BYTES = OFF_MISC + 64 + NST * 4;
   static constexpr int THREADS = 160;
   static constexpr int CTAS_PER_SM = enc_ctas_per_sm(D);
   static_assert(TMEM_COLS <= 512 / CTAS_PER_SM, "TMEM columns of the co-resident CTAs exceed 512");
+  static_assert(COL_O + NO <= TMEM_COLS, "score buffers and O exceed the allocation");
   static_assert(T % 16 == 0 && TILE_B % 256 == 0, "tile must hold whole swizzle atoms");
 };
 
@@ -70,7 +76,7 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
     encode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const EncodeParams p) {
   using Cfg = EncCfg<D>;
-  constexpr int NST = Cfg::NST, T = Cfg::T;
+  constexpr int NST = Cfg::NST, T = Cfg::T, NB = Cfg::NB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sq = sm + Cfg::OFF_Q;
@@ -79,10 +85,10 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Cfg::OFF_BAR);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;            // [NST] K/V tile landed
-  uint64_t* s_full = bars + 1 + NST;       // [2] score buffer computed
-  uint64_t* pv_done = s_full + 2;          // [2] value MMA done reading the buffer's P
-  uint64_t* p_full = s_full + 4;           // [2] P stored by every softmax warp (one arrive per warp)
-  uint64_t* o_full = s_full + 6;           // every MMA of the CTA done
+  uint64_t* s_full = bars + 1 + NST;       // [NB] score buffer computed
+  uint64_t* pv_done = s_full + NB;         // [NB] value MMA done reading the buffer's P
+  uint64_t* p_full = s_full + 2 * NB;      // [NB] P stored by every softmax warp (one arrive per warp)
+  uint64_t* o_full = s_full + 3 * NB;      // every MMA of the CTA done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(sm + Cfg::OFF_MISC + 4);
   float* red = reinterpret_cast<float*>(sm + Cfg::OFF_MISC + 16);
@@ -103,8 +109,10 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
   const int ntiles = max(0, t1 - t0);
   const int g = p.q_per_batch ? bh : h;
   float* part_base = p.part + static_cast<size_t>(bh * S + s) * p.M * (D + 2);
+  pdl_launch_dependents();
 
   if (ntiles == 0) {  // empty split: contributes nothing to the merge
+    pdl_wait();
     for (int r = threadIdx.x; r < kLatBlock; r += blockDim.x) {
       const int m = lb * kLatBlock + r;
       if (m < p.M) {
@@ -124,7 +132,7 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
       mbar_init(kv_full + i, 1);
       last_load[i] = -1;
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NB; ++i) {
       mbar_init(s_full + i, 1);
       mbar_init(pv_done + i, 1);
       mbar_init(p_full + i, 4);
@@ -145,6 +153,8 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // set-up done: from here on global memory that the previous kernel writes
+  pdl_wait();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{p.err, abort_flag, p.timeout_ns};
   // K and V of tile n into ring stage n % NST (one thread)
@@ -172,11 +182,11 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
       const uint64_t q_desc = umma_desc(smem_u32(sq), 16, Cfg::SBO, Cfg::LAYOUT);
       const uint64_t k_desc = umma_desc(smem_u32(sk), 16, Cfg::SBO, Cfg::LAYOUT);
       const uint64_t v_desc = umma_desc(smem_u32(sv), Cfg::TILE_B, Cfg::SBO, Cfg::LAYOUT);
-      // S_i into buffer i % 2, once tile i has landed and P_{i-2} has been consumed
+      // S_i into buffer i % NB, once tile i has landed and P_{i-NB} has been consumed
       auto issue_s = [&](int i) -> bool {
-        const int st = i % NST, buf = i & 1;
+        const int st = i % NST, buf = i % NB;
         if (!mbar_wait(kv_full + st, (i / NST) & 1, wc)) return false;
-        if (i >= 2 && !mbar_wait(pv_done + buf, ((i - 2) >> 1) & 1, wc)) return false;
+        if (i >= NB && !mbar_wait(pv_done + buf, ((i - NB) / NB) & 1, wc)) return false;
         tc_fence_after();
         const uint64_t kd = k_desc + static_cast<uint64_t>((st * Cfg::TILE_B) >> 4);
 #pragma unroll
@@ -187,8 +197,8 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
       };
       // O += P_i [V_i | 1] once every softmax warp has stored P_i
       auto issue_pv = [&](int i) -> bool {
-        const int buf = i & 1;
-        if (!mbar_wait(p_full + buf, (i >> 1) & 1, wc)) return false;
+        const int buf = i % NB;
+        if (!mbar_wait(p_full + buf, (i / NB) & 1, wc)) return false;
         tc_fence_after();
         const uint64_t vd = v_desc + static_cast<uint64_t>(((i % NST) * 2 * Cfg::TILE_B) >> 4);
 #pragma unroll
@@ -247,9 +257,8 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
     // the tile loop, with NP polynomial exp2 pairs out of every 32
     auto run_tiles = [&](auto np_tag) -> bool {
       constexpr int NP = decltype(np_tag)::value;
-      for (int i = 0; i < ntiles; ++i) {
-        const int buf = i & 1;
-        if (!mbar_wait_warp(s_full + buf, (i >> 1) & 1, wc)) return false;
+      for (int i = 0, buf = 0, use = 0; i < ntiles; ++i) {
+        if (!mbar_wait_warp(s_full + buf, use & 1, wc)) return false;
         tc_fence_after();
         const int valid = L - (t0 + i) * T;
         if (warp_live && FLARE_ENC_SPLIT_LD && valid >= T) {
@@ -261,7 +270,7 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
           tmem_ld_cols<R>(lane_base + buf * T + 16, s1);
           exp2_row<16, NP>(s0, c, U, *reinterpret_cast<uint32_t(*)[8]>(&pk[0]));
           tmem_wait_ld();
-          exp2_row<R, NP>(s1, c, U, *reinterpret_cast<uint32_t(*)[R / 2]>(&pk[8]));
+          exp2_row<R, NP, 8>(s1, c, U, *reinterpret_cast<uint32_t(*)[R / 2]>(&pk[8]));
           tmem_st_cols<T / 2>(lane_base + buf * T, pk);  // P_i over the first T/2 columns of S_i
           tmem_wait_st();
         } else if (warp_live) {
@@ -286,6 +295,10 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
         // S_i complete implies P_{i-2} V_{i-2} complete: its ring stage is free
         if (i >= 2 && i - 2 + NST < ntiles && wq == (i & 3) && lane == 0) load_tile(i - 2 + NST);
         __syncwarp();
+        if (++buf == NB) {
+          buf = 0;
+          ++use;
+        }
       }
       return true;
     };
@@ -340,21 +353,16 @@ size_t encode_smem_bytes(int D) {
 }
 
 cudaError_t launch_encode(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                          const EncodeParams& p, cudaStream_t s) {
+                          const EncodeParams& p, cudaStream_t s, bool pdl) {
   const size_t smem = encode_smem_bytes(p.D);
   const dim3 grid(static_cast<unsigned>(p.B * p.H * p.n_lblocks * p.n_splits));
-  if (p.D == 16) {
-    cudaError_t e = cudaFuncSetAttribute(encode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+  auto go = [&](auto kern, int threads) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    encode_kernel<16><<<grid, EncCfg<16>::THREADS, smem, s>>>(tm_q, tm_k, tm_v, p);
-  } else {
-    cudaError_t e = cudaFuncSetAttribute(encode_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    encode_kernel<32><<<grid, EncCfg<32>::THREADS, smem, s>>>(tm_q, tm_k, tm_v, p);
-  }
-  return cudaGetLastError();
+    LaunchCfg lc(grid, dim3(threads), smem, s, pdl);
+    return cudaLaunchKernelEx(&lc.cfg, kern, tm_q, tm_k, tm_v, p);
+  };
+  return p.D == 16 ? go(encode_kernel<16>, EncCfg<16>::THREADS) : go(encode_kernel<32>, EncCfg<32>::THREADS);
 }
 
 }  // namespace flare

@@ -34,20 +34,42 @@ constexpr int kDecTile = 128;      // tokens per decode tile (UMMA M)
 constexpr int kNormGroup = 32;     // tokens per key-norm group
 constexpr int kProjTile = 128;     // tokens per projection tile
 
-// Tokens per encoder tile.  The encoder keeps two score tiles and the
-// output accumulator in TMEM: 2 * 48 + 32 = 128 columns for D = 16, and
-// 2 * 64 + 48 (within 256) for D = 32.
-__host__ __device__ constexpr int enc_tile(int D) { return D == 16 ? 48 : 64; }
+// Tokens per encoder tile and score buffers in TMEM.  The encoder keeps
+// enc_bufs score tiles and the output accumulator (D + 16 columns) in TMEM:
+// 2 * 48 + 32 = 128 columns for D = 16 (four CTAs per SM), and 3 * 64 + 48
+// (within 256, two CTAs per SM) for D = 32.  Chosen by measurement on B200:
+// at D = 16 three 32-token buffers (the same 128 columns) were 12 % slower
+// than two 48-token ones.
+#ifndef FLARE_ENC_TILE_D16
+#define FLARE_ENC_TILE_D16 48
+#endif
+#ifndef FLARE_ENC_BUFS_D16
+#define FLARE_ENC_BUFS_D16 2
+#endif
+#ifndef FLARE_ENC_BUFS_D32
+#define FLARE_ENC_BUFS_D32 3
+#endif
+__host__ __device__ constexpr int enc_tile(int D) { return D == 16 ? FLARE_ENC_TILE_D16 : 64; }
+__host__ __device__ constexpr int enc_bufs(int D) { return D == 16 ? FLARE_ENC_BUFS_D16 : FLARE_ENC_BUFS_D32; }
 // Co-resident CTAs per SM of the encoder: 128 TMEM columns per CTA for
 // D = 16 (up to four CTAs), 256 for D = 32 (two).
 #ifndef FLARE_ENC_CTAS_D16
 #define FLARE_ENC_CTAS_D16 4
 #endif
 __host__ __device__ constexpr int enc_ctas_per_sm(int D) { return D == 16 ? FLARE_ENC_CTAS_D16 : 2; }
-// Latents per decoder chunk.  The decoder keeps two score chunks and the
-// output accumulator in TMEM: 2 * 48 + 32 = 128 columns for D = 16, and
-// 2 * 64 + 48 (within 256) for D = 32.
-__host__ __device__ constexpr int dec_chunk(int D) { return D == 16 ? 48 : 64; }
+// Latents per decoder chunk and score buffers, as for the encoder: 2 * 48
+// + 32 = 128 TMEM columns for D = 16, 3 * 64 + 48 (within 256) for D = 32.
+#ifndef FLARE_DEC_CHUNK_D16
+#define FLARE_DEC_CHUNK_D16 48
+#endif
+#ifndef FLARE_DEC_BUFS_D16
+#define FLARE_DEC_BUFS_D16 2
+#endif
+#ifndef FLARE_DEC_BUFS_D32
+#define FLARE_DEC_BUFS_D32 3
+#endif
+__host__ __device__ constexpr int dec_chunk(int D) { return D == 16 ? FLARE_DEC_CHUNK_D16 : 64; }
+__host__ __device__ constexpr int dec_bufs(int D) { return D == 16 ? FLARE_DEC_BUFS_D16 : FLARE_DEC_BUFS_D32; }
 // Co-resident CTAs per SM of the decoder (TMEM columns as for the encoder).
 #ifndef FLARE_DEC_CTAS_D16
 #define FLARE_DEC_CTAS_D16 4
@@ -55,10 +77,10 @@ __host__ __device__ constexpr int dec_chunk(int D) { return D == 16 ? 48 : 64; }
 __host__ __device__ constexpr int dec_ctas_per_sm(int D) { return D == 16 ? FLARE_DEC_CTAS_D16 : 2; }
 
 // Of every 32 score pairs of a softmax row, how many are exponentiated on
-// the FMA pipe (polynomial) instead of the MUFU; chosen by measurement on
-// B200 (the encoder gains with 4, the decoder loses).
+// the FMA pipe (polynomial, paired fp32 instructions) instead of the MUFU;
+// chosen by measurement on B200.
 #ifndef FLARE_ENC_POLY_PAIRS
-#define FLARE_ENC_POLY_PAIRS 4
+#define FLARE_ENC_POLY_PAIRS 10
 #endif
 // Encoder softmax: load the first 16 score columns, start their
 // exponentials while the rest of the tile is read from TMEM.
@@ -71,7 +93,7 @@ __host__ __device__ constexpr int dec_ctas_per_sm(int D) { return D == 16 ? FLAR
 #define FLARE_PROJ_EPI_HEADS 4
 #endif
 #ifndef FLARE_DEC_POLY_PAIRS
-#define FLARE_DEC_POLY_PAIRS 6
+#define FLARE_DEC_POLY_PAIRS 10
 #endif
 
 // ---------------------------------------------------------------------------
@@ -141,6 +163,9 @@ struct MergeParams {
   const uint16_t* v;    // bf16 values [B*H][N][D]
   float* out_f32;       // [B*H][M][D]
   uint16_t* out_bf16;   // [B*H][M][D]
+  const float* fix;     // context parallelism: every shard's exact partials of the rows that need
+                        // them, [n_ranks][B*H*M][D+2] rank-major, or nullptr
+  size_t fix_rank_stride;  // floats between consecutive shards' exact partials
 };
 
 // ---------------------------------------------------------------------------
@@ -168,15 +193,43 @@ struct DecodeParams {
   unsigned long long timeout_ns;
 };
 
-// Host-side launchers (each returns the cudaError_t of the launch).
+// Launch configuration of one kernel.  With pdl (programmatic dependent
+// launch) the kernel may begin -- its CTAs become resident and run their
+// set-up -- while the previous kernel on the stream is still finishing; every
+// kernel of this library calls pdl_wait() before its first access to global
+// memory that another kernel writes or reads, and calls
+// pdl_launch_dependents() early so that the next kernel can start.  Only a
+// kernel whose predecessor on the stream is a kernel of the same call is
+// launched with pdl.
+struct LaunchCfg {
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  LaunchCfg(dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl) {
+#ifdef FLARE_NO_PDL
+    pdl = false;
+#endif
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+  }
+};
+
+// Host-side launchers (each returns the cudaError_t of the launch; pdl as
+// for LaunchCfg).
 cudaError_t launch_project(const CUtensorMap& tm_x, const CUtensorMap (&tm_w)[4], const ProjParams& p,
-                           cudaStream_t s);
+                           cudaStream_t s, bool pdl = false);
 cudaError_t launch_knorm(const KnormParams& p, cudaStream_t s);
 cudaError_t launch_encode(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                          const EncodeParams& p, cudaStream_t s);
-cudaError_t launch_merge(const MergeParams& p, cudaStream_t s);
+                          const EncodeParams& p, cudaStream_t s, bool pdl = false);
+cudaError_t launch_merge(const MergeParams& p, cudaStream_t s, bool pdl = false);
+cudaError_t launch_cp_exact(const MergeParams& p, int rank, float* out, cudaStream_t s);
 cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_z, const CUtensorMap& tm_k,
-                          const DecodeParams& p, cudaStream_t s);
+                          const DecodeParams& p, cudaStream_t s, bool pdl = false);
 cudaError_t launch_wait_selftest(uint32_t* err, unsigned long long timeout_ns, cudaStream_t s);
 
 // Shared-memory footprints (bytes) of the pipelined kernels.

@@ -38,8 +38,9 @@ struct BwdPlan {
 
 BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C);
 
-// Number of token splits of a split-N pass (the encoder's wave cost model).
-int choose_splits(long units, long ntiles, long slots);
+// Number of token splits of a split-N pass (the encoder's wave cost model;
+// setup_tiles: a CTA's fixed cost in tiles of work).
+int choose_splits(long units, long ntiles, long slots, long setup_tiles);
 
 flare_status check_common(int B, int H, int N, int M, int D);
 float resolve_scale(float scale, int D);

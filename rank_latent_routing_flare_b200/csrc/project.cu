@@ -65,7 +65,11 @@ __global__ void __launch_bounds__(192, 1)
   const int grp = blockIdx.x / p.n_proj;
   const int H = p.H;
   const int my_tiles = (grp < p.n_tiles) ? (p.n_tiles - 1 - grp) / p.groups + 1 : 0;
-  if (my_tiles == 0) return;
+  pdl_launch_dependents();
+  if (my_tiles == 0) {
+    pdl_wait();
+    return;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(w_full, 1);
@@ -88,6 +92,8 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // set-up done: from here on global memory that the previous kernel writes
+  pdl_wait();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{p.err, abort_flag, p.timeout_ns};
 
@@ -222,19 +228,19 @@ __global__ void __launch_bounds__(192, 1)
 
 template <int C, int D>
 cudaError_t launch_project_cd(const CUtensorMap& tm_x, const CUtensorMap (&tm_w)[4], const ProjParams& p,
-                              cudaStream_t s) {
+                              cudaStream_t s, bool pdl) {
   const size_t smem = project_smem_bytes(C);
   cudaError_t e = cudaFuncSetAttribute(project_kernel<C, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  project_kernel<C, D><<<dim3(p.n_proj * p.groups), 192, smem, s>>>(tm_x, tm_w[0], tm_w[1], tm_w[2], tm_w[3], p);
-  return cudaGetLastError();
+  LaunchCfg lc(dim3(p.n_proj * p.groups), dim3(192), smem, s, pdl);
+  return cudaLaunchKernelEx(&lc.cfg, project_kernel<C, D>, tm_x, tm_w[0], tm_w[1], tm_w[2], tm_w[3], p);
 }
 
 template <int C>
 cudaError_t launch_project_c(const CUtensorMap& tm_x, const CUtensorMap (&tm_w)[4], const ProjParams& p,
-                             cudaStream_t s) {
-  return p.D == 16 ? launch_project_cd<C, 16>(tm_x, tm_w, p, s) : launch_project_cd<C, 32>(tm_x, tm_w, p, s);
+                             cudaStream_t s, bool pdl) {
+  return p.D == 16 ? launch_project_cd<C, 16>(tm_x, tm_w, p, s, pdl) : launch_project_cd<C, 32>(tm_x, tm_w, p, s, pdl);
 }
 
 }  // namespace
@@ -250,11 +256,11 @@ size_t project_smem_bytes(int C) {
 }
 
 cudaError_t launch_project(const CUtensorMap& tm_x, const CUtensorMap (&tm_w)[4], const ProjParams& p,
-                           cudaStream_t s) {
+                           cudaStream_t s, bool pdl) {
   switch (p.C) {
-    case 64: return launch_project_c<64>(tm_x, tm_w, p, s);
-    case 128: return launch_project_c<128>(tm_x, tm_w, p, s);
-    case 256: return launch_project_c<256>(tm_x, tm_w, p, s);
+    case 64: return launch_project_c<64>(tm_x, tm_w, p, s, pdl);
+    case 128: return launch_project_c<128>(tm_x, tm_w, p, s, pdl);
+    case 256: return launch_project_c<256>(tm_x, tm_w, p, s, pdl);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -117,6 +117,13 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   return true;
 }
 
+// Programmatic dependent launch (see LaunchCfg): wait until the previous
+// kernel on the stream has completed and its writes are visible (returns at
+// once for a kernel launched normally), and let the next kernel start
+// launching once every CTA of this grid has called it or exited.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -319,6 +326,47 @@ __device__ __forceinline__ float ex2_poly(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// ----------------------------------------------------------------------------
+// packed fp32 pairs (sm_100: one instruction computes two lanes' worth)
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+// a * b + c, elementwise, round to nearest
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// ex2_poly of two values with the paired instructions: the same operations,
+// each rounded as in ex2_poly, so the results are bitwise the same.
+__device__ __forceinline__ void ex2_poly_x2(float x0, float x1, float& e0, float& e1) {
+  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f), neg_magic = f2_pack(-12582912.0f, -12582912.0f);
+  const uint64_t x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t t = f2_add(x, magic);
+  const uint64_t r = f2_add(t, neg_magic);                       // t - magic, exact
+  const uint64_t f = f2_fma(r, f2_pack(-1.0f, -1.0f), x);       // x - r, exact
+  uint64_t p = f2_fma(f2_pack(0x1.c3f76p-5f, 0x1.c3f76p-5f), f, f2_pack(0x1.f0de1ap-3f, 0x1.f0de1ap-3f));
+  p = f2_fma(p, f, f2_pack(0x1.62f31ap-1f, 0x1.62f31ap-1f));
+  p = f2_fma(p, f, f2_pack(0x1.fff692p-1f, 0x1.fff692p-1f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  e0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  e1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 // Exponentials of one 64-column chunk of scores (raw fp32 bits in a[0..31],
 // b[0..31]): e = 2^(s * c - shift), packed to bf16 pairs.  NPOLY of the 32
 // pairs use ex2_poly (FMA pipe), spread evenly; the rest use the MUFU.
@@ -346,18 +394,36 @@ __device__ __forceinline__ void exp2_chunk64(const uint32_t (&a)[32], const uint
 
 // Exponentials of one row of NV scores (raw fp32 bits in s[0..NV)): e =
 // 2^(s * c - shift), packed to bf16 pairs pk[0..NV/2).  NPOLY of every 32
-// pairs use ex2_poly (FMA pipe), spread evenly; the rest use the MUFU.
-template <int NV, int NPOLY>
+// pairs use ex2_poly (FMA pipe), spread evenly; the rest use the MUFU.  A row
+// exponentiated in pieces passes each piece's first pair index as Q0, so the
+// pattern runs on across the pieces.
+#ifndef FLARE_PACKED_F32X2
+#define FLARE_PACKED_F32X2 1
+#endif
+template <int NV, int NPOLY, int Q0 = 0>
 __device__ __forceinline__ void exp2_row(const uint32_t (&s)[NV], float c, float shift, uint32_t (&pk)[NV / 2]) {
+#if FLARE_PACKED_F32X2
+  // the scale-and-shift of a pair of scores is one paired fma
+  const uint64_t c2 = f2_pack(c, c), ms2 = f2_pack(-shift, -shift);
+#endif
 #pragma unroll
   for (int q = 0; q < NV / 2; ++q) {
-    const float x0 = fmaf(__uint_as_float(s[2 * q]), c, -shift);
-    const float x1 = fmaf(__uint_as_float(s[2 * q + 1]), c, -shift);
-    const bool poly = (((q % 32) * NPOLY) % 32) < NPOLY;
+    float x0, x1;
+#if FLARE_PACKED_F32X2
+    f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * q]), __uint_as_float(s[2 * q + 1])), c2, ms2), x0, x1);
+#else
+    x0 = fmaf(__uint_as_float(s[2 * q]), c, -shift);
+    x1 = fmaf(__uint_as_float(s[2 * q + 1]), c, -shift);
+#endif
+    const bool poly = ((((q + Q0) % 32) * NPOLY) % 32) < NPOLY;
     float e0, e1;
     if (poly) {
+#if FLARE_PACKED_F32X2
+      ex2_poly_x2(x0, x1, e0, e1);
+#else
       e0 = ex2_poly(x0);
       e1 = ex2_poly(x1);
+#endif
     } else {
       e0 = ex2_mufu(x0);
       e1 = ex2_mufu(x1);

@@ -34,6 +34,7 @@ def test_header_declares_the_abi():
                             "flare_last_device_status", "flare_status_string",
                             "flare_selftest_wait_timeout", "flare_cp_partials_bytes", "flarepp_cp_begin",
                             "flarepp_cp_middle", "flarepp_cp_end", "flare_cp_begin", "flare_cp_end",
+                            "flare_cp_exact_bytes", "flarepp_cp_exact", "flare_cp_exact",
                             "flare_mixer_bwd", "flarepp_mixer_bwd", "flarepp_cp_bwd_exchange_bytes",
                             "flarepp_cp_bwd_phase", "flare_mixer_fwd_inspect", "flarepp_mixer_fwd_inspect",
                             "flare_static_last_device_status", "flare_probe_scratch_bytes",
@@ -198,12 +199,22 @@ def test_context_parallel_argument_errors():
     assert lib.flarepp_cp_begin(A, A, A, A, A, A, *args, 0, 1, 0.0, W, ws, None, None) == Status.ERR_NULL
     assert lib.flarepp_cp_begin(A, A, A, A, A, A, *args, 0, 1, 0.0, W, ws, None, A + 4) == Status.ERR_ALIGN
     assert lib.flarepp_cp_begin(A, A, A, A, A, A, *args, 0, 1, 0.0, W, ws - 256, None, A) == Status.ERR_WORKSPACE
-    assert lib.flarepp_cp_middle(A, *args, 0, 0, 0.0, W, ws, None, A, None) == Status.ERR_SHAPE   # world 0
-    assert lib.flarepp_cp_end(None, A, *args, 0, 1, 0.0, W, ws, None, None) == Status.ERR_NULL
+    assert lib.flarepp_cp_middle(A, A, *args, 0, 0, 0.0, W, ws, None, A, None) == Status.ERR_SHAPE   # world 0
+    assert lib.flarepp_cp_middle(A, A + 4, *args, 0, 1, 0.0, W, ws, None, A, None) == Status.ERR_ALIGN
+    assert lib.flarepp_cp_end(None, A, A, *args, 0, 1, 0.0, W, ws, None, None) == Status.ERR_NULL
+    # the exact step: pass 0 or 1 only, every pointer, alignment, workspace
+    assert lib.flare_cp_exact_bytes(1, 4, 32, 16) == 4 * 32 * 18 * 4
+    assert lib.flare_cp_exact_bytes(1, 4, 40, 16) == 0
+    assert lib.flarepp_cp_exact(2, A, A, A, A, A, A, *args, 0, 1, 0.0, W, ws, None, A) == Status.ERR_SHAPE
+    assert lib.flarepp_cp_exact(0, A, A, A, A, A, A, *args, 0, 1, 0.0, W, ws, None, None) == Status.ERR_NULL
+    assert lib.flarepp_cp_exact(1, A, A, A, A, A, A, *args, 0, 1, 0.0, W, ws, None, A + 4) == Status.ERR_ALIGN
+    assert lib.flarepp_cp_exact(1, A, A, A, A, A, A, *args, 0, 1, 0.0, W, ws - 256, None, A) == Status.ERR_WORKSPACE
     fargs = (1, 2, 100, 32, 16, None)
     fws = fl.flare_workspace_bytes(0, 1, 2, 100, 32, 16)
     assert lib.flare_cp_begin(A, A, A, *fargs, -1, 2, 0.0, W, fws, None, A) == Status.ERR_SHAPE
-    assert lib.flare_cp_end(A, A, A, None, *fargs, 0, 2, 0.0, W, fws, None, None) == Status.ERR_NULL
+    assert lib.flare_cp_end(A, None, A, A, None, *fargs, 0, 2, 0.0, W, fws, None, None) == Status.ERR_NULL
+    assert lib.flare_cp_exact(A, A, None, A, *fargs, 0, 2, 0.0, W, fws, None, A) == Status.ERR_NULL
+    assert lib.flare_cp_exact(A, A, A, A, *fargs, 2, 2, 0.0, W, fws, None, A) == Status.ERR_SHAPE
     assert fl.flare_status_string(8).startswith("FLARE_ERR_UNDERFLOW")
 
 
