@@ -354,6 +354,8 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
     const float c = p.c;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     // Epilogue of tile i: Y = acc / sum, zero rows for padding, bf16 stores.
+    // (Reading Y before the next tile's first exponentials instead, so that
+    // the next value MMA need not wait for it, measured 4 % slower.)
     auto epilogue = [&](int i) -> bool {
       if (!mbar_wait_warp(y_full, i & 1, wc)) return false;
       tc_fence_after();

@@ -80,7 +80,7 @@ __host__ __device__ constexpr int dec_ctas_per_sm(int D) { return D == 16 ? FLAR
 // the FMA pipe (polynomial, paired fp32 instructions) instead of the MUFU;
 // chosen by measurement on B200.
 #ifndef FLARE_ENC_POLY_PAIRS
-#define FLARE_ENC_POLY_PAIRS 10
+#define FLARE_ENC_POLY_PAIRS 11
 #endif
 // Encoder softmax: load the first 16 score columns, start their
 // exponentials while the rest of the tile is read from TMEM.

@@ -119,6 +119,10 @@ __device__ RowStats row_stats(const MergeParams& p, int bh, int m, int b, int la
   return {G, any, needs};
 }
 
+// From this many (shard, split) partials per row on, the merge gives every
+// lane whole splits (one round of loads) instead of one value of d.
+constexpr int kMergeLanesOverSplits = 12;
+
 template <int D>
 __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
   pdl_launch_dependents();
@@ -181,26 +185,63 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
       den += __shfl_xor_sync(0xffffffffu, den, o);
     }
     z = num / den;
+  } else if (G > -INFINITY && R * S < kMergeLanesOverSplits) {
+    // few splits: the 32 / D lane groups take the splits j = group,
+    // group + 32 / D, ..., each lane one value of d
+    float num = 0.f, den = 0.f;
+#pragma unroll 4
+    for (int j = grp; j < R * S; j += NG) {
+      const int r = j / S, s = j - r * S;
+      if (split_tiles(r, s) == 0) continue;
+      const float* e = part_of(r, s);  // (U, l, O[D])
+      const float2 ul = *reinterpret_cast<const float2*>(e);
+      if (!(ul.y > 0.f)) continue;
+      const float w = exp2f(ul.x - G);
+      den = fmaf(w, ul.y, den);
+      num = fmaf(w, e[2 + d], num);
+    }
+#pragma unroll
+    for (int o = D; o < 32; o <<= 1) {  // combine the groups (commutative adds: same bits in every lane)
+      num += __shfl_xor_sync(0xffffffffu, num, o);
+      den += __shfl_xor_sync(0xffffffffu, den, o);
+    }
+    z = num / den;
+    if (rs.needs_exact && lane == 0) atomicOr(p.err, FLARE_DEV_UNDERFLOW);
   } else {
     if (G > -INFINITY) {
-      float num = 0.f, den = 0.f;
-#pragma unroll 4
-      for (int j = grp; j < R * S; j += NG) {
+      // many splits: every lane takes whole splits j = lane, lane + 32, ...
+      // (one row of D + 2 floats each, all loads of the warp in flight at
+      // once), then a butterfly over the lanes; each step adds two lanes'
+      // values, a commutative operation, so every lane ends with the same bits
+      float num[D], den = 0.f;
+#pragma unroll
+      for (int k = 0; k < D; ++k) num[k] = 0.f;
+      for (int j = lane; j < R * S; j += 32) {
         const int r = j / S, s = j - r * S;
         if (split_tiles(r, s) == 0) continue;
-        const float* e = part_of(r, s);  // (U, l, O[D])
-        const float2 ul = *reinterpret_cast<const float2*>(e);
+        const float2* e = reinterpret_cast<const float2*>(part_of(r, s));  // (U, l), then O[D] as pairs
+        const float2 ul = e[0];
         if (!(ul.y > 0.f)) continue;
         const float w = exp2f(ul.x - G);
         den = fmaf(w, ul.y, den);
-        num = fmaf(w, e[2 + d], num);
+#pragma unroll
+        for (int k = 0; k < D / 2; ++k) {
+          const float2 o = e[1 + k];
+          num[2 * k] = fmaf(w, o.x, num[2 * k]);
+          num[2 * k + 1] = fmaf(w, o.y, num[2 * k + 1]);
+        }
       }
 #pragma unroll
-      for (int o = D; o < 32; o <<= 1) {  // combine the groups (commutative adds: same bits in every lane)
-        num += __shfl_xor_sync(0xffffffffu, num, o);
+      for (int o = 16; o > 0; o >>= 1) {
         den += __shfl_xor_sync(0xffffffffu, den, o);
+#pragma unroll
+        for (int k = 0; k < D; ++k) num[k] += __shfl_xor_sync(0xffffffffu, num[k], o);
       }
-      z = num / den;
+      float mine = 0.f;
+#pragma unroll
+      for (int k = 0; k < D; ++k)
+        if (k == d) mine = num[k];
+      z = mine / den;
     }
     // a row that needed the exact recomputation, with no exact partials of
     // the other shards at hand, is reported instead
