@@ -282,6 +282,29 @@ FLARE_API flare_status flarepp_cp_bwd_phase(int phase, const flare_bf16* X, cons
                                             void* stream);
 
 /*
+ * Context-parallel FLARE backward (token sharding as for flare_cp_begin /
+ * flare_cp_end; K, V, dY, dK and dV are the shard's rows, `lengths` counts
+ * tokens of the whole sequences).  The backward of flare_mixer_bwd runs in
+ * FLARE_CP_BWD_PHASES_FLARE phases with the same protocol as
+ * flarepp_cp_bwd_phase: phase p (< last) writes
+ * flare_cp_bwd_exchange_bytes(p, ...) bytes to `exchange`, the caller
+ * all-gathers them in rank order and passes the result as `gathered` to phase
+ * p + 1.  Every rank merges in ascending (rank, split) order, so every rank
+ * ends with bitwise the same dQ (written by the last phase); dK and dV hold
+ * the shard's rows (written by phase 2).  With world == 1 the result equals
+ * flare_mixer_bwd bit for bit (flare_mixer_bwd runs the same phases).  The
+ * phases of one rank share its workspace (FLARE_VARIANT_FLARE_BWD with the
+ * shard's N).  An out-of-range phase returns FLARE_ERR_SHAPE.
+ */
+#define FLARE_CP_BWD_PHASES_FLARE 4
+FLARE_API size_t flare_cp_bwd_exchange_bytes(int phase, int B, int H, int N, int M, int D);
+FLARE_API flare_status flare_cp_bwd_phase(int phase, const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q,
+                                          const flare_bf16* dY, const float* gathered, float* exchange,
+                                          flare_bf16* dK, flare_bf16* dV, float* dQ, int B, int H, int N, int M,
+                                          int D, const int32_t* lengths, int rank, int world, float scale,
+                                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream`, reads the device error word of `workspace` and
  * returns FLARE_OK, FLARE_ERR_TIMEOUT, FLARE_ERR_SHAPE (invalid lengths) or
  * FLARE_ERR_UNDERFLOW (context-parallel merges only).

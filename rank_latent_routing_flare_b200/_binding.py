@@ -96,6 +96,10 @@ def load_library(build_if_missing: bool = True):
         lib.flarepp_mixer_bwd.argtypes = [vp] * 13 + [i] * 6 + [vp, f, vp, sz, vp]
         lib.flarepp_cp_bwd_exchange_bytes.restype = sz
         lib.flarepp_cp_bwd_exchange_bytes.argtypes = [i] * 7
+        lib.flare_cp_bwd_exchange_bytes.restype = sz
+        lib.flare_cp_bwd_exchange_bytes.argtypes = [i] * 6
+        lib.flare_cp_bwd_phase.restype = i
+        lib.flare_cp_bwd_phase.argtypes = [i] + [vp] * 9 + [i] * 5 + [vp, i, i, f, vp, sz, vp]
         lib.flarepp_cp_bwd_phase.restype = i
         lib.flarepp_cp_bwd_phase.argtypes = [i] + [vp] * 15 + [i] * 6 + [vp, i, i, f, vp, sz, vp]
         lib.flarepp_mixer_out_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, f, vp, sz, vp]

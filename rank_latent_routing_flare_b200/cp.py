@@ -161,6 +161,47 @@ def flare_mixer_cp_fwd(K, V, Q, lengths=None, group=None, scale: float = 0.0, Y=
 
 
 FLARE_CP_BWD_PHASES = 7
+FLARE_CP_BWD_PHASES_FLARE = 4
+
+
+def flare_mixer_cp_bwd(K, V, Q, dY, lengths=None, group=None, scale: float = 0.0, workspace=None, stream=None,
+                       dK=None, dV=None, dQ=None, device_check=None):
+    """FLARE backward of this rank's token shard (the sharding of
+    flare_mixer_cp_fwd; K, V, dY [B, H, N, D] hold the shard's rows).
+    Returns (dK, dV) of the shard's rows (bf16) and dQ [H, M, D] (fp32,
+    bitwise the same on every rank).  Four phases with one all-gather of a
+    small fp32 buffer between two of them."""
+    torch = b._torch()
+    rank, world = _group_info(group)
+    B, H, N, D = K.shape
+    M = Q.shape[1]
+    dev = K.device
+    lib = b.load_library()
+    dK = torch.empty_like(K) if dK is None else dK
+    dV = torch.empty_like(K) if dV is None else dV
+    dQ = torch.empty((H, M, D), dtype=torch.float32, device=dev) if dQ is None else dQ
+    nbytes = b.flare_workspace_bytes(b.FLARE_VARIANT_FLARE_BWD, B, H, N, M, D)
+    ws = b._workspace(workspace, nbytes, dev)
+    if stream is not None and K.is_cuda:
+        ws.record_stream(stream)
+    st = b._stream_ptr(stream, dev)
+    ins = [b._ptr(t) for t in (K, V, Q, dY)]
+    outs = [b._ptr(t) for t in (dK, dV, dQ)]
+    gathered = None
+    for phase in range(FLARE_CP_BWD_PHASES_FLARE):
+        exch = None
+        if phase < FLARE_CP_BWD_PHASES_FLARE - 1:
+            nb = lib.flare_cp_bwd_exchange_bytes(phase, B, H, N, M, D)
+            if nb == 0:
+                raise ValueError("unsupported sizes")
+            exch = torch.empty(nb // 4, dtype=torch.float32, device=dev)
+        _status(lib.flare_cp_bwd_phase(phase, *ins, b._ptr(gathered), b._ptr(exch), *outs, B, H, N, M, D,
+                                       b._ptr(lengths), rank, world, float(scale), b._ptr(ws), ws.numel(), st),
+                f"flare_cp_bwd_phase({phase})")
+        if exch is not None:
+            gathered = allgather_partials(exch, world, group, stream)
+    _device_status(device_check, workspace is not None, ws, stream, "flare_mixer_cp_bwd")
+    return dK, dV, dQ
 
 
 def flarepp_mixer_cp_bwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, lengths=None, group=None, scale: float = 0.0,

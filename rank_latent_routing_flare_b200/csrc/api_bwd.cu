@@ -60,8 +60,10 @@ BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C) {
   if (pp) {
     bp.off_q0pad = take(static_cast<size_t>(H * M * (D + 4)) * 4);
     bp.off_dqxpad = take(padded);
-    bp.off_dqxdec = take(lat);
   }
+  // FLARE++: the decoder's part of dQ(X) [B*H][M][D]; FLARE: the decoder's
+  // part of dQ, summed over the batch [H][M][D]
+  bp.off_dqxdec = take(lat);
   if (pp) {
     bp.off_g32 = take(static_cast<size_t>(B * N) * 4 * C * 4);
     bp.off_dwpart = take(static_cast<size_t>(bp.dw_splits) * C * 4 * C * 4);
@@ -155,59 +157,118 @@ size_t part_floats(const BwdPlan& bp, int B, int H, int M, int D, bool recompute
   return static_cast<size_t>(B) * H * bp.S * M * (D + (recompute ? 2 : 0));
 }
 
-// FLARE (eq. 5-6) backward on one GPU: dK, dV to bf16 outputs, dQ summed
-// over the batch.
-flare_status flare_bwd_run(const BwdPlan& bp, uint8_t* ws, const float* q, const void* k, const void* v,
-                           const void* dy, uint16_t* dk, uint16_t* dv, float* dq, int B, int H, int N, int M, int D,
-                           const int32_t* lengths, float sc, cudaStream_t s) {
-  const Shard sh{0, N, 1};
+// ---------------------------------------------------------------------------
+// FLARE (eq. 5-6) backward in four phases, like the FLARE++ one below: between
+// two phases every shard's exchange buffer is all-gathered in rank order and
+// merged in ascending (rank, split) order, so every rank holds bitwise the
+// same Z, dZ and dQ.  On one GPU the phases run back to back with the
+// exchanges in the workspace.
+//   0: encoder recompute partials of the shard's tokens            -> E0
+//   1: merge E0 -> Z, L_m; decoder stats; decoder backward         -> E1 = [dZ | dQ_dec partials]
+//   2: dZ, gamma, scale * dQ_dec (summed over the batch); dK, dV of
+//      the shard's tokens (bf16 outputs); encoder dQ partials      -> E2
+//   3: dQ = scale * dQ_enc + the decoder part, summed over the batch
+// ---------------------------------------------------------------------------
+constexpr int kFlPhases = 4;
+
+struct FlArgs {
+  const flare_bf16 *K, *V, *Q, *dY;
+  flare_bf16 *dK, *dV;
+  float* dQ;
+  int B, H, N, M, D;
+  const int32_t* lengths;
+  float sc;
+  Shard sh;
+};
+
+size_t fl_exchange_floats(const BwdPlan& bp, int phase, int B, int H, int M, int D) {
+  switch (phase) {
+    case 0: return part_floats(bp, B, H, M, D, true);
+    case 1: return 2 * part_floats(bp, B, H, M, D, false);
+    case 2: return part_floats(bp, B, H, M, D, false);
+    default: return 0;
+  }
+}
+
+flare_status fl_phase(int phase, const BwdPlan& bp, uint8_t* ws, const FlArgs& a, const float* gathered, float* exch,
+                      cudaStream_t s) {
+  const int B = a.B, H = a.H, N = a.N, M = a.M, D = a.D;
   const long BH = static_cast<long>(B) * H;
+  const float sc = a.sc, c = sc * kLog2e;
+  const int R = a.sh.R;
+  float* q32 = reinterpret_cast<float*>(ws + bp.off_q32);
   float* z32 = reinterpret_cast<float*>(ws + bp.off_z32);
   float* lenc = reinterpret_cast<float*>(ws + bp.off_lenc);
+  float* ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
+  float* dtok = reinterpret_cast<float*>(ws + bp.off_dtok);
   float* dz32 = reinterpret_cast<float*>(ws + bp.off_dz32);
   float* gam = reinterpret_cast<float*>(ws + bp.off_gam);
-  float* pa = reinterpret_cast<float*>(ws + bp.off_pa);
-  float* pb = pa + part_floats(bp, B, H, M, D, false);
-  float* pc = reinterpret_cast<float*>(ws + bp.off_pc);
+  float* dqdec = reinterpret_cast<float*>(ws + bp.off_dqxdec);
   float* qpad = reinterpret_cast<float*>(ws + bp.off_qpad);
   float* zpad = reinterpret_cast<float*>(ws + bp.off_zpad);
   float* dzpad = reinterpret_cast<float*>(ws + bp.off_dzpad);
-  // encoder recompute: Z and the row normalisers
-  LatParams lf = lat_params(bp, ws, q, 0, k, B, H, N, M, D, lengths, sc, sh);
-  lf.v = static_cast<const uint16_t*>(v);
-  lf.part_a = reinterpret_cast<float*>(ws + bp.off_fpart);
-  if (launch_lat(kLatForward, lf, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  flare_status st = lat_merge(lf.part_a, 1, 0, static_cast<int>(BH), M, D, bp.S, z32, lenc, s);
-  if (st != FLARE_OK) return st;
-  if ((st = pad(q, qpad, static_cast<long>(H) * M, D, sc * kLog2e, s)) != FLARE_OK ||
-      (st = pad(z32, zpad, BH * M, D, 1.f, s)) != FLARE_OK)
-    return st;
-  // decoder recompute: L_n and delta_n
-  TokParams tp = tok_params(B, H, N, M, D, 0, lengths, sc, sh);
-  tp.qpad = qpad; tp.zpad = zpad; tp.dzpad = dzpad; tp.lm = lenc; tp.gam = gam;
-  tp.k = static_cast<const uint16_t*>(k);
-  tp.v = static_cast<const uint16_t*>(v);
-  tp.dy = static_cast<const uint16_t*>(dy);
-  tp.ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
-  tp.dtok = reinterpret_cast<float*>(ws + bp.off_dtok);
-  tp.dk16 = dk; tp.dv16 = dv;
-  if (launch_tok(kTokStats, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  // decoder backward, reductions over tokens: dZ and the decoder's dQ
-  LatParams ld = lat_params(bp, ws, q, 0, k, B, H, N, M, D, lengths, sc, sh);
-  ld.zrow = z32; ld.dy = tp.dy; ld.ltok = tp.ltok; ld.dtok = tp.dtok;
-  ld.part_a = pa; ld.part_b = pb;
-  if (launch_lat(kLatDecoder, ld, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  if ((st = lat_sum(B, H, M, D, bp.S, 0, 1.f, pa, nullptr, 1, 0, nullptr, z32, gam, dz32, s)) != FLARE_OK ||
-      (st = pad(dz32, dzpad, BH * M, D, 1.f, s)) != FLARE_OK)
-    return st;
-  // dK (both parts) and dV
-  if (launch_tok(kTokFull, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  // encoder backward: its dQ; dQ = scale * (decoder + encoder parts), summed over the batch
-  LatParams le = lat_params(bp, ws, q, 0, k, B, H, N, M, D, lengths, sc, sh);
-  le.zrow = dz32; le.lrow = lenc; le.grow = gam; le.v = tp.v;
-  le.part_b = pc;
-  if (launch_lat(kLatEncoder, le, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  return lat_sum(B, H, M, D, bp.S, 1, sc, pb, pc, 1, 0, nullptr, nullptr, nullptr, dq, s);
+  const uint16_t* k = reinterpret_cast<const uint16_t*>(a.K);
+  const uint16_t* v = reinterpret_cast<const uint16_t*>(a.V);
+  const uint16_t* dy = reinterpret_cast<const uint16_t*>(a.dY);
+  const size_t P = part_floats(bp, B, H, M, D, false);
+  const size_t stride = fl_exchange_floats(bp, phase - 1, B, H, M, D);  // of the gathered buffers
+  flare_status st = FLARE_OK;
+  switch (phase) {
+    case 0: {
+      if (cudaMemsetAsync(ws + bp.fwd.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+      const CvtParams cv{static_cast<long>(H) * M * D, reinterpret_cast<const uint16_t*>(a.Q), q32};
+      if (launch_cvt(cv, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+      // eq. 5 recomputed: the encoder partials of this shard
+      LatParams lf = lat_params(bp, ws, q32, 0, k, B, H, N, M, D, a.lengths, sc, a.sh);
+      lf.v = v;
+      lf.part_a = exch;
+      return launch_lat(kLatForward, lf, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+    }
+    case 1: {
+      if ((st = lat_merge(gathered, R, stride, static_cast<int>(BH), M, D, bp.S, z32, lenc, s)) != FLARE_OK ||
+          (st = pad(q32, qpad, static_cast<long>(H) * M, D, c, s)) != FLARE_OK ||
+          (st = pad(z32, zpad, BH * M, D, 1.f, s)) != FLARE_OK)
+        return st;
+      // eq. 6: the decoder's per-token normalisers and delta_n of this shard
+      TokParams tp = tok_params(B, H, N, M, D, 0, a.lengths, sc, a.sh);
+      tp.qpad = qpad; tp.zpad = zpad;
+      tp.k = k; tp.v = v; tp.dy = dy;
+      tp.ltok = ltok; tp.dtok = dtok;
+      if (launch_tok(kTokStats, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+      // decoder backward, reductions over this shard's tokens: dZ and dQ partials
+      LatParams ld = lat_params(bp, ws, q32, 0, k, B, H, N, M, D, a.lengths, sc, a.sh);
+      ld.zrow = z32; ld.dy = dy; ld.ltok = ltok; ld.dtok = dtok;
+      ld.part_a = exch; ld.part_b = exch + P;
+      return launch_lat(kLatDecoder, ld, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+    }
+    case 2: {
+      // dZ and gamma; the decoder's part of dQ, scaled and summed over the batch
+      if ((st = lat_sum(B, H, M, D, bp.S, 0, 1.f, gathered, nullptr, R, stride, nullptr, z32, gam, dz32, s)) !=
+              FLARE_OK ||
+          (st = lat_sum(B, H, M, D, bp.S, 1, sc, gathered + P, nullptr, R, stride, nullptr, nullptr, nullptr, dqdec,
+                        s)) != FLARE_OK ||
+          (st = pad(dz32, dzpad, BH * M, D, 1.f, s)) != FLARE_OK)
+        return st;
+      // dK (both parts) and dV of this shard's tokens
+      TokParams tp = tok_params(B, H, N, M, D, 0, a.lengths, sc, a.sh);
+      tp.qpad = qpad; tp.zpad = zpad; tp.dzpad = dzpad; tp.lm = lenc; tp.gam = gam;
+      tp.k = k; tp.v = v; tp.dy = dy;
+      tp.ltok = ltok; tp.dtok = dtok;
+      tp.dk16 = reinterpret_cast<uint16_t*>(a.dK);
+      tp.dv16 = reinterpret_cast<uint16_t*>(a.dV);
+      if (launch_tok(kTokFull, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+      // encoder backward: its dQ partials
+      LatParams le = lat_params(bp, ws, q32, 0, k, B, H, N, M, D, a.lengths, sc, a.sh);
+      le.zrow = dz32; le.lrow = lenc; le.grow = gam; le.v = v;
+      le.part_b = exch;
+      return launch_lat(kLatEncoder, le, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+    }
+    case 3:
+      // dQ = scale * (decoder + encoder parts), summed over the batch and the shards
+      return lat_sum(B, H, M, D, bp.S, 1, sc, gathered, nullptr, R, stride, dqdec, nullptr, nullptr, a.dQ, s);
+    default:
+      return FLARE_ERR_SHAPE;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -401,6 +462,18 @@ flare_status check_bwd_sizes(int B, int H, int N, int M, int D) {
   return static_cast<long>(B) * H > 65535 ? FLARE_ERR_UNSUPPORTED : FLARE_OK;
 }
 
+// Checks shared by the FLARE backward entry points.
+flare_status check_fl_bwd(const FlArgs& a, const void* workspace) {
+  if (!a.K || !a.V || !a.Q || !a.dY || !a.dK || !a.dV || !a.dQ || !workspace) return FLARE_ERR_NULL;
+  flare_status st = check_bwd_sizes(a.B, a.H, a.N, a.M, a.D);
+  if (st != FLARE_OK) return st;
+  if (!aligned16(a.K) || !aligned16(a.V) || !aligned16(a.Q) || !aligned16(a.dY) || !aligned16(a.dK) ||
+      !aligned16(a.dV) || !aligned16(a.dQ) || !aligned16(a.lengths) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FLARE_ERR_ALIGN;
+  return FLARE_OK;
+}
+
 // Checks shared by the FLARE++ backward entry points.
 flare_status check_pp_bwd(const PpArgs& a, const void* workspace) {
   flare_status st = check_flarepp(a.X, a.Wk, a.Wv, a.Wk_syn, a.Wv_syn, a.Q0, a.dY, a.B, a.N, a.C, a.H, a.M, a.D,
@@ -427,22 +500,48 @@ flare_status flare_mixer_bwd(const flare_bf16* K, const flare_bf16* V, const fla
                              flare_bf16* dK, flare_bf16* dV, float* dQ, int B, int H, int N, int M, int D,
                              const int32_t* lengths, float scale, void* workspace, size_t workspace_bytes,
                              void* stream) {
-  if (!K || !V || !Q || !dY || !dK || !dV || !dQ || !workspace) return FLARE_ERR_NULL;
-  flare_status st = check_bwd_sizes(B, H, N, M, D);
+  const FlArgs a{K, V, Q, dY, dK, dV, dQ, B, H, N, M, D, lengths, resolve_scale(scale, D), Shard{0, N, 1}};
+  flare_status st = check_fl_bwd(a, workspace);
   if (st != FLARE_OK) return st;
-  if (!aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(dY) || !aligned16(dK) || !aligned16(dV) ||
-      !aligned16(dQ) || !aligned16(lengths) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return FLARE_ERR_ALIGN;
   const BwdPlan bp = make_bwd_plan(false, B, H, N, M, D, 0);
   if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  if (cudaMemsetAsync(ws + bp.fwd.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  float* q32 = reinterpret_cast<float*>(ws + bp.off_q32);
-  const CvtParams cv{static_cast<long>(H) * M * D, reinterpret_cast<const uint16_t*>(Q), q32};
-  if (launch_cvt(cv, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  return flare_bwd_run(bp, ws, q32, K, V, dY, reinterpret_cast<uint16_t*>(dK), reinterpret_cast<uint16_t*>(dV), dQ, B,
-                       H, N, M, D, lengths, resolve_scale(scale, D), s);
+  // one shard: the exchanges stay in the workspace (each phase reads the
+  // previous phase's buffer and writes another one)
+  float* ex[kFlPhases - 1] = {reinterpret_cast<float*>(ws + bp.off_fpart), reinterpret_cast<float*>(ws + bp.off_pa),
+                              reinterpret_cast<float*>(ws + bp.off_pc)};
+  for (int ph = 0; ph < kFlPhases; ++ph) {
+    st = fl_phase(ph, bp, ws, a, ph > 0 ? ex[ph - 1] : nullptr, ph < kFlPhases - 1 ? ex[ph] : nullptr, s);
+    if (st != FLARE_OK) return st;
+  }
+  return FLARE_OK;
+}
+
+size_t flare_cp_bwd_exchange_bytes(int phase, int B, int H, int N, int M, int D) {
+  if (phase < 0 || phase >= kFlPhases - 1) return 0;
+  if (check_bwd_sizes(B, H, N, M, D) != FLARE_OK) return 0;
+  return fl_exchange_floats(make_bwd_plan(false, B, H, N, M, D, 0), phase, B, H, M, D) * sizeof(float);
+}
+
+flare_status flare_cp_bwd_phase(int phase, const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q,
+                                const flare_bf16* dY, const float* gathered, float* exchange, flare_bf16* dK,
+                                flare_bf16* dV, float* dQ, int B, int H, int N, int M, int D, const int32_t* lengths,
+                                int rank, int world, float scale, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  if (phase < 0 || phase >= kFlPhases) return FLARE_ERR_SHAPE;
+  if (world < 1 || rank < 0 || rank >= world) return FLARE_ERR_SHAPE;
+  if (static_cast<long>(N) * world >= (1L << 31)) return FLARE_ERR_UNSUPPORTED;
+  if ((phase > 0 && !gathered) || (phase < kFlPhases - 1 && !exchange)) return FLARE_ERR_NULL;
+  if (!aligned16(gathered) || !aligned16(exchange)) return FLARE_ERR_ALIGN;
+  const FlArgs a{K, V, Q, dY, dK, dV, dQ, B, H, N, M, D, lengths, resolve_scale(scale, D),
+                 Shard{rank * N, world * N, world}};
+  flare_status st = check_fl_bwd(a, workspace);
+  if (st != FLARE_OK) return st;
+  const BwdPlan bp = make_bwd_plan(false, B, H, N, M, D, 0);
+  if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
+  return fl_phase(phase, bp, static_cast<uint8_t*>(workspace), a, gathered, exchange,
+                  static_cast<cudaStream_t>(stream));
 }
 
 flare_status flarepp_mixer_bwd(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,

@@ -35,6 +35,7 @@ def test_header_declares_the_abi():
                             "flare_selftest_wait_timeout", "flare_cp_partials_bytes", "flarepp_cp_begin",
                             "flarepp_cp_middle", "flarepp_cp_end", "flare_cp_begin", "flare_cp_end",
                             "flare_cp_exact_bytes", "flarepp_cp_exact", "flare_cp_exact",
+                            "flare_cp_bwd_exchange_bytes", "flare_cp_bwd_phase",
                             "flare_mixer_bwd", "flarepp_mixer_bwd", "flarepp_cp_bwd_exchange_bytes",
                             "flarepp_cp_bwd_phase", "flare_mixer_fwd_inspect", "flarepp_mixer_fwd_inspect",
                             "flare_static_last_device_status", "flare_probe_scratch_bytes",
@@ -323,3 +324,34 @@ def test_cp_backward_valid_call_without_gpu_reports_launch_error():
         pytest.skip("a GPU is present")
     assert cp_bwd_call() == Status.ERR_LAUNCH
     assert cp_bwd_call(phase=6, gathered=A, exchange=None) == Status.ERR_LAUNCH
+
+
+def fl_cp_bwd_call(phase=0, gathered=None, exchange=A, rank=0, world=2, B=1, H=2, N=100, M=32, D=16, ws=W,
+                   ws_bytes=None, dK=A):
+    lib = fl.load_library()
+    if ws_bytes is None:
+        ws_bytes = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLARE_BWD, B, H, N, M, D) or (1 << 40)
+    return lib.flare_cp_bwd_phase(phase, A, A, A, A, gathered, exchange, dK, A, A, B, H, N, M, D, None, rank, world,
+                                  0.0, ws, ws_bytes, None)
+
+
+def test_flare_cp_backward_exchange_sizes():
+    lib = fl.load_library()
+    sizes = [lib.flare_cp_bwd_exchange_bytes(p, 1, 2, 1000, 32, 16) for p in range(5)]
+    assert all(x > 0 and x % 16 == 0 for x in sizes[:3]) and sizes[3] == 0 and sizes[4] == 0
+    assert sizes[1] == 2 * sizes[2]                       # [dZ | dQ] partials
+    assert sizes[0] * 16 == sizes[2] * 18                 # recompute partials carry D + 2 floats per row
+    assert lib.flare_cp_bwd_exchange_bytes(0, 1, 2, 1000, 40, 16) == 0      # M not a multiple of 16
+    assert lib.flare_cp_bwd_exchange_bytes(-1, 1, 2, 1000, 32, 16) == 0
+
+
+def test_flare_cp_backward_argument_errors():
+    assert fl_cp_bwd_call(phase=4) == Status.ERR_SHAPE
+    assert fl_cp_bwd_call(phase=-1) == Status.ERR_SHAPE
+    assert fl_cp_bwd_call(rank=2, world=2) == Status.ERR_SHAPE
+    assert fl_cp_bwd_call(phase=1, gathered=None) == Status.ERR_NULL
+    assert fl_cp_bwd_call(phase=0, exchange=None) == Status.ERR_NULL
+    assert fl_cp_bwd_call(phase=3, gathered=A, exchange=None, dK=None) == Status.ERR_NULL
+    assert fl_cp_bwd_call(phase=2, gathered=A + 4) == Status.ERR_ALIGN
+    need = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLARE_BWD, 1, 2, 100, 32, 16)
+    assert fl_cp_bwd_call(ws_bytes=need - 256) == Status.ERR_WORKSPACE

@@ -188,3 +188,76 @@ def test_a_caller_workspace_is_left_for_the_caller_to_check(monkeypatch):
     fake2 = _StatusLib(0)
     _run_single_rank_bwd(monkeypatch, fake2, workspace=ws, device_check=True)
     assert fake2.calls[-1] == ("status",)
+
+
+class _FakeFlareLib(_FakeLib):
+    """Stands in for libflare.so in the FLARE backward: exchange buffers get
+    (rank, phase) markers, and what each phase was handed is recorded."""
+
+    def flare_cp_bwd_exchange_bytes(self, phase, B, H, N, M, D):
+        return 4 * (2 + phase) if 0 <= phase < 3 else 0
+
+    def flare_cp_bwd_phase(self, phase, *args):
+        import ctypes
+        gathered, exchange = args[4], args[5]
+        rank_arg, world_arg = args[15], args[16]   # after B, H, N, M, D and lengths
+        seen = None
+        if gathered:
+            n = 2 * (2 + phase - 1)
+            seen = list((ctypes.c_float * n).from_address(gathered))
+        if exchange:
+            n = 2 + phase
+            buf = (ctypes.c_float * n).from_address(exchange)
+            for i in range(n):
+                buf[i] = 100 * self.rank + 10 * phase + i
+        self.calls.append((phase, rank_arg, world_arg, seen, bool(exchange)))
+        return 0
+
+
+def _flare_bwd_rank_main(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import torch.distributed as dist
+    from rank_latent_routing_flare_b200 import _binding, cp
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        fake = _FakeFlareLib(rank)
+        _binding.load_library = lambda *a, **k: fake
+        _binding.flare_workspace_bytes = lambda *a, **k: 256
+
+        class _Stream:
+            cuda_stream = 0
+        B, H, N, M, D = 1, 2, 4, 16, 16
+        K = torch.zeros((B, H, N, D), dtype=torch.bfloat16)
+        Q = torch.zeros((H, M, D), dtype=torch.bfloat16)
+        cp.flare_mixer_cp_bwd(K, K, Q, K, stream=_Stream())
+        out.put((rank, fake.calls))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_flare_backward_phases_run_in_order_with_rank_ordered_gathers():
+    world = 2
+    ctx = multiprocessing.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_flare_bwd_rank_main, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = sorted(out.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, calls in results:
+        assert calls[-1] == ("status",)
+        calls = calls[:-1]
+        assert [c[0] for c in calls] == list(range(4))
+        assert all(c[1] == rank and c[2] == world for c in calls)
+        assert calls[0][3] is None
+        assert [c[4] for c in calls] == [True] * 3 + [False]
+        for phase in range(1, 4):
+            n = 2 + phase - 1
+            want = [float(10 * (phase - 1) + i) for i in range(n)] + \
+                   [float(100 + 10 * (phase - 1) + i) for i in range(n)]
+            assert calls[phase][3] == want, (rank, phase)

@@ -106,3 +106,90 @@ def test_sharded_backward_matches_oracle(name, N, B, R, lengths):
     if lengths is not None:
         for b, L in enumerate(lengths):
             assert np.all(got["dX"][b, L:] == 0)
+
+
+# ---------------------------------------------------------------------------
+# FLARE (fixed queries): four phases of flare_cp_bwd_phase
+# ---------------------------------------------------------------------------
+
+FL_PHASES = 4
+
+
+def flare_case(B, H, N, M, D, seed, lengths=None):
+    from workloads import Workload, to_bf16_bits
+    rng = np.random.default_rng(seed)
+    w = Workload(name="flare_cp_bwd", variant="flare", B=B, H=H, N=N, C=H * D, D=D, M=M, seed=seed)
+    w.K = to_bf16_bits(rng.standard_normal((B, H, N, D)))
+    w.V = to_bf16_bits(rng.standard_normal((B, H, N, D)))
+    w.Q = to_bf16_bits(rng.standard_normal((H, M, D)))
+    w.lengths = None if lengths is None else np.asarray(lengths, np.int32)
+    return w
+
+
+def emulate_flare(w, dY, R):
+    lib = fl.load_library()
+    B, H, N, M, D = w.B, w.H, w.N // R, w.M, w.D
+    K, V, Q, dYd = dev_bf16(w.K), dev_bf16(w.V), dev_bf16(w.Q), dev_bf16(dY)
+    lengths = None if w.lengths is None else torch.from_numpy(w.lengths).cuda()
+    lp = None if lengths is None else lengths.data_ptr()
+    nbytes = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLARE_BWD, B, H, N, M, D)
+    st = torch.cuda.current_stream().cuda_stream
+    shard = lambda t, r: t[:, :, r * N:(r + 1) * N].contiguous()  # noqa: E731
+    Ks, Vs, dYs = [shard(K, r) for r in range(R)], [shard(V, r) for r in range(R)], [shard(dYd, r) for r in range(R)]
+    wss = [torch.empty(nbytes, dtype=torch.uint8, device="cuda") for _ in range(R)]
+    outs = [{"dK": torch.empty_like(Ks[r]), "dV": torch.empty_like(Ks[r]),
+             "dQ": torch.empty((H, M, D), dtype=torch.float32, device="cuda")} for r in range(R)]
+    gathered = None
+    for phase in range(FL_PHASES):
+        exch = [None] * R
+        if phase < FL_PHASES - 1:
+            nb = lib.flare_cp_bwd_exchange_bytes(phase, B, H, N, M, D)
+            assert nb > 0
+            exch = [torch.empty(nb // 4, dtype=torch.float32, device="cuda") for _ in range(R)]
+        for r in range(R):
+            rc = lib.flare_cp_bwd_phase(
+                phase, Ks[r].data_ptr(), Vs[r].data_ptr(), Q.data_ptr(), dYs[r].data_ptr(),
+                None if gathered is None else gathered.data_ptr(), None if exch[r] is None else exch[r].data_ptr(),
+                outs[r]["dK"].data_ptr(), outs[r]["dV"].data_ptr(), outs[r]["dQ"].data_ptr(), B, H, N, M, D, lp, r, R,
+                0.0, wss[r].data_ptr(), nbytes, st)
+            assert rc == 0, (phase, r, rc)
+        if phase < FL_PHASES - 1:
+            gathered = torch.cat(exch)
+    torch.cuda.synchronize()
+    for r in range(R):
+        assert fl.flare_last_device_status(wss[r]) == fl.Status.OK
+    return outs
+
+
+def test_flare_one_rank_reproduces_the_single_gpu_backward():
+    w = flare_case(2, 2, 1000, 64, 16, seed=5, lengths=[1000, 613])
+    dY = make_upstream_grad(w)
+    outs = emulate_flare(w, dY, 1)[0]
+    lengths = torch.from_numpy(w.lengths).cuda()
+    dK, dV, dQ = fl.flare_mixer_bwd(dev_bf16(w.K), dev_bf16(w.V), dev_bf16(w.Q), dev_bf16(dY), lengths=lengths)
+    torch.cuda.synchronize()
+    assert torch.equal(outs["dK"].view(torch.int16), dK.view(torch.int16))
+    assert torch.equal(outs["dV"].view(torch.int16), dV.view(torch.int16))
+    assert torch.equal(outs["dQ"], dQ)
+
+
+@pytest.mark.parametrize("B,H,N,M,D,R,lengths", [
+    (2, 2, 2048, 64, 16, 2, None),
+    (2, 3, 1536, 128, 16, 3, [1536, 500]),      # ranks 1 and 2 hold no valid token of sample 1
+    (1, 2, 1024, 96, 32, 4, None),              # D = 32
+])
+def test_flare_sharded_backward_matches_oracle(B, H, N, M, D, R, lengths):
+    w = flare_case(B, H, N, M, D, seed=N + R, lengths=lengths)
+    dY = make_upstream_grad(w)
+    outs = emulate_flare(w, dY, R)
+    for r in range(1, R):
+        assert torch.equal(outs[r]["dQ"], outs[0]["dQ"]), r
+    got = {"dK": np.concatenate([host_f64(outs[r]["dK"]) for r in range(R)], axis=2),
+           "dV": np.concatenate([host_f64(outs[r]["dV"]) for r in range(R)], axis=2),
+           "dQ": host_f64(outs[0]["dQ"])}
+    ref = oracle.backward_workload(w, dY)
+    for k in ("dK", "dV", "dQ"):
+        check(got[k], ref[k], f"flare {B}x{H}x{N} M={M} D={D} R={R} {k}")
+    if lengths is not None:
+        for b, L in enumerate(lengths):
+            assert np.all(got["dK"][b, :, L:] == 0) and np.all(got["dV"][b, :, L:] == 0)
