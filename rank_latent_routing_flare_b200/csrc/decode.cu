@@ -291,8 +291,8 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
       // P_{q-NB} has been consumed
       auto issue_s = [&](const Cursor& x) -> bool {
         const int buf = x.q % NB, st = x.tile % NST;
-        if (x.cc == 0 && !mbar_wait(k_full + st, (x.tile / NST) & 1, wc)) return false;
-        if (x.q >= NB && !mbar_wait(pv_done + buf, ((x.q - NB) / NB) & 1, wc)) return false;
+        if (x.cc == 0 && !mbar_wait_mma(k_full + st, (x.tile / NST) & 1, wc)) return false;
+        if (x.q >= NB && !mbar_wait_mma(pv_done + buf, ((x.q - NB) / NB) & 1, wc)) return false;
         tc_fence_after();
         const uint32_t idesc_s = x.cc == nc - 1 ? idesc_last : idesc_full;
         const uint64_t kd = k_desc + static_cast<uint64_t>(st) * (Cfg::KT_B >> 4);
@@ -307,8 +307,8 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
       // tile's first chunk, has read the previous tile's Y)
       auto issue_pv = [&](const Cursor& x) -> bool {
         const int buf = x.q % NB;
-        if (!mbar_wait(p_full + buf, (x.q / NB) & 1, wc)) return false;
-        if (x.cc == 0 && x.tile >= 1 && !mbar_wait(y_free, (x.tile - 1) & 1, wc)) return false;
+        if (!mbar_wait_mma(p_full + buf, (x.q / NB) & 1, wc)) return false;
+        if (x.cc == 0 && x.tile >= 1 && !mbar_wait_mma(y_free, (x.tile - 1) & 1, wc)) return false;
         tc_fence_after();
         const uint64_t step = static_cast<uint64_t>(x.cc) * CH_STEP;
         const uint64_t zd = z_desc + step - (step << 16);
@@ -323,7 +323,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
         return true;
       };
       Cursor cs{0, 0, 0}, cp{0, 0, 0};
-      bool ok = mbar_wait(qz_full, 0, wc) && issue_s(cs);
+      bool ok = mbar_wait_mma(qz_full, 0, wc) && issue_s(cs);
       advance(cs);
       if (ok && total > 1) ok = issue_s(cs);
       advance(cs);

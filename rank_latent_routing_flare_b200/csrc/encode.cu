@@ -185,8 +185,8 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
       // S_i into buffer i % NB, once tile i has landed and P_{i-NB} has been consumed
       auto issue_s = [&](int i) -> bool {
         const int st = i % NST, buf = i % NB;
-        if (!mbar_wait(kv_full + st, (i / NST) & 1, wc)) return false;
-        if (i >= NB && !mbar_wait(pv_done + buf, ((i - NB) / NB) & 1, wc)) return false;
+        if (!mbar_wait_mma(kv_full + st, (i / NST) & 1, wc)) return false;
+        if (i >= NB && !mbar_wait_mma(pv_done + buf, ((i - NB) / NB) & 1, wc)) return false;
         tc_fence_after();
         const uint64_t kd = k_desc + static_cast<uint64_t>((st * Cfg::TILE_B) >> 4);
 #pragma unroll
@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
       // O += P_i [V_i | 1] once every softmax warp has stored P_i
       auto issue_pv = [&](int i) -> bool {
         const int buf = i % NB;
-        if (!mbar_wait(p_full + buf, (i / NB) & 1, wc)) return false;
+        if (!mbar_wait_mma(p_full + buf, (i / NB) & 1, wc)) return false;
         tc_fence_after();
         const uint64_t vd = v_desc + static_cast<uint64_t>(((i % NST) * 2 * Cfg::TILE_B) >> 4);
 #pragma unroll
@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
         umma_commit(pv_done + buf);
         return true;
       };
-      bool ok = mbar_wait(q_full, 0, wc) && issue_s(0);
+      bool ok = mbar_wait_mma(q_full, 0, wc) && issue_s(0);
       if (ok && ntiles > 1) ok = issue_s(1);
       for (int i = 0; ok && i < ntiles; ++i) {
         ok = issue_pv(i);

@@ -99,6 +99,51 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// Wait of the single MMA-issuing thread.  A failed poll is followed by a
+// pause (FLARE_MMA_WAIT_SLEEP_NS nanoseconds, or a suspend-time hint of
+// FLARE_MMA_WAIT_HINT_NS on the poll itself), so that the polling does not
+// take the issue slots of the softmax warp that shares its sub-partition.
+#ifndef FLARE_MMA_WAIT_SLEEP_NS
+#define FLARE_MMA_WAIT_SLEEP_NS 0
+#endif
+#ifndef FLARE_MMA_WAIT_HINT_NS
+#define FLARE_MMA_WAIT_HINT_NS 0
+#endif
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_mma(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  uint32_t spins = 0;
+  while (true) {
+#if FLARE_MMA_WAIT_SLEEP_NS > 0
+    __nanosleep(FLARE_MMA_WAIT_SLEEP_NS);
+#endif
+#if FLARE_MMA_WAIT_HINT_NS > 0
+    if (mbar_try_wait_hint(bar, parity, FLARE_MMA_WAIT_HINT_NS)) return true;
+#else
+    if (mbar_try_wait(bar, parity)) return true;
+#endif
+    if ((++spins & 15u) == 0) {
+      if (*w.abort) return false;
+      if (global_timer_ns() - t0 > w.timeout_ns) {
+        atomicOr(w.gerr, FLARE_DEV_TIMEOUT);
+        *w.abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // Warp-collective wait (all 32 lanes call it): the verdict is made uniform
 // across the warp so that a following .sync.aligned instruction is never
 // executed by part of a warp.
