@@ -8,6 +8,7 @@ the synthesised queries, both log-sum-exp merges and the decode.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     python bench.py --backward [--workload NAME] ...   # the backward: its own JSON line
+    python bench.py --train [--workload NAME] ...      # a training step (forward + backward)
 
 Prints one JSON line (rank 0).  ``value`` is whole-job token*heads/s with the
 inputs resident in HBM, timed with CUDA events on the launching stream over
@@ -34,6 +35,11 @@ collective).
 FLARE workload) per step with a seeded upstream gradient dY, against the
 backward's own roofline (three exponentials per score, the tf32 tensor term,
 HBM); ``e2e`` then copies the inputs and dY in and every gradient out.
+``--train`` times a training step instead: the training forward
+(``flarepp_mixer_fwd_train``), which keeps its state, and the backward that
+reuses it (``flarepp_mixer_bwd_train``), against the sum of the forward's and
+the backward's rooflines; ``compare`` gives the plain forward + recomputing
+backward on the same inputs, timed after the timed region.
 """
 from __future__ import annotations
 
@@ -307,6 +313,11 @@ def cpu_model():
 BWD_METRIC = "mixer bwd token·heads/s at N=1M (1×B200) and % of roofline (HBM/MMA/MUFU)"
 BWD_LAUNCHES = 24        # kernels per FLARE++ backward call (projections, recompute, gradients, GEMMs)
 BWD_LAUNCHES_FLARE = 12  # kernels per FLARE backward call (recompute, gradients, merges, pads)
+# a training step: the training forward (the forward's kernels) and the
+# training backward (conversions, pads, delta, then the gradient passes)
+TRAIN_LAUNCHES = LAUNCHES_PER_STEP + 21
+TRAIN_LAUNCHES_FLARE = 5 + 12
+TRAIN_METRIC = "mixer training step (fwd+bwd) token·heads/s at N=1M (1×B200) and % of roofline"
 TF32_PER_BF16 = 0.5  # nominal dense tf32 : bf16 tensor throughput
 
 
@@ -368,6 +379,7 @@ def run_backward(args, rank, world, local_rank):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
 
     flare = w.variant == "flare"
+    train = args.train
     dY = to_dev(dY_bits)
     if flare:
         host_inputs = (w.K, w.V, w.Q)
@@ -382,17 +394,42 @@ def run_backward(args, rank, world, local_rank):
     ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     grads = None
+    Y = torch.empty((w.B, w.H, w.N, w.D), dtype=torch.bfloat16, device=dev)
 
-    def step():
+    def step(training=train, with_forward=train):
+        """One backward call; with ``with_forward`` a training step: the
+        forward, then the backward (the training pair if ``training``, else
+        the plain forward and the recomputing backward)."""
         nonlocal grads
         if flare:
+            if with_forward:
+                if training:
+                    fl.flare_mixer_fwd_train(*dev_inputs, lengths=lengths, Y=Y, workspace=ws, stream=stream,
+                                             check=False)
+                else:
+                    fl.flare_mixer_fwd(*dev_inputs, lengths=lengths, Y=Y, workspace=ws, stream=stream, check=False)
             out = (None, None, None) if grads is None else (grads["dK"], grads["dV"], grads["dQ"])
-            dK, dV, dQ = fl.flare_mixer_bwd(*dev_inputs, dY, lengths=lengths, workspace=ws, stream=stream,
-                                            dK=out[0], dV=out[1], dQ=out[2], check=False)
+            if training:
+                dK, dV, dQ = fl.flare_mixer_bwd_train(*dev_inputs, dY, ws, lengths=lengths, stream=stream,
+                                                      dK=out[0], dV=out[1], dQ=out[2], check=False)
+            else:
+                dK, dV, dQ = fl.flare_mixer_bwd(*dev_inputs, dY, lengths=lengths, workspace=ws, stream=stream,
+                                                dK=out[0], dV=out[1], dQ=out[2], check=False)
             grads = {"dK": dK, "dV": dV, "dQ": dQ}
         else:
-            grads = fl.flarepp_mixer_bwd(*dev_inputs, dY, lengths=lengths, workspace=ws, stream=stream,
-                                         grads=grads, check=False)
+            if with_forward:
+                if training:
+                    fl.flarepp_mixer_fwd_train(*dev_inputs, lengths=lengths, Y=Y, workspace=ws, stream=stream,
+                                               check=False)
+                else:
+                    fl.flarepp_mixer_fwd(*dev_inputs, lengths=lengths, Y=Y, workspace=ws, stream=stream,
+                                         check=False)
+            if training:
+                grads = fl.flarepp_mixer_bwd_train(*dev_inputs, dY, ws, lengths=lengths, stream=stream,
+                                                   grads=grads, check=False)
+            else:
+                grads = fl.flarepp_mixer_bwd(*dev_inputs, dY, lengths=lengths, workspace=ws, stream=stream,
+                                             grads=grads, check=False)
 
     for _ in range(args.warmup):
         step()
@@ -416,6 +453,21 @@ def run_backward(args, rank, world, local_rank):
     ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world, dev)
     th_per_rank = w.B * w.H * (w.valid_tokens() // w.B if w.lengths is not None else w.N)
     value = whole_job_rate(world, th_per_rank, ms)
+    compare = None
+    if train:
+        # the same training step with the plain forward and the recomputing
+        # backward, for comparison (after the timed region)
+        n_cmp = min(args.steps, 10)
+        step(training=False, with_forward=True)
+        torch.cuda.synchronize(dev)
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(n_cmp):
+            step(training=False, with_forward=True)
+        c1.record(stream)
+        torch.cuda.synchronize(dev)
+        compare = {"recomputing_pair_ms": round(max_over_ranks(c0.elapsed_time(c1) / n_cmp, world, dev), 4),
+                   "steps": n_cmp, "what": "flare(pp)_mixer_fwd + flare(pp)_mixer_bwd on the same inputs"}
 
     peaks = load_peaks()
     rates = pipe_rates(fl, dev)
@@ -424,6 +476,14 @@ def run_backward(args, rank, world, local_rank):
     wk = backward_work(w)
     terms = {"hbm": wk["bytes"] / (peaks["hbm_gbs"] * 1e9), "mma_tf32": wk["flops"] / tf32_peak,
              "mufu": wk["exps"] / mufu_peak}
+    if train:
+        # plus the forward: its exponentials, its bf16 tensor products and its
+        # HBM traffic (the stage model of the forward; FLARE: encode + decode)
+        sw = stage_work(w)
+        keys = ("encode", "merge", "decode") if flare else tuple(sw)
+        terms["hbm"] += sum(sw[k]["bytes"] for k in keys) / (peaks["hbm_gbs"] * 1e9)
+        terms["mma_tf32"] += sum(sw[k]["flops"] for k in keys) / (peaks["bf16_tflops"] * 1e12)
+        terms["mufu"] += sum(sw[k]["exps"] for k in keys) / mufu_peak
     t_roof = max(terms.values())
     bound = {"hbm": "hbm", "mma_tf32": "tensor", "mufu": "alu"}[max(terms, key=terms.get)]
 
@@ -461,14 +521,16 @@ def run_backward(args, rank, world, local_rank):
         if world == 1 and not args.no_cpu_baseline:
             rate, ns, t, threads = oracle_backward_rate(w, dY_bits, args.cpu_seconds)
             cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
-                   "sample": f"fp64 oracle, full {'FLARE' if flare else 'FLARE++'} backward on the first {ns} "
+                   "sample": f"fp64 oracle, full {'FLARE' if flare else 'FLARE++'} backward (which computes the "
+                             f"forward's values on the way) on the first {ns} "
                              f"of {w.N} tokens (B={w.B} H={w.H} M={w.M} D={w.D} C={w.C}) in {t:.1f} s; "
                              f"{cpu_model()}"}
         line = {
-            "metric": BWD_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "metric": TRAIN_METRIC if train else BWD_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "tf32", "data": "synthetic",
-            "config": {"workload": w.name, "pass": "backward", "B": w.B, "N": w.N, "C": w.C, "H": w.H,
+            "config": {"workload": w.name, "pass": "training step" if train else "backward", "B": w.B, "N": w.N, "C": w.C, "H": w.H,
                        "D": w.D, "M": w.M, "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": ("inputs larger than L2 (K, V, dY: " +
                               f"{3 * w.B * w.H * w.N * w.D * 2 / 2**20:.0f} MiB together)" if flare else
@@ -482,7 +544,9 @@ def run_backward(args, rank, world, local_rank):
             "cpu_baseline": cpu,
             "e2e": {"value": whole_job_rate(world, th_per_rank, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": (BWD_LAUNCHES_FLARE if flare else BWD_LAUNCHES) * args.steps,
+            "gpu_launches": ((TRAIN_LAUNCHES_FLARE if flare else TRAIN_LAUNCHES) if train else
+                             (BWD_LAUNCHES_FLARE if flare else BWD_LAUNCHES)) * args.steps,
+            "compare": compare,
             "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)
@@ -549,6 +613,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--backward", action="store_true",
                     help="time the FLARE++ backward (gradients) instead of the forward; its own JSON line")
+    ap.add_argument("--train", action="store_true",
+                    help="with --backward: time a training step, the training forward that keeps its state and "
+                         "the backward that reuses it (and, for comparison, the plain forward + backward)")
     ap.add_argument("--graph", action="store_true",
                     help="time replays of one step captured as a CUDA graph (no per-launch host cost); the "
                          "stage times come from as many eager steps with stage events after the timed region")
@@ -562,7 +629,7 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
-    if args.backward:
+    if args.backward or args.train:
         return run_backward(args, rank, world, local_rank)
 
     import torch

@@ -85,8 +85,10 @@ typedef enum {
   FLARE_ERR_WORKSPACE = 5,   /* workspace smaller than flare_workspace_bytes()    */
   FLARE_ERR_LAUNCH = 6,      /* CUDA error while enqueueing (no sm_100 device...) */
   FLARE_ERR_TIMEOUT = 7,     /* a device-side bounded wait expired                */
-  FLARE_ERR_UNDERFLOW = 8    /* context parallelism without the exact step: a merged
+  FLARE_ERR_UNDERFLOW = 8,   /* context parallelism without the exact step: a merged
                                 row's sums underflowed and were not recomputed  */
+  FLARE_ERR_NO_FORWARD = 9   /* a *_bwd_train call found no *_fwd_train state in
+                                its workspace (none run, or already used)       */
 } flare_status;
 
 /* Variant selector for flare_workspace_bytes(). */
@@ -243,6 +245,59 @@ FLARE_API flare_status flarepp_mixer_bwd(const flare_bf16* X, const flare_bf16* 
                                          float* dWk_syn, float* dWv_syn, float* dQ0, int B, int N, int C, int H,
                                          int M, int D, const int32_t* lengths, float scale, void* workspace,
                                          size_t workspace_bytes, void* stream);
+
+/*
+ * Training pair: a forward that keeps its state for the backward.
+ *
+ * The forward of a training step computes everything the backward would
+ * otherwise recompute: the projections K, V, K~, V~ (FLARE++), Q(X) and Z,
+ * the log-normaliser of every row of the three softmaxes (eq. 8, 10 and 11
+ * of the FLARE++ paper; eq. 5-6 of the FLARE paper) and Y itself.  The
+ * *_fwd_train calls run the forward and keep that state in the BACKWARD's
+ * workspace (flare_workspace_bytes(FLARE_VARIANT_FLAREPP_BWD or
+ * FLARE_VARIANT_FLARE_BWD, ...)); the *_bwd_train calls read it instead of
+ * recomputing the projections, the synthesis and encode passes and the
+ * decoder's statistics.
+ *
+ *   flarepp_mixer_fwd_train   arguments as flarepp_mixer_fwd; writes Y
+ *   flarepp_mixer_bwd_train   arguments as flarepp_mixer_bwd
+ *   flare_mixer_fwd_train     arguments as flare_mixer_fwd; writes Y
+ *   flare_mixer_bwd_train     arguments as flare_mixer_bwd
+ *
+ * A *_bwd_train call must get the same workspace, inputs, sizes, lengths
+ * and scale as the *_fwd_train call before it, with nothing else run in that
+ * workspace in between.  The forward marks the workspace; the backward checks
+ * the mark on the device (no host synchronisation) and clears it when done,
+ * so one forward serves one backward.  A backward without a mark still runs
+ * to its end on whatever the workspace holds and reports
+ * FLARE_ERR_NO_FORWARD through flare_last_device_status; its outputs are then
+ * meaningless.  Inputs changed between the two calls are not detected.
+ *
+ * The backward's score recomputations use the bf16 Q(X) and Z that the
+ * forward's tensor-core products used (flarepp_mixer_bwd recomputes them in
+ * fp32), so its gradients differ from flarepp_mixer_bwd's by rounding, within
+ * the same tolerance against the exact gradients.  Y is written by the
+ * forward exactly as flarepp_mixer_fwd (flare_mixer_fwd) writes it.
+ */
+FLARE_API flare_status flarepp_mixer_fwd_train(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                                               const flare_bf16* Wk_syn, const flare_bf16* Wv_syn,
+                                               const flare_bf16* Q0, flare_bf16* Y, int B, int N, int C, int H,
+                                               int M, int D, const int32_t* lengths, float scale, void* workspace,
+                                               size_t workspace_bytes, void* stream);
+FLARE_API flare_status flarepp_mixer_bwd_train(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                                               const flare_bf16* Wk_syn, const flare_bf16* Wv_syn,
+                                               const flare_bf16* Q0, const flare_bf16* dY, flare_bf16* dX,
+                                               float* dWk, float* dWv, float* dWk_syn, float* dWv_syn, float* dQ0,
+                                               int B, int N, int C, int H, int M, int D, const int32_t* lengths,
+                                               float scale, void* workspace, size_t workspace_bytes, void* stream);
+FLARE_API flare_status flare_mixer_fwd_train(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q,
+                                             flare_bf16* Y, int B, int H, int N, int M, int D,
+                                             const int32_t* lengths, float scale, void* workspace,
+                                             size_t workspace_bytes, void* stream);
+FLARE_API flare_status flare_mixer_bwd_train(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q,
+                                             const flare_bf16* dY, flare_bf16* dK, flare_bf16* dV, float* dQ, int B,
+                                             int H, int N, int M, int D, const int32_t* lengths, float scale,
+                                             void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Context-parallel FLARE++ backward (the token-sharded encoder of section

@@ -16,7 +16,9 @@ from ._binding import (  # noqa: F401
     Status,
     flare_last_device_status,
     flare_mixer_bwd,
+    flare_mixer_bwd_train,
     flare_mixer_fwd,
+    flare_mixer_fwd_train,
     flare_mixer_fwd_static,
     flare_probe_pipe_rates,
     flare_selftest_wait_timeout,
@@ -24,7 +26,9 @@ from ._binding import (  # noqa: F401
     flare_status_string,
     flare_workspace_bytes,
     flarepp_mixer_bwd,
+    flarepp_mixer_bwd_train,
     flarepp_mixer_fwd,
+    flarepp_mixer_fwd_train,
     flarepp_mixer_out_fwd,
     library_path,
     load_library,

@@ -29,6 +29,7 @@ class Status(enum.IntEnum):
     ERR_LAUNCH = 6
     ERR_TIMEOUT = 7
     ERR_UNDERFLOW = 8
+    ERR_NO_FORWARD = 9
 
 
 class FlareError(RuntimeError):
@@ -94,6 +95,14 @@ def load_library(build_if_missing: bool = True):
         lib.flare_mixer_bwd.argtypes = [vp] * 7 + [i] * 5 + [vp, f, vp, sz, vp]
         lib.flarepp_mixer_bwd.restype = i
         lib.flarepp_mixer_bwd.argtypes = [vp] * 13 + [i] * 6 + [vp, f, vp, sz, vp]
+        lib.flarepp_mixer_fwd_train.restype = i
+        lib.flarepp_mixer_fwd_train.argtypes = [vp] * 7 + [i] * 6 + [vp, f, vp, sz, vp]
+        lib.flarepp_mixer_bwd_train.restype = i
+        lib.flarepp_mixer_bwd_train.argtypes = lib.flarepp_mixer_bwd.argtypes
+        lib.flare_mixer_fwd_train.restype = i
+        lib.flare_mixer_fwd_train.argtypes = [vp] * 4 + [i] * 5 + [vp, f, vp, sz, vp]
+        lib.flare_mixer_bwd_train.restype = i
+        lib.flare_mixer_bwd_train.argtypes = lib.flare_mixer_bwd.argtypes
         lib.flarepp_cp_bwd_exchange_bytes.restype = sz
         lib.flarepp_cp_bwd_exchange_bytes.argtypes = [i] * 7
         lib.flare_cp_bwd_exchange_bytes.restype = sz
@@ -332,8 +341,46 @@ def flare_mixer_fwd_static(K, V, Q, lengths=None, scale: float = 0.0, Y=None, st
     return Y
 
 
+def flare_mixer_fwd_train(K, V, Q, lengths=None, scale: float = 0.0, Y=None, workspace=None, stream=None,
+                          check: bool = True, device_check=None):
+    """FLARE forward that keeps its state for ``flare_mixer_bwd_train``:
+    returns (Y, workspace), the workspace (FLARE_VARIANT_FLARE_BWD bytes)
+    holding that state.  Y is the same as flare_mixer_fwd's."""
+    torch = _torch()
+    B, H, N, D = K.shape
+    M = Q.shape[1]
+    if check:
+        _check_dev("K", K, torch.bfloat16)
+        _check_dev("V", V, torch.bfloat16, K.shape)
+        _check_dev("Q", Q, torch.bfloat16, (H, M, D))
+        _check_dev("lengths", lengths, torch.int32, (B,))
+        _check_dev("Y", Y, torch.bfloat16, K.shape)
+    if Y is None:
+        Y = torch.empty_like(K)
+    given = workspace is not None
+    workspace = _workspace(workspace, flare_workspace_bytes(FLARE_VARIANT_FLARE_BWD, B, H, N, M, D), K.device)
+    st = load_library().flare_mixer_fwd_train(_ptr(K), _ptr(V), _ptr(Q), _ptr(Y), B, H, N, M, D, _ptr(lengths),
+                                              float(scale), _ptr(workspace), workspace.numel(),
+                                              _stream_ptr(stream, K.device))
+    if st != 0:
+        raise FlareError(st, "flare_mixer_fwd_train")
+    _device_check(device_check, given, workspace, stream, "flare_mixer_fwd_train")
+    return Y, workspace
+
+
+def flare_mixer_bwd_train(K, V, Q, dY, workspace, lengths=None, scale: float = 0.0, stream=None,
+                          dK=None, dV=None, dQ=None, check: bool = True, device_check: bool = False):
+    """FLARE backward from the state that ``flare_mixer_fwd_train`` left in
+    ``workspace`` (same inputs, lengths and scale).  Returns (dK, dV, dQ) as
+    flare_mixer_bwd.  With ``device_check`` the device status is read after
+    the call (synchronises), which also reports a workspace without a
+    training forward's state (Status.ERR_NO_FORWARD)."""
+    return flare_mixer_bwd(K, V, Q, dY, lengths=lengths, scale=scale, workspace=workspace, stream=stream, dK=dK,
+                           dV=dV, dQ=dQ, check=check, device_check=device_check, _train=True)
+
+
 def flare_mixer_bwd(K, V, Q, dY, lengths=None, scale: float = 0.0, workspace=None, stream=None,
-                    dK=None, dV=None, dQ=None, check: bool = True, device_check=None):
+                    dK=None, dV=None, dQ=None, check: bool = True, device_check=None, _train: bool = False):
     """FLARE backward (gradients of eq. 5-6 given dY).  K, V, dY: [B,H,N,D] bf16;
     Q: [H,M,D] bf16 -> (dK, dV) [B,H,N,D] bf16 and dQ [H,M,D] float32."""
     torch = _torch()
@@ -352,17 +399,58 @@ def flare_mixer_bwd(K, V, Q, dY, lengths=None, scale: float = 0.0, workspace=Non
     nbytes = flare_workspace_bytes(FLARE_VARIANT_FLARE_BWD, B, H, N, M, D)
     given = workspace is not None
     workspace = _workspace(workspace, nbytes, K.device)
-    st = load_library().flare_mixer_bwd(_ptr(K), _ptr(V), _ptr(Q), _ptr(dY), _ptr(dK), _ptr(dV), _ptr(dQ),
-                                        B, H, N, M, D, _ptr(lengths), float(scale), _ptr(workspace),
-                                        workspace.numel(), _stream_ptr(stream, K.device))
+    fn = load_library().flare_mixer_bwd_train if _train else load_library().flare_mixer_bwd
+    where = "flare_mixer_bwd_train" if _train else "flare_mixer_bwd"
+    st = fn(_ptr(K), _ptr(V), _ptr(Q), _ptr(dY), _ptr(dK), _ptr(dV), _ptr(dQ), B, H, N, M, D, _ptr(lengths),
+            float(scale), _ptr(workspace), workspace.numel(), _stream_ptr(stream, K.device))
     if st != 0:
-        raise FlareError(st, "flare_mixer_bwd")
-    _device_check(device_check, given, workspace, stream, "flare_mixer_bwd")
+        raise FlareError(st, where)
+    _device_check(device_check, given, workspace, stream, where)
     return dK, dV, dQ
 
 
+def flarepp_mixer_fwd_train(X, Wk, Wv, Wk_syn, Wv_syn, Q0, lengths=None, scale: float = 0.0, Y=None,
+                            workspace=None, stream=None, check: bool = True, device_check=None):
+    """FLARE++ forward that keeps its state (projections, Q(X), Z, the
+    softmaxes' log-normalisers, fp32 Y) for ``flarepp_mixer_bwd_train``:
+    returns (Y, workspace), the workspace (FLARE_VARIANT_FLAREPP_BWD bytes)
+    holding that state.  Y is the same as flarepp_mixer_fwd's."""
+    torch = _torch()
+    B, N, C = X.shape
+    H, M, D = Q0.shape
+    if check:
+        _check_dev("X", X, torch.bfloat16)
+        for nm, w in (("Wk", Wk), ("Wv", Wv), ("Wk_syn", Wk_syn), ("Wv_syn", Wv_syn)):
+            _check_dev(nm, w, torch.bfloat16, (C, C))
+        _check_dev("Q0", Q0, torch.bfloat16)
+        _check_dev("lengths", lengths, torch.int32, (B,))
+        _check_dev("Y", Y, torch.bfloat16, (B, H, N, D))
+    if Y is None:
+        Y = torch.empty((B, H, N, D), dtype=torch.bfloat16, device=X.device)
+    given = workspace is not None
+    workspace = _workspace(workspace, flare_workspace_bytes(FLARE_VARIANT_FLAREPP_BWD, B, H, N, M, D, C), X.device)
+    st = load_library().flarepp_mixer_fwd_train(
+        _ptr(X), _ptr(Wk), _ptr(Wv), _ptr(Wk_syn), _ptr(Wv_syn), _ptr(Q0), _ptr(Y), B, N, C, H, M, D,
+        _ptr(lengths), float(scale), _ptr(workspace), workspace.numel(), _stream_ptr(stream, X.device))
+    if st != 0:
+        raise FlareError(st, "flarepp_mixer_fwd_train")
+    _device_check(device_check, given, workspace, stream, "flarepp_mixer_fwd_train")
+    return Y, workspace
+
+
+def flarepp_mixer_bwd_train(X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, workspace, lengths=None, scale: float = 0.0,
+                            stream=None, grads=None, check: bool = True, device_check: bool = False):
+    """FLARE++ backward from the state that ``flarepp_mixer_fwd_train`` left
+    in ``workspace`` (same inputs, lengths and scale).  Returns the gradients
+    as flarepp_mixer_bwd.  With ``device_check`` the device status is read
+    after the call (synchronises), which also reports a workspace without a
+    training forward's state (Status.ERR_NO_FORWARD)."""
+    return flarepp_mixer_bwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, lengths=lengths, scale=scale, workspace=workspace,
+                             stream=stream, grads=grads, check=check, device_check=device_check, _train=True)
+
+
 def flarepp_mixer_bwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, lengths=None, scale: float = 0.0, workspace=None,
-                      stream=None, grads=None, check: bool = True, device_check=None):
+                      stream=None, grads=None, check: bool = True, device_check=None, _train: bool = False):
     """FLARE++ backward (gradients of eq. 7-11 given dY [B,H,N,D] bf16).
     Returns a dict: dX [B,N,C] bf16; dWk, dWv, dWk_syn, dWv_syn [C,C] float32;
     dQ0 [H,M,D] float32.  ``grads`` may hold preallocated outputs by name."""
@@ -393,14 +481,16 @@ def flarepp_mixer_bwd(X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, lengths=None, scale: fl
     nbytes = flare_workspace_bytes(FLARE_VARIANT_FLAREPP_BWD, B, H, N, M, D, C)
     given = workspace is not None
     workspace = _workspace(workspace, nbytes, dev)
-    st = load_library().flarepp_mixer_bwd(
-        _ptr(X), _ptr(Wk), _ptr(Wv), _ptr(Wk_syn), _ptr(Wv_syn), _ptr(Q0), _ptr(dY), _ptr(g["dX"]),
-        _ptr(g["dWk"]), _ptr(g["dWv"]), _ptr(g["dWk_syn"]), _ptr(g["dWv_syn"]), _ptr(g["dQ0"]),
-        B, N, C, H, M, D, _ptr(lengths), float(scale), _ptr(workspace), workspace.numel(),
-        _stream_ptr(stream, dev))
+    lib = load_library()
+    fn, where = (lib.flarepp_mixer_bwd_train, "flarepp_mixer_bwd_train") if _train else \
+        (lib.flarepp_mixer_bwd, "flarepp_mixer_bwd")
+    st = fn(_ptr(X), _ptr(Wk), _ptr(Wv), _ptr(Wk_syn), _ptr(Wv_syn), _ptr(Q0), _ptr(dY), _ptr(g["dX"]),
+            _ptr(g["dWk"]), _ptr(g["dWv"]), _ptr(g["dWk_syn"]), _ptr(g["dWv_syn"]), _ptr(g["dQ0"]),
+            B, N, C, H, M, D, _ptr(lengths), float(scale), _ptr(workspace), workspace.numel(),
+            _stream_ptr(stream, dev))
     if st != 0:
-        raise FlareError(st, "flarepp_mixer_bwd")
-    _device_check(device_check, given, workspace, stream, "flarepp_mixer_bwd")
+        raise FlareError(st, where)
+    _device_check(device_check, given, workspace, stream, where)
     return g
 
 

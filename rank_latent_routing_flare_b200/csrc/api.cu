@@ -219,9 +219,10 @@ MergeParams merge_params(const Plan& pl, uint8_t* ws, const float* part, int R, 
 flare_status run_merge(const Plan& pl, uint8_t* ws, const float* part, int R, const void* q, int q_per_batch,
                        const void* k, const void* v, float* out32, uint16_t* out16, int B, int H, int N, int M,
                        int D, const int32_t* lengths, float scale, cudaStream_t st, void* const* ev, int ev_i,
-                       bool pdl, bool allow_exact = true, const float* exact = nullptr) {
-  const MergeParams mp =
+                       bool pdl, bool allow_exact = true, const float* exact = nullptr, float* lse_out = nullptr) {
+  MergeParams mp =
       merge_params(pl, ws, part, R, q, q_per_batch, k, v, out32, out16, B, H, N, M, D, lengths, scale, allow_exact, exact);
+  mp.lse_out = lse_out;
   if (launch_merge(mp, st, pdl) != cudaSuccess || !record(ev, ev_i, st)) return FLARE_ERR_LAUNCH;
   return FLARE_OK;
 }
@@ -239,19 +240,20 @@ flare_status run_cp_exact(const Plan& pl, uint8_t* ws, const float* part, int R,
 // Encoder pass + merge on one GPU (the whole sequence).
 flare_status run_encode(const Plan& pl, uint8_t* ws, const void* q, int q_per_batch, const void* k, const void* v,
                         const float* knorm, float* out32, uint16_t* out16, int B, int H, int N, int M, int D,
-                        const int32_t* lengths, float scale, cudaStream_t st, void* const* ev, int ev0, bool pdl) {
+                        const int32_t* lengths, float scale, cudaStream_t st, void* const* ev, int ev0, bool pdl,
+                        float* lse_out = nullptr) {
   float* part = reinterpret_cast<float*>(ws + pl.off_part);
   flare_status r = run_encode_partials(pl, ws, q, q_per_batch, k, v, knorm, part, B, H, N, M, D, lengths, 0, N,
                                        scale, st, ev, ev0, pdl);
   if (r != FLARE_OK) return r;
   return run_merge(pl, ws, part, 1, q, q_per_batch, k, v, out32, out16, B, H, N, M, D, lengths, scale, st, ev,
-                   ev0 + 1, pdl);
+                   ev0 + 1, pdl, true, nullptr, lse_out);
 }
 
 flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_batch, const uint16_t* z16,
                         const void* k, void* y, int y_token_major, int B, int H, int N, int M, int D,
                         const int32_t* lengths, float scale, cudaStream_t st, bool pdl, int tok_offset = 0,
-                        int n_global = -1, float* y_f32 = nullptr) {
+                        int n_global = -1, float* y_f32 = nullptr, float* ltok_out = nullptr) {
   const long BH = static_cast<long>(B) * H;
   const long G = q_per_batch ? BH : H;
   CUtensorMap tq, tz, tk;
@@ -272,6 +274,7 @@ flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
   dp.y = static_cast<uint16_t*>(y);
   dp.y_token_major = y_token_major;
   dp.y_f32 = y_f32;
+  dp.ltok_out = ltok_out;
   dp.tok_offset = tok_offset;
   dp.n_global = n_global < 0 ? N : n_global;
   dp.err = reinterpret_cast<uint32_t*>(ws + pl.off_err);
@@ -339,6 +342,8 @@ const char* flare_status_string(flare_status s) {
     case FLARE_ERR_TIMEOUT: return "FLARE_ERR_TIMEOUT: a device-side bounded wait expired";
     case FLARE_ERR_UNDERFLOW:
       return "FLARE_ERR_UNDERFLOW: a context-parallel merge found sums that underflowed (not recomputed)";
+    case FLARE_ERR_NO_FORWARD:
+      return "FLARE_ERR_NO_FORWARD: a training backward found no training forward's state in its workspace";
   }
   return "unknown flare_status";
 }
@@ -352,7 +357,7 @@ namespace flare {
 flare_status flare_fwd(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, flare_bf16* Y, int B, int H,
                        int N, int M, int D, const int32_t* lengths, float scale, void* workspace,
                        size_t workspace_bytes, void* stream, float* Z_out, float* Y_f32_out,
-                       void* const* stage_events) {
+                       void* const* stage_events, const FwdStats* stats) {
   if (!K || !V || !Q || !Y || !workspace) return FLARE_ERR_NULL;
   flare_status st = check_common(B, H, N, M, D);
   if (st != FLARE_OK) return st;
@@ -364,7 +369,7 @@ flare_status flare_fwd(const flare_bf16* K, const flare_bf16* V, const flare_bf1
   const float sc = resolve_scale(scale, D);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  if (cudaMemsetAsync(ws + pl.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  if (cudaMemsetAsync(ws + pl.off_err, 0, kErrClearBytes, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   if (!record(stage_events, 0, s)) return FLARE_ERR_LAUNCH;
   KnormParams kp{B * H, N, D, pl.G32, reinterpret_cast<const uint16_t*>(K), reinterpret_cast<float*>(ws + pl.off_kn)};
   if (launch_knorm(kp, s) != cudaSuccess || !record(stage_events, 1, s)) return FLARE_ERR_LAUNCH;
@@ -373,9 +378,11 @@ flare_status flare_fwd(const flare_bf16* K, const flare_bf16* V, const flare_bf1
   // kernels after the first start early (programmatic launch) unless stage
   // events sit between them
   const bool pdl = stage_events == nullptr;
-  st = run_encode(pl, ws, Q, 0, K, V, kp.knorm, z32, z16, B, H, N, M, D, lengths, sc, s, stage_events, 2, pdl);
+  st = run_encode(pl, ws, Q, 0, K, V, kp.knorm, z32, z16, B, H, N, M, D, lengths, sc, s, stage_events, 2, pdl,
+                  stats ? stats->lenc : nullptr);
   if (st != FLARE_OK) return st;
-  st = run_decode(pl, ws, Q, 0, z16, K, Y, 0, B, H, N, M, D, lengths, sc, s, pdl, 0, -1, Y_f32_out);
+  st = run_decode(pl, ws, Q, 0, z16, K, Y, 0, B, H, N, M, D, lengths, sc, s, pdl, 0, -1, Y_f32_out,
+                  stats ? stats->ltok : nullptr);
   if (st != FLARE_OK) return st;
   return record(stage_events, 4, s) ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
@@ -389,7 +396,7 @@ flare_status flare_mixer_fwd_profiled(const flare_bf16* K, const flare_bf16* V, 
                                       void* workspace, size_t workspace_bytes, void* stream, float* Z_out,
                                       void* const* stage_events) {
   return flare_fwd(K, V, Q, Y, B, H, N, M, D, lengths, scale, workspace, workspace_bytes, stream, Z_out, nullptr,
-                   stage_events);
+                   stage_events, nullptr);
 }
 
 flare_status flare_mixer_fwd_inspect(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, flare_bf16* Y,
@@ -398,7 +405,7 @@ flare_status flare_mixer_fwd_inspect(const flare_bf16* K, const flare_bf16* V, c
                                      float* Y_f32_out) {
   if (!Y_f32_out) return FLARE_ERR_NULL;
   return flare_fwd(K, V, Q, Y, B, H, N, M, D, lengths, scale, workspace, workspace_bytes, stream, Z_out, Y_f32_out,
-                   nullptr);
+                   nullptr, nullptr);
 }
 
 flare_status flare_mixer_fwd(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, flare_bf16* Y, int B,
@@ -496,8 +503,8 @@ flare_status flarepp_run(const Plan& pl, const flare_bf16* X, const flare_bf16* 
                          const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0, void* Y,
                          int y_token_major, int B, int N, int C, int H, int M, int D, const int32_t* lengths,
                          float sc, uint8_t* ws, cudaStream_t s, float* Qx_out, float* Z_out,
-                         void* const* stage_events, float* Y_f32_out = nullptr) {
-  if (cudaMemsetAsync(ws + pl.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+                         void* const* stage_events, float* Y_f32_out, const FwdStats* stats) {
+  if (cudaMemsetAsync(ws + pl.off_err, 0, kErrClearBytes, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   Projected pr;
   flare_status st = flarepp_project(pl, X, Wk, Wv, Wk_syn, Wv_syn, B, N, C, H, D, ws, s, stage_events, &pr);
   if (st != FLARE_OK) return st;
@@ -510,15 +517,18 @@ flare_status flarepp_run(const Plan& pl, const flare_bf16* X, const flare_bf16* 
   // eq. 8: query synthesis with the learned seeds
   float* qx32 = Qx_out ? Qx_out : reinterpret_cast<float*>(ws + pl.off_qx32);
   uint16_t* qx16 = reinterpret_cast<uint16_t*>(ws + pl.off_qx16);
-  st = run_encode(pl, ws, Q0, 0, kt, vt, kn_syn, qx32, qx16, B, H, N, M, D, lengths, sc, s, stage_events, 2, pdl);
+  st = run_encode(pl, ws, Q0, 0, kt, vt, kn_syn, qx32, qx16, B, H, N, M, D, lengths, sc, s, stage_events, 2, pdl,
+                  stats ? stats->lsyn : nullptr);
   if (st != FLARE_OK) return st;
   // eq. 10: encode with the synthesised queries
   float* z32 = Z_out ? Z_out : reinterpret_cast<float*>(ws + pl.off_z32);
   uint16_t* z16 = reinterpret_cast<uint16_t*>(ws + pl.off_z16);
-  st = run_encode(pl, ws, qx16, 1, kk, vv, kn, z32, z16, B, H, N, M, D, lengths, sc, s, stage_events, 4, pdl);
+  st = run_encode(pl, ws, qx16, 1, kk, vv, kn, z32, z16, B, H, N, M, D, lengths, sc, s, stage_events, 4, pdl,
+                  stats ? stats->lenc : nullptr);
   if (st != FLARE_OK) return st;
   // eq. 11: decode
-  st = run_decode(pl, ws, qx16, 1, z16, kk, Y, y_token_major, B, H, N, M, D, lengths, sc, s, pdl, 0, -1, Y_f32_out);
+  st = run_decode(pl, ws, qx16, 1, z16, kk, Y, y_token_major, B, H, N, M, D, lengths, sc, s, pdl, 0, -1, Y_f32_out,
+                  stats ? stats->ltok : nullptr);
   if (st != FLARE_OK) return st;
   return record(stage_events, 6, s) ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
@@ -540,7 +550,7 @@ flare_status flarepp_mixer_fwd_profiled(const flare_bf16* X, const flare_bf16* W
   if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
   return flarepp_run(pl, X, Wk, Wv, Wk_syn, Wv_syn, Q0, Y, 0, B, N, C, H, M, D, lengths, resolve_scale(scale, D),
                      static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream), Qx_out, Z_out,
-                     stage_events);
+                     stage_events, nullptr, nullptr);
 }
 
 flare_status flarepp_mixer_fwd_inspect(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
@@ -557,7 +567,7 @@ flare_status flarepp_mixer_fwd_inspect(const flare_bf16* X, const flare_bf16* Wk
   if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
   return flarepp_run(pl, X, Wk, Wv, Wk_syn, Wv_syn, Q0, Y, 0, B, N, C, H, M, D, lengths, resolve_scale(scale, D),
                      static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream), Qx_out, Z_out, nullptr,
-                     Y_f32_out);
+                     Y_f32_out, nullptr);
 }
 
 flare_status flarepp_mixer_out_fwd(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
@@ -576,7 +586,7 @@ flare_status flarepp_mixer_out_fwd(const flare_bf16* X, const flare_bf16* Wk, co
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint16_t* ycat = reinterpret_cast<uint16_t*>(ws + pl.off_ycat);  // [B][N][C], heads side by side
   st = flarepp_run(pl, X, Wk, Wv, Wk_syn, Wv_syn, Q0, ycat, 1, B, N, C, H, M, D, lengths, resolve_scale(scale, D),
-                   ws, s, nullptr, nullptr, nullptr);
+                   ws, s, nullptr, nullptr, nullptr, nullptr, nullptr);
   if (st != FLARE_OK) return st;
   // Out = concat_h(Y_h) W_O: the same tcgen05 projection with one weight and
   // token-major output rows
@@ -641,7 +651,7 @@ flare_status flarepp_cp_begin(const flare_bf16* X, const flare_bf16* Wk, const f
   if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(ws + pl.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  if (cudaMemsetAsync(ws + pl.off_err, 0, kErrClearBytes, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   Projected pr;
   if ((st = flarepp_project(pl, X, Wk, Wv, Wk_syn, Wv_syn, B, N, C, H, D, ws, s, nullptr, &pr)) != FLARE_OK)
     return st;
@@ -755,7 +765,7 @@ flare_status flare_cp_begin(const flare_bf16* K, const flare_bf16* V, const flar
   if (workspace_bytes < pl.total) return FLARE_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(ws + pl.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  if (cudaMemsetAsync(ws + pl.off_err, 0, kErrClearBytes, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   KnormParams kp{B * H, N, D, pl.G32, reinterpret_cast<const uint16_t*>(K), reinterpret_cast<float*>(ws + pl.off_kn)};
   if (launch_knorm(kp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   return run_encode_partials(pl, ws, Q, 0, K, V, kp.knorm, partials, B, H, N, M, D, lengths, rank * N, world * N,
@@ -812,6 +822,7 @@ flare_status flare_last_device_status(void* workspace, void* stream) {
   if (word & FLARE_DEV_TIMEOUT) return FLARE_ERR_TIMEOUT;
   if (word & FLARE_DEV_BAD_LENGTH) return FLARE_ERR_SHAPE;
   if (word & FLARE_DEV_UNDERFLOW) return FLARE_ERR_UNDERFLOW;
+  if (word & FLARE_DEV_NO_STATE) return FLARE_ERR_NO_FORWARD;
   return FLARE_OK;
 }
 

@@ -67,6 +67,11 @@ BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C) {
   if (pp) {
     bp.off_g32 = take(static_cast<size_t>(B * N) * 4 * C * 4);
     bp.off_dwpart = take(static_cast<size_t>(bp.dw_splits) * C * 4 * C * 4);
+    // a training forward's fp32 Y ([B*H][N][D]) waits in the gradient rows'
+    // space, which the backward fills only after it has used Y
+    bp.off_y32 = bp.off_g32;
+  } else {
+    bp.off_y32 = take(static_cast<size_t>(BH * N * D) * 4);
   }
   bp.total = off;
   return bp;
@@ -215,7 +220,7 @@ flare_status fl_phase(int phase, const BwdPlan& bp, uint8_t* ws, const FlArgs& a
   flare_status st = FLARE_OK;
   switch (phase) {
     case 0: {
-      if (cudaMemsetAsync(ws + bp.fwd.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+      if (cudaMemsetAsync(ws + bp.fwd.off_err, 0, kErrClearBytes, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
       const CvtParams cv{static_cast<long>(H) * M * D, reinterpret_cast<const uint16_t*>(a.Q), q32};
       if (launch_cvt(cv, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
       // eq. 5 recomputed: the encoder partials of this shard
@@ -345,7 +350,7 @@ flare_status pp_phase(int phase, const BwdPlan& bp, uint8_t* ws, const PpArgs& a
   flare_status st = FLARE_OK;
   switch (phase) {
     case 0: {
-      if (cudaMemsetAsync(ws + bp.fwd.off_err, 0, 8, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+      if (cudaMemsetAsync(ws + bp.fwd.off_err, 0, kErrClearBytes, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
       // eq. 7 and 9: the projections, recomputed (tcgen05, as in the forward)
       Projected pr;
       if ((st = flarepp_project(bp.fwd, a.X, a.Wk, a.Wv, a.Wk_syn, a.Wv_syn, B, N, C, H, D, ws, s, nullptr, &pr)) !=
@@ -569,6 +574,166 @@ flare_status flarepp_mixer_bwd(const flare_bf16* X, const flare_bf16* Wk, const 
     if (st != FLARE_OK) return st;
   }
   return FLARE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Training pair: a forward that keeps, in the backward's workspace, what the
+// backward would otherwise recompute (the projections, Q(X) and Z, the row
+// log-normalisers of every softmax and the fp32 Y), and the backward that
+// uses it.  The scores of the backward's passes then use the bf16 Q(X) and Z
+// that the forward's tensor-core products used, so that the saved
+// normalisers fit them.
+// ---------------------------------------------------------------------------
+namespace {
+
+flare_status set_train_tag(uint8_t* ws, const BwdPlan& bp, int value, cudaStream_t s) {
+  return cudaMemsetAsync(ws + bp.fwd.off_err + kTrainMarkOffset, value, 4, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+}
+
+flare_status widen(const uint16_t* src, float* dst, long n, cudaStream_t s) {
+  const CvtParams cv{n, src, dst};
+  return launch_cvt(cv, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+}
+
+flare_status delta(const BwdPlan& bp, uint8_t* ws, const flare_bf16* dY, int B, int H, int N, int D,
+                   const int32_t* lengths, cudaStream_t s) {
+  DeltaParams dp{};
+  dp.B = B; dp.H = H; dp.N = N; dp.D = D;
+  dp.tok_offset = 0; dp.n_global = N;
+  dp.lengths = lengths;
+  dp.y32 = reinterpret_cast<const float*>(ws + bp.off_y32);
+  dp.dy = reinterpret_cast<const uint16_t*>(dY);
+  dp.dtok = reinterpret_cast<float*>(ws + bp.off_dtok);
+  dp.tag = reinterpret_cast<const uint32_t*>(ws + bp.fwd.off_err + kTrainMarkOffset);
+  dp.err = reinterpret_cast<uint32_t*>(ws + bp.fwd.off_err);
+  return launch_delta(dp, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+}
+
+}  // namespace
+
+flare_status flarepp_mixer_fwd_train(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                                     const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0,
+                                     flare_bf16* Y, int B, int N, int C, int H, int M, int D, const int32_t* lengths,
+                                     float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  flare_status st = check_flarepp(X, Wk, Wv, Wk_syn, Wv_syn, Q0, Y, B, N, C, H, M, D, lengths, workspace, nullptr,
+                                  nullptr);
+  if (st != FLARE_OK) return st;
+  if ((st = check_bwd_sizes(B, H, N, M, D)) != FLARE_OK) return st;
+  const BwdPlan bp = make_bwd_plan(true, B, H, N, M, D, C);
+  if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FwdStats fs;
+  fs.lsyn = reinterpret_cast<float*>(ws + bp.off_lsyn);
+  fs.lenc = reinterpret_cast<float*>(ws + bp.off_lenc);
+  fs.ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
+  st = flarepp_run(bp.fwd, X, Wk, Wv, Wk_syn, Wv_syn, Q0, Y, 0, B, N, C, H, M, D, lengths, resolve_scale(scale, D), ws,
+                   s, nullptr, nullptr, nullptr, reinterpret_cast<float*>(ws + bp.off_y32), &fs);
+  if (st != FLARE_OK) return st;
+  return set_train_tag(ws, bp, kTrainStateByte, s);
+}
+
+flare_status flarepp_mixer_bwd_train(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                                     const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0,
+                                     const flare_bf16* dY, flare_bf16* dX, float* dWk, float* dWv, float* dWk_syn,
+                                     float* dWv_syn, float* dQ0, int B, int N, int C, int H, int M, int D,
+                                     const int32_t* lengths, float scale, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  const PpArgs a{X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, dX, dWk, dWv, dWk_syn, dWv_syn, dQ0,
+                 B, N, C, H, M, D, lengths, resolve_scale(scale, D), Shard{0, N, 1}};
+  flare_status st = check_pp_bwd(a, workspace);
+  if (st != FLARE_OK) return st;
+  const BwdPlan bp = make_bwd_plan(true, B, H, N, M, D, C);
+  if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const long BH = static_cast<long>(B) * H;
+  const float c = a.sc * 1.4426950408889634f;
+  if (cudaMemsetAsync(ws + bp.fwd.off_err, 0, kErrWordBytes, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  float* q32 = reinterpret_cast<float*>(ws + bp.off_q32);
+  float* qx32 = reinterpret_cast<float*>(ws + bp.off_qx32);
+  float* z32 = reinterpret_cast<float*>(ws + bp.off_z32);
+  // what the forward kept: Q0, Q(X) and Z as the bf16 values its products used
+  if ((st = widen(reinterpret_cast<const uint16_t*>(Q0), q32, static_cast<long>(H) * M * D, s)) != FLARE_OK ||
+      (st = widen(reinterpret_cast<const uint16_t*>(ws + bp.fwd.off_qx16), qx32, BH * M * D, s)) != FLARE_OK ||
+      (st = widen(reinterpret_cast<const uint16_t*>(ws + bp.fwd.off_z16), z32, BH * M * D, s)) != FLARE_OK ||
+      (st = pad(qx32, reinterpret_cast<float*>(ws + bp.off_qpad), BH * M, D, c, s)) != FLARE_OK ||
+      (st = pad(z32, reinterpret_cast<float*>(ws + bp.off_zpad), BH * M, D, 1.f, s)) != FLARE_OK ||
+      (st = delta(bp, ws, dY, B, H, N, D, lengths, s)) != FLARE_OK)
+    return st;
+  // the decoder backward (phase 2 of the seven, after its statistics)
+  float* pa = reinterpret_cast<float*>(ws + bp.off_pa);
+  LatParams ld = lat_params(bp, ws, qx32, 1, ws + bp.fwd.off_kp, B, H, N, M, D, lengths, a.sc, a.sh);
+  ld.zrow = z32;
+  ld.dy = reinterpret_cast<const uint16_t*>(dY);
+  ld.ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
+  ld.dtok = reinterpret_cast<float*>(ws + bp.off_dtok);
+  ld.part_a = pa;
+  ld.part_b = pa + part_floats(bp, B, H, M, D, false);
+  if (launch_lat(kLatDecoder, ld, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  float* ex[kPpPhases - 1] = {nullptr, nullptr, pa, reinterpret_cast<float*>(ws + bp.off_pc),
+                              reinterpret_cast<float*>(ws + bp.off_pc), reinterpret_cast<float*>(ws + bp.off_dwpart)};
+  for (int ph = 3; ph < kPpPhases; ++ph) {
+    st = pp_phase(ph, bp, ws, a, ex[ph - 1], ph < kPpPhases - 1 ? ex[ph] : nullptr, s);
+    if (st != FLARE_OK) return st;
+  }
+  return set_train_tag(ws, bp, 0, s);  // the state is used: a second backward needs a new forward
+}
+
+flare_status flare_mixer_fwd_train(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, flare_bf16* Y,
+                                   int B, int H, int N, int M, int D, const int32_t* lengths, float scale,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  if (!K || !V || !Q || !Y || !workspace) return FLARE_ERR_NULL;
+  flare_status st = check_bwd_sizes(B, H, N, M, D);
+  if (st != FLARE_OK) return st;
+  const BwdPlan bp = make_bwd_plan(false, B, H, N, M, D, 0);
+  if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  FwdStats fs;
+  fs.lenc = reinterpret_cast<float*>(ws + bp.off_lenc);
+  fs.ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
+  st = flare_fwd(K, V, Q, Y, B, H, N, M, D, lengths, scale, workspace, workspace_bytes, stream, nullptr,
+                 reinterpret_cast<float*>(ws + bp.off_y32), nullptr, &fs);
+  if (st != FLARE_OK) return st;
+  return set_train_tag(ws, bp, kTrainStateByte, static_cast<cudaStream_t>(stream));
+}
+
+flare_status flare_mixer_bwd_train(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, const flare_bf16* dY,
+                                   flare_bf16* dK, flare_bf16* dV, float* dQ, int B, int H, int N, int M, int D,
+                                   const int32_t* lengths, float scale, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  const FlArgs a{K, V, Q, dY, dK, dV, dQ, B, H, N, M, D, lengths, resolve_scale(scale, D), Shard{0, N, 1}};
+  flare_status st = check_fl_bwd(a, workspace);
+  if (st != FLARE_OK) return st;
+  const BwdPlan bp = make_bwd_plan(false, B, H, N, M, D, 0);
+  if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const long BH = static_cast<long>(B) * H;
+  const float c = a.sc * 1.4426950408889634f;
+  if (cudaMemsetAsync(ws + bp.fwd.off_err, 0, kErrWordBytes, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  float* q32 = reinterpret_cast<float*>(ws + bp.off_q32);
+  float* z32 = reinterpret_cast<float*>(ws + bp.off_z32);
+  if ((st = widen(reinterpret_cast<const uint16_t*>(Q), q32, static_cast<long>(H) * M * D, s)) != FLARE_OK ||
+      (st = widen(reinterpret_cast<const uint16_t*>(ws + bp.fwd.off_z16), z32, BH * M * D, s)) != FLARE_OK ||
+      (st = pad(q32, reinterpret_cast<float*>(ws + bp.off_qpad), static_cast<long>(H) * M, D, c, s)) != FLARE_OK ||
+      (st = pad(z32, reinterpret_cast<float*>(ws + bp.off_zpad), BH * M, D, 1.f, s)) != FLARE_OK ||
+      (st = delta(bp, ws, dY, B, H, N, D, lengths, s)) != FLARE_OK)
+    return st;
+  // the decoder backward (phase 1 of the four, after its statistics)
+  float* pa = reinterpret_cast<float*>(ws + bp.off_pa);
+  LatParams ld = lat_params(bp, ws, q32, 0, K, B, H, N, M, D, lengths, a.sc, a.sh);
+  ld.zrow = z32;
+  ld.dy = reinterpret_cast<const uint16_t*>(dY);
+  ld.ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
+  ld.dtok = reinterpret_cast<float*>(ws + bp.off_dtok);
+  ld.part_a = pa;
+  ld.part_b = pa + part_floats(bp, B, H, M, D, false);
+  if (launch_lat(kLatDecoder, ld, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  float* pc = reinterpret_cast<float*>(ws + bp.off_pc);
+  if ((st = fl_phase(2, bp, ws, a, pa, pc, s)) != FLARE_OK || (st = fl_phase(3, bp, ws, a, pc, nullptr, s)) != FLARE_OK)
+    return st;
+  return set_train_tag(ws, bp, 0, s);
 }
 
 size_t flarepp_cp_bwd_exchange_bytes(int phase, int B, int N, int C, int H, int M, int D) {

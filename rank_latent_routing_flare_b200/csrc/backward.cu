@@ -902,6 +902,27 @@ __global__ void __launch_bounds__(256) cvt_kernel(const CvtParams p) {
   if (i < p.n) p.dst[i] = bf(p.src[i]);
 }
 
+// delta_n = <dY_n, Y_n> (one thread per token of a head); thread 0 of the
+// first block also checks that a training forward left its state.
+template <int D>
+__global__ void __launch_bounds__(256) delta_kernel(const DeltaParams p) {
+  const long i = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i == 0 && *p.tag != kTrainStateTag) atomicOr(p.err, FLARE_DEV_NO_STATE);
+  if (i >= static_cast<long>(p.B) * p.H * p.N) return;
+  const long bh = i / p.N;
+  const int n = static_cast<int>(i % p.N);
+  bool bad = false;
+  const int L = shard_valid_len(p.lengths, static_cast<int>(bh / p.H), p.N, p.tok_offset, p.n_global, &bad);
+  float d = 0.f;
+  if (n < L) {
+    const float* y = p.y32 + i * D;
+    const uint16_t* g = p.dy + i * D;
+#pragma unroll
+    for (int k = 0; k < D; ++k) d = fmaf(bf(g[k]), y[k], d);
+  }
+  p.dtok[i] = d;
+}
+
 unsigned blocks_for(long n, int threads) { return static_cast<unsigned>((n + threads - 1) / threads); }
 
 }  // namespace
@@ -988,6 +1009,13 @@ cudaError_t launch_pad(const PadParams& p, cudaStream_t s) {
 
 cudaError_t launch_cvt(const CvtParams& p, cudaStream_t s) {
   cvt_kernel<<<blocks_for(p.n, 256), 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_delta(const DeltaParams& p, cudaStream_t s) {
+  const unsigned grid = blocks_for(static_cast<long>(p.B) * p.H * p.N, 256);
+  if (p.D == 16) delta_kernel<16><<<grid, 256, 0, s>>>(p);
+  else delta_kernel<32><<<grid, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -133,7 +133,23 @@ struct CvtParams {
   float* dst;
 };
 
+// delta_n = <dY_n, Y_n> per token of one shard from a training forward's fp32
+// Y (0 for padding tokens); also checks the state tag that the forward left.
+struct DeltaParams {
+  int B, H, N, D;
+  int tok_offset, n_global;
+  const int32_t* lengths;
+  const float* y32;             // [B*H][N][D]
+  const uint16_t* dy;           // bf16 [B*H][N][D]
+  float* dtok;                  // [B*H][N]
+  const uint32_t* tag;          // must hold kTrainStateTag
+  uint32_t* err;
+};
+constexpr int kTrainStateByte = 0xA5;               // written with a byte memset
+constexpr uint32_t kTrainStateTag = 0xA5A5A5A5u;    // kTrainStateByte in all four bytes
+
 cudaError_t launch_lat(int mode, const LatParams& p, cudaStream_t s);
+cudaError_t launch_delta(const DeltaParams& p, cudaStream_t s);
 cudaError_t launch_lat_merge(const LatMergeParams& p, cudaStream_t s);
 cudaError_t launch_lat_sum(const LatSumParams& p, cudaStream_t s);
 cudaError_t launch_tok(int mode, const TokParams& p, cudaStream_t s);

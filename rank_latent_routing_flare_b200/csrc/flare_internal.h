@@ -9,6 +9,7 @@
 #define FLARE_DEV_TIMEOUT 0x1u
 #define FLARE_DEV_BAD_LENGTH 0x2u
 #define FLARE_DEV_UNDERFLOW 0x4u   // a merged row lost mass and could not be recomputed exactly
+#define FLARE_DEV_NO_STATE 0x8u    // a backward that reuses a training forward's state found none
 
 namespace flare {
 
@@ -81,6 +82,17 @@ __host__ __device__ constexpr int dec_ctas_per_sm(int D) { return D == 16 ? FLAR
 // chosen by measurement on B200.
 #ifndef FLARE_ENC_POLY_PAIRS
 #define FLARE_ENC_POLY_PAIRS 11
+#endif
+// Encoder K/V ring refills: issued by the MMA thread once a tile's value MMA
+// is done (1), or by the softmax warps in rotation once the scores two tiles
+// later are ready (0).
+#ifndef FLARE_ENC_REFILL_MMA
+#define FLARE_ENC_REFILL_MMA 0
+#endif
+// Decoder key-ring refills: by the MMA thread once a tile's last value MMA
+// is done (1), or by the softmax warps in rotation (0).
+#ifndef FLARE_DEC_REFILL_MMA
+#define FLARE_DEC_REFILL_MMA 0
 #endif
 // Encoder softmax: load the first 16 score columns, start their
 // exponentials while the rest of the tile is read from TMEM.
@@ -166,6 +178,7 @@ struct MergeParams {
   const float* fix;     // context parallelism: every shard's exact partials of the rows that need
                         // them, [n_ranks][B*H*M][D+2] rank-major, or nullptr
   size_t fix_rank_stride;  // floats between consecutive shards' exact partials
+  float* lse_out;       // optional [B*H][M]: L_m = log2 sum_n 2^(c <q_m, k_n>), the row's log-normaliser
 };
 
 // ---------------------------------------------------------------------------
@@ -187,6 +200,7 @@ struct DecodeParams {
   uint16_t* y;          // bf16 [B*H][N][D], or [B][N][H*D] when y_token_major
   int y_token_major;
   float* y_f32;         // optional fp32 copy of Y ([B*H][N][D], the values Y is rounded from), or nullptr
+  float* ltok_out;      // optional [B*H][N]: L_n = log2 sum_m 2^(c <k_n, q_m>) per token (0 for padding)
   uint32_t* fb_count;   // number of listed tokens (zeroed before the decoder runs)
   uint64_t* fb_list;    // tokens (bh * N + n) whose row sum underflowed, capacity B*H*N
   uint32_t* err;

@@ -14,6 +14,16 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 inline long cdiv(long a, long b) { return (a + b - 1) / b; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The first bytes of every workspace: the device error word (offset 0), the
+// decoder's fallback counter (4) and the training forward's mark (8).  Every
+// entry point but the training backward clears all three when it starts, so
+// that any other call in a workspace invalidates a training forward's state;
+// the training backward clears only the first two (kErrWordBytes) and checks
+// the mark on the device.
+constexpr size_t kErrWordBytes = 8;
+constexpr size_t kTrainMarkOffset = 8;
+constexpr size_t kErrClearBytes = 16;
+
 // Workspace layout and launch shapes of the forward.
 struct Plan {
   int S = 1, tps = 1, LB = 1;            // encoder splits, tiles per split, latent blocks
@@ -32,8 +42,8 @@ struct BwdPlan {
   int S = 1, tps = 1, rpb = 32, LB = 1, dw_splits = 1;
   size_t off_q32 = 0, off_qx32 = 0, off_lsyn = 0, off_dqx32 = 0, off_gsyn = 0, off_z32 = 0, off_lenc = 0,
          off_ltok = 0, off_dtok = 0, off_dz32 = 0, off_gam = 0, off_fpart = 0, off_pa = 0, off_pc = 0,
-         off_g32 = 0, off_dwpart = 0, off_qpad = 0, off_q0pad = 0, off_zpad = 0, off_dzpad = 0, off_dqxpad = 0,
-         off_dqxdec = 0, total = 0;
+         off_g32 = 0, off_dwpart = 0, off_y32 = 0, off_qpad = 0, off_q0pad = 0, off_zpad = 0, off_dzpad = 0,
+         off_dqxpad = 0, off_dqxdec = 0, total = 0;
 };
 
 BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C);
@@ -47,6 +57,25 @@ float resolve_scale(float scale, int D);
 flare_status check_flarepp(const void* X, const void* Wk, const void* Wv, const void* Wk_syn, const void* Wv_syn,
                            const void* Q0, const void* Y, int B, int N, int C, int H, int M, int D,
                            const int32_t* lengths, const void* workspace, const float* Qx_out, const float* Z_out);
+
+// Statistics a training forward leaves for the backward (each optional):
+// the row log-normalisers of the synthesis and the encode ([B*H][M]) and the
+// decoder's per-token ones ([B*H][N]), in log2 units.
+struct FwdStats {
+  float *lsyn = nullptr, *lenc = nullptr, *ltok = nullptr;
+};
+
+// The FLARE forward (eq. 5-6) and the FLARE++ pipeline (eq. 7-11) after the
+// argument checks of their entry points; Y_f32_out and stats are optional.
+flare_status flare_fwd(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, flare_bf16* Y, int B, int H,
+                       int N, int M, int D, const int32_t* lengths, float scale, void* workspace,
+                       size_t workspace_bytes, void* stream, float* Z_out, float* Y_f32_out,
+                       void* const* stage_events, const FwdStats* stats);
+flare_status flarepp_run(const Plan& pl, const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
+                         const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0, void* Y,
+                         int y_token_major, int B, int N, int C, int H, int M, int D, const int32_t* lengths,
+                         float sc, uint8_t* ws, cudaStream_t s, float* Qx_out, float* Z_out,
+                         void* const* stage_events, float* Y_f32_out, const FwdStats* stats);
 
 // Outputs of the FLARE++ projections in the workspace.
 struct Projected {

@@ -69,15 +69,6 @@ __device__ ExactPartial exact_partial(const MergeParams& p, const uint16_t* qrow
   return {mx, den, acc};
 }
 
-// Exact encoder row: z = sum_n softmax_n(<q, k_n> * scale) v_n over n < L.
-template <int D>
-__device__ float merge_exact_row(const MergeParams& p, const uint16_t* qrow, const uint16_t* kh,
-                                 const uint16_t* vh, int L, int lane) {
-  if (L <= 0) return 0.f;
-  const ExactPartial e = exact_partial<D>(p, qrow, kh, vh, L, lane);
-  return e.acc / e.den;
-}
-
 // What the split partials of one row (b, h, m) say, identically in every
 // lane: G = log2 of the row's total weight, max over the splits of all
 // shards of U + log2 l (-inf if every sum is zero); has_tokens: some split
@@ -154,14 +145,18 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
   constexpr int NG = 32 / D;
   const int d = lane % D, grp = lane / D;
   float z = 0.f;
+  float lse = -INFINITY;  // log2 of the row's total weight, for lse_out
   const bool can_exact = R == 1 && p.allow_exact;
   if (!rs.has_tokens) {
     z = 0.f;
   } else if (rs.needs_exact && can_exact) {
     const int g = p.q_per_batch ? bh : h;
     const int L = shard_valid_len(p.lengths, b, p.N, 0, p.N, &bad);
-    z = merge_exact_row<D>(p, p.q + (static_cast<size_t>(g) * p.M + m) * D, p.k + static_cast<size_t>(bh) * p.N * D,
-                           p.v + static_cast<size_t>(bh) * p.N * D, L, lane);
+    const ExactPartial e =
+        exact_partial<D>(p, p.q + (static_cast<size_t>(g) * p.M + m) * D, p.k + static_cast<size_t>(bh) * p.N * D,
+                         p.v + static_cast<size_t>(bh) * p.N * D, L, lane);
+    z = L > 0 ? e.acc / e.den : 0.f;
+    lse = e.mx + log2f(e.den);
   } else if (rs.needs_exact && p.fix != nullptr) {
     // every shard's exact partial sums of this row: (mx, den, acc[D]), rank-major
     const float* fr = p.fix + static_cast<size_t>(row) * (D + 2);
@@ -185,6 +180,7 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
       den += __shfl_xor_sync(0xffffffffu, den, o);
     }
     z = num / den;
+    lse = G2 + log2f(den);
   } else if (G > -INFINITY && R * S < kMergeLanesOverSplits) {
     // few splits: the 32 / D lane groups take the splits j = group,
     // group + 32 / D, ..., each lane one value of d
@@ -206,6 +202,7 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
       den += __shfl_xor_sync(0xffffffffu, den, o);
     }
     z = num / den;
+    lse = G + log2f(den);
     if (rs.needs_exact && lane == 0) atomicOr(p.err, FLARE_DEV_UNDERFLOW);
   } else {
     if (G > -INFINITY) {
@@ -242,11 +239,13 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
       for (int k = 0; k < D; ++k)
         if (k == d) mine = num[k];
       z = mine / den;
+      lse = G + log2f(den);
     }
     // a row that needed the exact recomputation, with no exact partials of
     // the other shards at hand, is reported instead
     if (rs.needs_exact && lane == 0) atomicOr(p.err, FLARE_DEV_UNDERFLOW);
   }
+  if (p.lse_out != nullptr && lane == 0) p.lse_out[row] = lse;
   if (lane < D) {
     const size_t o = static_cast<size_t>(row) * D + lane;
     p.out_f32[o] = z;

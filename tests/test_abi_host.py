@@ -39,7 +39,8 @@ def test_header_declares_the_abi():
                             "flare_mixer_bwd", "flarepp_mixer_bwd", "flarepp_cp_bwd_exchange_bytes",
                             "flarepp_cp_bwd_phase", "flare_mixer_fwd_inspect", "flarepp_mixer_fwd_inspect",
                             "flare_static_last_device_status", "flare_probe_scratch_bytes",
-                            "flare_probe_pipe_rates"])
+                            "flare_probe_pipe_rates", "flarepp_mixer_fwd_train", "flarepp_mixer_bwd_train",
+                            "flare_mixer_fwd_train", "flare_mixer_bwd_train"])
 
 
 def test_library_loads_and_exports_every_declared_symbol():
@@ -285,6 +286,48 @@ def test_backward_valid_calls_without_gpu_report_launch_error():
     assert flarepp_bwd_call() == Status.ERR_LAUNCH
     # shared projections: the synthesis weight gradients may be NULL
     assert flarepp_bwd_call(Wks=A, Wvs=A, dWks=None, dWvs=None) == Status.ERR_LAUNCH
+
+
+def test_training_pair_argument_errors():
+    """The training pair takes the backward's workspace for both calls and
+    the backward's argument checks."""
+    lib = fl.load_library()
+    need_f = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLARE_BWD, 1, 2, 100, 32, 16)
+    need_p = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLAREPP_BWD, 1, 4, 100, 32, 16, 64)
+    fwd_f = lambda Y=A, ws=W, nb=need_f, D=16: lib.flare_mixer_fwd_train(A, A, A, Y, 1, 2, 100, 32, D, None, 0.0,
+                                                                         ws, nb, None)
+    fwd_p = lambda Y=A, ws=W, nb=need_p, C=64: lib.flarepp_mixer_fwd_train(A, A, A, A + 0x100, A + 0x200, A, Y, 1,
+                                                                           100, C, 4, 32, 16, None, 0.0, ws, nb,
+                                                                           None)
+    assert fwd_f(Y=None) == Status.ERR_NULL and fwd_p(Y=None) == Status.ERR_NULL
+    assert fwd_f(ws=None) == Status.ERR_NULL and fwd_p(ws=None) == Status.ERR_NULL
+    assert fwd_f(D=64) == Status.ERR_UNSUPPORTED
+    assert fwd_p(C=128) == Status.ERR_SHAPE
+    # the forward's own workspace is too small: the state lives in the backward's
+    small_f = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLARE, 1, 2, 100, 32, 16)
+    small_p = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLAREPP, 1, 4, 100, 32, 16, 64)
+    assert fwd_f(nb=small_f) == Status.ERR_WORKSPACE and fwd_p(nb=small_p) == Status.ERR_WORKSPACE
+    assert fwd_f(nb=need_f - 256) == Status.ERR_WORKSPACE and fwd_p(nb=need_p - 256) == Status.ERR_WORKSPACE
+    bwd_f = lambda dQ=A, nb=need_f: lib.flare_mixer_bwd_train(A, A, A, A, A, A, dQ, 1, 2, 100, 32, 16, None, 0.0, W,
+                                                             nb, None)
+    bwd_p = lambda dX=A, nb=need_p: lib.flarepp_mixer_bwd_train(A, A, A, A + 0x100, A + 0x200, A, A, dX, A, A, A,
+                                                               A, A, 1, 100, 64, 4, 32, 16, None, 0.0, W, nb,
+                                                               None)
+    assert bwd_f(dQ=None) == Status.ERR_NULL and bwd_p(dX=None) == Status.ERR_NULL
+    assert bwd_f(dQ=A + 4) == Status.ERR_ALIGN
+    assert bwd_f(nb=need_f - 256) == Status.ERR_WORKSPACE and bwd_p(nb=need_p - 256) == Status.ERR_WORKSPACE
+    import torch
+    if not torch.cuda.is_available():
+        assert fwd_f() == Status.ERR_LAUNCH and fwd_p() == Status.ERR_LAUNCH
+        assert bwd_f() == Status.ERR_LAUNCH and bwd_p() == Status.ERR_LAUNCH
+
+
+def test_flare_training_workspace_holds_fp32_y():
+    """FLARE's backward workspace grows by the training forward's fp32 Y
+    ([B][H][N][D] floats); FLARE++ keeps it in the gradient rows' space."""
+    a = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLARE_BWD, 1, 2, 10000, 32, 16)
+    b = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLARE_BWD, 1, 2, 20000, 32, 16)
+    assert b - a >= 2 * 10000 * 16 * 4
 
 
 def cp_bwd_call(phase=0, gathered=None, exchange=A, rank=0, world=2, B=1, N=100, C=64, H=4, M=32, D=16, ws=W,
