@@ -314,7 +314,8 @@ BWD_METRIC = "mixer bwd token·heads/s at N=1M (1×B200) and % of roofline (HBM/
 BWD_LAUNCHES = 24        # kernels per FLARE++ backward call (projections, recompute, gradients, GEMMs)
 BWD_LAUNCHES_FLARE = 12  # kernels per FLARE backward call (recompute, gradients, merges, pads)
 # a training step: the training forward (the forward's kernels) and the
-# training backward (conversions, pads, delta, then the gradient passes)
+# training backward (mark check, conversions, pads, decoder statistics and
+# backward, then the gradient passes)
 TRAIN_LAUNCHES = LAUNCHES_PER_STEP + 21
 TRAIN_LAUNCHES_FLARE = 5 + 12
 TRAIN_METRIC = "mixer training step (fwd+bwd) token·heads/s at N=1M (1×B200) and % of roofline"

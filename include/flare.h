@@ -249,15 +249,15 @@ FLARE_API flare_status flarepp_mixer_bwd(const flare_bf16* X, const flare_bf16* 
 /*
  * Training pair: a forward that keeps its state for the backward.
  *
- * The forward of a training step computes everything the backward would
+ * The forward of a training step computes most of what the backward would
  * otherwise recompute: the projections K, V, K~, V~ (FLARE++), Q(X) and Z,
- * the log-normaliser of every row of the three softmaxes (eq. 8, 10 and 11
- * of the FLARE++ paper; eq. 5-6 of the FLARE paper) and Y itself.  The
+ * and the log-normaliser of every row of the synthesis and encode softmaxes
+ * (eq. 8 and 10 of the FLARE++ paper; eq. 5 of the FLARE paper).  The
  * *_fwd_train calls run the forward and keep that state in the BACKWARD's
  * workspace (flare_workspace_bytes(FLARE_VARIANT_FLAREPP_BWD or
  * FLARE_VARIANT_FLARE_BWD, ...)); the *_bwd_train calls read it instead of
- * recomputing the projections, the synthesis and encode passes and the
- * decoder's statistics.
+ * recomputing the projections and the synthesis and encode passes.  The
+ * decoder's per-token statistics (eq. 11; eq. 6) are still recomputed.
  *
  *   flarepp_mixer_fwd_train   arguments as flarepp_mixer_fwd; writes Y
  *   flarepp_mixer_bwd_train   arguments as flarepp_mixer_bwd
@@ -266,18 +266,22 @@ FLARE_API flare_status flarepp_mixer_bwd(const flare_bf16* X, const flare_bf16* 
  *
  * A *_bwd_train call must get the same workspace, inputs, sizes, lengths
  * and scale as the *_fwd_train call before it, with nothing else run in that
- * workspace in between.  The forward marks the workspace; the backward checks
- * the mark on the device (no host synchronisation) and clears it when done,
- * so one forward serves one backward.  A backward without a mark still runs
- * to its end on whatever the workspace holds and reports
- * FLARE_ERR_NO_FORWARD through flare_last_device_status; its outputs are then
- * meaningless.  Inputs changed between the two calls are not detected.
+ * workspace in between.  The forward marks the workspace; every other entry
+ * point clears the mark when it starts, and the backward checks it on the
+ * device (no host synchronisation) and clears it when done, so one forward
+ * serves one backward.  A backward without the mark still runs to its end on
+ * whatever the workspace holds and reports FLARE_ERR_NO_FORWARD through
+ * flare_last_device_status; its outputs are then meaningless.  Inputs changed
+ * between the two calls are not detected.
  *
- * The backward's score recomputations use the bf16 Q(X) and Z that the
- * forward's tensor-core products used (flarepp_mixer_bwd recomputes them in
- * fp32), so its gradients differ from flarepp_mixer_bwd's by rounding, within
- * the same tolerance against the exact gradients.  Y is written by the
- * forward exactly as flarepp_mixer_fwd (flare_mixer_fwd) writes it.
+ * The backward's scores take the bf16 Q(X) that the forward's tensor-core
+ * products took (flarepp_mixer_bwd recomputes Q(X) in fp32), unscaled, with
+ * the scale applied to the fp32 product as in the forward, so that the
+ * forward's normalisers fit them; Z and the synthesis' gamma use the
+ * forward's fp32 Z and Q(X).  The gradients differ from flarepp_mixer_bwd's
+ * by rounding, within the same tolerance against the exact gradients.  Y is
+ * written by the forward exactly as flarepp_mixer_fwd (flare_mixer_fwd)
+ * writes it.
  */
 FLARE_API flare_status flarepp_mixer_fwd_train(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
                                                const flare_bf16* Wk_syn, const flare_bf16* Wv_syn,

@@ -411,8 +411,8 @@ def flare_mixer_bwd(K, V, Q, dY, lengths=None, scale: float = 0.0, workspace=Non
 
 def flarepp_mixer_fwd_train(X, Wk, Wv, Wk_syn, Wv_syn, Q0, lengths=None, scale: float = 0.0, Y=None,
                             workspace=None, stream=None, check: bool = True, device_check=None):
-    """FLARE++ forward that keeps its state (projections, Q(X), Z, the
-    softmaxes' log-normalisers, fp32 Y) for ``flarepp_mixer_bwd_train``:
+    """FLARE++ forward that keeps its state (projections, Q(X), Z and the
+    synthesis and encode log-normalisers) for ``flarepp_mixer_bwd_train``:
     returns (Y, workspace), the workspace (FLARE_VARIANT_FLAREPP_BWD bytes)
     holding that state.  Y is the same as flarepp_mixer_fwd's."""
     torch = _torch()

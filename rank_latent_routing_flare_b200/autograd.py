@@ -6,7 +6,7 @@ Argument marshalling only: the forward calls ``flarepp_mixer_fwd`` /
 statistics from the saved inputs, so only the inputs are kept for the
 backward).  With ``save_state=True`` the training pair runs instead
 (``*_fwd_train`` / ``*_bwd_train``): the forward keeps its projections,
-latents, normalisers and fp32 Y in the backward's workspace, which autograd
+latents and encoder normalisers in the backward's workspace, which autograd
 holds until the backward, and the backward skips their recomputation --
 less time, more memory held between the passes.  Gradients come back in the
 dtype of their inputs (the library's weight and seed gradients are fp32 and

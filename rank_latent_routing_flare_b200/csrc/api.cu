@@ -253,7 +253,7 @@ flare_status run_encode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
 flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_batch, const uint16_t* z16,
                         const void* k, void* y, int y_token_major, int B, int H, int N, int M, int D,
                         const int32_t* lengths, float scale, cudaStream_t st, bool pdl, int tok_offset = 0,
-                        int n_global = -1, float* y_f32 = nullptr, float* ltok_out = nullptr) {
+                        int n_global = -1, float* y_f32 = nullptr) {
   const long BH = static_cast<long>(B) * H;
   const long G = q_per_batch ? BH : H;
   CUtensorMap tq, tz, tk;
@@ -274,7 +274,6 @@ flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
   dp.y = static_cast<uint16_t*>(y);
   dp.y_token_major = y_token_major;
   dp.y_f32 = y_f32;
-  dp.ltok_out = ltok_out;
   dp.tok_offset = tok_offset;
   dp.n_global = n_global < 0 ? N : n_global;
   dp.err = reinterpret_cast<uint32_t*>(ws + pl.off_err);
@@ -381,8 +380,7 @@ flare_status flare_fwd(const flare_bf16* K, const flare_bf16* V, const flare_bf1
   st = run_encode(pl, ws, Q, 0, K, V, kp.knorm, z32, z16, B, H, N, M, D, lengths, sc, s, stage_events, 2, pdl,
                   stats ? stats->lenc : nullptr);
   if (st != FLARE_OK) return st;
-  st = run_decode(pl, ws, Q, 0, z16, K, Y, 0, B, H, N, M, D, lengths, sc, s, pdl, 0, -1, Y_f32_out,
-                  stats ? stats->ltok : nullptr);
+  st = run_decode(pl, ws, Q, 0, z16, K, Y, 0, B, H, N, M, D, lengths, sc, s, pdl, 0, -1, Y_f32_out);
   if (st != FLARE_OK) return st;
   return record(stage_events, 4, s) ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
@@ -527,8 +525,8 @@ flare_status flarepp_run(const Plan& pl, const flare_bf16* X, const flare_bf16* 
                   stats ? stats->lenc : nullptr);
   if (st != FLARE_OK) return st;
   // eq. 11: decode
-  st = run_decode(pl, ws, qx16, 1, z16, kk, Y, y_token_major, B, H, N, M, D, lengths, sc, s, pdl, 0, -1, Y_f32_out,
-                  stats ? stats->ltok : nullptr);
+  st = run_decode(pl, ws, qx16, 1, z16, kk, Y, y_token_major, B, H, N, M, D, lengths, sc, s, pdl, 0, -1,
+                  Y_f32_out);
   if (st != FLARE_OK) return st;
   return record(stage_events, 6, s) ? FLARE_OK : FLARE_ERR_LAUNCH;
 }

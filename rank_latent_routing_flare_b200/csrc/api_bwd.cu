@@ -67,11 +67,6 @@ BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C) {
   if (pp) {
     bp.off_g32 = take(static_cast<size_t>(B * N) * 4 * C * 4);
     bp.off_dwpart = take(static_cast<size_t>(bp.dw_splits) * C * 4 * C * 4);
-    // a training forward's fp32 Y ([B*H][N][D]) waits in the gradient rows'
-    // space, which the backward fills only after it has used Y
-    bp.off_y32 = bp.off_g32;
-  } else {
-    bp.off_y32 = take(static_cast<size_t>(BH * N * D) * 4);
   }
   bp.total = off;
   return bp;
@@ -109,7 +104,8 @@ LatParams lat_params(const BwdPlan& bp, uint8_t* ws, const float* q, int q_per_b
   lp.tok_offset = sh.tok_offset; lp.n_global = sh.n_global;
   lp.q_per_batch = q_per_batch;
   lp.n_splits = bp.S; lp.tiles_per_split = bp.tps; lp.rows_per_block = bp.rpb;
-  lp.c = sc * kLog2e;
+  lp.qmul = sc * kLog2e;
+  lp.smul = 1.f;
   lp.lengths = lengths;
   lp.q = q;
   lp.k = static_cast<const uint16_t*>(k);
@@ -123,7 +119,7 @@ TokParams tok_params(int B, int H, int N, int M, int D, int q_per_batch, const i
   tp.B = B; tp.H = H; tp.N = N; tp.M = M; tp.D = D;
   tp.tok_offset = sh.tok_offset; tp.n_global = sh.n_global;
   tp.q_per_batch = q_per_batch;
-  tp.c = sc * kLog2e;
+  tp.smul = 1.f;
   tp.lengths = lengths;
   return tp;
 }
@@ -149,6 +145,15 @@ flare_status lat_merge(const float* part, int R, size_t rank_stride, int BH, int
   mp.R = R; mp.rank_stride = rank_stride;
   mp.part = part; mp.z = z; mp.lse = lse;
   return launch_lat_merge(mp, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+}
+
+// Exact scores for the gradient modes (see LatParams): the query operand
+// unscaled, the scale applied to the fp32 product.  The training backward
+// uses them so that its scores match the forward's, whose normalisers it
+// reuses.
+void exact_scores(LatParams& lp, float sc) {
+  lp.qmul = 1.f;
+  lp.smul = sc * kLog2e;
 }
 
 flare_status pad(const float* src, float* dst, long rows, int D, float mul, cudaStream_t s) {
@@ -184,6 +189,7 @@ struct FlArgs {
   const int32_t* lengths;
   float sc;
   Shard sh;
+  bool exact = false;  // exact scores (the training backward), see exact_scores
 };
 
 size_t fl_exchange_floats(const BwdPlan& bp, int phase, int B, int H, int M, int D) {
@@ -261,10 +267,12 @@ flare_status fl_phase(int phase, const BwdPlan& bp, uint8_t* ws, const FlArgs& a
       tp.ltok = ltok; tp.dtok = dtok;
       tp.dk16 = reinterpret_cast<uint16_t*>(a.dK);
       tp.dv16 = reinterpret_cast<uint16_t*>(a.dV);
+      if (a.exact) tp.smul = c;
       if (launch_tok(kTokFull, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
       // encoder backward: its dQ partials
       LatParams le = lat_params(bp, ws, q32, 0, k, B, H, N, M, D, a.lengths, sc, a.sh);
       le.zrow = dz32; le.lrow = lenc; le.grow = gam; le.v = v;
+      if (a.exact) exact_scores(le, sc);
       le.part_b = exch;
       return launch_lat(kLatEncoder, le, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
     }
@@ -302,6 +310,7 @@ struct PpArgs {
   const int32_t* lengths;
   float sc;
   Shard sh;
+  bool exact = false;  // exact scores (the training backward), see exact_scores
 };
 
 size_t pp_exchange_floats(const BwdPlan& bp, int phase, int B, int H, int M, int D, int C) {
@@ -403,18 +412,23 @@ flare_status pp_phase(int phase, const BwdPlan& bp, uint8_t* ws, const PpArgs& a
       tp.k = kk; tp.v = vv; tp.dy = reinterpret_cast<const uint16_t*>(a.dY);
       tp.ltok = ltok; tp.dtok = dtok;
       tp.g32 = g32; tp.g_ld = 4 * C; tp.g_col_k = 0; tp.g_col_v = C;
+      if (a.exact) tp.smul = c;
       if (launch_tok(kTokFull, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
       // encoder backward: its dQ(X) partials
       LatParams le = lat_params(bp, ws, qx32, 1, kk, B, H, N, M, D, a.lengths, sc, a.sh);
       le.zrow = dz32; le.lrow = lenc; le.grow = gam; le.v = vv;
+      if (a.exact) exact_scores(le, sc);
       le.part_b = exch;
       return launch_lat(kLatEncoder, le, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
     }
     case 4: {
-      // dQ(X) = scale * (decoder + encoder parts); gamma of the synthesis
-      if ((st = lat_sum(B, H, M, D, bp.S, 0, sc, gathered, nullptr, R, stride, dqxdec, qx32, gsyn, dqx32, s)) !=
+      // dQ(X) = scale * (decoder + encoder parts); gamma of the synthesis,
+      // <dQ(X), Q(X)> with the synthesis' own fp32 output (the training
+      // backward's qx32 holds the bf16 Q(X) that the later passes' scores took)
+      const float* qx_syn = a.exact ? reinterpret_cast<const float*>(ws + bp.fwd.off_qx32) : qx32;
+      if ((st = lat_sum(B, H, M, D, bp.S, 0, sc, gathered, nullptr, R, stride, dqxdec, qx_syn, gsyn, dqx32, s)) !=
               FLARE_OK ||
-          (st = pad(q32, q0pad, static_cast<long>(H) * M, D, c, s)) != FLARE_OK ||
+          (st = pad(q32, q0pad, static_cast<long>(H) * M, D, a.exact ? 1.f : c, s)) != FLARE_OK ||
           (st = pad(dqx32, dqxpad, BH * M, D, 1.f, s)) != FLARE_OK)
         return st;
       // eq. 8 backward with dQ(X) as the upstream gradient: dK~, dV~ rows ...
@@ -422,10 +436,12 @@ flare_status pp_phase(int phase, const BwdPlan& bp, uint8_t* ws, const PpArgs& a
       tp.qpad = q0pad; tp.dzpad = dqxpad; tp.lm = lsyn; tp.gam = gsyn;
       tp.k = kt; tp.v = vt;
       tp.g32 = g32; tp.g_ld = 4 * C; tp.g_col_k = 2 * C; tp.g_col_v = 3 * C;
+      if (a.exact) tp.smul = c;
       if (launch_tok(kTokEncoder, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
       // ... and the partials of dQ0
       LatParams le = lat_params(bp, ws, q32, 0, kt, B, H, N, M, D, a.lengths, sc, a.sh);
       le.zrow = dqx32; le.lrow = lsyn; le.grow = gsyn; le.v = vt;
+      if (a.exact) exact_scores(le, sc);
       le.part_b = exch;
       return launch_lat(kLatEncoder, le, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
     }
@@ -578,16 +594,20 @@ flare_status flarepp_mixer_bwd(const flare_bf16* X, const flare_bf16* Wk, const 
 
 // ---------------------------------------------------------------------------
 // Training pair: a forward that keeps, in the backward's workspace, what the
-// backward would otherwise recompute (the projections, Q(X) and Z, the row
-// log-normalisers of every softmax and the fp32 Y), and the backward that
-// uses it.  The scores of the backward's passes then use the bf16 Q(X) and Z
-// that the forward's tensor-core products used, so that the saved
-// normalisers fit them.
+// backward would otherwise recompute (the projections, Q(X) and Z, and the
+// log-normalisers of the synthesis and encode softmaxes), and the backward
+// that uses it.  The backward's scores then take the bf16 Q(X) that the
+// forward's products used, unscaled, with the scale applied to the fp32
+// product (exact scores), so that the forward's normalisers fit them.  The
+// decoder's per-token statistics are recomputed: delta_n = <dY_n, Y_n> needs
+// Y from the fp32 Z (the forward's Y takes Z in bf16, which moves the
+// gradients of Q0 and W~_K by more than the tolerance).
 // ---------------------------------------------------------------------------
 namespace {
 
-flare_status set_train_tag(uint8_t* ws, const BwdPlan& bp, int value, cudaStream_t s) {
-  return cudaMemsetAsync(ws + bp.fwd.off_err + kTrainMarkOffset, value, 4, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+flare_status set_train_mark(uint8_t* ws, const BwdPlan& bp, int value, cudaStream_t s) {
+  return cudaMemsetAsync(ws + bp.fwd.off_err + kTrainMarkOffset, value, 4, s) == cudaSuccess ? FLARE_OK
+                                                                                             : FLARE_ERR_LAUNCH;
 }
 
 flare_status widen(const uint16_t* src, float* dst, long n, cudaStream_t s) {
@@ -595,18 +615,57 @@ flare_status widen(const uint16_t* src, float* dst, long n, cudaStream_t s) {
   return launch_cvt(cv, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
 
-flare_status delta(const BwdPlan& bp, uint8_t* ws, const flare_bf16* dY, int B, int H, int N, int D,
-                   const int32_t* lengths, cudaStream_t s) {
-  DeltaParams dp{};
-  dp.B = B; dp.H = H; dp.N = N; dp.D = D;
-  dp.tok_offset = 0; dp.n_global = N;
-  dp.lengths = lengths;
-  dp.y32 = reinterpret_cast<const float*>(ws + bp.off_y32);
-  dp.dy = reinterpret_cast<const uint16_t*>(dY);
-  dp.dtok = reinterpret_cast<float*>(ws + bp.off_dtok);
-  dp.tag = reinterpret_cast<const uint32_t*>(ws + bp.fwd.off_err + kTrainMarkOffset);
-  dp.err = reinterpret_cast<uint32_t*>(ws + bp.fwd.off_err);
-  return launch_delta(dp, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+// Start of a training backward: clear the error word (not the mark), check
+// the mark on the device, take Q0 (or Q) and Q(X) as fp32 images of their
+// bf16 values and the forward's fp32 Z, and pad them unscaled.
+flare_status train_prologue(const BwdPlan& bp, uint8_t* ws, const flare_bf16* Q, const uint16_t* qx16, long BH, int H,
+                            int M, int D, cudaStream_t s) {
+  if (cudaMemsetAsync(ws + bp.fwd.off_err, 0, kErrWordBytes, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  const MarkParams mk{reinterpret_cast<const uint32_t*>(ws + bp.fwd.off_err + kTrainMarkOffset),
+                      reinterpret_cast<uint32_t*>(ws + bp.fwd.off_err)};
+  if (launch_check_mark(mk, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  float* q32 = reinterpret_cast<float*>(ws + bp.off_q32);
+  float* z32 = reinterpret_cast<float*>(ws + bp.off_z32);
+  const size_t lat = static_cast<size_t>(BH) * M * D;
+  flare_status st;
+  if ((st = widen(reinterpret_cast<const uint16_t*>(Q), q32, static_cast<long>(H) * M * D, s)) != FLARE_OK) return st;
+  if (cudaMemcpyAsync(z32, ws + bp.fwd.off_z32, lat * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return FLARE_ERR_LAUNCH;
+  const float* qdec = q32;  // FLARE: the learned queries
+  if (qx16 != nullptr) {
+    float* qx32 = reinterpret_cast<float*>(ws + bp.off_qx32);
+    if ((st = widen(qx16, qx32, static_cast<long>(lat), s)) != FLARE_OK) return st;
+    qdec = qx32;
+  }
+  const long qrows = qx16 != nullptr ? BH * M : static_cast<long>(H) * M;
+  if ((st = pad(qdec, reinterpret_cast<float*>(ws + bp.off_qpad), qrows, D, 1.f, s)) != FLARE_OK) return st;
+  return pad(z32, reinterpret_cast<float*>(ws + bp.off_zpad), BH * M, D, 1.f, s);
+}
+
+// The decoder's statistics (L_n, delta_n) and its backward (the dZ and dQ
+// partials into `exch`), exact scores; q: the fp32 queries of the lat pass.
+flare_status train_decoder(const BwdPlan& bp, uint8_t* ws, const float* q, int q_per_batch, const void* k,
+                           const flare_bf16* dY, int B, int H, int N, int M, int D, const int32_t* lengths, float sc,
+                           float* exch, cudaStream_t s) {
+  const Shard sh{0, N, 1};
+  float* ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
+  float* dtok = reinterpret_cast<float*>(ws + bp.off_dtok);
+  TokParams tp = tok_params(B, H, N, M, D, q_per_batch, lengths, sc, sh);
+  tp.smul = sc * kLog2e;
+  tp.qpad = reinterpret_cast<const float*>(ws + bp.off_qpad);
+  tp.zpad = reinterpret_cast<const float*>(ws + bp.off_zpad);
+  tp.k = static_cast<const uint16_t*>(k);
+  tp.dy = reinterpret_cast<const uint16_t*>(dY);
+  tp.ltok = ltok; tp.dtok = dtok;
+  if (launch_tok(kTokStats, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  LatParams ld = lat_params(bp, ws, q, q_per_batch, k, B, H, N, M, D, lengths, sc, sh);
+  exact_scores(ld, sc);
+  ld.zrow = reinterpret_cast<const float*>(ws + bp.off_z32);
+  ld.dy = tp.dy;
+  ld.ltok = ltok; ld.dtok = dtok;
+  ld.part_a = exch;
+  ld.part_b = exch + part_floats(bp, B, H, M, D, false);
+  return launch_lat(kLatDecoder, ld, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
 
 }  // namespace
@@ -626,11 +685,10 @@ flare_status flarepp_mixer_fwd_train(const flare_bf16* X, const flare_bf16* Wk, 
   FwdStats fs;
   fs.lsyn = reinterpret_cast<float*>(ws + bp.off_lsyn);
   fs.lenc = reinterpret_cast<float*>(ws + bp.off_lenc);
-  fs.ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
   st = flarepp_run(bp.fwd, X, Wk, Wv, Wk_syn, Wv_syn, Q0, Y, 0, B, N, C, H, M, D, lengths, resolve_scale(scale, D), ws,
-                   s, nullptr, nullptr, nullptr, reinterpret_cast<float*>(ws + bp.off_y32), &fs);
+                   s, nullptr, nullptr, nullptr, nullptr, &fs);
   if (st != FLARE_OK) return st;
-  return set_train_tag(ws, bp, kTrainStateByte, s);
+  return set_train_mark(ws, bp, kTrainStateByte, s);
 }
 
 flare_status flarepp_mixer_bwd_train(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
@@ -639,8 +697,9 @@ flare_status flarepp_mixer_bwd_train(const flare_bf16* X, const flare_bf16* Wk, 
                                      float* dWv_syn, float* dQ0, int B, int N, int C, int H, int M, int D,
                                      const int32_t* lengths, float scale, void* workspace, size_t workspace_bytes,
                                      void* stream) {
-  const PpArgs a{X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, dX, dWk, dWv, dWk_syn, dWv_syn, dQ0,
-                 B, N, C, H, M, D, lengths, resolve_scale(scale, D), Shard{0, N, 1}};
+  PpArgs a{X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, dX, dWk, dWv, dWk_syn, dWv_syn, dQ0,
+           B, N, C, H, M, D, lengths, resolve_scale(scale, D), Shard{0, N, 1}};
+  a.exact = true;
   flare_status st = check_pp_bwd(a, workspace);
   if (st != FLARE_OK) return st;
   const BwdPlan bp = make_bwd_plan(true, B, H, N, M, D, C);
@@ -648,36 +707,18 @@ flare_status flarepp_mixer_bwd_train(const flare_bf16* X, const flare_bf16* Wk, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const long BH = static_cast<long>(B) * H;
-  const float c = a.sc * 1.4426950408889634f;
-  if (cudaMemsetAsync(ws + bp.fwd.off_err, 0, kErrWordBytes, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  float* q32 = reinterpret_cast<float*>(ws + bp.off_q32);
-  float* qx32 = reinterpret_cast<float*>(ws + bp.off_qx32);
-  float* z32 = reinterpret_cast<float*>(ws + bp.off_z32);
-  // what the forward kept: Q0, Q(X) and Z as the bf16 values its products used
-  if ((st = widen(reinterpret_cast<const uint16_t*>(Q0), q32, static_cast<long>(H) * M * D, s)) != FLARE_OK ||
-      (st = widen(reinterpret_cast<const uint16_t*>(ws + bp.fwd.off_qx16), qx32, BH * M * D, s)) != FLARE_OK ||
-      (st = widen(reinterpret_cast<const uint16_t*>(ws + bp.fwd.off_z16), z32, BH * M * D, s)) != FLARE_OK ||
-      (st = pad(qx32, reinterpret_cast<float*>(ws + bp.off_qpad), BH * M, D, c, s)) != FLARE_OK ||
-      (st = pad(z32, reinterpret_cast<float*>(ws + bp.off_zpad), BH * M, D, 1.f, s)) != FLARE_OK ||
-      (st = delta(bp, ws, dY, B, H, N, D, lengths, s)) != FLARE_OK)
-    return st;
-  // the decoder backward (phase 2 of the seven, after its statistics)
   float* pa = reinterpret_cast<float*>(ws + bp.off_pa);
-  LatParams ld = lat_params(bp, ws, qx32, 1, ws + bp.fwd.off_kp, B, H, N, M, D, lengths, a.sc, a.sh);
-  ld.zrow = z32;
-  ld.dy = reinterpret_cast<const uint16_t*>(dY);
-  ld.ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
-  ld.dtok = reinterpret_cast<float*>(ws + bp.off_dtok);
-  ld.part_a = pa;
-  ld.part_b = pa + part_floats(bp, B, H, M, D, false);
-  if (launch_lat(kLatDecoder, ld, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  float* ex[kPpPhases - 1] = {nullptr, nullptr, pa, reinterpret_cast<float*>(ws + bp.off_pc),
-                              reinterpret_cast<float*>(ws + bp.off_pc), reinterpret_cast<float*>(ws + bp.off_dwpart)};
-  for (int ph = 3; ph < kPpPhases; ++ph) {
-    st = pp_phase(ph, bp, ws, a, ex[ph - 1], ph < kPpPhases - 1 ? ex[ph] : nullptr, s);
-    if (st != FLARE_OK) return st;
-  }
-  return set_train_tag(ws, bp, 0, s);  // the state is used: a second backward needs a new forward
+  float* pc = reinterpret_cast<float*>(ws + bp.off_pc);
+  if ((st = train_prologue(bp, ws, Q0, reinterpret_cast<const uint16_t*>(ws + bp.fwd.off_qx16), BH, H, M, D, s)) !=
+          FLARE_OK ||
+      (st = train_decoder(bp, ws, reinterpret_cast<const float*>(ws + bp.off_qx32), 1, ws + bp.fwd.off_kp, dY, B, H, N,
+                          M, D, lengths, a.sc, pa, s)) != FLARE_OK)
+    return st;
+  // phases 3-6 of the seven (the exchanges stay in the workspace)
+  float* ex[kPpPhases - 1] = {nullptr, nullptr, pa, pc, pc, reinterpret_cast<float*>(ws + bp.off_dwpart)};
+  for (int ph = 3; ph < kPpPhases; ++ph)
+    if ((st = pp_phase(ph, bp, ws, a, ex[ph - 1], ph < kPpPhases - 1 ? ex[ph] : nullptr, s)) != FLARE_OK) return st;
+  return set_train_mark(ws, bp, 0, s);  // the state is used: a second backward needs a new forward
 }
 
 flare_status flare_mixer_fwd_train(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, flare_bf16* Y,
@@ -691,49 +732,32 @@ flare_status flare_mixer_fwd_train(const flare_bf16* K, const flare_bf16* V, con
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   FwdStats fs;
   fs.lenc = reinterpret_cast<float*>(ws + bp.off_lenc);
-  fs.ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
-  st = flare_fwd(K, V, Q, Y, B, H, N, M, D, lengths, scale, workspace, workspace_bytes, stream, nullptr,
-                 reinterpret_cast<float*>(ws + bp.off_y32), nullptr, &fs);
+  st = flare_fwd(K, V, Q, Y, B, H, N, M, D, lengths, scale, workspace, workspace_bytes, stream, nullptr, nullptr,
+                 nullptr, &fs);
   if (st != FLARE_OK) return st;
-  return set_train_tag(ws, bp, kTrainStateByte, static_cast<cudaStream_t>(stream));
+  return set_train_mark(ws, bp, kTrainStateByte, static_cast<cudaStream_t>(stream));
 }
 
 flare_status flare_mixer_bwd_train(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, const flare_bf16* dY,
                                    flare_bf16* dK, flare_bf16* dV, float* dQ, int B, int H, int N, int M, int D,
                                    const int32_t* lengths, float scale, void* workspace, size_t workspace_bytes,
                                    void* stream) {
-  const FlArgs a{K, V, Q, dY, dK, dV, dQ, B, H, N, M, D, lengths, resolve_scale(scale, D), Shard{0, N, 1}};
+  FlArgs a{K, V, Q, dY, dK, dV, dQ, B, H, N, M, D, lengths, resolve_scale(scale, D), Shard{0, N, 1}};
+  a.exact = true;
   flare_status st = check_fl_bwd(a, workspace);
   if (st != FLARE_OK) return st;
   const BwdPlan bp = make_bwd_plan(false, B, H, N, M, D, 0);
   if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const long BH = static_cast<long>(B) * H;
-  const float c = a.sc * 1.4426950408889634f;
-  if (cudaMemsetAsync(ws + bp.fwd.off_err, 0, kErrWordBytes, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  float* q32 = reinterpret_cast<float*>(ws + bp.off_q32);
-  float* z32 = reinterpret_cast<float*>(ws + bp.off_z32);
-  if ((st = widen(reinterpret_cast<const uint16_t*>(Q), q32, static_cast<long>(H) * M * D, s)) != FLARE_OK ||
-      (st = widen(reinterpret_cast<const uint16_t*>(ws + bp.fwd.off_z16), z32, BH * M * D, s)) != FLARE_OK ||
-      (st = pad(q32, reinterpret_cast<float*>(ws + bp.off_qpad), static_cast<long>(H) * M, D, c, s)) != FLARE_OK ||
-      (st = pad(z32, reinterpret_cast<float*>(ws + bp.off_zpad), BH * M, D, 1.f, s)) != FLARE_OK ||
-      (st = delta(bp, ws, dY, B, H, N, D, lengths, s)) != FLARE_OK)
-    return st;
-  // the decoder backward (phase 1 of the four, after its statistics)
   float* pa = reinterpret_cast<float*>(ws + bp.off_pa);
-  LatParams ld = lat_params(bp, ws, q32, 0, K, B, H, N, M, D, lengths, a.sc, a.sh);
-  ld.zrow = z32;
-  ld.dy = reinterpret_cast<const uint16_t*>(dY);
-  ld.ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
-  ld.dtok = reinterpret_cast<float*>(ws + bp.off_dtok);
-  ld.part_a = pa;
-  ld.part_b = pa + part_floats(bp, B, H, M, D, false);
-  if (launch_lat(kLatDecoder, ld, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   float* pc = reinterpret_cast<float*>(ws + bp.off_pc);
-  if ((st = fl_phase(2, bp, ws, a, pa, pc, s)) != FLARE_OK || (st = fl_phase(3, bp, ws, a, pc, nullptr, s)) != FLARE_OK)
+  if ((st = train_prologue(bp, ws, Q, nullptr, static_cast<long>(B) * H, H, M, D, s)) != FLARE_OK ||
+      (st = train_decoder(bp, ws, reinterpret_cast<const float*>(ws + bp.off_q32), 0, K, dY, B, H, N, M, D, lengths,
+                          a.sc, pa, s)) != FLARE_OK ||
+      (st = fl_phase(2, bp, ws, a, pa, pc, s)) != FLARE_OK || (st = fl_phase(3, bp, ws, a, pc, nullptr, s)) != FLARE_OK)
     return st;
-  return set_train_tag(ws, bp, 0, s);
+  return set_train_mark(ws, bp, 0, s);
 }
 
 size_t flarepp_cp_bwd_exchange_bytes(int phase, int B, int N, int C, int H, int M, int D) {

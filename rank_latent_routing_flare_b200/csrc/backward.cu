@@ -112,7 +112,8 @@ __device__ __forceinline__ void stage_bf16(float* dst, const uint16_t* src, int 
 // forward mode keeps MT = 1 for its online softmax), and walks the split's
 // valid tokens in tiles of 64 that the CTA stages in shared memory (double
 // buffered).  Per tile and 8-token column block:
-// scores S = (c Q) K^T on the tensor cores, then
+// scores S = smul (qmul Q) K^T on the tensor cores (qmul smul = scale log2(e);
+// the forward mode takes smul = 1), then
 //   forward:  online softmax over tokens, O += 2^(S - max) V
 //   decoder:  W = 2^(S - L_n), dS = W (Z dY^T - delta_n), dZ += W dY, dQ += dS K
 //   encoder:  W = 2^(S - L_m), dS = W (dZ V^T - gamma_m), dQ += dS K
@@ -168,10 +169,10 @@ __global__ void __launch_bounds__(256) lat_kernel(const LatParams p) {
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
       const int c = ks * 8 + t;
-      qa[mt][ks][0] = act[mt][0] ? tf32(p.c * qrow[0][c]) : 0u;
-      qa[mt][ks][1] = act[mt][1] ? tf32(p.c * qrow[1][c]) : 0u;
-      qa[mt][ks][2] = act[mt][0] ? tf32(p.c * qrow[0][c + 4]) : 0u;
-      qa[mt][ks][3] = act[mt][1] ? tf32(p.c * qrow[1][c + 4]) : 0u;
+      qa[mt][ks][0] = act[mt][0] ? tf32(p.qmul * qrow[0][c]) : 0u;
+      qa[mt][ks][1] = act[mt][1] ? tf32(p.qmul * qrow[1][c]) : 0u;
+      qa[mt][ks][2] = act[mt][0] ? tf32(p.qmul * qrow[0][c + 4]) : 0u;
+      qa[mt][ks][3] = act[mt][1] ? tf32(p.qmul * qrow[1][c + 4]) : 0u;
       if (MODE != kLatForward) {
         za[mt][ks][0] = act[mt][0] ? tf32(zrow[0][c]) : 0u;
         za[mt][ks][1] = act[mt][1] ? tf32(zrow[1][c]) : 0u;
@@ -332,10 +333,10 @@ __global__ void __launch_bounds__(256) lat_kernel(const LatParams p) {
           float w[4], ds[4];
           if (MODE == kLatDecoder) {
             // W = 2^(S - L_n) per token column, dS = W (<Z_m, dY_n> - delta_n)
-            w[0] = va ? ex2_mufu(s[0] - la) : 0.f;
-            w[1] = vb ? ex2_mufu(s[1] - lb) : 0.f;
-            w[2] = va ? ex2_mufu(s[2] - la) : 0.f;
-            w[3] = vb ? ex2_mufu(s[3] - lb) : 0.f;
+            w[0] = va ? ex2_mufu(fmaf(s[0], p.smul, -la)) : 0.f;
+            w[1] = vb ? ex2_mufu(fmaf(s[1], p.smul, -lb)) : 0.f;
+            w[2] = va ? ex2_mufu(fmaf(s[2], p.smul, -la)) : 0.f;
+            w[3] = vb ? ex2_mufu(fmaf(s[3], p.smul, -lb)) : 0.f;
             ds[0] = w[0] * (gg[0] - da);
             ds[1] = w[1] * (gg[1] - db);
             ds[2] = w[2] * (gg[2] - da);
@@ -346,10 +347,10 @@ __global__ void __launch_bounds__(256) lat_kernel(const LatParams p) {
             for (int nd = 0; nd < KS; ++nd) mma8(oa[mt][nd], wa, by[nd][0], by[nd][1]);
           } else {
             // W = 2^(S - L_m) per latent row, dS = W (<dZ_m, V_n> - gamma_m)
-            w[0] = va ? ex2_mufu(s[0] - lr[mt][0]) : 0.f;
-            w[1] = vb ? ex2_mufu(s[1] - lr[mt][0]) : 0.f;
-            w[2] = va ? ex2_mufu(s[2] - lr[mt][1]) : 0.f;
-            w[3] = vb ? ex2_mufu(s[3] - lr[mt][1]) : 0.f;
+            w[0] = va ? ex2_mufu(fmaf(s[0], p.smul, -lr[mt][0])) : 0.f;
+            w[1] = vb ? ex2_mufu(fmaf(s[1], p.smul, -lr[mt][0])) : 0.f;
+            w[2] = va ? ex2_mufu(fmaf(s[2], p.smul, -lr[mt][1])) : 0.f;
+            w[3] = vb ? ex2_mufu(fmaf(s[3], p.smul, -lr[mt][1])) : 0.f;
             ds[0] = w[0] * (gg[0] - gr[mt][0]);
             ds[1] = w[1] * (gg[1] - gr[mt][0]);
             ds[2] = w[2] * (gg[2] - gr[mt][1]);
@@ -482,7 +483,7 @@ __global__ void __launch_bounds__(256) lat_sum_kernel(const LatSumParams p) {
 // Token-parallel pass: a warp owns MT tiles of 16 token rows (a CTA 128 tokens)
 // of one head and walks all latents in chunks of 64 (32 for D = 32), copied
 // with cp.async from padded tf32 images into two shared-memory buffers.
-// Per 8-latent column block, on the tensor cores: S = K (c Q)^T, and
+// Per 8-latent column block, on the tensor cores: S = smul K (qpad's Q)^T, and
 //   stats:    online softmax over latents, Y += 2^(S - max) Z; at the end
 //             L_n = log2 sum 2^S and delta_n = <dY_n, Y_n>
 //   full:     A = 2^(S - L_m), P = 2^(S - L_n), dA = V dZ^T, dP = dY Z^T,
@@ -607,8 +608,10 @@ __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
       }
       tm0 = quad_max(tm0);
       tm1 = quad_max(tm1);
+      // running maximum of the unscaled products (smul > 0 keeps the order)
       const float nm0 = fmaxf(mx0, tm0), nm1 = fmaxf(mx1, tm1);
-      const float q0 = ex2_mufu(mx0 - nm0), q1 = ex2_mufu(mx1 - nm1);
+      const float q0 = ex2_mufu((mx0 - nm0) * p.smul), q1 = ex2_mufu((mx1 - nm1) * p.smul);
+      const float b0 = nm0 * p.smul, b1 = nm1 * p.smul;
       mx0 = nm0;
       mx1 = nm1;
       l0 *= q0;
@@ -621,8 +624,8 @@ __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
 #pragma unroll
       for (int nt = 0; nt < MC / 8; ++nt) {
         if (nt < ntl) {
-          const float p0 = ex2_mufu(s[nt][0] - nm0), p1 = ex2_mufu(s[nt][1] - nm0);
-          const float p2 = ex2_mufu(s[nt][2] - nm1), p3 = ex2_mufu(s[nt][3] - nm1);
+          const float p0 = ex2_mufu(fmaf(s[nt][0], p.smul, -b0)), p1 = ex2_mufu(fmaf(s[nt][1], p.smul, -b0));
+          const float p2 = ex2_mufu(fmaf(s[nt][2], p.smul, -b1)), p3 = ex2_mufu(fmaf(s[nt][3], p.smul, -b1));
           l0 += p0 + p1;
           l1 += p2 + p3;
           uint32_t pa[4];
@@ -669,10 +672,10 @@ __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
             mma8(da, va[mt][ks], bz[ks][0], bz[ks][1]);
           }
           float a[4], ds[4];
-          a[0] = ex2_mufu(s[0] - lma);
-          a[1] = ex2_mufu(s[1] - lmb);
-          a[2] = ex2_mufu(s[2] - lma);
-          a[3] = ex2_mufu(s[3] - lmb);
+          a[0] = ex2_mufu(fmaf(s[0], p.smul, -lma));
+          a[1] = ex2_mufu(fmaf(s[1], p.smul, -lmb));
+          a[2] = ex2_mufu(fmaf(s[2], p.smul, -lma));
+          a[3] = ex2_mufu(fmaf(s[3], p.smul, -lmb));
           ds[0] = a[0] * (da[0] - ga);
           ds[1] = a[1] * (da[1] - gb);
           ds[2] = a[2] * (da[2] - ga);
@@ -681,10 +684,10 @@ __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
             float dp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) mma8(dp, ya[mt][ks], bzz[ks][0], bzz[ks][1]);
-            ds[0] = fmaf(ex2_mufu(s[0] - ln[mt][0]), dp[0] - dl[mt][0], ds[0]);
-            ds[1] = fmaf(ex2_mufu(s[1] - ln[mt][0]), dp[1] - dl[mt][0], ds[1]);
-            ds[2] = fmaf(ex2_mufu(s[2] - ln[mt][1]), dp[2] - dl[mt][1], ds[2]);
-            ds[3] = fmaf(ex2_mufu(s[3] - ln[mt][1]), dp[3] - dl[mt][1], ds[3]);
+            ds[0] = fmaf(ex2_mufu(fmaf(s[0], p.smul, -ln[mt][0])), dp[0] - dl[mt][0], ds[0]);
+            ds[1] = fmaf(ex2_mufu(fmaf(s[1], p.smul, -ln[mt][0])), dp[1] - dl[mt][0], ds[1]);
+            ds[2] = fmaf(ex2_mufu(fmaf(s[2], p.smul, -ln[mt][1])), dp[2] - dl[mt][1], ds[2]);
+            ds[3] = fmaf(ex2_mufu(fmaf(s[3], p.smul, -ln[mt][1])), dp[3] - dl[mt][1], ds[3]);
           }
           uint32_t sa4[4], aa4[4];
           c_as_a(sa4, ds[0], ds[1], ds[2], ds[3]);
@@ -716,12 +719,19 @@ __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
     d0 = quad_sum(d0);
     d1 = quad_sum(d1);
     if (t == 0) {
-      if (in0) { p.ltok[tok0] = rr[0][0] < L ? mx0 + __log2f(l0) : 0.f; p.dtok[tok0] = rr[0][0] < L ? d0 : 0.f; }
-      if (in1) { p.ltok[tok1] = rr[0][1] < L ? mx1 + __log2f(l1) : 0.f; p.dtok[tok1] = rr[0][1] < L ? d1 : 0.f; }
+      if (in0) {
+        p.ltok[tok0] = rr[0][0] < L ? mx0 * p.smul + __log2f(l0) : 0.f;
+        p.dtok[tok0] = rr[0][0] < L ? d0 : 0.f;
+      }
+      if (in1) {
+        p.ltok[tok1] = rr[0][1] < L ? mx1 * p.smul + __log2f(l1) : 0.f;
+        p.dtok[tok1] = rr[0][1] < L ? d1 : 0.f;
+      }
     }
     return;
   }
-  // dK = scale sum dS q = ln2 sum dS (scale log2(e) q); padding tokens get zeros
+  // dK = scale sum dS q = ln2 smul sum dS (qpad's q); padding tokens get zeros
+  const float kdk = kLn2 * p.smul;
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -731,7 +741,7 @@ __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
 #pragma unroll
       for (int nd = 0; nd < KS; ++nd) {
         const int c = nd * 8 + 2 * t;
-        const float2 kk = v ? make_float2(oa[mt][nd][2 * i] * kLn2, oa[mt][nd][2 * i + 1] * kLn2)
+        const float2 kk = v ? make_float2(oa[mt][nd][2 * i] * kdk, oa[mt][nd][2 * i + 1] * kdk)
                             : make_float2(0.f, 0.f);
         const float2 vv = v ? make_float2(ob[mt][nd][2 * i], ob[mt][nd][2 * i + 1]) : make_float2(0.f, 0.f);
         if (p.g32 != nullptr) {
@@ -902,25 +912,9 @@ __global__ void __launch_bounds__(256) cvt_kernel(const CvtParams p) {
   if (i < p.n) p.dst[i] = bf(p.src[i]);
 }
 
-// delta_n = <dY_n, Y_n> (one thread per token of a head); thread 0 of the
-// first block also checks that a training forward left its state.
-template <int D>
-__global__ void __launch_bounds__(256) delta_kernel(const DeltaParams p) {
-  const long i = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i == 0 && *p.tag != kTrainStateTag) atomicOr(p.err, FLARE_DEV_NO_STATE);
-  if (i >= static_cast<long>(p.B) * p.H * p.N) return;
-  const long bh = i / p.N;
-  const int n = static_cast<int>(i % p.N);
-  bool bad = false;
-  const int L = shard_valid_len(p.lengths, static_cast<int>(bh / p.H), p.N, p.tok_offset, p.n_global, &bad);
-  float d = 0.f;
-  if (n < L) {
-    const float* y = p.y32 + i * D;
-    const uint16_t* g = p.dy + i * D;
-#pragma unroll
-    for (int k = 0; k < D; ++k) d = fmaf(bf(g[k]), y[k], d);
-  }
-  p.dtok[i] = d;
+// Whether a training forward left its state in the workspace.
+__global__ void check_mark_kernel(const MarkParams p) {
+  if (*p.mark != kTrainStateTag) atomicOr(p.err, FLARE_DEV_NO_STATE);
 }
 
 unsigned blocks_for(long n, int threads) { return static_cast<unsigned>((n + threads - 1) / threads); }
@@ -1012,10 +1006,8 @@ cudaError_t launch_cvt(const CvtParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_delta(const DeltaParams& p, cudaStream_t s) {
-  const unsigned grid = blocks_for(static_cast<long>(p.B) * p.H * p.N, 256);
-  if (p.D == 16) delta_kernel<16><<<grid, 256, 0, s>>>(p);
-  else delta_kernel<32><<<grid, 256, 0, s>>>(p);
+cudaError_t launch_check_mark(const MarkParams& p, cudaStream_t s) {
+  check_mark_kernel<<<1, 1, 0, s>>>(p);
   return cudaGetLastError();
 }
 

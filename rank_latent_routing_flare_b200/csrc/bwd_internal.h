@@ -26,7 +26,12 @@ struct LatParams {
   int tok_offset, n_global;     // this shard holds tokens [tok_offset, tok_offset + N) of n_global
   int q_per_batch;              // queries [G][M][D] with G = B*H (1) or H (0)
   int n_splits, tiles_per_split, rows_per_block;   // rows_per_block: 16 per warp, at most 128
-  float c;                      // scale * log2(e)
+  // scores in log2 units: t = smul * <qmul * q, k>, qmul * smul = scale * log2(e).
+  // qmul = scale * log2(e), smul = 1: the query operand is pre-scaled (rounded
+  // to tf32 with the scale); qmul = 1, smul = scale * log2(e): the product of
+  // bf16-exact queries and keys is exact and the scale follows in fp32, as in
+  // the forward's kernels (the gradient modes only)
+  float qmul, smul;
   const int32_t* lengths;
   const float* q;               // fp32 queries [G][M][D]
   const float* zrow;            // decoder: Z [B*H][M][D]; encoder: dZ [B*H][M][D]
@@ -77,10 +82,10 @@ struct TokParams {
   int B, H, N, M, D;
   int tok_offset, n_global;     // this shard holds tokens [tok_offset, tok_offset + N) of n_global
   int q_per_batch;
-  float c;
+  float smul;                   // score multiplier: qpad holds (scale * log2(e) / smul) * q
   const int32_t* lengths;
   // padded tf32 images ([rows][D + 4], see PadParams)
-  const float* qpad;            // log2-scaled queries [G][M][D + 4]
+  const float* qpad;            // scaled queries [G][M][D + 4]
   const float* zpad;            // Z [B*H][M][D + 4] (stats, full)
   const float* dzpad;           // dZ [B*H][M][D + 4] (full, encoder)
   const float* lm;              // encoder row log2-normaliser [B*H][M]
@@ -133,23 +138,17 @@ struct CvtParams {
   float* dst;
 };
 
-// delta_n = <dY_n, Y_n> per token of one shard from a training forward's fp32
-// Y (0 for padding tokens); also checks the state tag that the forward left.
-struct DeltaParams {
-  int B, H, N, D;
-  int tok_offset, n_global;
-  const int32_t* lengths;
-  const float* y32;             // [B*H][N][D]
-  const uint16_t* dy;           // bf16 [B*H][N][D]
-  float* dtok;                  // [B*H][N]
-  const uint32_t* tag;          // must hold kTrainStateTag
+// The mark a training forward leaves in its workspace; a training backward
+// that does not find it sets FLARE_DEV_NO_STATE in the error word.
+struct MarkParams {
+  const uint32_t* mark;         // must hold kTrainStateTag
   uint32_t* err;
 };
 constexpr int kTrainStateByte = 0xA5;               // written with a byte memset
 constexpr uint32_t kTrainStateTag = 0xA5A5A5A5u;    // kTrainStateByte in all four bytes
 
 cudaError_t launch_lat(int mode, const LatParams& p, cudaStream_t s);
-cudaError_t launch_delta(const DeltaParams& p, cudaStream_t s);
+cudaError_t launch_check_mark(const MarkParams& p, cudaStream_t s);
 cudaError_t launch_lat_merge(const LatMergeParams& p, cudaStream_t s);
 cudaError_t launch_lat_sum(const LatSumParams& p, cudaStream_t s);
 cudaError_t launch_tok(int mode, const TokParams& p, cudaStream_t s);

@@ -131,7 +131,6 @@ __global__ void __launch_bounds__(128) decode_fallback_kernel(const DecodeParams
       for (int d = 0; d < D; ++d) y[d] = fmaf(w, __uint_as_float(static_cast<uint32_t>(zh[m * D + d]) << 16), y[d]);
     }
     const float inv = 1.f / den;
-    if (p.ltok_out != nullptr) p.ltok_out[static_cast<size_t>(bh) * p.N + n] = mx + log2f(den);
     if (p.y_f32 != nullptr) {
       float4* d32 = reinterpret_cast<float4*>(p.y_f32 + (static_cast<size_t>(bh) * p.N + n) * D);
 #pragma unroll
@@ -294,16 +293,6 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
         const int buf = x.q % NB, st = x.tile % NST;
         if (x.cc == 0 && !mbar_wait_mma(k_full + st, (x.tile / NST) & 1, wc)) return false;
         if (x.q >= NB && !mbar_wait_mma(pv_done + buf, ((x.q - NB) / NB) & 1, wc)) return false;
-#if FLARE_DEC_REFILL_MMA
-        // chunk q - NB's value MMA is done, and so is every MMA before it: if
-        // that chunk was the last of its tile, the tile's ring stage is free
-        // (every softmax warp read the tile's key norms before handing over the
-        // tile's first P)
-        if (x.q >= NB) {
-          const int qd = x.q - NB, td = qd / nc;
-          if (qd - td * nc == nc - 1 && td + NST < ntiles) load_tile(td + NST);
-        }
-#endif
         tc_fence_after();
         const uint32_t idesc_s = x.cc == nc - 1 ? idesc_last : idesc_full;
         const uint64_t kd = k_desc + static_cast<uint64_t>(st) * (Cfg::KT_B >> 4);
@@ -367,7 +356,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
     // Epilogue of tile i: Y = acc / sum, zero rows for padding, bf16 stores.
     // (Reading Y before the next tile's first exponentials instead, so that
     // the next value MMA need not wait for it, measured 4 % slower.)
-    auto epilogue = [&](int i, float nu_i) -> bool {
+    auto epilogue = [&](int i) -> bool {
       if (!mbar_wait_warp(y_full, i & 1, wc)) return false;
       tc_fence_after();
       uint32_t o[32];
@@ -400,8 +389,6 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
 #pragma unroll
         for (int d = 0; d < D; ++d) y[d] = 0.f;
       }
-      if (p.ltok_out != nullptr && n < p.N && !exact)
-        p.ltok_out[static_cast<size_t>(bh) * p.N + n] = n < L ? nu_i + log2f(l) : 0.f;
       if (exact) {  // recomputed exactly by decode_fallback_kernel
         const uint32_t e = atomicAdd(p.fb_count, 1u);
         p.fb_list[e] = static_cast<uint64_t>(bh) * p.N + n;
@@ -440,7 +427,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
       tmem_wait_st();
     };
     bool ok = true;
-    float nu = 0.f, nu_prev = 0.f;  // shift bounds of the current and the previous tile
+    float nu = 0.f;
     for (int q = 0, tile = 0, cc = 0, buf = 0, use = 0; q < total; ++q) {
       if (!mbar_wait_warp(s_full + buf, use & 1, wc)) { ok = false; break; }
       tc_fence_after();
@@ -450,7 +437,6 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
         // tile's stage is refilled only after every warp is past this point
         if (!mbar_wait_warp(k_full + tile % NST, (tile / NST) & 1, wc)) { ok = false; break; }
         const uint4* krow_s = reinterpret_cast<const uint4*>(sk + (tile % NST) * Cfg::KT_B + r * Cfg::ROWB);
-        nu_prev = nu;
         nu = c * sqrtf(bf16_row_norm2(krow_s, D / 8)) * qm;
       }
       const int cn = min(C, p.M - cc * C);
@@ -461,12 +447,10 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
       else run_chunk(std::integral_constant<int, 16>{}, cb, nu);
       tc_fence_before();
       mbar_arrive_warp(p_full + buf);
-#if !FLARE_DEC_REFILL_MMA
       if (cc == 0 && tile >= 2 && tile - 2 + NST < ntiles && wq == (tile & 3) && lane == 0)
         load_tile(tile - 2 + NST);  // every MMA and norm read of tile - 2 is done
-#endif
       __syncwarp();
-      if (cc == 0 && tile >= 1 && !epilogue(tile - 1, nu_prev)) { ok = false; break; }
+      if (cc == 0 && tile >= 1 && !epilogue(tile - 1)) { ok = false; break; }
       if (++cc == nc) {
         cc = 0;
         ++tile;
@@ -476,7 +460,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
         ++use;
       }
     }
-    if (ok) epilogue(ntiles - 1, nu);
+    if (ok) epilogue(ntiles - 1);
   }
   tc_fence_before();
   __syncthreads();

@@ -187,10 +187,6 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
         const int st = i % NST, buf = i % NB;
         if (!mbar_wait_mma(kv_full + st, (i / NST) & 1, wc)) return false;
         if (i >= NB && !mbar_wait_mma(pv_done + buf, ((i - NB) / NB) & 1, wc)) return false;
-#if FLARE_ENC_REFILL_MMA
-        // the value MMA of tile i - NB is done: its ring stage takes tile i - NB + NST
-        if (i >= NB && i - NB + NST < ntiles) load_tile(i - NB + NST);
-#endif
         tc_fence_after();
         const uint64_t kd = k_desc + static_cast<uint64_t>((st * Cfg::TILE_B) >> 4);
 #pragma unroll
@@ -297,9 +293,7 @@ __global__ void __launch_bounds__(EncCfg<D>::THREADS, EncCfg<D>::CTAS_PER_SM)
         tc_fence_before();
         mbar_arrive_warp(p_full + buf);
         // S_i complete implies P_{i-2} V_{i-2} complete: its ring stage is free
-#if !FLARE_ENC_REFILL_MMA
         if (i >= 2 && i - 2 + NST < ntiles && wq == (i & 3) && lane == 0) load_tile(i - 2 + NST);
-#endif
         __syncwarp();
         if (++buf == NB) {
           buf = 0;

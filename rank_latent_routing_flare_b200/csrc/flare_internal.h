@@ -83,17 +83,6 @@ __host__ __device__ constexpr int dec_ctas_per_sm(int D) { return D == 16 ? FLAR
 #ifndef FLARE_ENC_POLY_PAIRS
 #define FLARE_ENC_POLY_PAIRS 11
 #endif
-// Encoder K/V ring refills: issued by the MMA thread once a tile's value MMA
-// is done (1), or by the softmax warps in rotation once the scores two tiles
-// later are ready (0).
-#ifndef FLARE_ENC_REFILL_MMA
-#define FLARE_ENC_REFILL_MMA 0
-#endif
-// Decoder key-ring refills: by the MMA thread once a tile's last value MMA
-// is done (1), or by the softmax warps in rotation (0).
-#ifndef FLARE_DEC_REFILL_MMA
-#define FLARE_DEC_REFILL_MMA 0
-#endif
 // Encoder softmax: load the first 16 score columns, start their
 // exponentials while the rest of the tile is read from TMEM.
 #ifndef FLARE_ENC_SPLIT_LD
@@ -103,6 +92,11 @@ __host__ __device__ constexpr int dec_ctas_per_sm(int D) { return D == 16 ? FLAR
 // from TMEM per wait.
 #ifndef FLARE_PROJ_EPI_HEADS
 #define FLARE_PROJ_EPI_HEADS 4
+#endif
+// Epilogue warpgroups of the projection kernel (1 or 2), each reading and
+// storing its own block of heads from the shared TMEM accumulator.
+#ifndef FLARE_PROJ_EPI_WG
+#define FLARE_PROJ_EPI_WG 1
 #endif
 #ifndef FLARE_DEC_POLY_PAIRS
 #define FLARE_DEC_POLY_PAIRS 10
@@ -200,7 +194,6 @@ struct DecodeParams {
   uint16_t* y;          // bf16 [B*H][N][D], or [B][N][H*D] when y_token_major
   int y_token_major;
   float* y_f32;         // optional fp32 copy of Y ([B*H][N][D], the values Y is rounded from), or nullptr
-  float* ltok_out;      // optional [B*H][N]: L_n = log2 sum_m 2^(c <k_n, q_m>) per token (0 for padding)
   uint32_t* fb_count;   // number of listed tokens (zeroed before the decoder runs)
   uint64_t* fb_list;    // tokens (bh * N + n) whose row sum underflowed, capacity B*H*N
   uint32_t* err;

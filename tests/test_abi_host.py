@@ -322,14 +322,6 @@ def test_training_pair_argument_errors():
         assert bwd_f() == Status.ERR_LAUNCH and bwd_p() == Status.ERR_LAUNCH
 
 
-def test_flare_training_workspace_holds_fp32_y():
-    """FLARE's backward workspace grows by the training forward's fp32 Y
-    ([B][H][N][D] floats); FLARE++ keeps it in the gradient rows' space."""
-    a = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLARE_BWD, 1, 2, 10000, 32, 16)
-    b = fl.flare_workspace_bytes(fl.FLARE_VARIANT_FLARE_BWD, 1, 2, 20000, 32, 16)
-    assert b - a >= 2 * 10000 * 16 * 4
-
-
 def cp_bwd_call(phase=0, gathered=None, exchange=A, rank=0, world=2, B=1, N=100, C=64, H=4, M=32, D=16, ws=W,
                 ws_bytes=None, dX=A):
     lib = fl.load_library()
