@@ -93,11 +93,6 @@ __host__ __device__ constexpr int dec_ctas_per_sm(int D) { return D == 16 ? FLAR
 #ifndef FLARE_PROJ_EPI_HEADS
 #define FLARE_PROJ_EPI_HEADS 4
 #endif
-// Epilogue warpgroups of the projection kernel (1 or 2), each reading and
-// storing its own block of heads from the shared TMEM accumulator.
-#ifndef FLARE_PROJ_EPI_WG
-#define FLARE_PROJ_EPI_WG 1
-#endif
 #ifndef FLARE_DEC_POLY_PAIRS
 #define FLARE_DEC_POLY_PAIRS 10
 #endif

@@ -12,8 +12,7 @@
 // every 32-token group (used by the encoder as its softmax shift bound).
 //
 // Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer + TMEM owner,
-// warps 2.. = FLARE_PROJ_EPI_WG epilogue warpgroups (thread <-> TMEM lane <->
-// token), warpgroup e taking the e-th block of H / FLARE_PROJ_EPI_WG heads.
+// warps 2..5 = epilogue (thread <-> TMEM lane <-> token).
 #include "ptx.cuh"
 
 namespace flare {
@@ -38,12 +37,10 @@ struct ProjCfg {
   static constexpr int OFF_MISC = OFF_BAR + 8 * 32;
   static constexpr int BYTES = OFF_MISC + 64;
   static constexpr uint32_t TMEM_COLS = (2 * C < 32) ? 32 : 2 * C;  // two accumulators of C columns
-  static constexpr int EWG = FLARE_PROJ_EPI_WG;       // epilogue warpgroups
-  static constexpr int THREADS = 64 + 128 * EWG;
 };
 
 template <int C, int D>
-__global__ void __launch_bounds__(ProjCfg<C>::THREADS, ProjCfg<C>::EWG > 1 ? 2 : 1)
+__global__ void __launch_bounds__(192, 1)
     project_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w0,
                    const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__ CUtensorMap tm_w2,
                    const __grid_constant__ CUtensorMap tm_w3, const ProjParams p) {
@@ -82,7 +79,7 @@ __global__ void __launch_bounds__(ProjCfg<C>::THREADS, ProjCfg<C>::EWG > 1 ? 2 :
     }
     for (int j = 0; j < 2; ++j) {
       mbar_init(acc_full + j, 1);
-      mbar_init(acc_free + j, 4 * Cfg::EWG);
+      mbar_init(acc_free + j, 4);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -169,8 +166,6 @@ __global__ void __launch_bounds__(ProjCfg<C>::THREADS, ProjCfg<C>::EWG > 1 ? 2 :
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const int eg = (warp - 2) >> 2;
-    const int h_begin = eg * H / Cfg::EWG, h_end = (eg + 1) * H / Cfg::EWG;
     uint16_t* out = proj == 0 ? p.out[0] : proj == 1 ? p.out[1] : proj == 2 ? p.out[2] : p.out[3];
     float* knorm = proj == 0 ? p.knorm[0] : proj == 1 ? p.knorm[1] : proj == 2 ? p.knorm[2] : p.knorm[3];
     for (int i = 0; i < my_tiles; ++i) {
@@ -183,16 +178,16 @@ __global__ void __launch_bounds__(ProjCfg<C>::THREADS, ProjCfg<C>::EWG > 1 ? 2 :
       tc_fence_after();
       // G heads per TMEM read (one wait per G heads; G * D columns)
       constexpr int G = D == 16 ? FLARE_PROJ_EPI_HEADS : (FLARE_PROJ_EPI_HEADS + 1) / 2;
-      for (int h0 = h_begin; h0 < h_end; h0 += G) {
+      for (int h0 = 0; h0 < H; h0 += G) {
         uint32_t v[G][D];
 #pragma unroll
         for (int j = 0; j < G; ++j)
-          if (h0 + j < h_end) tmem_ld_cols<D>(lane_base + ab * C + (h0 + j) * D, v[j]);
+          if (h0 + j < H) tmem_ld_cols<D>(lane_base + ab * C + (h0 + j) * D, v[j]);
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < G; ++j) {
           const int hh = h0 + j;
-          if (hh >= h_end) break;
+          if (hh >= H) break;
           uint32_t pk[D / 2];
           float nrm = 0.f;
 #pragma unroll
@@ -238,7 +233,7 @@ cudaError_t launch_project_cd(const CUtensorMap& tm_x, const CUtensorMap (&tm_w)
   cudaError_t e = cudaFuncSetAttribute(project_kernel<C, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  LaunchCfg lc(dim3(p.n_proj * p.groups), dim3(ProjCfg<C>::THREADS), smem, s, pdl);
+  LaunchCfg lc(dim3(p.n_proj * p.groups), dim3(192), smem, s, pdl);
   return cudaLaunchKernelEx(&lc.cfg, project_kernel<C, D>, tm_x, tm_w[0], tm_w[1], tm_w[2], tm_w[3], p);
 }
 
