@@ -66,12 +66,14 @@ MUFU_PER_CLK_PER_SM = 16          # nominal ex2 results per clock per SM (used o
 FMA_PER_CLK_PER_SM = 128          # nominal fp32 fma per clock per SM (ditto)
 NUM_SM = 148
 # Issue-slot cost of the softmax's own arithmetic per score (the kernels'
-# exponential step): one FFMA for the scale-and-shift and half a bf16x2 pack,
-# plus the exponential itself -- one MUFU instruction, or the 9 instructions
-# of the FMA-pipe polynomial (clamp, two adds and a subtract for the range
-# reduction, three FFMAs, a shift and an integer add for the exponent).
-SOFTMAX_BASE_OPS = 1.5
-POLY_EXP_OPS = 9.0
+# exponential step, thread instructions, with the paired fp32x2 forms the
+# kernels use): half a paired FFMA for the scale-and-shift and half a bf16x2
+# pack, plus the exponential itself -- one MUFU instruction, or 6 for the
+# FMA-pipe polynomial (per pair of scores: 2 clamps, 2 paired adds for the
+# range reduction, 4 paired FFMAs for the remainder and the cubic, 2 shifts
+# and 2 integer adds for the exponent: 12).
+SOFTMAX_BASE_OPS = 1.0
+POLY_EXP_OPS = 6.0
 STAGES_PP = ["project", "synth_encode", "synth_merge", "encode", "merge", "decode"]
 KERNEL_SOURCES = {"project": "project.cu", "synth_encode": "encode.cu", "encode": "encode.cu",
                   "synth_merge": "merge.cu", "merge": "merge.cu", "decode": "decode.cu"}
