@@ -68,6 +68,13 @@ BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C) {
     bp.off_g32 = take(static_cast<size_t>(B * N) * 4 * C * 4);
     bp.off_dwpart = take(static_cast<size_t>(bp.dw_splits) * C * 4 * C * 4);
   }
+  // the training pair at D = 16: the low part of Z and the forward's fp32 Y
+  // (FLARE++: in the gradient rows' space, which the backward fills only
+  // after it has taken delta_n from Y)
+  if (D == 16) {
+    bp.off_zlo16 = take(static_cast<size_t>(BH * M * D) * 2);
+    bp.off_y32 = pp ? bp.off_g32 : take(static_cast<size_t>(BH * N * D) * 4);
+  }
   bp.total = off;
   return bp;
 }
@@ -599,11 +606,25 @@ flare_status flarepp_mixer_bwd(const flare_bf16* X, const flare_bf16* Wk, const 
 // that uses it.  The backward's scores then take the bf16 Q(X) that the
 // forward's products used, unscaled, with the scale applied to the fp32
 // product (exact scores), so that the forward's normalisers fit them.  The
-// decoder's per-token statistics are recomputed: delta_n = <dY_n, Y_n> needs
-// Y from the fp32 Z (the forward's Y takes Z in bf16, which moves the
-// gradients of Q0 and W~_K by more than the tolerance).
+// decoder's delta_n = <dY_n, Y_n> needs Y from the fp32 Z (a Y from the bf16
+// Z moves the gradients of Q0 and W~_K by more than the tolerance): at D = 16
+// the training forward's decoder adds the low bf16 part of Z and keeps the
+// fp32 Y and the per-token normalisers L_n; at D = 32 (no shared memory for
+// the low part) the backward recomputes L_n and delta_n.
 // ---------------------------------------------------------------------------
 namespace {
+
+// What a training forward keeps besides the synthesis normalisers.
+FwdStats train_stats(const BwdPlan& bp, uint8_t* ws, int D) {
+  FwdStats fs;
+  fs.lenc = reinterpret_cast<float*>(ws + bp.off_lenc);
+  if (D == 16) {
+    fs.zlo = reinterpret_cast<uint16_t*>(ws + bp.off_zlo16);
+    fs.y32 = reinterpret_cast<float*>(ws + bp.off_y32);
+    fs.ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
+  }
+  return fs;
+}
 
 flare_status set_train_mark(uint8_t* ws, const BwdPlan& bp, int value, cudaStream_t s) {
   return cudaMemsetAsync(ws + bp.fwd.off_err + kTrainMarkOffset, value, 4, s) == cudaSuccess ? FLARE_OK
@@ -642,26 +663,38 @@ flare_status train_prologue(const BwdPlan& bp, uint8_t* ws, const flare_bf16* Q,
   return pad(z32, reinterpret_cast<float*>(ws + bp.off_zpad), BH * M, D, 1.f, s);
 }
 
-// The decoder's statistics (L_n, delta_n) and its backward (the dZ and dQ
-// partials into `exch`), exact scores; q: the fp32 queries of the lat pass.
+// The decoder's statistics (L_n, delta_n: from the training forward at
+// D = 16, recomputed otherwise) and its backward (the dZ and dQ partials into
+// `exch`), exact scores; q: the fp32 queries of the lat pass.
 flare_status train_decoder(const BwdPlan& bp, uint8_t* ws, const float* q, int q_per_batch, const void* k,
                            const flare_bf16* dY, int B, int H, int N, int M, int D, const int32_t* lengths, float sc,
                            float* exch, cudaStream_t s) {
   const Shard sh{0, N, 1};
   float* ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
   float* dtok = reinterpret_cast<float*>(ws + bp.off_dtok);
-  TokParams tp = tok_params(B, H, N, M, D, q_per_batch, lengths, sc, sh);
-  tp.smul = sc * kLog2e;
-  tp.qpad = reinterpret_cast<const float*>(ws + bp.off_qpad);
-  tp.zpad = reinterpret_cast<const float*>(ws + bp.off_zpad);
-  tp.k = static_cast<const uint16_t*>(k);
-  tp.dy = reinterpret_cast<const uint16_t*>(dY);
-  tp.ltok = ltok; tp.dtok = dtok;
-  if (launch_tok(kTokStats, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  if (D == 16) {  // L_n is the forward's; delta_n from its fp32 Y
+    DeltaParams dp{};
+    dp.B = B; dp.H = H; dp.N = N; dp.D = D;
+    dp.tok_offset = 0; dp.n_global = N;
+    dp.lengths = lengths;
+    dp.y32 = reinterpret_cast<const float*>(ws + bp.off_y32);
+    dp.dy = reinterpret_cast<const uint16_t*>(dY);
+    dp.dtok = dtok;
+    if (launch_delta(dp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  } else {
+    TokParams tp = tok_params(B, H, N, M, D, q_per_batch, lengths, sc, sh);
+    tp.smul = sc * kLog2e;
+    tp.qpad = reinterpret_cast<const float*>(ws + bp.off_qpad);
+    tp.zpad = reinterpret_cast<const float*>(ws + bp.off_zpad);
+    tp.k = static_cast<const uint16_t*>(k);
+    tp.dy = reinterpret_cast<const uint16_t*>(dY);
+    tp.ltok = ltok; tp.dtok = dtok;
+    if (launch_tok(kTokStats, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  }
   LatParams ld = lat_params(bp, ws, q, q_per_batch, k, B, H, N, M, D, lengths, sc, sh);
   exact_scores(ld, sc);
   ld.zrow = reinterpret_cast<const float*>(ws + bp.off_z32);
-  ld.dy = tp.dy;
+  ld.dy = reinterpret_cast<const uint16_t*>(dY);
   ld.ltok = ltok; ld.dtok = dtok;
   ld.part_a = exch;
   ld.part_b = exch + part_floats(bp, B, H, M, D, false);
@@ -682,9 +715,8 @@ flare_status flarepp_mixer_fwd_train(const flare_bf16* X, const flare_bf16* Wk, 
   if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  FwdStats fs;
+  FwdStats fs = train_stats(bp, ws, D);
   fs.lsyn = reinterpret_cast<float*>(ws + bp.off_lsyn);
-  fs.lenc = reinterpret_cast<float*>(ws + bp.off_lenc);
   st = flarepp_run(bp.fwd, X, Wk, Wv, Wk_syn, Wv_syn, Q0, Y, 0, B, N, C, H, M, D, lengths, resolve_scale(scale, D), ws,
                    s, nullptr, nullptr, nullptr, nullptr, &fs);
   if (st != FLARE_OK) return st;
@@ -730,8 +762,7 @@ flare_status flare_mixer_fwd_train(const flare_bf16* K, const flare_bf16* V, con
   const BwdPlan bp = make_bwd_plan(false, B, H, N, M, D, 0);
   if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  FwdStats fs;
-  fs.lenc = reinterpret_cast<float*>(ws + bp.off_lenc);
+  FwdStats fs = train_stats(bp, ws, D);
   st = flare_fwd(K, V, Q, Y, B, H, N, M, D, lengths, scale, workspace, workspace_bytes, stream, nullptr, nullptr,
                  nullptr, &fs);
   if (st != FLARE_OK) return st;

@@ -912,6 +912,36 @@ __global__ void __launch_bounds__(256) cvt_kernel(const CvtParams p) {
   if (i < p.n) p.dst[i] = bf(p.src[i]);
 }
 
+// delta_n = <dY_n, Y_n>, one thread per token of a head.
+template <int D>
+__global__ void __launch_bounds__(256) delta_kernel(const DeltaParams p) {
+  const long i = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= static_cast<long>(p.B) * p.H * p.N) return;
+  const long bh = i / p.N;
+  const int n = static_cast<int>(i % p.N);
+  bool bad = false;
+  const int L = shard_valid_len(p.lengths, static_cast<int>(bh / p.H), p.N, p.tok_offset, p.n_global, &bad);
+  float d = 0.f;
+  if (n < L) {
+    const float4* y = reinterpret_cast<const float4*>(p.y32 + i * D);
+    const uint4* g = reinterpret_cast<const uint4*>(p.dy + i * D);
+#pragma unroll
+    for (int u = 0; u < D / 8; ++u) {
+      const uint4 gv = g[u];
+      const float4 y0 = y[2 * u], y1 = y[2 * u + 1];
+      d = fmaf(bf16_lo(gv.x), y0.x, d);
+      d = fmaf(bf16_hi(gv.x), y0.y, d);
+      d = fmaf(bf16_lo(gv.y), y0.z, d);
+      d = fmaf(bf16_hi(gv.y), y0.w, d);
+      d = fmaf(bf16_lo(gv.z), y1.x, d);
+      d = fmaf(bf16_hi(gv.z), y1.y, d);
+      d = fmaf(bf16_lo(gv.w), y1.z, d);
+      d = fmaf(bf16_hi(gv.w), y1.w, d);
+    }
+  }
+  p.dtok[i] = d;
+}
+
 // Whether a training forward left its state in the workspace.
 __global__ void check_mark_kernel(const MarkParams p) {
   if (*p.mark != kTrainStateTag) atomicOr(p.err, FLARE_DEV_NO_STATE);
@@ -1003,6 +1033,13 @@ cudaError_t launch_pad(const PadParams& p, cudaStream_t s) {
 
 cudaError_t launch_cvt(const CvtParams& p, cudaStream_t s) {
   cvt_kernel<<<blocks_for(p.n, 256), 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_delta(const DeltaParams& p, cudaStream_t s) {
+  const unsigned grid = blocks_for(static_cast<long>(p.B) * p.H * p.N, 256);
+  if (p.D == 16) delta_kernel<16><<<grid, 256, 0, s>>>(p);
+  else delta_kernel<32><<<grid, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 

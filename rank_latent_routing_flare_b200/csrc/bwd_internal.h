@@ -138,6 +138,18 @@ struct CvtParams {
   float* dst;
 };
 
+// delta_n = <dY_n, Y_n> per token from a training forward's fp32 Y (0 for
+// padding tokens).
+struct DeltaParams {
+  int B, H, N, D;
+  int tok_offset, n_global;
+  const int32_t* lengths;
+  const float* y32;             // [B*H][N][D]
+  const uint16_t* dy;           // bf16 [B*H][N][D]
+  float* dtok;                  // [B*H][N]
+};
+cudaError_t launch_delta(const DeltaParams& p, cudaStream_t s);
+
 // The mark a training forward leaves in its workspace; a training backward
 // that does not find it sets FLARE_DEV_NO_STATE in the error word.
 struct MarkParams {

@@ -26,6 +26,13 @@
 // full phase ahead of the party that waits on it.  The epilogue of a tile
 // (Y / sum, bf16 stores) runs after the first chunk of the next tile.
 //
+// With ZLO (the training forward, D = 16) Z also has a low part Zlo =
+// Z - bf16(Z) in shared memory and each chunk adds P Zlo_c into Y (a second
+// value MMA of N = D, no ones block), so that Y, and the fp32 copy the
+// backward takes delta_n from, see Z to fp32 accuracy; the epilogue also
+// writes L_n.  The extra 16 KB of shared memory leave room for three CTAs per
+// SM instead of four.
+//
 // Warp roles (5 warps): warp 0 lane 0 is the MMA thread (it also loads Q, Z
 // and the first key tiles).  Warps 1..4 are the softmax warps (thread <->
 // TMEM lane <-> token); one of them, in rotation, refills the key ring.  A
@@ -38,8 +45,9 @@
 namespace flare {
 namespace {
 
-template <int D>
+template <int D, bool ZLO>
 struct DecCfg {
+  static_assert(!ZLO || D == 16, "the low part of Z is kept for D = 16 only");
   static constexpr int C = dec_chunk(D);                // latents per chunk
   static constexpr int ROWB = D * 2;
   static constexpr int KT_B = kDecTile * ROWB;          // one key tile
@@ -51,7 +59,8 @@ struct DecCfg {
   static constexpr int NB = dec_bufs(D);                // score buffers
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_Z = OFF_Q + QZ_B;
-  static constexpr int OFF_ONES = OFF_Z + QZ_B;         // C x ROWB block of ones
+  static constexpr int OFF_ZLO = OFF_Z + QZ_B;          // (ZLO) the low part of Z
+  static constexpr int OFF_ONES = OFF_ZLO + (ZLO ? QZ_B : 0);  // C x ROWB block of ones
   static constexpr int OFF_K = OFF_ONES + C * ROWB;     // NST * KT_B
   static constexpr int OFF_BAR = OFF_K + NST * KT_B;
   static constexpr int OFF_MISC = OFF_BAR + 8 * (4 + NST + 3 * NB);
@@ -60,7 +69,7 @@ struct DecCfg {
   static constexpr uint32_t COL_Y = NB * C;
   static constexpr uint32_t TMEM_COLS = (COL_Y + NY <= 128) ? 128 : 256;
   static constexpr int THREADS = 160;
-  static constexpr int CTAS_PER_SM = dec_ctas_per_sm(D);
+  static constexpr int CTAS_PER_SM = ZLO ? 3 : dec_ctas_per_sm(D);
   static_assert(TMEM_COLS <= 512 / CTAS_PER_SM, "TMEM columns of the co-resident CTAs exceed 512");
   static_assert(COL_Y + NY <= TMEM_COLS, "score buffers and Y exceed the allocation");
   static_assert(OFF_K % 512 == 0 || D == 16, "key tiles must start on a swizzle atom");
@@ -108,6 +117,7 @@ __global__ void __launch_bounds__(128) decode_fallback_kernel(const DecodeParams
     const uint16_t* krow = p.k + (static_cast<size_t>(bh) * p.N + n) * D;
     const uint16_t* qg = p.q + static_cast<size_t>(g) * p.M * D;
     const uint16_t* zh = p.z + static_cast<size_t>(bh) * p.M * D;
+    const uint16_t* zl = p.zlo != nullptr ? p.zlo + static_cast<size_t>(bh) * p.M * D : nullptr;
     float k[D], y[D];
 #pragma unroll
     for (int d = 0; d < D; ++d) k[d] = __uint_as_float(static_cast<uint32_t>(krow[d]) << 16);
@@ -129,8 +139,13 @@ __global__ void __launch_bounds__(128) decode_fallback_kernel(const DecodeParams
       den += w;
 #pragma unroll
       for (int d = 0; d < D; ++d) y[d] = fmaf(w, __uint_as_float(static_cast<uint32_t>(zh[m * D + d]) << 16), y[d]);
+      if (zl != nullptr) {
+#pragma unroll
+        for (int d = 0; d < D; ++d) y[d] = fmaf(w, __uint_as_float(static_cast<uint32_t>(zl[m * D + d]) << 16), y[d]);
+      }
     }
     const float inv = 1.f / den;
+    if (p.ltok_out != nullptr) p.ltok_out[static_cast<size_t>(bh) * p.N + n] = mx + log2f(den);
     if (p.y_f32 != nullptr) {
       float4* d32 = reinterpret_cast<float4*>(p.y_f32 + (static_cast<size_t>(bh) * p.N + n) * D);
 #pragma unroll
@@ -147,16 +162,18 @@ __global__ void __launch_bounds__(128) decode_fallback_kernel(const DecodeParams
   }
 }
 
-template <int D>
-__global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
+template <int D, bool ZLO>
+__global__ void __launch_bounds__(DecCfg<D, ZLO>::THREADS, DecCfg<D, ZLO>::CTAS_PER_SM)
     decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_z,
-                  const __grid_constant__ CUtensorMap tm_k, const DecodeParams p) {
-  using Cfg = DecCfg<D>;
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_zlo,
+                  const DecodeParams p) {
+  using Cfg = DecCfg<D, ZLO>;
   constexpr int NST = Cfg::NST, C = Cfg::C, NB = Cfg::NB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sq = sm + Cfg::OFF_Q;
   uint8_t* sz = sm + Cfg::OFF_Z;
+  uint8_t* szlo = sm + Cfg::OFF_ZLO;
   uint8_t* sones = sm + Cfg::OFF_ONES;
   uint8_t* sk = sm + Cfg::OFF_K;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Cfg::OFF_BAR);
@@ -258,11 +275,14 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_z);
       tma_prefetch_desc(&tm_k);
+      if constexpr (ZLO) tma_prefetch_desc(&tm_zlo);
       const int nbox = (p.M + p.qz_box_rows - 1) / p.qz_box_rows;
-      mbar_arrive_expect_tx(qz_full, 2 * nbox * p.qz_box_rows * Cfg::ROWB);
+      mbar_arrive_expect_tx(qz_full, (ZLO ? 3 : 2) * nbox * p.qz_box_rows * Cfg::ROWB);
       for (int bx = 0; bx < nbox; ++bx) {
         tma_load_3d(sq + bx * p.qz_box_rows * Cfg::ROWB, &tm_q, qz_full, 0, bx * p.qz_box_rows, g);
         tma_load_3d(sz + bx * p.qz_box_rows * Cfg::ROWB, &tm_z, qz_full, 0, bx * p.qz_box_rows, bh);
+        if constexpr (ZLO)
+          tma_load_3d(szlo + bx * p.qz_box_rows * Cfg::ROWB, &tm_zlo, qz_full, 0, bx * p.qz_box_rows, bh);
       }
       for (int n = 0; n < min(NST, ntiles); ++n) load_tile(n);
       const uint32_t idesc_y = idesc_bf16_f32(128, Cfg::NY, false, true);
@@ -287,6 +307,9 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
       // [Z_c | 1]: chunk c starts CH_STEP * c further on, and its ones block
       // (leading byte offset) is that much closer
       const uint64_t z_desc = umma_desc(sz_a, ones_a - sz_a, Cfg::SBO, Cfg::LAYOUT);
+      // Zlo_c alone (N = D: one block, its leading byte offset unused)
+      const uint64_t zlo_desc = umma_desc(smem_u32(szlo), 16, Cfg::SBO, Cfg::LAYOUT);
+      const uint32_t idesc_ylo = idesc_bf16_f32(128, D, false, true);
       // S_q = K_tile Q_c^T into buffer q % NB, once the key tile has landed and
       // P_{q-NB} has been consumed
       auto issue_s = [&](const Cursor& x) -> bool {
@@ -318,6 +341,14 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
           if (ks < nks)
             umma_ts(tmem + Cfg::COL_Y, tmem + buf * C + ks * 8,
                     zd + static_cast<uint64_t>((ks * 16 * Cfg::ROWB) >> 4), idesc_y, (x.cc > 0 || ks > 0) ? 1u : 0u);
+        if constexpr (ZLO) {
+          const uint64_t zld = zlo_desc + step;
+#pragma unroll
+          for (int ks = 0; ks < C / 16; ++ks)
+            if (ks < nks)
+              umma_ts(tmem + Cfg::COL_Y, tmem + buf * C + ks * 8,
+                      zld + static_cast<uint64_t>((ks * 16 * Cfg::ROWB) >> 4), idesc_ylo, 1u);
+        }
         umma_commit(pv_done + buf);
         if (x.cc == nc - 1) umma_commit(y_full);
         return true;
@@ -356,7 +387,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
     // Epilogue of tile i: Y = acc / sum, zero rows for padding, bf16 stores.
     // (Reading Y before the next tile's first exponentials instead, so that
     // the next value MMA need not wait for it, measured 4 % slower.)
-    auto epilogue = [&](int i) -> bool {
+    auto epilogue = [&](int i, float nu_i) -> bool {
       if (!mbar_wait_warp(y_full, i & 1, wc)) return false;
       tc_fence_after();
       uint32_t o[32];
@@ -388,6 +419,10 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
       } else {
 #pragma unroll
         for (int d = 0; d < D; ++d) y[d] = 0.f;
+      }
+      if constexpr (ZLO) {  // L_n for the training backward
+        if (p.ltok_out != nullptr && n < p.N && !exact)
+          p.ltok_out[static_cast<size_t>(bh) * p.N + n] = n < L ? nu_i + log2f(l) : 0.f;
       }
       if (exact) {  // recomputed exactly by decode_fallback_kernel
         const uint32_t e = atomicAdd(p.fb_count, 1u);
@@ -427,7 +462,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
       tmem_wait_st();
     };
     bool ok = true;
-    float nu = 0.f;
+    float nu = 0.f, nu_prev = 0.f;  // shift bounds of the current and the previous tile
     for (int q = 0, tile = 0, cc = 0, buf = 0, use = 0; q < total; ++q) {
       if (!mbar_wait_warp(s_full + buf, use & 1, wc)) { ok = false; break; }
       tc_fence_after();
@@ -437,6 +472,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
         // tile's stage is refilled only after every warp is past this point
         if (!mbar_wait_warp(k_full + tile % NST, (tile / NST) & 1, wc)) { ok = false; break; }
         const uint4* krow_s = reinterpret_cast<const uint4*>(sk + (tile % NST) * Cfg::KT_B + r * Cfg::ROWB);
+        if constexpr (ZLO) nu_prev = nu;
         nu = c * sqrtf(bf16_row_norm2(krow_s, D / 8)) * qm;
       }
       const int cn = min(C, p.M - cc * C);
@@ -450,7 +486,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
       if (cc == 0 && tile >= 2 && tile - 2 + NST < ntiles && wq == (tile & 3) && lane == 0)
         load_tile(tile - 2 + NST);  // every MMA and norm read of tile - 2 is done
       __syncwarp();
-      if (cc == 0 && tile >= 1 && !epilogue(tile - 1)) { ok = false; break; }
+      if (cc == 0 && tile >= 1 && !epilogue(tile - 1, nu_prev)) { ok = false; break; }
       if (++cc == nc) {
         cc = 0;
         ++tile;
@@ -460,7 +496,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
         ++use;
       }
     }
-    if (ok) epilogue(ntiles - 1);
+    if (ok) epilogue(ntiles - 1, nu);
   }
   tc_fence_before();
   __syncthreads();
@@ -477,25 +513,33 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, DecCfg<D>::CTAS_PER_SM)
 
 }  // namespace
 
-size_t decode_smem_bytes(int D, int /*M*/) {
-  const size_t need = (D == 16 ? DecCfg<16>::BYTES : DecCfg<32>::BYTES) + 1024;
-  // at most dec_ctas_per_sm(D) CTAs per SM (228 KB each, 1 KB of it
-  // reserved per CTA), so that every resident CTA finds its TMEM columns free
-  const size_t floor = (228 * 1024) / (dec_ctas_per_sm(D) + 1) + 1024;
+size_t decode_smem_bytes(int D, bool zlo) {
+  const size_t need =
+      (D == 16 ? (zlo ? DecCfg<16, true>::BYTES : DecCfg<16, false>::BYTES) : DecCfg<32, false>::BYTES) + 1024;
+  // at most as many CTAs per SM as the kernel's launch bounds name (228 KB
+  // each, 1 KB of it reserved per CTA), so that every resident CTA finds its
+  // TMEM columns free
+  const int ctas = D == 16 ? (zlo ? DecCfg<16, true>::CTAS_PER_SM : DecCfg<16, false>::CTAS_PER_SM)
+                           : DecCfg<32, false>::CTAS_PER_SM;
+  const size_t floor = (228 * 1024) / (ctas + 1) + 1024;
   return need > floor ? need : floor;
 }
 
 cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_z, const CUtensorMap& tm_k,
-                          const DecodeParams& p, cudaStream_t s, bool pdl) {
-  const size_t smem = decode_smem_bytes(p.D, p.M);
+                          const CUtensorMap* tm_zlo, const DecodeParams& p, cudaStream_t s, bool pdl) {
+  const bool zlo = tm_zlo != nullptr;
+  if (zlo && (p.D != 16 || p.zlo == nullptr)) return cudaErrorInvalidValue;
+  const size_t smem = decode_smem_bytes(p.D, zlo);
   const dim3 grid(static_cast<unsigned>(p.B * p.H * p.ctas_per_head));
   auto go = [&](auto kern, int threads) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     LaunchCfg lc(grid, dim3(threads), smem, s, pdl);
-    return cudaLaunchKernelEx(&lc.cfg, kern, tm_q, tm_z, tm_k, p);
+    return cudaLaunchKernelEx(&lc.cfg, kern, tm_q, tm_z, tm_k, zlo ? *tm_zlo : tm_z, p);
   };
-  cudaError_t e = p.D == 16 ? go(decode_kernel<16>, DecCfg<16>::THREADS) : go(decode_kernel<32>, DecCfg<32>::THREADS);
+  cudaError_t e = p.D != 16 ? go(decode_kernel<32, false>, DecCfg<32, false>::THREADS)
+                  : zlo     ? go(decode_kernel<16, true>, DecCfg<16, true>::THREADS)
+                            : go(decode_kernel<16, false>, DecCfg<16, false>::THREADS);
   if (e != cudaSuccess) return e;
   // the fallback follows the decoder on the same stream: always programmatic
   LaunchCfg fb(dim3(kNumSM), dim3(128), 0, s, true);

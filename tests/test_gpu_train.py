@@ -1,11 +1,15 @@
 """GPU parity of the training pair (flarepp_mixer_fwd_train / _bwd_train and
 the FLARE ones) against the fp64 oracle and against the stand-alone calls.
 
-The training forward writes the same Y as flarepp_mixer_fwd (bit for bit:
-the same kernels, with the normalisers and the fp32 Y also stored); its
-backward reuses the forward's state instead of recomputing it, and its
-gradients are held to the backward's tolerance against the oracle:
-rel-L2 <= 5e-3 and max |error| <= 3e-2 * max |reference| per tensor.
+At D = 32 the training forward writes the same Y as flarepp_mixer_fwd (bit
+for bit: the same kernels, the normalisers also stored).  At D = 16 its
+decoder also adds the low bf16 part of Z (so that the fp32 Y it keeps for the
+backward sees Z to fp32 accuracy): Y is then held to the forward's own parity
+criteria against the oracle (``tests/parity.py``) and is at least as close to
+it as the plain forward's.  The backward reuses the forward's state instead
+of recomputing it; its gradients are held to the backward's tolerance
+against the oracle: rel-L2 <= 5e-3 and max |error| <= 3e-2 * max |reference|
+per tensor.
 """
 import numpy as np
 import pytest
@@ -13,7 +17,7 @@ import torch
 
 import oracle
 import rank_latent_routing_flare_b200 as fl
-from tests.gpu_util import dev_bf16, host_f64, rel_l2
+from tests.gpu_util import compare, dev_bf16, host_f64, rel_l2
 from tests.test_gpu_backward import check, flare_case, lengths_dev, run_flare_bwd, run_flarepp_bwd
 from workloads import make_upstream_grad, make_workload
 
@@ -48,6 +52,21 @@ def run_flare_train(w, dY):
 PP_KEYS = ("dX", "dWk", "dWv", "dWk_syn", "dWv_syn", "dQ0")
 
 
+def check_train_y(w, Y, Y_plain, label):
+    """The training forward's Y: bitwise the plain forward's at D = 32; at
+    D = 16 (the decoder adds the low part of Z) within the forward's parity
+    criteria and no further from the oracle than the plain forward's Y."""
+    if w.D != 16:
+        assert torch.equal(Y.view(torch.int16), Y_plain.view(torch.int16)), label
+        return
+    ref = oracle.forward_workload(w)
+    got, plain = host_f64(Y), host_f64(Y_plain)
+    compare({"Y": got}, ref, label=label, lengths=w.lengths)
+    e_train, e_plain = rel_l2(got, ref["Y"]), rel_l2(plain, ref["Y"])
+    print(f"{label}: Y rel-L2 training forward {e_train:.3e}, plain forward {e_plain:.3e}")
+    assert e_train <= e_plain * 1.02 + 1e-6, (label, e_train, e_plain)
+
+
 @pytest.mark.parametrize("name,N,B", [
     ("flarepp_n1k", None, None),
     ("flarepp_n8k_mesh2d", 1500, 2),
@@ -59,7 +78,7 @@ def test_flarepp_training_pair_matches_oracle(name, N, B):
     dY = make_upstream_grad(w)
     Y, got, _ = run_flarepp_train(w, dY)
     Y_ref = fl.flarepp_mixer_fwd(*flarepp_inputs(w), lengths=lengths_dev(w))
-    assert torch.equal(Y.view(torch.int16), Y_ref.view(torch.int16)), "training forward changed Y"
+    check_train_y(w, Y, Y_ref, f"train {name} forward")
     ref = oracle.backward_workload(w, dY)
     plain = run_flarepp_bwd(w, dY)
     for k in PP_KEYS:
@@ -82,7 +101,7 @@ def test_flare_training_pair_matches_oracle(B, H, N, M, D, lengths):
     dY = make_upstream_grad(w)
     Y, got, _ = run_flare_train(w, dY)
     Y_ref = fl.flare_mixer_fwd(dev_bf16(w.K), dev_bf16(w.V), dev_bf16(w.Q), lengths=lengths_dev(w))
-    assert torch.equal(Y.view(torch.int16), Y_ref.view(torch.int16))
+    check_train_y(w, Y, Y_ref, f"train FLARE forward D{D}")
     ref = oracle.backward_workload(w, dY)
     plain = run_flare_bwd(w, dY)
     for k in ("dK", "dV", "dQ"):
