@@ -70,6 +70,19 @@ bool map2d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint32_t 
 
 CUtensorMapSwizzle row_swizzle(int D) { return D == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B; }
 
+// 2-D fp32 tensor map: dims (d0 innermost, d1), dense, box (b0, b1), no swizzle.
+bool map2d_f32(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint32_t b0, uint32_t b1) {
+  EncodeTiledFn fn = tensor_map_encoder();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {d0, d1};
+  const cuuint64_t strides[1] = {d0 * 4};
+  const cuuint32_t box[2] = {b0, b1};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 
 // Number of token splits of the encoder.  Cost model: the CTAs run in
 // waves of `slots` (CTAs resident on the whole GPU); a wave lasts as long as

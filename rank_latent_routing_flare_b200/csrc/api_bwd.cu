@@ -73,6 +73,9 @@ BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C) {
   // after it has taken delta_n from Y)
   if (D == 16) {
     bp.off_zlo16 = take(static_cast<size_t>(BH * M * D) * 2);
+    // the high and low bf16 parts of dZ (then of dQ(X)) for the tcgen05 passes
+    bp.off_xhi16 = take(static_cast<size_t>(BH * M * D) * 2);
+    bp.off_xlo16 = take(static_cast<size_t>(BH * M * D) * 2);
     bp.off_y32 = pp ? bp.off_g32 : take(static_cast<size_t>(BH * N * D) * 4);
   }
   bp.total = off;
@@ -161,6 +164,56 @@ flare_status lat_merge(const float* part, int R, size_t rank_stride, int BH, int
 void exact_scores(LatParams& lp, float sc) {
   lp.qmul = 1.f;
   lp.smul = sc * kLog2e;
+}
+
+#ifndef FLARE_LAT_TC
+#define FLARE_LAT_TC 1
+#endif
+// The training backward's latent-parallel passes at D = 16 run on tcgen05
+// (lat_tc.cu) unless built with FLARE_LAT_TC=0 (the tf32 passes, kept for D = 32
+// and the self-contained backward).
+bool use_lat_tc(bool exact, int D) { return FLARE_LAT_TC && exact && D == 16; }
+
+// One tcgen05 latent-parallel pass: q16 bf16 queries ([G][M][D]), xa16 / xb16
+// the high and low parts of dZ (encoder) or Z (decoder), k16 / u16 the token
+// rows (K and V, or K and dY), and for the decoder L_n, delta_n; partials as
+// the tf32 passes write them ([B*H][S][M][D], S = bp.S splits of bp.tps
+// 64-token tiles).
+flare_status lat_tc(int mode, const BwdPlan& bp, uint8_t* ws, const void* q16, int q_per_batch, const void* xa16,
+                    const void* xb16, const void* k16, const void* u16, const float* ltok, const float* dtok,
+                    const float* lrow, const float* grow, float* part_q, float* part_z, int B, int H, int N, int M,
+                    int D, const int32_t* lengths, float sc, cudaStream_t s) {
+  const long BH = static_cast<long>(B) * H;
+  const long G = q_per_batch ? BH : H;
+  const int qrows = std::min(M, kLatBlock), T = lat_tc_tile();
+  LatTcMaps mp;
+  if (!map3d(&mp.q, q16, D, M, G, D, qrows, row_swizzle(D)) || !map3d(&mp.xa, xa16, D, M, BH, D, qrows, row_swizzle(D)) ||
+      !map3d(&mp.xb, xb16, D, M, BH, D, qrows, row_swizzle(D)) || !map3d(&mp.k, k16, D, N, BH, D, T, row_swizzle(D)) ||
+      !map3d(&mp.u, u16, D, N, BH, D, T, row_swizzle(D)))
+    return FLARE_ERR_LAUNCH;
+  if (mode == kLatTcDecoder && (!map2d_f32(&mp.l, ltok, N, BH, T, 1) || !map2d_f32(&mp.d, dtok, N, BH, T, 1)))
+    return FLARE_ERR_LAUNCH;
+  LatTcParams p{};
+  p.B = B; p.H = H; p.N = N; p.M = M; p.D = D;
+  p.q_per_batch = q_per_batch;
+  p.n_lblocks = static_cast<int>(cdiv(M, kLatBlock));
+  p.n_splits = bp.S;
+  p.split_tokens = bp.tps * kBwdTokTile;
+  p.q_rows = qrows;
+  p.c = sc * kLog2e;
+  p.lengths = lengths;
+  p.lrow = lrow; p.grow = grow;
+  p.part_q = part_q; p.part_z = part_z;
+  p.err = reinterpret_cast<uint32_t*>(ws + bp.fwd.off_err);
+  p.timeout_ns = wait_timeout_ns();
+  return launch_lat_tc(mode, mp, p, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+}
+
+// x (fp32 [rows][D]) into the high and low bf16 parts kept for the tcgen05 passes.
+flare_status split_hilo(const BwdPlan& bp, uint8_t* ws, const float* x, long n, cudaStream_t s) {
+  const SplitHiLoParams sp{n, x, reinterpret_cast<uint16_t*>(ws + bp.off_xhi16),
+                           reinterpret_cast<uint16_t*>(ws + bp.off_xlo16)};
+  return launch_split_hilo(sp, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
 
 flare_status pad(const float* src, float* dst, long rows, int D, float mul, cudaStream_t s) {
@@ -277,6 +330,11 @@ flare_status fl_phase(int phase, const BwdPlan& bp, uint8_t* ws, const FlArgs& a
       if (a.exact) tp.smul = c;
       if (launch_tok(kTokFull, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
       // encoder backward: its dQ partials
+      if (use_lat_tc(a.exact, D)) {
+        if ((st = split_hilo(bp, ws, dz32, BH * M * D, s)) != FLARE_OK) return st;
+        return lat_tc(kLatTcEncoder, bp, ws, a.Q, 0, ws + bp.off_xhi16, ws + bp.off_xlo16, k, v, nullptr, nullptr,
+                      lenc, gam, exch, nullptr, B, H, N, M, D, a.lengths, sc, s);
+      }
       LatParams le = lat_params(bp, ws, q32, 0, k, B, H, N, M, D, a.lengths, sc, a.sh);
       le.zrow = dz32; le.lrow = lenc; le.grow = gam; le.v = v;
       if (a.exact) exact_scores(le, sc);
@@ -421,7 +479,13 @@ flare_status pp_phase(int phase, const BwdPlan& bp, uint8_t* ws, const PpArgs& a
       tp.g32 = g32; tp.g_ld = 4 * C; tp.g_col_k = 0; tp.g_col_v = C;
       if (a.exact) tp.smul = c;
       if (launch_tok(kTokFull, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-      // encoder backward: its dQ(X) partials
+      // encoder backward: its dQ(X) partials (the tcgen05 pass takes the
+      // forward's bf16 Q(X))
+      if (use_lat_tc(a.exact, D)) {
+        if ((st = split_hilo(bp, ws, dz32, BH * M * D, s)) != FLARE_OK) return st;
+        return lat_tc(kLatTcEncoder, bp, ws, ws + bp.fwd.off_qx16, 1, ws + bp.off_xhi16, ws + bp.off_xlo16, kk, vv,
+                      nullptr, nullptr, lenc, gam, exch, nullptr, B, H, N, M, D, a.lengths, sc, s);
+      }
       LatParams le = lat_params(bp, ws, qx32, 1, kk, B, H, N, M, D, a.lengths, sc, a.sh);
       le.zrow = dz32; le.lrow = lenc; le.grow = gam; le.v = vv;
       if (a.exact) exact_scores(le, sc);
@@ -446,6 +510,11 @@ flare_status pp_phase(int phase, const BwdPlan& bp, uint8_t* ws, const PpArgs& a
       if (a.exact) tp.smul = c;
       if (launch_tok(kTokEncoder, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
       // ... and the partials of dQ0
+      if (use_lat_tc(a.exact, D)) {
+        if ((st = split_hilo(bp, ws, dqx32, BH * M * D, s)) != FLARE_OK) return st;
+        return lat_tc(kLatTcEncoder, bp, ws, a.Q0, 0, ws + bp.off_xhi16, ws + bp.off_xlo16, kt, vt, nullptr, nullptr,
+                      lsyn, gsyn, exch, nullptr, B, H, N, M, D, a.lengths, sc, s);
+      }
       LatParams le = lat_params(bp, ws, q32, 0, kt, B, H, N, M, D, a.lengths, sc, a.sh);
       le.zrow = dqx32; le.lrow = lsyn; le.grow = gsyn; le.v = vt;
       if (a.exact) exact_scores(le, sc);
@@ -666,9 +735,9 @@ flare_status train_prologue(const BwdPlan& bp, uint8_t* ws, const flare_bf16* Q,
 // The decoder's statistics (L_n, delta_n: from the training forward at
 // D = 16, recomputed otherwise) and its backward (the dZ and dQ partials into
 // `exch`), exact scores; q: the fp32 queries of the lat pass.
-flare_status train_decoder(const BwdPlan& bp, uint8_t* ws, const float* q, int q_per_batch, const void* k,
-                           const flare_bf16* dY, int B, int H, int N, int M, int D, const int32_t* lengths, float sc,
-                           float* exch, cudaStream_t s) {
+flare_status train_decoder(const BwdPlan& bp, uint8_t* ws, const float* q, const void* q16, int q_per_batch,
+                           const void* k, const flare_bf16* dY, int B, int H, int N, int M, int D,
+                           const int32_t* lengths, float sc, float* exch, cudaStream_t s) {
   const Shard sh{0, N, 1};
   float* ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
   float* dtok = reinterpret_cast<float*>(ws + bp.off_dtok);
@@ -691,13 +760,20 @@ flare_status train_decoder(const BwdPlan& bp, uint8_t* ws, const float* q, int q
     tp.ltok = ltok; tp.dtok = dtok;
     if (launch_tok(kTokStats, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   }
+  const size_t P = part_floats(bp, B, H, M, D, false);
+  // Z as the forward's bf16 Z and the low part it kept; the per-token L_n and
+  // delta_n rows go through fp32 tensor maps, whose row stride (4N bytes)
+  // must be a multiple of 16
+  if (use_lat_tc(true, D) && N % 4 == 0)
+    return lat_tc(kLatTcDecoder, bp, ws, q16, q_per_batch, ws + bp.fwd.off_z16, ws + bp.off_zlo16, k, dY, ltok, dtok,
+                  nullptr, nullptr, exch + P, exch, B, H, N, M, D, lengths, sc, s);
   LatParams ld = lat_params(bp, ws, q, q_per_batch, k, B, H, N, M, D, lengths, sc, sh);
   exact_scores(ld, sc);
   ld.zrow = reinterpret_cast<const float*>(ws + bp.off_z32);
   ld.dy = reinterpret_cast<const uint16_t*>(dY);
   ld.ltok = ltok; ld.dtok = dtok;
   ld.part_a = exch;
-  ld.part_b = exch + part_floats(bp, B, H, M, D, false);
+  ld.part_b = exch + P;
   return launch_lat(kLatDecoder, ld, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
 
@@ -743,8 +819,8 @@ flare_status flarepp_mixer_bwd_train(const flare_bf16* X, const flare_bf16* Wk, 
   float* pc = reinterpret_cast<float*>(ws + bp.off_pc);
   if ((st = train_prologue(bp, ws, Q0, reinterpret_cast<const uint16_t*>(ws + bp.fwd.off_qx16), BH, H, M, D, s)) !=
           FLARE_OK ||
-      (st = train_decoder(bp, ws, reinterpret_cast<const float*>(ws + bp.off_qx32), 1, ws + bp.fwd.off_kp, dY, B, H, N,
-                          M, D, lengths, a.sc, pa, s)) != FLARE_OK)
+      (st = train_decoder(bp, ws, reinterpret_cast<const float*>(ws + bp.off_qx32), ws + bp.fwd.off_qx16, 1,
+                          ws + bp.fwd.off_kp, dY, B, H, N, M, D, lengths, a.sc, pa, s)) != FLARE_OK)
     return st;
   // phases 3-6 of the seven (the exchanges stay in the workspace)
   float* ex[kPpPhases - 1] = {nullptr, nullptr, pa, pc, pc, reinterpret_cast<float*>(ws + bp.off_dwpart)};
@@ -784,8 +860,8 @@ flare_status flare_mixer_bwd_train(const flare_bf16* K, const flare_bf16* V, con
   float* pa = reinterpret_cast<float*>(ws + bp.off_pa);
   float* pc = reinterpret_cast<float*>(ws + bp.off_pc);
   if ((st = train_prologue(bp, ws, Q, nullptr, static_cast<long>(B) * H, H, M, D, s)) != FLARE_OK ||
-      (st = train_decoder(bp, ws, reinterpret_cast<const float*>(ws + bp.off_q32), 0, K, dY, B, H, N, M, D, lengths,
-                          a.sc, pa, s)) != FLARE_OK ||
+      (st = train_decoder(bp, ws, reinterpret_cast<const float*>(ws + bp.off_q32), Q, 0, K, dY, B, H, N, M, D,
+                          lengths, a.sc, pa, s)) != FLARE_OK ||
       (st = fl_phase(2, bp, ws, a, pa, pc, s)) != FLARE_OK || (st = fl_phase(3, bp, ws, a, pc, nullptr, s)) != FLARE_OK)
     return st;
   return set_train_mark(ws, bp, 0, s);

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace flare {
@@ -137,6 +138,44 @@ struct CvtParams {
   const uint16_t* src;
   float* dst;
 };
+
+// Latent-parallel backward passes on tcgen05 (lat_tc.cu; D = 16, bf16
+// queries, exact scores): the encoder's dQ partials, or the decoder's dQ and
+// dZ partials, per (head, 128-latent block, token split).
+constexpr int kLatTcEncoder = 0;
+constexpr int kLatTcDecoder = 1;
+struct LatTcParams {
+  int B, H, N, M, D;
+  int q_per_batch;              // queries [G][M][D] with G = B*H (1) or H (0)
+  int n_lblocks, n_splits;
+  int split_tokens;             // tokens per split (split s: [s*split_tokens, ...))
+  int q_rows;                   // rows of one query box: min(M, kLatBlock)
+  float c;                      // scale * log2(e), applied to the fp32 product
+  const int32_t* lengths;
+  const float* lrow;            // encoder: row log2-normaliser L_m [B*H][M]
+  const float* grow;            // encoder: gamma_m [B*H][M]
+  float* part_q;                // dQ partials [B*H][S][M][D]
+  float* part_z;                // decoder: dZ partials [B*H][S][M][D]
+  uint32_t* err;
+  unsigned long long timeout_ns;
+};
+// Tensor maps: q (bf16 [G][M][D]); xa, xb (bf16 [B*H][M][D]: the high and low
+// parts of dZ for the encoder, of Z for the decoder); k, u (bf16 [B*H][N][D]:
+// K and V for the encoder, K and dY for the decoder); l, d (fp32 [B*H][N]:
+// the decoder's L_n and delta_n).
+struct LatTcMaps {
+  CUtensorMap q, xa, xb, k, u, l, d;
+};
+cudaError_t launch_lat_tc(int mode, const LatTcMaps& m, const LatTcParams& p, cudaStream_t s);
+size_t lat_tc_smem_bytes();
+int lat_tc_tile();
+// hi[i] = bf16(x[i]), lo[i] = bf16(x[i] - hi[i]) for i < n (n even)
+struct SplitHiLoParams {
+  long n;
+  const float* x;
+  uint16_t *hi, *lo;
+};
+cudaError_t launch_split_hilo(const SplitHiLoParams& p, cudaStream_t s);
 
 // delta_n = <dY_n, Y_n> per token from a training forward's fp32 Y (0 for
 // padding tokens).

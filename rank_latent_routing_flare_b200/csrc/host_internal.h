@@ -11,6 +11,14 @@
 namespace flare {
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Tensor maps (api.cu): bf16 3-D [d2][d1][d0] with box (b0, b1, 1); fp32 2-D
+// [d1][d0] with box (b0, b1); the row swizzle of a D-wide bf16 operand.
+bool map3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1,
+           CUtensorMapSwizzle sw);
+bool map2d_f32(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint32_t b0, uint32_t b1);
+CUtensorMapSwizzle row_swizzle(int D);
+unsigned long long wait_timeout_ns();
 inline long cdiv(long a, long b) { return (a + b - 1) / b; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -42,7 +50,7 @@ struct BwdPlan {
   int S = 1, tps = 1, rpb = 32, LB = 1, dw_splits = 1;
   size_t off_q32 = 0, off_qx32 = 0, off_lsyn = 0, off_dqx32 = 0, off_gsyn = 0, off_z32 = 0, off_lenc = 0,
          off_ltok = 0, off_dtok = 0, off_dz32 = 0, off_gam = 0, off_fpart = 0, off_pa = 0, off_pc = 0,
-         off_g32 = 0, off_dwpart = 0, off_y32 = 0, off_zlo16 = 0, off_qpad = 0, off_q0pad = 0, off_zpad = 0, off_dzpad = 0,
+         off_g32 = 0, off_dwpart = 0, off_y32 = 0, off_zlo16 = 0, off_xhi16 = 0, off_xlo16 = 0, off_qpad = 0, off_q0pad = 0, off_zpad = 0, off_dzpad = 0,
          off_dqxpad = 0, off_dqxdec = 0, total = 0;
 };
 
