@@ -266,15 +266,14 @@ flare_status run_encode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
 flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_batch, const uint16_t* z16,
                         const void* k, void* y, int y_token_major, int B, int H, int N, int M, int D,
                         const int32_t* lengths, float scale, cudaStream_t st, bool pdl, int tok_offset = 0,
-                        int n_global = -1, float* y_f32 = nullptr, const uint16_t* zlo16 = nullptr,
+                        int n_global = -1, float* y_f32 = nullptr, int z_f16 = 0, const float* z32 = nullptr,
                         float* ltok_out = nullptr) {
   const long BH = static_cast<long>(B) * H;
   const long G = q_per_batch ? BH : H;
-  CUtensorMap tq, tz, tk, tzlo;
+  CUtensorMap tq, tz, tk;
   const int box_rows = std::min(M, 256);
   if (!map3d(&tq, q, D, M, G, D, box_rows, row_swizzle(D)) || !map3d(&tz, z16, D, M, BH, D, box_rows, row_swizzle(D)) ||
-      !map3d(&tk, k, D, N, BH, D, kDecTile, row_swizzle(D)) ||
-      (zlo16 != nullptr && !map3d(&tzlo, zlo16, D, M, BH, D, box_rows, row_swizzle(D))))
+      !map3d(&tk, k, D, N, BH, D, kDecTile, row_swizzle(D)))
     return FLARE_ERR_LAUNCH;
   DecodeParams dp{};
   dp.B = B; dp.H = H; dp.N = N; dp.M = M; dp.D = D;
@@ -289,7 +288,8 @@ flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
   dp.y = static_cast<uint16_t*>(y);
   dp.y_token_major = y_token_major;
   dp.y_f32 = y_f32;
-  dp.zlo = zlo16;
+  dp.z_f16 = z_f16;
+  dp.z32 = z32;
   dp.ltok_out = ltok_out;
   dp.tok_offset = tok_offset;
   dp.n_global = n_global < 0 ? N : n_global;
@@ -297,8 +297,7 @@ flare_status run_decode(const Plan& pl, uint8_t* ws, const void* q, int q_per_ba
   dp.fb_count = reinterpret_cast<uint32_t*>(ws + pl.off_err) + 1;
   dp.fb_list = reinterpret_cast<uint64_t*>(ws + pl.off_fb);
   dp.timeout_ns = wait_timeout_ns();
-  if (launch_decode(tq, tz, tk, zlo16 != nullptr ? &tzlo : nullptr, dp, st, pdl) != cudaSuccess)
-    return FLARE_ERR_LAUNCH;
+  if (launch_decode(tq, tz, tk, dp, st, pdl) != cudaSuccess) return FLARE_ERR_LAUNCH;
   return FLARE_OK;
 }
 
@@ -370,14 +369,13 @@ const char* flare_status_string(flare_status s) {
 namespace flare {
 
 // The FLARE forward (eq. 5-6) after nothing but the caller's arguments:
-// A training forward's decoder (FwdStats with zlo, D = 16) adds the low part
-// of Z: split it off the merged fp32 Z first.
-flare_status train_decode_inputs(const FwdStats* stats, const float* z32, const uint16_t* z16, int B, int H, int M,
-                                 int D, cudaStream_t s) {
-  if (stats == nullptr || stats->zlo == nullptr) return FLARE_OK;
+// A training forward's decoder (FwdStats with zf16, D = 16) takes Z in fp16:
+// convert the merged fp32 Z first.
+flare_status train_decode_inputs(const FwdStats* stats, const float* z32, int B, int H, int M, int D, cudaStream_t s) {
+  if (stats == nullptr || stats->zf16 == nullptr) return FLARE_OK;
   if (D != 16) return FLARE_ERR_UNSUPPORTED;
-  const SplitLoParams sp{static_cast<long>(B) * H * M * D, z32, z16, stats->zlo};
-  return launch_split_lo(sp, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+  const ToF16Params tp{static_cast<long>(B) * H * M * D, z32, stats->zf16};
+  return launch_to_f16(tp, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
 
 // checks, then key norms | encode | merge | decode on `stream`.
@@ -408,11 +406,11 @@ flare_status flare_fwd(const flare_bf16* K, const flare_bf16* V, const flare_bf1
   st = run_encode(pl, ws, Q, 0, K, V, kp.knorm, z32, z16, B, H, N, M, D, lengths, sc, s, stage_events, 2, pdl,
                   stats ? stats->lenc : nullptr);
   if (st != FLARE_OK) return st;
-  st = train_decode_inputs(stats, z32, z16, B, H, M, D, s);
+  st = train_decode_inputs(stats, z32, B, H, M, D, s);
   if (st != FLARE_OK) return st;
-  const bool lo = stats != nullptr && stats->zlo != nullptr;
-  st = run_decode(pl, ws, Q, 0, z16, K, Y, 0, B, H, N, M, D, lengths, sc, s, pdl, 0, -1, lo ? stats->y32 : Y_f32_out,
-                  lo ? stats->zlo : nullptr, lo ? stats->ltok : nullptr);
+  const bool f16 = stats != nullptr && stats->zf16 != nullptr;
+  st = run_decode(pl, ws, Q, 0, f16 ? stats->zf16 : z16, K, Y, 0, B, H, N, M, D, lengths, sc, s, pdl, 0, -1,
+                  f16 ? stats->y32 : Y_f32_out, f16 ? 1 : 0, f16 ? z32 : nullptr, f16 ? stats->ltok : nullptr);
   if (st != FLARE_OK) return st;
   return record(stage_events, 4, s) ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
@@ -557,11 +555,12 @@ flare_status flarepp_run(const Plan& pl, const flare_bf16* X, const flare_bf16* 
                   stats ? stats->lenc : nullptr);
   if (st != FLARE_OK) return st;
   // eq. 11: decode
-  st = train_decode_inputs(stats, z32, z16, B, H, M, D, s);
+  st = train_decode_inputs(stats, z32, B, H, M, D, s);
   if (st != FLARE_OK) return st;
-  const bool lo = stats != nullptr && stats->zlo != nullptr;
-  st = run_decode(pl, ws, qx16, 1, z16, kk, Y, y_token_major, B, H, N, M, D, lengths, sc, s, pdl, 0, -1,
-                  lo ? stats->y32 : Y_f32_out, lo ? stats->zlo : nullptr, lo ? stats->ltok : nullptr);
+  const bool f16 = stats != nullptr && stats->zf16 != nullptr;
+  st = run_decode(pl, ws, qx16, 1, f16 ? stats->zf16 : z16, kk, Y, y_token_major, B, H, N, M, D, lengths, sc, s, pdl,
+                  0, -1, f16 ? stats->y32 : Y_f32_out, f16 ? 1 : 0, f16 ? z32 : nullptr,
+                  f16 ? stats->ltok : nullptr);
   if (st != FLARE_OK) return st;
   return record(stage_events, 6, s) ? FLARE_OK : FLARE_ERR_LAUNCH;
 }

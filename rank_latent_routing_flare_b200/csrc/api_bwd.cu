@@ -68,11 +68,11 @@ BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C) {
     bp.off_g32 = take(static_cast<size_t>(B * N) * 4 * C * 4);
     bp.off_dwpart = take(static_cast<size_t>(bp.dw_splits) * C * 4 * C * 4);
   }
-  // the training pair at D = 16: the low part of Z and the forward's fp32 Y
+  // the training pair at D = 16: the forward's fp16 copy of Z and its fp32 Y
   // (FLARE++: in the gradient rows' space, which the backward fills only
   // after it has taken delta_n from Y)
   if (D == 16) {
-    bp.off_zlo16 = take(static_cast<size_t>(BH * M * D) * 2);
+    bp.off_zf16 = take(static_cast<size_t>(BH * M * D) * 2);
     // the high and low bf16 parts of dZ (then of dQ(X)) for the tcgen05 passes
     bp.off_xhi16 = take(static_cast<size_t>(BH * M * D) * 2);
     bp.off_xlo16 = take(static_cast<size_t>(BH * M * D) * 2);
@@ -688,7 +688,7 @@ FwdStats train_stats(const BwdPlan& bp, uint8_t* ws, int D) {
   FwdStats fs;
   fs.lenc = reinterpret_cast<float*>(ws + bp.off_lenc);
   if (D == 16) {
-    fs.zlo = reinterpret_cast<uint16_t*>(ws + bp.off_zlo16);
+    fs.zf16 = reinterpret_cast<uint16_t*>(ws + bp.off_zf16);
     fs.y32 = reinterpret_cast<float*>(ws + bp.off_y32);
     fs.ltok = reinterpret_cast<float*>(ws + bp.off_ltok);
   }
@@ -761,12 +761,16 @@ flare_status train_decoder(const BwdPlan& bp, uint8_t* ws, const float* q, const
     if (launch_tok(kTokStats, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
   }
   const size_t P = part_floats(bp, B, H, M, D, false);
-  // Z as the forward's bf16 Z and the low part it kept; the per-token L_n and
+  // Z as the high and low bf16 parts of the fp32 Z; the per-token L_n and
   // delta_n rows go through fp32 tensor maps, whose row stride (4N bytes)
   // must be a multiple of 16
-  if (use_lat_tc(true, D) && N % 4 == 0)
-    return lat_tc(kLatTcDecoder, bp, ws, q16, q_per_batch, ws + bp.fwd.off_z16, ws + bp.off_zlo16, k, dY, ltok, dtok,
+  if (use_lat_tc(true, D) && N % 4 == 0) {
+    flare_status st = split_hilo(bp, ws, reinterpret_cast<const float*>(ws + bp.off_z32),
+                                 static_cast<long>(B) * H * M * D, s);
+    if (st != FLARE_OK) return st;
+    return lat_tc(kLatTcDecoder, bp, ws, q16, q_per_batch, ws + bp.off_xhi16, ws + bp.off_xlo16, k, dY, ltok, dtok,
                   nullptr, nullptr, exch + P, exch, B, H, N, M, D, lengths, sc, s);
+  }
   LatParams ld = lat_params(bp, ws, q, q_per_batch, k, B, H, N, M, D, lengths, sc, sh);
   exact_scores(ld, sc);
   ld.zrow = reinterpret_cast<const float*>(ws + bp.off_z32);

@@ -26,12 +26,13 @@
 // full phase ahead of the party that waits on it.  The epilogue of a tile
 // (Y / sum, bf16 stores) runs after the first chunk of the next tile.
 //
-// With ZLO (the training forward, D = 16) Z also has a low part Zlo =
-// Z - bf16(Z) in shared memory and each chunk adds P Zlo_c into Y (a second
-// value MMA of N = D, no ones block), so that Y, and the fp32 copy the
-// backward takes delta_n from, see Z to fp32 accuracy; the epilogue also
-// writes L_n.  The extra 16 KB of shared memory leave room for three CTAs per
-// SM instead of four.
+// With F16 (the training forward, D = 16) the value product runs on fp16
+// operands: Z as fp16 (11-bit mantissa instead of bf16's 8) and the weights
+// as fp16 P' = 2^(S c - nu + 14), scaled by 2^14 so that weights down to
+// 2^-28 of the bound keep full fp16 precision (the scale cancels in Y = acc /
+// sum).  Y, and the fp32 copy the backward takes delta_n from, then see Z to
+// 2^-12; the epilogue also writes L_n.  Rows whose scaled sum falls below
+// 2^-14 (a bound looser than 28 in log2 units) go to the exact fallback.
 //
 // Warp roles (5 warps): warp 0 lane 0 is the MMA thread (it also loads Q, Z
 // and the first key tiles).  Warps 1..4 are the softmax warps (thread <->
@@ -45,9 +46,9 @@
 namespace flare {
 namespace {
 
-template <int D, bool ZLO>
+template <int D, bool F16>
 struct DecCfg {
-  static_assert(!ZLO || D == 16, "the low part of Z is kept for D = 16 only");
+  static_assert(!F16 || D == 16, "the fp16 value product is built for D = 16 only");
   static constexpr int C = dec_chunk(D);                // latents per chunk
   static constexpr int ROWB = D * 2;
   static constexpr int KT_B = kDecTile * ROWB;          // one key tile
@@ -59,8 +60,7 @@ struct DecCfg {
   static constexpr int NB = dec_bufs(D);                // score buffers
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_Z = OFF_Q + QZ_B;
-  static constexpr int OFF_ZLO = OFF_Z + QZ_B;          // (ZLO) the low part of Z
-  static constexpr int OFF_ONES = OFF_ZLO + (ZLO ? QZ_B : 0);  // C x ROWB block of ones
+  static constexpr int OFF_ONES = OFF_Z + QZ_B;         // C x ROWB block of ones
   static constexpr int OFF_K = OFF_ONES + C * ROWB;     // NST * KT_B
   static constexpr int OFF_BAR = OFF_K + NST * KT_B;
   static constexpr int OFF_MISC = OFF_BAR + 8 * (4 + NST + 3 * NB);
@@ -69,7 +69,7 @@ struct DecCfg {
   static constexpr uint32_t COL_Y = NB * C;
   static constexpr uint32_t TMEM_COLS = (COL_Y + NY <= 128) ? 128 : 256;
   static constexpr int THREADS = 160;
-  static constexpr int CTAS_PER_SM = ZLO ? 3 : dec_ctas_per_sm(D);
+  static constexpr int CTAS_PER_SM = dec_ctas_per_sm(D);
   static_assert(TMEM_COLS <= 512 / CTAS_PER_SM, "TMEM columns of the co-resident CTAs exceed 512");
   static_assert(COL_Y + NY <= TMEM_COLS, "score buffers and Y exceed the allocation");
   static_assert(OFF_K % 512 == 0 || D == 16, "key tiles must start on a swizzle atom");
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(128) decode_fallback_kernel(const DecodeParams
     const uint16_t* krow = p.k + (static_cast<size_t>(bh) * p.N + n) * D;
     const uint16_t* qg = p.q + static_cast<size_t>(g) * p.M * D;
     const uint16_t* zh = p.z + static_cast<size_t>(bh) * p.M * D;
-    const uint16_t* zl = p.zlo != nullptr ? p.zlo + static_cast<size_t>(bh) * p.M * D : nullptr;
+    const float* zf = p.z32 != nullptr ? p.z32 + static_cast<size_t>(bh) * p.M * D : nullptr;
     float k[D], y[D];
 #pragma unroll
     for (int d = 0; d < D; ++d) k[d] = __uint_as_float(static_cast<uint32_t>(krow[d]) << 16);
@@ -137,11 +137,12 @@ __global__ void __launch_bounds__(128) decode_fallback_kernel(const DecodeParams
       for (int d = 0; d < D; ++d) s = fmaf(k[d], __uint_as_float(static_cast<uint32_t>(qg[m * D + d]) << 16), s);
       const float w = exp2f(s * p.c - mx);
       den += w;
+      if (zf != nullptr) {
 #pragma unroll
-      for (int d = 0; d < D; ++d) y[d] = fmaf(w, __uint_as_float(static_cast<uint32_t>(zh[m * D + d]) << 16), y[d]);
-      if (zl != nullptr) {
+        for (int d = 0; d < D; ++d) y[d] = fmaf(w, zf[m * D + d], y[d]);
+      } else {
 #pragma unroll
-        for (int d = 0; d < D; ++d) y[d] = fmaf(w, __uint_as_float(static_cast<uint32_t>(zl[m * D + d]) << 16), y[d]);
+        for (int d = 0; d < D; ++d) y[d] = fmaf(w, __uint_as_float(static_cast<uint32_t>(zh[m * D + d]) << 16), y[d]);
       }
     }
     const float inv = 1.f / den;
@@ -162,18 +163,16 @@ __global__ void __launch_bounds__(128) decode_fallback_kernel(const DecodeParams
   }
 }
 
-template <int D, bool ZLO>
-__global__ void __launch_bounds__(DecCfg<D, ZLO>::THREADS, DecCfg<D, ZLO>::CTAS_PER_SM)
+template <int D, bool F16>
+__global__ void __launch_bounds__(DecCfg<D, F16>::THREADS, DecCfg<D, F16>::CTAS_PER_SM)
     decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_z,
-                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_zlo,
-                  const DecodeParams p) {
-  using Cfg = DecCfg<D, ZLO>;
+                  const __grid_constant__ CUtensorMap tm_k, const DecodeParams p) {
+  using Cfg = DecCfg<D, F16>;
   constexpr int NST = Cfg::NST, C = Cfg::C, NB = Cfg::NB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sq = sm + Cfg::OFF_Q;
   uint8_t* sz = sm + Cfg::OFF_Z;
-  uint8_t* szlo = sm + Cfg::OFF_ZLO;
   uint8_t* sones = sm + Cfg::OFF_ONES;
   uint8_t* sk = sm + Cfg::OFF_K;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Cfg::OFF_BAR);
@@ -246,7 +245,7 @@ __global__ void __launch_bounds__(DecCfg<D, ZLO>::THREADS, DecCfg<D, ZLO>::CTAS_
     fence_mbar_init();
   }
   for (int i = threadIdx.x; i < C * Cfg::ROWB / 4; i += blockDim.x)
-    reinterpret_cast<uint32_t*>(sones)[i] = 0x3F803F80u;  // bf16 1.0 pairs
+    reinterpret_cast<uint32_t*>(sones)[i] = F16 ? 0x3C003C00u : 0x3F803F80u;  // 1.0 pairs (fp16 or bf16)
   fence_proxy_async_smem();
   if (warp == 0) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
@@ -275,17 +274,14 @@ __global__ void __launch_bounds__(DecCfg<D, ZLO>::THREADS, DecCfg<D, ZLO>::CTAS_
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_z);
       tma_prefetch_desc(&tm_k);
-      if constexpr (ZLO) tma_prefetch_desc(&tm_zlo);
       const int nbox = (p.M + p.qz_box_rows - 1) / p.qz_box_rows;
-      mbar_arrive_expect_tx(qz_full, (ZLO ? 3 : 2) * nbox * p.qz_box_rows * Cfg::ROWB);
+      mbar_arrive_expect_tx(qz_full, 2 * nbox * p.qz_box_rows * Cfg::ROWB);
       for (int bx = 0; bx < nbox; ++bx) {
         tma_load_3d(sq + bx * p.qz_box_rows * Cfg::ROWB, &tm_q, qz_full, 0, bx * p.qz_box_rows, g);
         tma_load_3d(sz + bx * p.qz_box_rows * Cfg::ROWB, &tm_z, qz_full, 0, bx * p.qz_box_rows, bh);
-        if constexpr (ZLO)
-          tma_load_3d(szlo + bx * p.qz_box_rows * Cfg::ROWB, &tm_zlo, qz_full, 0, bx * p.qz_box_rows, bh);
       }
       for (int n = 0; n < min(NST, ntiles); ++n) load_tile(n);
-      const uint32_t idesc_y = idesc_bf16_f32(128, Cfg::NY, false, true);
+      const uint32_t idesc_y = F16 ? idesc_f16_f32(128, Cfg::NY, false, true) : idesc_bf16_f32(128, Cfg::NY, false, true);
       const uint32_t sz_a = smem_u32(sz), ones_a = smem_u32(sones);
       const uint64_t q_desc = umma_desc(smem_u32(sq), 16, Cfg::SBO, Cfg::LAYOUT);
       const uint64_t k_desc = umma_desc(smem_u32(sk), 16, Cfg::SBO, Cfg::LAYOUT);
@@ -307,9 +303,6 @@ __global__ void __launch_bounds__(DecCfg<D, ZLO>::THREADS, DecCfg<D, ZLO>::CTAS_
       // [Z_c | 1]: chunk c starts CH_STEP * c further on, and its ones block
       // (leading byte offset) is that much closer
       const uint64_t z_desc = umma_desc(sz_a, ones_a - sz_a, Cfg::SBO, Cfg::LAYOUT);
-      // Zlo_c alone (N = D: one block, its leading byte offset unused)
-      const uint64_t zlo_desc = umma_desc(smem_u32(szlo), 16, Cfg::SBO, Cfg::LAYOUT);
-      const uint32_t idesc_ylo = idesc_bf16_f32(128, D, false, true);
       // S_q = K_tile Q_c^T into buffer q % NB, once the key tile has landed and
       // P_{q-NB} has been consumed
       auto issue_s = [&](const Cursor& x) -> bool {
@@ -341,14 +334,6 @@ __global__ void __launch_bounds__(DecCfg<D, ZLO>::THREADS, DecCfg<D, ZLO>::CTAS_
           if (ks < nks)
             umma_ts(tmem + Cfg::COL_Y, tmem + buf * C + ks * 8,
                     zd + static_cast<uint64_t>((ks * 16 * Cfg::ROWB) >> 4), idesc_y, (x.cc > 0 || ks > 0) ? 1u : 0u);
-        if constexpr (ZLO) {
-          const uint64_t zld = zlo_desc + step;
-#pragma unroll
-          for (int ks = 0; ks < C / 16; ++ks)
-            if (ks < nks)
-              umma_ts(tmem + Cfg::COL_Y, tmem + buf * C + ks * 8,
-                      zld + static_cast<uint64_t>((ks * 16 * Cfg::ROWB) >> 4), idesc_ylo, 1u);
-        }
         umma_commit(pv_done + buf);
         if (x.cc == nc - 1) umma_commit(y_full);
         return true;
@@ -411,7 +396,9 @@ __global__ void __launch_bounds__(DecCfg<D, ZLO>::THREADS, DecCfg<D, ZLO>::CTAS_
       mbar_arrive_warp(y_free);  // the next tile's first value MMA may overwrite Y
       const int n = (ta + i) * kDecTile + r;
       // lost mass < M * 2^-126 per token; 2^-90 keeps it below 2^-27 relative
-      const bool exact = n < L && !(l >= 0x1p-90f);
+      // F16: the weights carry 2^14, and a sum below 2^-14 means weights in
+      // fp16's subnormal range
+      const bool exact = n < L && !(l >= (F16 ? 0x1p-14f : 0x1p-90f));
       if (n < L) {
         const float inv = 1.f / l;
 #pragma unroll
@@ -420,9 +407,9 @@ __global__ void __launch_bounds__(DecCfg<D, ZLO>::THREADS, DecCfg<D, ZLO>::CTAS_
 #pragma unroll
         for (int d = 0; d < D; ++d) y[d] = 0.f;
       }
-      if constexpr (ZLO) {  // L_n for the training backward
+      if constexpr (F16) {  // L_n for the training backward (the weights carry 2^14)
         if (p.ltok_out != nullptr && n < p.N && !exact)
-          p.ltok_out[static_cast<size_t>(bh) * p.N + n] = n < L ? nu_i + log2f(l) : 0.f;
+          p.ltok_out[static_cast<size_t>(bh) * p.N + n] = n < L ? nu_i - 14.f + log2f(l) : 0.f;
       }
       if (exact) {  // recomputed exactly by decode_fallback_kernel
         const uint32_t e = atomicAdd(p.fb_count, 1u);
@@ -445,18 +432,19 @@ __global__ void __launch_bounds__(DecCfg<D, ZLO>::THREADS, DecCfg<D, ZLO>::CTAS_
     // first 16 columns are exponentiated while the rest are read from TMEM
     auto run_chunk = [&](auto cn_tag, uint32_t cb, float nu) {
       constexpr int CN = decltype(cn_tag)::value;
+      const float nu_p = F16 ? nu - 14.f : nu;  // F16: weights scaled by 2^14
       uint32_t s0[16], pk[CN / 2];
       tmem_ld16(cb, s0);
       tmem_wait_ld();
       if constexpr (CN > 16) {
         uint32_t s1[CN - 16];
         tmem_ld_cols<CN - 16>(cb + 16, s1);
-        exp2_row<16, FLARE_DEC_POLY_PAIRS>(s0, c, nu, *reinterpret_cast<uint32_t(*)[8]>(&pk[0]));
+        exp2_row<16, FLARE_DEC_POLY_PAIRS, 0, F16>(s0, c, nu_p, *reinterpret_cast<uint32_t(*)[8]>(&pk[0]));
         tmem_wait_ld();
-        exp2_row<CN - 16, FLARE_DEC_POLY_PAIRS, 8>(s1, c, nu,
+        exp2_row<CN - 16, FLARE_DEC_POLY_PAIRS, 8, F16>(s1, c, nu_p,
                                                    *reinterpret_cast<uint32_t(*)[(CN - 16) / 2]>(&pk[8]));
       } else {
-        exp2_row<16, FLARE_DEC_POLY_PAIRS>(s0, c, nu, pk);
+        exp2_row<16, FLARE_DEC_POLY_PAIRS, 0, F16>(s0, c, nu_p, pk);
       }
       tmem_st_cols<CN / 2>(cb, pk);  // P over the first CN/2 columns of the chunk's scores
       tmem_wait_st();
@@ -472,7 +460,7 @@ __global__ void __launch_bounds__(DecCfg<D, ZLO>::THREADS, DecCfg<D, ZLO>::CTAS_
         // tile's stage is refilled only after every warp is past this point
         if (!mbar_wait_warp(k_full + tile % NST, (tile / NST) & 1, wc)) { ok = false; break; }
         const uint4* krow_s = reinterpret_cast<const uint4*>(sk + (tile % NST) * Cfg::KT_B + r * Cfg::ROWB);
-        if constexpr (ZLO) nu_prev = nu;
+        if constexpr (F16) nu_prev = nu;
         nu = c * sqrtf(bf16_row_norm2(krow_s, D / 8)) * qm;
       }
       const int cn = min(C, p.M - cc * C);
@@ -513,32 +501,27 @@ __global__ void __launch_bounds__(DecCfg<D, ZLO>::THREADS, DecCfg<D, ZLO>::CTAS_
 
 }  // namespace
 
-size_t decode_smem_bytes(int D, bool zlo) {
-  const size_t need =
-      (D == 16 ? (zlo ? DecCfg<16, true>::BYTES : DecCfg<16, false>::BYTES) : DecCfg<32, false>::BYTES) + 1024;
-  // at most as many CTAs per SM as the kernel's launch bounds name (228 KB
-  // each, 1 KB of it reserved per CTA), so that every resident CTA finds its
-  // TMEM columns free
-  const int ctas = D == 16 ? (zlo ? DecCfg<16, true>::CTAS_PER_SM : DecCfg<16, false>::CTAS_PER_SM)
-                           : DecCfg<32, false>::CTAS_PER_SM;
-  const size_t floor = (228 * 1024) / (ctas + 1) + 1024;
+size_t decode_smem_bytes(int D) {
+  const size_t need = (D == 16 ? DecCfg<16, false>::BYTES : DecCfg<32, false>::BYTES) + 1024;
+  // at most dec_ctas_per_sm(D) CTAs per SM (228 KB each, 1 KB of it
+  // reserved per CTA), so that every resident CTA finds its TMEM columns free
+  const size_t floor = (228 * 1024) / (dec_ctas_per_sm(D) + 1) + 1024;
   return need > floor ? need : floor;
 }
 
 cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_z, const CUtensorMap& tm_k,
-                          const CUtensorMap* tm_zlo, const DecodeParams& p, cudaStream_t s, bool pdl) {
-  const bool zlo = tm_zlo != nullptr;
-  if (zlo && (p.D != 16 || p.zlo == nullptr)) return cudaErrorInvalidValue;
-  const size_t smem = decode_smem_bytes(p.D, zlo);
+                          const DecodeParams& p, cudaStream_t s, bool pdl) {
+  if (p.z_f16 && p.D != 16) return cudaErrorInvalidValue;
+  const size_t smem = decode_smem_bytes(p.D);
   const dim3 grid(static_cast<unsigned>(p.B * p.H * p.ctas_per_head));
   auto go = [&](auto kern, int threads) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     LaunchCfg lc(grid, dim3(threads), smem, s, pdl);
-    return cudaLaunchKernelEx(&lc.cfg, kern, tm_q, tm_z, tm_k, zlo ? *tm_zlo : tm_z, p);
+    return cudaLaunchKernelEx(&lc.cfg, kern, tm_q, tm_z, tm_k, p);
   };
   cudaError_t e = p.D != 16 ? go(decode_kernel<32, false>, DecCfg<32, false>::THREADS)
-                  : zlo     ? go(decode_kernel<16, true>, DecCfg<16, true>::THREADS)
+                  : p.z_f16 ? go(decode_kernel<16, true>, DecCfg<16, true>::THREADS)
                             : go(decode_kernel<16, false>, DecCfg<16, false>::THREADS);
   if (e != cudaSuccess) return e;
   // the fallback follows the decoder on the same stream: always programmatic

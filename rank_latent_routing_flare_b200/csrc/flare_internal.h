@@ -189,9 +189,11 @@ struct DecodeParams {
   uint16_t* y;          // bf16 [B*H][N][D], or [B][N][H*D] when y_token_major
   int y_token_major;
   float* y_f32;         // optional fp32 copy of Y ([B*H][N][D], the values Y is rounded from), or nullptr
-  // optional (the training forward, D = 16): the low bf16 part of Z
-  // (Z - bf16(Z), [B*H][M][D]); Y then takes Z as the sum of both parts
-  const uint16_t* zlo;
+  // the training forward's variant (D = 16): z holds fp16 bits of Z and the
+  // softmax weights enter the value product in fp16 (scaled by 2^14), so
+  // that Y sees Z to 2^-12; the exact fallback takes z32 (fp32 Z)
+  int z_f16;
+  const float* z32;
   float* ltok_out;      // optional [B*H][N]: L_n = log2 sum_m 2^(c <k_n, q_m>) per token (0 for padding)
   uint32_t* fb_count;   // number of listed tokens (zeroed before the decoder runs)
   uint64_t* fb_list;    // tokens (bh * N + n) whose row sum underflowed, capacity B*H*N
@@ -233,24 +235,21 @@ cudaError_t launch_knorm(const KnormParams& p, cudaStream_t s);
 cudaError_t launch_encode(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                           const EncodeParams& p, cudaStream_t s, bool pdl = false);
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t s, bool pdl = false);
-// lo[i] = bf16(full[i] - hi[i]) for i < n (n even): the low bf16 part of an
-// fp32 tensor whose high part hi = bf16(full) is stored.
-struct SplitLoParams {
+// dst[i] = fp16(src[i]) for i < n (n even).
+struct ToF16Params {
   long n;
-  const float* full;
-  const uint16_t* hi;
-  uint16_t* lo;
+  const float* src;
+  uint16_t* dst;
 };
-cudaError_t launch_split_lo(const SplitLoParams& p, cudaStream_t s);
+cudaError_t launch_to_f16(const ToF16Params& p, cudaStream_t s);
 cudaError_t launch_cp_exact(const MergeParams& p, int rank, float* out, cudaStream_t s);
-// tm_zlo: the low part of Z (the training forward's variant, D = 16), or nullptr.
 cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_z, const CUtensorMap& tm_k,
-                          const CUtensorMap* tm_zlo, const DecodeParams& p, cudaStream_t s, bool pdl = false);
+                          const DecodeParams& p, cudaStream_t s, bool pdl = false);
 cudaError_t launch_wait_selftest(uint32_t* err, unsigned long long timeout_ns, cudaStream_t s);
 
 // Shared-memory footprints (bytes) of the pipelined kernels.
 size_t encode_smem_bytes(int D);
-size_t decode_smem_bytes(int D, bool zlo);
+size_t decode_smem_bytes(int D);
 size_t project_smem_bytes(int C);
 
 }  // namespace flare

@@ -50,7 +50,7 @@ struct BwdPlan {
   int S = 1, tps = 1, rpb = 32, LB = 1, dw_splits = 1;
   size_t off_q32 = 0, off_qx32 = 0, off_lsyn = 0, off_dqx32 = 0, off_gsyn = 0, off_z32 = 0, off_lenc = 0,
          off_ltok = 0, off_dtok = 0, off_dz32 = 0, off_gam = 0, off_fpart = 0, off_pa = 0, off_pc = 0,
-         off_g32 = 0, off_dwpart = 0, off_y32 = 0, off_zlo16 = 0, off_xhi16 = 0, off_xlo16 = 0, off_qpad = 0, off_q0pad = 0, off_zpad = 0, off_dzpad = 0,
+         off_g32 = 0, off_dwpart = 0, off_y32 = 0, off_zf16 = 0, off_xhi16 = 0, off_xlo16 = 0, off_qpad = 0, off_q0pad = 0, off_zpad = 0, off_dzpad = 0,
          off_dqxpad = 0, off_dqxdec = 0, total = 0;
 };
 
@@ -68,12 +68,12 @@ flare_status check_flarepp(const void* X, const void* Wk, const void* Wv, const 
 
 // Statistics a training forward leaves for the backward (each optional):
 // the row log-normalisers of the synthesis and the encode ([B*H][M]), in
-// log2 units; and, with zlo (D = 16), the low bf16 part of Z that the decoder
-// adds so that Y sees Z to fp32 accuracy, the fp32 Y and the decoder's
-// per-token log-normalisers ([B*H][N]).
+// log2 units; and, with zf16 (D = 16), where the decoder's fp16 copy of Z
+// goes (its value product then runs in fp16, so that Y sees Z to 2^-12), the
+// fp32 Y and the decoder's per-token log-normalisers ([B*H][N]).
 struct FwdStats {
   float *lsyn = nullptr, *lenc = nullptr;
-  uint16_t* zlo = nullptr;
+  uint16_t* zf16 = nullptr;
   float *y32 = nullptr, *ltok = nullptr;
 };
 

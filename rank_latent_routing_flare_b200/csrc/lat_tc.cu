@@ -20,37 +20,43 @@
 // score scale c = scale log2(e) is applied to the fp32 product, as in the
 // forward's kernels, so that the forward's normalisers L_m fit these scores.
 //
-// Tiles of T = 32 tokens stream through a TMA ring (K and V, or K and dY,
-// plus L_n and delta_n for the decoder).  TMEM holds two score buffers, S and
-// G of a tile each (buffer b: S at column 64b, G at 64b + 32), and the dQ
-// (column 128) and dZ (144) accumulators: 256 columns, two CTAs per SM.  Tile
-// i uses buffer i % 2 and is worked on by softmax warpgroup i % 2, so one
-// warpgroup's exponentials overlap the MMAs of the other's tile.  The softmax
-// threads read a tile's S and G in 16-column pieces and write, over the piece
-// they have read, dS as bf16 high and low parts (S columns [16j, 16j+8) and
+// Tiles of T = 48 tokens stream through a TMA ring (K and V, or K and dY,
+// plus L_n and delta_n for the decoder).  TMEM: S at column 0, G at 48, dQ at
+// 96, dZ at 112 (128 columns: four CTAs per SM).  The softmax threads read a
+// tile's S and G in three 16-column pieces (the next piece's TMEM load in
+// flight while the current one is computed) and write, over the piece they
+// have read, dS as bf16 high and low parts (S columns [16j, 16j+8) and
 // [16j+8, 16j+16)) and, for the decoder, W in bf16 (G columns [16j, 16j+8)):
 // each 16-token k-step of the value MMAs then takes its A operand from 8
-// consecutive columns.  The MMA thread issues S and G of tile i, then the
-// value MMAs of tile i - 1 once its warpgroup has stored dS, and reuses a
-// buffer once the value MMAs that read it are done.
+// consecutive columns.  One score buffer: the MMA thread issues the next
+// tile's S and G once the value MMAs of the previous tile are done; the four
+// co-resident CTAs of an SM fill each other's gaps.
 //
-// Warp roles (9 warps): warp 0 lane 0 issues the TMA loads and the MMAs;
-// warps 1..4 and 5..8 are the two softmax warpgroups (thread <-> TMEM lane
-// <-> latent row).
+// Warp roles (5 warps): warp 0 lane 0 issues the TMA loads and the MMAs;
+// warps 1..4 are the softmax warps (thread <-> TMEM lane <-> latent row).
 #include "bwd_internal.h"
 #include "ptx.cuh"
 
 namespace flare {
 namespace {
 
+// After tcgen05.wait::ld: the registers a TMEM load wrote are defined here,
+// so that no use of them is scheduled before the wait.
+__device__ __forceinline__ void regs_defined(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]));
+}
+
 struct LatTcCfg {
   static constexpr int D = 16;
-  static constexpr int T = 32;                          // tokens per tile
+  static constexpr int T = 48;                          // tokens per tile
   static constexpr int ROWB = D * 2;                    // bytes of one bf16 row
   static constexpr int TILE_B = T * ROWB;               // one K, V or dY tile
   static constexpr int ROWS_B = kLatBlock * ROWB;       // Q, or one part of dZ / Z
   static constexpr int LD_B = 256;                      // one tile's L_n or delta_n (T floats, padded)
-  static constexpr int NST = 8;                         // ring stages
+  static constexpr int NST = 6;                         // ring stages
   static constexpr uint32_t LAYOUT = LAYOUT_SW32;
   static constexpr uint32_t SBO = 8 * ROWB;
   static constexpr int OFF_Q = 0;
@@ -60,13 +66,12 @@ struct LatTcCfg {
   static constexpr int OFF_U = OFF_K + NST * TILE_B;    // NST x (V or dY) tile
   static constexpr int OFF_LD = OFF_U + NST * TILE_B;   // NST x (L_n | delta_n)
   static constexpr int OFF_BAR = OFF_LD + NST * 2 * LD_B;
-  static constexpr int OFF_MISC = OFF_BAR + 8 * (8 + NST);
+  static constexpr int OFF_MISC = OFF_BAR + 8 * (6 + NST);
   static constexpr int BYTES = OFF_MISC + 64 + NST * 4;
-  static constexpr uint32_t BUF = 2 * T;                // columns of one score buffer (S | G)
-  static constexpr uint32_t COL_S = 0, COL_G = T, COL_DQ = 2 * BUF, COL_DZ = 2 * BUF + D;
-  static constexpr uint32_t TMEM_COLS = 256;
-  static constexpr int THREADS = 288;
-  static constexpr int CTAS_PER_SM = 2;
+  static constexpr uint32_t COL_S = 0, COL_G = T, COL_DQ = 2 * T, COL_DZ = 2 * T + D;
+  static constexpr uint32_t TMEM_COLS = 128;
+  static constexpr int THREADS = 160;
+  static constexpr int CTAS_PER_SM = 4;
   static_assert(COL_DZ + D <= TMEM_COLS, "TMEM columns");
   static_assert(TILE_B % 256 == 0 && ROWS_B % 1024 == 0, "tiles must hold whole swizzle atoms");
   static_assert(T % 16 == 0 && T * 4 <= LD_B, "tile of L_n / delta_n");
@@ -91,11 +96,11 @@ __global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
   uint8_t* sld = sm + Cfg::OFF_LD;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Cfg::OFF_BAR);
   uint64_t* q_full = bars;                 // Q and both parts of dZ / Z landed
-  uint64_t* o_full = bars + 1;             // every MMA of the CTA done
-  uint64_t* s_full = bars + 2;             // [2] S and G of the buffer's tile computed
-  uint64_t* p_full = bars + 4;             // [2] dS (and W) stored by the buffer's warpgroup
-  uint64_t* pv_done = bars + 6;            // [2] the value MMAs reading the buffer done
-  uint64_t* kv_full = bars + 8;            // [NST] ring stage landed
+  uint64_t* s_full = bars + 1;             // S and G of the current tile computed
+  uint64_t* p_full = bars + 2;             // dS (and W) stored by every softmax warp
+  uint64_t* pv_done = bars + 3;            // the value MMAs of the tile done
+  uint64_t* o_full = bars + 4;             // every MMA of the CTA done
+  uint64_t* kv_full = bars + 6;            // [NST] ring stage landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(sm + Cfg::OFF_MISC + 4);
   volatile int* last_load = reinterpret_cast<volatile int*>(sm + Cfg::OFF_MISC + 64);  // per stage
@@ -131,12 +136,10 @@ __global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(pv_done, 1);
     mbar_init(o_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(s_full + i, 1);
-      mbar_init(p_full + i, 4);
-      mbar_init(pv_done + i, 1);
-    }
     for (int i = 0; i < NST; ++i) {
       mbar_init(kv_full + i, 1);
       last_load[i] = -1;
@@ -192,49 +195,40 @@ __global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
       const uint64_t k_desc = umma_desc(smem_u32(sk), 16, Cfg::SBO, Cfg::LAYOUT);
       const uint64_t u_desc = umma_desc(smem_u32(su), 16, Cfg::SBO, Cfg::LAYOUT);
       constexpr uint64_t STAGE = Cfg::TILE_B >> 4, KSTEP = (16 * Cfg::ROWB) >> 4;
-      // the value MMAs of tile j (buffer j % 2, ring stage j % NST), once its
-      // warpgroup has stored dS (and W)
-      auto issue_values = [&](int j) -> bool {
-        const int bj = j & 1, sj = j % NST;
-        if (!mbar_wait_mma(p_full + bj, (j >> 1) & 1, wc)) return false;
-        tc_fence_after();
-        const uint64_t kd = k_desc + sj * STAGE, ud = u_desc + sj * STAGE;
-        const uint32_t cs = tmem + bj * Cfg::BUF + Cfg::COL_S, cg = tmem + bj * Cfg::BUF + Cfg::COL_G;
-#pragma unroll
-        for (int ks = 0; ks < T / 16; ++ks) {
-          umma_ts(tmem + Cfg::COL_DQ, cs + 16 * ks, kd + ks * KSTEP, idesc_v, (j > 0 || ks > 0) ? 1u : 0u);  // dShi K
-          umma_ts(tmem + Cfg::COL_DQ, cs + 16 * ks + 8, kd + ks * KSTEP, idesc_v, 1u);                      // dSlo K
-          if (DEC)
-            umma_ts(tmem + Cfg::COL_DZ, cg + 16 * ks, ud + ks * KSTEP, idesc_v, (j > 0 || ks > 0) ? 1u : 0u);  // W dY
-        }
-        umma_commit(pv_done + bj);
-        return true;
-      };
       bool ok = mbar_wait_mma(q_full, 0, wc);
       for (int i = 0; ok && i < ntiles; ++i) {
-        const int bi = i & 1, st = i % NST;
-        if (i >= 2) {
-          // the value MMAs of tile i - 2 are done: its buffer may be
-          // overwritten, and its ring stage takes tile i - 2 + NST
-          if (!mbar_wait_mma(pv_done + bi, ((i - 2) >> 1) & 1, wc)) { ok = false; break; }
-          if (i - 2 + NST < ntiles) load_tile(i - 2 + NST);
+        const int st = i % NST;
+        if (i > 0) {
+          // the value MMAs of tile i - 1 are done: S and G may be overwritten,
+          // and tile i - 1's stage takes tile i - 1 + NST
+          if (!mbar_wait_mma(pv_done, (i - 1) & 1, wc)) { ok = false; break; }
+          if (i - 1 + NST < ntiles) load_tile(i - 1 + NST);
         }
         if (!mbar_wait_mma(kv_full + st, (i / NST) & 1, wc)) { ok = false; break; }
         tc_fence_after();
         const uint64_t kd = k_desc + st * STAGE, ud = u_desc + st * STAGE;
-        umma_ss(tmem + bi * Cfg::BUF + Cfg::COL_S, q_desc, kd, idesc_s, 0u);
-        umma_ss(tmem + bi * Cfg::BUF + Cfg::COL_G, xa_desc, ud, idesc_s, 0u);
-        umma_ss(tmem + bi * Cfg::BUF + Cfg::COL_G, xb_desc, ud, idesc_s, 1u);
-        umma_commit(s_full + bi);
-        if (i >= 1 && !issue_values(i - 1)) { ok = false; break; }
+        umma_ss(tmem + Cfg::COL_S, q_desc, kd, idesc_s, 0u);
+        umma_ss(tmem + Cfg::COL_G, xa_desc, ud, idesc_s, 0u);
+        umma_ss(tmem + Cfg::COL_G, xb_desc, ud, idesc_s, 1u);
+        umma_commit(s_full);
+        if (!mbar_wait_mma(p_full, i & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < T / 16; ++ks) {
+          const uint32_t a = tmem + Cfg::COL_S + 16 * ks;
+          umma_ts(tmem + Cfg::COL_DQ, a, kd + ks * KSTEP, idesc_v, (i > 0 || ks > 0) ? 1u : 0u);  // dShi K
+          umma_ts(tmem + Cfg::COL_DQ, a + 8, kd + ks * KSTEP, idesc_v, 1u);                      // dSlo K
+          if (DEC)
+            umma_ts(tmem + Cfg::COL_DZ, tmem + Cfg::COL_G + 16 * ks, ud + ks * KSTEP, idesc_v,
+                    (i > 0 || ks > 0) ? 1u : 0u);                                                // W dY
+        }
+        umma_commit(pv_done);
       }
-      if (ok) issue_values(ntiles - 1);
       umma_commit(o_full);  // completes once every MMA issued above is done
       mbar_wait_drain(o_full, 0, p.timeout_ns);
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int wg = (warp - 1) >> 2;           // softmax warpgroup: tiles i with i % 2 == wg
     const int wq = warp & 3;                  // TMEM lane quarter of this warp
     const int r = wq * 32 + lane;             // latent row within the block
     const int m = lb * kLatBlock + r;
@@ -248,20 +242,27 @@ __global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
       grow = p.grow[static_cast<size_t>(bh) * p.M + m];
     }
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const uint32_t buf_base = lane_base + wg * Cfg::BUF;
     bool ok = true;
-    for (int i = wg; i < ntiles; i += 2) {
-      if (!mbar_wait_warp(s_full + wg, (i >> 1) & 1, wc)) { ok = false; break; }
+    for (int i = 0; i < ntiles; ++i) {
+      if (!mbar_wait_warp(s_full, i & 1, wc)) { ok = false; break; }
       tc_fence_after();
       const int valid = min(T, n_end - (n_begin + i * T));
       const float* sl = reinterpret_cast<const float*>(sld + (i % NST) * 2 * Cfg::LD_B);
       if (warp_live) {
+        uint32_t sv[2][16], gv[2][16];
+        tmem_ld16(lane_base + Cfg::COL_S, sv[0]);
+        tmem_ld16(lane_base + Cfg::COL_G, gv[0]);
+        tmem_wait_ld();
+        regs_defined(sv[0]);
+        regs_defined(gv[0]);
 #pragma unroll
         for (int j = 0; j < T / 16; ++j) {
-          uint32_t sv[16], gv[16], hi[8], lo[8], wp[8];
-          tmem_ld16(buf_base + Cfg::COL_S + 16 * j, sv);
-          tmem_ld16(buf_base + Cfg::COL_G + 16 * j, gv);
-          tmem_wait_ld();
+          uint32_t hi[8], lo[8], wp[8];
+          const int cb = j & 1, nb = cb ^ 1;
+          if (j + 1 < T / 16) {  // the next piece, while this one is computed
+            tmem_ld16(lane_base + Cfg::COL_S + 16 * (j + 1), sv[nb]);
+            tmem_ld16(lane_base + Cfg::COL_G + 16 * (j + 1), gv[nb]);
+          }
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const int c0 = 16 * j + 2 * k;
@@ -269,15 +270,15 @@ __global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
             if (DEC) {  // L_n, delta_n of the two token columns (shared-memory broadcast)
               const float2 ln = *reinterpret_cast<const float2*>(sl + c0);
               const float2 dl = *reinterpret_cast<const float2*>(sl + Cfg::LD_B / 4 + c0);
-              w0 = ex2_mufu(fmaf(__uint_as_float(sv[2 * k]), c, -ln.x));
-              w1 = ex2_mufu(fmaf(__uint_as_float(sv[2 * k + 1]), c, -ln.y));
-              d0 = w0 * (__uint_as_float(gv[2 * k]) - dl.x);
-              d1 = w1 * (__uint_as_float(gv[2 * k + 1]) - dl.y);
+              w0 = ex2_mufu(fmaf(__uint_as_float(sv[cb][2 * k]), c, -ln.x));
+              w1 = ex2_mufu(fmaf(__uint_as_float(sv[cb][2 * k + 1]), c, -ln.y));
+              d0 = w0 * (__uint_as_float(gv[cb][2 * k]) - dl.x);
+              d1 = w1 * (__uint_as_float(gv[cb][2 * k + 1]) - dl.y);
             } else {
-              w0 = ex2_mufu(fmaf(__uint_as_float(sv[2 * k]), c, -lrow));
-              w1 = ex2_mufu(fmaf(__uint_as_float(sv[2 * k + 1]), c, -lrow));
-              d0 = w0 * (__uint_as_float(gv[2 * k]) - grow);
-              d1 = w1 * (__uint_as_float(gv[2 * k + 1]) - grow);
+              w0 = ex2_mufu(fmaf(__uint_as_float(sv[cb][2 * k]), c, -lrow));
+              w1 = ex2_mufu(fmaf(__uint_as_float(sv[cb][2 * k + 1]), c, -lrow));
+              d0 = w0 * (__uint_as_float(gv[cb][2 * k]) - grow);
+              d1 = w1 * (__uint_as_float(gv[cb][2 * k + 1]) - grow);
             }
             if (c0 >= valid) { w0 = 0.f; d0 = 0.f; }
             if (c0 + 1 >= valid) { w1 = 0.f; d1 = 0.f; }
@@ -286,19 +287,24 @@ __global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
             if (DEC) wp[k] = pack_bf16x2(w0, w1);
           }
           // over the 16 columns just read: dS high and low parts (and W)
-          tmem_st8(buf_base + Cfg::COL_S + 16 * j, hi);
-          tmem_st8(buf_base + Cfg::COL_S + 16 * j + 8, lo);
-          if (DEC) tmem_st8(buf_base + Cfg::COL_G + 16 * j, wp);
+          tmem_st8(lane_base + Cfg::COL_S + 16 * j, hi);
+          tmem_st8(lane_base + Cfg::COL_S + 16 * j + 8, lo);
+          if (DEC) tmem_st8(lane_base + Cfg::COL_G + 16 * j, wp);
+          if (j + 1 < T / 16) {
+            tmem_wait_ld();
+            regs_defined(sv[nb]);
+            regs_defined(gv[nb]);
+          }
         }
         tmem_wait_st();
       }
       tc_fence_before();
-      mbar_arrive_warp(p_full + wg);
+      mbar_arrive_warp(p_full);
       __syncwarp();
     }
     if (ok && mbar_wait_warp(o_full, 0, wc)) {
       tc_fence_after();
-      if (wg == 0 && warp_live) {  // warpgroup 0 writes the partials
+      if (warp_live) {
         uint32_t dq[16], dz[16];
         tmem_ld16(lane_base + Cfg::COL_DQ, dq);
         if (DEC) tmem_ld16(lane_base + Cfg::COL_DZ, dz);

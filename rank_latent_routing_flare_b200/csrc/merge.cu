@@ -326,19 +326,18 @@ __global__ void wait_selftest_kernel(uint32_t* err, unsigned long long timeout_n
   }
 }
 
-__global__ void __launch_bounds__(256) split_lo_kernel(const SplitLoParams p) {
+__global__ void __launch_bounds__(256) to_f16_kernel(const ToF16Params p) {
   const long i = 2 * (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x);
   if (i >= p.n) return;
-  const uint32_t h = *reinterpret_cast<const uint32_t*>(p.hi + i);
-  const float2 f = *reinterpret_cast<const float2*>(p.full + i);
-  *reinterpret_cast<uint32_t*>(p.lo + i) = pack_bf16x2(f.x - bf16_lo(h), f.y - bf16_hi(h));
+  const float2 f = *reinterpret_cast<const float2*>(p.src + i);
+  *reinterpret_cast<uint32_t*>(p.dst + i) = pack_f16x2(f.x, f.y);
 }
 
 }  // namespace
 
-cudaError_t launch_split_lo(const SplitLoParams& p, cudaStream_t s) {
+cudaError_t launch_to_f16(const ToF16Params& p, cudaStream_t s) {
   const long pairs = p.n / 2;
-  split_lo_kernel<<<static_cast<unsigned>((pairs + 255) / 256), 256, 0, s>>>(p);
+  to_f16_kernel<<<static_cast<unsigned>((pairs + 255) / 256), 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -269,6 +269,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
+// The same with fp16 A/B (type fields 0).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return idesc_bf16_f32(M, N, a_mn_major, b_mn_major) & ~((7u << 7) | (7u << 10));
+}
 
 // ----------------------------------------------------------------------------
 // TMEM <-> registers, 32 lanes x 32 bit per warp (thread i <-> lane base+i)
@@ -348,6 +352,12 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 // arithmetic helpers
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi);
+// Pack two floats to fp16x2 (round to nearest even): lo -> bits [0,16), hi -> [16,32).
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
 
 // 2^x on the special-function unit (flushes subnormal results to zero).
 __device__ __forceinline__ float ex2_mufu(float x) {
@@ -445,7 +455,7 @@ __device__ __forceinline__ void exp2_chunk64(const uint32_t (&a)[32], const uint
 #ifndef FLARE_PACKED_F32X2
 #define FLARE_PACKED_F32X2 1
 #endif
-template <int NV, int NPOLY, int Q0 = 0>
+template <int NV, int NPOLY, int Q0 = 0, bool F16 = false>
 __device__ __forceinline__ void exp2_row(const uint32_t (&s)[NV], float c, float shift, uint32_t (&pk)[NV / 2]) {
 #if FLARE_PACKED_F32X2
   // the scale-and-shift of a pair of scores is one paired fma
@@ -473,7 +483,7 @@ __device__ __forceinline__ void exp2_row(const uint32_t (&s)[NV], float c, float
       e0 = ex2_mufu(x0);
       e1 = ex2_mufu(x1);
     }
-    pk[q] = pack_bf16x2(e0, e1);
+    pk[q] = F16 ? pack_f16x2(e0, e1) : pack_bf16x2(e0, e1);
   }
 }
 
