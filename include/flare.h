@@ -257,11 +257,11 @@ FLARE_API flare_status flarepp_mixer_bwd(const flare_bf16* X, const flare_bf16* 
  * workspace (flare_workspace_bytes(FLARE_VARIANT_FLAREPP_BWD or
  * FLARE_VARIANT_FLARE_BWD, ...)); the *_bwd_train calls read it instead of
  * recomputing the projections and the synthesis and encode passes.  At
- * D = 16 the training forward's decoder also adds the low bf16 part of Z
- * (Z - bf16(Z)) so that Y sees Z to fp32 accuracy, and keeps the fp32 Y and
- * the decoder's per-token log-normalisers (eq. 11; eq. 6), which the
- * backward then takes instead of recomputing them; at D = 32 the backward
- * recomputes those.
+ * D = 16 the training forward's decoder runs its value product on fp16
+ * operands (Z and the softmax weights in fp16 instead of bf16) so that Y sees
+ * Z to 2^-12, and keeps the fp32 Y and the decoder's per-token
+ * log-normalisers (eq. 11; eq. 6), which the backward then takes instead of
+ * recomputing them; at D = 32 the backward recomputes those.
  *
  *   flarepp_mixer_fwd_train   arguments as flarepp_mixer_fwd; writes Y
  *   flarepp_mixer_bwd_train   arguments as flarepp_mixer_bwd
@@ -285,9 +285,9 @@ FLARE_API flare_status flarepp_mixer_bwd(const flare_bf16* X, const flare_bf16* 
  * forward's fp32 Z and Q(X).  The gradients differ from flarepp_mixer_bwd's
  * by rounding, within the same tolerance against the exact gradients.  At
  * D = 32 Y is written by the forward exactly as flarepp_mixer_fwd
- * (flare_mixer_fwd) writes it; at D = 16 it is the bf16 rounding of a Y that
- * used Z unrounded, within the forward's tolerance and no further from the
- * exact Y.
+ * (flare_mixer_fwd) writes it; at D = 16 it is the bf16 rounding of a Y
+ * computed with fp16 Z and weights, within the forward's tolerance and no
+ * further from the exact Y.
  */
 FLARE_API flare_status flarepp_mixer_fwd_train(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
                                                const flare_bf16* Wk_syn, const flare_bf16* Wv_syn,

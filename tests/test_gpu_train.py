@@ -3,10 +3,10 @@ the FLARE ones) against the fp64 oracle and against the stand-alone calls.
 
 At D = 32 the training forward writes the same Y as flarepp_mixer_fwd (bit
 for bit: the same kernels, the normalisers also stored).  At D = 16 its
-decoder also adds the low bf16 part of Z (so that the fp32 Y it keeps for the
-backward sees Z to fp32 accuracy): Y is then held to the forward's own parity
-criteria against the oracle (``tests/parity.py``) and is at least as close to
-it as the plain forward's.  The backward reuses the forward's state instead
+decoder runs the value product on fp16 Z and weights (so that the fp32 Y it
+keeps for the backward sees Z to 2^-12): Y is then held to the forward's own
+parity criteria against the oracle (``tests/parity.py``) and is at least as
+close to it as the plain forward's.  The backward reuses the forward's state instead
 of recomputing it; its gradients are held to the backward's tolerance
 against the oracle: rel-L2 <= 5e-3 and max |error| <= 3e-2 * max |reference|
 per tensor.
@@ -54,7 +54,7 @@ PP_KEYS = ("dX", "dWk", "dWv", "dWk_syn", "dWv_syn", "dQ0")
 
 def check_train_y(w, Y, Y_plain, label):
     """The training forward's Y: bitwise the plain forward's at D = 32; at
-    D = 16 (the decoder adds the low part of Z) within the forward's parity
+    D = 16 (the decoder's value product in fp16) within the forward's parity
     criteria and no further from the oracle than the plain forward's Y."""
     if w.D != 16:
         assert torch.equal(Y.view(torch.int16), Y_plain.view(torch.int16)), label
