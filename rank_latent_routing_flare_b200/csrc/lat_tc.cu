@@ -242,6 +242,46 @@ __global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
       grow = p.grow[static_cast<size_t>(bh) * p.M + m];
     }
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    // One 16-column piece: scores s and products g (raw fp32 bits), for the
+    // decoder its tokens' L_n at ld[0..16) and delta_n at ld[LD_B/4 ..); dS =
+    // W (g - delta) with W = 2^(s c - L) out as bf16 high and low parts (and
+    // W in bf16).  Pairs of columns go through the paired fp32x2 forms.
+    const uint64_t c2 = f2_pack(c, c), m1 = f2_pack(-1.f, -1.f), zero2 = f2_pack(0.f, 0.f);
+    const uint64_t neg_l2 = f2_pack(-lrow, -lrow), neg_g2 = f2_pack(-grow, -grow);
+    auto piece = [&](const uint32_t (&sp)[16], const uint32_t (&gp)[16], const float* ld, uint32_t (&hi)[8],
+                     uint32_t (&lo)[8], uint32_t (&wp)[8]) {
+      float4 lq = make_float4(0.f, 0.f, 0.f, 0.f), dq = lq;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint64_t s2 = f2_pack(__uint_as_float(sp[2 * k]), __uint_as_float(sp[2 * k + 1]));
+        const uint64_t g2 = f2_pack(__uint_as_float(gp[2 * k]), __uint_as_float(gp[2 * k + 1]));
+        uint64_t t2, e2;
+        if (DEC) {  // L_n, delta_n of the pair's token columns (shared-memory broadcast, four at a time)
+          if ((k & 1) == 0) {
+            lq = *reinterpret_cast<const float4*>(ld + 2 * k);
+            dq = *reinterpret_cast<const float4*>(ld + Cfg::LD_B / 4 + 2 * k);
+          }
+          const uint64_t l2 = (k & 1) ? f2_pack(lq.z, lq.w) : f2_pack(lq.x, lq.y);
+          const uint64_t d2 = (k & 1) ? f2_pack(dq.z, dq.w) : f2_pack(dq.x, dq.y);
+          t2 = f2_fma(l2, m1, f2_fma(s2, c2, zero2));   // s c - L_n
+          e2 = f2_fma(d2, m1, g2);                       // g - delta_n
+        } else {
+          t2 = f2_fma(s2, c2, neg_l2);                   // s c - L_m
+          e2 = f2_add(g2, neg_g2);                       // g - gamma_m
+        }
+        float t0, t1;
+        f2_unpack(t2, t0, t1);
+        const float w0 = ex2_mufu(t0), w1 = ex2_mufu(t1);
+        const uint64_t d2 = f2_fma(f2_pack(w0, w1), e2, zero2);  // dS = W (g - .)
+        float d0, d1;
+        f2_unpack(d2, d0, d1);
+        hi[k] = pack_bf16x2(d0, d1);
+        float r0, r1;
+        f2_unpack(f2_fma(f2_pack(bf16_lo(hi[k]), bf16_hi(hi[k])), m1, d2), r0, r1);  // dS - hi
+        lo[k] = pack_bf16x2(r0, r1);
+        if (DEC) wp[k] = pack_bf16x2(w0, w1);
+      }
+    };
     bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
       if (!mbar_wait_warp(s_full, i & 1, wc)) { ok = false; break; }
@@ -249,6 +289,7 @@ __global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
       const int valid = min(T, n_end - (n_begin + i * T));
       const float* sl = reinterpret_cast<const float*>(sld + (i % NST) * 2 * Cfg::LD_B);
       if (warp_live) {
+        const bool full = valid >= T;  // every token column of the tile is valid
         uint32_t sv[2][16], gv[2][16];
         tmem_ld16(lane_base + Cfg::COL_S, sv[0]);
         tmem_ld16(lane_base + Cfg::COL_G, gv[0]);
@@ -263,28 +304,16 @@ __global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
             tmem_ld16(lane_base + Cfg::COL_S + 16 * (j + 1), sv[nb]);
             tmem_ld16(lane_base + Cfg::COL_G + 16 * (j + 1), gv[nb]);
           }
+          piece(sv[cb], gv[cb], sl + 16 * j, hi, lo, wp);
+          if (!full) {  // the tile's last valid token column is in this tile: zero the columns past it
+            const int nv = valid - 16 * j;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int c0 = 16 * j + 2 * k;
-            float w0, w1, d0, d1;
-            if (DEC) {  // L_n, delta_n of the two token columns (shared-memory broadcast)
-              const float2 ln = *reinterpret_cast<const float2*>(sl + c0);
-              const float2 dl = *reinterpret_cast<const float2*>(sl + Cfg::LD_B / 4 + c0);
-              w0 = ex2_mufu(fmaf(__uint_as_float(sv[cb][2 * k]), c, -ln.x));
-              w1 = ex2_mufu(fmaf(__uint_as_float(sv[cb][2 * k + 1]), c, -ln.y));
-              d0 = w0 * (__uint_as_float(gv[cb][2 * k]) - dl.x);
-              d1 = w1 * (__uint_as_float(gv[cb][2 * k + 1]) - dl.y);
-            } else {
-              w0 = ex2_mufu(fmaf(__uint_as_float(sv[cb][2 * k]), c, -lrow));
-              w1 = ex2_mufu(fmaf(__uint_as_float(sv[cb][2 * k + 1]), c, -lrow));
-              d0 = w0 * (__uint_as_float(gv[cb][2 * k]) - grow);
-              d1 = w1 * (__uint_as_float(gv[cb][2 * k + 1]) - grow);
+            for (int k = 0; k < 8; ++k) {
+              const uint32_t keep = 2 * k + 1 < nv ? 0xFFFFFFFFu : 2 * k < nv ? 0x0000FFFFu : 0u;
+              hi[k] &= keep;
+              lo[k] &= keep;
+              wp[k] &= keep;
             }
-            if (c0 >= valid) { w0 = 0.f; d0 = 0.f; }
-            if (c0 + 1 >= valid) { w1 = 0.f; d1 = 0.f; }
-            hi[k] = pack_bf16x2(d0, d1);
-            lo[k] = pack_bf16x2(d0 - bf16_lo(hi[k]), d1 - bf16_hi(hi[k]));
-            if (DEC) wp[k] = pack_bf16x2(w0, w1);
           }
           // over the 16 columns just read: dS high and low parts (and W)
           tmem_st8(lane_base + Cfg::COL_S + 16 * j, hi);
