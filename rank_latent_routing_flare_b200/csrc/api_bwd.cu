@@ -76,6 +76,9 @@ BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C) {
     // the high and low bf16 parts of dZ (then of dQ(X)) for the tcgen05 passes
     bp.off_xhi16 = take(static_cast<size_t>(BH * M * D) * 2);
     bp.off_xlo16 = take(static_cast<size_t>(BH * M * D) * 2);
+    // and of Z
+    bp.off_zhi16 = take(static_cast<size_t>(BH * M * D) * 2);
+    bp.off_zlo16 = take(static_cast<size_t>(BH * M * D) * 2);
     bp.off_y32 = pp ? bp.off_g32 : take(static_cast<size_t>(BH * N * D) * 4);
   }
   bp.total = off;
@@ -209,11 +212,44 @@ flare_status lat_tc(int mode, const BwdPlan& bp, uint8_t* ws, const void* q16, i
   return launch_lat_tc(mode, mp, p, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
 
-// x (fp32 [rows][D]) into the high and low bf16 parts kept for the tcgen05 passes.
-flare_status split_hilo(const BwdPlan& bp, uint8_t* ws, const float* x, long n, cudaStream_t s) {
-  const SplitHiLoParams sp{n, x, reinterpret_cast<uint16_t*>(ws + bp.off_xhi16),
-                           reinterpret_cast<uint16_t*>(ws + bp.off_xlo16)};
+// x (fp32 [rows][D]) into the high and low bf16 parts kept for the tcgen05
+// passes (dZ, then dQ(X): the x buffers; Z: the z buffers).
+flare_status split_hilo(const BwdPlan& bp, uint8_t* ws, const float* x, long n, cudaStream_t s, bool z = false) {
+  const SplitHiLoParams sp{n, x, reinterpret_cast<uint16_t*>(ws + (z ? bp.off_zhi16 : bp.off_xhi16)),
+                           reinterpret_cast<uint16_t*>(ws + (z ? bp.off_zlo16 : bp.off_xlo16))};
   return launch_split_hilo(sp, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+}
+
+// One tcgen05 token-parallel pass (see TokTcParams): dK, dV rows into g32
+// (token-major fp32 rows) or into bf16 dk16 / dv16.  Full: z parts from the
+// z buffers, L_n and delta_n; both modes: the dZ (or dQ(X)) parts from the x
+// buffers, L_m and gamma_m.
+flare_status tok_tc(int mode, const BwdPlan& bp, uint8_t* ws, const void* k16, const void* v16, const void* dy16,
+                    const void* q16, int q_per_batch, const float* ltok, const float* dtok, const float* lm,
+                    const float* gm, float* g32, int g_ld, int g_col_k, int g_col_v, uint16_t* dk16, uint16_t* dv16,
+                    int B, int H, int N, int M, int D, const int32_t* lengths, float sc, cudaStream_t s) {
+  const long BH = static_cast<long>(B) * H;
+  const long G = q_per_batch ? BH : H;
+  const CUtensorMapSwizzle sw = row_swizzle(D);
+  TokTcMaps mp;
+  const bool full = mode == kTokTcFull;
+  if (!map3d(&mp.k, k16, D, N, BH, D, kBwdTokBlock, sw) || !map3d(&mp.v, v16, D, N, BH, D, kBwdTokBlock, sw) ||
+      !map3d(&mp.y, full ? dy16 : k16, D, N, BH, D, kBwdTokBlock, sw) || !map3d(&mp.q, q16, D, M, G, D, 32, sw) ||
+      !map3d(&mp.zh, ws + bp.off_zhi16, D, M, BH, D, 32, sw) || !map3d(&mp.zl, ws + bp.off_zlo16, D, M, BH, D, 32, sw) ||
+      !map3d(&mp.dh, ws + bp.off_xhi16, D, M, BH, D, 32, sw) || !map3d(&mp.dl, ws + bp.off_xlo16, D, M, BH, D, 32, sw) ||
+      !map2d_f32(&mp.lm, lm, M, BH, 32, 1) || !map2d_f32(&mp.gm, gm, M, BH, 32, 1))
+    return FLARE_ERR_LAUNCH;
+  TokTcParams p{};
+  p.B = B; p.H = H; p.N = N; p.M = M; p.D = D;
+  p.q_per_batch = q_per_batch;
+  p.c = sc * kLog2e;
+  p.lengths = lengths;
+  p.ltok = ltok; p.dtok = dtok;
+  p.g32 = g32; p.g_ld = g_ld; p.g_col_k = g_col_k; p.g_col_v = g_col_v;
+  p.dk16 = dk16; p.dv16 = dv16;
+  p.err = reinterpret_cast<uint32_t*>(ws + bp.fwd.off_err);
+  p.timeout_ns = wait_timeout_ns();
+  return launch_tok_tc(mode, mp, p, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
 
 flare_status pad(const float* src, float* dst, long rows, int D, float mul, cudaStream_t s) {
@@ -327,14 +363,18 @@ flare_status fl_phase(int phase, const BwdPlan& bp, uint8_t* ws, const FlArgs& a
       tp.ltok = ltok; tp.dtok = dtok;
       tp.dk16 = reinterpret_cast<uint16_t*>(a.dK);
       tp.dv16 = reinterpret_cast<uint16_t*>(a.dV);
-      if (a.exact) tp.smul = c;
-      if (launch_tok(kTokFull, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-      // encoder backward: its dQ partials
-      if (use_lat_tc(a.exact, D)) {
-        if ((st = split_hilo(bp, ws, dz32, BH * M * D, s)) != FLARE_OK) return st;
+      if (use_lat_tc(a.exact, D)) {  // both passes on tcgen05, from the parts of dZ (and Z)
+        if ((st = split_hilo(bp, ws, dz32, BH * M * D, s)) != FLARE_OK ||
+            (st = tok_tc(kTokTcFull, bp, ws, k, v, dy, a.Q, 0, ltok, dtok, lenc, gam, nullptr, 0, 0, 0,
+                         reinterpret_cast<uint16_t*>(a.dK), reinterpret_cast<uint16_t*>(a.dV), B, H, N, M, D,
+                         a.lengths, sc, s)) != FLARE_OK)
+          return st;
         return lat_tc(kLatTcEncoder, bp, ws, a.Q, 0, ws + bp.off_xhi16, ws + bp.off_xlo16, k, v, nullptr, nullptr,
                       lenc, gam, exch, nullptr, B, H, N, M, D, a.lengths, sc, s);
       }
+      if (a.exact) tp.smul = c;
+      if (launch_tok(kTokFull, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+      // encoder backward: its dQ partials
       LatParams le = lat_params(bp, ws, q32, 0, k, B, H, N, M, D, a.lengths, sc, a.sh);
       le.zrow = dz32; le.lrow = lenc; le.grow = gam; le.v = v;
       if (a.exact) exact_scores(le, sc);
@@ -477,15 +517,17 @@ flare_status pp_phase(int phase, const BwdPlan& bp, uint8_t* ws, const PpArgs& a
       tp.k = kk; tp.v = vv; tp.dy = reinterpret_cast<const uint16_t*>(a.dY);
       tp.ltok = ltok; tp.dtok = dtok;
       tp.g32 = g32; tp.g_ld = 4 * C; tp.g_col_k = 0; tp.g_col_v = C;
-      if (a.exact) tp.smul = c;
-      if (launch_tok(kTokFull, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-      // encoder backward: its dQ(X) partials (the tcgen05 pass takes the
-      // forward's bf16 Q(X))
-      if (use_lat_tc(a.exact, D)) {
-        if ((st = split_hilo(bp, ws, dz32, BH * M * D, s)) != FLARE_OK) return st;
+      if (use_lat_tc(a.exact, D)) {  // both passes on tcgen05 (the forward's bf16 Q(X), the parts of dZ and Z)
+        if ((st = split_hilo(bp, ws, dz32, BH * M * D, s)) != FLARE_OK ||
+            (st = tok_tc(kTokTcFull, bp, ws, kk, vv, a.dY, ws + bp.fwd.off_qx16, 1, ltok, dtok, lenc, gam, g32,
+                         4 * C, 0, C, nullptr, nullptr, B, H, N, M, D, a.lengths, sc, s)) != FLARE_OK)
+          return st;
         return lat_tc(kLatTcEncoder, bp, ws, ws + bp.fwd.off_qx16, 1, ws + bp.off_xhi16, ws + bp.off_xlo16, kk, vv,
                       nullptr, nullptr, lenc, gam, exch, nullptr, B, H, N, M, D, a.lengths, sc, s);
       }
+      if (a.exact) tp.smul = c;
+      if (launch_tok(kTokFull, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+      // encoder backward: its dQ(X) partials
       LatParams le = lat_params(bp, ws, qx32, 1, kk, B, H, N, M, D, a.lengths, sc, a.sh);
       le.zrow = dz32; le.lrow = lenc; le.grow = gam; le.v = vv;
       if (a.exact) exact_scores(le, sc);
@@ -507,14 +549,17 @@ flare_status pp_phase(int phase, const BwdPlan& bp, uint8_t* ws, const PpArgs& a
       tp.qpad = q0pad; tp.dzpad = dqxpad; tp.lm = lsyn; tp.gam = gsyn;
       tp.k = kt; tp.v = vt;
       tp.g32 = g32; tp.g_ld = 4 * C; tp.g_col_k = 2 * C; tp.g_col_v = 3 * C;
-      if (a.exact) tp.smul = c;
-      if (launch_tok(kTokEncoder, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-      // ... and the partials of dQ0
-      if (use_lat_tc(a.exact, D)) {
-        if ((st = split_hilo(bp, ws, dqx32, BH * M * D, s)) != FLARE_OK) return st;
+      if (use_lat_tc(a.exact, D)) {  // both passes on tcgen05, from the parts of dQ(X)
+        if ((st = split_hilo(bp, ws, dqx32, BH * M * D, s)) != FLARE_OK ||
+            (st = tok_tc(kTokTcEncoder, bp, ws, kt, vt, nullptr, a.Q0, 0, nullptr, nullptr, lsyn, gsyn, g32, 4 * C,
+                         2 * C, 3 * C, nullptr, nullptr, B, H, N, M, D, a.lengths, sc, s)) != FLARE_OK)
+          return st;
         return lat_tc(kLatTcEncoder, bp, ws, a.Q0, 0, ws + bp.off_xhi16, ws + bp.off_xlo16, kt, vt, nullptr, nullptr,
                       lsyn, gsyn, exch, nullptr, B, H, N, M, D, a.lengths, sc, s);
       }
+      if (a.exact) tp.smul = c;
+      if (launch_tok(kTokEncoder, tp, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+      // ... and the partials of dQ0
       LatParams le = lat_params(bp, ws, q32, 0, kt, B, H, N, M, D, a.lengths, sc, a.sh);
       le.zrow = dqx32; le.lrow = lsyn; le.grow = gsyn; le.v = vt;
       if (a.exact) exact_scores(le, sc);
@@ -729,6 +774,7 @@ flare_status train_prologue(const BwdPlan& bp, uint8_t* ws, const flare_bf16* Q,
   }
   const long qrows = qx16 != nullptr ? BH * M : static_cast<long>(H) * M;
   if ((st = pad(qdec, reinterpret_cast<float*>(ws + bp.off_qpad), qrows, D, 1.f, s)) != FLARE_OK) return st;
+  if (use_lat_tc(true, D) && (st = split_hilo(bp, ws, z32, static_cast<long>(lat), s, true)) != FLARE_OK) return st;
   return pad(z32, reinterpret_cast<float*>(ws + bp.off_zpad), BH * M, D, 1.f, s);
 }
 
@@ -765,10 +811,7 @@ flare_status train_decoder(const BwdPlan& bp, uint8_t* ws, const float* q, const
   // delta_n rows go through fp32 tensor maps, whose row stride (4N bytes)
   // must be a multiple of 16
   if (use_lat_tc(true, D) && N % 4 == 0) {
-    flare_status st = split_hilo(bp, ws, reinterpret_cast<const float*>(ws + bp.off_z32),
-                                 static_cast<long>(B) * H * M * D, s);
-    if (st != FLARE_OK) return st;
-    return lat_tc(kLatTcDecoder, bp, ws, q16, q_per_batch, ws + bp.off_xhi16, ws + bp.off_xlo16, k, dY, ltok, dtok,
+    return lat_tc(kLatTcDecoder, bp, ws, q16, q_per_batch, ws + bp.off_zhi16, ws + bp.off_zlo16, k, dY, ltok, dtok,
                   nullptr, nullptr, exch + P, exch, B, H, N, M, D, lengths, sc, s);
   }
   LatParams ld = lat_params(bp, ws, q, q_per_batch, k, B, H, N, M, D, lengths, sc, sh);

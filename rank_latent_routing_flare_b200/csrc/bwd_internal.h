@@ -169,6 +169,35 @@ struct LatTcMaps {
 cudaError_t launch_lat_tc(int mode, const LatTcMaps& m, const LatTcParams& p, cudaStream_t s);
 size_t lat_tc_smem_bytes();
 int lat_tc_tile();
+// Token-parallel backward passes on tcgen05 (tok_tc.cu; D = 16, bf16
+// queries, exact scores): dK and dV rows of 128-token tiles, the decoder and
+// encoder parts (kTokTcFull) or the encoder part alone (kTokTcEncoder: the
+// query synthesis).
+constexpr int kTokTcFull = 0;
+constexpr int kTokTcEncoder = 1;
+struct TokTcParams {
+  int B, H, N, M, D;
+  int q_per_batch;              // queries [G][M][D] with G = B*H (1) or H (0)
+  float c;                      // scale * log2(e), applied to the fp32 product
+  const int32_t* lengths;
+  const float* ltok;            // full: L_n [B*H][N]
+  const float* dtok;            // full: delta_n [B*H][N]
+  float* g32;                   // token-major fp32 gradient rows [B][N][g_ld] or NULL
+  int g_ld, g_col_k, g_col_v;   // row stride and column offsets of dK and dV (head h adds h*D)
+  uint16_t *dk16, *dv16;        // or bf16 [B*H][N][D] outputs
+  uint32_t* err;
+  unsigned long long timeout_ns;
+};
+// Tensor maps: k, v, y (bf16 [B*H][N][D], 128-token boxes: K, V, dY); q (bf16
+// [G][M][D]); zh, zl (Z's bf16 parts), dh, dl (dZ's, or dQ(X)'s for the
+// synthesis) (bf16 [B*H][M][D]); lm, gm (fp32 [B*H][M]: L_m, gamma_m); all
+// latent boxes 32 rows.
+struct TokTcMaps {
+  CUtensorMap k, v, y, q, zh, zl, dh, dl, lm, gm;
+};
+cudaError_t launch_tok_tc(int mode, const TokTcMaps& m, const TokTcParams& p, cudaStream_t s);
+size_t tok_tc_smem_bytes();
+
 // hi[i] = bf16(x[i]), lo[i] = bf16(x[i] - hi[i]) for i < n (n even)
 struct SplitHiLoParams {
   long n;
