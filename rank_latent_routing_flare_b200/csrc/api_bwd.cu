@@ -233,11 +233,12 @@ flare_status tok_tc(int mode, const BwdPlan& bp, uint8_t* ws, const void* k16, c
   const CUtensorMapSwizzle sw = row_swizzle(D);
   TokTcMaps mp;
   const bool full = mode == kTokTcFull;
+  const uint32_t ch = static_cast<uint32_t>(tok_tc_chunk(mode));
   if (!map3d(&mp.k, k16, D, N, BH, D, kBwdTokBlock, sw) || !map3d(&mp.v, v16, D, N, BH, D, kBwdTokBlock, sw) ||
-      !map3d(&mp.y, full ? dy16 : k16, D, N, BH, D, kBwdTokBlock, sw) || !map3d(&mp.q, q16, D, M, G, D, 32, sw) ||
-      !map3d(&mp.zh, ws + bp.off_zhi16, D, M, BH, D, 32, sw) || !map3d(&mp.zl, ws + bp.off_zlo16, D, M, BH, D, 32, sw) ||
-      !map3d(&mp.dh, ws + bp.off_xhi16, D, M, BH, D, 32, sw) || !map3d(&mp.dl, ws + bp.off_xlo16, D, M, BH, D, 32, sw) ||
-      !map2d_f32(&mp.lm, lm, M, BH, 32, 1) || !map2d_f32(&mp.gm, gm, M, BH, 32, 1))
+      !map3d(&mp.y, full ? dy16 : k16, D, N, BH, D, kBwdTokBlock, sw) || !map3d(&mp.q, q16, D, M, G, D, ch, sw) ||
+      !map3d(&mp.zh, ws + bp.off_zhi16, D, M, BH, D, ch, sw) || !map3d(&mp.zl, ws + bp.off_zlo16, D, M, BH, D, ch, sw) ||
+      !map3d(&mp.dh, ws + bp.off_xhi16, D, M, BH, D, ch, sw) || !map3d(&mp.dl, ws + bp.off_xlo16, D, M, BH, D, ch, sw) ||
+      !map2d_f32(&mp.lm, lm, M, BH, ch, 1) || !map2d_f32(&mp.gm, gm, M, BH, ch, 1))
     return FLARE_ERR_LAUNCH;
   TokTcParams p{};
   p.B = B; p.H = H; p.N = N; p.M = M; p.D = D;

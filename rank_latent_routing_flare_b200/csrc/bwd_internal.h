@@ -191,12 +191,13 @@ struct TokTcParams {
 // Tensor maps: k, v, y (bf16 [B*H][N][D], 128-token boxes: K, V, dY); q (bf16
 // [G][M][D]); zh, zl (Z's bf16 parts), dh, dl (dZ's, or dQ(X)'s for the
 // synthesis) (bf16 [B*H][M][D]); lm, gm (fp32 [B*H][M]: L_m, gamma_m); all
-// latent boxes 32 rows.
+// latent boxes tok_tc_chunk(mode) rows.
 struct TokTcMaps {
   CUtensorMap k, v, y, q, zh, zl, dh, dl, lm, gm;
 };
 cudaError_t launch_tok_tc(int mode, const TokTcMaps& m, const TokTcParams& p, cudaStream_t s);
-size_t tok_tc_smem_bytes();
+size_t tok_tc_smem_bytes(int mode);
+int tok_tc_chunk(int mode);  // latents per chunk (the latent tensor maps' box rows)
 
 // hi[i] = bf16(x[i]), lo[i] = bf16(x[i] - hi[i]) for i < n (n even)
 struct SplitHiLoParams {

@@ -2,7 +2,9 @@
 // key and value rows for the training backward, whose queries are bf16
 // values (Q(X), Q0 or the learned Q) so that the score products are exact.
 // One CTA owns a tile of 128 tokens of one head (thread <-> TMEM lane <->
-// token) and walks the latents in chunks of C = 32:
+// token) and walks the latents in chunks of C = 32 (full) or 48 (encoder
+// only: half the work per score, so longer chunks amortise the per-chunk
+// hand-offs):
 //
 //   full (kTokTcFull: decoder and encoder, FLARE++ paper eq. 10-11; FLARE
 //   paper eq. 5-6), per chunk:
@@ -20,8 +22,8 @@
 //
 // The token tile's K, V and dY stay in shared memory; the latent chunks
 // (Q_c, the parts of Z_c and dZ_c, L_m and gamma_m) stream through a TMA
-// ring.  TMEM: S at column 0, dA at 32, dP at 64, dK at 96, dV at 112 (128
-// columns: four CTAs per SM).  The softmax threads read a chunk in 16-column
+// ring.  TMEM: S at column 0, dA at C, dP at 2C (full), dK at 96, dV at 112
+// (128 columns: four CTAs per SM).  The softmax threads read a chunk in 16-column
 // pieces and write, over the piece they have read, dS as bf16 high and low
 // parts (S columns [16j, 16j+8) and [16j+8, 16j+16)) and A in bf16 (dA
 // columns [16j, 16j+8)); each 16-latent k-step of the value MMAs takes its A
@@ -44,42 +46,46 @@ __device__ __forceinline__ void regs_defined16(uint32_t (&r)[16]) {
                  "+r"(r[15]));
 }
 
+template <int MODE>
 struct TokTcCfg {
+  static constexpr bool FULL = MODE == kTokTcFull;
   static constexpr int D = 16;
-  static constexpr int C = 32;                          // latents per chunk
+  static constexpr int C = FULL ? 32 : 48;              // latents per chunk
   static constexpr int TT = kBwdTokBlock;               // tokens per CTA (128)
   static constexpr int ROWB = D * 2;
   static constexpr int TOK_B = TT * ROWB;               // one token tile (K, V or dY)
   static constexpr int CH_B = C * ROWB;                 // one latent chunk of Q, Zhi, Zlo, dZhi or dZlo
-  static constexpr int ST_B = 5 * CH_B + 2 * 256;       // a ring stage: five chunks, L_m, gamma_m
+  static constexpr int NCH = FULL ? 5 : 3;              // chunks per ring stage
+  static constexpr int ST_B = NCH * CH_B + 2 * 256;     // a ring stage: the chunks, L_m, gamma_m
   static constexpr int NST = 6;
   static constexpr uint32_t LAYOUT = LAYOUT_SW32;
   static constexpr uint32_t SBO = 8 * ROWB;
   static constexpr int OFF_TK = 0, OFF_TV = TOK_B, OFF_TY = 2 * TOK_B;
-  static constexpr int OFF_RING = 3 * TOK_B;
+  static constexpr int OFF_RING = (FULL ? 3 : 2) * TOK_B;
   // within a stage
-  static constexpr int S_Q = 0, S_ZH = CH_B, S_ZL = 2 * CH_B, S_DH = 3 * CH_B, S_DL = 4 * CH_B;
-  static constexpr int S_LM = 5 * CH_B, S_GM = 5 * CH_B + 256;
+  static constexpr int S_Q = 0, S_DH = CH_B, S_DL = 2 * CH_B, S_ZH = 3 * CH_B, S_ZL = 4 * CH_B;
+  static constexpr int S_LM = NCH * CH_B, S_GM = NCH * CH_B + 256;
   static constexpr int OFF_BAR = OFF_RING + NST * ST_B;
   static constexpr int OFF_MISC = OFF_BAR + 8 * (6 + NST);
   static constexpr int BYTES = OFF_MISC + 64 + NST * 4;
-  static constexpr uint32_t COL_S = 0, COL_DA = C, COL_DP = 2 * C, COL_DK = 3 * C, COL_DV = 3 * C + D;
+  static constexpr uint32_t COL_S = 0, COL_DA = C, COL_DP = 2 * C, COL_DK = 96, COL_DV = 96 + D;
   static constexpr uint32_t TMEM_COLS = 128;
   static constexpr int THREADS = 160;
   static constexpr int CTAS_PER_SM = 4;
-  static_assert(COL_DV + D <= TMEM_COLS, "TMEM columns");
+  static_assert(COL_DV + D <= TMEM_COLS && (FULL ? 3 : 2) * C <= static_cast<int>(COL_DK), "TMEM columns");
   static_assert(TOK_B % 1024 == 0 && CH_B % 256 == 0 && ST_B % 256 == 0, "tiles must hold whole swizzle atoms");
+  static_assert(C * 4 <= 256, "L_m / gamma_m of a chunk");
 };
 
 template <int MODE>
-__global__ void __launch_bounds__(TokTcCfg::THREADS, TokTcCfg::CTAS_PER_SM)
+__global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_PER_SM)
     tok_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_zh, const __grid_constant__ CUtensorMap tm_zl,
                   const __grid_constant__ CUtensorMap tm_dh, const __grid_constant__ CUtensorMap tm_dl,
                   const __grid_constant__ CUtensorMap tm_lm, const __grid_constant__ CUtensorMap tm_gm,
                   const TokTcParams p) {
-  using Cfg = TokTcCfg;
+  using Cfg = TokTcCfg<MODE>;
   constexpr int D = Cfg::D, C = Cfg::C, NST = Cfg::NST;
   constexpr bool FULL = MODE == kTokTcFull;
   extern __shared__ uint8_t smem_raw[];
@@ -192,8 +198,6 @@ __global__ void __launch_bounds__(TokTcCfg::THREADS, TokTcCfg::CTAS_PER_SM)
       tma_load_3d(stv, &tm_v, tok_full, 0, n0, bh);
       if (FULL) tma_load_3d(sty, &tm_y, tok_full, 0, n0, bh);
       for (int j = 0; j < min(NST, nchunks); ++j) load_chunk(j);
-      const uint32_t idesc_full = idesc_bf16_f32(128, C, false, false);
-      const uint32_t idesc_half = idesc_bf16_f32(128, C / 2, false, false);
       const uint32_t idesc_v = idesc_bf16_f32(128, D, false, true);
       const uint64_t tk_desc = umma_desc(smem_u32(stk), 16, Cfg::SBO, Cfg::LAYOUT);
       const uint64_t tv_desc = umma_desc(smem_u32(stv), 16, Cfg::SBO, Cfg::LAYOUT);
@@ -208,7 +212,7 @@ __global__ void __launch_bounds__(TokTcCfg::THREADS, TokTcCfg::CTAS_PER_SM)
       bool ok = mbar_wait_mma(tok_full, 0, wc);
       for (int j = 0; ok && j < nchunks; ++j) {
         const int st = j % NST;
-        const int cn = min(C, p.M - j * C);  // 32, or 16 for a last half chunk
+        const int cn = min(C, p.M - j * C);  // C, or a multiple of 16 for the last chunk
         if (j > 0) {
           // the value MMAs of chunk j - 1 are done: S, dA, dP may be
           // overwritten, and its ring stage takes chunk j - 1 + NST
@@ -218,7 +222,7 @@ __global__ void __launch_bounds__(TokTcCfg::THREADS, TokTcCfg::CTAS_PER_SM)
         if (!mbar_wait_mma(lat_full + st, (j / NST) & 1, wc)) { ok = false; break; }
         tc_fence_after();
         const uint64_t rd = r_desc + st * STAGE;
-        const uint32_t idesc_s = cn == C ? idesc_full : idesc_half;
+        const uint32_t idesc_s = idesc_bf16_f32(128, cn, false, false);
         umma_ss(tmem + Cfg::COL_S, tk_desc, rd + OQ, idesc_s, 0u);    // K Q_c^T
         umma_ss(tmem + Cfg::COL_DA, tv_desc, rd + ODH, idesc_s, 0u);  // V dZhi_c^T
         umma_ss(tmem + Cfg::COL_DA, tv_desc, rd + ODL, idesc_s, 1u);  // + V dZlo_c^T
@@ -355,26 +359,29 @@ __global__ void __launch_bounds__(TokTcCfg::THREADS, TokTcCfg::CTAS_PER_SM)
 
 }  // namespace
 
-size_t tok_tc_smem_bytes() {
-  const size_t need = TokTcCfg::BYTES + 1024;
+size_t tok_tc_smem_bytes(int mode) {
+  const size_t need = (mode == kTokTcFull ? TokTcCfg<kTokTcFull>::BYTES : TokTcCfg<kTokTcEncoder>::BYTES) + 1024;
   // at most CTAS_PER_SM CTAs per SM (228 KB each, 1 KB of it reserved per
   // CTA), so that every resident CTA finds its TMEM columns free
-  const size_t floor = (228 * 1024) / (TokTcCfg::CTAS_PER_SM + 1) + 1024;
+  const size_t floor = (228 * 1024) / (TokTcCfg<kTokTcFull>::CTAS_PER_SM + 1) + 1024;
   return need > floor ? need : floor;
 }
 
+int tok_tc_chunk(int mode) { return mode == kTokTcFull ? TokTcCfg<kTokTcFull>::C : TokTcCfg<kTokTcEncoder>::C; }
+
 cudaError_t launch_tok_tc(int mode, const TokTcMaps& m, const TokTcParams& p, cudaStream_t s) {
   if (p.D != 16) return cudaErrorInvalidValue;
-  const size_t smem = tok_tc_smem_bytes();
-  const int tiles = (p.N + TokTcCfg::TT - 1) / TokTcCfg::TT;
+  const size_t smem = tok_tc_smem_bytes(mode);
+  const int tiles = (p.N + kBwdTokBlock - 1) / kBwdTokBlock;
   const dim3 grid(static_cast<unsigned>(static_cast<long>(p.B) * p.H * tiles));
-  auto go = [&](auto kern) {
+  auto go = [&](auto kern, int threads) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid, TokTcCfg::THREADS, smem, s>>>(m.k, m.v, m.y, m.q, m.zh, m.zl, m.dh, m.dl, m.lm, m.gm, p);
+    kern<<<grid, threads, smem, s>>>(m.k, m.v, m.y, m.q, m.zh, m.zl, m.dh, m.dl, m.lm, m.gm, p);
     return cudaGetLastError();
   };
-  return mode == kTokTcFull ? go(tok_tc_kernel<kTokTcFull>) : go(tok_tc_kernel<kTokTcEncoder>);
+  return mode == kTokTcFull ? go(tok_tc_kernel<kTokTcFull>, TokTcCfg<kTokTcFull>::THREADS)
+                            : go(tok_tc_kernel<kTokTcEncoder>, TokTcCfg<kTokTcEncoder>::THREADS);
 }
 
 }  // namespace flare
