@@ -313,14 +313,14 @@ def cpu_model():
 # ---------------------------------------------------------------------------
 
 BWD_METRIC = "mixer bwd token·heads/s at N=1M (1×B200) and % of roofline (HBM/MMA/MUFU)"
-BWD_LAUNCHES = 24        # kernels per FLARE++ backward call (projections, recompute, gradients, GEMMs)
-BWD_LAUNCHES_FLARE = 12  # kernels per FLARE backward call (recompute, gradients, merges, pads)
 # a training step, by (variant, D): the training forward (the forward's
 # kernels; at D = 16 plus the fp16 copy of Z) and the training backward (mark
 # check, conversions, pads, the decoder's delta or statistics, the latent- and
 # token-parallel passes with their sums and operand splits, the projection
 # gradients)
 TRAIN_LAUNCHES = {("flarepp", 16): 8 + 24, ("flarepp", 32): 7 + 21, ("flare", 16): 6 + 14, ("flare", 32): 5 + 12}
+# a self-contained backward call runs the same launches without the mark check
+BWD_LAUNCHES = {k: v - 1 for k, v in TRAIN_LAUNCHES.items()}
 TRAIN_METRIC = "mixer training step (fwd+bwd) token·heads/s at N=1M (1×B200) and % of roofline"
 TF32_PER_BF16 = 0.5  # nominal dense tf32 : bf16 tensor throughput
 
@@ -548,8 +548,7 @@ def run_backward(args, rank, world, local_rank):
             "cpu_baseline": cpu,
             "e2e": {"value": whole_job_rate(world, th_per_rank, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": (TRAIN_LAUNCHES[(w.variant, w.D)] if train else
-                             (BWD_LAUNCHES_FLARE if flare else BWD_LAUNCHES)) * args.steps,
+            "gpu_launches": (TRAIN_LAUNCHES if train else BWD_LAUNCHES)[(w.variant, w.D)] * args.steps,
             "compare": compare,
             "clocks": clocks.summary(),
         }

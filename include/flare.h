@@ -203,16 +203,20 @@ FLARE_API flare_status flarepp_mixer_fwd_inspect(const flare_bf16* X, const flar
  * compute the SDPA backward of each step (for O = softmax_rows(s Qa Ka^T) Va:
  * dVa = P^T dO, dS = P (dO Va^T - rowsum(P (dO Va^T))), dQa = s dS Ka,
  * dKa = s dS^T Qa), chained through the mixer.  Each call is
- * self-contained: it recomputes what the forward produced (the projections,
- * Q(X), Z and the softmax normalisers, all in fp32) from the inputs, so it
- * takes the forward's inputs and dY, not the forward's outputs.  Outputs are
+ * self-contained: it takes the forward's inputs and dY, not the forward's
+ * outputs, and first runs the training forward's kernels (below) into its
+ * workspace without storing Y, so that what the forward produced (the
+ * projections, Q(X), Z and the softmax normalisers) comes from the forward's
+ * own launches; then the training backward's launches.  The gradients equal
+ * those of the training pair on the same inputs bit for bit.  Outputs are
  * written (not accumulated).  Rows of dY for padding tokens are ignored;
  * padding tokens get zero gradients.  Same size limits as the forward, and
- * B*H <= 65535.  Arithmetic: the score and gradient products on the tensor
- * cores with tf32 operands (bf16 inputs are exact in tf32) and fp32
- * accumulation; softmax weights, normalisers and every reduction in fp32;
- * the FLARE++ projections recomputed in bf16 as in the forward.
- * Deterministic like the forward.
+ * B*H <= 65535.  Arithmetic: at D = 16 the score and gradient products of
+ * the four softmax passes on the tcgen05 tensor cores with each fp32 operand
+ * as the sum of two bf16 parts (high and low) and fp32 accumulation; at
+ * D = 32 and for the projection gradients, tensor-core products with tf32
+ * operands (bf16 inputs are exact in tf32); softmax weights, normalisers and
+ * every reduction in fp32.  Deterministic like the forward.
  *
  * flare_mixer_bwd (FLARE, eq. 5-6), workspace variant FLARE_VARIANT_FLARE_BWD:
  *   K, V, Q, lengths, scale   as in flare_mixer_fwd
@@ -279,11 +283,10 @@ FLARE_API flare_status flarepp_mixer_bwd(const flare_bf16* X, const flare_bf16* 
  * between the two calls are not detected.
  *
  * The backward's scores take the bf16 Q(X) that the forward's tensor-core
- * products took (flarepp_mixer_bwd recomputes Q(X) in fp32), unscaled, with
- * the scale applied to the fp32 product as in the forward, so that the
- * forward's normalisers fit them; Z and the synthesis' gamma use the
- * forward's fp32 Z and Q(X).  The gradients differ from flarepp_mixer_bwd's
- * by rounding, within the same tolerance against the exact gradients.  At
+ * products took, unscaled, with the scale applied to the fp32 product as in
+ * the forward, so that the forward's normalisers fit them; Z and the
+ * synthesis' gamma use the forward's fp32 Z and Q(X).  The gradients equal
+ * flarepp_mixer_bwd's (flare_mixer_bwd's) bit for bit.  At
  * D = 32 Y is written by the forward exactly as flarepp_mixer_fwd
  * (flare_mixer_fwd) writes it; at D = 16 it is the bf16 rounding of a Y
  * computed with fp16 Z and weights, within the forward's tolerance and no
@@ -329,8 +332,11 @@ FLARE_API flare_status flare_mixer_bwd_train(const flare_bf16* K, const flare_bf
  * NULL for the last phase).  Every rank merges the gathered buffers in the
  * same ascending (rank, split) order, so every rank ends with bitwise the
  * same dW_K, dW_V, dW~_K, dW~_V and dQ0 (written by the last two phases);
- * dX holds the shard's rows.  With world == 1 the result equals
- * flarepp_mixer_bwd bit for bit.  The phases of one rank share its workspace
+ * dX holds the shard's rows.  The phases recompute the forward's state
+ * themselves (the projections, then Q(X), Z and the normalisers with the
+ * backward's own tensor-core passes), so with world == 1 the result matches
+ * flarepp_mixer_bwd to rounding, not bit for bit; both are within the same
+ * tolerance of the exact gradients.  The phases of one rank share its workspace
  * (flare_workspace_bytes(FLARE_VARIANT_FLAREPP_BWD, ...) with the shard's N)
  * and carry the shard's state in it; the other arguments are as for
  * flarepp_mixer_bwd.  An out-of-range phase returns FLARE_ERR_SHAPE.
@@ -356,9 +362,9 @@ FLARE_API flare_status flarepp_cp_bwd_phase(int phase, const flare_bf16* X, cons
  * all-gathers them in rank order and passes the result as `gathered` to phase
  * p + 1.  Every rank merges in ascending (rank, split) order, so every rank
  * ends with bitwise the same dQ (written by the last phase); dK and dV hold
- * the shard's rows (written by phase 2).  With world == 1 the result equals
- * flare_mixer_bwd bit for bit (flare_mixer_bwd runs the same phases).  The
- * phases of one rank share its workspace (FLARE_VARIANT_FLARE_BWD with the
+ * the shard's rows (written by phase 2).  As for FLARE++, the phases
+ * recompute the encoder's state, so with world == 1 the result matches
+ * flare_mixer_bwd to rounding.  The phases of one rank share its workspace (FLARE_VARIANT_FLARE_BWD with the
  * shard's N).  An out-of-range phase returns FLARE_ERR_SHAPE.
  */
 #define FLARE_CP_BWD_PHASES_FLARE 4

@@ -383,7 +383,9 @@ flare_status flare_fwd(const flare_bf16* K, const flare_bf16* V, const flare_bf1
                        int N, int M, int D, const int32_t* lengths, float scale, void* workspace,
                        size_t workspace_bytes, void* stream, float* Z_out, float* Y_f32_out,
                        void* const* stage_events, const FwdStats* stats) {
-  if (!K || !V || !Q || !Y || !workspace) return FLARE_ERR_NULL;
+  // Y may be null only for a training forward run inside a backward call,
+  // which needs the kept state and not Y
+  if (!K || !V || !Q || (!Y && !stats) || !workspace) return FLARE_ERR_NULL;
   flare_status st = check_common(B, H, N, M, D);
   if (st != FLARE_OK) return st;
   if (!aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(Y) || !aligned16(lengths) || !aligned16(Z_out) ||

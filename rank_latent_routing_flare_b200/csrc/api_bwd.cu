@@ -637,28 +637,35 @@ flare_status check_pp_bwd(const PpArgs& a, const void* workspace) {
 
 using namespace flare;
 
+namespace {
+// The training pair's launch sequences (defined with the training entry
+// points below); the single-GPU backward runs them back to back.
+flare_status pp_train_forward(const BwdPlan& bp, uint8_t* ws, const PpArgs& a, flare_bf16* Y, cudaStream_t s);
+flare_status pp_train_backward(const BwdPlan& bp, uint8_t* ws, const PpArgs& a, bool check_state, cudaStream_t s);
+flare_status fl_train_forward(const BwdPlan& bp, uint8_t* ws, const FlArgs& a, flare_bf16* Y, size_t workspace_bytes,
+                              cudaStream_t s);
+flare_status fl_train_backward(const BwdPlan& bp, uint8_t* ws, const FlArgs& a, bool check_state, cudaStream_t s);
+
+}  // namespace
+
 extern "C" {
 
 flare_status flare_mixer_bwd(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, const flare_bf16* dY,
                              flare_bf16* dK, flare_bf16* dV, float* dQ, int B, int H, int N, int M, int D,
                              const int32_t* lengths, float scale, void* workspace, size_t workspace_bytes,
                              void* stream) {
-  const FlArgs a{K, V, Q, dY, dK, dV, dQ, B, H, N, M, D, lengths, resolve_scale(scale, D), Shard{0, N, 1}};
+  FlArgs a{K, V, Q, dY, dK, dV, dQ, B, H, N, M, D, lengths, resolve_scale(scale, D), Shard{0, N, 1}};
+  a.exact = true;
   flare_status st = check_fl_bwd(a, workspace);
   if (st != FLARE_OK) return st;
   const BwdPlan bp = make_bwd_plan(false, B, H, N, M, D, 0);
   if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  // one shard: the exchanges stay in the workspace (each phase reads the
-  // previous phase's buffer and writes another one)
-  float* ex[kFlPhases - 1] = {reinterpret_cast<float*>(ws + bp.off_fpart), reinterpret_cast<float*>(ws + bp.off_pa),
-                              reinterpret_cast<float*>(ws + bp.off_pc)};
-  for (int ph = 0; ph < kFlPhases; ++ph) {
-    st = fl_phase(ph, bp, ws, a, ph > 0 ? ex[ph - 1] : nullptr, ph < kFlPhases - 1 ? ex[ph] : nullptr, s);
-    if (st != FLARE_OK) return st;
-  }
-  return FLARE_OK;
+  // the statistics come from the forward kernels (a training forward that
+  // stores no Y), then the training backward's launches
+  if ((st = fl_train_forward(bp, ws, a, nullptr, workspace_bytes, s)) != FLARE_OK) return st;
+  return fl_train_backward(bp, ws, a, false, s);
 }
 
 size_t flare_cp_bwd_exchange_bytes(int phase, int B, int H, int N, int M, int D) {
@@ -693,26 +700,23 @@ flare_status flarepp_mixer_bwd(const flare_bf16* X, const flare_bf16* Wk, const 
                                float* dWv_syn, float* dQ0, int B, int N, int C, int H, int M, int D,
                                const int32_t* lengths, float scale, void* workspace, size_t workspace_bytes,
                                void* stream) {
-  const PpArgs a{X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, dX, dWk, dWv, dWk_syn, dWv_syn, dQ0,
-                 B, N, C, H, M, D, lengths, resolve_scale(scale, D), Shard{0, N, 1}};
+  PpArgs a{X, Wk, Wv, Wk_syn, Wv_syn, Q0, dY, dX, dWk, dWv, dWk_syn, dWv_syn, dQ0,
+           B, N, C, H, M, D, lengths, resolve_scale(scale, D), Shard{0, N, 1}};
+  a.exact = true;
   flare_status st = check_pp_bwd(a, workspace);
   if (st != FLARE_OK) return st;
   const BwdPlan bp = make_bwd_plan(true, B, H, N, M, D, C);
   if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  // one shard: the exchanges stay in the workspace (stream order makes every
-  // reuse safe: a buffer is read by the next phase's first launches before
-  // that phase writes its own exchange)
-  float* ex[kPpPhases - 1] = {reinterpret_cast<float*>(ws + bp.off_fpart), reinterpret_cast<float*>(ws + bp.off_fpart),
-                              reinterpret_cast<float*>(ws + bp.off_pa),    reinterpret_cast<float*>(ws + bp.off_pc),
-                              reinterpret_cast<float*>(ws + bp.off_pc),    reinterpret_cast<float*>(ws + bp.off_dwpart)};
-  for (int ph = 0; ph < kPpPhases; ++ph) {
-    st = pp_phase(ph, bp, ws, a, ph > 0 ? ex[ph - 1] : nullptr, ph < kPpPhases - 1 ? ex[ph] : nullptr, s);
-    if (st != FLARE_OK) return st;
-  }
-  return FLARE_OK;
+  // the projections, Q(X), Z and the statistics come from the forward
+  // kernels (a training forward that stores no Y), then the training
+  // backward's launches
+  if ((st = pp_train_forward(bp, ws, a, nullptr, s)) != FLARE_OK) return st;
+  return pp_train_backward(bp, ws, a, false, s);
 }
+
+}  // extern "C"
 
 // ---------------------------------------------------------------------------
 // Training pair: a forward that keeps, in the backward's workspace, what the
@@ -752,14 +756,18 @@ flare_status widen(const uint16_t* src, float* dst, long n, cudaStream_t s) {
 }
 
 // Start of a training backward: clear the error word (not the mark), check
-// the mark on the device, take Q0 (or Q) and Q(X) as fp32 images of their
-// bf16 values and the forward's fp32 Z, and pad them unscaled.
+// the mark on the device (check_state; not when the state comes from this
+// call's own forward, whose error word is kept), take Q0 (or Q) and Q(X) as
+// fp32 images of their bf16 values and the forward's fp32 Z, and pad them
+// unscaled.
 flare_status train_prologue(const BwdPlan& bp, uint8_t* ws, const flare_bf16* Q, const uint16_t* qx16, long BH, int H,
-                            int M, int D, cudaStream_t s) {
-  if (cudaMemsetAsync(ws + bp.fwd.off_err, 0, kErrWordBytes, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-  const MarkParams mk{reinterpret_cast<const uint32_t*>(ws + bp.fwd.off_err + kTrainMarkOffset),
-                      reinterpret_cast<uint32_t*>(ws + bp.fwd.off_err)};
-  if (launch_check_mark(mk, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+                            int M, int D, bool check_state, cudaStream_t s) {
+  if (check_state) {
+    if (cudaMemsetAsync(ws + bp.fwd.off_err, 0, kErrWordBytes, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+    const MarkParams mk{reinterpret_cast<const uint32_t*>(ws + bp.fwd.off_err + kTrainMarkOffset),
+                        reinterpret_cast<uint32_t*>(ws + bp.fwd.off_err)};
+    if (launch_check_mark(mk, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+  }
   float* q32 = reinterpret_cast<float*>(ws + bp.off_q32);
   float* z32 = reinterpret_cast<float*>(ws + bp.off_z32);
   const size_t lat = static_cast<size_t>(BH) * M * D;
@@ -825,7 +833,58 @@ flare_status train_decoder(const BwdPlan& bp, uint8_t* ws, const float* q, const
   return launch_lat(kLatDecoder, ld, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
 
+// The training forward's launches (FLARE++): the mixer forward that also
+// keeps the backward's state; Y may be null (not stored).
+flare_status pp_train_forward(const BwdPlan& bp, uint8_t* ws, const PpArgs& a, flare_bf16* Y, cudaStream_t s) {
+  FwdStats fs = train_stats(bp, ws, a.D);
+  fs.lsyn = reinterpret_cast<float*>(ws + bp.off_lsyn);
+  return flarepp_run(bp.fwd, a.X, a.Wk, a.Wv, a.Wk_syn, a.Wv_syn, a.Q0, Y, 0, a.B, a.N, a.C, a.H, a.M, a.D,
+                     a.lengths, a.sc, ws, s, nullptr, nullptr, nullptr, nullptr, &fs);
+}
+
+// The training backward's launches after the argument checks (FLARE++).
+flare_status pp_train_backward(const BwdPlan& bp, uint8_t* ws, const PpArgs& a, bool check_state, cudaStream_t s) {
+  const long BH = static_cast<long>(a.B) * a.H;
+  float* pa = reinterpret_cast<float*>(ws + bp.off_pa);
+  float* pc = reinterpret_cast<float*>(ws + bp.off_pc);
+  flare_status st;
+  if ((st = train_prologue(bp, ws, a.Q0, reinterpret_cast<const uint16_t*>(ws + bp.fwd.off_qx16), BH, a.H, a.M, a.D,
+                           check_state, s)) != FLARE_OK ||
+      (st = train_decoder(bp, ws, reinterpret_cast<const float*>(ws + bp.off_qx32), ws + bp.fwd.off_qx16, 1,
+                          ws + bp.fwd.off_kp, a.dY, a.B, a.H, a.N, a.M, a.D, a.lengths, a.sc, pa, s)) != FLARE_OK)
+    return st;
+  // phases 3-6 of the seven (the exchanges stay in the workspace)
+  float* ex[kPpPhases - 1] = {nullptr, nullptr, pa, pc, pc, reinterpret_cast<float*>(ws + bp.off_dwpart)};
+  for (int ph = 3; ph < kPpPhases; ++ph)
+    if ((st = pp_phase(ph, bp, ws, a, ex[ph - 1], ph < kPpPhases - 1 ? ex[ph] : nullptr, s)) != FLARE_OK) return st;
+  return FLARE_OK;
+}
+
+// The training forward's launches (FLARE); Y may be null (not stored).
+flare_status fl_train_forward(const BwdPlan& bp, uint8_t* ws, const FlArgs& a, flare_bf16* Y, size_t workspace_bytes,
+                              cudaStream_t s) {
+  FwdStats fs = train_stats(bp, ws, a.D);
+  return flare_fwd(a.K, a.V, a.Q, Y, a.B, a.H, a.N, a.M, a.D, a.lengths, a.sc, ws, workspace_bytes, s, nullptr,
+                   nullptr, nullptr, &fs);
+}
+
+// The training backward's launches after the argument checks (FLARE).
+flare_status fl_train_backward(const BwdPlan& bp, uint8_t* ws, const FlArgs& a, bool check_state, cudaStream_t s) {
+  float* pa = reinterpret_cast<float*>(ws + bp.off_pa);
+  float* pc = reinterpret_cast<float*>(ws + bp.off_pc);
+  flare_status st;
+  if ((st = train_prologue(bp, ws, a.Q, nullptr, static_cast<long>(a.B) * a.H, a.H, a.M, a.D, check_state, s)) !=
+          FLARE_OK ||
+      (st = train_decoder(bp, ws, reinterpret_cast<const float*>(ws + bp.off_q32), a.Q, 0, a.K, a.dY, a.B, a.H, a.N,
+                          a.M, a.D, a.lengths, a.sc, pa, s)) != FLARE_OK ||
+      (st = fl_phase(2, bp, ws, a, pa, pc, s)) != FLARE_OK || (st = fl_phase(3, bp, ws, a, pc, nullptr, s)) != FLARE_OK)
+    return st;
+  return FLARE_OK;
+}
+
 }  // namespace
+
+extern "C" {
 
 flare_status flarepp_mixer_fwd_train(const flare_bf16* X, const flare_bf16* Wk, const flare_bf16* Wv,
                                      const flare_bf16* Wk_syn, const flare_bf16* Wv_syn, const flare_bf16* Q0,
@@ -839,11 +898,9 @@ flare_status flarepp_mixer_fwd_train(const flare_bf16* X, const flare_bf16* Wk, 
   if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  FwdStats fs = train_stats(bp, ws, D);
-  fs.lsyn = reinterpret_cast<float*>(ws + bp.off_lsyn);
-  st = flarepp_run(bp.fwd, X, Wk, Wv, Wk_syn, Wv_syn, Q0, Y, 0, B, N, C, H, M, D, lengths, resolve_scale(scale, D), ws,
-                   s, nullptr, nullptr, nullptr, nullptr, &fs);
-  if (st != FLARE_OK) return st;
+  const PpArgs a{X, Wk, Wv, Wk_syn, Wv_syn, Q0, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                 B, N, C, H, M, D, lengths, resolve_scale(scale, D), Shard{0, N, 1}};
+  if ((st = pp_train_forward(bp, ws, a, Y, s)) != FLARE_OK) return st;
   return set_train_mark(ws, bp, kTrainStateByte, s);
 }
 
@@ -862,18 +919,7 @@ flare_status flarepp_mixer_bwd_train(const flare_bf16* X, const flare_bf16* Wk, 
   if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const long BH = static_cast<long>(B) * H;
-  float* pa = reinterpret_cast<float*>(ws + bp.off_pa);
-  float* pc = reinterpret_cast<float*>(ws + bp.off_pc);
-  if ((st = train_prologue(bp, ws, Q0, reinterpret_cast<const uint16_t*>(ws + bp.fwd.off_qx16), BH, H, M, D, s)) !=
-          FLARE_OK ||
-      (st = train_decoder(bp, ws, reinterpret_cast<const float*>(ws + bp.off_qx32), ws + bp.fwd.off_qx16, 1,
-                          ws + bp.fwd.off_kp, dY, B, H, N, M, D, lengths, a.sc, pa, s)) != FLARE_OK)
-    return st;
-  // phases 3-6 of the seven (the exchanges stay in the workspace)
-  float* ex[kPpPhases - 1] = {nullptr, nullptr, pa, pc, pc, reinterpret_cast<float*>(ws + bp.off_dwpart)};
-  for (int ph = 3; ph < kPpPhases; ++ph)
-    if ((st = pp_phase(ph, bp, ws, a, ex[ph - 1], ph < kPpPhases - 1 ? ex[ph] : nullptr, s)) != FLARE_OK) return st;
+  if ((st = pp_train_backward(bp, ws, a, true, s)) != FLARE_OK) return st;
   return set_train_mark(ws, bp, 0, s);  // the state is used: a second backward needs a new forward
 }
 
@@ -886,11 +932,11 @@ flare_status flare_mixer_fwd_train(const flare_bf16* K, const flare_bf16* V, con
   const BwdPlan bp = make_bwd_plan(false, B, H, N, M, D, 0);
   if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  FwdStats fs = train_stats(bp, ws, D);
-  st = flare_fwd(K, V, Q, Y, B, H, N, M, D, lengths, scale, workspace, workspace_bytes, stream, nullptr, nullptr,
-                 nullptr, &fs);
-  if (st != FLARE_OK) return st;
-  return set_train_mark(ws, bp, kTrainStateByte, static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const FlArgs a{K, V, Q, nullptr, nullptr, nullptr, nullptr, B, H, N, M, D, lengths, resolve_scale(scale, D),
+                 Shard{0, N, 1}};
+  if ((st = fl_train_forward(bp, ws, a, Y, workspace_bytes, s)) != FLARE_OK) return st;
+  return set_train_mark(ws, bp, kTrainStateByte, s);
 }
 
 flare_status flare_mixer_bwd_train(const flare_bf16* K, const flare_bf16* V, const flare_bf16* Q, const flare_bf16* dY,
@@ -905,13 +951,7 @@ flare_status flare_mixer_bwd_train(const flare_bf16* K, const flare_bf16* V, con
   if (workspace_bytes < bp.total) return FLARE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* pa = reinterpret_cast<float*>(ws + bp.off_pa);
-  float* pc = reinterpret_cast<float*>(ws + bp.off_pc);
-  if ((st = train_prologue(bp, ws, Q, nullptr, static_cast<long>(B) * H, H, M, D, s)) != FLARE_OK ||
-      (st = train_decoder(bp, ws, reinterpret_cast<const float*>(ws + bp.off_q32), Q, 0, K, dY, B, H, N, M, D,
-                          lengths, a.sc, pa, s)) != FLARE_OK ||
-      (st = fl_phase(2, bp, ws, a, pa, pc, s)) != FLARE_OK || (st = fl_phase(3, bp, ws, a, pc, nullptr, s)) != FLARE_OK)
-    return st;
+  if ((st = fl_train_backward(bp, ws, a, true, s)) != FLARE_OK) return st;
   return set_train_mark(ws, bp, 0, s);
 }
 

@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(128) decode_fallback_kernel(const DecodeParams
       for (int u = 0; u < D / 4; ++u)
         d32[u] = make_float4(y[4 * u] * inv, y[4 * u + 1] * inv, y[4 * u + 2] * inv, y[4 * u + 3] * inv);
     }
+    if (p.y == nullptr) continue;
     uint4* dst = reinterpret_cast<uint4*>(y_row<D>(p, bh, n));
 #pragma unroll
     for (int u = 0; u < D / 8; ++u)
@@ -211,9 +212,10 @@ __global__ void __launch_bounds__(DecCfg<D, F16>::THREADS, DecCfg<D, F16>::CTAS_
     const int z0 = max(ta, tiles_valid) * kDecTile;
     const int z1 = min(tb * kDecTile, p.N);
     const uint4 zero = make_uint4(0, 0, 0, 0);
-    for (size_t e = static_cast<size_t>(z0) * (D / 8) + threadIdx.x; e < static_cast<size_t>(z1) * (D / 8);
-         e += blockDim.x)
-      reinterpret_cast<uint4*>(y_row<D>(p, bh, static_cast<int>(e / (D / 8))))[e % (D / 8)] = zero;
+    if (p.y != nullptr)
+      for (size_t e = static_cast<size_t>(z0) * (D / 8) + threadIdx.x; e < static_cast<size_t>(z1) * (D / 8);
+           e += blockDim.x)
+        reinterpret_cast<uint4*>(y_row<D>(p, bh, static_cast<int>(e / (D / 8))))[e % (D / 8)] = zero;
     if (p.y_f32 != nullptr) {
       uint4* d32 = reinterpret_cast<uint4*>(p.y_f32 + static_cast<size_t>(bh) * p.N * D);
       for (size_t e = static_cast<size_t>(z0) * (D / 4) + threadIdx.x; e < static_cast<size_t>(z1) * (D / 4);
@@ -420,11 +422,13 @@ __global__ void __launch_bounds__(DecCfg<D, F16>::THREADS, DecCfg<D, F16>::CTAS_
 #pragma unroll
           for (int u = 0; u < D / 4; ++u) d32[u] = make_float4(y[4 * u], y[4 * u + 1], y[4 * u + 2], y[4 * u + 3]);
         }
-        uint4* dst = reinterpret_cast<uint4*>(y_row<D>(p, bh, n));
+        if (p.y != nullptr) {
+          uint4* dst = reinterpret_cast<uint4*>(y_row<D>(p, bh, n));
 #pragma unroll
-        for (int u = 0; u < D / 8; ++u)
-          dst[u] = make_uint4(pack_bf16x2(y[8 * u + 0], y[8 * u + 1]), pack_bf16x2(y[8 * u + 2], y[8 * u + 3]),
-                              pack_bf16x2(y[8 * u + 4], y[8 * u + 5]), pack_bf16x2(y[8 * u + 6], y[8 * u + 7]));
+          for (int u = 0; u < D / 8; ++u)
+            dst[u] = make_uint4(pack_bf16x2(y[8 * u + 0], y[8 * u + 1]), pack_bf16x2(y[8 * u + 2], y[8 * u + 3]),
+                                pack_bf16x2(y[8 * u + 4], y[8 * u + 5]), pack_bf16x2(y[8 * u + 6], y[8 * u + 7]));
+        }
       }
       return true;
     };

@@ -186,7 +186,7 @@ struct DecodeParams {
   const uint16_t* q;    // bf16 [G][M][D]
   const uint16_t* z;    // bf16 [B*H][M][D]
   const uint16_t* k;    // bf16 [B*H][N][D]
-  uint16_t* y;          // bf16 [B*H][N][D], or [B][N][H*D] when y_token_major
+  uint16_t* y;          // bf16 [B*H][N][D], or [B][N][H*D] when y_token_major; null: not stored
   int y_token_major;
   float* y_f32;         // optional fp32 copy of Y ([B*H][N][D], the values Y is rounded from), or nullptr
   // the training forward's variant (D = 16): z holds fp16 bits of Z and the

@@ -183,8 +183,9 @@ def test_backward_reports_bad_lengths():
 
 
 def test_backward_cuda_graph_replays_the_same_bits():
-    """The backward call only enqueues kernels and a memset on its stream, so
-    it can be captured into a CUDA graph; a replay gives the eager bits."""
+    """The backward call only enqueues kernels, memsets and a device-to-device
+    copy on its stream, so it can be captured into a CUDA graph; a replay
+    gives the eager bits."""
     w = make_workload("flarepp_n8k_mesh2d", N=1024, B=2)
     dY = dev_bf16(make_upstream_grad(w))
     X, Q0 = dev_bf16(w.X), dev_bf16(w.Q0)

@@ -5,8 +5,9 @@ and its backward).
 One GPU plays R ranks: each rank runs the seven phases of
 flarepp_cp_bwd_phase through the C ABI on its own token shard and workspace,
 and the all-gather between two phases is a concatenation in rank order.
-Checked: with one rank the phases reproduce flarepp_mixer_bwd bit for bit;
-with several ranks every rank holds bitwise the same weight and seed
+Checked: with one rank the phases match the fp64 oracle and flarepp_mixer_bwd
+(which takes the forward's state from the forward kernels, so the two agree
+to rounding, not bit for bit); with several ranks every rank holds bitwise the same weight and seed
 gradients, and the gradients (dX from the shards' rows) match the fp64
 oracle on the whole sequences, including a rank whose shard has no valid
 token of a sample.
@@ -72,18 +73,17 @@ def emulate(w, dY, R):
     return outs
 
 
-def test_one_rank_reproduces_the_single_gpu_backward():
+def test_one_rank_matches_the_single_gpu_backward():
     w = make_workload("flarepp_n1k", N=900)
     dY = make_upstream_grad(w)
     outs = emulate(w, dY, 1)[0]
     g = fl.flarepp_mixer_bwd(dev_bf16(w.X), dev_bf16(w.Wk), dev_bf16(w.Wv), dev_bf16(w.Wk_syn),
                              dev_bf16(w.Wv_syn), dev_bf16(w.Q0), dev_bf16(dY))
     torch.cuda.synchronize()
+    ref = oracle.backward_workload(w, dY)
     for k in KEYS:
-        a, b = outs[k], g[k]
-        if a.dtype == torch.bfloat16:
-            a, b = a.view(torch.int16), b.view(torch.int16)
-        assert torch.equal(a, b), k
+        check(host_f64(outs[k]), ref[k], f"one rank {k} vs oracle")
+        check(host_f64(outs[k]), host_f64(g[k]), f"one rank {k} vs flarepp_mixer_bwd")
 
 
 @pytest.mark.parametrize("name,N,B,R,lengths", [
@@ -161,16 +161,19 @@ def emulate_flare(w, dY, R):
     return outs
 
 
-def test_flare_one_rank_reproduces_the_single_gpu_backward():
+def test_flare_one_rank_matches_the_single_gpu_backward():
     w = flare_case(2, 2, 1000, 64, 16, seed=5, lengths=[1000, 613])
     dY = make_upstream_grad(w)
     outs = emulate_flare(w, dY, 1)[0]
     lengths = torch.from_numpy(w.lengths).cuda()
     dK, dV, dQ = fl.flare_mixer_bwd(dev_bf16(w.K), dev_bf16(w.V), dev_bf16(w.Q), dev_bf16(dY), lengths=lengths)
     torch.cuda.synchronize()
-    assert torch.equal(outs["dK"].view(torch.int16), dK.view(torch.int16))
-    assert torch.equal(outs["dV"].view(torch.int16), dV.view(torch.int16))
-    assert torch.equal(outs["dQ"], dQ)
+    ref = oracle.backward_workload(w, dY)
+    for k, single in (("dK", dK), ("dV", dV), ("dQ", dQ)):
+        check(host_f64(outs[k]), ref[k], f"flare one rank {k} vs oracle")
+        check(host_f64(outs[k]), host_f64(single), f"flare one rank {k} vs flare_mixer_bwd")
+    for b, L in enumerate(w.lengths):
+        assert torch.all(outs["dK"][b, :, L:] == 0) and torch.all(dK[b, :, L:] == 0)
 
 
 @pytest.mark.parametrize("B,H,N,M,D,R,lengths", [
