@@ -65,6 +65,8 @@ BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C) {
   // part of dQ, summed over the batch [H][M][D]
   bp.off_dqxdec = take(lat);
   if (pp) {
+    // the gradient rows [B*N][4C] = [dK | dV | dK~ | dV~] as two bf16 planes
+    // (high and low parts), read by the projection gradients
     bp.off_g32 = take(static_cast<size_t>(B * N) * 4 * C * 4);
     bp.off_dwpart = take(static_cast<size_t>(bp.dw_splits) * C * 4 * C * 4);
   }
@@ -220,13 +222,13 @@ flare_status split_hilo(const BwdPlan& bp, uint8_t* ws, const float* x, long n, 
   return launch_split_hilo(sp, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
 }
 
-// One tcgen05 token-parallel pass (see TokTcParams): dK, dV rows into g32
-// (token-major fp32 rows) or into bf16 dk16 / dv16.  Full: z parts from the
+// One tcgen05 token-parallel pass (see TokTcParams): dK, dV rows into ghi /
+// glo (token-major rows as bf16 high and low parts) or into bf16 dk16 / dv16.  Full: z parts from the
 // z buffers, L_n and delta_n; both modes: the dZ (or dQ(X)) parts from the x
 // buffers, L_m and gamma_m.
 flare_status tok_tc(int mode, const BwdPlan& bp, uint8_t* ws, const void* k16, const void* v16, const void* dy16,
                     const void* q16, int q_per_batch, const float* ltok, const float* dtok, const float* lm,
-                    const float* gm, float* g32, int g_ld, int g_col_k, int g_col_v, uint16_t* dk16, uint16_t* dv16,
+                    const float* gm, uint16_t* ghi, uint16_t* glo, int g_ld, int g_col_k, int g_col_v, uint16_t* dk16, uint16_t* dv16,
                     int B, int H, int N, int M, int D, const int32_t* lengths, float sc, cudaStream_t s) {
   const long BH = static_cast<long>(B) * H;
   const long G = q_per_batch ? BH : H;
@@ -246,7 +248,7 @@ flare_status tok_tc(int mode, const BwdPlan& bp, uint8_t* ws, const void* k16, c
   p.c = sc * kLog2e;
   p.lengths = lengths;
   p.ltok = ltok; p.dtok = dtok;
-  p.g32 = g32; p.g_ld = g_ld; p.g_col_k = g_col_k; p.g_col_v = g_col_v;
+  p.ghi = ghi; p.glo = glo; p.g_ld = g_ld; p.g_col_k = g_col_k; p.g_col_v = g_col_v;
   p.dk16 = dk16; p.dv16 = dv16;
   p.err = reinterpret_cast<uint32_t*>(ws + bp.fwd.off_err);
   p.timeout_ns = wait_timeout_ns();
@@ -366,7 +368,7 @@ flare_status fl_phase(int phase, const BwdPlan& bp, uint8_t* ws, const FlArgs& a
       tp.dv16 = reinterpret_cast<uint16_t*>(a.dV);
       if (use_lat_tc(a.exact, D)) {  // both passes on tcgen05, from the parts of dZ (and Z)
         if ((st = split_hilo(bp, ws, dz32, BH * M * D, s)) != FLARE_OK ||
-            (st = tok_tc(kTokTcFull, bp, ws, k, v, dy, a.Q, 0, ltok, dtok, lenc, gam, nullptr, 0, 0, 0,
+            (st = tok_tc(kTokTcFull, bp, ws, k, v, dy, a.Q, 0, ltok, dtok, lenc, gam, nullptr, nullptr, 0, 0, 0,
                          reinterpret_cast<uint16_t*>(a.dK), reinterpret_cast<uint16_t*>(a.dV), B, H, N, M, D,
                          a.lengths, sc, s)) != FLARE_OK)
           return st;
@@ -459,7 +461,9 @@ flare_status pp_phase(int phase, const BwdPlan& bp, uint8_t* ws, const PpArgs& a
   float* dzpad = reinterpret_cast<float*>(ws + bp.off_dzpad);
   float* q0pad = reinterpret_cast<float*>(ws + bp.off_q0pad);
   float* dqxpad = reinterpret_cast<float*>(ws + bp.off_dqxpad);
-  float* g32 = reinterpret_cast<float*>(ws + bp.off_g32);
+  // the gradient rows [B*N][4C] as bf16 high and low planes
+  uint16_t* ghi = reinterpret_cast<uint16_t*>(ws + bp.off_g32);
+  uint16_t* glo = ghi + static_cast<size_t>(B) * N * 4 * C;
   const size_t P = part_floats(bp, B, H, M, D, false);
   const size_t stride = pp_exchange_floats(bp, phase - 1, B, H, M, D, C);  // of the gathered buffers
   flare_status st = FLARE_OK;
@@ -517,10 +521,10 @@ flare_status pp_phase(int phase, const BwdPlan& bp, uint8_t* ws, const PpArgs& a
       tp.qpad = qpad; tp.zpad = zpad; tp.dzpad = dzpad; tp.lm = lenc; tp.gam = gam;
       tp.k = kk; tp.v = vv; tp.dy = reinterpret_cast<const uint16_t*>(a.dY);
       tp.ltok = ltok; tp.dtok = dtok;
-      tp.g32 = g32; tp.g_ld = 4 * C; tp.g_col_k = 0; tp.g_col_v = C;
+      tp.ghi = ghi; tp.glo = glo; tp.g_ld = 4 * C; tp.g_col_k = 0; tp.g_col_v = C;
       if (use_lat_tc(a.exact, D)) {  // both passes on tcgen05 (the forward's bf16 Q(X), the parts of dZ and Z)
         if ((st = split_hilo(bp, ws, dz32, BH * M * D, s)) != FLARE_OK ||
-            (st = tok_tc(kTokTcFull, bp, ws, kk, vv, a.dY, ws + bp.fwd.off_qx16, 1, ltok, dtok, lenc, gam, g32,
+            (st = tok_tc(kTokTcFull, bp, ws, kk, vv, a.dY, ws + bp.fwd.off_qx16, 1, ltok, dtok, lenc, gam, ghi, glo,
                          4 * C, 0, C, nullptr, nullptr, B, H, N, M, D, a.lengths, sc, s)) != FLARE_OK)
           return st;
         return lat_tc(kLatTcEncoder, bp, ws, ws + bp.fwd.off_qx16, 1, ws + bp.off_xhi16, ws + bp.off_xlo16, kk, vv,
@@ -549,10 +553,10 @@ flare_status pp_phase(int phase, const BwdPlan& bp, uint8_t* ws, const PpArgs& a
       TokParams tp = tok_params(B, H, N, M, D, 0, a.lengths, sc, a.sh);
       tp.qpad = q0pad; tp.dzpad = dqxpad; tp.lm = lsyn; tp.gam = gsyn;
       tp.k = kt; tp.v = vt;
-      tp.g32 = g32; tp.g_ld = 4 * C; tp.g_col_k = 2 * C; tp.g_col_v = 3 * C;
+      tp.ghi = ghi; tp.glo = glo; tp.g_ld = 4 * C; tp.g_col_k = 2 * C; tp.g_col_v = 3 * C;
       if (use_lat_tc(a.exact, D)) {  // both passes on tcgen05, from the parts of dQ(X)
         if ((st = split_hilo(bp, ws, dqx32, BH * M * D, s)) != FLARE_OK ||
-            (st = tok_tc(kTokTcEncoder, bp, ws, kt, vt, nullptr, a.Q0, 0, nullptr, nullptr, lsyn, gsyn, g32, 4 * C,
+            (st = tok_tc(kTokTcEncoder, bp, ws, kt, vt, nullptr, a.Q0, 0, nullptr, nullptr, lsyn, gsyn, ghi, glo, 4 * C,
                          2 * C, 3 * C, nullptr, nullptr, B, H, N, M, D, a.lengths, sc, s)) != FLARE_OK)
           return st;
         return lat_tc(kLatTcEncoder, bp, ws, a.Q0, 0, ws + bp.off_xhi16, ws + bp.off_xlo16, kt, vt, nullptr, nullptr,
@@ -572,18 +576,30 @@ flare_status pp_phase(int phase, const BwdPlan& bp, uint8_t* ws, const PpArgs& a
       if ((st = lat_sum(B, H, M, D, bp.S, 1, sc, gathered, nullptr, R, stride, nullptr, nullptr, nullptr, a.dQ0, s)) !=
           FLARE_OK)
         return st;
-      // projections backward on this shard's rows: dX = G [Wk | Wv | Wk~ | Wv~]^T, partials of X^T G
+      // projections backward on this shard's rows (tcgen05): dX = G [Wk | Wv | Wk~ | Wv~]^T and the
+      // split partials of (X^T G)^T
       const long rows = static_cast<long>(B) * N;
-      DxParams dx{};
-      dx.R = static_cast<int>(rows); dx.C = C; dx.nw = 4;
-      dx.g = g32;
+      const CUtensorMapSwizzle sw128 = CU_TENSOR_MAP_SWIZZLE_128B;
       const flare_bf16* w4[4] = {a.Wk, a.Wv, a.Wk_syn, a.Wv_syn};
-      for (int i = 0; i < 4; ++i) dx.w[i] = reinterpret_cast<const uint16_t*>(w4[i]);
+      DxTcMaps xm;
+      DwTcMaps wm;
+      if (!map2d(&xm.ghi, ghi, 4 * C, rows, 64, 128, sw128) || !map2d(&xm.glo, glo, 4 * C, rows, 64, 128, sw128) ||
+          !map2d(&wm.ghi, ghi, 4 * C, rows, 64, 32, sw128) || !map2d(&wm.glo, glo, 4 * C, rows, 64, 32, sw128) ||
+          !map2d(&wm.x, a.X, C, rows, 64, 32, sw128))
+        return FLARE_ERR_LAUNCH;
+      for (int i = 0; i < 4; ++i)
+        if (!map2d(&xm.w[i], w4[i], C, C, 64, C, sw128)) return FLARE_ERR_LAUNCH;
+      uint32_t* err = reinterpret_cast<uint32_t*>(ws + bp.fwd.off_err);
+      DxTcParams dx{};
+      dx.R = static_cast<int>(rows); dx.C = C;
       dx.dx = reinterpret_cast<uint16_t*>(a.dX);
-      if (launch_dx(dx, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
-      const DwParams dw{static_cast<int>(rows), C, 4 * C, bp.dw_splits, reinterpret_cast<const uint16_t*>(a.X), g32,
-                        exch};
-      return launch_dw(dw, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+      dx.err = err; dx.timeout_ns = wait_timeout_ns();
+      if (launch_dx_tc(xm, dx, s) != cudaSuccess) return FLARE_ERR_LAUNCH;
+      DwTcParams dw{};
+      dw.R = static_cast<int>(rows); dw.C = C; dw.n_splits = bp.dw_splits; dw.rows_per_split = kBwdDwRows;
+      dw.part = exch;
+      dw.err = err; dw.timeout_ns = wait_timeout_ns();
+      return launch_dw_tc(wm, dw, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
     }
     case 6: {
       // dW: the partials of every shard's rows (rank-major, so the splits of all
@@ -592,7 +608,7 @@ flare_status pp_phase(int phase, const BwdPlan& bp, uint8_t* ws, const PpArgs& a
       dr.C = C; dr.J = 4 * C; dr.n_splits = R * bp.dw_splits; dr.shared = shared ? 1 : 0;
       dr.part = gathered;
       dr.dw[0] = a.dWk; dr.dw[1] = a.dWv; dr.dw[2] = a.dWk_syn; dr.dw[3] = a.dWv_syn;
-      return launch_dw_reduce(dr, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
+      return launch_dw_tc_reduce(dr, s) == cudaSuccess ? FLARE_OK : FLARE_ERR_LAUNCH;
     }
     default:
       return FLARE_ERR_SHAPE;

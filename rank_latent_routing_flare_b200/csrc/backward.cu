@@ -25,7 +25,6 @@
 //   tok_kernel<., kTokFull, .>       dK (decoder + encoder) and dV
 //   lat_kernel<., kLatEncoder, .>    the encoder's dQ (per split)
 //   tok_kernel<., kTokEncoder, .>    dK, dV of the query synthesis
-//   dx_kernel / dw_kernel / dw_reduce_kernel   projection gradients
 // Every reduction has a fixed order: the results are bitwise reproducible.
 // No kernel waits on another CTA or on a flag: there are no spin loops.
 #include "bwd_internal.h"
@@ -744,156 +743,19 @@ __global__ void __launch_bounds__(256) tok_kernel(const TokParams p) {
         const float2 kk = v ? make_float2(oa[mt][nd][2 * i] * kdk, oa[mt][nd][2 * i + 1] * kdk)
                             : make_float2(0.f, 0.f);
         const float2 vv = v ? make_float2(ob[mt][nd][2 * i], ob[mt][nd][2 * i + 1]) : make_float2(0.f, 0.f);
-        if (p.g32 != nullptr) {
-          float* o = p.g32 + (static_cast<size_t>(b) * p.N + rr[mt][i]) * p.g_ld + h * D + c;
-          *reinterpret_cast<float2*>(o + p.g_col_k) = kk;
-          *reinterpret_cast<float2*>(o + p.g_col_v) = vv;
+        if (p.ghi != nullptr) {
+          const size_t o = (static_cast<size_t>(b) * p.N + rr[mt][i]) * p.g_ld + h * D + c;
+          const uint32_t kh = pack_bf16x2(kk.x, kk.y), vh = pack_bf16x2(vv.x, vv.y);
+          *reinterpret_cast<uint32_t*>(p.ghi + o + p.g_col_k) = kh;
+          *reinterpret_cast<uint32_t*>(p.glo + o + p.g_col_k) = pack_bf16x2(kk.x - bf16_lo(kh), kk.y - bf16_hi(kh));
+          *reinterpret_cast<uint32_t*>(p.ghi + o + p.g_col_v) = vh;
+          *reinterpret_cast<uint32_t*>(p.glo + o + p.g_col_v) = pack_bf16x2(vv.x - bf16_lo(vh), vv.y - bf16_hi(vh));
         } else {
           *reinterpret_cast<uint32_t*>(p.dk16 + tk[mt][i] * D + c) = pack_bf16x2(kk.x, kk.y);
           *reinterpret_cast<uint32_t*>(p.dv16 + tk[mt][i] * D + c) = pack_bf16x2(vv.x, vv.y);
         }
       }
     }
-}
-
-// ---------------------------------------------------------------------------
-// Projection gradients (eq. 7 and 9 run backwards) on the tensor cores: a CTA
-// of 8 warps computes a 128 x 128 output tile, a warp 16 rows of it, over
-// k-steps of 32 staged in shared memory (fp32, tf32-rounded; bf16 values are
-// exact in tf32).
-// ---------------------------------------------------------------------------
-constexpr int kGT = 128;       // output tile rows and columns
-constexpr int kGK = 32;        // k-step
-constexpr int kGLD = kGK + 4;  // padded row of a [row][k] tile (conflict-free fragments)
-constexpr int kGLT = kGT + 8;  // padded row of a [k][col] tile
-
-// dX[r][c] = sum_j G[r][j] Wcat[c][j], Wcat = [W_0 | W_1 | ...] (each [C][C]).
-// A = G rows ([row][k] tile), B[k][n] = W_q[c][j] ([c][k] tile).
-__global__ void __launch_bounds__(256) dx_kernel(const DxParams p) {
-  __shared__ __align__(16) float sG[kGT * kGLD];
-  __shared__ __align__(16) float sW[kGT * kGLD];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const long r0 = static_cast<long>(blockIdx.x) * kGT;
-  const int c0 = blockIdx.y * kGT;
-  const int J = p.nw * p.C;
-  float acc[kGT / 8][4];
-#pragma unroll
-  for (int nt = 0; nt < kGT / 8; ++nt)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-  for (int j0 = 0; j0 < J; j0 += kGK) {
-    const int q = j0 / p.C, jj0 = j0 - q * p.C;
-    __syncthreads();
-    for (int i = threadIdx.x; i < kGT * kGK / 4; i += blockDim.x) {
-      const int row = i / (kGK / 4), c4 = (i - row * (kGK / 4)) * 4;
-      const long gr = r0 + row;
-      float4 v = gr < p.R ? *reinterpret_cast<const float4*>(p.g + gr * J + j0 + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
-      v = make_float4(__uint_as_float(tf32(v.x)), __uint_as_float(tf32(v.y)), __uint_as_float(tf32(v.z)),
-                      __uint_as_float(tf32(v.w)));
-      *reinterpret_cast<float4*>(&sG[row * kGLD + c4]) = v;
-    }
-    for (int i = threadIdx.x; i < kGT * kGK / 8; i += blockDim.x) {
-      const int c = i / (kGK / 8), k8 = (i - c * (kGK / 8)) * 8;
-      uint4 w = make_uint4(0u, 0u, 0u, 0u);
-      if (c0 + c < p.C) w = *reinterpret_cast<const uint4*>(p.w[q] + static_cast<size_t>(c0 + c) * p.C + jj0 + k8);
-      float4* d = reinterpret_cast<float4*>(&sW[c * kGLD + k8]);
-      d[0] = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
-      d[1] = make_float4(bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w));
-    }
-    __syncthreads();
-#pragma unroll
-    for (int ks = 0; ks < kGK / 8; ++ks) {
-      const float* ar = sG + (warp * 16 + g) * kGLD + ks * 8 + t;
-      const uint32_t a[4] = {fbits(ar), fbits(ar + 8 * kGLD), fbits(ar + 4), fbits(ar + 8 * kGLD + 4)};
-#pragma unroll
-      for (int nt = 0; nt < kGT / 8; ++nt) {
-        const float* br = sW + (nt * 8 + g) * kGLD + ks * 8 + t;
-        mma8(acc[nt], a, fbits(br), fbits(br + 4));
-      }
-    }
-  }
-  const long ra = r0 + warp * 16 + g, rb = ra + 8;
-#pragma unroll
-  for (int nt = 0; nt < kGT / 8; ++nt) {
-    const int c = c0 + nt * 8 + 2 * t;
-    if (c >= p.C) continue;
-    if (ra < p.R) *reinterpret_cast<uint32_t*>(p.dx + ra * p.C + c) = pack_bf16x2(acc[nt][0], acc[nt][1]);
-    if (rb < p.R) *reinterpret_cast<uint32_t*>(p.dx + rb * p.C + c) = pack_bf16x2(acc[nt][2], acc[nt][3]);
-  }
-}
-
-// part[split][c][j] = sum over the split's rows r of X[r][c] G[r][j].
-// A[c][k = r] = X[r][c] and B[k = r][j] = G[r][j], both from [k][col] tiles.
-__global__ void __launch_bounds__(256) dw_kernel(const DwParams p) {
-  __shared__ __align__(16) float sX[kGK * kGLT];
-  __shared__ __align__(16) float sG[kGK * kGLT];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int c0 = blockIdx.x * kGT, j0 = blockIdx.y * kGT, split = blockIdx.z;
-  const long rs = static_cast<long>(split) * kBwdDwRows;
-  const long re = min(rs + kBwdDwRows, static_cast<long>(p.R));
-  float acc[kGT / 8][4];
-#pragma unroll
-  for (int nt = 0; nt < kGT / 8; ++nt)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-  for (long r = rs; r < re; r += kGK) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < kGK * kGT / 8; i += blockDim.x) {
-      const int k = i / (kGT / 8), c8 = (i - k * (kGT / 8)) * 8;
-      uint4 w = make_uint4(0u, 0u, 0u, 0u);
-      if (r + k < re && c0 + c8 < p.C) w = *reinterpret_cast<const uint4*>(p.x + (r + k) * p.C + c0 + c8);
-      float4* d = reinterpret_cast<float4*>(&sX[k * kGLT + c8]);
-      d[0] = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
-      d[1] = make_float4(bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w));
-    }
-    for (int i = threadIdx.x; i < kGK * kGT / 4; i += blockDim.x) {
-      const int k = i / (kGT / 4), j4 = (i - k * (kGT / 4)) * 4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r + k < re && j0 + j4 < p.J) v = *reinterpret_cast<const float4*>(p.g + (r + k) * p.J + j0 + j4);
-      v = make_float4(__uint_as_float(tf32(v.x)), __uint_as_float(tf32(v.y)), __uint_as_float(tf32(v.z)),
-                      __uint_as_float(tf32(v.w)));
-      *reinterpret_cast<float4*>(&sG[k * kGLT + j4]) = v;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int ks = 0; ks < kGK / 8; ++ks) {
-      const float* ar = sX + (ks * 8 + t) * kGLT + warp * 16 + g;
-      const uint32_t a[4] = {fbits(ar), fbits(ar + 8), fbits(ar + 4 * kGLT), fbits(ar + 4 * kGLT + 8)};
-#pragma unroll
-      for (int nt = 0; nt < kGT / 8; ++nt) {
-        const float* br = sG + (ks * 8 + t) * kGLT + nt * 8 + g;
-        mma8(acc[nt], a, fbits(br), fbits(br + 4 * kGLT));
-      }
-    }
-  }
-  const int ca = c0 + warp * 16 + g, cb = ca + 8;
-#pragma unroll
-  for (int nt = 0; nt < kGT / 8; ++nt) {
-    const int j = j0 + nt * 8 + 2 * t;
-    if (j >= p.J) continue;
-    if (ca < p.C)
-      *reinterpret_cast<float2*>(p.part + (static_cast<size_t>(split) * p.C + ca) * p.J + j) =
-          make_float2(acc[nt][0], acc[nt][1]);
-    if (cb < p.C)
-      *reinterpret_cast<float2*>(p.part + (static_cast<size_t>(split) * p.C + cb) * p.J + j) =
-          make_float2(acc[nt][2], acc[nt][3]);
-  }
-}
-
-__global__ void __launch_bounds__(256) dw_reduce_kernel(const DwReduceParams p) {
-  const int ncols = p.shared ? 2 * p.C : p.J;
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= p.C * ncols) return;
-  const int c = idx / ncols, j = idx % ncols;
-  float s = 0.f;
-  for (int sp = 0; sp < p.n_splits; ++sp) {
-    const float* row = p.part + (static_cast<size_t>(sp) * p.C + c) * p.J;
-    s += row[j];
-    if (p.shared) s += row[j + 2 * p.C];
-  }
-  const int q = j / p.C, jj = j % p.C;
-  if (p.dw[q]) p.dw[q][static_cast<size_t>(c) * p.C + jj] = s;
-  if (p.shared && p.dw[q + 2]) p.dw[q + 2][static_cast<size_t>(c) * p.C + jj] = s;
 }
 
 // dst[r][0..LD) = (tf32(mul * src[r][c]) for c < D, then zeros): the padded
@@ -1005,24 +867,6 @@ cudaError_t launch_tok(int mode, const TokParams& p, cudaStream_t s) {
     else FLARE_TOK(32, kTokEncoder, 1);
   }
 #undef FLARE_TOK
-  return cudaGetLastError();
-}
-
-cudaError_t launch_dx(const DxParams& p, cudaStream_t s) {
-  const dim3 grid(blocks_for(p.R, kGT), blocks_for(p.C, kGT));
-  dx_kernel<<<grid, 256, 0, s>>>(p);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_dw(const DwParams& p, cudaStream_t s) {
-  const dim3 grid(blocks_for(p.C, kGT), blocks_for(p.J, kGT), p.n_splits);
-  dw_kernel<<<grid, 256, 0, s>>>(p);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_dw_reduce(const DwReduceParams& p, cudaStream_t s) {
-  const long n = static_cast<long>(p.C) * (p.shared ? 2 * p.C : p.J);
-  dw_reduce_kernel<<<blocks_for(n, 256), 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 

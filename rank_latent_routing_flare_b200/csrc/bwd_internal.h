@@ -94,29 +94,40 @@ struct TokParams {
   const uint16_t *k, *v, *dy;   // bf16 [B*H][N][D]
   float* ltok;                  // [B*H][N]: written (stats), read (full)
   float* dtok;                  // [B*H][N]: written (stats), read (full)
-  float* g32;                   // token-major fp32 gradient rows [B][N][g_ld] or NULL
+  uint16_t *ghi, *glo;          // token-major gradient rows [B][N][g_ld] as bf16 high and low parts, or NULL
   int g_ld, g_col_k, g_col_v;   // row stride and column offsets of dK and dV (head h adds h*D)
   uint16_t* dk16;               // or bf16 [B*H][N][D] outputs
   uint16_t* dv16;
 };
 
-// dX[r][c] = sum_q sum_j G[r][q*C + j] W_q[c][j]   (r < R = B*N, q < nw)
-struct DxParams {
-  int R, C, nw;
-  const float* g;               // [R][nw*C]
-  const uint16_t* w[4];         // bf16 [C][C]
+// Projection gradients on tcgen05 (proj_grad.cu).  G: the token-major
+// gradient rows [R][4C] = [dK | dV | dK~ | dV~] (R = B*N) as two bf16
+// planes, high and low parts; Wcat = [W_K | W_V | W~_K | W~_V], each [C][C].
+// dX[r][c] = sum_j G[r][j] Wcat[c][j].
+struct DxTcParams {
+  int R, C;
   uint16_t* dx;                 // bf16 [R][C]
+  uint32_t* err;
+  unsigned long long timeout_ns;
+};
+// ghi, glo: [R][4C] bf16, 64 x 128 boxes, SW128; w[q]: W_q [C][C] bf16, 64 x C boxes, SW128.
+struct DxTcMaps {
+  CUtensorMap ghi, glo, w[4];
+};
+// Partials of the transposed weight gradient over splits of rows_per_split
+// token rows: part[s][j][c] = sum_{r in split s} G[r][j] X[r][c].
+struct DwTcParams {
+  int R, C, n_splits, rows_per_split;
+  float* part;                  // [n_splits][4C][C]
+  uint32_t* err;
+  unsigned long long timeout_ns;
+};
+// ghi, glo: [R][4C] bf16 and x: X [R][C] bf16, all 64 x 32 boxes, SW128.
+struct DwTcMaps {
+  CUtensorMap ghi, glo, x;
 };
 
-// Partial weight gradients dWcat[c][j] = sum_{r in split} X[r][c] G[r][j].
-struct DwParams {
-  int R, C, J, n_splits;
-  const uint16_t* x;            // bf16 [R][C]
-  const float* g;               // [R][J]
-  float* part;                  // [n_splits][C][J]
-};
-
-// dW_q[c][j] = sum_splits part[.][c][q*C + j] (+ part[.][c][(q+2)*C + j]
+// dW_q[c][j] = sum_splits part[.][q*C + j][c] (+ part[.][(q+2)*C + j][c]
 // when the synthesis weights are the encode weights).
 struct DwReduceParams {
   int C, J, n_splits, shared;
@@ -182,7 +193,7 @@ struct TokTcParams {
   const int32_t* lengths;
   const float* ltok;            // full: L_n [B*H][N]
   const float* dtok;            // full: delta_n [B*H][N]
-  float* g32;                   // token-major fp32 gradient rows [B][N][g_ld] or NULL
+  uint16_t *ghi, *glo;          // token-major gradient rows [B][N][g_ld] as bf16 high and low parts, or NULL
   int g_ld, g_col_k, g_col_v;   // row stride and column offsets of dK and dV (head h adds h*D)
   uint16_t *dk16, *dv16;        // or bf16 [B*H][N][D] outputs
   uint32_t* err;
@@ -233,9 +244,9 @@ cudaError_t launch_check_mark(const MarkParams& p, cudaStream_t s);
 cudaError_t launch_lat_merge(const LatMergeParams& p, cudaStream_t s);
 cudaError_t launch_lat_sum(const LatSumParams& p, cudaStream_t s);
 cudaError_t launch_tok(int mode, const TokParams& p, cudaStream_t s);
-cudaError_t launch_dx(const DxParams& p, cudaStream_t s);
-cudaError_t launch_dw(const DwParams& p, cudaStream_t s);
-cudaError_t launch_dw_reduce(const DwReduceParams& p, cudaStream_t s);
+cudaError_t launch_dx_tc(const DxTcMaps& m, const DxTcParams& p, cudaStream_t s);
+cudaError_t launch_dw_tc(const DwTcMaps& m, const DwTcParams& p, cudaStream_t s);
+cudaError_t launch_dw_tc_reduce(const DwReduceParams& p, cudaStream_t s);
 cudaError_t launch_pad(const PadParams& p, cudaStream_t s);
 cudaError_t launch_cvt(const CvtParams& p, cudaStream_t s);
 

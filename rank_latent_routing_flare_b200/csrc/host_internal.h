@@ -16,6 +16,8 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // [d1][d0] with box (b0, b1); the row swizzle of a D-wide bf16 operand.
 bool map3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1,
            CUtensorMapSwizzle sw);
+bool map2d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint32_t b0, uint32_t b1,
+           CUtensorMapSwizzle sw);
 bool map2d_f32(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint32_t b0, uint32_t b1);
 CUtensorMapSwizzle row_swizzle(int D);
 unsigned long long wait_timeout_ns();

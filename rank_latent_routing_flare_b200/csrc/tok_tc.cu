@@ -120,13 +120,25 @@ __global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_
 
   // one token row of the outputs (zeros for padding tokens)
   auto store_row = [&](int n, const float (&dk)[D], const float (&dv)[D]) {
-    if (p.g32 != nullptr) {
-      float* o = p.g32 + (static_cast<size_t>(b) * p.N + n) * p.g_ld + h * D;
+    if (p.ghi != nullptr) {  // high and low bf16 parts of the fp32 rows
+      const size_t o = (static_cast<size_t>(b) * p.N + n) * p.g_ld + h * D;
+      auto put = [&](int col, const float (&x)[D]) {
+        uint32_t hi[D / 2], lo[D / 2];
 #pragma unroll
-      for (int u = 0; u < D / 4; ++u) {
-        reinterpret_cast<float4*>(o + p.g_col_k)[u] = make_float4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
-        reinterpret_cast<float4*>(o + p.g_col_v)[u] = make_float4(dv[4 * u], dv[4 * u + 1], dv[4 * u + 2], dv[4 * u + 3]);
-      }
+        for (int k = 0; k < D / 2; ++k) {
+          hi[k] = pack_bf16x2(x[2 * k], x[2 * k + 1]);
+          lo[k] = pack_bf16x2(x[2 * k] - bf16_lo(hi[k]), x[2 * k + 1] - bf16_hi(hi[k]));
+        }
+        uint4* dh = reinterpret_cast<uint4*>(p.ghi + o + col);
+        uint4* dl = reinterpret_cast<uint4*>(p.glo + o + col);
+#pragma unroll
+        for (int u = 0; u < D / 8; ++u) {
+          dh[u] = make_uint4(hi[4 * u], hi[4 * u + 1], hi[4 * u + 2], hi[4 * u + 3]);
+          dl[u] = make_uint4(lo[4 * u], lo[4 * u + 1], lo[4 * u + 2], lo[4 * u + 3]);
+        }
+      };
+      put(p.g_col_k, dk);
+      put(p.g_col_v, dv);
     } else {
       uint4* ok = reinterpret_cast<uint4*>(p.dk16 + (static_cast<size_t>(bh) * p.N + n) * D);
       uint4* ov = reinterpret_cast<uint4*>(p.dv16 + (static_cast<size_t>(bh) * p.N + n) * D);
