@@ -102,21 +102,28 @@ def test_flarepp_backward_matches_oracle(name, N, B):
             assert np.all(got["dX"][b, L:] == 0)
 
 
-def storage_model_bwd(w, dY):
+def storage_model_bwd(w, dY, p_round=False):
     """The oracle's FLARE++ backward in fp64 on the bf16 tensors that the
     forward stores and the backward reuses: the projections K~, V~, K, V and
     the synthesised queries Q(X), which the encode and the decode scores take
     in bf16 (eq. 10-11 on the forward's stored Q(X); its gradient passes
     through the rounding unchanged).  Everything else is kept in fp32 on the
-    GPU and in fp64 here."""
+    GPU and in fp64 here.  With ``p_round`` Q(X) and Z come from the forward
+    storage model that also rounds the softmax weights of the value products
+    to bf16 (as the forward's kernels read them)."""
+    from tests.parity import storage_model
     from workloads import bf16_bits_to_f64 as f64, to_bf16_bits
     r = lambda a: f64(to_bf16_bits(a.astype(np.float32)))
     X, Q0, dy = f64(w.X), f64(w.Q0), f64(dY)
     Wk, Wv, Wks, Wvs = (f64(a) for a in (w.Wk, w.Wv, w.Wk_syn, w.Wv_syn))
     Kt, Vt = r(oracle.project(X, Wks, w.H)), r(oracle.project(X, Wvs, w.H))
     K, V = r(oracle.project(X, Wk, w.H)), r(oracle.project(X, Wv, w.H))
-    Qx = r(oracle.encode(Q0, Kt, Vt, w.lengths))
-    Z = oracle.encode(Qx, K, V, w.lengths)
+    if p_round:
+        fwd = storage_model(w, oracle, p_round=True)
+        Qx, Z = r(fwd["Qx"]), fwd["Z"]
+    else:
+        Qx = r(oracle.encode(Q0, Kt, Vt, w.lengths))
+        Z = oracle.encode(Qx, K, V, w.lengths)
     dK, dQx, dZ = oracle.decode_bwd(K, Qx, Z, dy, w.lengths)
     dQx_e, dK_e, dV = oracle.encode_bwd(Qx, K, V, dZ, w.lengths)
     dQ0, dKt, dVt = oracle.encode_bwd(Q0, Kt, Vt, dQx + dQx_e, w.lengths)
@@ -131,21 +138,25 @@ def test_flarepp_backward_sharp_matches_bf16_storage_model():
     """Diagnostic with all weights ~ N(0, 16/C) (not a graded workload): the
     sharp softmaxes make the gradients sensitive to the bf16 storage of the
     projections and of Q(X), which alone moves them by 2-11 % from the exact
-    fp64 values (Q(X) in bf16 accounts for up to 3 % of it).  The rest of
-    the GPU path (the forward's softmax weights in bf16 for its value
-    products, fp32 everything else) moves them by well under 1e-2 more.
-    Checked: the GPU within 1e-2 (rel-L2) of the storage model, and no
-    further from the exact gradients than the storage model plus 1e-2; both
-    distances are printed."""
+    fp64 values (Q(X) in bf16 accounts for up to 3 % of it).  The forward
+    also rounds its softmax weights to bf16 for the value products that give
+    Q(X) and Z; that rounding is random (its pattern depends on the shift,
+    which differs between the kernels and any model), so it is bounded by its
+    size in the model: r_P = rel-L2 between the storage model with and
+    without it (1-2 % here).  Checked: the GPU within 1e-2 + 1.5 r_P (rel-L2)
+    of the storage model, and no further from the exact gradients than the
+    storage model plus 1e-2; the distances are printed."""
     w = make_workload("flarepp_n8k_sharp", N=1200, B=2)
     dY = make_upstream_grad(w)
     got = run_flarepp_bwd(w, dY)
     model = storage_model_bwd(w, dY)
+    model_p = storage_model_bwd(w, dY, p_round=True)
     exact = oracle.backward_workload(w, dY)
     for k in ("dX", "dWk", "dWv", "dWk_syn", "dWv_syn", "dQ0"):
+        r_p = rel_l2(model_p[k], model[k])
         print(f"sharp {k}: storage model vs exact {rel_l2(model[k], exact[k]):.3e}, "
-              f"gpu vs exact {rel_l2(got[k], exact[k]):.3e}")
-        check(got[k], model[k], f"sharp {k} vs storage model", rel_bound=1e-2, max_bound=5e-2)
+              f"gpu vs exact {rel_l2(got[k], exact[k]):.3e}, weight rounding r_P {r_p:.3e}")
+        check(got[k], model[k], f"sharp {k} vs storage model", rel_bound=1e-2 + 1.5 * r_p, max_bound=5e-2)
         assert rel_l2(got[k], exact[k]) <= rel_l2(model[k], exact[k]) + 1e-2
 
 
