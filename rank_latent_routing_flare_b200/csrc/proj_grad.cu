@@ -4,7 +4,8 @@
 // Wcat = [W_K | W_V | W~_K | W~_V] (each [C][C], K = X W_K):
 //   dX = G Wcat^T               (dx_tc_kernel)
 //   dWcat = X^T G               (dw_tc_kernel: per-split partials of its
-//                                transpose, then dw_tc_reduce_kernel)
+//                                transpose, then dw_tc_reduce_kernel sums
+//                                them in a fixed order)
 // G arrives as two bf16 planes, high and low parts (G = Ghi + Glo to about
 // 2^-16 relative), so every product runs as two kind::f16 MMAs on operands
 // the tensor core reads straight from their bf16 storage (X and W are bf16
@@ -344,23 +345,35 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-// dW_q[c][jj] = sum over splits (ascending) of part[s][q*C + jj][c] (+ the
-// (q+2) block when the synthesis weights are the encode weights): one
-// thread per output, consecutive threads along c so that the reads coalesce.
+// dW_q[c][jj] = sum over the splits of part[s][q*C + jj][c] (+ the (q+2)
+// block when the synthesis weights are the encode weights).  A block of 256
+// threads owns 32 consecutive c of one row j: its eight warps sum the splits
+// w, w + 8, w + 16, ... (lanes along c, so the reads coalesce) and the eight
+// partial sums are then added in warp order: a fixed order, so the result
+// does not depend on timing.
+constexpr int kRedGroups = 8;
+
 __global__ void __launch_bounds__(256) dw_tc_reduce_kernel(const DwReduceParams p) {
-  const int ncols = p.shared ? 2 * p.C : p.J;
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= p.C * ncols) return;
-  const int c = idx % p.C, j = idx / p.C;
+  __shared__ float red[kRedGroups][32];
+  const int cblocks = p.C / 32;
+  const int j = blockIdx.x / cblocks;
+  const int lane = threadIdx.x & 31, g = threadIdx.x >> 5;
+  const int c = (blockIdx.x % cblocks) * 32 + lane;
   float s = 0.f;
-  for (int sp = 0; sp < p.n_splits; ++sp) {
+  for (int sp = g; sp < p.n_splits; sp += kRedGroups) {
     const float* blk = p.part + static_cast<size_t>(sp) * p.J * p.C;
     s += blk[static_cast<size_t>(j) * p.C + c];
     if (p.shared) s += blk[static_cast<size_t>(j + 2 * p.C) * p.C + c];
   }
+  red[g][lane] = s;
+  __syncthreads();
+  if (g != 0) return;
+  float t = red[0][lane];
+#pragma unroll
+  for (int k = 1; k < kRedGroups; ++k) t += red[k][lane];
   const int q = j / p.C, jj = j % p.C;
-  if (p.dw[q]) p.dw[q][static_cast<size_t>(c) * p.C + jj] = s;
-  if (p.shared && p.dw[q + 2]) p.dw[q + 2][static_cast<size_t>(c) * p.C + jj] = s;
+  if (p.dw[q]) p.dw[q][static_cast<size_t>(c) * p.C + jj] = t;
+  if (p.shared && p.dw[q + 2]) p.dw[q + 2][static_cast<size_t>(c) * p.C + jj] = t;
 }
 
 template <class Cfg>
@@ -404,8 +417,9 @@ cudaError_t launch_dw_tc(const DwTcMaps& m, const DwTcParams& p, cudaStream_t s)
 }
 
 cudaError_t launch_dw_tc_reduce(const DwReduceParams& p, cudaStream_t s) {
-  const long n = static_cast<long>(p.C) * (p.shared ? 2 * p.C : p.J);
-  dw_tc_reduce_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(p);
+  if (p.C % 32 != 0) return cudaErrorInvalidValue;
+  const long rows = p.shared ? 2 * p.C : p.J;
+  dw_tc_reduce_kernel<<<static_cast<unsigned>(rows * (p.C / 32)), kRedGroups * 32, 0, s>>>(p);
   return cudaGetLastError();
 }
 

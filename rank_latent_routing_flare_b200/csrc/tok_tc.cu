@@ -2,13 +2,11 @@
 // key and value rows for the training backward, whose queries are bf16
 // values (Q(X), Q0 or the learned Q) so that the score products are exact.
 // One CTA owns a tile of 128 tokens of one head (thread <-> TMEM lane <->
-// token) and walks the latents in chunks of C = 32 (full) or 48 (encoder
-// only: half the work per score, so longer chunks amortise the per-chunk
-// hand-offs):
+// token) and walks the latents in chunks of C = 16:
 //
 //   full (kTokTcFull: decoder and encoder, FLARE++ paper eq. 10-11; FLARE
 //   paper eq. 5-6), per chunk:
-//     S = K Q_c^T, dA = V dZ_c^T, dP = dY Z_c^T     UMMA M=128 x N=C, fp32 TMEM
+//     S = K Q_c^T, dA = V dZ_c^T, dP = dY Z_c^T     UMMA M=128 x N=16, fp32 TMEM
 //       (dZ and Z fp32, each as two bf16 parts: two UMMAs)
 //     A = 2^(S c - L_m), P = 2^(S c - L_n)
 //     dS = A (dA - gamma_m) + P (dP - delta_n)       softmax threads
@@ -20,16 +18,16 @@
 // padding tokens are zero.  The score scale is applied to the fp32 product,
 // as in the forward, so that the forward's normalisers L_m fit these scores.
 //
-// The token tile's K, V and dY stay in shared memory; the latent chunks
-// (Q_c, the parts of Z_c and dZ_c, L_m and gamma_m) stream through a TMA
-// ring.  TMEM: S at column 0, dA at C, dP at 2C (full), dK at 96, dV at 112
-// (128 columns: four CTAs per SM).  The softmax threads read a chunk in 16-column
-// pieces and write, over the piece they have read, dS as bf16 high and low
-// parts (S columns [16j, 16j+8) and [16j+8, 16j+16)) and A in bf16 (dA
-// columns [16j, 16j+8)); each 16-latent k-step of the value MMAs takes its A
-// operand from 8 consecutive columns.  One score buffer: the MMA thread
-// issues the next chunk's products once the value MMAs of the previous one
-// are done; the four co-resident CTAs of an SM fill each other's gaps.
+// The token tile's K, V and dY stay in shared memory; the latents (Q, the
+// parts of Z and dZ, L_m and gamma_m) stream through a TMA ring of 32-latent
+// stages (two chunks each).  TMEM holds two score buffers (S, dA and, full,
+// dP: 16 columns each) and the dK, dV accumulators at columns 96 and 112
+// (128 columns: four CTAs per SM).  The MMA thread issues chunk j + 1's score
+// products into the other buffer before it waits for the softmax threads to
+// finish chunk j, so the score products of one chunk overlap the softmax of
+// the previous one.  The softmax threads write, over the columns they have
+// read, dS as bf16 high and low parts (S columns [0, 8) and [8, 16)) and A in
+// bf16 (dA columns [0, 8)); the value MMAs take them as TMEM A operands.
 //
 // Warp roles (5 warps): warp 0 lane 0 issues the TMA loads and the MMAs;
 // warps 1..4 are the softmax warps.
@@ -50,13 +48,14 @@ template <int MODE>
 struct TokTcCfg {
   static constexpr bool FULL = MODE == kTokTcFull;
   static constexpr int D = 16;
-  static constexpr int C = FULL ? 32 : 48;              // latents per chunk
+  static constexpr int C = 16;                          // latents per chunk (one k-step of the value MMAs)
+  static constexpr int CR = 2 * C;                      // latents per ring stage
   static constexpr int TT = kBwdTokBlock;               // tokens per CTA (128)
   static constexpr int ROWB = D * 2;
   static constexpr int TOK_B = TT * ROWB;               // one token tile (K, V or dY)
-  static constexpr int CH_B = C * ROWB;                 // one latent chunk of Q, Zhi, Zlo, dZhi or dZlo
-  static constexpr int NCH = FULL ? 5 : 3;              // chunks per ring stage
-  static constexpr int ST_B = NCH * CH_B + 2 * 256;     // a ring stage: the chunks, L_m, gamma_m
+  static constexpr int CH_B = CR * ROWB;                // a stage's rows of Q, Zhi, Zlo, dZhi or dZlo
+  static constexpr int NCH = FULL ? 5 : 3;              // latent tensors per ring stage
+  static constexpr int ST_B = NCH * CH_B + 2 * 256;     // a ring stage: the tensors, L_m, gamma_m
   static constexpr int NST = 6;
   static constexpr uint32_t LAYOUT = LAYOUT_SW32;
   static constexpr uint32_t SBO = 8 * ROWB;
@@ -66,15 +65,18 @@ struct TokTcCfg {
   static constexpr int S_Q = 0, S_DH = CH_B, S_DL = 2 * CH_B, S_ZH = 3 * CH_B, S_ZL = 4 * CH_B;
   static constexpr int S_LM = NCH * CH_B, S_GM = NCH * CH_B + 256;
   static constexpr int OFF_BAR = OFF_RING + NST * ST_B;
-  static constexpr int OFF_MISC = OFF_BAR + 8 * (6 + NST);
+  static constexpr int OFF_MISC = OFF_BAR + 8 * (8 + NST);
   static constexpr int BYTES = OFF_MISC + 64 + NST * 4;
+  // one score buffer: S, dA (and dP) of a chunk
+  static constexpr uint32_t BUF = FULL ? 3 * C : 2 * C;
   static constexpr uint32_t COL_S = 0, COL_DA = C, COL_DP = 2 * C, COL_DK = 96, COL_DV = 96 + D;
   static constexpr uint32_t TMEM_COLS = 128;
   static constexpr int THREADS = 160;
   static constexpr int CTAS_PER_SM = 4;
-  static_assert(COL_DV + D <= TMEM_COLS && (FULL ? 3 : 2) * C <= static_cast<int>(COL_DK), "TMEM columns");
-  static_assert(TOK_B % 1024 == 0 && CH_B % 256 == 0 && ST_B % 256 == 0, "tiles must hold whole swizzle atoms");
-  static_assert(C * 4 <= 256, "L_m / gamma_m of a chunk");
+  static_assert(COL_DV + D <= TMEM_COLS && 2 * BUF <= COL_DK, "TMEM columns");
+  static_assert(TOK_B % 1024 == 0 && CH_B % 256 == 0 && ST_B % 256 == 0 && (C * ROWB) % 256 == 0,
+                "tiles and chunks must hold whole swizzle atoms");
+  static_assert(CR * 4 <= 256, "L_m / gamma_m of a stage");
 };
 
 template <int MODE>
@@ -96,11 +98,11 @@ __global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_
   uint8_t* ring = sm + Cfg::OFF_RING;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Cfg::OFF_BAR);
   uint64_t* tok_full = bars;               // the token tile landed
-  uint64_t* s_full = bars + 1;             // the chunk's S, dA (dP) computed
-  uint64_t* p_full = bars + 2;             // dS and A stored by every softmax warp
-  uint64_t* pv_done = bars + 3;            // the chunk's value MMAs done
-  uint64_t* o_full = bars + 4;             // every MMA of the CTA done
-  uint64_t* lat_full = bars + 6;           // [NST] ring stage landed
+  uint64_t* s_full = bars + 1;             // [2] a buffer's S, dA (dP) computed
+  uint64_t* p_full = bars + 3;             // [2] dS and A of a buffer stored by every softmax warp
+  uint64_t* pv_done = bars + 5;            // [2] a buffer's value MMAs done
+  uint64_t* o_full = bars + 7;             // every MMA of the CTA done
+  uint64_t* lat_full = bars + 8;           // [NST] ring stage landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(sm + Cfg::OFF_MISC + 4);
   volatile int* last_load = reinterpret_cast<volatile int*>(sm + Cfg::OFF_MISC + 64);  // per stage
@@ -115,7 +117,8 @@ __global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_
   const int L = shard_valid_len(p.lengths, b, p.N, 0, p.N, &bad_len);
   if (bad_len && threadIdx.x == 0) atomicOr(p.err, FLARE_DEV_BAD_LENGTH);
   const int n0 = tile * Cfg::TT;
-  const int nchunks = (p.M + C - 1) / C;
+  const int nchunks = p.M / C;              // M is a multiple of 16
+  const int nstages = (p.M + Cfg::CR - 1) / Cfg::CR;
   pdl_launch_dependents();
 
   // one token row of the outputs (zeros for padding tokens)
@@ -164,9 +167,11 @@ __global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_
 
   if (threadIdx.x == 0) {
     mbar_init(tok_full, 1);
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full + b, 1);
+      mbar_init(p_full + b, 4);
+      mbar_init(pv_done + b, 1);
+    }
     mbar_init(o_full, 1);
     for (int i = 0; i < NST; ++i) {
       mbar_init(lat_full + i, 1);
@@ -185,11 +190,11 @@ __global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_
   pdl_wait();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{p.err, abort_flag, p.timeout_ns};
-  // latent chunk j into ring stage j % NST (one thread)
-  auto load_chunk = [&](int j) {
-    const int st = j % NST, m0 = j * C;
+  // latents [32 j, 32 j + 32) into ring stage j % NST (one thread)
+  auto load_stage = [&](int j) {
+    const int st = j % NST, m0 = j * Cfg::CR;
     uint8_t* sb = ring + st * Cfg::ST_B;
-    mbar_arrive_expect_tx(lat_full + st, (FULL ? 5 : 3) * Cfg::CH_B + 2 * C * 4);
+    mbar_arrive_expect_tx(lat_full + st, (FULL ? 5 : 3) * Cfg::CH_B + 2 * Cfg::CR * 4);
     tma_load_3d(sb + Cfg::S_Q, &tm_q, lat_full + st, 0, m0, g);
     tma_load_3d(sb + Cfg::S_DH, &tm_dh, lat_full + st, 0, m0, bh);
     tma_load_3d(sb + Cfg::S_DL, &tm_dl, lat_full + st, 0, m0, bh);
@@ -209,51 +214,58 @@ __global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_
       tma_load_3d(stk, &tm_k, tok_full, 0, n0, bh);
       tma_load_3d(stv, &tm_v, tok_full, 0, n0, bh);
       if (FULL) tma_load_3d(sty, &tm_y, tok_full, 0, n0, bh);
-      for (int j = 0; j < min(NST, nchunks); ++j) load_chunk(j);
+      for (int j = 0; j < min(NST, nstages); ++j) load_stage(j);
       const uint32_t idesc_v = idesc_bf16_f32(128, D, false, true);
+      const uint32_t idesc_s = idesc_bf16_f32(128, C, false, false);
       const uint64_t tk_desc = umma_desc(smem_u32(stk), 16, Cfg::SBO, Cfg::LAYOUT);
       const uint64_t tv_desc = umma_desc(smem_u32(stv), 16, Cfg::SBO, Cfg::LAYOUT);
       const uint64_t ty_desc = umma_desc(smem_u32(sty), 16, Cfg::SBO, Cfg::LAYOUT);
-      // a chunk as the K-major B operand of a score product (N = C latents)
-      // and as the MN-major B operand of a value product (N = D, k-steps of
-      // 16 latents); a stage's descriptor adds its offset >> 4
+      // a chunk as the K-major B operand of a score product (N = 16 latents)
+      // and as the MN-major B operand of a value product (N = D, one k-step
+      // of 16 latents); a chunk's descriptor adds its offset >> 4
       const uint64_t r_desc = umma_desc(smem_u32(ring), 16, Cfg::SBO, Cfg::LAYOUT);
-      constexpr uint64_t STAGE = Cfg::ST_B >> 4, KSTEP = (16 * Cfg::ROWB) >> 4;
+      constexpr uint64_t STAGE = Cfg::ST_B >> 4, HALF = (Cfg::C * Cfg::ROWB) >> 4;
       constexpr uint64_t OQ = Cfg::S_Q >> 4, OZH = Cfg::S_ZH >> 4, OZL = Cfg::S_ZL >> 4, ODH = Cfg::S_DH >> 4,
                          ODL = Cfg::S_DL >> 4;
-      bool ok = mbar_wait_mma(tok_full, 0, wc);
-      for (int j = 0; ok && j < nchunks; ++j) {
-        const int st = j % NST;
-        const int cn = min(C, p.M - j * C);  // C, or a multiple of 16 for the last chunk
-        if (j > 0) {
-          // the value MMAs of chunk j - 1 are done: S, dA, dP may be
-          // overwritten, and its ring stage takes chunk j - 1 + NST
-          if (!mbar_wait_mma(pv_done, (j - 1) & 1, wc)) { ok = false; break; }
-          if (j - 1 + NST < nchunks) load_chunk(j - 1 + NST);
-        }
-        if (!mbar_wait_mma(lat_full + st, (j / NST) & 1, wc)) { ok = false; break; }
+      auto chunk_desc = [&](int j) { return r_desc + ((j >> 1) % NST) * STAGE + (j & 1) * HALF; };
+      // the score products of chunk j into buffer j & 1
+      auto scores = [&](int j) -> bool {
+        const int sj = j >> 1;
+        if (!mbar_wait_mma(lat_full + sj % NST, (sj / NST) & 1, wc)) return false;
         tc_fence_after();
-        const uint64_t rd = r_desc + st * STAGE;
-        const uint32_t idesc_s = idesc_bf16_f32(128, cn, false, false);
-        umma_ss(tmem + Cfg::COL_S, tk_desc, rd + OQ, idesc_s, 0u);    // K Q_c^T
-        umma_ss(tmem + Cfg::COL_DA, tv_desc, rd + ODH, idesc_s, 0u);  // V dZhi_c^T
-        umma_ss(tmem + Cfg::COL_DA, tv_desc, rd + ODL, idesc_s, 1u);  // + V dZlo_c^T
+        const uint64_t rd = chunk_desc(j);
+        const uint32_t tb = tmem + (j & 1) * Cfg::BUF;
+        umma_ss(tb + Cfg::COL_S, tk_desc, rd + OQ, idesc_s, 0u);    // K Q_c^T
+        umma_ss(tb + Cfg::COL_DA, tv_desc, rd + ODH, idesc_s, 0u);  // V dZhi_c^T
+        umma_ss(tb + Cfg::COL_DA, tv_desc, rd + ODL, idesc_s, 1u);  // + V dZlo_c^T
         if (FULL) {
-          umma_ss(tmem + Cfg::COL_DP, ty_desc, rd + OZH, idesc_s, 0u);  // dY Zhi_c^T
-          umma_ss(tmem + Cfg::COL_DP, ty_desc, rd + OZL, idesc_s, 1u);  // + dY Zlo_c^T
+          umma_ss(tb + Cfg::COL_DP, ty_desc, rd + OZH, idesc_s, 0u);  // dY Zhi_c^T
+          umma_ss(tb + Cfg::COL_DP, ty_desc, rd + OZL, idesc_s, 1u);  // + dY Zlo_c^T
         }
-        umma_commit(s_full);
-        if (!mbar_wait_mma(p_full, j & 1, wc)) { ok = false; break; }
+        umma_commit(s_full + (j & 1));
+        return true;
+      };
+      bool ok = mbar_wait_mma(tok_full, 0, wc) && scores(0);
+      for (int j = 0; ok && j < nchunks; ++j) {
+        if (j + 1 < nchunks) {
+          if (j >= 1) {
+            // chunk j - 1's value MMAs are done: its buffer takes chunk j + 1,
+            // and once both chunks of a stage are done the stage is refilled
+            if (!mbar_wait_mma(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, wc)) { ok = false; break; }
+            if (((j - 1) & 1) && ((j - 1) >> 1) + NST < nstages) load_stage(((j - 1) >> 1) + NST);
+          }
+          if (!scores(j + 1)) { ok = false; break; }
+        }
+        if (!mbar_wait_mma(p_full + (j & 1), (j >> 1) & 1, wc)) { ok = false; break; }
         tc_fence_after();
-        for (int ks = 0; ks < cn / 16; ++ks) {
-          const uint32_t as = tmem + Cfg::COL_S + 16 * ks, aa = tmem + Cfg::COL_DA + 16 * ks;
-          const uint32_t acc0 = (j > 0 || ks > 0) ? 1u : 0u;
-          umma_ts(tmem + Cfg::COL_DK, as, rd + OQ + ks * KSTEP, idesc_v, acc0);       // dShi Q_c
-          umma_ts(tmem + Cfg::COL_DK, as + 8, rd + OQ + ks * KSTEP, idesc_v, 1u);     // dSlo Q_c
-          umma_ts(tmem + Cfg::COL_DV, aa, rd + ODH + ks * KSTEP, idesc_v, acc0);      // A dZhi_c
-          umma_ts(tmem + Cfg::COL_DV, aa, rd + ODL + ks * KSTEP, idesc_v, 1u);        // A dZlo_c
-        }
-        umma_commit(pv_done);
+        const uint64_t rd = chunk_desc(j);
+        const uint32_t tb = tmem + (j & 1) * Cfg::BUF;
+        const uint32_t acc0 = j > 0 ? 1u : 0u;
+        umma_ts(tmem + Cfg::COL_DK, tb + Cfg::COL_S, rd + OQ, idesc_v, acc0);        // dShi Q_c
+        umma_ts(tmem + Cfg::COL_DK, tb + Cfg::COL_S + 8, rd + OQ, idesc_v, 1u);      // dSlo Q_c
+        umma_ts(tmem + Cfg::COL_DV, tb + Cfg::COL_DA, rd + ODH, idesc_v, acc0);      // A dZhi_c
+        umma_ts(tmem + Cfg::COL_DV, tb + Cfg::COL_DA, rd + ODL, idesc_v, 1u);        // A dZlo_c
+        umma_commit(pv_done + (j & 1));
       }
       umma_commit(o_full);  // completes once every MMA issued above is done
       mbar_wait_drain(o_full, 0, p.timeout_ns);
@@ -313,29 +325,28 @@ __global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_
     };
     bool ok = true;
     for (int j = 0; j < nchunks; ++j) {
-      if (!mbar_wait_warp(s_full, j & 1, wc)) { ok = false; break; }
+      const int b = j & 1;
+      if (!mbar_wait_warp(s_full + b, (j >> 1) & 1, wc)) { ok = false; break; }
       tc_fence_after();
-      const int cn = min(C, p.M - j * C);
-      const uint8_t* sb = ring + (j % NST) * Cfg::ST_B;
-      const float* lm = reinterpret_cast<const float*>(sb + Cfg::S_LM);
-      const float* gm = reinterpret_cast<const float*>(sb + Cfg::S_GM);
-      for (int q = 0; q < cn / 16; ++q) {
-        uint32_t sv[16], av[16], pv[16], hi[8], lo[8], wa[8];
-        tmem_ld16(lane_base + Cfg::COL_S + 16 * q, sv);
-        tmem_ld16(lane_base + Cfg::COL_DA + 16 * q, av);
-        if (FULL) tmem_ld16(lane_base + Cfg::COL_DP + 16 * q, pv);
-        tmem_wait_ld();
-        regs_defined16(sv);
-        regs_defined16(av);
-        if (FULL) regs_defined16(pv);
-        piece(sv, av, pv, lm + 16 * q, gm + 16 * q, hi, lo, wa);
-        tmem_st8(lane_base + Cfg::COL_S + 16 * q, hi);
-        tmem_st8(lane_base + Cfg::COL_S + 16 * q + 8, lo);
-        tmem_st8(lane_base + Cfg::COL_DA + 16 * q, wa);
-      }
+      const uint8_t* sb = ring + ((j >> 1) % NST) * Cfg::ST_B;
+      const float* lm = reinterpret_cast<const float*>(sb + Cfg::S_LM) + b * C;
+      const float* gm = reinterpret_cast<const float*>(sb + Cfg::S_GM) + b * C;
+      const uint32_t tb = lane_base + b * Cfg::BUF;
+      uint32_t sv[16], av[16], pv[16], hi[8], lo[8], wa[8];
+      tmem_ld16(tb + Cfg::COL_S, sv);
+      tmem_ld16(tb + Cfg::COL_DA, av);
+      if (FULL) tmem_ld16(tb + Cfg::COL_DP, pv);
+      tmem_wait_ld();
+      regs_defined16(sv);
+      regs_defined16(av);
+      if (FULL) regs_defined16(pv);
+      piece(sv, av, pv, lm, gm, hi, lo, wa);
+      tmem_st8(tb + Cfg::COL_S, hi);
+      tmem_st8(tb + Cfg::COL_S + 8, lo);
+      tmem_st8(tb + Cfg::COL_DA, wa);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive_warp(p_full);
+      mbar_arrive_warp(p_full + b);
       __syncwarp();
     }
     if (ok && mbar_wait_warp(o_full, 0, wc)) {
@@ -379,7 +390,7 @@ size_t tok_tc_smem_bytes(int mode) {
   return need > floor ? need : floor;
 }
 
-int tok_tc_chunk(int mode) { return mode == kTokTcFull ? TokTcCfg<kTokTcFull>::C : TokTcCfg<kTokTcEncoder>::C; }
+int tok_tc_chunk(int mode) { return mode == kTokTcFull ? TokTcCfg<kTokTcFull>::CR : TokTcCfg<kTokTcEncoder>::CR; }
 
 cudaError_t launch_tok_tc(int mode, const TokTcMaps& m, const TokTcParams& p, cudaStream_t s) {
   if (p.D != 16) return cudaErrorInvalidValue;
