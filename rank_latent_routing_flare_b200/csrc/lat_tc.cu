@@ -20,17 +20,17 @@
 // score scale c = scale log2(e) is applied to the fp32 product, as in the
 // forward's kernels, so that the forward's normalisers L_m fit these scores.
 //
-// The split's tokens stream through a TMA ring in stages of 32 (K and V, or K
-// and dY, plus L_n and delta_n for the decoder) and are worked on in tiles of
-// T = 16 tokens.  TMEM holds two score buffers (S and G of a tile, 16
-// columns each, at columns 0 and 32) and the dQ, dZ accumulators at 96 and
-// 112 (128 columns: four CTAs per SM).  The MMA thread issues tile i + 1's S
-// and G into the other buffer before it waits for the softmax threads to
-// finish tile i, so the score products of one tile overlap the softmax of the
-// previous one.  The softmax threads write, over the columns they have read,
-// dS as bf16 high and low parts (S columns [0, 8) and [8, 16)) and, for the
-// decoder, W in bf16 (G columns [0, 8)); the value MMAs (one 16-token k-step)
-// take them as TMEM A operands.
+// Tiles of T = 48 tokens stream through a TMA ring (K and V, or K and dY,
+// plus L_n and delta_n for the decoder).  TMEM: S at column 0, G at 48, dQ at
+// 96, dZ at 112 (128 columns: four CTAs per SM).  The softmax threads read a
+// tile's S and G in three 16-column pieces (the next piece's TMEM load in
+// flight while the current one is computed) and write, over the piece they
+// have read, dS as bf16 high and low parts (S columns [16j, 16j+8) and
+// [16j+8, 16j+16)) and, for the decoder, W in bf16 (G columns [16j, 16j+8)):
+// each 16-token k-step of the value MMAs then takes its A operand from 8
+// consecutive columns.  One score buffer: the MMA thread issues the next
+// tile's S and G once the value MMAs of the previous tile are done; the four
+// co-resident CTAs of an SM fill each other's gaps.
 //
 // Warp roles (5 warps): warp 0 lane 0 issues the TMA loads and the MMAs;
 // warps 1..4 are the softmax warps (thread <-> TMEM lane <-> latent row).
@@ -51,33 +51,30 @@ __device__ __forceinline__ void regs_defined(uint32_t (&r)[16]) {
 
 struct LatTcCfg {
   static constexpr int D = 16;
-  static constexpr int T = 16;                          // tokens per tile (one k-step of the value MMAs)
-  static constexpr int TR = 2 * T;                      // tokens per ring stage
+  static constexpr int T = 48;                          // tokens per tile
   static constexpr int ROWB = D * 2;                    // bytes of one bf16 row
-  static constexpr int TILE_B = TR * ROWB;              // one stage's K, V or dY rows
+  static constexpr int TILE_B = T * ROWB;               // one K, V or dY tile
   static constexpr int ROWS_B = kLatBlock * ROWB;       // Q, or one part of dZ / Z
-  static constexpr int LD_B = 256;                      // one stage's L_n or delta_n (TR floats, padded)
-  static constexpr int NST = 8;                         // ring stages
+  static constexpr int LD_B = 256;                      // one tile's L_n or delta_n (T floats, padded)
+  static constexpr int NST = 6;                         // ring stages
   static constexpr uint32_t LAYOUT = LAYOUT_SW32;
   static constexpr uint32_t SBO = 8 * ROWB;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_XA = OFF_Q + ROWS_B;         // dZhi (encoder) or Zhi (decoder)
   static constexpr int OFF_XB = OFF_XA + ROWS_B;        // the low parts
-  static constexpr int OFF_K = OFF_XB + ROWS_B;         // NST x K rows
-  static constexpr int OFF_U = OFF_K + NST * TILE_B;    // NST x (V or dY) rows
+  static constexpr int OFF_K = OFF_XB + ROWS_B;         // NST x K tile
+  static constexpr int OFF_U = OFF_K + NST * TILE_B;    // NST x (V or dY) tile
   static constexpr int OFF_LD = OFF_U + NST * TILE_B;   // NST x (L_n | delta_n)
   static constexpr int OFF_BAR = OFF_LD + NST * 2 * LD_B;
-  static constexpr int OFF_MISC = OFF_BAR + 8 * (8 + NST);
+  static constexpr int OFF_MISC = OFF_BAR + 8 * (6 + NST);
   static constexpr int BYTES = OFF_MISC + 64 + NST * 4;
-  static constexpr uint32_t BUF = 2 * T;                // one score buffer: S and G of a tile
-  static constexpr uint32_t COL_S = 0, COL_G = T, COL_DQ = 96, COL_DZ = 96 + D;
+  static constexpr uint32_t COL_S = 0, COL_G = T, COL_DQ = 2 * T, COL_DZ = 2 * T + D;
   static constexpr uint32_t TMEM_COLS = 128;
   static constexpr int THREADS = 160;
   static constexpr int CTAS_PER_SM = 4;
-  static_assert(COL_DZ + D <= TMEM_COLS && 2 * BUF <= COL_DQ, "TMEM columns");
-  static_assert(TILE_B % 256 == 0 && (T * ROWB) % 256 == 0 && ROWS_B % 1024 == 0,
-                "tiles must hold whole swizzle atoms");
-  static_assert(TR * 4 <= LD_B, "a stage of L_n / delta_n");
+  static_assert(COL_DZ + D <= TMEM_COLS, "TMEM columns");
+  static_assert(TILE_B % 256 == 0 && ROWS_B % 1024 == 0, "tiles must hold whole swizzle atoms");
+  static_assert(T % 16 == 0 && T * 4 <= LD_B, "tile of L_n / delta_n");
 };
 
 template <int MODE>
@@ -99,11 +96,11 @@ __global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
   uint8_t* sld = sm + Cfg::OFF_LD;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Cfg::OFF_BAR);
   uint64_t* q_full = bars;                 // Q and both parts of dZ / Z landed
-  uint64_t* s_full = bars + 1;             // [2] S and G of a buffer computed
-  uint64_t* p_full = bars + 3;             // [2] dS (and W) of a buffer stored by every softmax warp
-  uint64_t* pv_done = bars + 5;            // [2] the value MMAs of a buffer done
-  uint64_t* o_full = bars + 7;             // every MMA of the CTA done
-  uint64_t* kv_full = bars + 8;            // [NST] ring stage landed
+  uint64_t* s_full = bars + 1;             // S and G of the current tile computed
+  uint64_t* p_full = bars + 2;             // dS (and W) stored by every softmax warp
+  uint64_t* pv_done = bars + 3;            // the value MMAs of the tile done
+  uint64_t* o_full = bars + 4;             // every MMA of the CTA done
+  uint64_t* kv_full = bars + 6;            // [NST] ring stage landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(sm + Cfg::OFF_MISC + 4);
   volatile int* last_load = reinterpret_cast<volatile int*>(sm + Cfg::OFF_MISC + 64);  // per stage
@@ -122,7 +119,6 @@ __global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
   const int n_begin = s * p.split_tokens;
   const int n_end = min(n_begin + p.split_tokens, L);
   const int ntiles = n_end > n_begin ? (n_end - n_begin + T - 1) / T : 0;
-  const int nstages = (ntiles + 1) / 2;
   const size_t part_row0 = (static_cast<size_t>(bh) * S + s) * p.M;
   pdl_launch_dependents();
 
@@ -140,11 +136,9 @@ __global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(s_full + i, 1);
-      mbar_init(p_full + i, 4);
-      mbar_init(pv_done + i, 1);
-    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(pv_done, 1);
     mbar_init(o_full, 1);
     for (int i = 0; i < NST; ++i) {
       mbar_init(kv_full + i, 1);
@@ -163,11 +157,11 @@ __global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
   pdl_wait();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{p.err, abort_flag, p.timeout_ns};
-  // the split's tokens [32 n, 32 n + 32) into ring stage n % NST (one thread)
-  auto load_stage = [&](int n) {
+  // tile n of the split into ring stage n % NST (one thread)
+  auto load_tile = [&](int n) {
     const int st = n % NST;
-    const int tok = n_begin + n * Cfg::TR;
-    mbar_arrive_expect_tx(kv_full + st, 2 * Cfg::TILE_B + (DEC ? 2 * Cfg::TR * 4 : 0));
+    const int tok = n_begin + n * T;
+    mbar_arrive_expect_tx(kv_full + st, 2 * Cfg::TILE_B + (DEC ? 2 * T * 4 : 0));
     tma_load_3d(sk + st * Cfg::TILE_B, &tm_k, kv_full + st, 0, tok, bh);
     tma_load_3d(su + st * Cfg::TILE_B, &tm_u, kv_full + st, 0, tok, bh);
     if (DEC) {
@@ -189,52 +183,46 @@ __global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
       tma_load_3d(sq, &tm_q, q_full, 0, lb * kLatBlock, g);
       tma_load_3d(sxa, &tm_xa, q_full, 0, lb * kLatBlock, bh);
       tma_load_3d(sxb, &tm_xb, q_full, 0, lb * kLatBlock, bh);
-      for (int n = 0; n < min(NST, nstages); ++n) load_stage(n);
+      for (int n = 0; n < min(NST, ntiles); ++n) load_tile(n);
       const uint32_t idesc_s = idesc_bf16_f32(128, T, false, false);
       const uint32_t idesc_v = idesc_bf16_f32(128, D, false, true);
       const uint64_t q_desc = umma_desc(smem_u32(sq), 16, Cfg::SBO, Cfg::LAYOUT);
       const uint64_t xa_desc = umma_desc(smem_u32(sxa), 16, Cfg::SBO, Cfg::LAYOUT);
       const uint64_t xb_desc = umma_desc(smem_u32(sxb), 16, Cfg::SBO, Cfg::LAYOUT);
-      // a tile's rows as the K-major B operand of a score product (N = 16
-      // tokens) and as the MN-major B operand of a value product (N = D, one
-      // k-step of 16 tokens); a tile's descriptor adds its offset >> 4
+      // a ring tile as the K-major B operand of a score product (N = T
+      // tokens) and as the MN-major B operand of a value product (N = D,
+      // k-steps of 16 tokens); a stage's descriptor adds its offset >> 4
       const uint64_t k_desc = umma_desc(smem_u32(sk), 16, Cfg::SBO, Cfg::LAYOUT);
       const uint64_t u_desc = umma_desc(smem_u32(su), 16, Cfg::SBO, Cfg::LAYOUT);
-      constexpr uint64_t STAGE = Cfg::TILE_B >> 4, HALF = (T * Cfg::ROWB) >> 4;
-      auto tile_off = [&](int i) -> uint64_t { return ((i >> 1) % NST) * STAGE + (i & 1) * HALF; };
-      // S and G of tile i into buffer i & 1
-      auto scores = [&](int i) -> bool {
-        const int si = i >> 1;
-        if (!mbar_wait_mma(kv_full + si % NST, (si / NST) & 1, wc)) return false;
-        tc_fence_after();
-        const uint64_t off = tile_off(i);
-        const uint32_t tb = tmem + (i & 1) * Cfg::BUF;
-        umma_ss(tb + Cfg::COL_S, q_desc, k_desc + off, idesc_s, 0u);
-        umma_ss(tb + Cfg::COL_G, xa_desc, u_desc + off, idesc_s, 0u);
-        umma_ss(tb + Cfg::COL_G, xb_desc, u_desc + off, idesc_s, 1u);
-        umma_commit(s_full + (i & 1));
-        return true;
-      };
-      bool ok = mbar_wait_mma(q_full, 0, wc) && scores(0);
+      constexpr uint64_t STAGE = Cfg::TILE_B >> 4, KSTEP = (16 * Cfg::ROWB) >> 4;
+      bool ok = mbar_wait_mma(q_full, 0, wc);
       for (int i = 0; ok && i < ntiles; ++i) {
-        if (i + 1 < ntiles) {
-          if (i >= 1) {
-            // tile i - 1's value MMAs are done: its buffer takes tile i + 1,
-            // and once both tiles of a stage are done the stage is refilled
-            if (!mbar_wait_mma(pv_done + ((i - 1) & 1), ((i - 1) >> 1) & 1, wc)) { ok = false; break; }
-            if (((i - 1) & 1) && ((i - 1) >> 1) + NST < nstages) load_stage(((i - 1) >> 1) + NST);
-          }
-          if (!scores(i + 1)) { ok = false; break; }
+        const int st = i % NST;
+        if (i > 0) {
+          // the value MMAs of tile i - 1 are done: S and G may be overwritten,
+          // and tile i - 1's stage takes tile i - 1 + NST
+          if (!mbar_wait_mma(pv_done, (i - 1) & 1, wc)) { ok = false; break; }
+          if (i - 1 + NST < ntiles) load_tile(i - 1 + NST);
         }
-        if (!mbar_wait_mma(p_full + (i & 1), (i >> 1) & 1, wc)) { ok = false; break; }
+        if (!mbar_wait_mma(kv_full + st, (i / NST) & 1, wc)) { ok = false; break; }
         tc_fence_after();
-        const uint64_t off = tile_off(i);
-        const uint32_t tb = tmem + (i & 1) * Cfg::BUF;
-        const uint32_t acc0 = i > 0 ? 1u : 0u;
-        umma_ts(tmem + Cfg::COL_DQ, tb + Cfg::COL_S, k_desc + off, idesc_v, acc0);       // dShi K
-        umma_ts(tmem + Cfg::COL_DQ, tb + Cfg::COL_S + 8, k_desc + off, idesc_v, 1u);     // dSlo K
-        if (DEC) umma_ts(tmem + Cfg::COL_DZ, tb + Cfg::COL_G, u_desc + off, idesc_v, acc0);  // W dY
-        umma_commit(pv_done + (i & 1));
+        const uint64_t kd = k_desc + st * STAGE, ud = u_desc + st * STAGE;
+        umma_ss(tmem + Cfg::COL_S, q_desc, kd, idesc_s, 0u);
+        umma_ss(tmem + Cfg::COL_G, xa_desc, ud, idesc_s, 0u);
+        umma_ss(tmem + Cfg::COL_G, xb_desc, ud, idesc_s, 1u);
+        umma_commit(s_full);
+        if (!mbar_wait_mma(p_full, i & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < T / 16; ++ks) {
+          const uint32_t a = tmem + Cfg::COL_S + 16 * ks;
+          umma_ts(tmem + Cfg::COL_DQ, a, kd + ks * KSTEP, idesc_v, (i > 0 || ks > 0) ? 1u : 0u);  // dShi K
+          umma_ts(tmem + Cfg::COL_DQ, a + 8, kd + ks * KSTEP, idesc_v, 1u);                      // dSlo K
+          if (DEC)
+            umma_ts(tmem + Cfg::COL_DZ, tmem + Cfg::COL_G + 16 * ks, ud + ks * KSTEP, idesc_v,
+                    (i > 0 || ks > 0) ? 1u : 0u);                                                // W dY
+        }
+        umma_commit(pv_done);
       }
       umma_commit(o_full);  // completes once every MMA issued above is done
       mbar_wait_drain(o_full, 0, p.timeout_ns);
@@ -296,38 +284,51 @@ __global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
     };
     bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
-      const int bb = i & 1;
-      if (!mbar_wait_warp(s_full + bb, (i >> 1) & 1, wc)) { ok = false; break; }
+      if (!mbar_wait_warp(s_full, i & 1, wc)) { ok = false; break; }
       tc_fence_after();
       const int valid = min(T, n_end - (n_begin + i * T));
-      // this tile's L_n at sl[0..16), delta_n at sl[LD_B/4 ..)
-      const float* sl = reinterpret_cast<const float*>(sld + ((i >> 1) % NST) * 2 * Cfg::LD_B) + bb * T;
+      const float* sl = reinterpret_cast<const float*>(sld + (i % NST) * 2 * Cfg::LD_B);
       if (warp_live) {
-        const uint32_t tb = lane_base + bb * Cfg::BUF;
-        uint32_t sv[16], gv[16], hi[8], lo[8], wp[8];
-        tmem_ld16(tb + Cfg::COL_S, sv);
-        tmem_ld16(tb + Cfg::COL_G, gv);
+        const bool full = valid >= T;  // every token column of the tile is valid
+        uint32_t sv[2][16], gv[2][16];
+        tmem_ld16(lane_base + Cfg::COL_S, sv[0]);
+        tmem_ld16(lane_base + Cfg::COL_G, gv[0]);
         tmem_wait_ld();
-        regs_defined(sv);
-        regs_defined(gv);
-        piece(sv, gv, sl, hi, lo, wp);
-        if (valid < T) {  // the split's last valid token is in this tile: zero the columns past it
+        regs_defined(sv[0]);
+        regs_defined(gv[0]);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint32_t keep = 2 * k + 1 < valid ? 0xFFFFFFFFu : 2 * k < valid ? 0x0000FFFFu : 0u;
-            hi[k] &= keep;
-            lo[k] &= keep;
-            wp[k] &= keep;
+        for (int j = 0; j < T / 16; ++j) {
+          uint32_t hi[8], lo[8], wp[8];
+          const int cb = j & 1, nb = cb ^ 1;
+          if (j + 1 < T / 16) {  // the next piece, while this one is computed
+            tmem_ld16(lane_base + Cfg::COL_S + 16 * (j + 1), sv[nb]);
+            tmem_ld16(lane_base + Cfg::COL_G + 16 * (j + 1), gv[nb]);
+          }
+          piece(sv[cb], gv[cb], sl + 16 * j, hi, lo, wp);
+          if (!full) {  // the tile's last valid token column is in this tile: zero the columns past it
+            const int nv = valid - 16 * j;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const uint32_t keep = 2 * k + 1 < nv ? 0xFFFFFFFFu : 2 * k < nv ? 0x0000FFFFu : 0u;
+              hi[k] &= keep;
+              lo[k] &= keep;
+              wp[k] &= keep;
+            }
+          }
+          // over the 16 columns just read: dS high and low parts (and W)
+          tmem_st8(lane_base + Cfg::COL_S + 16 * j, hi);
+          tmem_st8(lane_base + Cfg::COL_S + 16 * j + 8, lo);
+          if (DEC) tmem_st8(lane_base + Cfg::COL_G + 16 * j, wp);
+          if (j + 1 < T / 16) {
+            tmem_wait_ld();
+            regs_defined(sv[nb]);
+            regs_defined(gv[nb]);
           }
         }
-        // over the columns just read: dS high and low parts (and W)
-        tmem_st8(tb + Cfg::COL_S, hi);
-        tmem_st8(tb + Cfg::COL_S + 8, lo);
-        if (DEC) tmem_st8(tb + Cfg::COL_G, wp);
         tmem_wait_st();
       }
       tc_fence_before();
-      mbar_arrive_warp(p_full + bb);
+      mbar_arrive_warp(p_full);
       __syncwarp();
     }
     if (ok && mbar_wait_warp(o_full, 0, wc)) {
@@ -392,7 +393,7 @@ size_t lat_tc_smem_bytes() {
   return need > floor ? need : floor;
 }
 
-int lat_tc_tile() { return LatTcCfg::TR; }
+int lat_tc_tile() { return LatTcCfg::T; }
 
 cudaError_t launch_lat_tc(int mode, const LatTcMaps& m, const LatTcParams& p, cudaStream_t s) {
   if (p.D != 16) return cudaErrorInvalidValue;

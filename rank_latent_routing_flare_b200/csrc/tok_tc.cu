@@ -2,11 +2,12 @@
 // key and value rows for the training backward, whose queries are bf16
 // values (Q(X), Q0 or the learned Q) so that the score products are exact.
 // One CTA owns a tile of 128 tokens of one head (thread <-> TMEM lane <->
-// token) and walks the latents in chunks of C = 16:
+// token) and walks the latents in chunks of C = 16 (full) or 48 (encoder
+// only):
 //
 //   full (kTokTcFull: decoder and encoder, FLARE++ paper eq. 10-11; FLARE
 //   paper eq. 5-6), per chunk:
-//     S = K Q_c^T, dA = V dZ_c^T, dP = dY Z_c^T     UMMA M=128 x N=16, fp32 TMEM
+//     S = K Q_c^T, dA = V dZ_c^T, dP = dY Z_c^T     UMMA M=128 x N=C, fp32 TMEM
 //       (dZ and Z fp32, each as two bf16 parts: two UMMAs)
 //     A = 2^(S c - L_m), P = 2^(S c - L_n)
 //     dS = A (dA - gamma_m) + P (dP - delta_n)       softmax threads
@@ -19,15 +20,22 @@
 // as in the forward, so that the forward's normalisers L_m fit these scores.
 //
 // The token tile's K, V and dY stay in shared memory; the latents (Q, the
-// parts of Z and dZ, L_m and gamma_m) stream through a TMA ring of 32-latent
-// stages (two chunks each).  TMEM holds two score buffers (S, dA and, full,
-// dP: 16 columns each) and the dK, dV accumulators at columns 96 and 112
-// (128 columns: four CTAs per SM).  The MMA thread issues chunk j + 1's score
-// products into the other buffer before it waits for the softmax threads to
-// finish chunk j, so the score products of one chunk overlap the softmax of
-// the previous one.  The softmax threads write, over the columns they have
-// read, dS as bf16 high and low parts (S columns [0, 8) and [8, 16)) and A in
-// bf16 (dA columns [0, 8)); the value MMAs take them as TMEM A operands.
+// parts of Z and dZ, L_m and gamma_m) stream through a TMA ring (stages of 32
+// latents, two chunks, in the full pass; of one 48-latent chunk in the
+// encoder-only one).  The dK, dV accumulators sit at TMEM columns 96 and 112
+// (128 columns: four CTAs per SM).  Full pass: two score buffers (S, dA, dP:
+// 16 columns each); the MMA thread issues chunk j + 1's score products into
+// the other buffer before it waits for the softmax threads to finish chunk
+// j, so the score products of one chunk overlap the softmax of the previous
+// one (measured: 4.39 against 5.02 ms per million-token launch with one
+// buffer of 32-latent chunks).  Encoder-only pass: one buffer (S at 0, dA at
+// 48), read in 16-column pieces, the next chunk's products issued once the
+// value products of the previous one are done (with half the work per
+// score, two buffers of 16-latent chunks measured slower: 3.64 against 3.36
+// ms).  The softmax threads write, over each 16-column piece they have read,
+// dS as bf16 high and low parts (S columns [0, 8) and [8, 16) of the piece)
+// and A in bf16 (dA columns [0, 8)); the value MMAs take them as TMEM A
+// operands, one 16-latent k-step per piece.
 //
 // Warp roles (5 warps): warp 0 lane 0 issues the TMA loads and the MMAs;
 // warps 1..4 are the softmax warps.
@@ -48,8 +56,10 @@ template <int MODE>
 struct TokTcCfg {
   static constexpr bool FULL = MODE == kTokTcFull;
   static constexpr int D = 16;
-  static constexpr int C = 16;                          // latents per chunk (one k-step of the value MMAs)
-  static constexpr int CR = 2 * C;                      // latents per ring stage
+  static constexpr bool DB = FULL;                      // two score buffers
+  static constexpr int C = FULL ? 16 : 48;              // latents per chunk
+  static constexpr int CR = FULL ? 2 * C : C;           // latents per ring stage
+  static constexpr int CPS = CR / C;                    // chunks per ring stage
   static constexpr int TT = kBwdTokBlock;               // tokens per CTA (128)
   static constexpr int ROWB = D * 2;
   static constexpr int TOK_B = TT * ROWB;               // one token tile (K, V or dY)
@@ -69,11 +79,12 @@ struct TokTcCfg {
   static constexpr int BYTES = OFF_MISC + 64 + NST * 4;
   // one score buffer: S, dA (and dP) of a chunk
   static constexpr uint32_t BUF = FULL ? 3 * C : 2 * C;
+  static constexpr int NBUF = DB ? 2 : 1;
   static constexpr uint32_t COL_S = 0, COL_DA = C, COL_DP = 2 * C, COL_DK = 96, COL_DV = 96 + D;
   static constexpr uint32_t TMEM_COLS = 128;
   static constexpr int THREADS = 160;
   static constexpr int CTAS_PER_SM = 4;
-  static_assert(COL_DV + D <= TMEM_COLS && 2 * BUF <= COL_DK, "TMEM columns");
+  static_assert(COL_DV + D <= TMEM_COLS && NBUF * BUF <= COL_DK, "TMEM columns");
   static_assert(TOK_B % 1024 == 0 && CH_B % 256 == 0 && ST_B % 256 == 0 && (C * ROWB) % 256 == 0,
                 "tiles and chunks must hold whole swizzle atoms");
   static_assert(CR * 4 <= 256, "L_m / gamma_m of a stage");
@@ -117,7 +128,7 @@ __global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_
   const int L = shard_valid_len(p.lengths, b, p.N, 0, p.N, &bad_len);
   if (bad_len && threadIdx.x == 0) atomicOr(p.err, FLARE_DEV_BAD_LENGTH);
   const int n0 = tile * Cfg::TT;
-  const int nchunks = p.M / C;              // M is a multiple of 16
+  const int nchunks = (p.M + C - 1) / C;   // M is a multiple of 16: so is a last partial chunk
   const int nstages = (p.M + Cfg::CR - 1) / Cfg::CR;
   pdl_launch_dependents();
 
@@ -220,52 +231,88 @@ __global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_
       const uint64_t tk_desc = umma_desc(smem_u32(stk), 16, Cfg::SBO, Cfg::LAYOUT);
       const uint64_t tv_desc = umma_desc(smem_u32(stv), 16, Cfg::SBO, Cfg::LAYOUT);
       const uint64_t ty_desc = umma_desc(smem_u32(sty), 16, Cfg::SBO, Cfg::LAYOUT);
-      // a chunk as the K-major B operand of a score product (N = 16 latents)
-      // and as the MN-major B operand of a value product (N = D, one k-step
-      // of 16 latents); a chunk's descriptor adds its offset >> 4
+      // a chunk as the K-major B operand of a score product (N = C latents)
+      // and as the MN-major B operand of a value product (N = D, k-steps of
+      // 16 latents); a chunk's descriptor adds its offset >> 4
       const uint64_t r_desc = umma_desc(smem_u32(ring), 16, Cfg::SBO, Cfg::LAYOUT);
       constexpr uint64_t STAGE = Cfg::ST_B >> 4, HALF = (Cfg::C * Cfg::ROWB) >> 4;
       constexpr uint64_t OQ = Cfg::S_Q >> 4, OZH = Cfg::S_ZH >> 4, OZL = Cfg::S_ZL >> 4, ODH = Cfg::S_DH >> 4,
                          ODL = Cfg::S_DL >> 4;
-      auto chunk_desc = [&](int j) { return r_desc + ((j >> 1) % NST) * STAGE + (j & 1) * HALF; };
-      // the score products of chunk j into buffer j & 1
-      auto scores = [&](int j) -> bool {
-        const int sj = j >> 1;
-        if (!mbar_wait_mma(lat_full + sj % NST, (sj / NST) & 1, wc)) return false;
-        tc_fence_after();
-        const uint64_t rd = chunk_desc(j);
-        const uint32_t tb = tmem + (j & 1) * Cfg::BUF;
-        umma_ss(tb + Cfg::COL_S, tk_desc, rd + OQ, idesc_s, 0u);    // K Q_c^T
-        umma_ss(tb + Cfg::COL_DA, tv_desc, rd + ODH, idesc_s, 0u);  // V dZhi_c^T
-        umma_ss(tb + Cfg::COL_DA, tv_desc, rd + ODL, idesc_s, 1u);  // + V dZlo_c^T
-        if (FULL) {
-          umma_ss(tb + Cfg::COL_DP, ty_desc, rd + OZH, idesc_s, 0u);  // dY Zhi_c^T
-          umma_ss(tb + Cfg::COL_DP, ty_desc, rd + OZL, idesc_s, 1u);  // + dY Zlo_c^T
-        }
-        umma_commit(s_full + (j & 1));
-        return true;
-      };
-      bool ok = mbar_wait_mma(tok_full, 0, wc) && scores(0);
-      for (int j = 0; ok && j < nchunks; ++j) {
-        if (j + 1 < nchunks) {
-          if (j >= 1) {
-            // chunk j - 1's value MMAs are done: its buffer takes chunk j + 1,
-            // and once both chunks of a stage are done the stage is refilled
-            if (!mbar_wait_mma(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, wc)) { ok = false; break; }
-            if (((j - 1) & 1) && ((j - 1) >> 1) + NST < nstages) load_stage(((j - 1) >> 1) + NST);
+      constexpr int CPS = Cfg::CPS;
+      auto chunk_desc = [&](int j) { return r_desc + ((j / CPS) % NST) * STAGE + (j % CPS) * HALF; };
+      bool ok = mbar_wait_mma(tok_full, 0, wc);
+      if constexpr (Cfg::DB) {
+        // the score products of chunk j into buffer j & 1
+        auto scores = [&](int j) -> bool {
+          const int sj = j / CPS;
+          if (!mbar_wait_mma(lat_full + sj % NST, (sj / NST) & 1, wc)) return false;
+          tc_fence_after();
+          const uint64_t rd = chunk_desc(j);
+          const uint32_t tb = tmem + (j & 1) * Cfg::BUF;
+          umma_ss(tb + Cfg::COL_S, tk_desc, rd + OQ, idesc_s, 0u);    // K Q_c^T
+          umma_ss(tb + Cfg::COL_DA, tv_desc, rd + ODH, idesc_s, 0u);  // V dZhi_c^T
+          umma_ss(tb + Cfg::COL_DA, tv_desc, rd + ODL, idesc_s, 1u);  // + V dZlo_c^T
+          if (FULL) {
+            umma_ss(tb + Cfg::COL_DP, ty_desc, rd + OZH, idesc_s, 0u);  // dY Zhi_c^T
+            umma_ss(tb + Cfg::COL_DP, ty_desc, rd + OZL, idesc_s, 1u);  // + dY Zlo_c^T
           }
-          if (!scores(j + 1)) { ok = false; break; }
+          umma_commit(s_full + (j & 1));
+          return true;
+        };
+        ok = ok && scores(0);
+        for (int j = 0; ok && j < nchunks; ++j) {
+          if (j + 1 < nchunks) {
+            if (j >= 1) {
+              // chunk j - 1's value MMAs are done: its buffer takes chunk
+              // j + 1, and once every chunk of a stage is done the stage is
+              // refilled
+              if (!mbar_wait_mma(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, wc)) { ok = false; break; }
+              if ((j - 1) % CPS == CPS - 1 && (j - 1) / CPS + NST < nstages) load_stage((j - 1) / CPS + NST);
+            }
+            if (!scores(j + 1)) { ok = false; break; }
+          }
+          if (!mbar_wait_mma(p_full + (j & 1), (j >> 1) & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t rd = chunk_desc(j);
+          const uint32_t tb = tmem + (j & 1) * Cfg::BUF;
+          const uint32_t acc0 = j > 0 ? 1u : 0u;
+          umma_ts(tmem + Cfg::COL_DK, tb + Cfg::COL_S, rd + OQ, idesc_v, acc0);        // dShi Q_c
+          umma_ts(tmem + Cfg::COL_DK, tb + Cfg::COL_S + 8, rd + OQ, idesc_v, 1u);      // dSlo Q_c
+          umma_ts(tmem + Cfg::COL_DV, tb + Cfg::COL_DA, rd + ODH, idesc_v, acc0);      // A dZhi_c
+          umma_ts(tmem + Cfg::COL_DV, tb + Cfg::COL_DA, rd + ODL, idesc_v, 1u);        // A dZlo_c
+          umma_commit(pv_done + (j & 1));
         }
-        if (!mbar_wait_mma(p_full + (j & 1), (j >> 1) & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-        const uint64_t rd = chunk_desc(j);
-        const uint32_t tb = tmem + (j & 1) * Cfg::BUF;
-        const uint32_t acc0 = j > 0 ? 1u : 0u;
-        umma_ts(tmem + Cfg::COL_DK, tb + Cfg::COL_S, rd + OQ, idesc_v, acc0);        // dShi Q_c
-        umma_ts(tmem + Cfg::COL_DK, tb + Cfg::COL_S + 8, rd + OQ, idesc_v, 1u);      // dSlo Q_c
-        umma_ts(tmem + Cfg::COL_DV, tb + Cfg::COL_DA, rd + ODH, idesc_v, acc0);      // A dZhi_c
-        umma_ts(tmem + Cfg::COL_DV, tb + Cfg::COL_DA, rd + ODL, idesc_v, 1u);        // A dZlo_c
-        umma_commit(pv_done + (j & 1));
+      } else {
+        constexpr uint64_t KSTEP = (16 * Cfg::ROWB) >> 4;
+        for (int j = 0; ok && j < nchunks; ++j) {
+          const int st = j % NST;
+          const int cn = min(C, p.M - j * C);  // C, or a multiple of 16 for the last chunk
+          if (j > 0) {
+            // the value MMAs of chunk j - 1 are done: S and dA may be
+            // overwritten, and its ring stage takes chunk j - 1 + NST
+            if (!mbar_wait_mma(pv_done, (j - 1) & 1, wc)) { ok = false; break; }
+            if (j - 1 + NST < nstages) load_stage(j - 1 + NST);
+          }
+          if (!mbar_wait_mma(lat_full + st, (j / NST) & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t rd = chunk_desc(j);
+          const uint32_t idesc_c = idesc_bf16_f32(128, cn, false, false);
+          umma_ss(tmem + Cfg::COL_S, tk_desc, rd + OQ, idesc_c, 0u);    // K Q_c^T
+          umma_ss(tmem + Cfg::COL_DA, tv_desc, rd + ODH, idesc_c, 0u);  // V dZhi_c^T
+          umma_ss(tmem + Cfg::COL_DA, tv_desc, rd + ODL, idesc_c, 1u);  // + V dZlo_c^T
+          umma_commit(s_full);
+          if (!mbar_wait_mma(p_full, j & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+          for (int ks = 0; ks < cn / 16; ++ks) {
+            const uint32_t as = tmem + Cfg::COL_S + 16 * ks, aa = tmem + Cfg::COL_DA + 16 * ks;
+            const uint32_t acc0 = (j > 0 || ks > 0) ? 1u : 0u;
+            umma_ts(tmem + Cfg::COL_DK, as, rd + OQ + ks * KSTEP, idesc_v, acc0);       // dShi Q_c
+            umma_ts(tmem + Cfg::COL_DK, as + 8, rd + OQ + ks * KSTEP, idesc_v, 1u);     // dSlo Q_c
+            umma_ts(tmem + Cfg::COL_DV, aa, rd + ODH + ks * KSTEP, idesc_v, acc0);      // A dZhi_c
+            umma_ts(tmem + Cfg::COL_DV, aa, rd + ODL + ks * KSTEP, idesc_v, 1u);        // A dZlo_c
+          }
+          umma_commit(pv_done);
+        }
       }
       umma_commit(o_full);  // completes once every MMA issued above is done
       mbar_wait_drain(o_full, 0, p.timeout_ns);
@@ -324,30 +371,57 @@ __global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_
       }
     };
     bool ok = true;
-    for (int j = 0; j < nchunks; ++j) {
-      const int b = j & 1;
-      if (!mbar_wait_warp(s_full + b, (j >> 1) & 1, wc)) { ok = false; break; }
-      tc_fence_after();
-      const uint8_t* sb = ring + ((j >> 1) % NST) * Cfg::ST_B;
-      const float* lm = reinterpret_cast<const float*>(sb + Cfg::S_LM) + b * C;
-      const float* gm = reinterpret_cast<const float*>(sb + Cfg::S_GM) + b * C;
-      const uint32_t tb = lane_base + b * Cfg::BUF;
-      uint32_t sv[16], av[16], pv[16], hi[8], lo[8], wa[8];
-      tmem_ld16(tb + Cfg::COL_S, sv);
-      tmem_ld16(tb + Cfg::COL_DA, av);
-      if (FULL) tmem_ld16(tb + Cfg::COL_DP, pv);
-      tmem_wait_ld();
-      regs_defined16(sv);
-      regs_defined16(av);
-      if (FULL) regs_defined16(pv);
-      piece(sv, av, pv, lm, gm, hi, lo, wa);
-      tmem_st8(tb + Cfg::COL_S, hi);
-      tmem_st8(tb + Cfg::COL_S + 8, lo);
-      tmem_st8(tb + Cfg::COL_DA, wa);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive_warp(p_full + b);
-      __syncwarp();
+    if constexpr (Cfg::DB) {
+      for (int j = 0; j < nchunks; ++j) {
+        const int b = j & 1;
+        if (!mbar_wait_warp(s_full + b, (j >> 1) & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        const uint8_t* sb = ring + ((j / Cfg::CPS) % NST) * Cfg::ST_B;
+        const float* lm = reinterpret_cast<const float*>(sb + Cfg::S_LM) + (j % Cfg::CPS) * C;
+        const float* gm = reinterpret_cast<const float*>(sb + Cfg::S_GM) + (j % Cfg::CPS) * C;
+        const uint32_t tb = lane_base + b * Cfg::BUF;
+        uint32_t sv[16], av[16], pv[16], hi[8], lo[8], wa[8];
+        tmem_ld16(tb + Cfg::COL_S, sv);
+        tmem_ld16(tb + Cfg::COL_DA, av);
+        if (FULL) tmem_ld16(tb + Cfg::COL_DP, pv);
+        tmem_wait_ld();
+        regs_defined16(sv);
+        regs_defined16(av);
+        if (FULL) regs_defined16(pv);
+        piece(sv, av, pv, lm, gm, hi, lo, wa);
+        tmem_st8(tb + Cfg::COL_S, hi);
+        tmem_st8(tb + Cfg::COL_S + 8, lo);
+        tmem_st8(tb + Cfg::COL_DA, wa);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive_warp(p_full + b);
+        __syncwarp();
+      }
+    } else {
+      for (int j = 0; j < nchunks; ++j) {
+        if (!mbar_wait_warp(s_full, j & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        const int cn = min(C, p.M - j * C);
+        const uint8_t* sb = ring + (j % NST) * Cfg::ST_B;
+        const float* lm = reinterpret_cast<const float*>(sb + Cfg::S_LM);
+        const float* gm = reinterpret_cast<const float*>(sb + Cfg::S_GM);
+        for (int q = 0; q < cn / 16; ++q) {
+          uint32_t sv[16], av[16], pv[16], hi[8], lo[8], wa[8];
+          tmem_ld16(lane_base + Cfg::COL_S + 16 * q, sv);
+          tmem_ld16(lane_base + Cfg::COL_DA + 16 * q, av);
+          tmem_wait_ld();
+          regs_defined16(sv);
+          regs_defined16(av);
+          piece(sv, av, pv, lm + 16 * q, gm + 16 * q, hi, lo, wa);
+          tmem_st8(lane_base + Cfg::COL_S + 16 * q, hi);
+          tmem_st8(lane_base + Cfg::COL_S + 16 * q + 8, lo);
+          tmem_st8(lane_base + Cfg::COL_DA + 16 * q, wa);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive_warp(p_full);
+        __syncwarp();
+      }
     }
     if (ok && mbar_wait_warp(o_full, 0, wc)) {
       tc_fence_after();
