@@ -211,13 +211,13 @@ FLARE_API flare_status flarepp_mixer_fwd_inspect(const flare_bf16* X, const flar
  * those of the training pair on the same inputs bit for bit.  Outputs are
  * written (not accumulated).  Rows of dY for padding tokens are ignored;
  * padding tokens get zero gradients.  Same size limits as the forward, and
- * B*H <= 65535.  Arithmetic: at D = 16 the score and gradient products of
- * the four softmax passes, and at every D the projection gradients dX and
- * dW, on the tcgen05 tensor cores with each fp32 operand as the sum of two
- * bf16 parts (high and low) and fp32 accumulation; at D = 32 the softmax
- * passes' products with tf32 operands (bf16 inputs are exact in tf32);
- * softmax weights, normalisers and every reduction in fp32.  Deterministic
- * like the forward.
+ * B*H <= 65535.  Arithmetic: the score and gradient products of the four
+ * softmax passes and the projection gradients dX and dW on the tcgen05
+ * tensor cores, each fp32 operand as the sum of two bf16 parts (high and
+ * low), fp32 accumulation; softmax weights, normalisers and every reduction
+ * in fp32.  (The context-parallel phases below recompute the forward's state
+ * and run their softmax passes with tf32 tensor-core products; bf16 inputs
+ * are exact in tf32.)  Deterministic like the forward.
  *
  * flare_mixer_bwd (FLARE, eq. 5-6), workspace variant FLARE_VARIANT_FLARE_BWD:
  *   K, V, Q, lengths, scale   as in flare_mixer_fwd

@@ -70,17 +70,17 @@ BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C) {
     bp.off_g32 = take(static_cast<size_t>(B * N) * 4 * C * 4);
     bp.off_dwpart = take(static_cast<size_t>(bp.dw_splits) * C * 4 * C * 4);
   }
+  // the high and low bf16 parts of dZ (then of dQ(X)) and of Z for the
+  // tcgen05 passes of the training backward
+  bp.off_xhi16 = take(static_cast<size_t>(BH * M * D) * 2);
+  bp.off_xlo16 = take(static_cast<size_t>(BH * M * D) * 2);
+  bp.off_zhi16 = take(static_cast<size_t>(BH * M * D) * 2);
+  bp.off_zlo16 = take(static_cast<size_t>(BH * M * D) * 2);
   // the training pair at D = 16: the forward's fp16 copy of Z and its fp32 Y
   // (FLARE++: in the gradient rows' space, which the backward fills only
   // after it has taken delta_n from Y)
   if (D == 16) {
     bp.off_zf16 = take(static_cast<size_t>(BH * M * D) * 2);
-    // the high and low bf16 parts of dZ (then of dQ(X)) for the tcgen05 passes
-    bp.off_xhi16 = take(static_cast<size_t>(BH * M * D) * 2);
-    bp.off_xlo16 = take(static_cast<size_t>(BH * M * D) * 2);
-    // and of Z
-    bp.off_zhi16 = take(static_cast<size_t>(BH * M * D) * 2);
-    bp.off_zlo16 = take(static_cast<size_t>(BH * M * D) * 2);
     bp.off_y32 = pp ? bp.off_g32 : take(static_cast<size_t>(BH * N * D) * 4);
   }
   bp.total = off;
@@ -177,7 +177,7 @@ void exact_scores(LatParams& lp, float sc) {
 // The training backward's latent-parallel passes at D = 16 run on tcgen05
 // (lat_tc.cu) unless built with FLARE_LAT_TC=0 (the tf32 passes, kept for D = 32
 // and the self-contained backward).
-bool use_lat_tc(bool exact, int D) { return FLARE_LAT_TC && exact && D == 16; }
+bool use_lat_tc(bool exact, int D) { return FLARE_LAT_TC && exact && (D == 16 || D == 32); }
 
 // One tcgen05 latent-parallel pass: q16 bf16 queries ([G][M][D]), xa16 / xb16
 // the high and low parts of dZ (encoder) or Z (decoder), k16 / u16 the token
@@ -190,7 +190,7 @@ flare_status lat_tc(int mode, const BwdPlan& bp, uint8_t* ws, const void* q16, i
                     int D, const int32_t* lengths, float sc, cudaStream_t s) {
   const long BH = static_cast<long>(B) * H;
   const long G = q_per_batch ? BH : H;
-  const int qrows = std::min(M, kLatBlock), T = lat_tc_tile();
+  const int qrows = std::min(M, kLatBlock), T = lat_tc_tile(D);
   LatTcMaps mp;
   if (!map3d(&mp.q, q16, D, M, G, D, qrows, row_swizzle(D)) || !map3d(&mp.xa, xa16, D, M, BH, D, qrows, row_swizzle(D)) ||
       !map3d(&mp.xb, xb16, D, M, BH, D, qrows, row_swizzle(D)) || !map3d(&mp.k, k16, D, N, BH, D, T, row_swizzle(D)) ||
@@ -235,7 +235,7 @@ flare_status tok_tc(int mode, const BwdPlan& bp, uint8_t* ws, const void* k16, c
   const CUtensorMapSwizzle sw = row_swizzle(D);
   TokTcMaps mp;
   const bool full = mode == kTokTcFull;
-  const uint32_t ch = static_cast<uint32_t>(tok_tc_chunk(mode));
+  const uint32_t ch = static_cast<uint32_t>(tok_tc_chunk(mode, D));
   if (!map3d(&mp.k, k16, D, N, BH, D, kBwdTokBlock, sw) || !map3d(&mp.v, v16, D, N, BH, D, kBwdTokBlock, sw) ||
       !map3d(&mp.y, full ? dy16 : k16, D, N, BH, D, kBwdTokBlock, sw) || !map3d(&mp.q, q16, D, M, G, D, ch, sw) ||
       !map3d(&mp.zh, ws + bp.off_zhi16, D, M, BH, D, ch, sw) || !map3d(&mp.zl, ws + bp.off_zlo16, D, M, BH, D, ch, sw) ||

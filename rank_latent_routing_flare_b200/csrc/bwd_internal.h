@@ -178,8 +178,8 @@ struct LatTcMaps {
   CUtensorMap q, xa, xb, k, u, l, d;
 };
 cudaError_t launch_lat_tc(int mode, const LatTcMaps& m, const LatTcParams& p, cudaStream_t s);
-size_t lat_tc_smem_bytes();
-int lat_tc_tile();
+size_t lat_tc_smem_bytes(int D);
+int lat_tc_tile(int D);  // tokens per tile (the token maps' box rows)
 // Token-parallel backward passes on tcgen05 (tok_tc.cu; D = 16, bf16
 // queries, exact scores): dK and dV rows of 128-token tiles, the decoder and
 // encoder parts (kTokTcFull) or the encoder part alone (kTokTcEncoder: the
@@ -207,8 +207,8 @@ struct TokTcMaps {
   CUtensorMap k, v, y, q, zh, zl, dh, dl, lm, gm;
 };
 cudaError_t launch_tok_tc(int mode, const TokTcMaps& m, const TokTcParams& p, cudaStream_t s);
-size_t tok_tc_smem_bytes(int mode);
-int tok_tc_chunk(int mode);  // latents per chunk (the latent tensor maps' box rows)
+size_t tok_tc_smem_bytes(int mode, int D);
+int tok_tc_chunk(int mode, int D);  // latents per ring stage (the latent tensor maps' box rows)
 
 // hi[i] = bf16(x[i]), lo[i] = bf16(x[i] - hi[i]) for i < n (n even)
 struct SplitHiLoParams {

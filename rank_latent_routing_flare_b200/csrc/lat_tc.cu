@@ -1,4 +1,4 @@
-// Latent-parallel backward passes on tcgen05 (D = 16): the gradients of the
+// Latent-parallel backward passes on tcgen05 (D = 16 or 32): the gradients of the
 // encoder softmax with respect to its queries (FLARE++ paper, eq. 8 and 10;
 // FLARE paper, eq. 5) and of the decoder softmax with respect to its queries
 // and latent values (eq. 11; eq. 6), for the training backward, whose
@@ -20,9 +20,10 @@
 // score scale c = scale log2(e) is applied to the fp32 product, as in the
 // forward's kernels, so that the forward's normalisers L_m fit these scores.
 //
-// Tiles of T = 48 tokens stream through a TMA ring (K and V, or K and dY,
-// plus L_n and delta_n for the decoder).  TMEM: S at column 0, G at 48, dQ at
-// 96, dZ at 112 (128 columns: four CTAs per SM).  The softmax threads read a
+// Tiles of T = 48 tokens (32 at D = 32) stream through a TMA ring (K and V,
+// or K and dY, plus L_n and delta_n for the decoder).  TMEM: S at column 0,
+// G at T, dQ at 2T, dZ at 2T + D (128 columns: four CTAs per SM).  The score
+// products take K = D in k-steps of 16.  The softmax threads read a
 // tile's S and G in three 16-column pieces (the next piece's TMEM load in
 // flight while the current one is computed) and write, over the piece they
 // have read, dS as bf16 high and low parts (S columns [16j, 16j+8) and
@@ -49,15 +50,16 @@ __device__ __forceinline__ void regs_defined(uint32_t (&r)[16]) {
                  "+r"(r[15]));
 }
 
+template <int D_>
 struct LatTcCfg {
-  static constexpr int D = 16;
-  static constexpr int T = 48;                          // tokens per tile
+  static constexpr int D = D_;
+  static constexpr int T = D == 16 ? 48 : 32;           // tokens per tile
   static constexpr int ROWB = D * 2;                    // bytes of one bf16 row
   static constexpr int TILE_B = T * ROWB;               // one K, V or dY tile
   static constexpr int ROWS_B = kLatBlock * ROWB;       // Q, or one part of dZ / Z
   static constexpr int LD_B = 256;                      // one tile's L_n or delta_n (T floats, padded)
   static constexpr int NST = 6;                         // ring stages
-  static constexpr uint32_t LAYOUT = LAYOUT_SW32;
+  static constexpr uint32_t LAYOUT = D == 16 ? LAYOUT_SW32 : LAYOUT_SW64;
   static constexpr uint32_t SBO = 8 * ROWB;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_XA = OFF_Q + ROWS_B;         // dZhi (encoder) or Zhi (decoder)
@@ -73,17 +75,17 @@ struct LatTcCfg {
   static constexpr int THREADS = 160;
   static constexpr int CTAS_PER_SM = 4;
   static_assert(COL_DZ + D <= TMEM_COLS, "TMEM columns");
-  static_assert(TILE_B % 256 == 0 && ROWS_B % 1024 == 0, "tiles must hold whole swizzle atoms");
+  static_assert(TILE_B % (8 * ROWB) == 0 && ROWS_B % 1024 == 0, "tiles must hold whole swizzle atoms");
   static_assert(T % 16 == 0 && T * 4 <= LD_B, "tile of L_n / delta_n");
 };
 
-template <int MODE>
-__global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
+template <int MODE, int DD>
+__global__ void __launch_bounds__(LatTcCfg<DD>::THREADS, LatTcCfg<DD>::CTAS_PER_SM)
     lat_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_xa,
                   const __grid_constant__ CUtensorMap tm_xb, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_l,
                   const __grid_constant__ CUtensorMap tm_d, const LatTcParams p) {
-  using Cfg = LatTcCfg;
+  using Cfg = LatTcCfg<DD>;
   constexpr int D = Cfg::D, T = Cfg::T, NST = Cfg::NST;
   constexpr bool DEC = MODE == kLatTcDecoder;
   extern __shared__ uint8_t smem_raw[];
@@ -207,9 +209,13 @@ __global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
         if (!mbar_wait_mma(kv_full + st, (i / NST) & 1, wc)) { ok = false; break; }
         tc_fence_after();
         const uint64_t kd = k_desc + st * STAGE, ud = u_desc + st * STAGE;
-        umma_ss(tmem + Cfg::COL_S, q_desc, kd, idesc_s, 0u);
-        umma_ss(tmem + Cfg::COL_G, xa_desc, ud, idesc_s, 0u);
-        umma_ss(tmem + Cfg::COL_G, xb_desc, ud, idesc_s, 1u);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {  // k-steps of 16 along D: 32 bytes inside the row
+          const uint64_t ko = 2 * kk;
+          umma_ss(tmem + Cfg::COL_S, q_desc + ko, kd + ko, idesc_s, kk > 0 ? 1u : 0u);
+          umma_ss(tmem + Cfg::COL_G, xa_desc + ko, ud + ko, idesc_s, kk > 0 ? 1u : 0u);
+          umma_ss(tmem + Cfg::COL_G, xb_desc + ko, ud + ko, idesc_s, 1u);
+        }
         umma_commit(s_full);
         if (!mbar_wait_mma(p_full, i & 1, wc)) { ok = false; break; }
         tc_fence_after();
@@ -334,9 +340,9 @@ __global__ void __launch_bounds__(LatTcCfg::THREADS, LatTcCfg::CTAS_PER_SM)
     if (ok && mbar_wait_warp(o_full, 0, wc)) {
       tc_fence_after();
       if (warp_live) {
-        uint32_t dq[16], dz[16];
-        tmem_ld16(lane_base + Cfg::COL_DQ, dq);
-        if (DEC) tmem_ld16(lane_base + Cfg::COL_DZ, dz);
+        uint32_t dq[D], dz[D];
+        tmem_ld_cols<D>(lane_base + Cfg::COL_DQ, dq);
+        if (DEC) tmem_ld_cols<D>(lane_base + Cfg::COL_DZ, dz);
         tmem_wait_ld();
         if (row_ok) {
           float4* oq = reinterpret_cast<float4*>(p.part_q + (part_row0 + m) * D);
@@ -385,28 +391,30 @@ cudaError_t launch_split_hilo(const SplitHiLoParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-size_t lat_tc_smem_bytes() {
-  const size_t need = LatTcCfg::BYTES + 1024;
+size_t lat_tc_smem_bytes(int D) {
+  const size_t need = (D == 16 ? LatTcCfg<16>::BYTES : LatTcCfg<32>::BYTES) + 1024;
   // at most CTAS_PER_SM CTAs per SM (228 KB each, 1 KB of it reserved per
   // CTA), so that every resident CTA finds its TMEM columns free
-  const size_t floor = (228 * 1024) / (LatTcCfg::CTAS_PER_SM + 1) + 1024;
+  const size_t floor = (228 * 1024) / (LatTcCfg<16>::CTAS_PER_SM + 1) + 1024;
   return need > floor ? need : floor;
 }
 
-int lat_tc_tile() { return LatTcCfg::T; }
+int lat_tc_tile(int D) { return D == 16 ? LatTcCfg<16>::T : LatTcCfg<32>::T; }
 
 cudaError_t launch_lat_tc(int mode, const LatTcMaps& m, const LatTcParams& p, cudaStream_t s) {
-  if (p.D != 16) return cudaErrorInvalidValue;
-  const size_t smem = lat_tc_smem_bytes();
+  if (p.D != 16 && p.D != 32) return cudaErrorInvalidValue;
+  const size_t smem = lat_tc_smem_bytes(p.D);
   const dim3 grid(static_cast<unsigned>(p.B * p.H * p.n_lblocks * p.n_splits));
   auto go = [&](auto kern) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid, LatTcCfg::THREADS, smem, s>>>(m.q, m.xa, m.xb, m.k, m.u, mode == kLatTcDecoder ? m.l : m.k,
-                                               mode == kLatTcDecoder ? m.d : m.k, p);
+    kern<<<grid, LatTcCfg<16>::THREADS, smem, s>>>(m.q, m.xa, m.xb, m.k, m.u, mode == kLatTcDecoder ? m.l : m.k,
+                                                   mode == kLatTcDecoder ? m.d : m.k, p);
     return cudaGetLastError();
   };
-  return mode == kLatTcDecoder ? go(lat_tc_kernel<kLatTcDecoder>) : go(lat_tc_kernel<kLatTcEncoder>);
+  if (p.D == 16)
+    return mode == kLatTcDecoder ? go(lat_tc_kernel<kLatTcDecoder, 16>) : go(lat_tc_kernel<kLatTcEncoder, 16>);
+  return mode == kLatTcDecoder ? go(lat_tc_kernel<kLatTcDecoder, 32>) : go(lat_tc_kernel<kLatTcEncoder, 32>);
 }
 
 }  // namespace flare

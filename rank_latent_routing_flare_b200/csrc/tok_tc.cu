@@ -1,9 +1,9 @@
-// Token-parallel backward passes on tcgen05 (D = 16): the gradients of the
+// Token-parallel backward passes on tcgen05 (D = 16 or 32): the gradients of the
 // key and value rows for the training backward, whose queries are bf16
 // values (Q(X), Q0 or the learned Q) so that the score products are exact.
 // One CTA owns a tile of 128 tokens of one head (thread <-> TMEM lane <->
 // token) and walks the latents in chunks of C = 16 (full) or 48 (encoder
-// only):
+// only; 32 at D = 32):
 //
 //   full (kTokTcFull: decoder and encoder, FLARE++ paper eq. 10-11; FLARE
 //   paper eq. 5-6), per chunk:
@@ -22,8 +22,9 @@
 // The token tile's K, V and dY stay in shared memory; the latents (Q, the
 // parts of Z and dZ, L_m and gamma_m) stream through a TMA ring (stages of 32
 // latents, two chunks, in the full pass; of one 48-latent chunk in the
-// encoder-only one).  The dK, dV accumulators sit at TMEM columns 96 and 112
-// (128 columns: four CTAs per SM).  Full pass: two score buffers (S, dA, dP:
+// encoder-only one).  The dK, dV accumulators sit at TMEM columns 128 - 2D
+// and 128 - D (128 columns: four CTAs per SM).  Full pass at D = 16: two
+// score buffers (S, dA, dP:
 // 16 columns each); the MMA thread issues chunk j + 1's score products into
 // the other buffer before it waits for the softmax threads to finish chunk
 // j, so the score products of one chunk overlap the softmax of the previous
@@ -32,7 +33,10 @@
 // 48), read in 16-column pieces, the next chunk's products issued once the
 // value products of the previous one are done (with half the work per
 // score, two buffers of 16-latent chunks measured slower: 3.64 against 3.36
-// ms).  The softmax threads write, over each 16-column piece they have read,
+// ms).  At D = 32 the accumulators take 64 columns, which leaves room for
+// one score buffer: 16-latent chunks for the full pass, 32 for the encoder
+// only.  The score products take K = D in k-steps of 16.  The softmax
+// threads write, over each 16-column piece they have read,
 // dS as bf16 high and low parts (S columns [0, 8) and [8, 16) of the piece)
 // and A in bf16 (dA columns [0, 8)); the value MMAs take them as TMEM A
 // operands, one 16-latent k-step per piece.
@@ -52,13 +56,13 @@ __device__ __forceinline__ void regs_defined16(uint32_t (&r)[16]) {
                  "+r"(r[15]));
 }
 
-template <int MODE>
+template <int MODE, int D_>
 struct TokTcCfg {
   static constexpr bool FULL = MODE == kTokTcFull;
-  static constexpr int D = 16;
-  static constexpr bool DB = FULL;                      // two score buffers
-  static constexpr int C = FULL ? 16 : 48;              // latents per chunk
-  static constexpr int CR = FULL ? 2 * C : C;           // latents per ring stage
+  static constexpr int D = D_;
+  static constexpr bool DB = FULL && D == 16;           // two score buffers
+  static constexpr int C = FULL ? 16 : (D == 16 ? 48 : 32);  // latents per chunk
+  static constexpr int CR = DB ? 2 * C : C;             // latents per ring stage
   static constexpr int CPS = CR / C;                    // chunks per ring stage
   static constexpr int TT = kBwdTokBlock;               // tokens per CTA (128)
   static constexpr int ROWB = D * 2;
@@ -66,8 +70,8 @@ struct TokTcCfg {
   static constexpr int CH_B = CR * ROWB;                // a stage's rows of Q, Zhi, Zlo, dZhi or dZlo
   static constexpr int NCH = FULL ? 5 : 3;              // latent tensors per ring stage
   static constexpr int ST_B = NCH * CH_B + 2 * 256;     // a ring stage: the tensors, L_m, gamma_m
-  static constexpr int NST = 6;
-  static constexpr uint32_t LAYOUT = LAYOUT_SW32;
+  static constexpr int NST = D == 16 ? 6 : 4;
+  static constexpr uint32_t LAYOUT = D == 16 ? LAYOUT_SW32 : LAYOUT_SW64;
   static constexpr uint32_t SBO = 8 * ROWB;
   static constexpr int OFF_TK = 0, OFF_TV = TOK_B, OFF_TY = 2 * TOK_B;
   static constexpr int OFF_RING = (FULL ? 3 : 2) * TOK_B;
@@ -80,25 +84,25 @@ struct TokTcCfg {
   // one score buffer: S, dA (and dP) of a chunk
   static constexpr uint32_t BUF = FULL ? 3 * C : 2 * C;
   static constexpr int NBUF = DB ? 2 : 1;
-  static constexpr uint32_t COL_S = 0, COL_DA = C, COL_DP = 2 * C, COL_DK = 96, COL_DV = 96 + D;
+  static constexpr uint32_t COL_S = 0, COL_DA = C, COL_DP = 2 * C, COL_DK = 128 - 2 * D, COL_DV = 128 - D;
   static constexpr uint32_t TMEM_COLS = 128;
   static constexpr int THREADS = 160;
   static constexpr int CTAS_PER_SM = 4;
   static_assert(COL_DV + D <= TMEM_COLS && NBUF * BUF <= COL_DK, "TMEM columns");
-  static_assert(TOK_B % 1024 == 0 && CH_B % 256 == 0 && ST_B % 256 == 0 && (C * ROWB) % 256 == 0,
+  static_assert(TOK_B % 1024 == 0 && CH_B % (8 * ROWB) == 0 && ST_B % 256 == 0 && (C * ROWB) % (8 * ROWB) == 0,
                 "tiles and chunks must hold whole swizzle atoms");
   static_assert(CR * 4 <= 256, "L_m / gamma_m of a stage");
 };
 
-template <int MODE>
-__global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_PER_SM)
+template <int MODE, int DD>
+__global__ void __launch_bounds__(TokTcCfg<MODE, DD>::THREADS, TokTcCfg<MODE, DD>::CTAS_PER_SM)
     tok_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_zh, const __grid_constant__ CUtensorMap tm_zl,
                   const __grid_constant__ CUtensorMap tm_dh, const __grid_constant__ CUtensorMap tm_dl,
                   const __grid_constant__ CUtensorMap tm_lm, const __grid_constant__ CUtensorMap tm_gm,
                   const TokTcParams p) {
-  using Cfg = TokTcCfg<MODE>;
+  using Cfg = TokTcCfg<MODE, DD>;
   constexpr int D = Cfg::D, C = Cfg::C, NST = Cfg::NST;
   constexpr bool FULL = MODE == kTokTcFull;
   extern __shared__ uint8_t smem_raw[];
@@ -239,6 +243,23 @@ __global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_
       constexpr uint64_t OQ = Cfg::S_Q >> 4, OZH = Cfg::S_ZH >> 4, OZL = Cfg::S_ZL >> 4, ODH = Cfg::S_DH >> 4,
                          ODL = Cfg::S_DL >> 4;
       constexpr int CPS = Cfg::CPS;
+      // S = K Q_c^T, dA = V dZ_c^T (two parts) and, full, dP = dY Z_c^T (two
+      // parts) into the buffer at tb; K = D in k-steps of 16 (32 bytes inside
+      // the rows)
+      auto score_products = [&](uint32_t tb, uint64_t rd, uint32_t idesc) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ko = 2 * kk;
+          const uint32_t a0 = kk > 0 ? 1u : 0u;
+          umma_ss(tb + Cfg::COL_S, tk_desc + ko, rd + OQ + ko, idesc, a0);
+          umma_ss(tb + Cfg::COL_DA, tv_desc + ko, rd + ODH + ko, idesc, a0);
+          umma_ss(tb + Cfg::COL_DA, tv_desc + ko, rd + ODL + ko, idesc, 1u);
+          if (FULL) {
+            umma_ss(tb + Cfg::COL_DP, ty_desc + ko, rd + OZH + ko, idesc, a0);
+            umma_ss(tb + Cfg::COL_DP, ty_desc + ko, rd + OZL + ko, idesc, 1u);
+          }
+        }
+      };
       auto chunk_desc = [&](int j) { return r_desc + ((j / CPS) % NST) * STAGE + (j % CPS) * HALF; };
       bool ok = mbar_wait_mma(tok_full, 0, wc);
       if constexpr (Cfg::DB) {
@@ -249,13 +270,7 @@ __global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_
           tc_fence_after();
           const uint64_t rd = chunk_desc(j);
           const uint32_t tb = tmem + (j & 1) * Cfg::BUF;
-          umma_ss(tb + Cfg::COL_S, tk_desc, rd + OQ, idesc_s, 0u);    // K Q_c^T
-          umma_ss(tb + Cfg::COL_DA, tv_desc, rd + ODH, idesc_s, 0u);  // V dZhi_c^T
-          umma_ss(tb + Cfg::COL_DA, tv_desc, rd + ODL, idesc_s, 1u);  // + V dZlo_c^T
-          if (FULL) {
-            umma_ss(tb + Cfg::COL_DP, ty_desc, rd + OZH, idesc_s, 0u);  // dY Zhi_c^T
-            umma_ss(tb + Cfg::COL_DP, ty_desc, rd + OZL, idesc_s, 1u);  // + dY Zlo_c^T
-          }
+          score_products(tb, rd, idesc_s);
           umma_commit(s_full + (j & 1));
           return true;
         };
@@ -297,9 +312,7 @@ __global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_
           tc_fence_after();
           const uint64_t rd = chunk_desc(j);
           const uint32_t idesc_c = idesc_bf16_f32(128, cn, false, false);
-          umma_ss(tmem + Cfg::COL_S, tk_desc, rd + OQ, idesc_c, 0u);    // K Q_c^T
-          umma_ss(tmem + Cfg::COL_DA, tv_desc, rd + ODH, idesc_c, 0u);  // V dZhi_c^T
-          umma_ss(tmem + Cfg::COL_DA, tv_desc, rd + ODL, idesc_c, 1u);  // + V dZlo_c^T
+          score_products(tmem, rd, idesc_c);
           umma_commit(s_full);
           if (!mbar_wait_mma(p_full, j & 1, wc)) { ok = false; break; }
           tc_fence_after();
@@ -409,9 +422,11 @@ __global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_
           uint32_t sv[16], av[16], pv[16], hi[8], lo[8], wa[8];
           tmem_ld16(lane_base + Cfg::COL_S + 16 * q, sv);
           tmem_ld16(lane_base + Cfg::COL_DA + 16 * q, av);
+          if (FULL) tmem_ld16(lane_base + Cfg::COL_DP + 16 * q, pv);
           tmem_wait_ld();
           regs_defined16(sv);
           regs_defined16(av);
+          if (FULL) regs_defined16(pv);
           piece(sv, av, pv, lm + 16 * q, gm + 16 * q, hi, lo, wa);
           tmem_st8(lane_base + Cfg::COL_S + 16 * q, hi);
           tmem_st8(lane_base + Cfg::COL_S + 16 * q + 8, lo);
@@ -425,9 +440,9 @@ __global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_
     }
     if (ok && mbar_wait_warp(o_full, 0, wc)) {
       tc_fence_after();
-      uint32_t kv[16], vv[16];
-      tmem_ld16(lane_base + Cfg::COL_DK, kv);
-      tmem_ld16(lane_base + Cfg::COL_DV, vv);
+      uint32_t kv[D], vv[D];
+      tmem_ld_cols<D>(lane_base + Cfg::COL_DK, kv);
+      tmem_ld_cols<D>(lane_base + Cfg::COL_DV, vv);
       tmem_wait_ld();
       if (n < p.N) {
         float dk[D], dv[D];
@@ -456,29 +471,40 @@ __global__ void __launch_bounds__(TokTcCfg<MODE>::THREADS, TokTcCfg<MODE>::CTAS_
 
 }  // namespace
 
-size_t tok_tc_smem_bytes(int mode) {
-  const size_t need = (mode == kTokTcFull ? TokTcCfg<kTokTcFull>::BYTES : TokTcCfg<kTokTcEncoder>::BYTES) + 1024;
+template <int MODE, int D>
+size_t tok_tc_smem() {
+  const size_t need = TokTcCfg<MODE, D>::BYTES + 1024;
   // at most CTAS_PER_SM CTAs per SM (228 KB each, 1 KB of it reserved per
   // CTA), so that every resident CTA finds its TMEM columns free
-  const size_t floor = (228 * 1024) / (TokTcCfg<kTokTcFull>::CTAS_PER_SM + 1) + 1024;
+  const size_t floor = (228 * 1024) / (TokTcCfg<MODE, D>::CTAS_PER_SM + 1) + 1024;
   return need > floor ? need : floor;
 }
 
-int tok_tc_chunk(int mode) { return mode == kTokTcFull ? TokTcCfg<kTokTcFull>::CR : TokTcCfg<kTokTcEncoder>::CR; }
+size_t tok_tc_smem_bytes(int mode, int D) {
+  if (D == 16) return mode == kTokTcFull ? tok_tc_smem<kTokTcFull, 16>() : tok_tc_smem<kTokTcEncoder, 16>();
+  return mode == kTokTcFull ? tok_tc_smem<kTokTcFull, 32>() : tok_tc_smem<kTokTcEncoder, 32>();
+}
+
+int tok_tc_chunk(int mode, int D) {
+  if (D == 16) return mode == kTokTcFull ? TokTcCfg<kTokTcFull, 16>::CR : TokTcCfg<kTokTcEncoder, 16>::CR;
+  return mode == kTokTcFull ? TokTcCfg<kTokTcFull, 32>::CR : TokTcCfg<kTokTcEncoder, 32>::CR;
+}
 
 cudaError_t launch_tok_tc(int mode, const TokTcMaps& m, const TokTcParams& p, cudaStream_t s) {
-  if (p.D != 16) return cudaErrorInvalidValue;
-  const size_t smem = tok_tc_smem_bytes(mode);
+  if (p.D != 16 && p.D != 32) return cudaErrorInvalidValue;
+  const size_t smem = tok_tc_smem_bytes(mode, p.D);
   const int tiles = (p.N + kBwdTokBlock - 1) / kBwdTokBlock;
   const dim3 grid(static_cast<unsigned>(static_cast<long>(p.B) * p.H * tiles));
-  auto go = [&](auto kern, int threads) {
+  auto go = [&](auto kern) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid, threads, smem, s>>>(m.k, m.v, m.y, m.q, m.zh, m.zl, m.dh, m.dl, m.lm, m.gm, p);
+    kern<<<grid, TokTcCfg<kTokTcFull, 16>::THREADS, smem, s>>>(m.k, m.v, m.y, m.q, m.zh, m.zl, m.dh, m.dl, m.lm,
+                                                               m.gm, p);
     return cudaGetLastError();
   };
-  return mode == kTokTcFull ? go(tok_tc_kernel<kTokTcFull>, TokTcCfg<kTokTcFull>::THREADS)
-                            : go(tok_tc_kernel<kTokTcEncoder>, TokTcCfg<kTokTcEncoder>::THREADS);
+  if (p.D == 16)
+    return mode == kTokTcFull ? go(tok_tc_kernel<kTokTcFull, 16>) : go(tok_tc_kernel<kTokTcEncoder, 16>);
+  return mode == kTokTcFull ? go(tok_tc_kernel<kTokTcFull, 32>) : go(tok_tc_kernel<kTokTcEncoder, 32>);
 }
 
 }  // namespace flare
