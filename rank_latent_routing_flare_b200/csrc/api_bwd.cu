@@ -190,7 +190,7 @@ flare_status lat_tc(int mode, const BwdPlan& bp, uint8_t* ws, const void* q16, i
                     int D, const int32_t* lengths, float sc, cudaStream_t s) {
   const long BH = static_cast<long>(B) * H;
   const long G = q_per_batch ? BH : H;
-  const int qrows = std::min(M, kLatBlock), T = lat_tc_tile(mode, D);
+  const int qrows = std::min(M, kLatBlock), T = lat_tc_tile(D);
   LatTcMaps mp;
   if (!map3d(&mp.q, q16, D, M, G, D, qrows, row_swizzle(D)) || !map3d(&mp.xa, xa16, D, M, BH, D, qrows, row_swizzle(D)) ||
       !map3d(&mp.xb, xb16, D, M, BH, D, qrows, row_swizzle(D)) || !map3d(&mp.k, k16, D, N, BH, D, T, row_swizzle(D)) ||

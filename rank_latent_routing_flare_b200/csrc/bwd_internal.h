@@ -178,8 +178,8 @@ struct LatTcMaps {
   CUtensorMap q, xa, xb, k, u, l, d;
 };
 cudaError_t launch_lat_tc(int mode, const LatTcMaps& m, const LatTcParams& p, cudaStream_t s);
-size_t lat_tc_smem_bytes(int mode, int D);
-int lat_tc_tile(int mode, int D);  // tokens per tile (the token maps' box rows)
+size_t lat_tc_smem_bytes(int D);
+int lat_tc_tile(int D);  // tokens per tile (the token maps' box rows)
 // Token-parallel backward passes on tcgen05 (tok_tc.cu; D = 16, bf16
 // queries, exact scores): dK and dV rows of 128-token tiles, the decoder and
 // encoder parts (kTokTcFull) or the encoder part alone (kTokTcEncoder: the

@@ -50,14 +50,10 @@ __device__ __forceinline__ void regs_defined(uint32_t (&r)[16]) {
                  "+r"(r[15]));
 }
 
-template <int MODE, int D_>
+template <int D_>
 struct LatTcCfg {
   static constexpr int D = D_;
-  // encoder: dS in columns of its own, so that the next tile's S and G can
-  // be issued right behind the value MMAs (which read dS), without waiting
-  // for them to complete
-  static constexpr bool SEP = MODE == kLatTcEncoder;
-  static constexpr int T = (SEP || D == 32) ? 32 : 48;  // tokens per tile
+  static constexpr int T = D == 16 ? 48 : 32;           // tokens per tile
   static constexpr int ROWB = D * 2;                    // bytes of one bf16 row
   static constexpr int TILE_B = T * ROWB;               // one K, V or dY tile
   static constexpr int ROWS_B = kLatBlock * ROWB;       // Q, or one part of dZ / Z
@@ -74,23 +70,22 @@ struct LatTcCfg {
   static constexpr int OFF_BAR = OFF_LD + NST * 2 * LD_B;
   static constexpr int OFF_MISC = OFF_BAR + 8 * (6 + NST);
   static constexpr int BYTES = OFF_MISC + 64 + NST * 4;
-  static constexpr uint32_t COL_S = 0, COL_G = T, COL_DS = SEP ? 2 * T : 0, COL_DQ = SEP ? 3 * T : 2 * T,
-                            COL_DZ = 2 * T + D;
+  static constexpr uint32_t COL_S = 0, COL_G = T, COL_DQ = 2 * T, COL_DZ = 2 * T + D;
   static constexpr uint32_t TMEM_COLS = 128;
   static constexpr int THREADS = 160;
   static constexpr int CTAS_PER_SM = 4;
-  static_assert(COL_DQ + D <= TMEM_COLS && (SEP || COL_DZ + D <= TMEM_COLS), "TMEM columns");
+  static_assert(COL_DZ + D <= TMEM_COLS, "TMEM columns");
   static_assert(TILE_B % (8 * ROWB) == 0 && ROWS_B % 1024 == 0, "tiles must hold whole swizzle atoms");
   static_assert(T % 16 == 0 && T * 4 <= LD_B, "tile of L_n / delta_n");
 };
 
 template <int MODE, int DD>
-__global__ void __launch_bounds__(LatTcCfg<MODE, DD>::THREADS, LatTcCfg<MODE, DD>::CTAS_PER_SM)
+__global__ void __launch_bounds__(LatTcCfg<DD>::THREADS, LatTcCfg<DD>::CTAS_PER_SM)
     lat_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_xa,
                   const __grid_constant__ CUtensorMap tm_xb, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_l,
                   const __grid_constant__ CUtensorMap tm_d, const LatTcParams p) {
-  using Cfg = LatTcCfg<MODE, DD>;
+  using Cfg = LatTcCfg<DD>;
   constexpr int D = Cfg::D, T = Cfg::T, NST = Cfg::NST;
   constexpr bool DEC = MODE == kLatTcDecoder;
   extern __shared__ uint8_t smem_raw[];
@@ -202,30 +197,31 @@ __global__ void __launch_bounds__(LatTcCfg<MODE, DD>::THREADS, LatTcCfg<MODE, DD
       const uint64_t k_desc = umma_desc(smem_u32(sk), 16, Cfg::SBO, Cfg::LAYOUT);
       const uint64_t u_desc = umma_desc(smem_u32(su), 16, Cfg::SBO, Cfg::LAYOUT);
       constexpr uint64_t STAGE = Cfg::TILE_B >> 4, KSTEP = (16 * Cfg::ROWB) >> 4;
-      // S = Q K_i^T and G = X U_i^T (two parts) of tile i; K = D in k-steps
-      // of 16 (32 bytes inside the rows)
-      auto scores = [&](int i) -> bool {
+      bool ok = mbar_wait_mma(q_full, 0, wc);
+      for (int i = 0; ok && i < ntiles; ++i) {
         const int st = i % NST;
-        if (!mbar_wait_mma(kv_full + st, (i / NST) & 1, wc)) return false;
+        if (i > 0) {
+          // the value MMAs of tile i - 1 are done: S and G may be overwritten,
+          // and tile i - 1's stage takes tile i - 1 + NST
+          if (!mbar_wait_mma(pv_done, (i - 1) & 1, wc)) { ok = false; break; }
+          if (i - 1 + NST < ntiles) load_tile(i - 1 + NST);
+        }
+        if (!mbar_wait_mma(kv_full + st, (i / NST) & 1, wc)) { ok = false; break; }
         tc_fence_after();
         const uint64_t kd = k_desc + st * STAGE, ud = u_desc + st * STAGE;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {  // k-steps of 16 along D: 32 bytes inside the row
           const uint64_t ko = 2 * kk;
           umma_ss(tmem + Cfg::COL_S, q_desc + ko, kd + ko, idesc_s, kk > 0 ? 1u : 0u);
           umma_ss(tmem + Cfg::COL_G, xa_desc + ko, ud + ko, idesc_s, kk > 0 ? 1u : 0u);
           umma_ss(tmem + Cfg::COL_G, xb_desc + ko, ud + ko, idesc_s, 1u);
         }
         umma_commit(s_full);
-        return true;
-      };
-      // dQ += dS K_i (two parts of dS) and, decoder, dZ += W U_i
-      auto values = [&](int i) {
-        const int st = i % NST;
-        const uint64_t kd = k_desc + st * STAGE, ud = u_desc + st * STAGE;
+        if (!mbar_wait_mma(p_full, i & 1, wc)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < T / 16; ++ks) {
-          const uint32_t a = tmem + Cfg::COL_DS + 16 * ks;
+          const uint32_t a = tmem + Cfg::COL_S + 16 * ks;
           umma_ts(tmem + Cfg::COL_DQ, a, kd + ks * KSTEP, idesc_v, (i > 0 || ks > 0) ? 1u : 0u);  // dShi K
           umma_ts(tmem + Cfg::COL_DQ, a + 8, kd + ks * KSTEP, idesc_v, 1u);                      // dSlo K
           if (DEC)
@@ -233,37 +229,6 @@ __global__ void __launch_bounds__(LatTcCfg<MODE, DD>::THREADS, LatTcCfg<MODE, DD
                     (i > 0 || ks > 0) ? 1u : 0u);                                                // W dY
         }
         umma_commit(pv_done);
-      };
-      bool ok = mbar_wait_mma(q_full, 0, wc);
-      if constexpr (Cfg::SEP) {
-        // the next tile's S and G go right behind this tile's value MMAs:
-        // they overwrite only columns the softmax threads have read, and
-        // their completion (s_full) implies the value MMAs' (in issue order),
-        // so dS may be rewritten once s_full is seen
-        ok = ok && scores(0);
-        for (int i = 0; ok && i < ntiles; ++i) {
-          if (i > 0) {  // tile i - 1's value MMAs are done: its stage takes tile i - 1 + NST
-            if (!mbar_wait_mma(pv_done, (i - 1) & 1, wc)) { ok = false; break; }
-            if (i - 1 + NST < ntiles) load_tile(i - 1 + NST);
-          }
-          if (!mbar_wait_mma(p_full, i & 1, wc)) { ok = false; break; }
-          tc_fence_after();
-          values(i);
-          if (i + 1 < ntiles && !scores(i + 1)) { ok = false; break; }
-        }
-      } else {
-        for (int i = 0; ok && i < ntiles; ++i) {
-          if (i > 0) {
-            // the value MMAs of tile i - 1 are done: S and G may be
-            // overwritten, and tile i - 1's stage takes tile i - 1 + NST
-            if (!mbar_wait_mma(pv_done, (i - 1) & 1, wc)) { ok = false; break; }
-            if (i - 1 + NST < ntiles) load_tile(i - 1 + NST);
-          }
-          if (!scores(i)) { ok = false; break; }
-          if (!mbar_wait_mma(p_full, i & 1, wc)) { ok = false; break; }
-          tc_fence_after();
-          values(i);
-        }
       }
       umma_commit(o_full);  // completes once every MMA issued above is done
       mbar_wait_drain(o_full, 0, p.timeout_ns);
@@ -357,8 +322,8 @@ __global__ void __launch_bounds__(LatTcCfg<MODE, DD>::THREADS, LatTcCfg<MODE, DD
             }
           }
           // over the 16 columns just read: dS high and low parts (and W)
-          tmem_st8(lane_base + Cfg::COL_DS + 16 * j, hi);
-          tmem_st8(lane_base + Cfg::COL_DS + 16 * j + 8, lo);
+          tmem_st8(lane_base + Cfg::COL_S + 16 * j, hi);
+          tmem_st8(lane_base + Cfg::COL_S + 16 * j + 8, lo);
           if (DEC) tmem_st8(lane_base + Cfg::COL_G + 16 * j, wp);
           if (j + 1 < T / 16) {
             tmem_wait_ld();
@@ -426,33 +391,24 @@ cudaError_t launch_split_hilo(const SplitHiLoParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-template <int MODE, int D>
-size_t lat_tc_smem() {
-  const size_t need = LatTcCfg<MODE, D>::BYTES + 1024;
+size_t lat_tc_smem_bytes(int D) {
+  const size_t need = (D == 16 ? LatTcCfg<16>::BYTES : LatTcCfg<32>::BYTES) + 1024;
   // at most CTAS_PER_SM CTAs per SM (228 KB each, 1 KB of it reserved per
   // CTA), so that every resident CTA finds its TMEM columns free
-  const size_t floor = (228 * 1024) / (LatTcCfg<MODE, D>::CTAS_PER_SM + 1) + 1024;
+  const size_t floor = (228 * 1024) / (LatTcCfg<16>::CTAS_PER_SM + 1) + 1024;
   return need > floor ? need : floor;
 }
 
-size_t lat_tc_smem_bytes(int mode, int D) {
-  if (D == 16) return mode == kLatTcDecoder ? lat_tc_smem<kLatTcDecoder, 16>() : lat_tc_smem<kLatTcEncoder, 16>();
-  return mode == kLatTcDecoder ? lat_tc_smem<kLatTcDecoder, 32>() : lat_tc_smem<kLatTcEncoder, 32>();
-}
-
-int lat_tc_tile(int mode, int D) {
-  if (D == 16) return mode == kLatTcDecoder ? LatTcCfg<kLatTcDecoder, 16>::T : LatTcCfg<kLatTcEncoder, 16>::T;
-  return mode == kLatTcDecoder ? LatTcCfg<kLatTcDecoder, 32>::T : LatTcCfg<kLatTcEncoder, 32>::T;
-}
+int lat_tc_tile(int D) { return D == 16 ? LatTcCfg<16>::T : LatTcCfg<32>::T; }
 
 cudaError_t launch_lat_tc(int mode, const LatTcMaps& m, const LatTcParams& p, cudaStream_t s) {
   if (p.D != 16 && p.D != 32) return cudaErrorInvalidValue;
-  const size_t smem = lat_tc_smem_bytes(mode, p.D);
+  const size_t smem = lat_tc_smem_bytes(p.D);
   const dim3 grid(static_cast<unsigned>(p.B * p.H * p.n_lblocks * p.n_splits));
   auto go = [&](auto kern) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid, LatTcCfg<kLatTcEncoder, 16>::THREADS, smem, s>>>(m.q, m.xa, m.xb, m.k, m.u, mode == kLatTcDecoder ? m.l : m.k,
+    kern<<<grid, LatTcCfg<16>::THREADS, smem, s>>>(m.q, m.xa, m.xb, m.k, m.u, mode == kLatTcDecoder ? m.l : m.k,
                                                    mode == kLatTcDecoder ? m.d : m.k, p);
     return cudaGetLastError();
   };
