@@ -33,13 +33,15 @@ collective).
 
 ``--backward`` times one ``flarepp_mixer_bwd`` call (``flare_mixer_bwd`` for a
 FLARE workload) per step with a seeded upstream gradient dY, against the
-backward's own roofline (three exponentials per score, the tf32 tensor term,
-HBM); ``e2e`` then copies the inputs and dY in and every gradient out.
+backward's own roofline (three exponentials per score, the tensor term at half
+the bf16 rate, HBM); ``e2e`` then copies the inputs and dY in and every
+gradient out.
 ``--train`` times a training step instead: the training forward
 (``flarepp_mixer_fwd_train``), which keeps its state, and the backward that
 reuses it (``flarepp_mixer_bwd_train``), against the sum of the forward's and
-the backward's rooflines; ``compare`` gives the plain forward + recomputing
-backward on the same inputs, timed after the timed region.
+the backward's rooflines; ``compare`` gives the plain forward + the
+self-contained backward (which runs the forward's kernels again) on the same
+inputs, timed after the timed region.
 """
 from __future__ import annotations
 
@@ -322,7 +324,10 @@ TRAIN_LAUNCHES = {("flarepp", 16): 8 + 24, ("flarepp", 32): 7 + 24, ("flare", 16
 # a self-contained backward call runs the same launches without the mark check
 BWD_LAUNCHES = {k: v - 1 for k, v in TRAIN_LAUNCHES.items()}
 TRAIN_METRIC = "mixer training step (fwd+bwd) token·heads/s at N=1M (1×B200) and % of roofline"
-TF32_PER_BF16 = 0.5  # nominal dense tf32 : bf16 tensor throughput
+# The backward's products take one operand (Z, dZ, dQ(X), dS or the gradient
+# rows, fp32) as two bf16 parts, so most of them cost two bf16 MMAs: half the
+# bf16 rate per useful flop (the nominal dense tf32 : bf16 ratio as well)
+SPLIT_PER_BF16 = 0.5
 
 
 def backward_work(w):
@@ -476,9 +481,9 @@ def run_backward(args, rank, world, local_rank):
     peaks = load_peaks()
     rates = pipe_rates(fl, dev)
     mufu_peak = rates["ex2"] * NUM_SM * peaks["sm_max_mhz"] * 1e6
-    tf32_peak = peaks["bf16_tflops"] * 1e12 * TF32_PER_BF16
+    split_peak = peaks["bf16_tflops"] * 1e12 * SPLIT_PER_BF16
     wk = backward_work(w)
-    terms = {"hbm": wk["bytes"] / (peaks["hbm_gbs"] * 1e9), "mma_tf32": wk["flops"] / tf32_peak,
+    terms = {"hbm": wk["bytes"] / (peaks["hbm_gbs"] * 1e9), "mma": wk["flops"] / split_peak,
              "mufu": wk["exps"] / mufu_peak}
     if train:
         # plus the forward: its exponentials, its bf16 tensor products and its
@@ -486,10 +491,10 @@ def run_backward(args, rank, world, local_rank):
         sw = stage_work(w)
         keys = ("encode", "merge", "decode") if flare else tuple(sw)
         terms["hbm"] += sum(sw[k]["bytes"] for k in keys) / (peaks["hbm_gbs"] * 1e9)
-        terms["mma_tf32"] += sum(sw[k]["flops"] for k in keys) / (peaks["bf16_tflops"] * 1e12)
+        terms["mma"] += sum(sw[k]["flops"] for k in keys) / (peaks["bf16_tflops"] * 1e12)
         terms["mufu"] += sum(sw[k]["exps"] for k in keys) / mufu_peak
     t_roof = max(terms.values())
-    bound = {"hbm": "hbm", "mma_tf32": "tensor", "mufu": "alu"}[max(terms, key=terms.get)]
+    bound = {"hbm": "hbm", "mma": "tensor", "mufu": "alu"}[max(terms, key=terms.get)]
 
     # end to end: inputs and dY in from pinned host memory, gradients back out,
     # all inside the timed region on the call's stream
@@ -533,17 +538,18 @@ def run_backward(args, rank, world, local_rank):
             "metric": TRAIN_METRIC if train else BWD_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "tf32", "data": "synthetic",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "pass": "training step" if train else "backward", "B": w.B, "N": w.N, "C": w.C, "H": w.H,
                        "D": w.D, "M": w.M, "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": ("inputs larger than L2 (K, V, dY: " +
                               f"{3 * w.B * w.H * w.N * w.D * 2 / 2**20:.0f} MiB together)" if flare else
-                              "inputs larger than L2 (X 256 MiB, dY 256 MiB, fp32 gradient rows 2 GiB)")},
+                              "inputs larger than L2 (X 256 MiB, dY 256 MiB, gradient rows 2 GiB)")},
             "step_roofline": {"t_roof_ms": round(t_roof * 1e3, 4), "frac": round(t_roof / (ms * 1e-3), 4),
                               "bound": bound, "terms_ms": {k: round(v * 1e3, 4) for k, v in terms.items()},
                               "peak_basis": f"MUFU {rates['ex2']:.2f} ex2/clk/SM ({rates['source']}) x {NUM_SM} x "
-                                            f"{peaks['sm_max_mhz']:.0f} MHz; tf32 = {TF32_PER_BF16} x measured "
-                                            f"bf16 {peaks['bf16_tflops']} TFLOP/s; HBM {peaks['hbm_gbs']} GB/s "
+                                            f"{peaks['sm_max_mhz']:.0f} MHz; tensor = {SPLIT_PER_BF16} x measured "
+                                            f"bf16 {peaks['bf16_tflops']} TFLOP/s (fp32 operands as two bf16 parts); "
+                                            f"HBM {peaks['hbm_gbs']} GB/s "
                                             f"({peaks['source']})"},
             "cpu_baseline": cpu,
             "e2e": {"value": whole_job_rate(world, th_per_rank, e2e_ms), "unit": UNIT,
