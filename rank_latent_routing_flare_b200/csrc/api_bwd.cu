@@ -67,7 +67,7 @@ BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C) {
   if (pp) {
     // the gradient rows [B*N][4C] = [dK | dV | dK~ | dV~] as two bf16 planes
     // (high and low parts), read by the projection gradients
-    bp.off_g32 = take(static_cast<size_t>(B * N) * 4 * C * 4);
+    bp.off_grows = take(static_cast<size_t>(B * N) * 4 * C * 4);
     bp.off_dwpart = take(static_cast<size_t>(bp.dw_splits) * C * 4 * C * 4);
   }
   // the high and low bf16 parts of dZ (then of dQ(X)) and of Z for the
@@ -81,7 +81,7 @@ BwdPlan make_bwd_plan(bool pp, long B, long H, long N, long M, long D, long C) {
   // after it has taken delta_n from Y)
   if (D == 16) {
     bp.off_zf16 = take(static_cast<size_t>(BH * M * D) * 2);
-    bp.off_y32 = pp ? bp.off_g32 : take(static_cast<size_t>(BH * N * D) * 4);
+    bp.off_y32 = pp ? bp.off_grows : take(static_cast<size_t>(BH * N * D) * 4);
   }
   bp.total = off;
   return bp;
@@ -462,7 +462,7 @@ flare_status pp_phase(int phase, const BwdPlan& bp, uint8_t* ws, const PpArgs& a
   float* q0pad = reinterpret_cast<float*>(ws + bp.off_q0pad);
   float* dqxpad = reinterpret_cast<float*>(ws + bp.off_dqxpad);
   // the gradient rows [B*N][4C] as bf16 high and low planes
-  uint16_t* ghi = reinterpret_cast<uint16_t*>(ws + bp.off_g32);
+  uint16_t* ghi = reinterpret_cast<uint16_t*>(ws + bp.off_grows);
   uint16_t* glo = ghi + static_cast<size_t>(B) * N * 4 * C;
   const size_t P = part_floats(bp, B, H, M, D, false);
   const size_t stride = pp_exchange_floats(bp, phase - 1, B, H, M, D, C);  // of the gathered buffers

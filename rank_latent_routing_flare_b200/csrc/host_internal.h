@@ -52,7 +52,7 @@ struct BwdPlan {
   int S = 1, tps = 1, rpb = 32, LB = 1, dw_splits = 1;
   size_t off_q32 = 0, off_qx32 = 0, off_lsyn = 0, off_dqx32 = 0, off_gsyn = 0, off_z32 = 0, off_lenc = 0,
          off_ltok = 0, off_dtok = 0, off_dz32 = 0, off_gam = 0, off_fpart = 0, off_pa = 0, off_pc = 0,
-         off_g32 = 0, off_dwpart = 0, off_y32 = 0, off_zf16 = 0, off_xhi16 = 0, off_xlo16 = 0, off_zhi16 = 0, off_zlo16 = 0, off_qpad = 0, off_q0pad = 0, off_zpad = 0, off_dzpad = 0,
+         off_grows = 0, off_dwpart = 0, off_y32 = 0, off_zf16 = 0, off_xhi16 = 0, off_xlo16 = 0, off_zhi16 = 0, off_zlo16 = 0, off_qpad = 0, off_q0pad = 0, off_zpad = 0, off_dzpad = 0,
          off_dqxpad = 0, off_dqxdec = 0, total = 0;
 };
 
